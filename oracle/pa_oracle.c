@@ -1,0 +1,292 @@
+/*
+ * pa_oracle.c -- the oracle for the paged KV-cache hot path.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path may call, link or
+ * load this file; only the tests, the smoke check and the benchmark's CPU
+ * baseline do.  It shares no code with the CUDA library: it has its own
+ * 16-bit float decoders, its own slot arithmetic and its own attention.
+ *
+ * Plain C, fp64 arithmetic, no fast-math, no blocking, no fusion.  Each
+ * function restates one step as the pages describe it:
+ *
+ *   orc_slot_mapping      "PagedAttention" (shubhamtatvamasi), "How attention
+ *                         reads paged memory" + the block-size-4 figure: a
+ *                         block table maps logical block i to a physical
+ *                         block id; token p of a sequence lives in logical
+ *                         block p / block_size at offset p % block_size.
+ *   orc_reshape_and_cache "How PagedAttention Works in vLLM to Maximize
+ *                         Memory Efficiency", "write_to_paged_cache: Direct
+ *                         In-Place Updates" and "Code Example": new K/V rows
+ *                         [num_tokens, num_kv_heads, head_size] are scattered
+ *                         into the pool at the flat slots of slot_mapping.
+ *   orc_copy_blocks       "PagedAttention", "How does copy-on-write work for
+ *                         parallel sampling?": allocate a block, copy the
+ *                         shared block's contents into it.
+ *   orc_decode            "PagedAttention", "How attention reads paged
+ *                         memory": for each query token walk the sequence's
+ *                         block table, gather every block's keys and values,
+ *                         and run attention over them.  The oracle gathers
+ *                         into one contiguous buffer and evaluates plain
+ *                         softmax(scale * q K^T) V in double precision (the
+ *                         exact quantity that an online softmax reaches up to
+ *                         rounding order).
+ *
+ * Pool layout (one tensor for K, one for V):
+ *   [num_blocks, block_size, num_kv_heads, head_dim]  -- "PagedAttention",
+ *   "How attention reads paged memory"; the same as one half of the flash
+ *   layout (2, num_blocks, block_size, num_kv_heads, head_size) on the vLLM
+ *   page, "Flash Layout: The Canonical Storage Format".
+ *
+ * Readings where the pages are silent (grouped-query head mapping, empty
+ * sequences) are stated at the function that takes them.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORC_F16 0
+#define ORC_BF16 1
+
+/* ---------------------------------------------------------------------------
+ * 16-bit float decoders, written from the IEEE 754 binary16 definition and
+ * the bfloat16 definition (the upper half of an IEEE binary32).
+ * ------------------------------------------------------------------------- */
+double orc_half_to_double(uint16_t h) {
+  int sign = (h >> 15) & 1;
+  int e = (h >> 10) & 0x1f;
+  int m = h & 0x3ff;
+  double v;
+  if (e == 0) {
+    v = ldexp((double)m, -24); /* subnormal: m * 2^-14 * 2^-10 */
+  } else if (e == 31) {
+    v = (m == 0) ? INFINITY : NAN;
+  } else {
+    v = ldexp((double)(1024 + m), e - 25); /* (1 + m/2^10) * 2^(e-15) */
+  }
+  return sign ? -v : v;
+}
+
+double orc_bf16_to_double(uint16_t b) {
+  int sign = (b >> 15) & 1;
+  int e = (b >> 7) & 0xff;
+  int m = b & 0x7f;
+  double v;
+  if (e == 0) {
+    v = ldexp((double)m, -133); /* subnormal: m * 2^-126 * 2^-7 */
+  } else if (e == 255) {
+    v = (m == 0) ? INFINITY : NAN;
+  } else {
+    v = ldexp((double)(128 + m), e - 134); /* (1 + m/2^7) * 2^(e-127) */
+  }
+  return sign ? -v : v;
+}
+
+static double orc_decode16(uint16_t bits, int dtype) {
+  return dtype == ORC_BF16 ? orc_bf16_to_double(bits) : orc_half_to_double(bits);
+}
+
+/* ---------------------------------------------------------------------------
+ * Slot of token position `pos` of a sequence whose block-table row is
+ * `table_row`: the physical block holding logical block pos / block_size,
+ * times block_size, plus the offset pos % block_size.
+ * ------------------------------------------------------------------------- */
+int64_t orc_slot_of(const int32_t* table_row, int64_t pos, int32_t block_size) {
+  int64_t logical_block = pos / block_size;
+  int64_t offset = pos % block_size;
+  return (int64_t)table_row[logical_block] * block_size + offset;
+}
+
+/* slots[i] = slot of position pos[i] of sequence seq_idx[i]; the table is
+ * row-major with `table_stride` entries per sequence. */
+void orc_slot_mapping(const int32_t* block_tables, int64_t table_stride,
+                      const int32_t* seq_idx, const int32_t* pos, int64_t n,
+                      int32_t block_size, int64_t* slots) {
+  for (int64_t i = 0; i < n; ++i) {
+    const int32_t* row = block_tables + (int64_t)seq_idx[i] * table_stride;
+    slots[i] = orc_slot_of(row, pos[i], block_size);
+  }
+}
+
+/* ---------------------------------------------------------------------------
+ * reshape_and_cache: for every new token t whose slot s = slot_mapping[t] is
+ * non-negative, copy key[t, h, :] to key_cache[s / bs, s % bs, h, :] for every
+ * KV head h, and the same for the values.  A negative slot is a padding token
+ * and writes nothing.  The copy is of the raw 16-bit words, so the cache ends
+ * up bit-identical to the input rows.
+ * key/value rows are `key_stride_t` / `value_stride_t` elements apart.
+ * ------------------------------------------------------------------------- */
+void orc_reshape_and_cache(const uint16_t* key, const uint16_t* value,
+                           int64_t key_stride_t, int64_t value_stride_t,
+                           uint16_t* key_cache, uint16_t* value_cache,
+                           const int32_t* slot_mapping, int64_t num_tokens,
+                           int32_t block_size, int32_t num_kv_heads,
+                           int32_t head_dim) {
+  for (int64_t t = 0; t < num_tokens; ++t) {
+    int64_t s = slot_mapping[t];
+    if (s < 0) continue;
+    int64_t block = s / block_size;
+    int64_t offset = s % block_size;
+    for (int32_t h = 0; h < num_kv_heads; ++h) {
+      int64_t dst = ((block * block_size + offset) * num_kv_heads + h) * head_dim;
+      for (int32_t d = 0; d < head_dim; ++d) {
+        key_cache[dst + d] = key[t * key_stride_t + (int64_t)h * head_dim + d];
+        value_cache[dst + d] = value[t * value_stride_t + (int64_t)h * head_dim + d];
+      }
+    }
+  }
+}
+
+/* ---------------------------------------------------------------------------
+ * copy_blocks (copy-on-write): for every (src, dst) pair, the whole physical
+ * block dst of every layer's K and V pool becomes a byte copy of block src.
+ * `caches` holds 2 * num_layers base pointers: K of layer 0, V of layer 0,
+ * K of layer 1, ...
+ * ------------------------------------------------------------------------- */
+void orc_copy_blocks(uint8_t* const* caches, int32_t num_layers,
+                     const int32_t* block_mapping, int64_t num_pairs,
+                     int64_t block_bytes) {
+  for (int64_t i = 0; i < num_pairs; ++i) {
+    int64_t src = block_mapping[2 * i];
+    int64_t dst = block_mapping[2 * i + 1];
+    for (int32_t c = 0; c < 2 * num_layers; ++c) {
+      memcpy(caches[c] + dst * block_bytes, caches[c] + src * block_bytes,
+             (size_t)block_bytes);
+    }
+  }
+}
+
+/* ---------------------------------------------------------------------------
+ * Decode attention, one query token per sequence.
+ *
+ *   out[b, h, :] = sum_t p_t V_b[t] / sum_t p_t,
+ *   p_t = exp(s_t - max_u s_u),  s_t = scale * <q[b, h, :], K_b[t]>,
+ *
+ * where K_b, V_b are sequence b's first seq_lens[b] tokens gathered through
+ * its block table into contiguous buffers.
+ *
+ * Readings where the pages are silent:
+ *  - grouped-query attention: query head h reads KV head h / (Hq / Hkv)
+ *    (consecutive query heads share one KV head);
+ *  - a sequence with seq_len 0 attends to nothing: its output is all zeros.
+ * Inputs q [B, Hq, D] and the pools hold 16-bit floats (`dtype`); the output
+ * is double [B, Hq, D].  Sequences are independent, so `nthreads` worker
+ * threads take whole sequences; the arithmetic per sequence is unchanged.
+ * ------------------------------------------------------------------------- */
+typedef struct {
+  double* out;
+  const uint16_t* q;
+  const uint16_t* key_cache;
+  const uint16_t* value_cache;
+  const int32_t* block_tables;
+  int64_t table_stride;
+  const int32_t* seq_lens;
+  int32_t num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, dtype;
+  double scale;
+  int32_t next_seq; /* work counter, guarded by mu */
+  pthread_mutex_t mu;
+  int32_t failed;
+} orc_decode_job;
+
+static int orc_decode_one(orc_decode_job* j, int32_t b) {
+  const int32_t Hq = j->num_q_heads, Hkv = j->num_kv_heads, D = j->head_dim;
+  const int32_t bs = j->block_size;
+  const int32_t group = Hq / Hkv;
+  const int64_t L = j->seq_lens[b];
+  double* outb = j->out + (int64_t)b * Hq * D;
+  if (L <= 0) {
+    for (int64_t i = 0; i < (int64_t)Hq * D; ++i) outb[i] = 0.0;
+    return 0;
+  }
+  const int32_t* row = j->block_tables + (int64_t)b * j->table_stride;
+  /* Gather this sequence's K and V into contiguous [L, Hkv, D] buffers. */
+  double* Kc = (double*)malloc(sizeof(double) * (size_t)(L * Hkv * D));
+  double* Vc = (double*)malloc(sizeof(double) * (size_t)(L * Hkv * D));
+  double* s = (double*)malloc(sizeof(double) * (size_t)L);
+  if (!Kc || !Vc || !s) {
+    free(Kc); free(Vc); free(s);
+    return 1;
+  }
+  for (int64_t t = 0; t < L; ++t) {
+    int64_t slot = orc_slot_of(row, t, bs);
+    for (int32_t g = 0; g < Hkv; ++g) {
+      for (int32_t d = 0; d < D; ++d) {
+        int64_t src = (slot * Hkv + g) * D + d;
+        Kc[(t * Hkv + g) * D + d] = orc_decode16(j->key_cache[src], j->dtype);
+        Vc[(t * Hkv + g) * D + d] = orc_decode16(j->value_cache[src], j->dtype);
+      }
+    }
+  }
+  for (int32_t h = 0; h < Hq; ++h) {
+    const int32_t g = h / group;
+    const uint16_t* qh = j->q + ((int64_t)b * Hq + h) * D;
+    double m = -INFINITY;
+    for (int64_t t = 0; t < L; ++t) {
+      double dot = 0.0;
+      for (int32_t d = 0; d < D; ++d)
+        dot += orc_decode16(qh[d], j->dtype) * Kc[(t * Hkv + g) * D + d];
+      s[t] = j->scale * dot;
+      if (s[t] > m) m = s[t];
+    }
+    double denom = 0.0;
+    for (int64_t t = 0; t < L; ++t) {
+      s[t] = exp(s[t] - m);
+      denom += s[t];
+    }
+    for (int32_t d = 0; d < D; ++d) {
+      double acc = 0.0;
+      for (int64_t t = 0; t < L; ++t) acc += s[t] * Vc[(t * Hkv + g) * D + d];
+      outb[(int64_t)h * D + d] = acc / denom;
+    }
+  }
+  free(Kc); free(Vc); free(s);
+  return 0;
+}
+
+static void* orc_decode_worker(void* arg) {
+  orc_decode_job* j = (orc_decode_job*)arg;
+  for (;;) {
+    pthread_mutex_lock(&j->mu);
+    int32_t b = j->next_seq++;
+    pthread_mutex_unlock(&j->mu);
+    if (b >= j->num_seqs) break;
+    if (orc_decode_one(j, b)) {
+      pthread_mutex_lock(&j->mu);
+      j->failed = 1;
+      pthread_mutex_unlock(&j->mu);
+    }
+  }
+  return NULL;
+}
+
+/* Returns 0 on success, 1 on allocation failure, 2 on a bad argument. */
+int orc_decode(double* out, const uint16_t* q, const uint16_t* key_cache,
+               const uint16_t* value_cache, const int32_t* block_tables,
+               int64_t table_stride, const int32_t* seq_lens, int32_t num_seqs,
+               int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+               int32_t block_size, double scale, int32_t dtype,
+               int32_t nthreads) {
+  if (num_kv_heads <= 0 || num_q_heads % num_kv_heads != 0 || block_size <= 0)
+    return 2;
+  orc_decode_job j;
+  j.out = out; j.q = q; j.key_cache = key_cache; j.value_cache = value_cache;
+  j.block_tables = block_tables; j.table_stride = table_stride;
+  j.seq_lens = seq_lens; j.num_seqs = num_seqs; j.num_q_heads = num_q_heads;
+  j.num_kv_heads = num_kv_heads; j.head_dim = head_dim;
+  j.block_size = block_size; j.dtype = dtype; j.scale = scale;
+  j.next_seq = 0; j.failed = 0;
+  pthread_mutex_init(&j.mu, NULL);
+  if (nthreads <= 1) {
+    orc_decode_worker(&j);
+  } else {
+    pthread_t* th = (pthread_t*)malloc(sizeof(pthread_t) * (size_t)nthreads);
+    if (!th) { pthread_mutex_destroy(&j.mu); return 1; }
+    for (int32_t i = 0; i < nthreads; ++i)
+      pthread_create(&th[i], NULL, orc_decode_worker, &j);
+    for (int32_t i = 0; i < nthreads; ++i) pthread_join(th[i], NULL);
+    free(th);
+  }
+  pthread_mutex_destroy(&j.mu);
+  return j.failed ? 1 : 0;
+}
