@@ -1,0 +1,520 @@
+"""Benchmark of the paged decode hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one decode step of the workload over its whole batch:
+copy_blocks (only where the workload has copy-on-write pairs) ->
+reshape_and_cache of the step's new K/V rows -> decode_attention (plan, main,
+combine).  Inputs are resident in HBM when the timed region starts; block
+tables and slots come from the native host block manager.
+
+Prints ONE JSON line (rank 0).  `value` is KV-read GB/s: the algorithmic KV
+bytes of a step (sum of seq_len * 2 * Hkv * D * 2 bytes, valid tokens only)
+times the steps and ranks, divided by the device time (CUDA events, max over
+ranks).  `--impl reference` times the fp64 CPU oracle instead, on bounded
+samples of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import pa_workloads as W  # noqa: E402
+
+METRIC = "paged decode attention KV-read GB/s (% of B200 HBM peak); decode tokens/s"
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "decode_main_llama8b.md")
+KERNEL_SOURCES = [os.path.join(ROOT, "paged_kv_cache_343_b200", "csrc", f)
+                  for f in ("pa_decode.cu", "pa_device.cuh")]
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return json.load(f), "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def profiled_traffic():
+    """DRAM bytes per launch of the main kernel from the committed ncu summary,
+    or None if there is none or the kernel changed since it was taken."""
+    if not os.path.exists(PROFILE_SUMMARY):
+        return None
+    txt = open(PROFILE_SUMMARY).read()
+    m_hash = re.search(r"kernel_source_hash:\s*([0-9a-f]+)", txt)
+    m_bytes = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", txt)
+    if not m_hash or not m_bytes or m_hash.group(1) != kernel_source_hash():
+        return None
+    return float(m_bytes.group(1))
+
+
+# --------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.rows = []
+        self.proc = None
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.rows.append((time.time(), line.strip()))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        if self.thread is not None:
+            self.thread.join(timeout=2)
+
+    def summary(self, t0: float, t1: float):
+        def parse(r):
+            parts = [x.strip() for x in r.split(",")]
+            try:
+                return {"sm": float(parts[1]), "max": float(parts[2]), "active": parts[4],
+                        "hw": parts[5], "hwt": parts[6], "swt": parts[7], "pcap": parts[8]}
+            except (ValueError, IndexError):
+                return None
+        inside = [parse(r) for (t, r) in self.rows if t0 <= t <= t1]
+        inside = [x for x in inside if x]
+        window = "timed region"
+        if not inside:  # region shorter than the sampling period: nearest samples
+            near = sorted(self.rows, key=lambda tr: min(abs(tr[0] - t0), abs(tr[0] - t1)))[:3]
+            inside = [x for x in (parse(r) for _, r in near) if x]
+            window = "nearest samples (timed region shorter than the 50 ms period)"
+        if not inside:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        reasons = set()
+        for x in inside:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
+                              ("swt", "sw_thermal_slowdown"), ("pcap", "sw_power_cap")):
+                if x[key].lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(x["sm"] for x in inside),
+                "sm_max_mhz": max(x["max"] for x in inside), "reasons": sorted(reasons),
+                "samples": len(inside), "window": window}
+
+
+# --------------------------------------------------------------------------- workload
+def kv_bytes(spec, lens) -> int:
+    return int(np.sum(lens.astype(np.int64))) * 2 * spec.num_kv_heads * spec.head_dim * spec.elem_bytes
+
+
+def build_workload(spec, pa):
+    """Seeded inputs and metadata from the native block manager.
+
+    Plain workloads: every sequence holds seq_len - 1 tokens and the step
+    appends its current token (position seq_len - 1), which the attention then
+    reads.  shared_prefix: prompts forked into samples, each sample appending
+    its extra tokens (copy-on-write on the first append)."""
+    case = W.draw(spec)
+    bs = spec.block_size
+    bm = pa.BlockManager(case.num_blocks, bs, case.free_order)
+    B = spec.num_seqs
+    lens = case.seq_lens.astype(np.int32)
+    cow = []
+    if spec.len_dist == "shared_prefix":
+        sid = 0
+        for _ in range(spec.prompts):
+            bm.add_sequence(sid, spec.prompt_len)
+            for s in range(1, spec.samples):
+                bm.fork(sid, sid + s)
+            sid += spec.samples
+        slots = []
+        for b in range(B):
+            for _ in range(int(case.extra_tokens[b])):
+                slot, c = bm.append_slot(b)
+                slots.append(slot)
+                if c is not None:
+                    cow.append(c)
+        new_k, new_v = case.new_k, case.new_v
+    else:
+        slots = []
+        for b in range(B):
+            bm.add_sequence(b, int(lens[b]) - 1)
+            slots.append(bm.append_slot(b)[0])
+        g = torch.Generator().manual_seed(spec.seed + 7)
+        new_k = W.randn_bits((B, spec.num_kv_heads, spec.head_dim), spec.dtype, g)
+        new_v = W.randn_bits((B, spec.num_kv_heads, spec.head_dim), spec.dtype, g)
+    width = max(len(bm.block_table(b)) for b in range(B))
+    tables = bm.tables(list(range(B)), width).numpy()
+    return dict(case=case, lens=lens, tables=tables, slots=np.array(slots, np.int32),
+                cow=np.array(cow, np.int32).reshape(-1, 2), new_k=new_k, new_v=new_v)
+
+
+def unique_kv_bytes(spec, wl) -> int:
+    """KV bytes of distinct (block, offset) slots read by the step."""
+    bs = spec.block_size
+    seen = set()
+    for b in range(spec.num_seqs):
+        L = int(wl["lens"][b])
+        for i in range(-(-L // bs)):
+            blk = int(wl["tables"][b, i])
+            n = min(bs, L - i * bs)
+            seen.add((blk, n))
+    slots = {}
+    for blk, n in seen:
+        slots[blk] = max(slots.get(blk, 0), n)
+    return sum(slots.values()) * 2 * spec.num_kv_heads * spec.head_dim * spec.elem_bytes
+
+
+# --------------------------------------------------------------------------- our arm
+def run_ours(args, rank, world, local_rank):
+    import paged_kv_cache_343_b200 as pa
+
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    spec = W.WORKLOADS[args.workload]
+    if world > 1:
+        spec = spec.replace(seed=spec.seed + 100 * rank)
+    wl = build_workload(spec, pa)
+    case = wl["case"]
+    td = {"f16": torch.float16, "bf16": torch.bfloat16}[spec.dtype]
+
+    def dev_bits(a):
+        return torch.from_numpy(np.ascontiguousarray(a)).view(torch.int16).view(td).to(device)
+
+    k_cache, v_cache = dev_bits(case.k_pool), dev_bits(case.v_pool)
+    q = dev_bits(case.q)
+    new_k, new_v = dev_bits(wl["new_k"]), dev_bits(wl["new_v"])
+    slots = torch.from_numpy(wl["slots"]).to(device)
+    tables = torch.from_numpy(wl["tables"]).to(device)
+    lens = torch.from_numpy(wl["lens"]).to(device)
+    cow = torch.from_numpy(wl["cow"]).to(device) if wl["cow"].size else None
+    out = torch.empty_like(q)
+    B, Hq, D = q.shape
+    max_len = int(wl["lens"].max())
+    psize = spec.partition_size
+    ws = pa.alloc_workspace(pa.decode_workspace_bytes(B, Hq, spec.num_kv_heads, D, spec.block_size,
+                                                      max_len, psize), device)
+    flag = torch.zeros(1, dtype=torch.int32, device=device)
+    scale = W.scale_of(spec)
+    stream = torch.cuda.current_stream(device)
+    launches_per_step = 1 + 3 + (1 if cow is not None else 0)
+
+    def step(ev0=None, ev1=None):
+        if cow is not None:
+            pa.copy_blocks([k_cache], [v_cache], cow, error_flag=flag)
+        pa.reshape_and_cache(new_k, new_v, k_cache, v_cache, slots, error_flag=flag)
+        if ev0 is not None:
+            ev0.record(stream)
+        pa.decode_attention(out, q, k_cache, v_cache, tables, lens, max_len, scale, psize, ws,
+                            error_flag=flag)
+        if ev1 is not None:
+            ev1.record(stream)
+
+    bytes_step = kv_bytes(spec, wl["lens"])
+    clocks = ClockSampler(local_rank if "CUDA_VISIBLE_DEVICES" not in os.environ
+                          else int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local_rank]))
+    clocks.start()
+    time.sleep(1.0)  # let nvidia-smi attach
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if int(flag.item()) != 0:
+        raise RuntimeError("device error flag %#x during warm-up" % int(flag.item()))
+
+    ev_att = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    wall0 = time.time()
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(*ev_att[i])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    wall1 = time.time()
+    if world > 1:
+        torch.distributed.barrier()
+    clock_info = clocks.summary(wall0, wall1)
+    clocks.stop()
+    elapsed_ms = t_start.elapsed_time(t_end)
+    att_ms = [a.elapsed_time(b) for a, b in ev_att]
+    att_avg_ms = sum(att_ms) / len(att_ms)
+    if int(flag.item()) != 0:
+        raise RuntimeError("device error flag %#x in the timed region" % int(flag.item()))
+
+    # ---------------- end to end: pinned host buffers through the public API
+    e2e_steps = max(1, min(args.steps, args.e2e_steps))
+    runner = pa.PagedDecodeStep(k_cache, v_cache, B, Hq, wl["tables"].shape[1], max_len, scale,
+                                psize)
+
+    def pinned(a, dtype=None):
+        t = torch.from_numpy(np.ascontiguousarray(a))
+        if dtype is not None:
+            t = t.view(torch.int16).view(dtype)
+        return t.pin_memory()
+
+    hq, hk, hv = pinned(case.q, td), pinned(wl["new_k"], td), pinned(wl["new_v"], td)
+    hs, ht, hl = pinned(wl["slots"]), pinned(wl["tables"]), pinned(wl["lens"])
+    hout = torch.empty(q.shape, dtype=td).pin_memory()
+    e2e_ok = wl["slots"].shape[0] == B and cow is None
+    e2e = None
+    if e2e_ok:
+        for _ in range(2):
+            runner(hq, hk, hv, hs, ht, hl, hout)
+        if world > 1:
+            torch.distributed.barrier()
+        t0 = time.perf_counter()
+        for _ in range(e2e_steps):
+            runner(hq, hk, hv, hs, ht, hl, hout)
+        e2e_s = time.perf_counter() - t0
+        e2e_s = max_over_ranks(e2e_s, world, device)
+        e2e = {"value": round(bytes_step * e2e_steps * world / e2e_s / 1e9, 2), "unit": "GB/s",
+               "h2d_bytes_per_step": runner.h2d_bytes(), "d2h_bytes_per_step": runner.d2h_bytes(),
+               "steps": e2e_steps, "ms_per_step": round(e2e_s * 1e3 / e2e_steps, 4)}
+
+    elapsed_ms = max_over_ranks(elapsed_ms, world, device)
+    att_avg_ms = max_over_ranks(att_avg_ms, world, device)
+    total_bytes = sum_over_ranks(float(bytes_step), world, device)
+    if rank != 0:
+        return None
+    peaks, peak_kind = load_peaks()
+    ms_per_step = elapsed_ms / args.steps
+    value = total_bytes * args.steps / (elapsed_ms / 1e3) / 1e9
+    achieved = bytes_step / (att_avg_ms / 1e3) / 1e9
+    peak = float(peaks["hbm_gbs"])
+    traffic = profiled_traffic() if args.workload == "llama8b" else None
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": spec.dtype,
+        "data": "synthetic (seeded N(0,1) values; lengths, placement and sharing per workload)",
+        "config": {
+            "workload": "%s: B %d, Hq %d / Hkv %d, D %d, block %d, %s, lengths %s" % (
+                spec.name, spec.num_seqs, spec.num_q_heads, spec.num_kv_heads, spec.head_dim,
+                spec.block_size, spec.dtype, describe_lengths(spec)),
+            "global_batch": spec.num_seqs * world, "kv_bytes_per_step": bytes_step,
+            "sum_seq_len": int(wl["lens"].sum()), "partition_size": psize,
+            "num_blocks": case.num_blocks, "parallelism": "dp%d (independent batches)" % world,
+            "l2": "no flush: each step reads %.0f MB of KV, more than the 126 MB L2" % (bytes_step / 1e6),
+        },
+        "decode_tokens_per_s": round(spec.num_seqs * world / (ms_per_step / 1e3), 1),
+        "attention_gbs": round(achieved, 2),
+        "pct_of_8tbs": round(100.0 * value / 8000.0, 2),
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "traffic": traffic,
+                     "kernel": "pa_decode_attention (plan + main + combine launches)",
+                     "peak_kind": peak_kind + " (MEASURED_PEAKS hbm_gbs, copy read+write)"},
+        "clocks": clock_info,
+        "e2e": e2e,
+        "gpu_launches": launches_per_step * args.steps,
+    }
+    if spec.len_dist == "shared_prefix":
+        ub = unique_kv_bytes(spec, wl)
+        line["config"]["unique_kv_bytes_per_step"] = ub
+        line["unique_gbs"] = round(ub * args.steps / (elapsed_ms / 1e3) / 1e9, 2)
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(spec, wl, budget_s=args.cpu_budget)
+    return line
+
+
+def describe_lengths(spec):
+    if spec.len_dist == "uniform":
+        return "U[%d, %d]" % (spec.len_lo, spec.len_hi)
+    if spec.len_dist == "lognormal":
+        return "lognormal(median %g, sigma %g) clipped [%d, %d]" % (
+            spec.lognormal_median, spec.lognormal_sigma, spec.len_lo, spec.len_hi)
+    if spec.len_dist == "shared_prefix":
+        return "%d-token prompt x %d samples + U[%d, %d]" % (spec.prompt_len, spec.samples,
+                                                            spec.extra_lo, spec.extra_hi)
+    return "fixed %s" % (sorted(set(spec.fixed_lens)),)
+
+
+def max_over_ranks(x, world, device):
+    if world == 1:
+        return x
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x, world, device):
+    if world == 1:
+        return x
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.SUM)
+    return float(t.item())
+
+
+# --------------------------------------------------------------------------- oracle
+def _oracle_sample(spec, wl, seqs):
+    """One oracle step over the sequences `seqs`: the writes of their new rows,
+    then fp64 attention.  Returns (seconds, kv bytes)."""
+    import oracle
+    case = wl["case"]
+    k, v = case.k_pool, case.v_pool
+    threads = len(os.sched_getaffinity(0))
+    t0 = time.perf_counter()
+    if spec.len_dist != "shared_prefix":
+        oracle.reshape_and_cache(wl["new_k"][seqs], wl["new_v"][seqs], k, v, wl["slots"][seqs])
+    oracle.decode(case.q[seqs], k, v, wl["tables"][seqs], wl["lens"][seqs], W.scale_of(spec),
+                  spec.dtype, nthreads=threads)
+    return time.perf_counter() - t0, kv_bytes(spec, wl["lens"][seqs])
+
+
+def cpu_baseline(spec, wl, budget_s=20.0):
+    """The oracle, as it stands, on all host cores, over a bounded sample:
+    whole-batch steps repeated while they fit in the budget (at least one)."""
+    B = spec.num_seqs
+    threads = len(os.sched_getaffinity(0))
+    total_t, total_b, n = 0.0, 0, 0
+    seqs = np.arange(B)
+    while True:
+        t, b = _oracle_sample(spec, wl, seqs)
+        total_t += t
+        total_b += b
+        n += 1
+        if total_t + t > budget_s or n >= 5:
+            break
+    return {"value": round(total_b / total_t / 1e9, 4), "unit": "GB/s", "cores": threads,
+            "kind": "oracle",
+            "sample": "%d full step(s) of the %s batch (%d sequences, %d tokens each step): "
+                      "reshape_and_cache + fp64 decode, %.1f s" % (
+                          n, spec.name, B, int(wl["lens"].sum()), total_t)}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    spec = W.WORKLOADS[args.workload]
+
+    # the oracle's own block manager builds the metadata for the reference arm
+    from oracle.blockmgr import RefBlockManager
+    case = W.draw(spec)
+    bm = RefBlockManager(case.num_blocks, spec.block_size, case.free_order)
+    lens = case.seq_lens.astype(np.int32)
+    slots = []
+    for b in range(spec.num_seqs):
+        bm.add_sequence(b, int(lens[b]) - 1)
+        slots.append(bm.append_slot(b)[0])
+    g = torch.Generator().manual_seed(spec.seed + 7)
+    new_k = W.randn_bits((spec.num_seqs, spec.num_kv_heads, spec.head_dim), spec.dtype, g)
+    new_v = W.randn_bits((spec.num_seqs, spec.num_kv_heads, spec.head_dim), spec.dtype, g)
+    width = max(len(bm.block_table(b)) for b in range(spec.num_seqs))
+    tables = np.full((spec.num_seqs, width), -1, np.int32)
+    for b in range(spec.num_seqs):
+        t = bm.block_table(b)
+        tables[b, :len(t)] = t
+    wl = dict(case=case, lens=lens, tables=tables, slots=np.array(slots, np.int32),
+              new_k=new_k, new_v=new_v)
+    # size each step so warm-up + timed steps take about args.ref_budget seconds
+    B = spec.num_seqs
+    t1, _ = _oracle_sample(spec, wl, np.arange(1))
+    per_seq = max(t1, 1e-4)
+    n_steps = args.warmup + args.steps
+    per_step = max(1, min(B, int(args.ref_budget / n_steps / per_seq)))
+    rng = np.random.default_rng(0)
+    for _ in range(args.warmup):
+        _oracle_sample(spec, wl, np.sort(rng.choice(B, per_step, replace=False)))
+    tt, tb = 0.0, 0
+    for _ in range(args.steps):
+        t, b = _oracle_sample(spec, wl, np.sort(rng.choice(B, per_step, replace=False)))
+        tt += t
+        tb += b
+    value = tb / tt / 1e9
+    threads = len(os.sched_getaffinity(0))
+    sample = "%d of %d sequences per step (random, seeded), reshape_and_cache + fp64 decode" % (
+        per_step, B)
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(tt * 1e3 / args.steps, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded N(0,1) values; lengths and placement per workload)",
+        "config": {"workload": spec.name, "global_batch": spec.num_seqs,
+                   "parallelism": "host cores"},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": threads,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default="llama8b", choices=sorted(W.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=200)
+    ap.add_argument("--cpu-budget", type=float, default=20.0)
+    ap.add_argument("--ref-budget", type=float, default=90.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return 0
+
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        line = run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+    if line is not None:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,226 @@
+/*
+ * pagedattn.h -- C ABI of libpagedattn.so, the paged KV-cache decode hot path
+ * for NVIDIA B200 (sm_100a).
+ *
+ * The operations follow three public pages on PagedAttention:
+ *   [vLLM]  "How PagedAttention Works in vLLM to Maximize Memory Efficiency"
+ *   [PA]    "PagedAttention" (shubhamtatvamasi.com)
+ *   [KV]    "KV cache and PagedAttention: how vLLM uses GPU memory more
+ *           efficiently" (suenot.com)
+ *
+ * Conventions shared by every entry point
+ *  - Pointers named *_cache, key, value, query, out, block_tables, seq_lens,
+ *    slot_mapping, block_mapping and workspace are DEVICE pointers; the caller
+ *    owns every buffer (the library allocates no device memory in these calls
+ *    and keeps no state except a small host-side cache of TMA descriptors).
+ *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *    default stream).  Arguments are validated on the host before any launch;
+ *    a rejected call launches nothing.
+ *  - KV pool layout, one tensor for K and one for V ([PA] "How attention reads
+ *    paged memory"; identical to one half of the flash layout
+ *    (2, num_blocks, block_size, num_kv_heads, head_size), [vLLM] "Flash
+ *    Layout: The Canonical Storage Format"):
+ *        [num_blocks, block_size, num_kv_heads, head_dim], contiguous,
+ *    16-bit elements (fp16 or bf16), base address 16-byte aligned.
+ *  - Optional `device_error_flag` (int32, device): kernels OR PA_DEVERR_* bits
+ *    into it when they meet bad data (an out-of-range block id or slot, a
+ *    sequence longer than max_seq_len, a pipeline wait that ran out).  The
+ *    offending element is skipped; nothing traps.  Read it after the stream
+ *    has synchronised.  NULL disables reporting (skipping still happens).
+ */
+#ifndef PAGEDATTN_H_
+#define PAGEDATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* pa_stream_t; /* == cudaStream_t */
+
+typedef enum {
+  PA_OK = 0,
+  PA_ERR_INVALID_ARG = 1,   /* null pointer, bad size, misalignment, ...   */
+  PA_ERR_UNSUPPORTED = 2,   /* valid but outside the built shapes/dtypes   */
+  PA_ERR_CUDA = 3,          /* a CUDA runtime call or launch failed        */
+  PA_ERR_OUT_OF_BLOCKS = 4, /* block manager: the free list is empty       */
+  PA_ERR_NOT_FOUND = 5      /* block manager: unknown sequence id          */
+} pa_status;
+
+typedef enum { PA_F16 = 0, PA_BF16 = 1, PA_F32 = 2 } pa_dtype;
+
+/* Cache storage type of write_to_paged_cache's kv_cache_dtype ([vLLM]
+ * "write_to_paged_cache: Direct In-Place Updates"); only "auto" (the cache
+ * holds the model's 16-bit type) is built. */
+typedef enum { PA_KV_AUTO = 0 } pa_kv_cache_dtype;
+
+#define PA_DEVERR_BAD_BLOCK 0x1   /* block-table entry outside [0, num_blocks) */
+#define PA_DEVERR_BAD_SLOT 0x2    /* slot / block id outside the pool          */
+#define PA_DEVERR_BAD_SEQLEN 0x4  /* seq_len < 0 or > max_seq_len              */
+#define PA_DEVERR_TIMEOUT 0x8     /* a bounded pipeline wait gave up           */
+
+/* Human-readable name of a status code (static storage). */
+const char* pa_status_string(pa_status status);
+
+/* Library version as major*10000 + minor*100 + patch. */
+int32_t pa_version(void);
+
+/* ---------------------------------------------------------------------------
+ * pa_reshape_and_cache -- [vLLM] "write_to_paged_cache: Direct In-Place
+ * Updates" (write_to_paged_cache -> ops.reshape_and_cache) and "Code Example".
+ *
+ * For every new token t with s = slot_mapping[t] >= 0, for every KV head h:
+ *     key_cache  [s / block_size, s % block_size, h, :] = key  [t, h, :]
+ *     value_cache[s / block_size, s % block_size, h, :] = value[t, h, :]
+ * as a raw copy of the 16-bit words (bit-exact).  A negative slot marks a
+ * padding token and writes nothing.
+ *
+ *  key, value      [num_tokens, num_kv_heads, head_dim]; rows are
+ *                  key_stride_t / value_stride_t ELEMENTS apart (heads and
+ *                  head_dim contiguous inside a row).
+ *  key_cache, value_cache  the pools (layout above), num_blocks blocks.
+ *  slot_mapping    int32 [num_tokens], flat slot = block * block_size + offset.
+ *  dtype           PA_F16 or PA_BF16 (both sides hold the same type).
+ *  kv_cache_dtype  PA_KV_AUTO only; k_scale / v_scale are accepted and
+ *                  ignored under AUTO (may be NULL).
+ * Errors: PA_ERR_INVALID_ARG for null pointers or non-positive sizes;
+ * PA_ERR_UNSUPPORTED for kv_cache_dtype != AUTO or dtype F32.  A slot at or
+ * beyond num_blocks*block_size is skipped and flagged PA_DEVERR_BAD_SLOT.
+ * Two tokens with the same slot: the surviving row is unspecified.
+ * ------------------------------------------------------------------------- */
+pa_status pa_reshape_and_cache(const void* key, const void* value,
+                               int64_t key_stride_t, int64_t value_stride_t,
+                               void* key_cache, void* value_cache,
+                               const int32_t* slot_mapping, int32_t num_tokens,
+                               int32_t num_blocks, int32_t block_size,
+                               int32_t num_kv_heads, int32_t head_dim,
+                               pa_dtype dtype, pa_kv_cache_dtype kv_cache_dtype,
+                               const float* k_scale, const float* v_scale,
+                               int32_t* device_error_flag, pa_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * pa_copy_blocks -- copy-on-write, [PA] "Sharing and copy-on-write" and "How
+ * does copy-on-write work for parallel sampling?" ([KV] "Shared prompts and
+ * continuous batching").
+ *
+ * For each pair i, block_mapping[2i] = src, block_mapping[2i+1] = dst:
+ * block dst of every listed K and V pool becomes a byte copy of block src
+ * (the whole block, so dst is bit-identical to src).
+ *
+ *  key_caches, value_caches  HOST arrays of num_layers DEVICE pointers.
+ *  block_mapping   int32 device [num_pairs, 2].
+ *  block_bytes     bytes of one block of one pool
+ *                  (block_size * num_kv_heads * head_dim * element size).
+ * Preconditions (caller's): dst ids are distinct and no id is both a src and
+ * a dst in the same call; otherwise the result is unspecified.
+ * Errors: PA_ERR_INVALID_ARG for null pointers or non-positive sizes; a pair
+ * with an id outside [0, num_blocks) is skipped and flagged PA_DEVERR_BAD_SLOT.
+ * ------------------------------------------------------------------------- */
+pa_status pa_copy_blocks(void* const* key_caches, void* const* value_caches,
+                         int32_t num_layers, const int32_t* block_mapping,
+                         int32_t num_pairs, int32_t num_blocks,
+                         int64_t block_bytes, int32_t* device_error_flag,
+                         pa_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * pa_decode_workspace_bytes -- device scratch that pa_decode_attention needs
+ * for the given shape: per-sequence work prefix sums and the split-KV
+ * partials (o, m, l) in fp32.  Depends on the SM count of the CURRENT device.
+ * partition_size as in pa_decode_attention.  Writes the size to *bytes.
+ * ------------------------------------------------------------------------- */
+pa_status pa_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads,
+                                    int32_t num_kv_heads, int32_t head_dim,
+                                    int32_t block_size, int32_t max_seq_len,
+                                    int32_t partition_size, size_t* bytes);
+
+/* ---------------------------------------------------------------------------
+ * pa_decode_attention -- paged decode attention with split-KV and a combine
+ * pass.  [PA] "How attention reads paged memory": for each query token, walk
+ * the sequence's block table (logical block i -> physical block id), gather
+ * each block's keys and values from the pool, and run attention over them
+ * with an online softmax.  One query token per sequence:
+ *
+ *   out[b, h, :] = sum_t softmax_t(scale * <query[b, h, :], K_b[t]>) V_b[t]
+ *
+ * over t < seq_lens[b], where K_b[t] = key_cache[table[b][t / bs], t % bs,
+ * h / (Hq / Hkv), :] (query heads grouped consecutively onto KV heads).
+ *
+ *  out             [num_seqs, num_q_heads, head_dim], out_dtype (F16, BF16
+ *                  or F32), contiguous.  A sequence with seq_len 0 gets zeros.
+ *  query           [num_seqs, num_q_heads, head_dim], kv_dtype, contiguous.
+ *  block_tables    int32 [num_seqs, block_table_stride], row-major; entries
+ *                  past ceil(seq_len / block_size) are never read.
+ *  seq_lens        int32 [num_seqs], device; each in [0, max_seq_len].
+ *  max_seq_len     host-side upper bound of seq_lens (sizes the workspace).
+ *  scale           softmax scale (e.g. 1/sqrt(head_dim)).
+ *  kv_dtype        PA_F16 or PA_BF16 (query, K and V share it).
+ *  partition_size  0: automatic split of the whole batch's work into equal
+ *                  shares per SM; > 0: in addition no partial covers more
+ *                  than partition_size tokens (a multiple of 16 and of
+ *                  block_size).  Partials are merged by the combine pass.
+ *  workspace       device scratch of at least pa_decode_workspace_bytes(),
+ *                  256-byte aligned; contents need no initialisation.
+ * Built shapes: head_dim 64 or 128; block_size 4..128 (power of two);
+ * num_q_heads / num_kv_heads <= 8.  Other shapes: PA_ERR_UNSUPPORTED.
+ * Errors: PA_ERR_INVALID_ARG for null pointers, num_q_heads % num_kv_heads,
+ * block_table_stride < ceil(max_seq_len / block_size), a partition_size that
+ * is not block aligned, misaligned pointers or a small workspace.  On the
+ * device, a table entry outside [0, num_blocks) is flagged
+ * PA_DEVERR_BAD_BLOCK and its tokens are left out of the softmax.
+ * ------------------------------------------------------------------------- */
+pa_status pa_decode_attention(void* out, pa_dtype out_dtype, const void* query,
+                              const void* key_cache, const void* value_cache,
+                              const int32_t* block_tables,
+                              int32_t block_table_stride,
+                              const int32_t* seq_lens, int32_t num_seqs,
+                              int32_t max_seq_len, int32_t num_q_heads,
+                              int32_t num_kv_heads, int32_t head_dim,
+                              int32_t num_blocks, int32_t block_size,
+                              float scale, pa_dtype kv_dtype,
+                              int32_t partition_size, void* workspace,
+                              size_t workspace_bytes,
+                              int32_t* device_error_flag, pa_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Host block manager -- [PA] "The idea: page the KV cache" (allocate a block
+ * when the previous one is full, from a free list, from anywhere in memory),
+ * "Sharing and copy-on-write" (per-block reference counts; full blocks are
+ * never written again) and "How does copy-on-write work for parallel
+ * sampling?" (allocate, copy, decrement, write into the copy).
+ *
+ * Host-only, not thread-safe (one manager per scheduler thread).  Block ids
+ * leave the free list in `free_order` (a permutation of [0, num_blocks);
+ * NULL = 0, 1, 2, ...); freed blocks go to its back.  Sequence ids are any
+ * int64 values chosen by the caller.
+ * ------------------------------------------------------------------------- */
+typedef struct pa_block_manager pa_block_manager;
+
+pa_status pa_bm_create(int32_t num_blocks, int32_t block_size,
+                       const int32_t* free_order, pa_block_manager** out);
+void pa_bm_destroy(pa_block_manager* bm);
+/* A new sequence that already holds num_tokens tokens: ceil(n / bs) blocks. */
+pa_status pa_bm_add_sequence(pa_block_manager* bm, int64_t seq, int64_t num_tokens);
+/* child shares all of parent's blocks (each refcount + 1). */
+pa_status pa_bm_fork(pa_block_manager* bm, int64_t parent, int64_t child);
+/* Reserve the slot of seq's next token.  *slot gets the flat slot; if the
+ * last block was shared and partially filled, a copy-on-write happened and
+ * (*cow_src, *cow_dst) name the copy the device must make first (else -1). */
+pa_status pa_bm_append_slot(pa_block_manager* bm, int64_t seq, int64_t* slot,
+                            int32_t* cow_src, int32_t* cow_dst);
+pa_status pa_bm_free_sequence(pa_block_manager* bm, int64_t seq);
+/* Copies at most `capacity` entries of seq's table to `out` (host);
+ * *num_blocks gets the table length, *num_tokens the sequence length. */
+pa_status pa_bm_block_table(const pa_block_manager* bm, int64_t seq,
+                            int32_t* out, int32_t capacity,
+                            int32_t* num_blocks, int64_t* num_tokens);
+/* Reference count of a physical block (-1 if out of range). */
+int32_t pa_bm_refcount(const pa_block_manager* bm, int32_t block);
+int32_t pa_bm_num_free(const pa_block_manager* bm);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAGEDATTN_H_ */

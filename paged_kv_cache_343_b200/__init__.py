@@ -1,0 +1,333 @@
+"""paged_kv_cache_343_b200 -- Python binding of libpagedattn.so.
+
+The library is the product: hand-written sm_100a CUDA kernels behind a C ABI
+(``include/pagedattn.h``).  This module only marshals arguments: it turns
+torch tensors into pointers, sizes and the current CUDA stream, calls the C
+entry point of the same name and raises on a non-OK status.  Every step of
+the hot path runs in the library's kernels; there is no fallback.  Importing
+this package fails loudly if the library has not been built
+(``python -m paged_kv_cache_343_b200.build``).
+
+Entry points (see the header for argument meaning, layout and errors):
+
+* ``reshape_and_cache`` -- scatter new K/V rows into pool slots
+  ("How PagedAttention Works in vLLM ...", "write_to_paged_cache").
+* ``copy_blocks``       -- copy-on-write block copies ("PagedAttention",
+  "How does copy-on-write work for parallel sampling?").
+* ``decode_attention``  -- paged decode attention with split-KV partials and a
+  combine pass ("PagedAttention", "How attention reads paged memory").
+* ``BlockManager``      -- the native host block manager (free list,
+  refcounts, copy-on-write planning).
+* ``PagedDecodeStep``   -- one decode step from pinned host buffers: copies in,
+  the two kernels, copy out (the end-to-end call).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+import torch
+
+__all__ = [
+    "LIB_PATH", "PagedAttnError", "reshape_and_cache", "copy_blocks", "decode_attention",
+    "decode_workspace_bytes", "BlockManager", "PagedDecodeStep", "DEVERR_BAD_BLOCK",
+    "DEVERR_BAD_SLOT", "DEVERR_BAD_SEQLEN", "DEVERR_TIMEOUT", "version",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpagedattn.so")
+
+DEVERR_BAD_BLOCK = 0x1
+DEVERR_BAD_SLOT = 0x2
+DEVERR_BAD_SEQLEN = 0x4
+DEVERR_TIMEOUT = 0x8
+
+_PA_F16, _PA_BF16, _PA_F32 = 0, 1, 2
+_DTYPE_CODE = {torch.float16: _PA_F16, torch.bfloat16: _PA_BF16, torch.float32: _PA_F32}
+
+
+class PagedAttnError(RuntimeError):
+    """A libpagedattn entry point returned a status other than PA_OK."""
+
+    def __init__(self, what: str, status: int, name: str):
+        super().__init__("%s failed: %s (%d)" % (what, name, status))
+        self.status = status
+        self.name = name
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError("libpagedattn.so is missing at %s; build it with "
+                          "`python -m paged_kv_cache_343_b200.build`" % LIB_PATH)
+    lib = ctypes.CDLL(LIB_PATH)
+    i32, i64, p, sz = ctypes.c_int32, ctypes.c_int64, ctypes.c_void_p, ctypes.c_size_t
+    lib.pa_status_string.restype = ctypes.c_char_p
+    lib.pa_status_string.argtypes = [ctypes.c_int]
+    lib.pa_version.restype = i32
+    lib.pa_version.argtypes = []
+    lib.pa_reshape_and_cache.restype = ctypes.c_int
+    lib.pa_reshape_and_cache.argtypes = [p, p, i64, i64, p, p, p, i32, i32, i32, i32, i32,
+                                         ctypes.c_int, ctypes.c_int, p, p, p, p]
+    lib.pa_copy_blocks.restype = ctypes.c_int
+    lib.pa_copy_blocks.argtypes = [p, p, i32, p, i32, i32, i64, p, p]
+    lib.pa_decode_workspace_bytes.restype = ctypes.c_int
+    lib.pa_decode_workspace_bytes.argtypes = [i32, i32, i32, i32, i32, i32, i32,
+                                              ctypes.POINTER(sz)]
+    lib.pa_decode_attention.restype = ctypes.c_int
+    lib.pa_decode_attention.argtypes = [p, ctypes.c_int, p, p, p, p, i32, p, i32, i32, i32, i32,
+                                        i32, i32, i32, ctypes.c_float, ctypes.c_int, i32, p, sz,
+                                        p, p]
+    lib.pa_bm_create.restype = ctypes.c_int
+    lib.pa_bm_create.argtypes = [i32, i32, p, ctypes.POINTER(p)]
+    lib.pa_bm_destroy.restype = None
+    lib.pa_bm_destroy.argtypes = [p]
+    lib.pa_bm_add_sequence.restype = ctypes.c_int
+    lib.pa_bm_add_sequence.argtypes = [p, i64, i64]
+    lib.pa_bm_fork.restype = ctypes.c_int
+    lib.pa_bm_fork.argtypes = [p, i64, i64]
+    lib.pa_bm_append_slot.restype = ctypes.c_int
+    lib.pa_bm_append_slot.argtypes = [p, i64, ctypes.POINTER(i64), ctypes.POINTER(i32),
+                                      ctypes.POINTER(i32)]
+    lib.pa_bm_free_sequence.restype = ctypes.c_int
+    lib.pa_bm_free_sequence.argtypes = [p, i64]
+    lib.pa_bm_block_table.restype = ctypes.c_int
+    lib.pa_bm_block_table.argtypes = [p, i64, p, i32, ctypes.POINTER(i32), ctypes.POINTER(i64)]
+    lib.pa_bm_refcount.restype = i32
+    lib.pa_bm_refcount.argtypes = [p, i32]
+    lib.pa_bm_num_free.restype = i32
+    lib.pa_bm_num_free.argtypes = [p]
+    return lib
+
+
+lib = _load()
+
+
+def version() -> int:
+    return int(lib.pa_version())
+
+
+def _check(status: int, what: str) -> None:
+    if status != 0:
+        raise PagedAttnError(what, status, lib.pa_status_string(status).decode())
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_handle(stream: Optional[torch.cuda.Stream]):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need(cond: bool, msg: str) -> None:
+    if not cond:
+        raise ValueError(msg)
+
+
+def reshape_and_cache(key: torch.Tensor, value: torch.Tensor, key_cache: torch.Tensor,
+                      value_cache: torch.Tensor, slot_mapping: torch.Tensor,
+                      kv_cache_dtype: str = "auto", k_scale: Optional[torch.Tensor] = None,
+                      v_scale: Optional[torch.Tensor] = None,
+                      error_flag: Optional[torch.Tensor] = None,
+                      stream: Optional[torch.cuda.Stream] = None) -> None:
+    """key/value [T, Hkv, D] (rows may be strided), caches [nb, bs, Hkv, D], slot_mapping int32 [T]."""
+    _need(kv_cache_dtype == "auto", "only kv_cache_dtype='auto' is built")
+    _need(key.dim() == 3 and value.shape == key.shape, "key/value must be [T, Hkv, D]")
+    _need(key.stride(2) == 1 and key.stride(1) == key.shape[2] and
+          value.stride(2) == 1 and value.stride(1) == value.shape[2],
+          "heads and head_dim must be contiguous inside a row")
+    _need(key_cache.is_contiguous() and value_cache.is_contiguous(), "caches must be contiguous")
+    _need(slot_mapping.dtype == torch.int32 and slot_mapping.is_contiguous(), "slot_mapping int32")
+    _need(key.dtype == key_cache.dtype == value.dtype == value_cache.dtype, "dtype mismatch")
+    nb, bs, hkv, d = key_cache.shape
+    _check(lib.pa_reshape_and_cache(
+        _ptr(key), _ptr(value), key.stride(0), value.stride(0), _ptr(key_cache),
+        _ptr(value_cache), _ptr(slot_mapping), key.shape[0], nb, bs, hkv, d,
+        _DTYPE_CODE[key.dtype], 0, _ptr(k_scale), _ptr(v_scale), _ptr(error_flag),
+        _stream_handle(stream)), "pa_reshape_and_cache")
+
+
+def copy_blocks(key_caches: Sequence[torch.Tensor], value_caches: Sequence[torch.Tensor],
+                block_mapping: torch.Tensor, error_flag: Optional[torch.Tensor] = None,
+                stream: Optional[torch.cuda.Stream] = None) -> None:
+    """block_mapping int32 [N, 2] (src, dst) on the device; one K and one V pool per layer."""
+    _need(len(key_caches) == len(value_caches) and len(key_caches) > 0, "one K and V pool per layer")
+    _need(block_mapping.dtype == torch.int32 and block_mapping.is_contiguous(), "mapping int32 [N,2]")
+    k0 = key_caches[0]
+    block_bytes = k0[0].numel() * k0.element_size()
+    for c in list(key_caches) + list(value_caches):
+        _need(c.is_contiguous() and c.shape == k0.shape and c.dtype == k0.dtype, "pool shapes differ")
+    n = len(key_caches)
+    karr = (ctypes.c_void_p * n)(*[c.data_ptr() for c in key_caches])
+    varr = (ctypes.c_void_p * n)(*[c.data_ptr() for c in value_caches])
+    _check(lib.pa_copy_blocks(ctypes.cast(karr, ctypes.c_void_p), ctypes.cast(varr, ctypes.c_void_p),
+                              n, _ptr(block_mapping), block_mapping.numel() // 2, k0.shape[0],
+                              block_bytes, _ptr(error_flag), _stream_handle(stream)),
+           "pa_copy_blocks")
+
+
+def decode_workspace_bytes(num_seqs: int, num_q_heads: int, num_kv_heads: int, head_dim: int,
+                           block_size: int, max_seq_len: int, partition_size: int = 0) -> int:
+    out = ctypes.c_size_t(0)
+    _check(lib.pa_decode_workspace_bytes(num_seqs, num_q_heads, num_kv_heads, head_dim,
+                                         block_size, max_seq_len, partition_size,
+                                         ctypes.byref(out)), "pa_decode_workspace_bytes")
+    return int(out.value)
+
+
+def alloc_workspace(nbytes: int, device) -> torch.Tensor:
+    """A device buffer of nbytes, 256-byte aligned (torch's allocator aligns to 512)."""
+    return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+
+
+def decode_attention(out: torch.Tensor, query: torch.Tensor, key_cache: torch.Tensor,
+                     value_cache: torch.Tensor, block_tables: torch.Tensor,
+                     seq_lens: torch.Tensor, max_seq_len: int, scale: float,
+                     partition_size: int = 0, workspace: Optional[torch.Tensor] = None,
+                     error_flag: Optional[torch.Tensor] = None,
+                     stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """out/query [B, Hq, D]; caches [nb, bs, Hkv, D]; block_tables int32 [B, W]; seq_lens int32 [B]."""
+    _need(query.dim() == 3 and query.is_contiguous(), "query must be contiguous [B, Hq, D]")
+    _need(out.shape == query.shape and out.is_contiguous(), "out must be contiguous [B, Hq, D]")
+    _need(key_cache.is_contiguous() and value_cache.is_contiguous(), "caches must be contiguous")
+    _need(key_cache.shape == value_cache.shape, "K and V pools differ")
+    _need(block_tables.dtype == torch.int32 and block_tables.dim() == 2 and
+          block_tables.stride(1) == 1, "block_tables int32 [B, W], rows contiguous")
+    _need(seq_lens.dtype == torch.int32 and seq_lens.is_contiguous(), "seq_lens int32")
+    _need(query.dtype == key_cache.dtype == value_cache.dtype, "query and caches share a dtype")
+    B, hq, d = query.shape
+    nb, bs, hkv, _ = key_cache.shape
+    if workspace is None:
+        workspace = alloc_workspace(decode_workspace_bytes(B, hq, hkv, d, bs, max_seq_len,
+                                                           partition_size), query.device)
+    _check(lib.pa_decode_attention(
+        _ptr(out), _DTYPE_CODE[out.dtype], _ptr(query), _ptr(key_cache), _ptr(value_cache),
+        _ptr(block_tables), block_tables.stride(0), _ptr(seq_lens), B, int(max_seq_len), hq, hkv,
+        d, nb, bs, float(scale), _DTYPE_CODE[query.dtype], int(partition_size), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _ptr(error_flag), _stream_handle(stream)),
+        "pa_decode_attention")
+    return out
+
+
+class BlockManager:
+    """Native host block manager (pa_bm_*): free list, refcounts, copy-on-write."""
+
+    def __init__(self, num_blocks: int, block_size: int, free_order=None):
+        self.block_size = int(block_size)
+        self.num_blocks = int(num_blocks)
+        h = ctypes.c_void_p()
+        if free_order is not None:
+            order = torch.as_tensor(free_order, dtype=torch.int32).contiguous()
+            _check(lib.pa_bm_create(num_blocks, block_size, _ptr(order), ctypes.byref(h)),
+                   "pa_bm_create")
+        else:
+            _check(lib.pa_bm_create(num_blocks, block_size, None, ctypes.byref(h)), "pa_bm_create")
+        self._h = h
+
+    def __del__(self):
+        h = getattr(self, "_h", None)
+        if h is not None and h.value:
+            lib.pa_bm_destroy(h)
+            self._h = None
+
+    def add_sequence(self, seq: int, num_tokens: int) -> None:
+        _check(lib.pa_bm_add_sequence(self._h, seq, num_tokens), "pa_bm_add_sequence")
+
+    def fork(self, parent: int, child: int) -> None:
+        _check(lib.pa_bm_fork(self._h, parent, child), "pa_bm_fork")
+
+    def append_slot(self, seq: int):
+        slot = ctypes.c_int64()
+        src, dst = ctypes.c_int32(), ctypes.c_int32()
+        _check(lib.pa_bm_append_slot(self._h, seq, ctypes.byref(slot), ctypes.byref(src),
+                                     ctypes.byref(dst)), "pa_bm_append_slot")
+        return int(slot.value), (None if src.value < 0 else (int(src.value), int(dst.value)))
+
+    def free_sequence(self, seq: int) -> None:
+        _check(lib.pa_bm_free_sequence(self._h, seq), "pa_bm_free_sequence")
+
+    def block_table(self, seq: int):
+        n = ctypes.c_int32()
+        toks = ctypes.c_int64()
+        _check(lib.pa_bm_block_table(self._h, seq, None, 0, ctypes.byref(n), ctypes.byref(toks)),
+               "pa_bm_block_table")
+        buf = (ctypes.c_int32 * max(1, n.value))()
+        _check(lib.pa_bm_block_table(self._h, seq, ctypes.cast(buf, ctypes.c_void_p), n.value,
+                                     ctypes.byref(n), ctypes.byref(toks)), "pa_bm_block_table")
+        return [int(buf[i]) for i in range(n.value)]
+
+    def seq_len(self, seq: int) -> int:
+        n = ctypes.c_int32()
+        toks = ctypes.c_int64()
+        _check(lib.pa_bm_block_table(self._h, seq, None, 0, ctypes.byref(n), ctypes.byref(toks)),
+               "pa_bm_block_table")
+        return int(toks.value)
+
+    def refcount(self, block: int) -> int:
+        return int(lib.pa_bm_refcount(self._h, block))
+
+    def num_free(self) -> int:
+        return int(lib.pa_bm_num_free(self._h))
+
+    def tables(self, seqs: Sequence[int], width: int) -> torch.Tensor:
+        """int32 [len(seqs), width] host tensor of block tables, padded with -1."""
+        t = torch.full((len(seqs), width), -1, dtype=torch.int32)
+        for i, s in enumerate(seqs):
+            row = self.block_table(s)
+            t[i, :len(row)] = torch.tensor(row, dtype=torch.int32)
+        return t
+
+
+class PagedDecodeStep:
+    """One decode step driven from pinned host memory (the end-to-end call).
+
+    Holds device buffers for a fixed batch shape.  ``__call__`` copies the
+    step's inputs host->device (query, new K/V rows, slot_mapping, block
+    tables, seq_lens), writes the new rows into the pools with
+    reshape_and_cache, runs decode_attention, and copies the output back
+    device->host, all on one stream, then waits for it."""
+
+    def __init__(self, key_cache: torch.Tensor, value_cache: torch.Tensor, num_seqs: int,
+                 num_q_heads: int, table_width: int, max_seq_len: int, scale: float,
+                 partition_size: int = 0, out_dtype: Optional[torch.dtype] = None,
+                 stream: Optional[torch.cuda.Stream] = None):
+        self.k, self.v = key_cache, value_cache
+        nb, bs, hkv, d = key_cache.shape
+        dev = key_cache.device
+        dt = key_cache.dtype
+        self.shape = (num_seqs, num_q_heads, d)
+        self.max_seq_len, self.scale, self.partition_size = max_seq_len, scale, partition_size
+        self.stream = stream if stream is not None else torch.cuda.Stream(device=dev)
+        self.q = torch.empty(self.shape, dtype=dt, device=dev)
+        self.new_k = torch.empty((num_seqs, hkv, d), dtype=dt, device=dev)
+        self.new_v = torch.empty((num_seqs, hkv, d), dtype=dt, device=dev)
+        self.slots = torch.empty(num_seqs, dtype=torch.int32, device=dev)
+        self.tables = torch.empty((num_seqs, table_width), dtype=torch.int32, device=dev)
+        self.lens = torch.empty(num_seqs, dtype=torch.int32, device=dev)
+        self.out = torch.empty(self.shape, dtype=out_dtype or dt, device=dev)
+        self.ws = alloc_workspace(decode_workspace_bytes(num_seqs, num_q_heads, hkv, d, bs,
+                                                         max_seq_len, partition_size), dev)
+
+    def h2d_bytes(self) -> int:
+        return sum(t.numel() * t.element_size()
+                   for t in (self.q, self.new_k, self.new_v, self.slots, self.tables, self.lens))
+
+    def d2h_bytes(self) -> int:
+        return self.out.numel() * self.out.element_size()
+
+    def __call__(self, q_host, new_k_host, new_v_host, slots_host, tables_host, lens_host,
+                 out_host) -> None:
+        s = self.stream
+        with torch.cuda.stream(s):
+            self.q.copy_(q_host, non_blocking=True)
+            self.new_k.copy_(new_k_host, non_blocking=True)
+            self.new_v.copy_(new_v_host, non_blocking=True)
+            self.slots.copy_(slots_host, non_blocking=True)
+            self.tables.copy_(tables_host, non_blocking=True)
+            self.lens.copy_(lens_host, non_blocking=True)
+            reshape_and_cache(self.new_k, self.new_v, self.k, self.v, self.slots, stream=s)
+            decode_attention(self.out, self.q, self.k, self.v, self.tables, self.lens,
+                             self.max_seq_len, self.scale, self.partition_size, self.ws, stream=s)
+            out_host.copy_(self.out, non_blocking=True)
+        s.synchronize()

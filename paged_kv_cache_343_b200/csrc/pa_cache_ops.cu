@@ -1,0 +1,175 @@
+// pa_cache_ops.cu -- the two cache-maintenance kernels of the hot path.
+//
+// reshape_and_cache ("How PagedAttention Works in vLLM to Maximize Memory
+// Efficiency", "write_to_paged_cache: Direct In-Place Updates"): new K/V rows
+// go straight into their pool slots, no staging buffer.  With the pool laid
+// out [num_blocks, block_size, Hkv, D], slot s = block * block_size + offset
+// starts s * Hkv * D elements into the pool, so each token is one contiguous
+// row copy of Hkv * D 16-bit words for K and one for V.
+//
+// copy_blocks ("PagedAttention", "How does copy-on-write work for parallel
+// sampling?"): the copy step of copy-on-write, a whole physical block per
+// (src, dst) pair and pool.
+#include <cuda_runtime.h>
+
+#include "pa_device.cuh"
+#include "pa_host.h"
+
+namespace pa {
+
+constexpr int kRowThreads = 128;
+constexpr int kCopyThreads = 256;
+constexpr int kMaxCopyCaches = 128;  // pointers per copy_blocks launch (64 layers of K and V)
+
+template <int VEC>
+struct Vec;
+template <>
+struct Vec<8> {
+  using T = uint4;
+};
+template <>
+struct Vec<1> {
+  using T = uint16_t;
+};
+
+// One CTA per token (grid-stride); the block's threads split the K and V rows.
+template <int VEC>
+__global__ void __launch_bounds__(kRowThreads)
+    pa_reshape_and_cache_kernel(const uint16_t* __restrict__ key,
+                                const uint16_t* __restrict__ value, int64_t key_stride,
+                                int64_t value_stride, uint16_t* __restrict__ key_cache,
+                                uint16_t* __restrict__ value_cache,
+                                const int32_t* __restrict__ slot_mapping, int32_t num_tokens,
+                                int64_t num_slots, int32_t row_elems, int32_t* err) {
+  using T = typename Vec<VEC>::T;
+  const int32_t nvec = row_elems / VEC;
+  for (int64_t t = blockIdx.x; t < num_tokens; t += gridDim.x) {
+    const int64_t slot = slot_mapping[t];
+    if (slot < 0) continue;  // padding token
+    if (slot >= num_slots) {
+      if (threadIdx.x == 0) flag_error(err, PA_DEVERR_BAD_SLOT);
+      continue;
+    }
+    const T* ks = reinterpret_cast<const T*>(key + t * key_stride);
+    const T* vs = reinterpret_cast<const T*>(value + t * value_stride);
+    T* kd = reinterpret_cast<T*>(key_cache + slot * row_elems);
+    T* vd = reinterpret_cast<T*>(value_cache + slot * row_elems);
+    for (int32_t i = threadIdx.x; i < 2 * nvec; i += kRowThreads) {
+      if (i < nvec) {
+        kd[i] = ks[i];
+      } else {
+        vd[i - nvec] = vs[i - nvec];
+      }
+    }
+  }
+}
+
+struct CopyPtrs {
+  uint8_t* p[kMaxCopyCaches];
+};
+
+// grid (num_pairs, num_caches): one CTA copies one block of one pool.
+template <bool kVec16>
+__global__ void __launch_bounds__(kCopyThreads)
+    pa_copy_blocks_kernel(const CopyPtrs ptrs, const int32_t* __restrict__ mapping,
+                          int32_t num_blocks, int64_t block_bytes, int32_t* err) {
+  const int64_t pair = blockIdx.x;
+  const int32_t src = mapping[2 * pair], dst = mapping[2 * pair + 1];
+  if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) {
+    if (threadIdx.x == 0 && blockIdx.y == 0) flag_error(err, PA_DEVERR_BAD_SLOT);
+    return;
+  }
+  uint8_t* base = ptrs.p[blockIdx.y];
+  if constexpr (kVec16) {
+    const uint4* s = reinterpret_cast<const uint4*>(base + src * block_bytes);
+    uint4* d = reinterpret_cast<uint4*>(base + dst * block_bytes);
+    const int64_t n = block_bytes / 16;
+    for (int64_t i = threadIdx.x; i < n; i += kCopyThreads) d[i] = s[i];
+  } else {
+    const uint8_t* s = base + src * block_bytes;
+    uint8_t* d = base + dst * block_bytes;
+    for (int64_t i = threadIdx.x; i < block_bytes; i += kCopyThreads) d[i] = s[i];
+  }
+}
+
+}  // namespace pa
+
+using namespace pa;
+
+extern "C" pa_status pa_reshape_and_cache(const void* key, const void* value,
+                                          int64_t key_stride_t, int64_t value_stride_t,
+                                          void* key_cache, void* value_cache,
+                                          const int32_t* slot_mapping, int32_t num_tokens,
+                                          int32_t num_blocks, int32_t block_size,
+                                          int32_t num_kv_heads, int32_t head_dim,
+                                          pa_dtype dtype, pa_kv_cache_dtype kv_cache_dtype,
+                                          const float* k_scale, const float* v_scale,
+                                          int32_t* device_error_flag, pa_stream_t stream) {
+  (void)k_scale;
+  (void)v_scale;
+  if (num_tokens < 0 || num_blocks <= 0 || block_size <= 0 || num_kv_heads <= 0 ||
+      head_dim <= 0)
+    return PA_ERR_INVALID_ARG;
+  if (dtype != PA_F16 && dtype != PA_BF16) return PA_ERR_UNSUPPORTED;
+  if (kv_cache_dtype != PA_KV_AUTO) return PA_ERR_UNSUPPORTED;
+  if (num_tokens == 0) return PA_OK;
+  if (!key || !value || !key_cache || !value_cache || !slot_mapping) return PA_ERR_INVALID_ARG;
+  const int64_t row = static_cast<int64_t>(num_kv_heads) * head_dim;
+  if (row > INT32_MAX || key_stride_t < row || value_stride_t < row) return PA_ERR_INVALID_ARG;
+  if (!aligned(key, 2) || !aligned(value, 2) || !aligned(key_cache, 2) ||
+      !aligned(value_cache, 2) || !aligned(slot_mapping, 4))
+    return PA_ERR_INVALID_ARG;
+  const int64_t num_slots = static_cast<int64_t>(num_blocks) * block_size;
+  const bool vec = aligned(key, 16) && aligned(value, 16) && aligned(key_cache, 16) &&
+                   aligned(value_cache, 16) && key_stride_t % 8 == 0 &&
+                   value_stride_t % 8 == 0 && row % 8 == 0;
+  const int grid = num_tokens < (1 << 20) ? num_tokens : (1 << 20);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (vec) {
+    pa_reshape_and_cache_kernel<8><<<grid, kRowThreads, 0, s>>>(
+        static_cast<const uint16_t*>(key), static_cast<const uint16_t*>(value), key_stride_t,
+        value_stride_t, static_cast<uint16_t*>(key_cache), static_cast<uint16_t*>(value_cache),
+        slot_mapping, num_tokens, num_slots, static_cast<int32_t>(row), device_error_flag);
+  } else {
+    pa_reshape_and_cache_kernel<1><<<grid, kRowThreads, 0, s>>>(
+        static_cast<const uint16_t*>(key), static_cast<const uint16_t*>(value), key_stride_t,
+        value_stride_t, static_cast<uint16_t*>(key_cache), static_cast<uint16_t*>(value_cache),
+        slot_mapping, num_tokens, num_slots, static_cast<int32_t>(row), device_error_flag);
+  }
+  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+extern "C" pa_status pa_copy_blocks(void* const* key_caches, void* const* value_caches,
+                                    int32_t num_layers, const int32_t* block_mapping,
+                                    int32_t num_pairs, int32_t num_blocks, int64_t block_bytes,
+                                    int32_t* device_error_flag, pa_stream_t stream) {
+  if (num_layers < 0 || num_pairs < 0 || num_blocks <= 0 || block_bytes <= 0)
+    return PA_ERR_INVALID_ARG;
+  if (num_layers == 0 || num_pairs == 0) return PA_OK;
+  if (!key_caches || !value_caches || !block_mapping || !aligned(block_mapping, 4))
+    return PA_ERR_INVALID_ARG;
+  bool vec = block_bytes % 16 == 0;
+  for (int32_t l = 0; l < num_layers; ++l) {
+    if (!key_caches[l] || !value_caches[l]) return PA_ERR_INVALID_ARG;
+    vec = vec && aligned(key_caches[l], 16) && aligned(value_caches[l], 16);
+  }
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int layers_per_launch = kMaxCopyCaches / 2;
+  for (int32_t l0 = 0; l0 < num_layers; l0 += layers_per_launch) {
+    const int32_t nl = num_layers - l0 < layers_per_launch ? num_layers - l0 : layers_per_launch;
+    CopyPtrs ptrs;
+    for (int32_t l = 0; l < nl; ++l) {
+      ptrs.p[2 * l] = static_cast<uint8_t*>(key_caches[l0 + l]);
+      ptrs.p[2 * l + 1] = static_cast<uint8_t*>(value_caches[l0 + l]);
+    }
+    const dim3 grid(num_pairs, 2 * nl);
+    if (vec) {
+      pa_copy_blocks_kernel<true><<<grid, kCopyThreads, 0, s>>>(ptrs, block_mapping, num_blocks,
+                                                                 block_bytes, device_error_flag);
+    } else {
+      pa_copy_blocks_kernel<false><<<grid, kCopyThreads, 0, s>>>(ptrs, block_mapping, num_blocks,
+                                                                  block_bytes, device_error_flag);
+    }
+  }
+  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}

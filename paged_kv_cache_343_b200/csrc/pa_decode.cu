@@ -1,0 +1,828 @@
+// pa_decode.cu -- paged decode attention for sm_100a ("PagedAttention",
+// section "How attention reads paged memory": for each query token walk the
+// sequence's block table, gather each block's keys and values from the shared
+// pool and run attention over them with an online softmax).
+//
+// Three launches per call, all on the caller's stream:
+//   1. plan     (1 CTA)   per-sequence prefix sums of 16-token tiles and of
+//                         partitions, written to the workspace;
+//   2. main     (1 CTA per SM and head group, persistent)  the batch's tiles
+//                         laid end to end are cut into equal shares, one per
+//                         CTA; a producer warp streams each tile's K and V
+//                         from the pool into shared memory with 5-D TMA loads
+//                         (one block-table lookup per block), and one consumer
+//                         warp per KV head computes S^T = K Q^T and
+//                         O^T += V^T P^T on the tensor cores (grouped query
+//                         heads packed into the MMA's N dimension) with an
+//                         fp32 online softmax;
+//   3. combine            merges the (o, m, l) partials of every sequence
+//                         whose tiles were split across CTAs or partitions.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <climits>
+#include <cstring>
+#include <mutex>
+
+#include "pa_device.cuh"
+#include "pa_host.h"
+
+namespace pa {
+
+constexpr int kTile = 16;            // tokens per tile (MMA M of the score product)
+constexpr int kPlanThreads = 1024;
+constexpr int kCombineWarps = 4;
+
+enum : int32_t {
+  kNewSeq = 1,    // first tile of a sequence in this CTA: reload Q
+  kSegStart = 2,  // reset the online-softmax state
+  kSegEnd = 4,    // finalise and write the segment
+  kDirect = 8,    // the segment is the whole sequence: write `out` directly
+};
+
+struct TileInfo {
+  int32_t b;       // sequence
+  int32_t valid;   // tokens of this tile inside the sequence (1..16)
+  int32_t mask;    // bit t set: token t takes part (valid and its block id is good)
+  int32_t seg;     // segment id inside this head group
+  int32_t flags;
+  int32_t pad[3];
+};
+
+struct DecodeParams {
+  void* out;
+  const uint16_t* query;
+  const int32_t* block_tables;
+  const int32_t* seq_lens;
+  int64_t table_stride;
+  int32_t out_dtype;
+  int32_t num_seqs, max_seq_len, num_q_heads, group, num_blocks, block_size;
+  int32_t tiles_per_part;  // partition length in tiles (INT_MAX: no partitions)
+  float scale_log2;        // scale * log2(e)
+  int32_t ctas_per_group;  // CTAs sharing one head group's tiles
+  int32_t heads_per_cta;   // KV heads per CTA (HG)
+  int32_t nseg_cap;        // partial slots per head group
+  int32_t stages;
+  int32_t tok_box;         // tokens per TMA box: min(block_size, 16)
+  int32_t tma_mode;        // 0: one box per block per tile, 1: one per (head, d-half)
+  int32_t* plan_tiles;     // [num_seqs + 1]
+  int32_t* plan_parts;     // [num_seqs + 1]
+  float* part_o;           // [groups][nseg_cap][HG * group][head_dim]
+  float* part_ml;          // [groups][nseg_cap][HG * group][2]  (m in log2 units, l)
+  int32_t* err;
+};
+
+__device__ __forceinline__ int32_t clamp_len(int32_t L, int32_t max_len) {
+  return L < 0 ? 0 : (L > max_len ? max_len : L);
+}
+
+// CTA whose share [c*N/C, (c+1)*N/C) holds global tile t.
+__device__ __forceinline__ int32_t cta_of_tile(int64_t t, int64_t N, int64_t C) {
+  return static_cast<int32_t>(((t + 1) * C - 1) / N);
+}
+
+// ---------------------------------------------------------------------------
+// plan: tiles[b] = sum_{b'<b} ceil(L_b'/16); parts[b] = sum_{b'<b} max(1, ceil(n_b'/tpp))
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kPlanThreads) pa_plan_kernel(DecodeParams p) {
+  __shared__ int32_t warp_t[kPlanThreads / 32], warp_p[kPlanThreads / 32];
+  __shared__ int32_t carry[2];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (tid == 0) carry[0] = carry[1] = 0;
+  __syncthreads();
+  for (int base = 0; base < p.num_seqs; base += kPlanThreads) {
+    const int b = base + tid;
+    int32_t nt = 0, np = 0;
+    if (b < p.num_seqs) {
+      const int32_t raw = p.seq_lens[b];
+      if (raw < 0 || raw > p.max_seq_len) flag_error(p.err, PA_DEVERR_BAD_SEQLEN);
+      const int32_t L = clamp_len(raw, p.max_seq_len);
+      nt = (L + kTile - 1) / kTile;
+      np = nt == 0 ? 1 : (p.tiles_per_part == INT_MAX ? 1 : (nt + p.tiles_per_part - 1) / p.tiles_per_part);
+    }
+    int32_t it = nt, ip = np;  // inclusive warp scan
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int32_t vt = __shfl_up_sync(0xffffffffu, it, o);
+      const int32_t vp = __shfl_up_sync(0xffffffffu, ip, o);
+      if (lane >= o) { it += vt; ip += vp; }
+    }
+    if (lane == 31) { warp_t[warp] = it; warp_p[warp] = ip; }
+    __syncthreads();
+    if (warp == 0) {
+      int32_t wt = warp_t[lane], wp = warp_p[lane];
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int32_t vt = __shfl_up_sync(0xffffffffu, wt, o);
+        const int32_t vp = __shfl_up_sync(0xffffffffu, wp, o);
+        if (lane >= o) { wt += vt; wp += vp; }
+      }
+      warp_t[lane] = wt;  // inclusive over warps
+      warp_p[lane] = wp;
+    }
+    __syncthreads();
+    const int32_t before_t = carry[0] + (warp > 0 ? warp_t[warp - 1] : 0);
+    const int32_t before_p = carry[1] + (warp > 0 ? warp_p[warp - 1] : 0);
+    if (b < p.num_seqs) {
+      p.plan_tiles[b] = before_t + it - nt;
+      p.plan_parts[b] = before_p + ip - np;
+    }
+    __syncthreads();
+    if (tid == 0) {
+      carry[0] += warp_t[kPlanThreads / 32 - 1];
+      carry[1] += warp_p[kPlanThreads / 32 - 1];
+    }
+    __syncthreads();
+  }
+  if (tid == 0) {
+    p.plan_tiles[p.num_seqs] = carry[0];
+    p.plan_parts[p.num_seqs] = carry[1];
+  }
+}
+
+// ---------------------------------------------------------------------------
+// main kernel
+// ---------------------------------------------------------------------------
+template <int D, int HG, bool kBF16>
+__global__ void __launch_bounds__((HG + 1) * 32, 1)
+    pa_decode_main_kernel(const __grid_constant__ CUtensorMap tmK,
+                          const __grid_constant__ CUtensorMap tmV, const DecodeParams p) {
+  constexpr int DC = D / 64;                       // 128-byte column chunks of a row
+  constexpr int KSTEPS = D / 16;                   // k16 steps of S^T = K Q^T
+  constexpr int MTILES = D / 16;                   // m16 tiles of O^T = V^T P^T
+  constexpr uint32_t kTileBytes = kTile * HG * D * 2;  // K (or V) bytes per stage
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const int NS = p.stages;
+  TileInfo* info = reinterpret_cast<TileInfo*>(smem + static_cast<size_t>(NS) * 2 * kTileBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(info + NS);
+  const uint32_t smem_base = smem_u32(smem);
+  const uint32_t bar_base = smem_u32(bars);
+  auto full_k = [&](int s) { return bar_base + 8u * s; };
+  auto full_v = [&](int s) { return bar_base + 8u * (NS + s); };
+  auto empty = [&](int s) { return bar_base + 8u * (2 * NS + s); };
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int hg = blockIdx.y;
+  const int64_t C = p.ctas_per_group;
+  const int c = blockIdx.x;
+  const int B = p.num_seqs;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(full_k(s), 1);
+      mbar_init(full_v(s), 1);
+      mbar_init(empty(s), HG);
+    }
+    fence_mbar_init();
+  }
+  if (warp == HG && lane == 0) {
+    prefetch_tmap(&tmK);
+    prefetch_tmap(&tmV);
+  }
+  __syncthreads();
+
+  const int64_t N = p.plan_tiles[B];
+  const int64_t lo = static_cast<int64_t>(c) * N / C;
+  const int64_t hi = static_cast<int64_t>(c + 1) * N / C;
+  if (lo >= hi) return;
+
+  // first sequence with tiles[b + 1] > lo
+  int b0;
+  {
+    int l = 0, r = B - 1;
+    while (l < r) {
+      const int mid = (l + r) >> 1;
+      if (p.plan_tiles[mid + 1] > lo) r = mid; else l = mid + 1;
+    }
+    b0 = l;
+  }
+
+  if (warp == HG) {
+    // ======================= producer =======================
+    if (lane != 0) return;
+    const uint64_t policy = l2_policy_evict_first();
+    const int bs = p.block_size;
+    const int TB = p.tok_box;
+    const uint32_t box_bytes = static_cast<uint32_t>(HG * DC * TB * 128);
+    const int bpt = bs < kTile ? kTile / bs : 1;  // blocks per tile
+    int b = b0;
+    int32_t t_first = p.plan_tiles[b];
+    int32_t n_b = p.plan_tiles[b + 1] - t_first;
+    int32_t L_b = clamp_len(p.seq_lens[b], p.max_seq_len);
+    int32_t parts_b = p.plan_parts[b];
+    int32_t nparts_b = p.plan_parts[b + 1] - parts_b;
+    const int32_t* row = p.block_tables + static_cast<int64_t>(b) * p.table_stride;
+    int32_t i = static_cast<int32_t>(lo - t_first);
+    bool new_seq = true;
+    int stage = 0;
+    uint32_t phase = 0;
+    int64_t issued = 0;
+    for (int64_t t = lo; t < hi; ++t, ++i) {
+      while (i >= n_b) {  // next sequence that has tiles
+        ++b;
+        t_first = p.plan_tiles[b];
+        n_b = p.plan_tiles[b + 1] - t_first;
+        L_b = clamp_len(p.seq_lens[b], p.max_seq_len);
+        parts_b = p.plan_parts[b];
+        nparts_b = p.plan_parts[b + 1] - parts_b;
+        row = p.block_tables + static_cast<int64_t>(b) * p.table_stride;
+        i = 0;
+        new_seq = true;
+      }
+      if (!mbar_wait(empty(stage), phase ^ 1u, p.err)) break;
+
+      const int32_t valid = min(kTile, L_b - i * kTile);
+      const int32_t j = (p.tiles_per_part == INT_MAX) ? 0 : i / p.tiles_per_part;
+      const int64_t part_lo = t_first + static_cast<int64_t>(j) *
+                                            (p.tiles_per_part == INT_MAX ? 0 : p.tiles_per_part);
+      const int64_t part_hi = (p.tiles_per_part == INT_MAX)
+                                  ? t_first + n_b
+                                  : min(static_cast<int64_t>(t_first) + n_b,
+                                        part_lo + p.tiles_per_part);
+      const int64_t seg_lo = max(part_lo, lo), seg_hi = min(part_hi, hi);
+      int32_t flags = 0;
+      if (new_seq) flags |= kNewSeq;
+      if (t == seg_lo) flags |= kSegStart;
+      if (t == seg_hi - 1) flags |= kSegEnd;
+      if (nparts_b == 1 && seg_lo == t_first && seg_hi == t_first + n_b) flags |= kDirect;
+      new_seq = false;
+
+      uint32_t mask = valid >= kTile ? 0xffffu : ((1u << valid) - 1u);
+      // block-table lookups first, so the expected byte count is known
+      int32_t phys[kTile / 4];
+      int32_t tok_off[kTile / 4];
+      int nbox = 0;
+      uint32_t bytes = 0;
+      if (bs <= kTile) {
+        for (int k = 0; k < bpt; ++k) {
+          const int tok0 = k * bs;
+          if (tok0 >= valid) break;
+          const int32_t id = __ldg(row + static_cast<int64_t>(i) * bpt + k);
+          if (id < 0 || id >= p.num_blocks) {
+            flag_error(p.err, PA_DEVERR_BAD_BLOCK);
+            mask &= ~(((1u << bs) - 1u) << tok0);
+            phys[k] = -1;
+            continue;
+          }
+          phys[k] = id;
+          tok_off[k] = 0;
+          nbox = k + 1;
+          bytes += box_bytes;
+        }
+      } else {
+        const int64_t tok = static_cast<int64_t>(i) * kTile;
+        const int32_t id = __ldg(row + tok / bs);
+        tok_off[0] = static_cast<int32_t>(tok % bs);
+        if (id < 0 || id >= p.num_blocks) {
+          flag_error(p.err, PA_DEVERR_BAD_BLOCK);
+          mask = 0;
+          phys[0] = -1;
+        } else {
+          phys[0] = id;
+          nbox = 1;
+          bytes = box_bytes;
+        }
+      }
+      TileInfo& ti = info[stage];
+      ti.b = b;
+      ti.valid = valid;
+      ti.mask = static_cast<int32_t>(mask);
+      ti.seg = parts_b + j + c;
+      ti.flags = flags;
+      mbar_arrive_expect_tx(full_k(stage), bytes);
+      mbar_arrive_expect_tx(full_v(stage), bytes);
+      const uint32_t kdst = smem_base + static_cast<uint32_t>(stage) * 2u * kTileBytes;
+      const uint32_t vdst = kdst + kTileBytes;
+      for (int k = 0; k < nbox; ++k) {
+        if (phys[k] < 0) continue;
+        if (p.tma_mode == 0) {
+          tma_load_5d(kdst + k * box_bytes, &tmK, full_k(stage), 0, tok_off[k], 0, hg * HG,
+                      phys[k], policy);
+          tma_load_5d(vdst + k * box_bytes, &tmV, full_v(stage), 0, tok_off[k], 0, hg * HG,
+                      phys[k], policy);
+        } else {
+          for (int hh = 0; hh < HG; ++hh) {
+            for (int dc = 0; dc < DC; ++dc) {
+              const uint32_t off = k * box_bytes + ((hh * DC + dc) * TB) * 128u;
+              tma_load_5d(kdst + off, &tmK, full_k(stage), 0, dc, hg * HG + hh, tok_off[k],
+                          phys[k], policy);
+              tma_load_5d(vdst + off, &tmV, full_v(stage), 0, dc, hg * HG + hh, tok_off[k],
+                          phys[k], policy);
+            }
+          }
+        }
+      }
+      ++issued;
+      if (++stage == NS) { stage = 0; phase ^= 1u; }
+    }
+    // Wait (bounded) until every load this warp issued has landed, so that no
+    // copy is in flight into shared memory when the CTA retires.
+    for (int64_t k = (issued > NS ? issued - NS : 0); k < issued; ++k) {
+      const int s = static_cast<int>(k % NS);
+      const uint32_t par = static_cast<uint32_t>((k / NS) & 1);
+      if (!mbar_wait(full_k(s), par, p.err)) break;
+      if (!mbar_wait(full_v(s), par, p.err)) break;
+    }
+    return;
+  }
+
+  // ======================= consumers: one warp per KV head =======================
+  const int g = warp;                         // KV head inside the group
+  const int kvh = hg * HG + g;                // KV head
+  const int G = p.group;
+  const int HGq = HG * G;                     // query heads of this CTA's group
+  const int quad = lane & 3, grp = lane >> 2;
+  const int TB = p.tok_box;
+  const int tb_shift = TB == 16 ? 4 : (TB == 8 ? 3 : 2);
+
+  // Per-lane row indices of the ldmatrix addresses (see the layout note in
+  // the producer: rows of 128 bytes ordered [box][head][d-chunk][token]).
+  auto row_of = [&](int tok, int dc) {
+    return ((tok >> tb_shift) * HG * DC + g * DC + dc) * TB + (tok & (TB - 1));
+  };
+  const int mi = lane >> 3, rr = lane & 7;
+  const int k_tok = rr + 8 * (mi & 1), k_chunk = mi >> 1;   // K: non-transposed
+  const int v_tok = rr + 8 * (mi >> 1), v_chunk = mi & 1;   // V: transposed
+  int k_row[DC], v_row[DC];
+#pragma unroll
+  for (int dc = 0; dc < DC; ++dc) {
+    k_row[dc] = row_of(k_tok, dc);
+    v_row[dc] = row_of(v_tok, dc);
+  }
+
+  uint32_t qf[KSTEPS][2];
+  float acc[MTILES][4];
+  float m_run[2], l_part[2];
+  int stage = 0;
+  uint32_t phase = 0;
+  const float sl2 = p.scale_log2;
+
+  for (int64_t t = lo; t < hi; ++t) {
+    if (!mbar_wait(full_k(stage), phase, p.err)) break;
+    const TileInfo ti = info[stage];
+    if (ti.flags & kNewSeq) {
+      const uint16_t* qb = p.query + (static_cast<int64_t>(ti.b) * p.num_q_heads + kvh * G) * D;
+#pragma unroll
+      for (int kc = 0; kc < KSTEPS; ++kc) {
+        if (grp < G) {
+          const uint16_t* qp = qb + grp * D + kc * 16 + quad * 2;
+          qf[kc][0] = *reinterpret_cast<const uint32_t*>(qp);
+          qf[kc][1] = *reinterpret_cast<const uint32_t*>(qp + 8);
+        } else {
+          qf[kc][0] = 0u;
+          qf[kc][1] = 0u;
+        }
+      }
+    }
+    if (ti.flags & kSegStart) {
+#pragma unroll
+      for (int mt = 0; mt < MTILES; ++mt)
+        acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
+      m_run[0] = m_run[1] = -INFINITY;
+      l_part[0] = l_part[1] = 0.f;
+    }
+    const uint32_t kbase = smem_base + static_cast<uint32_t>(stage) * 2u * kTileBytes;
+    const uint32_t vbase = kbase + kTileBytes;
+
+    // ---- S^T[16 tok x 8 heads] = K[16 x D] * Q^T[D x 8]
+    float s[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int kc = 0; kc < KSTEPS; ++kc) {
+      const int dc = kc >> 2;
+      const int r = k_row[dc];
+      const uint32_t chunk = static_cast<uint32_t>((2 * (kc & 3) + k_chunk) ^ (r & 7));
+      uint32_t a0, a1, a2, a3;
+      ldmatrix_x4(kbase + static_cast<uint32_t>(r) * 128u + chunk * 16u, a0, a1, a2, a3);
+      mma_16816<kBF16>(s, a0, a1, a2, a3, qf[kc][0], qf[kc][1]);
+    }
+    // ---- online softmax (base 2), masked by selection
+    const uint32_t mask = static_cast<uint32_t>(ti.mask);
+    const bool ok0 = (mask >> grp) & 1u, ok1 = (mask >> (grp + 8)) & 1u;
+    s[0] = ok0 ? s[0] * sl2 : -INFINITY;
+    s[1] = ok0 ? s[1] * sl2 : -INFINITY;
+    s[2] = ok1 ? s[2] * sl2 : -INFINITY;
+    s[3] = ok1 ? s[3] * sl2 : -INFINITY;
+    float mx0 = fmaxf(s[0], s[2]), mx1 = fmaxf(s[1], s[3]);
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+    }
+    const float mn0 = fmaxf(m_run[0], mx0), mn1 = fmaxf(m_run[1], mx1);
+    const float alpha0 = (mn0 == m_run[0]) ? 1.f : ex2(m_run[0] - mn0);
+    const float alpha1 = (mn1 == m_run[1]) ? 1.f : ex2(m_run[1] - mn1);
+    m_run[0] = mn0;
+    m_run[1] = mn1;
+    const float p0 = (s[0] == -INFINITY) ? 0.f : ex2(s[0] - mn0);
+    const float p1 = (s[1] == -INFINITY) ? 0.f : ex2(s[1] - mn1);
+    const float p2 = (s[2] == -INFINITY) ? 0.f : ex2(s[2] - mn0);
+    const float p3 = (s[3] == -INFINITY) ? 0.f : ex2(s[3] - mn1);
+    // P in two 16-bit halves, P = hi + lo, so the P.V product keeps about
+    // 16 significant bits of every weight instead of the storage type's 8 or 11.
+    const uint32_t pt0 = pack2<kBF16>(p0, p1);  // P^T row grp     (heads 2q, 2q+1)
+    const uint32_t pt1 = pack2<kBF16>(p2, p3);  // P^T row grp + 8
+    const uint32_t pl0 = pack2<kBF16>(p0 - lo_to_float<kBF16>(pt0), p1 - hi_to_float<kBF16>(pt0));
+    const uint32_t pl1 = pack2<kBF16>(p2 - lo_to_float<kBF16>(pt1), p3 - hi_to_float<kBF16>(pt1));
+    l_part[0] = l_part[0] * alpha0 + (p0 + p2);
+    l_part[1] = l_part[1] * alpha1 + (p1 + p3);
+    if (__any_sync(0xffffffffu, alpha0 != 1.f || alpha1 != 1.f)) {
+#pragma unroll
+      for (int mt = 0; mt < MTILES; ++mt) {
+        acc[mt][0] *= alpha0;
+        acc[mt][1] *= alpha1;
+        acc[mt][2] *= alpha0;
+        acc[mt][3] *= alpha1;
+      }
+    }
+    // P^T as the B operand (k = token, n = head): transpose the 8x8 halves
+    const uint32_t pb0 = movmatrix_trans(pt0);
+    const uint32_t pb1 = movmatrix_trans(pt1);
+    const uint32_t pc0 = movmatrix_trans(pl0);
+    const uint32_t pc1 = movmatrix_trans(pl1);
+
+    // ---- O^T[D x 8] += V^T[D x 16 tok] * P^T[16 tok x 8]
+    if (!mbar_wait(full_v(stage), phase, p.err)) break;
+    const bool partial = mask != 0xffffu;
+    uint32_t z01 = 0xffffffffu, z23 = 0xffffffffu;
+    if (partial) {
+      const int tk = 2 * quad;
+      z01 = (((mask >> tk) & 1u) ? 0x0000ffffu : 0u) | (((mask >> (tk + 1)) & 1u) ? 0xffff0000u : 0u);
+      z23 = (((mask >> (tk + 8)) & 1u) ? 0x0000ffffu : 0u) |
+            (((mask >> (tk + 9)) & 1u) ? 0xffff0000u : 0u);
+    }
+#pragma unroll
+    for (int mt = 0; mt < MTILES; ++mt) {
+      const int dc = mt >> 2;
+      const int r = v_row[dc];
+      const uint32_t chunk = static_cast<uint32_t>((2 * (mt & 3) + v_chunk) ^ (r & 7));
+      uint32_t a0, a1, a2, a3;
+      ldmatrix_x4_trans(vbase + static_cast<uint32_t>(r) * 128u + chunk * 16u, a0, a1, a2, a3);
+      // masked tokens may hold anything (NaN included): zero them, never multiply
+      a0 &= z01;
+      a1 &= z01;
+      a2 &= z23;
+      a3 &= z23;
+      mma_16816<kBF16>(acc[mt], a0, a1, a2, a3, pb0, pb1);
+      mma_16816<kBF16>(acc[mt], a0, a1, a2, a3, pc0, pc1);
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(empty(stage));
+    if (++stage == NS) { stage = 0; phase ^= 1u; }
+
+    if (ti.flags & kSegEnd) {
+      float l0 = l_part[0], l1 = l_part[1];
+#pragma unroll
+      for (int o = 4; o < 32; o <<= 1) {
+        l0 += __shfl_xor_sync(0xffffffffu, l0, o);
+        l1 += __shfl_xor_sync(0xffffffffu, l1, o);
+      }
+      const float inv0 = l0 > 0.f ? 1.f / l0 : 0.f;
+      const float inv1 = l1 > 0.f ? 1.f / l1 : 0.f;
+      const int h0 = 2 * quad, h1 = h0 + 1;
+      if (ti.flags & kDirect) {
+        const int64_t obase = (static_cast<int64_t>(ti.b) * p.num_q_heads + kvh * G) * D;
+#pragma unroll
+        for (int mt = 0; mt < MTILES; ++mt) {
+          const int d = mt * 16 + grp;
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            const int h = hh ? h1 : h0;
+            if (h >= G) continue;
+            const float inv = hh ? inv1 : inv0;
+            const float v0 = acc[mt][hh] * inv, v1 = acc[mt][2 + hh] * inv;
+            const int64_t o = obase + static_cast<int64_t>(h) * D + d;
+            if (p.out_dtype == PA_F32) {
+              float* op = static_cast<float*>(p.out);
+              op[o] = v0;
+              op[o + 8] = v1;
+            } else if (p.out_dtype == PA_BF16) {
+              __nv_bfloat16* op = static_cast<__nv_bfloat16*>(p.out);
+              op[o] = __float2bfloat16_rn(v0);
+              op[o + 8] = __float2bfloat16_rn(v1);
+            } else {
+              __half* op = static_cast<__half*>(p.out);
+              op[o] = __float2half_rn(v0);
+              op[o + 8] = __float2half_rn(v1);
+            }
+          }
+        }
+      } else if (ti.seg < p.nseg_cap) {
+        const int64_t sbase = static_cast<int64_t>(hg) * p.nseg_cap + ti.seg;
+        float* po = p.part_o + (sbase * HGq + g * G) * D;
+#pragma unroll
+        for (int mt = 0; mt < MTILES; ++mt) {
+          const int d = mt * 16 + grp;
+          if (h0 < G) {
+            po[h0 * D + d] = acc[mt][0] * inv0;
+            po[h0 * D + d + 8] = acc[mt][2] * inv0;
+          }
+          if (h1 < G) {
+            po[h1 * D + d] = acc[mt][1] * inv1;
+            po[h1 * D + d + 8] = acc[mt][3] * inv1;
+          }
+        }
+        if (grp == 0) {
+          float* pm = p.part_ml + (sbase * HGq + g * G) * 2;
+          if (h0 < G) {
+            pm[h0 * 2] = l0 > 0.f ? m_run[0] : -INFINITY;
+            pm[h0 * 2 + 1] = l0;
+          }
+          if (h1 < G) {
+            pm[h1 * 2] = l1 > 0.f ? m_run[1] : -INFINITY;
+            pm[h1 * 2 + 1] = l1;
+          }
+        }
+      } else {
+        flag_error(p.err, PA_DEVERR_BAD_SEQLEN);
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// combine: out[b, h] = sum_j w_j o_j / sum_j w_j,  w_j = l_j 2^(m_j - M)
+// grid (B, ceil(Hq / kCombineWarps)), one warp per query head
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(kCombineWarps * 32) pa_combine_kernel(const DecodeParams p) {
+  constexpr int V = D / 32;  // floats per lane
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int b = blockIdx.x;
+  const int qh = blockIdx.y * kCombineWarps + warp;
+  if (qh >= p.num_q_heads) return;
+  const int G = p.group, HG = p.heads_per_cta;
+  const int kvh = qh / G, hg = kvh / HG;
+  const int HGq = HG * G;
+  const int qloc = qh - hg * HGq;
+  const int64_t C = p.ctas_per_group;
+  const int64_t N = p.plan_tiles[p.num_seqs];
+  const int32_t t0 = p.plan_tiles[b], t1 = p.plan_tiles[b + 1];
+  const int32_t pp0 = p.plan_parts[b], npart = p.plan_parts[b + 1] - pp0;
+  const int64_t obase = (static_cast<int64_t>(b) * p.num_q_heads + qh) * D + lane * V;
+
+  float acc[V];
+#pragma unroll
+  for (int k = 0; k < V; ++k) acc[k] = 0.f;
+  float M = -INFINITY, Wsum = 0.f;
+  if (t1 > t0) {
+    if (npart == 1 && cta_of_tile(t0, N, C) == cta_of_tile(t1 - 1, N, C)) return;  // written by main
+    const int64_t tpp = (p.tiles_per_part == INT_MAX) ? (t1 - t0) : p.tiles_per_part;
+    for (int32_t j = 0; j < npart; ++j) {
+      const int64_t a = t0 + j * tpp;
+      const int64_t e = min(static_cast<int64_t>(t1), a + tpp);
+      const int32_t c0 = cta_of_tile(a, N, C), c1 = cta_of_tile(e - 1, N, C);
+      for (int32_t cc = c0; cc <= c1; ++cc) {
+        if (cc * N / C == (cc + 1) * N / C) continue;  // a CTA with an empty share wrote nothing
+        const int64_t seg = pp0 + j + cc;
+        if (seg >= p.nseg_cap) continue;
+        const int64_t sidx = (static_cast<int64_t>(hg) * p.nseg_cap + seg) * HGq + qloc;
+        const float m = p.part_ml[sidx * 2];
+        const float l = p.part_ml[sidx * 2 + 1];
+        if (!(l > 0.f)) continue;
+        const float* po = p.part_o + sidx * D + lane * V;
+        float o[V];
+        if constexpr (V == 4) {
+          const float4 v = *reinterpret_cast<const float4*>(po);
+          o[0] = v.x; o[1] = v.y; o[2] = v.z; o[3] = v.w;
+        } else {
+          const float2 v = *reinterpret_cast<const float2*>(po);
+          o[0] = v.x; o[1] = v.y;
+        }
+        if (m > M) {
+          const float r = (M == -INFINITY) ? 0.f : ex2(M - m);
+#pragma unroll
+          for (int k = 0; k < V; ++k) acc[k] *= r;
+          Wsum *= r;
+          M = m;
+        }
+        const float w = l * ex2(m - M);
+#pragma unroll
+        for (int k = 0; k < V; ++k) acc[k] += w * o[k];
+        Wsum += w;
+      }
+    }
+  }
+  const float inv = Wsum > 0.f ? 1.f / Wsum : 0.f;
+#pragma unroll
+  for (int k = 0; k < V; ++k) {
+    const float v = acc[k] * inv;
+    if (p.out_dtype == PA_F32) {
+      static_cast<float*>(p.out)[obase + k] = v;
+    } else if (p.out_dtype == PA_BF16) {
+      static_cast<__nv_bfloat16*>(p.out)[obase + k] = __float2bfloat16_rn(v);
+    } else {
+      static_cast<__half*>(p.out)[obase + k] = __float2half_rn(v);
+    }
+  }
+}
+
+// ===========================================================================
+// host side
+// ===========================================================================
+namespace {
+
+using MainKernel = void (*)(const CUtensorMap, const CUtensorMap, const DecodeParams);
+
+template <int D, int HG, bool BF>
+MainKernel main_kernel_ptr() {
+  return pa_decode_main_kernel<D, HG, BF>;
+}
+
+MainKernel select_main(int D, int HG, bool bf16) {
+#define PA_SEL(d, hg)                                                      \
+  if (D == d && HG == hg) return bf16 ? main_kernel_ptr<d, hg, true>()     \
+                                      : main_kernel_ptr<d, hg, false>();
+  PA_SEL(64, 1) PA_SEL(64, 2) PA_SEL(64, 4) PA_SEL(64, 8)
+  PA_SEL(128, 1) PA_SEL(128, 2) PA_SEL(128, 4) PA_SEL(128, 8)
+#undef PA_SEL
+  return nullptr;
+}
+
+struct LaunchPlan {
+  int HG = 0, groups = 0, stages = 0, tok_box = 0, threads = 0;
+  int ctas_per_group = 0, tiles_per_part = INT_MAX, nseg_cap = 0;
+  size_t smem = 0;
+  size_t off_tiles = 0, off_parts = 0, off_o = 0, off_ml = 0, total = 0;
+  MainKernel kernel = nullptr;
+};
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
+
+pa_status make_plan(int32_t num_seqs, int32_t Hq, int32_t Hkv, int32_t D, int32_t bs,
+                    int32_t max_seq_len, int32_t partition_size, bool bf16, LaunchPlan* lp) {
+  if (num_seqs < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || bs <= 0 || max_seq_len < 0 ||
+      partition_size < 0)
+    return PA_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return PA_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return PA_ERR_UNSUPPORTED;
+  if (!is_pow2(bs) || bs < 4 || bs > 128) return PA_ERR_UNSUPPORTED;
+  const int G = Hq / Hkv;
+  if (G > 8) return PA_ERR_UNSUPPORTED;
+  if (partition_size > 0 && (partition_size % kTile != 0 || partition_size % bs != 0))
+    return PA_ERR_INVALID_ARG;
+  int HG = 8;
+  while (Hkv % HG != 0) HG >>= 1;
+  const int DC = D / 64;
+  const int TB = bs < kTile ? bs : kTile;
+  if ((HG * DC * TB * 128) % 1024 != 0) return PA_ERR_UNSUPPORTED;
+  lp->HG = HG;
+  lp->groups = Hkv / HG;
+  lp->tok_box = TB;
+  lp->threads = (HG + 1) * 32;
+  const size_t tile_bytes = static_cast<size_t>(kTile) * HG * D * 2;
+  const size_t budget = 200 * 1024;
+  int stages = static_cast<int>(budget / (2 * tile_bytes));
+  if (stages > 6) stages = 6;
+  if (stages < 2) return PA_ERR_UNSUPPORTED;
+  lp->stages = stages;
+  lp->smem = 1024 + static_cast<size_t>(stages) * 2 * tile_bytes + stages * sizeof(TileInfo) +
+             3 * stages * sizeof(uint64_t);
+  lp->kernel = select_main(D, HG, bf16);
+  if (lp->kernel == nullptr) return PA_ERR_UNSUPPORTED;
+
+  const DeviceInfo* dev = current_device_info();
+  if (dev == nullptr) return PA_ERR_CUDA;
+  if (!ensure_smem_attr(reinterpret_cast<const void*>(lp->kernel), lp->smem)) return PA_ERR_CUDA;
+  const int per_sm = ctas_per_sm(reinterpret_cast<const void*>(lp->kernel), lp->threads, lp->smem);
+  if (per_sm < 1) return PA_ERR_CUDA;
+  const int total_ctas = dev->num_sms * per_sm;
+  lp->ctas_per_group = total_ctas / lp->groups > 0 ? total_ctas / lp->groups : 1;
+
+  const int64_t max_tiles = (static_cast<int64_t>(max_seq_len) + kTile - 1) / kTile;
+  int64_t parts_per_seq = 1;
+  if (partition_size > 0) {
+    lp->tiles_per_part = partition_size / kTile;
+    parts_per_seq = (max_tiles + lp->tiles_per_part - 1) / lp->tiles_per_part;
+    if (parts_per_seq < 1) parts_per_seq = 1;
+  }
+  const int64_t nseg = static_cast<int64_t>(num_seqs) * parts_per_seq + lp->ctas_per_group;
+  if (nseg > INT_MAX / 2) return PA_ERR_UNSUPPORTED;
+  lp->nseg_cap = static_cast<int>(nseg);
+  lp->off_tiles = 0;
+  lp->off_parts = align_up(static_cast<size_t>(num_seqs + 1) * 4, 256);
+  lp->off_o = lp->off_parts + align_up(static_cast<size_t>(num_seqs + 1) * 4, 256);
+  const size_t o_bytes = static_cast<size_t>(lp->groups) * nseg * HG * G * D * sizeof(float);
+  lp->off_ml = lp->off_o + align_up(o_bytes, 256);
+  const size_t ml_bytes = static_cast<size_t>(lp->groups) * nseg * HG * G * 2 * sizeof(float);
+  lp->total = lp->off_ml + align_up(ml_bytes, 256);
+  return PA_OK;
+}
+
+}  // namespace
+}  // namespace pa
+
+using namespace pa;
+
+extern "C" pa_status pa_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads,
+                                               int32_t num_kv_heads, int32_t head_dim,
+                                               int32_t block_size, int32_t max_seq_len,
+                                               int32_t partition_size, size_t* bytes) {
+  if (bytes == nullptr) return PA_ERR_INVALID_ARG;
+  LaunchPlan lp;
+  const pa_status st = make_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
+                                 max_seq_len, partition_size, true, &lp);
+  if (st != PA_OK) return st;
+  *bytes = lp.total;
+  return PA_OK;
+}
+
+extern "C" pa_status pa_decode_attention(
+    void* out, pa_dtype out_dtype, const void* query, const void* key_cache,
+    const void* value_cache, const int32_t* block_tables, int32_t block_table_stride,
+    const int32_t* seq_lens, int32_t num_seqs, int32_t max_seq_len, int32_t num_q_heads,
+    int32_t num_kv_heads, int32_t head_dim, int32_t num_blocks, int32_t block_size, float scale,
+    pa_dtype kv_dtype, int32_t partition_size, void* workspace, size_t workspace_bytes,
+    int32_t* device_error_flag, pa_stream_t stream) {
+  if (num_seqs < 0) return PA_ERR_INVALID_ARG;
+  if (num_seqs == 0) return PA_OK;
+  if (!out || !query || !key_cache || !value_cache || !block_tables || !seq_lens || !workspace)
+    return PA_ERR_INVALID_ARG;
+  if (kv_dtype != PA_F16 && kv_dtype != PA_BF16) return PA_ERR_UNSUPPORTED;
+  if (out_dtype != PA_F16 && out_dtype != PA_BF16 && out_dtype != PA_F32)
+    return PA_ERR_INVALID_ARG;
+  if (num_blocks <= 0 || !(scale == scale)) return PA_ERR_INVALID_ARG;
+  LaunchPlan lp;
+  pa_status st = make_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
+                           max_seq_len, partition_size, kv_dtype == PA_BF16, &lp);
+  if (st != PA_OK) return st;
+  const int64_t need_blocks = (static_cast<int64_t>(max_seq_len) + block_size - 1) / block_size;
+  if (block_table_stride < need_blocks) return PA_ERR_INVALID_ARG;
+  if (workspace_bytes < lp.total) return PA_ERR_INVALID_ARG;
+  if (!aligned(key_cache, 16) || !aligned(value_cache, 16) || !aligned(query, 16) ||
+      !aligned(workspace, 256) || !aligned(out, out_dtype == PA_F32 ? 4 : 2) ||
+      !aligned(block_tables, 4) || !aligned(seq_lens, 4))
+    return PA_ERR_INVALID_ARG;
+
+  const int HG = lp.HG, D = head_dim, DC = D / 64;
+  const uint64_t e = 2;
+  CUtensorMap tmK, tmV;
+  int mode = 0;
+  {
+    // mode 0: dims {64 d, tokens, d-chunks, heads, blocks}, box {64, TB, DC, HG, 1}
+    const uint64_t dims0[5] = {64, (uint64_t)block_size, (uint64_t)DC, (uint64_t)num_kv_heads,
+                               (uint64_t)num_blocks};
+    const uint64_t str0[4] = {num_kv_heads * D * e, 128, D * e, block_size * num_kv_heads * D * e};
+    const uint32_t box0[5] = {64, (uint32_t)lp.tok_box, (uint32_t)DC, (uint32_t)HG, 1};
+    // mode 1: dims {64 d, d-chunks, heads, tokens, blocks}, box {64, 1, 1, TB, 1}
+    const uint64_t dims1[5] = {64, (uint64_t)DC, (uint64_t)num_kv_heads, (uint64_t)block_size,
+                               (uint64_t)num_blocks};
+    const uint64_t str1[4] = {128, D * e, num_kv_heads * D * e, block_size * num_kv_heads * D * e};
+    const uint32_t box1[5] = {64, 1, 1, (uint32_t)lp.tok_box, 1};
+    if (get_tensor_map(&tmK, key_cache, dims0, str0, box0) &&
+        get_tensor_map(&tmV, value_cache, dims0, str0, box0)) {
+      mode = 0;
+    } else if (lp.tok_box * 128 % 1024 == 0 && get_tensor_map(&tmK, key_cache, dims1, str1, box1) &&
+               get_tensor_map(&tmV, value_cache, dims1, str1, box1)) {
+      mode = 1;
+    } else {
+      return PA_ERR_UNSUPPORTED;
+    }
+  }
+
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  DecodeParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.out = out;
+  p.query = static_cast<const uint16_t*>(query);
+  p.block_tables = block_tables;
+  p.seq_lens = seq_lens;
+  p.table_stride = block_table_stride;
+  p.out_dtype = out_dtype;
+  p.num_seqs = num_seqs;
+  p.max_seq_len = max_seq_len;
+  p.num_q_heads = num_q_heads;
+  p.group = num_q_heads / num_kv_heads;
+  p.num_blocks = num_blocks;
+  p.block_size = block_size;
+  p.tiles_per_part = lp.tiles_per_part;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.ctas_per_group = lp.ctas_per_group;
+  p.heads_per_cta = HG;
+  p.nseg_cap = lp.nseg_cap;
+  p.stages = lp.stages;
+  p.tok_box = lp.tok_box;
+  p.tma_mode = mode;
+  p.plan_tiles = reinterpret_cast<int32_t*>(ws + lp.off_tiles);
+  p.plan_parts = reinterpret_cast<int32_t*>(ws + lp.off_parts);
+  p.part_o = reinterpret_cast<float*>(ws + lp.off_o);
+  p.part_ml = reinterpret_cast<float*>(ws + lp.off_ml);
+  p.err = device_error_flag;
+
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  pa_plan_kernel<<<1, kPlanThreads, 0, s>>>(p);
+  lp.kernel<<<dim3(lp.ctas_per_group, lp.groups), lp.threads, lp.smem, s>>>(tmK, tmV, p);
+  const dim3 cgrid(num_seqs, (num_q_heads + kCombineWarps - 1) / kCombineWarps);
+  if (D == 128) {
+    pa_combine_kernel<128><<<cgrid, kCombineWarps * 32, 0, s>>>(p);
+  } else {
+    pa_combine_kernel<64><<<cgrid, kCombineWarps * 32, 0, s>>>(p);
+  }
+  if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
+  return PA_OK;
+}

@@ -1,0 +1,43 @@
+// pa_host.h -- host-side helpers shared by the library's entry points:
+// per-device attributes, dynamic shared-memory opt-in, alignment checks and a
+// small cache of TMA tensor descriptors keyed by pool address and shape.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstddef>
+#include <cstdint>
+
+#include "../../include/pagedattn.h"
+
+namespace pa {
+
+struct DeviceInfo {
+  int device = -1;
+  int num_sms = 0;
+  int max_smem_optin = 0;
+  int l2_bytes = 0;
+};
+
+// Attributes of the current device (cached per device); nullptr on failure.
+const DeviceInfo* current_device_info();
+
+// Opts `func` into `bytes` of dynamic shared memory on the current device.
+bool ensure_smem_attr(const void* func, size_t bytes);
+
+// Resident CTAs per SM of `func` at this launch shape on the current device
+// (cached); 0 on failure.
+int ctas_per_sm(const void* func, int threads, size_t smem);
+
+inline bool aligned(const void* p, size_t a) {
+  return (reinterpret_cast<uintptr_t>(p) % a) == 0;
+}
+
+// 5-D tiled 16-bit tensor map with 128-byte swizzle over `base`.
+// dims: innermost first; strides: bytes of dims 1..4; box: elements per dim.
+// Returns false if the driver rejects the description.
+bool get_tensor_map(CUtensorMap* out, const void* base, const uint64_t dims[5],
+                    const uint64_t strides[4], const uint32_t box[5]);
+
+}  // namespace pa

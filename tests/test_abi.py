@@ -1,0 +1,124 @@
+"""The C-ABI library on the CPU: it loads, exports every entry point the header
+declares, and rejects bad arguments on the host before any launch.  Also the
+native block manager against the reference block manager, table for table."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "pagedattn.h")
+
+
+@pytest.fixture(scope="module")
+def pa():
+    from paged_kv_cache_343_b200 import build
+    build.build()
+    import paged_kv_cache_343_b200 as pa
+    return pa
+
+
+def _declared():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(pa_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol(pa):
+    names = _declared()
+    assert "pa_decode_attention" in names and "pa_reshape_and_cache" in names
+    assert "pa_copy_blocks" in names
+    lib = ctypes.CDLL(pa.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_status_strings(pa):
+    assert pa.lib.pa_status_string(0) == b"PA_OK"
+    assert pa.lib.pa_status_string(1) == b"PA_ERR_INVALID_ARG"
+    assert pa.version() >= 100
+
+
+def test_host_validation_without_gpu(pa):
+    lib = pa.lib
+    # null pointers are refused before anything touches the device
+    st = lib.pa_decode_attention(None, 1, None, None, None, None, 1, None, 4, 16, 4, 2, 64, 8,
+                                 4, 0.125, 1, 0, None, 0, None, None)
+    assert st == 1
+    st = lib.pa_reshape_and_cache(None, None, 128, 128, None, None, None, 4, 8, 4, 2, 64, 0, 0,
+                                  None, None, None, None)
+    assert st == 1
+    # fp8 cache types are not built
+    st = lib.pa_reshape_and_cache(None, None, 128, 128, None, None, None, 4, 8, 4, 2, 64, 0, 1,
+                                  None, None, None, None)
+    assert st == 2
+    # zero work is a no-op
+    assert lib.pa_decode_attention(None, 1, None, None, None, None, 1, None, 0, 16, 4, 2, 64, 8,
+                                   4, 0.125, 1, 0, None, 0, None, None) == 0
+    assert lib.pa_copy_blocks(None, None, 1, None, 0, 8, 1024, None, None) == 0
+    # bad sizes
+    assert lib.pa_copy_blocks(None, None, 1, None, 3, 0, 1024, None, None) == 1
+
+
+def test_workspace_shape_checks_without_gpu(pa):
+    out = ctypes.c_size_t(0)
+    lib = pa.lib
+    # Hq not a multiple of Hkv
+    assert lib.pa_decode_workspace_bytes(4, 6, 4, 128, 16, 512, 0, ctypes.byref(out)) == 1
+    # unsupported head_dim / block size / group
+    assert lib.pa_decode_workspace_bytes(4, 8, 2, 96, 16, 512, 0, ctypes.byref(out)) == 2
+    assert lib.pa_decode_workspace_bytes(4, 8, 2, 128, 12, 512, 0, ctypes.byref(out)) == 2
+    assert lib.pa_decode_workspace_bytes(4, 32, 2, 128, 16, 512, 0, ctypes.byref(out)) == 2
+    # partition not block aligned
+    assert lib.pa_decode_workspace_bytes(4, 8, 2, 128, 32, 512, 48, ctypes.byref(out)) == 1
+
+
+def _ops_trace(seed, num_blocks=64, bs=4):
+    rng = np.random.default_rng(seed)
+    order = rng.permutation(num_blocks).astype(np.int32)
+    ops = [("add", 0, 7), ("add", 1, 4), ("fork", 0, 2), ("fork", 0, 3)]
+    for _ in range(40):
+        ops.append(("append", int(rng.integers(0, 4)), None))
+    ops += [("free", 1, None), ("add", 4, 9), ("fork", 2, 5)]
+    for _ in range(20):
+        ops.append(("append", int(rng.choice([0, 2, 3, 4, 5])), None))
+    return order, ops
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_native_block_manager_matches_reference(pa, seed):
+    from oracle.blockmgr import RefBlockManager
+    order, ops = _ops_trace(seed)
+    ref = RefBlockManager(64, 4, order)
+    nat = pa.BlockManager(64, 4, order)
+    live = set()
+    for op, a, b in ops:
+        if op == "add":
+            ref.add_sequence(a, b); nat.add_sequence(a, b); live.add(a)
+        elif op == "fork":
+            ref.fork(a, b); nat.fork(a, b); live.add(b)
+        elif op == "free":
+            ref.free_sequence(a); nat.free_sequence(a); live.discard(a)
+        else:
+            assert ref.append_slot(a) == nat.append_slot(a)
+        for s in live:
+            assert ref.block_table(s) == nat.block_table(s)
+            assert ref.lengths[s] == nat.seq_len(s)
+        ref.check_invariants()
+    assert [ref.refcount[i] for i in range(64)] == [nat.refcount(i) for i in range(64)]
+    assert len(ref.free) == nat.num_free()
+
+
+def test_native_block_manager_errors(pa):
+    bm = pa.BlockManager(2, 4)
+    bm.add_sequence(0, 8)
+    with pytest.raises(pa.PagedAttnError) as e:
+        bm.append_slot(0)
+    assert e.value.name == "PA_ERR_OUT_OF_BLOCKS"
+    with pytest.raises(pa.PagedAttnError) as e:
+        bm.append_slot(7)
+    assert e.value.name == "PA_ERR_NOT_FOUND"
+    with pytest.raises(pa.PagedAttnError):
+        pa.BlockManager(3, 4, [0, 0, 1])  # not a permutation

@@ -1,0 +1,264 @@
+"""Paged decode attention on the GPU against the fp64 oracle.
+
+Tolerances: outputs stored in the 16-bit input type must be within 2e-3
+max-abs of the oracle (fp16/bf16 storage, fp32 accumulation); the fp32-output
+mode, which removes the final storage rounding, must be within 1e-4.  Pools are
+NaN-poisoned in every slot that holds no token, so any read past a sequence's
+end or of a block outside its table shows up as NaN."""
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import pa_workloads as W
+from harness import as_f64, prepare, to_dev
+
+pytestmark = pytest.mark.gpu
+
+TOL_STORED = 2e-3
+TOL_F32 = 1e-4
+NTHREADS = max(1, len(os.sched_getaffinity(0)))
+
+
+@pytest.fixture(scope="module")
+def pa():
+    import paged_kv_cache_343_b200 as pa
+    return pa
+
+
+def _run(pa, prep, lens=None, out_dtype=None, partition_size=None, k=None, v=None, tables=None,
+         flag=None):
+    s = prep.case.spec
+    lens = prep.seq_lens if lens is None else lens
+    q = to_dev(prep.case.q, s.dtype)
+    dk = to_dev(prep.k_pool, s.dtype) if k is None else k
+    dv = to_dev(prep.v_pool, s.dtype) if v is None else v
+    tb = to_dev(prep.tables if tables is None else tables)
+    out = torch.empty(q.shape, dtype=out_dtype or q.dtype, device="cuda")
+    ps = s.partition_size if partition_size is None else partition_size
+    pa.decode_attention(out, q, dk, dv, tb, to_dev(lens.astype(np.int32)), int(lens.max()),
+                        W.scale_of(s), partition_size=ps, error_flag=flag)
+    torch.cuda.synchronize()
+    return out
+
+
+def _oracle(orc, prep, lens=None, k=None, v=None, tables=None, seqs=None):
+    s = prep.case.spec
+    lens = prep.seq_lens if lens is None else lens
+    tables = prep.tables if tables is None else tables
+    q = prep.case.q
+    if seqs is not None:
+        q, tables, lens = q[seqs], tables[seqs], lens[seqs]
+    return orc.decode(q, prep.k_pool if k is None else k, prep.v_pool if v is None else v,
+                      tables, lens, W.scale_of(s), s.dtype, nthreads=NTHREADS)
+
+
+def _maxerr(out, ref, seqs=None):
+    o = as_f64(out)
+    if seqs is not None:
+        o = o[seqs]
+    assert np.all(np.isfinite(o)), "non-finite output"
+    return float(np.max(np.abs(o - ref)))
+
+
+def half_ulp(ref: np.ndarray, dtype: str) -> np.ndarray:
+    """Half a unit in the last place of the 16-bit storage type at |ref|: the
+    rounding that storing an exact result in that type may add."""
+    mant, emin = (7, -126) if dtype == "bf16" else (10, -14)
+    e = np.floor(np.log2(np.maximum(np.abs(ref), 2.0 ** emin)))
+    return 0.5 * np.exp2(e - mant)
+
+
+def _stored_within(out, ref, dtype):
+    """Stored outputs: the fp32-path error plus the storage rounding."""
+    o = as_f64(out)
+    assert np.all(np.isfinite(o))
+    return bool(np.all(np.abs(o - ref) <= TOL_F32 + half_ulp(ref, dtype)))
+
+
+def _reduced(name):
+    base = W.WORKLOADS[name]
+    if name == "llama8b":
+        return base.replace(num_seqs=6, len_lo=512, len_hi=1100)
+    if name == "longtail":
+        return base.replace(num_seqs=40, new_rows=40)
+    if name == "longctx":
+        return base.replace(num_seqs=2, fixed_lens=(4096, 4096))
+    if name == "shared_prefix":
+        return base.replace(prompts=2, num_seqs=16)
+    return base
+
+
+@pytest.mark.parametrize("name", ["tiny", "llama8b", "longtail", "longctx", "shared_prefix"])
+def test_decode_reduced(pa, orc, name):
+    """Every workload's shape at a size the oracle runs in seconds (several tiles
+    per sequence, ragged last tiles), stored and fp32 outputs."""
+    prep = prepare(_reduced(name))
+    s = prep.case.spec
+    k, v = prep.k_pool, prep.v_pool
+    if prep.cow_pairs is not None:
+        # the decode step sees the pool after copy-on-write and the appends
+        import oracle
+        k, v = k.copy(), v.copy()
+        oracle.copy_blocks([k, v], prep.cow_pairs, int(np.prod(k.shape[1:])) * 2)
+        oracle.reshape_and_cache(prep.case.new_k, prep.case.new_v, k, v, prep.new_slots)
+    ref = _oracle(orc, prep, k=k, v=v)
+    dk, dv = to_dev(k, s.dtype), to_dev(v, s.dtype)
+    flag = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = _run(pa, prep, k=dk, v=dv, flag=flag)
+    assert _maxerr(out, ref) <= TOL_STORED
+    out32 = _run(pa, prep, k=dk, v=dv, out_dtype=torch.float32)
+    assert _maxerr(out32, ref) <= TOL_F32
+    assert int(flag.item()) == 0
+
+
+def test_tiny_write_then_attend(pa, orc):
+    """Tiny workload: reshape_and_cache of the 4 new tokens at their next slots
+    (the 16-token sequence first gets a fifth block), then attention over
+    lengths + 1 reads them back."""
+    prep = prepare(W.WORKLOADS["tiny"])
+    s = prep.case.spec
+    k, v = prep.k_pool.copy(), prep.v_pool.copy()
+    orc.reshape_and_cache(prep.case.new_k, prep.case.new_v, k, v, prep.new_slots)
+    lens1 = prep.seq_lens + 1
+    ref = _oracle(orc, prep, lens=lens1, k=k, v=v)
+    dk, dv = to_dev(prep.k_pool, s.dtype), to_dev(prep.v_pool, s.dtype)
+    pa.reshape_and_cache(to_dev(prep.case.new_k, s.dtype), to_dev(prep.case.new_v, s.dtype),
+                         dk, dv, to_dev(prep.new_slots))
+    out = _run(pa, prep, lens=lens1, k=dk, v=dv, out_dtype=torch.float32)
+    assert _maxerr(out, ref) <= TOL_F32
+    # the 16-token sequence's new token sits in a fifth block
+    assert prep.tables[2, 4] >= 0
+
+
+@pytest.mark.parametrize("psize", [0, 16, 32, 64, 512, 4096])
+def test_partition_sizes_agree(pa, orc, psize):
+    spec = W.WORKLOADS["llama8b"].replace(num_seqs=5, len_lo=1, len_hi=1500, seed=77)
+    prep = prepare(spec)
+    ref = _oracle(orc, prep)
+    out32 = _run(pa, prep, out_dtype=torch.float32, partition_size=psize)
+    assert _maxerr(out32, ref) <= TOL_F32
+
+
+@pytest.mark.parametrize("bs,dtype,hq,hkv,d", [
+    (4, "bf16", 8, 2, 128), (8, "f16", 16, 4, 64), (32, "f16", 8, 8, 128),
+    (64, "bf16", 16, 2, 128), (128, "bf16", 4, 1, 64), (16, "f16", 24, 8, 128),
+    (16, "bf16", 64, 8, 128),
+])
+def test_shapes(pa, orc, bs, dtype, hq, hkv, d):
+    spec = W.Spec("shape", 7, hq, hkv, d, bs, dtype, seed=bs * 7 + hq, len_dist="uniform",
+                  len_lo=1, len_hi=700)
+    prep = prepare(spec)
+    ref = _oracle(orc, prep)
+    out32 = _run(pa, prep, out_dtype=torch.float32)
+    assert _maxerr(out32, ref) <= TOL_F32
+    # lengths down to 1 give |out| near 1-2, where one storage ulp of bf16 alone
+    # exceeds 2e-3: the stored check is the fp32 bound plus half an ulp
+    out = _run(pa, prep)
+    assert _stored_within(out, ref, dtype)
+
+
+def test_empty_and_single_token_sequences(pa, orc):
+    spec = W.Spec("edge", 6, 8, 2, 128, 16, "bf16", seed=5, len_dist="fixed",
+                  fixed_lens=(0, 1, 16, 17, 0, 33))
+    prep = prepare(spec)
+    ref = _oracle(orc, prep)
+    out32 = _run(pa, prep, out_dtype=torch.float32)
+    o = as_f64(out32)
+    assert np.all(o[0] == 0) and np.all(o[4] == 0)
+    assert _maxerr(out32, ref) <= TOL_F32
+    # seq_len 1: the output is that token's value row, exactly (fp32 out)
+    vrow = prep.v_pool[prep.tables[1, 0], 0]  # [Hkv, D] bits
+    import oracle
+    vv = oracle.bf16_to_double(vrow)
+    for h in range(8):
+        assert np.array_equal(o[1, h], vv[h // 4])
+
+
+def test_placement_invariance_bitwise(pa):
+    """Relabelling physical blocks (data and tables together) leaves the GPU
+    output bit-identical: the summation order does not depend on placement."""
+    spec = W.WORKLOADS["llama8b"].replace(num_seqs=4, len_lo=100, len_hi=900, seed=9)
+    prep = prepare(spec)
+    out_a = _run(pa, prep, out_dtype=torch.float32)
+    nb = prep.case.num_blocks
+    perm = np.random.default_rng(4).permutation(nb)
+    kp, vp = np.empty_like(prep.k_pool), np.empty_like(prep.v_pool)
+    kp[perm], vp[perm] = prep.k_pool, prep.v_pool
+    tp = np.where(prep.tables >= 0, perm[np.maximum(prep.tables, 0)], -1).astype(np.int32)
+    out_b = _run(pa, prep, out_dtype=torch.float32, k=to_dev(kp, "bf16"), v=to_dev(vp, "bf16"),
+                 tables=tp)
+    assert torch.equal(out_a, out_b)
+
+
+def test_repeat_runs_bitwise_identical(pa):
+    spec = W.WORKLOADS["longtail"].replace(num_seqs=64, new_rows=0, seed=3)
+    prep = prepare(spec)
+    a = _run(pa, prep)
+    b = _run(pa, prep)
+    assert torch.equal(a, b)
+
+
+def test_bad_block_id_flagged_and_skipped(pa, orc):
+    spec = W.WORKLOADS["llama8b"].replace(num_seqs=3, len_lo=64, len_hi=64, seed=12)
+    prep = prepare(spec)
+    tables = prep.tables.copy()
+    tables[1, 2] = prep.case.num_blocks + 5       # tokens 32..47 of sequence 1 are unreachable
+    flag = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = _run(pa, prep, out_dtype=torch.float32, tables=tables, flag=flag)
+    assert int(flag.item()) & pa.DEVERR_BAD_BLOCK
+    # the other sequences are unaffected
+    ref = _oracle(orc, prep)
+    o = as_f64(out)
+    assert np.max(np.abs(o[[0, 2]] - ref[[0, 2]])) <= TOL_F32
+    # sequence 1 equals attention over its 48 reachable tokens
+    import oracle
+    keep = [t for t in range(64) if not (32 <= t < 48)]
+    t1 = prep.tables[1]
+    blk = np.array([t1[t // 16] for t in keep])
+    off = np.array([t % 16 for t in keep])
+    k = np.ascontiguousarray(prep.k_pool[blk, off][:, None])   # [48, 1, Hkv, D]: block size 1
+    v = np.ascontiguousarray(prep.v_pool[blk, off][:, None])
+    ref1 = oracle.decode(prep.case.q[1:2], k, v, np.arange(48, dtype=np.int32)[None],
+                         np.array([48], np.int32), W.scale_of(spec), "bf16")
+    assert np.max(np.abs(o[1] - ref1[0])) <= TOL_F32
+
+
+def test_seq_len_above_max_is_flagged(pa):
+    spec = W.WORKLOADS["llama8b"].replace(num_seqs=2, len_lo=40, len_hi=40, seed=13)
+    prep = prepare(spec)
+    s = prep.case.spec
+    flag = torch.zeros(1, dtype=torch.int32, device="cuda")
+    q = to_dev(prep.case.q, s.dtype)
+    out = torch.empty_like(q)
+    pa.decode_attention(out, q, to_dev(prep.k_pool, s.dtype), to_dev(prep.v_pool, s.dtype),
+                        to_dev(prep.tables), to_dev(prep.seq_lens), 32, W.scale_of(s),
+                        error_flag=flag)
+    torch.cuda.synchronize()
+    assert int(flag.item()) & pa.DEVERR_BAD_SEQLEN
+    assert torch.isfinite(out.float()).all()
+
+
+# --------------------------------------------------------------------------
+# full sizes, in the launch configuration the benchmark times
+# --------------------------------------------------------------------------
+@pytest.mark.slow
+@pytest.mark.parametrize("name", ["llama8b", "longtail", "longctx", "shared_prefix"])
+def test_decode_full_size(pa, orc, name):
+    prep = prepare(W.WORKLOADS[name])
+    s = prep.case.spec
+    k, v = prep.k_pool, prep.v_pool
+    if prep.cow_pairs is not None:
+        import oracle
+        k, v = k.copy(), v.copy()
+        oracle.copy_blocks([k, v], prep.cow_pairs, int(np.prod(k.shape[1:])) * 2)
+        oracle.reshape_and_cache(prep.case.new_k, prep.case.new_v, k, v, prep.new_slots)
+    rng = np.random.default_rng(0)
+    seqs = np.sort(rng.choice(s.num_seqs, size=min(s.num_seqs, 24), replace=False))
+    ref = _oracle(orc, prep, k=k, v=v, seqs=seqs)
+    dk, dv = to_dev(k, s.dtype), to_dev(v, s.dtype)
+    out = _run(pa, prep, k=dk, v=dv)
+    assert _maxerr(out, ref, seqs) <= TOL_STORED
+    assert torch.isfinite(out.float()).all()
