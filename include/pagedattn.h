@@ -46,7 +46,9 @@ typedef enum {
   PA_ERR_UNSUPPORTED = 2,   /* valid but outside the built shapes/dtypes   */
   PA_ERR_CUDA = 3,          /* a CUDA runtime call or launch failed        */
   PA_ERR_OUT_OF_BLOCKS = 4, /* block manager: the free list is empty       */
-  PA_ERR_NOT_FOUND = 5      /* block manager: unknown sequence id          */
+  PA_ERR_NOT_FOUND = 5,     /* block manager: unknown sequence id          */
+  PA_ERR_TOO_LARGE = 6      /* needs more scratch than the library's static
+                               buffer holds (pa_decode_attention_noalloc)  */
 } pa_status;
 
 typedef enum { PA_F16 = 0, PA_BF16 = 1, PA_F32 = 2 } pa_dtype;
@@ -182,6 +184,44 @@ pa_status pa_decode_attention(void* out, pa_dtype out_dtype, const void* query,
                               int32_t partition_size, void* workspace,
                               size_t workspace_bytes,
                               int32_t* device_error_flag, pa_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * pa_decode_attention_noalloc -- pa_decode_attention for callers that cannot
+ * allocate device memory.  The pages have no counterpart of this entry point;
+ * it exists for callers such as plugins whose host framework owns every device
+ * allocation and forbids direct cudaMalloc, driver-style or embedded callers
+ * that have no allocator to hand, and loops where cudaMalloc/cudaFree (which
+ * may synchronise the whole device) cannot be afforded.
+ *
+ * Same arguments, meaning and errors as pa_decode_attention, minus the
+ * workspace: the scratch is a static device array inside the library, of
+ * PA_NOALLOC_SCRATCH_BYTES bytes on every GPU that loads the library, held
+ * until the process exits.  A shape whose pa_decode_workspace_bytes() exceeds
+ * that size is rejected with PA_ERR_TOO_LARGE before anything is launched.
+ * The call allocates nothing (no cudaMalloc, cudaFree or allocating library
+ * routine).
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    before any stream capture.
+ *  - All calls on a device share the one array and it keeps the last call's
+ *    contents.  Nothing in it needs to start at zero: each call's first
+ *    kernel rewrites the per-call bookkeeping before the others read it.
+ *    Calls that overlap on the GPU (other streams, or other host threads
+ *    without ordering) race on the array and give wrong results: order them.
+ * ------------------------------------------------------------------------- */
+#define PA_NOALLOC_SCRATCH_BYTES (16u << 20) /* 16 MiB per device */
+
+pa_status pa_decode_attention_noalloc(void* out, pa_dtype out_dtype, const void* query,
+                                      const void* key_cache, const void* value_cache,
+                                      const int32_t* block_tables,
+                                      int32_t block_table_stride,
+                                      const int32_t* seq_lens, int32_t num_seqs,
+                                      int32_t max_seq_len, int32_t num_q_heads,
+                                      int32_t num_kv_heads, int32_t head_dim,
+                                      int32_t num_blocks, int32_t block_size,
+                                      float scale, pa_dtype kv_dtype,
+                                      int32_t partition_size,
+                                      int32_t* device_error_flag, pa_stream_t stream);
 
 /* ---------------------------------------------------------------------------
  * Host block manager -- [PA] "The idea: page the KV cache" (allocate a block

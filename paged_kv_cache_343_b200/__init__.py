@@ -77,6 +77,10 @@ def _load() -> ctypes.CDLL:
     lib.pa_decode_attention.argtypes = [p, ctypes.c_int, p, p, p, p, i32, p, i32, i32, i32, i32,
                                         i32, i32, i32, ctypes.c_float, ctypes.c_int, i32, p, sz,
                                         p, p]
+    lib.pa_decode_attention_noalloc.restype = ctypes.c_int
+    lib.pa_decode_attention_noalloc.argtypes = [p, ctypes.c_int, p, p, p, p, i32, p, i32, i32, i32,
+                                                i32, i32, i32, i32, ctypes.c_float, ctypes.c_int,
+                                                i32, p, p]
     lib.pa_bm_create.restype = ctypes.c_int
     lib.pa_bm_create.argtypes = [i32, i32, p, ctypes.POINTER(p)]
     lib.pa_bm_destroy.restype = None
@@ -207,6 +211,30 @@ def decode_attention(out: torch.Tensor, query: torch.Tensor, key_cache: torch.Te
         d, nb, bs, float(scale), _DTYPE_CODE[query.dtype], int(partition_size), _ptr(workspace),
         workspace.numel() * workspace.element_size(), _ptr(error_flag), _stream_handle(stream)),
         "pa_decode_attention")
+    return out
+
+
+# Bytes of the library's static scratch array used by decode_attention_noalloc.
+NOALLOC_SCRATCH_BYTES = 16 << 20
+
+
+def decode_attention_noalloc(out: torch.Tensor, query: torch.Tensor, key_cache: torch.Tensor,
+                             value_cache: torch.Tensor, block_tables: torch.Tensor,
+                             seq_lens: torch.Tensor, max_seq_len: int, scale: float,
+                             partition_size: int = 0, error_flag: Optional[torch.Tensor] = None,
+                             stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """decode_attention for callers that must not allocate device memory: the
+    scratch is the library's static per-device array (NOALLOC_SCRATCH_BYTES),
+    so this wrapper allocates nothing either.  Shapes needing more scratch raise
+    PagedAttnError PA_ERR_TOO_LARGE.  Calls overlapping on the GPU share the
+    array and race; the first call on a device should precede stream capture."""
+    B, hq, d = query.shape
+    nb, bs, hkv, _ = key_cache.shape
+    _check(lib.pa_decode_attention_noalloc(
+        _ptr(out), _DTYPE_CODE[out.dtype], _ptr(query), _ptr(key_cache), _ptr(value_cache),
+        _ptr(block_tables), block_tables.stride(0), _ptr(seq_lens), B, int(max_seq_len), hq, hkv,
+        d, nb, bs, float(scale), _DTYPE_CODE[query.dtype], int(partition_size),
+        _ptr(error_flag), _stream_handle(stream)), "pa_decode_attention_noalloc")
     return out
 
 

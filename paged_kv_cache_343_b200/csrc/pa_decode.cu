@@ -826,3 +826,58 @@ extern "C" pa_status pa_decode_attention(
   if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
   return PA_OK;
 }
+
+// ===========================================================================
+// No-allocation variant: the same launches with the workspace in a static
+// device array of this file instead of caller-provided memory, for callers
+// that may not allocate device memory (see pa_decode_attention_noalloc in the
+// header).  In host code the array's name is only a host-side stand-in, so its
+// device address is looked up once per device and passed to the kernels.
+// ===========================================================================
+static __device__ __align__(256) unsigned char g_noalloc_scratch[PA_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[64] = {};  // device address of g_noalloc_scratch, per device
+
+// Looks the array's address up on the current device the first time; later
+// calls on that device reuse it.
+pa_status noalloc_scratch(void** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return PA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+      return PA_ERR_CUDA;
+    g_noalloc_addr[dev] = p;
+  }
+  *out = g_noalloc_addr[dev];
+  return PA_OK;
+}
+
+}  // namespace
+
+extern "C" pa_status pa_decode_attention_noalloc(
+    void* out, pa_dtype out_dtype, const void* query, const void* key_cache,
+    const void* value_cache, const int32_t* block_tables, int32_t block_table_stride,
+    const int32_t* seq_lens, int32_t num_seqs, int32_t max_seq_len, int32_t num_q_heads,
+    int32_t num_kv_heads, int32_t head_dim, int32_t num_blocks, int32_t block_size, float scale,
+    pa_dtype kv_dtype, int32_t partition_size, int32_t* device_error_flag, pa_stream_t stream) {
+  if (num_seqs < 0) return PA_ERR_INVALID_ARG;
+  if (num_seqs == 0) return PA_OK;
+  size_t need = 0;
+  pa_status st = pa_decode_workspace_bytes(num_seqs, num_q_heads, num_kv_heads, head_dim,
+                                           block_size, max_seq_len, partition_size, &need);
+  if (st != PA_OK) return st;
+  if (need > PA_NOALLOC_SCRATCH_BYTES) return PA_ERR_TOO_LARGE;
+  void* scratch = nullptr;
+  st = noalloc_scratch(&scratch);
+  if (st != PA_OK) return st;
+  return pa_decode_attention(out, out_dtype, query, key_cache, value_cache, block_tables,
+                             block_table_stride, seq_lens, num_seqs, max_seq_len, num_q_heads,
+                             num_kv_heads, head_dim, num_blocks, block_size, scale, kv_dtype,
+                             partition_size, scratch, PA_NOALLOC_SCRATCH_BYTES, device_error_flag,
+                             stream);
+}

@@ -168,6 +168,7 @@ extern "C" const char* pa_status_string(pa_status status) {
     case PA_ERR_CUDA: return "PA_ERR_CUDA";
     case PA_ERR_OUT_OF_BLOCKS: return "PA_ERR_OUT_OF_BLOCKS";
     case PA_ERR_NOT_FOUND: return "PA_ERR_NOT_FOUND";
+    case PA_ERR_TOO_LARGE: return "PA_ERR_TOO_LARGE";
   }
   return "PA_ERR_UNKNOWN";
 }
