@@ -43,6 +43,8 @@ __global__ void __launch_bounds__(kRowThreads)
                                 int64_t num_slots, int32_t row_elems, int32_t* err) {
   using T = typename Vec<VEC>::T;
   const int32_t nvec = row_elems / VEC;
+  griddep_launch_dependents();
+  griddep_wait();
   for (int64_t t = blockIdx.x; t < num_tokens; t += gridDim.x) {
     const int64_t slot = slot_mapping[t];
     if (slot < 0) continue;  // padding token
@@ -74,6 +76,8 @@ __global__ void __launch_bounds__(kCopyThreads)
     pa_copy_blocks_kernel(const CopyPtrs ptrs, const int32_t* __restrict__ mapping,
                           int32_t num_blocks, int64_t block_bytes, int32_t* err) {
   const int64_t pair = blockIdx.x;
+  griddep_launch_dependents();
+  griddep_wait();
   const int32_t src = mapping[2 * pair], dst = mapping[2 * pair + 1];
   if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) {
     if (threadIdx.x == 0 && blockIdx.y == 0) flag_error(err, PA_DEVERR_BAD_SLOT);
@@ -124,19 +128,18 @@ extern "C" pa_status pa_reshape_and_cache(const void* key, const void* value,
                    aligned(value_cache, 16) && key_stride_t % 8 == 0 &&
                    value_stride_t % 8 == 0 && row % 8 == 0;
   const int grid = num_tokens < (1 << 20) ? num_tokens : (1 << 20);
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (vec) {
-    pa_reshape_and_cache_kernel<8><<<grid, kRowThreads, 0, s>>>(
-        static_cast<const uint16_t*>(key), static_cast<const uint16_t*>(value), key_stride_t,
-        value_stride_t, static_cast<uint16_t*>(key_cache), static_cast<uint16_t*>(value_cache),
-        slot_mapping, num_tokens, num_slots, static_cast<int32_t>(row), device_error_flag);
-  } else {
-    pa_reshape_and_cache_kernel<1><<<grid, kRowThreads, 0, s>>>(
-        static_cast<const uint16_t*>(key), static_cast<const uint16_t*>(value), key_stride_t,
-        value_stride_t, static_cast<uint16_t*>(key_cache), static_cast<uint16_t*>(value_cache),
-        slot_mapping, num_tokens, num_slots, static_cast<int32_t>(row), device_error_flag);
-  }
-  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+  PdlLaunch launch(reinterpret_cast<cudaStream_t>(stream), dim3(grid), dim3(kRowThreads));
+  const uint16_t* k = static_cast<const uint16_t*>(key);
+  const uint16_t* v = static_cast<const uint16_t*>(value);
+  uint16_t* kc = static_cast<uint16_t*>(key_cache);
+  uint16_t* vc = static_cast<uint16_t*>(value_cache);
+  const int32_t re = static_cast<int32_t>(row);
+  const cudaError_t e =
+      vec ? launch(pa_reshape_and_cache_kernel<8>, k, v, key_stride_t, value_stride_t, kc, vc,
+                   slot_mapping, num_tokens, num_slots, re, device_error_flag)
+          : launch(pa_reshape_and_cache_kernel<1>, k, v, key_stride_t, value_stride_t, kc, vc,
+                   slot_mapping, num_tokens, num_slots, re, device_error_flag);
+  return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
 extern "C" pa_status pa_copy_blocks(void* const* key_caches, void* const* value_caches,
@@ -162,14 +165,13 @@ extern "C" pa_status pa_copy_blocks(void* const* key_caches, void* const* value_
       ptrs.p[2 * l] = static_cast<uint8_t*>(key_caches[l0 + l]);
       ptrs.p[2 * l + 1] = static_cast<uint8_t*>(value_caches[l0 + l]);
     }
-    const dim3 grid(num_pairs, 2 * nl);
-    if (vec) {
-      pa_copy_blocks_kernel<true><<<grid, kCopyThreads, 0, s>>>(ptrs, block_mapping, num_blocks,
-                                                                 block_bytes, device_error_flag);
-    } else {
-      pa_copy_blocks_kernel<false><<<grid, kCopyThreads, 0, s>>>(ptrs, block_mapping, num_blocks,
-                                                                  block_bytes, device_error_flag);
-    }
+    PdlLaunch launch(s, dim3(num_pairs, 2 * nl), dim3(kCopyThreads));
+    const cudaError_t e =
+        vec ? launch(pa_copy_blocks_kernel<true>, ptrs, block_mapping, num_blocks, block_bytes,
+                     device_error_flag)
+            : launch(pa_copy_blocks_kernel<false>, ptrs, block_mapping, num_blocks, block_bytes,
+                     device_error_flag);
+    if (e != cudaSuccess) return PA_ERR_CUDA;
   }
-  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+  return PA_OK;
 }

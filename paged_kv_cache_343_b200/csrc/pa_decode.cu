@@ -31,7 +31,7 @@
 namespace pa {
 
 constexpr int kTile = 16;            // tokens per tile (MMA M of the score product)
-constexpr int kPlanThreads = 1024;
+constexpr int kPlanThreads = 256;
 constexpr int kCombineWarps = 4;
 
 enum : int32_t {
@@ -66,8 +66,10 @@ struct DecodeParams {
   int32_t stages;
   int32_t tok_box;         // tokens per TMA box: min(block_size, 16)
   int32_t tma_mode;        // 0: one box per block per tile, 1: one per (head, d-half)
-  int32_t* plan_tiles;     // [num_seqs + 1]
-  int32_t* plan_parts;     // [num_seqs + 1]
+  int32_t* plan_tiles;     // [num_seqs + 1] tile prefix sums
+  int32_t* seg_base;       // [num_seqs + 1] segment prefix sums (partial slots)
+  int32_t* start_seq;      // [ctas_per_group] sequence holding each CTA's first tile
+  int32_t* first_k;        // [ctas_per_group] index of that tile's segment in its sequence
   float* part_o;           // [groups][nseg_cap][HG * group][head_dim]
   float* part_ml;          // [groups][nseg_cap][HG * group][2]  (m in log2 units, l)
   int32_t* err;
@@ -77,68 +79,118 @@ __device__ __forceinline__ int32_t clamp_len(int32_t L, int32_t max_len) {
   return L < 0 ? 0 : (L > max_len ? max_len : L);
 }
 
-// CTA whose share [c*N/C, (c+1)*N/C) holds global tile t.
-__device__ __forceinline__ int32_t cta_of_tile(int64_t t, int64_t N, int64_t C) {
-  return static_cast<int32_t>(((t + 1) * C - 1) / N);
-}
 
 // ---------------------------------------------------------------------------
-// plan: tiles[b] = sum_{b'<b} ceil(L_b'/16); parts[b] = sum_{b'<b} max(1, ceil(n_b'/tpp))
+// plan (one CTA)
+//   tiles[b]    = sum_{b' < b} ceil(L_b' / 16)          (N = tiles[B] in all)
+//   segments    a sequence's tiles are cut wherever a partition starts
+//               (every tiles_per_part tiles from its first tile) or a CTA's
+//               share starts (lo(c) = floor(c N / C)); each piece is one
+//               segment, numbered 0, 1, ... within the sequence;
+//   seg_base[b] = sum_{b' < b} (segments of b'), so the partials of sequence
+//               b occupy slots seg_base[b] .. seg_base[b + 1] - 1;
+//   start_seq[c], first_k[c]: the sequence holding lo(c) and the number of
+//               that sequence's segments that start before lo(c).
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(kPlanThreads) pa_plan_kernel(DecodeParams p) {
-  __shared__ int32_t warp_t[kPlanThreads / 32], warp_p[kPlanThreads / 32];
-  __shared__ int32_t carry[2];
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  if (tid == 0) carry[0] = carry[1] = 0;
+constexpr int kPlanWarps = kPlanThreads / 32;
+
+// Exclusive block-wide prefix sum of one value per thread; *total gets the sum.
+__device__ __forceinline__ int32_t block_exclusive_scan(int32_t v, int32_t* warp_buf,
+                                                        int32_t* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int32_t inc = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int32_t u = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += u;
+  }
+  if (lane == 31) warp_buf[warp] = inc;
   __syncthreads();
+  if (warp == 0) {
+    int32_t w = lane < kPlanWarps ? warp_buf[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int32_t u = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += u;
+    }
+    if (lane < kPlanWarps) warp_buf[lane] = w;  // inclusive over warps
+  }
+  __syncthreads();
+  const int32_t before = (warp > 0 ? warp_buf[warp - 1] : 0) + inc - v;
+  *total = warp_buf[kPlanWarps - 1];
+  __syncthreads();  // warp_buf is reused by the next call
+  return before;
+}
+
+// Walks the segment starts of sequence b (tiles [t0, t1)) in order: the
+// partition starts and the CTA-share starts, equal points counted once.
+// Records start_seq / first_k for every CTA whose share starts inside b and
+// returns the number of segments.
+__device__ int32_t plan_sequence_segments(const DecodeParams& p, int32_t b, int64_t t0,
+                                          int64_t t1, int64_t N, int64_t C) {
+  const int64_t q = N / C, r = N % C;
+  int64_t c = (t0 * C + N - 1) / N;  // first CTA with lo(c) >= t0
+  int64_t lo_c = c * q + (c * r) / C;
+  int64_t rem = (c * r) % C;         // lo(c + 1) = lo(c) + q + [rem + r >= C]
+  int64_t part = t0;                 // next partition start
+  const int64_t tpp = p.tiles_per_part;
+  int32_t count = 0;
+  int64_t last = -1;
+  while (true) {
+    const int64_t cta_pt = (c < C && lo_c < t1) ? lo_c : INT64_MAX;
+    const int64_t part_pt = part < t1 ? part : INT64_MAX;
+    if (cta_pt == INT64_MAX && part_pt == INT64_MAX) break;
+    if (cta_pt <= part_pt) {
+      const int32_t idx = (cta_pt == last) ? count - 1 : count;
+      if (cta_pt != last) { ++count; last = cta_pt; }
+      p.start_seq[c] = b;
+      p.first_k[c] = idx;
+      ++c;
+      rem += r;
+      lo_c += q;
+      if (rem >= C) { rem -= C; ++lo_c; }
+    } else {
+      if (part_pt != last) { ++count; last = part_pt; }
+      part = (tpp == INT_MAX) ? INT64_MAX : part + tpp;
+    }
+  }
+  return count;
+}
+
+__global__ void __launch_bounds__(kPlanThreads) pa_plan_kernel(DecodeParams p) {
+  __shared__ int32_t warp_buf[kPlanWarps];
+  const int tid = threadIdx.x;
+  griddep_launch_dependents();
+  griddep_wait();  // seq_lens may come from the previous kernel on the stream
+  int32_t carry = 0, total = 0;
   for (int base = 0; base < p.num_seqs; base += kPlanThreads) {
     const int b = base + tid;
-    int32_t nt = 0, np = 0;
+    int32_t nt = 0;
     if (b < p.num_seqs) {
       const int32_t raw = p.seq_lens[b];
       if (raw < 0 || raw > p.max_seq_len) flag_error(p.err, PA_DEVERR_BAD_SEQLEN);
-      const int32_t L = clamp_len(raw, p.max_seq_len);
-      nt = (L + kTile - 1) / kTile;
-      np = nt == 0 ? 1 : (p.tiles_per_part == INT_MAX ? 1 : (nt + p.tiles_per_part - 1) / p.tiles_per_part);
+      nt = (clamp_len(raw, p.max_seq_len) + kTile - 1) / kTile;
     }
-    int32_t it = nt, ip = np;  // inclusive warp scan
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int32_t vt = __shfl_up_sync(0xffffffffu, it, o);
-      const int32_t vp = __shfl_up_sync(0xffffffffu, ip, o);
-      if (lane >= o) { it += vt; ip += vp; }
-    }
-    if (lane == 31) { warp_t[warp] = it; warp_p[warp] = ip; }
-    __syncthreads();
-    if (warp == 0) {
-      int32_t wt = warp_t[lane], wp = warp_p[lane];
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int32_t vt = __shfl_up_sync(0xffffffffu, wt, o);
-        const int32_t vp = __shfl_up_sync(0xffffffffu, wp, o);
-        if (lane >= o) { wt += vt; wp += vp; }
-      }
-      warp_t[lane] = wt;  // inclusive over warps
-      warp_p[lane] = wp;
-    }
-    __syncthreads();
-    const int32_t before_t = carry[0] + (warp > 0 ? warp_t[warp - 1] : 0);
-    const int32_t before_p = carry[1] + (warp > 0 ? warp_p[warp - 1] : 0);
-    if (b < p.num_seqs) {
-      p.plan_tiles[b] = before_t + it - nt;
-      p.plan_parts[b] = before_p + ip - np;
-    }
-    __syncthreads();
-    if (tid == 0) {
-      carry[0] += warp_t[kPlanThreads / 32 - 1];
-      carry[1] += warp_p[kPlanThreads / 32 - 1];
-    }
-    __syncthreads();
+    const int32_t ex = block_exclusive_scan(nt, warp_buf, &total);
+    if (b < p.num_seqs) p.plan_tiles[b] = carry + ex;
+    carry += total;
   }
-  if (tid == 0) {
-    p.plan_tiles[p.num_seqs] = carry[0];
-    p.plan_parts[p.num_seqs] = carry[1];
+  if (tid == 0) p.plan_tiles[p.num_seqs] = carry;
+  __syncthreads();
+  const int64_t N = carry, C = p.ctas_per_group;
+  int32_t seg_carry = 0;
+  for (int base = 0; base < p.num_seqs; base += kPlanThreads) {
+    const int b = base + tid;
+    int32_t ns = 0;
+    if (b < p.num_seqs && N > 0) {
+      const int64_t t0 = p.plan_tiles[b], t1 = p.plan_tiles[b + 1];
+      if (t1 > t0) ns = plan_sequence_segments(p, b, t0, t1, N, C);
+    }
+    const int32_t ex = block_exclusive_scan(ns, warp_buf, &total);
+    if (b < p.num_seqs) p.seg_base[b] = seg_carry + ex;
+    seg_carry += total;
   }
+  if (tid == 0) p.seg_base[p.num_seqs] = seg_carry;
 }
 
 // ---------------------------------------------------------------------------
@@ -184,22 +236,13 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
     prefetch_tmap(&tmV);
   }
   __syncthreads();
+  griddep_launch_dependents();
+  griddep_wait();  // the plan (and all earlier work on the stream) is complete
 
   const int64_t N = p.plan_tiles[B];
   const int64_t lo = static_cast<int64_t>(c) * N / C;
   const int64_t hi = static_cast<int64_t>(c + 1) * N / C;
   if (lo >= hi) return;
-
-  // first sequence with tiles[b + 1] > lo
-  int b0;
-  {
-    int l = 0, r = B - 1;
-    while (l < r) {
-      const int mid = (l + r) >> 1;
-      if (p.plan_tiles[mid + 1] > lo) r = mid; else l = mid + 1;
-    }
-    b0 = l;
-  }
 
   if (warp == HG) {
     // ======================= producer =======================
@@ -209,12 +252,13 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
     const int TB = p.tok_box;
     const uint32_t box_bytes = static_cast<uint32_t>(HG * DC * TB * 128);
     const int bpt = bs < kTile ? kTile / bs : 1;  // blocks per tile
-    int b = b0;
+    int b = p.start_seq[c];
     int32_t t_first = p.plan_tiles[b];
     int32_t n_b = p.plan_tiles[b + 1] - t_first;
     int32_t L_b = clamp_len(p.seq_lens[b], p.max_seq_len);
-    int32_t parts_b = p.plan_parts[b];
-    int32_t nparts_b = p.plan_parts[b + 1] - parts_b;
+    int32_t seg_b = p.seg_base[b];
+    int32_t nseg_b = p.seg_base[b + 1] - seg_b;
+    int32_t k = p.first_k[c] - 1;  // segment index inside the sequence (advanced at starts)
     const int32_t* row = p.block_tables + static_cast<int64_t>(b) * p.table_stride;
     int32_t i = static_cast<int32_t>(lo - t_first);
     bool new_seq = true;
@@ -227,8 +271,9 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
         t_first = p.plan_tiles[b];
         n_b = p.plan_tiles[b + 1] - t_first;
         L_b = clamp_len(p.seq_lens[b], p.max_seq_len);
-        parts_b = p.plan_parts[b];
-        nparts_b = p.plan_parts[b + 1] - parts_b;
+        seg_b = p.seg_base[b];
+        nseg_b = p.seg_base[b + 1] - seg_b;
+        k = -1;
         row = p.block_tables + static_cast<int64_t>(b) * p.table_stride;
         i = 0;
         new_seq = true;
@@ -246,9 +291,12 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
       const int64_t seg_lo = max(part_lo, lo), seg_hi = min(part_hi, hi);
       int32_t flags = 0;
       if (new_seq) flags |= kNewSeq;
-      if (t == seg_lo) flags |= kSegStart;
+      if (t == seg_lo) {
+        flags |= kSegStart;
+        ++k;
+      }
       if (t == seg_hi - 1) flags |= kSegEnd;
-      if (nparts_b == 1 && seg_lo == t_first && seg_hi == t_first + n_b) flags |= kDirect;
+      if (nseg_b == 1) flags |= kDirect;
       new_seq = false;
 
       uint32_t mask = valid >= kTile ? 0xffffu : ((1u << valid) - 1u);
@@ -291,7 +339,7 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
       ti.b = b;
       ti.valid = valid;
       ti.mask = static_cast<int32_t>(mask);
-      ti.seg = parts_b + j + c;
+      ti.seg = seg_b + k;
       ti.flags = flags;
       mbar_arrive_expect_tx(full_k(stage), bytes);
       mbar_arrive_expect_tx(full_v(stage), bytes);
@@ -544,8 +592,11 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
 }
 
 // ---------------------------------------------------------------------------
-// combine: out[b, h] = sum_j w_j o_j / sum_j w_j,  w_j = l_j 2^(m_j - M)
-// grid (B, ceil(Hq / kCombineWarps)), one warp per query head
+// combine: out[b, h] = sum_k w_k o_k / sum_k w_k,  w_k = l_k 2^(m_k - M),
+// M = max_k m_k over the segments k of sequence b (slots seg_base[b] ..).
+// grid (B, ceil(Hq / kCombineWarps)), one warp per query head; the weights are
+// found with the lanes spread over segments, then the lanes (spread over
+// head_dim) stream the partial outputs with no dependence between segments.
 // ---------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(kCombineWarps * 32) pa_combine_kernel(const DecodeParams p) {
@@ -553,69 +604,56 @@ __global__ void __launch_bounds__(kCombineWarps * 32) pa_combine_kernel(const De
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int b = blockIdx.x;
   const int qh = blockIdx.y * kCombineWarps + warp;
+  griddep_wait();  // the main kernel's partials are complete and visible
   if (qh >= p.num_q_heads) return;
   const int G = p.group, HG = p.heads_per_cta;
-  const int kvh = qh / G, hg = kvh / HG;
+  const int hg = (qh / G) / HG;
   const int HGq = HG * G;
   const int qloc = qh - hg * HGq;
-  const int64_t C = p.ctas_per_group;
-  const int64_t N = p.plan_tiles[p.num_seqs];
-  const int32_t t0 = p.plan_tiles[b], t1 = p.plan_tiles[b + 1];
-  const int32_t pp0 = p.plan_parts[b], npart = p.plan_parts[b + 1] - pp0;
+  const int32_t s0 = p.seg_base[b], ns = p.seg_base[b + 1] - s0;
+  if (ns == 1) return;  // the main kernel wrote this sequence directly
   const int64_t obase = (static_cast<int64_t>(b) * p.num_q_heads + qh) * D + lane * V;
+  const int64_t sidx0 = (static_cast<int64_t>(hg) * p.nseg_cap + s0) * HGq + qloc;
+  const int32_t nvalid = (s0 + ns <= p.nseg_cap) ? ns : 0;
 
+  float M = -INFINITY;
+  for (int k = lane; k < nvalid; k += 32) {
+    const float m = p.part_ml[(sidx0 + static_cast<int64_t>(k) * HGq) * 2];
+    const float l = p.part_ml[(sidx0 + static_cast<int64_t>(k) * HGq) * 2 + 1];
+    if (l > 0.f) M = fmaxf(M, m);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
   float acc[V];
 #pragma unroll
-  for (int k = 0; k < V; ++k) acc[k] = 0.f;
-  float M = -INFINITY, Wsum = 0.f;
-  if (t1 > t0) {
-    if (npart == 1 && cta_of_tile(t0, N, C) == cta_of_tile(t1 - 1, N, C)) return;  // written by main
-    const int64_t tpp = (p.tiles_per_part == INT_MAX) ? (t1 - t0) : p.tiles_per_part;
-    for (int32_t j = 0; j < npart; ++j) {
-      const int64_t a = t0 + j * tpp;
-      const int64_t e = min(static_cast<int64_t>(t1), a + tpp);
-      const int32_t c0 = cta_of_tile(a, N, C), c1 = cta_of_tile(e - 1, N, C);
-      for (int32_t cc = c0; cc <= c1; ++cc) {
-        if (cc * N / C == (cc + 1) * N / C) continue;  // a CTA with an empty share wrote nothing
-        const int64_t seg = pp0 + j + cc;
-        if (seg >= p.nseg_cap) continue;
-        const int64_t sidx = (static_cast<int64_t>(hg) * p.nseg_cap + seg) * HGq + qloc;
-        const float m = p.part_ml[sidx * 2];
-        const float l = p.part_ml[sidx * 2 + 1];
-        if (!(l > 0.f)) continue;
-        const float* po = p.part_o + sidx * D + lane * V;
-        float o[V];
-        if constexpr (V == 4) {
-          const float4 v = *reinterpret_cast<const float4*>(po);
-          o[0] = v.x; o[1] = v.y; o[2] = v.z; o[3] = v.w;
-        } else {
-          const float2 v = *reinterpret_cast<const float2*>(po);
-          o[0] = v.x; o[1] = v.y;
-        }
-        if (m > M) {
-          const float r = (M == -INFINITY) ? 0.f : ex2(M - m);
-#pragma unroll
-          for (int k = 0; k < V; ++k) acc[k] *= r;
-          Wsum *= r;
-          M = m;
-        }
-        const float w = l * ex2(m - M);
-#pragma unroll
-        for (int k = 0; k < V; ++k) acc[k] += w * o[k];
-        Wsum += w;
-      }
-    }
-  }
-  const float inv = Wsum > 0.f ? 1.f / Wsum : 0.f;
-#pragma unroll
-  for (int k = 0; k < V; ++k) {
-    const float v = acc[k] * inv;
-    if (p.out_dtype == PA_F32) {
-      static_cast<float*>(p.out)[obase + k] = v;
-    } else if (p.out_dtype == PA_BF16) {
-      static_cast<__nv_bfloat16*>(p.out)[obase + k] = __float2bfloat16_rn(v);
+  for (int v = 0; v < V; ++v) acc[v] = 0.f;
+  float W = 0.f;
+#pragma unroll 4
+  for (int k = 0; k < nvalid; ++k) {
+    const int64_t sidx = sidx0 + static_cast<int64_t>(k) * HGq;
+    const float m = p.part_ml[sidx * 2];
+    const float l = p.part_ml[sidx * 2 + 1];
+    const float w = l > 0.f ? l * ex2(m - M) : 0.f;
+    const float* po = p.part_o + sidx * D + lane * V;
+    if constexpr (V == 4) {
+      const float4 o4 = *reinterpret_cast<const float4*>(po);
+      acc[0] += w * o4.x; acc[1] += w * o4.y; acc[2] += w * o4.z; acc[3] += w * o4.w;
     } else {
-      static_cast<__half*>(p.out)[obase + k] = __float2half_rn(v);
+      const float2 o2 = *reinterpret_cast<const float2*>(po);
+      acc[0] += w * o2.x; acc[1] += w * o2.y;
+    }
+    W += w;
+  }
+  const float inv = W > 0.f ? 1.f / W : 0.f;
+#pragma unroll
+  for (int v = 0; v < V; ++v) {
+    const float x = acc[v] * inv;
+    if (p.out_dtype == PA_F32) {
+      static_cast<float*>(p.out)[obase + v] = x;
+    } else if (p.out_dtype == PA_BF16) {
+      static_cast<__nv_bfloat16*>(p.out)[obase + v] = __float2bfloat16_rn(x);
+    } else {
+      static_cast<__half*>(p.out)[obase + v] = __float2half_rn(x);
     }
   }
 }
@@ -646,7 +684,8 @@ struct LaunchPlan {
   int HG = 0, groups = 0, stages = 0, tok_box = 0, threads = 0;
   int ctas_per_group = 0, tiles_per_part = INT_MAX, nseg_cap = 0;
   size_t smem = 0;
-  size_t off_tiles = 0, off_parts = 0, off_o = 0, off_ml = 0, total = 0;
+  size_t off_tiles = 0, off_segs = 0, off_start = 0, off_firstk = 0, off_o = 0, off_ml = 0,
+         total = 0;
   MainKernel kernel = nullptr;
 };
 
@@ -705,8 +744,10 @@ pa_status make_plan(int32_t num_seqs, int32_t Hq, int32_t Hkv, int32_t D, int32_
   if (nseg > INT_MAX / 2) return PA_ERR_UNSUPPORTED;
   lp->nseg_cap = static_cast<int>(nseg);
   lp->off_tiles = 0;
-  lp->off_parts = align_up(static_cast<size_t>(num_seqs + 1) * 4, 256);
-  lp->off_o = lp->off_parts + align_up(static_cast<size_t>(num_seqs + 1) * 4, 256);
+  lp->off_segs = align_up(static_cast<size_t>(num_seqs + 1) * 4, 256);
+  lp->off_start = lp->off_segs + align_up(static_cast<size_t>(num_seqs + 1) * 4, 256);
+  lp->off_firstk = lp->off_start + align_up(static_cast<size_t>(lp->ctas_per_group) * 4, 256);
+  lp->off_o = lp->off_firstk + align_up(static_cast<size_t>(lp->ctas_per_group) * 4, 256);
   const size_t o_bytes = static_cast<size_t>(lp->groups) * nseg * HG * G * D * sizeof(float);
   lp->off_ml = lp->off_o + align_up(o_bytes, 256);
   const size_t ml_bytes = static_cast<size_t>(lp->groups) * nseg * HG * G * 2 * sizeof(float);
@@ -809,22 +850,26 @@ extern "C" pa_status pa_decode_attention(
   p.tok_box = lp.tok_box;
   p.tma_mode = mode;
   p.plan_tiles = reinterpret_cast<int32_t*>(ws + lp.off_tiles);
-  p.plan_parts = reinterpret_cast<int32_t*>(ws + lp.off_parts);
+  p.seg_base = reinterpret_cast<int32_t*>(ws + lp.off_segs);
+  p.start_seq = reinterpret_cast<int32_t*>(ws + lp.off_start);
+  p.first_k = reinterpret_cast<int32_t*>(ws + lp.off_firstk);
   p.part_o = reinterpret_cast<float*>(ws + lp.off_o);
   p.part_ml = reinterpret_cast<float*>(ws + lp.off_ml);
   p.err = device_error_flag;
 
+  // All three launches use programmatic dependent launch: each may start while
+  // its predecessor runs and waits (griddepcontrol.wait) before touching data.
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  pa_plan_kernel<<<1, kPlanThreads, 0, s>>>(p);
-  lp.kernel<<<dim3(lp.ctas_per_group, lp.groups), lp.threads, lp.smem, s>>>(tmK, tmV, p);
-  const dim3 cgrid(num_seqs, (num_q_heads + kCombineWarps - 1) / kCombineWarps);
-  if (D == 128) {
-    pa_combine_kernel<128><<<cgrid, kCombineWarps * 32, 0, s>>>(p);
-  } else {
-    pa_combine_kernel<64><<<cgrid, kCombineWarps * 32, 0, s>>>(p);
-  }
-  if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
-  return PA_OK;
+  if (PdlLaunch(s, dim3(1), dim3(kPlanThreads))(pa_plan_kernel, p) != cudaSuccess)
+    return PA_ERR_CUDA;
+  if (PdlLaunch(s, dim3(lp.ctas_per_group, lp.groups), dim3(lp.threads), lp.smem)(
+          lp.kernel, tmK, tmV, p) != cudaSuccess)
+    return PA_ERR_CUDA;
+  PdlLaunch combine(s, dim3(num_seqs, (num_q_heads + kCombineWarps - 1) / kCombineWarps),
+                    dim3(kCombineWarps * 32));
+  const cudaError_t e3 =
+      D == 128 ? combine(pa_combine_kernel<128>, p) : combine(pa_combine_kernel<64>, p);
+  return e3 == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
 // ===========================================================================

@@ -8,6 +8,7 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <utility>
 
 #include "../../include/pagedattn.h"
 
@@ -39,5 +40,28 @@ inline bool aligned(const void* p, size_t a) {
 // Returns false if the driver rejects the description.
 bool get_tensor_map(CUtensorMap* out, const void* base, const uint64_t dims[5],
                     const uint64_t strides[4], const uint32_t box[5]);
+
+// Launches kernels with programmatic dependent launch on `stream`: the kernel
+// may start while the previous kernel on the stream finishes and must call
+// griddepcontrol.wait before it touches memory that kernel may write.
+struct PdlLaunch {
+  cudaLaunchConfig_t cfg;
+  cudaLaunchAttribute attr;
+  PdlLaunch(cudaStream_t stream, dim3 grid, dim3 block, size_t smem = 0) {
+    attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr.val.programmaticStreamSerializationAllowed = 1;
+    cfg = cudaLaunchConfig_t{};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+  }
+  template <typename... KArgs, typename... Args>
+  cudaError_t operator()(void (*kernel)(KArgs...), Args&&... args) {
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+  }
+};
 
 }  // namespace pa
