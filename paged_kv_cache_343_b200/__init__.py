@@ -310,52 +310,79 @@ class BlockManager:
 class PagedDecodeStep:
     """One decode step driven from pinned host memory (the end-to-end call).
 
-    Holds device buffers for a fixed batch shape.  ``__call__`` copies the
-    step's inputs host->device (query, new K/V rows, slot_mapping, block
-    tables, seq_lens), writes the new rows into the pools with
-    reshape_and_cache, runs decode_attention, and copies the output back
-    device->host, all on one stream, then waits for it."""
+    Holds, for a fixed batch shape, one pinned host staging buffer and a device
+    buffer of the same layout.  The caller writes the step's inputs into the
+    views of ``host`` (``q``, ``new_k``, ``new_v``, ``slots``, ``tables``,
+    ``lens``); a call copies the whole staging buffer host->device in one copy,
+    writes the new rows into the pools with reshape_and_cache, runs
+    decode_attention, copies the output into the pinned ``host_out`` in one copy
+    and waits for the stream.  With ``use_graph`` (default) the first call runs
+    eagerly and captures the step (copies and kernels) into a CUDA graph that
+    later calls replay."""
+
+    _ALIGN = 256
 
     def __init__(self, key_cache: torch.Tensor, value_cache: torch.Tensor, num_seqs: int,
                  num_q_heads: int, table_width: int, max_seq_len: int, scale: float,
                  partition_size: int = 0, out_dtype: Optional[torch.dtype] = None,
-                 stream: Optional[torch.cuda.Stream] = None):
+                 stream: Optional[torch.cuda.Stream] = None, use_graph: bool = True):
         self.k, self.v = key_cache, value_cache
         nb, bs, hkv, d = key_cache.shape
         dev = key_cache.device
         dt = key_cache.dtype
-        self.shape = (num_seqs, num_q_heads, d)
         self.max_seq_len, self.scale, self.partition_size = max_seq_len, scale, partition_size
         self.stream = stream if stream is not None else torch.cuda.Stream(device=dev)
-        self.q = torch.empty(self.shape, dtype=dt, device=dev)
-        self.new_k = torch.empty((num_seqs, hkv, d), dtype=dt, device=dev)
-        self.new_v = torch.empty((num_seqs, hkv, d), dtype=dt, device=dev)
-        self.slots = torch.empty(num_seqs, dtype=torch.int32, device=dev)
-        self.tables = torch.empty((num_seqs, table_width), dtype=torch.int32, device=dev)
-        self.lens = torch.empty(num_seqs, dtype=torch.int32, device=dev)
-        self.out = torch.empty(self.shape, dtype=out_dtype or dt, device=dev)
+        self.use_graph = use_graph
+        self.graph = None
+        fields = [("q", (num_seqs, num_q_heads, d), dt), ("new_k", (num_seqs, hkv, d), dt),
+                  ("new_v", (num_seqs, hkv, d), dt), ("slots", (num_seqs,), torch.int32),
+                  ("tables", (num_seqs, table_width), torch.int32),
+                  ("lens", (num_seqs,), torch.int32)]
+        layout, off = [], 0
+        for name, shape, dtype in fields:
+            nbytes = int(torch.Size(shape).numel()) * torch.empty((), dtype=dtype).element_size()
+            layout.append((name, shape, dtype, off, nbytes))
+            off += -(-nbytes // self._ALIGN) * self._ALIGN
+        self._nbytes = off
+        self._host_buf = torch.empty(off, dtype=torch.uint8).pin_memory()
+        self._dev_buf = torch.empty(off, dtype=torch.uint8, device=dev)
+
+        def views(buf):
+            return {name: buf[o:o + n].view(dtype).view(shape) for name, shape, dtype, o, n in layout}
+
+        self.host = views(self._host_buf)
+        self.dev = views(self._dev_buf)
+        self.out = torch.empty((num_seqs, num_q_heads, d), dtype=out_dtype or dt, device=dev)
+        self.host_out = torch.empty(self.out.shape, dtype=self.out.dtype).pin_memory()
         self.ws = alloc_workspace(decode_workspace_bytes(num_seqs, num_q_heads, hkv, d, bs,
                                                          max_seq_len, partition_size), dev)
 
     def h2d_bytes(self) -> int:
-        return sum(t.numel() * t.element_size()
-                   for t in (self.q, self.new_k, self.new_v, self.slots, self.tables, self.lens))
+        return self._nbytes
 
     def d2h_bytes(self) -> int:
         return self.out.numel() * self.out.element_size()
 
-    def __call__(self, q_host, new_k_host, new_v_host, slots_host, tables_host, lens_host,
-                 out_host) -> None:
-        s = self.stream
-        with torch.cuda.stream(s):
-            self.q.copy_(q_host, non_blocking=True)
-            self.new_k.copy_(new_k_host, non_blocking=True)
-            self.new_v.copy_(new_v_host, non_blocking=True)
-            self.slots.copy_(slots_host, non_blocking=True)
-            self.tables.copy_(tables_host, non_blocking=True)
-            self.lens.copy_(lens_host, non_blocking=True)
-            reshape_and_cache(self.new_k, self.new_v, self.k, self.v, self.slots, stream=s)
-            decode_attention(self.out, self.q, self.k, self.v, self.tables, self.lens,
-                             self.max_seq_len, self.scale, self.partition_size, self.ws, stream=s)
-            out_host.copy_(self.out, non_blocking=True)
-        s.synchronize()
+    def _enqueue(self) -> None:
+        dv = self.dev
+        self._dev_buf.copy_(self._host_buf, non_blocking=True)
+        reshape_and_cache(dv["new_k"], dv["new_v"], self.k, self.v, dv["slots"])
+        decode_attention(self.out, dv["q"], self.k, self.v, dv["tables"], dv["lens"],
+                         self.max_seq_len, self.scale, self.partition_size, self.ws)
+        self.host_out.copy_(self.out, non_blocking=True)
+
+    def __call__(self) -> torch.Tensor:
+        if self.graph is not None:
+            with torch.cuda.stream(self.stream):
+                self.graph.replay()
+            self.stream.synchronize()
+            return self.host_out
+        with torch.cuda.stream(self.stream):
+            self._enqueue()
+        self.stream.synchronize()
+        if self.use_graph:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=self.stream, capture_error_mode="thread_local"):
+                self._enqueue()
+            self.graph = g
+        return self.host_out

@@ -157,14 +157,19 @@ __device__ int32_t plan_sequence_segments(const DecodeParams& p, int32_t b, int6
   return count;
 }
 
+constexpr int kPlanRegChunks = 8;  // batches up to 8 x 256 sequences keep their counts in registers
+
 __global__ void __launch_bounds__(kPlanThreads) pa_plan_kernel(DecodeParams p) {
   __shared__ int32_t warp_buf[kPlanWarps];
   const int tid = threadIdx.x;
   griddep_launch_dependents();
   griddep_wait();  // seq_lens may come from the previous kernel on the stream
+  const int nchunks = (p.num_seqs + kPlanThreads - 1) / kPlanThreads;
+  const bool in_regs = nchunks <= kPlanRegChunks;
+  int32_t t_reg[kPlanRegChunks], n_reg[kPlanRegChunks];
   int32_t carry = 0, total = 0;
-  for (int base = 0; base < p.num_seqs; base += kPlanThreads) {
-    const int b = base + tid;
+  for (int ch = 0; ch < nchunks; ++ch) {
+    const int b = ch * kPlanThreads + tid;
     int32_t nt = 0;
     if (b < p.num_seqs) {
       const int32_t raw = p.seq_lens[b];
@@ -173,17 +178,36 @@ __global__ void __launch_bounds__(kPlanThreads) pa_plan_kernel(DecodeParams p) {
     }
     const int32_t ex = block_exclusive_scan(nt, warp_buf, &total);
     if (b < p.num_seqs) p.plan_tiles[b] = carry + ex;
+#pragma unroll
+    for (int r = 0; r < kPlanRegChunks; ++r) {
+      if (r == ch) {
+        t_reg[r] = carry + ex;
+        n_reg[r] = nt;
+      }
+    }
     carry += total;
   }
   if (tid == 0) p.plan_tiles[p.num_seqs] = carry;
-  __syncthreads();
+  if (!in_regs) __syncthreads();  // the global copy is read back below
   const int64_t N = carry, C = p.ctas_per_group;
   int32_t seg_carry = 0;
-  for (int base = 0; base < p.num_seqs; base += kPlanThreads) {
-    const int b = base + tid;
+  for (int ch = 0; ch < nchunks; ++ch) {
+    const int b = ch * kPlanThreads + tid;
     int32_t ns = 0;
     if (b < p.num_seqs && N > 0) {
-      const int64_t t0 = p.plan_tiles[b], t1 = p.plan_tiles[b + 1];
+      int64_t t0 = 0, t1 = 0;
+      if (in_regs) {
+#pragma unroll
+        for (int r = 0; r < kPlanRegChunks; ++r) {
+          if (r == ch) {
+            t0 = t_reg[r];
+            t1 = t0 + n_reg[r];
+          }
+        }
+      } else {
+        t0 = p.plan_tiles[b];
+        t1 = p.plan_tiles[b + 1];
+      }
       if (t1 > t0) ns = plan_sequence_segments(p, b, t0, t1, N, C);
     }
     const int32_t ex = block_exclusive_scan(ns, warp_buf, &total);

@@ -262,3 +262,103 @@ def test_decode_full_size(pa, orc, name):
     out = _run(pa, prep, k=dk, v=dv)
     assert _maxerr(out, ref, seqs) <= TOL_STORED
     assert torch.isfinite(out.float()).all()
+
+
+def test_copy_on_write_step_end_to_end(pa, orc):
+    """Parallel sampling with a shared prompt, all on the GPU: the native block
+    manager plans the step (same tables, slots and copy pairs as the reference
+    manager), copy_blocks makes the copies, reshape_and_cache writes every
+    sample's new tokens, decode attends -- against the oracle doing the same
+    three steps.  Invariants: shared full prompt blocks are untouched, at most one
+    copy per sequence, copy targets are distinct, refcounts match the tables."""
+    import oracle
+    spec = W.WORKLOADS["shared_prefix"].replace(prompts=3, num_seqs=24, seed=71)
+    prep = prepare(spec)
+    s = prep.case.spec
+    bm_ref = prep.extra["bm"]
+    # the native manager, driven by the same operations
+    bm = pa.BlockManager(prep.case.num_blocks, s.block_size, prep.case.free_order)
+    sid = 0
+    for _ in range(s.prompts):
+        bm.add_sequence(sid, s.prompt_len)
+        for k in range(1, s.samples):
+            bm.fork(sid, sid + k)
+        sid += s.samples
+    slots, cow = [], []
+    for b in range(s.num_seqs):
+        for _ in range(int(prep.case.extra_tokens[b])):
+            slot, c = bm.append_slot(b)
+            slots.append(slot)
+            if c is not None:
+                cow.append(c)
+    assert slots == prep.new_slots.tolist()
+    assert cow == [tuple(x) for x in prep.cow_pairs.tolist()]
+    for b in range(s.num_seqs):
+        assert bm.block_table(b) == bm_ref.block_table(b)
+    assert all(bm.refcount(i) == bm_ref.refcount[i] for i in range(prep.case.num_blocks))
+    # invariants of the plan
+    dst = [d for _, d in cow]
+    assert len(set(dst)) == len(dst)
+    assert len(cow) <= s.num_seqs and len(cow) == s.prompts * (s.samples - 1)
+    full_prompt_blocks = sorted({blk for b in range(0, s.num_seqs, s.samples)
+                                 for blk in bm_ref.block_table(b)[: s.prompt_len // s.block_size]})
+    for blk in full_prompt_blocks:
+        assert bm.refcount(blk) == s.samples
+    # oracle chain
+    k, v = prep.k_pool.copy(), prep.v_pool.copy()
+    block_bytes = int(np.prod(k.shape[1:])) * 2
+    oracle.copy_blocks([k, v], prep.cow_pairs, block_bytes)
+    oracle.reshape_and_cache(prep.case.new_k, prep.case.new_v, k, v, prep.new_slots)
+    ref = _oracle(orc, prep, k=k, v=v)
+    # GPU chain
+    dk, dv = to_dev(prep.k_pool, s.dtype), to_dev(prep.v_pool, s.dtype)
+    flag = torch.zeros(1, dtype=torch.int32, device="cuda")
+    pa.copy_blocks([dk], [dv], to_dev(prep.cow_pairs), error_flag=flag)
+    pa.reshape_and_cache(to_dev(prep.case.new_k, s.dtype), to_dev(prep.case.new_v, s.dtype),
+                         dk, dv, to_dev(prep.new_slots), error_flag=flag)
+    out = _run(pa, prep, k=dk, v=dv, out_dtype=torch.float32, flag=flag)
+    assert int(flag.item()) == 0
+    from harness import bits_of
+    assert np.array_equal(bits_of(dk), k) and np.array_equal(bits_of(dv), v)
+    # shared full blocks are bit-identical to their initial contents
+    assert np.array_equal(bits_of(dk)[full_prompt_blocks], prep.k_pool[full_prompt_blocks])
+    assert np.array_equal(bits_of(dv)[full_prompt_blocks], prep.v_pool[full_prompt_blocks])
+    assert _maxerr(out, ref) <= TOL_F32
+
+
+@pytest.mark.parametrize("use_graph", [False, True])
+def test_end_to_end_step_from_host_buffers(pa, orc, use_graph):
+    """PagedDecodeStep: pinned host inputs -> reshape_and_cache + decode ->
+    pinned host output, three steps in a row with new inputs each step."""
+    spec = W.WORKLOADS["llama8b"].replace(num_seqs=5, len_lo=40, len_hi=600, seed=41)
+    prep = prepare(spec)
+    s = prep.case.spec
+    B = s.num_seqs
+    bm = prep.extra["bm"]
+    dk, dv = to_dev(prep.k_pool, s.dtype), to_dev(prep.v_pool, s.dtype)
+    k_ref, v_ref = prep.k_pool.copy(), prep.v_pool.copy()
+    width = prep.tables.shape[1] + 4
+    step = pa.PagedDecodeStep(dk, dv, B, s.num_q_heads, width, int(prep.seq_lens.max()) + 8,
+                              W.scale_of(s), use_graph=use_graph)
+    td = {"bf16": torch.bfloat16, "f16": torch.float16}[s.dtype]
+    h = step.host
+    g = torch.Generator().manual_seed(3)
+    for it in range(3):
+        slots = np.array([bm.append_slot(b)[0] for b in range(B)], np.int32)
+        lens = np.array([bm.lengths[b] for b in range(B)], np.int32)
+        tables = np.full((B, width), -1, np.int32)
+        for b in range(B):
+            t = bm.block_table(b)
+            tables[b, :len(t)] = t
+        q = W.randn_bits((B, s.num_q_heads, s.head_dim), s.dtype, g)
+        nk = W.randn_bits((B, s.num_kv_heads, s.head_dim), s.dtype, g)
+        nv = W.randn_bits((B, s.num_kv_heads, s.head_dim), s.dtype, g)
+        for name, src in (("q", q), ("new_k", nk), ("new_v", nv)):
+            h[name].copy_(torch.from_numpy(src).view(torch.int16).view(td))
+        h["slots"].copy_(torch.from_numpy(slots))
+        h["tables"].copy_(torch.from_numpy(tables))
+        h["lens"].copy_(torch.from_numpy(lens))
+        out = step()
+        orc.reshape_and_cache(nk, nv, k_ref, v_ref, slots)
+        ref = orc.decode(q, k_ref, v_ref, tables, lens, W.scale_of(s), s.dtype, nthreads=4)
+        assert np.max(np.abs(out.double().numpy() - ref)) <= TOL_STORED
