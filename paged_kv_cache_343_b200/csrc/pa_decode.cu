@@ -657,7 +657,8 @@ __global__ void __launch_bounds__(kCombineWarps * 32) pa_combine_kernel(const De
     const int64_t sidx = sidx0 + static_cast<int64_t>(k) * HGq;
     const float m = p.part_ml[sidx * 2];
     const float l = p.part_ml[sidx * 2 + 1];
-    const float w = l > 0.f ? l * ex2(m - M) : 0.f;
+    if (!(l > 0.f)) continue;  // nothing attended in this partial: skip it, never 0 * o
+    const float w = l * ex2(m - M);
     const float* po = p.part_o + sidx * D + lane * V;
     if constexpr (V == 4) {
       const float4 o4 = *reinterpret_cast<const float4*>(po);
