@@ -18,6 +18,10 @@ What each function follows (page title and section):
   parallel sampling?".
 * ``decode``         -- "PagedAttention", "How attention reads paged memory":
   gather through the block table, then softmax(scale q K^T) V in fp64.
+* ``reshape_and_cache_fp8`` / ``decode_fp8`` -- the same over a cache of 8-bit
+  E4M3 codes ("write_to_paged_cache" takes kv_cache_dtype, k_scale, v_scale;
+  the pages show only "auto", so the fp8 rule is a reading: the cache holds
+  e4m3(x / scale) and reads back code * scale).
 
 Pins (tests/test_oracle.py): the pages' worked example and code example, a
 pure-Python ``math.fsum`` brute force (``oracle.brute``), the float64 library
@@ -72,6 +76,16 @@ def _load():
                                               i32, i32, i32]
         lib.orc_copy_blocks.restype = None
         lib.orc_copy_blocks.argtypes = [p, i32, p, i64, i64]
+        lib.orc_e4m3_to_double.restype = ctypes.c_double
+        lib.orc_e4m3_to_double.argtypes = [ctypes.c_uint8]
+        lib.orc_float_to_e4m3.restype = ctypes.c_uint8
+        lib.orc_float_to_e4m3.argtypes = [ctypes.c_float]
+        lib.orc_reshape_and_cache_fp8.restype = None
+        lib.orc_reshape_and_cache_fp8.argtypes = [p, p, i64, i64, p, p, p, i64, i32, i32, i32,
+                                                  i32, ctypes.c_float, ctypes.c_float]
+        lib.orc_decode_fp8.restype = ctypes.c_int
+        lib.orc_decode_fp8.argtypes = [p, p, p, p, ctypes.c_double, ctypes.c_double, p, i64, p,
+                                       i32, i32, i32, i32, i32, ctypes.c_double, i32, i32]
         lib.orc_decode.restype = ctypes.c_int
         lib.orc_decode.argtypes = [p, p, p, p, p, i64, p, i32, i32, i32, i32,
                                    i32, ctypes.c_double, i32, i32]
@@ -163,4 +177,62 @@ def decode(q: np.ndarray, key_cache: np.ndarray, value_cache: np.ndarray,
                         float(scale), _dtype_code(dtype), int(nthreads))
     if rc != 0:
         raise RuntimeError("orc_decode failed with code %d" % rc)
+    return out
+
+
+# --------------------------------------------------------------------------
+# fp8 (E4M3) cache: codes = e4m3(x / scale) taken in float; reads code * scale
+# --------------------------------------------------------------------------
+def e4m3_to_double(codes) -> np.ndarray:
+    """Decode E4M3 codes (uint8), element by element."""
+    lib = _load()
+    flat = np.asarray(codes, dtype=np.uint8).ravel()
+    return np.array([lib.orc_e4m3_to_double(int(c)) for c in flat],
+                    dtype=np.float64).reshape(np.shape(codes))
+
+
+def float_to_e4m3(x) -> np.ndarray:
+    """Nearest E4M3 code of each float32 value (ties to even, saturating at 448)."""
+    lib = _load()
+    flat = np.asarray(x, dtype=np.float32).ravel()
+    return np.array([lib.orc_float_to_e4m3(float(v)) for v in flat],
+                    dtype=np.uint8).reshape(np.shape(x))
+
+
+def reshape_and_cache_fp8(key: np.ndarray, value: np.ndarray, key_cache: np.ndarray,
+                          value_cache: np.ndarray, slot_mapping: np.ndarray, dtype,
+                          k_scale: float, v_scale: float) -> None:
+    """Write key/value [T, Hkv, D] (uint16 bits of ``dtype``) into uint8 code
+    pools [num_blocks, block_size, Hkv, D] in place."""
+    lib = _load()
+    assert key_cache.dtype == np.uint8 and key_cache.flags.c_contiguous
+    assert value_cache.dtype == np.uint8 and value_cache.flags.c_contiguous
+    k = np.ascontiguousarray(key, dtype=np.uint16)
+    v = np.ascontiguousarray(value, dtype=np.uint16)
+    sm = np.ascontiguousarray(slot_mapping, dtype=np.int32)
+    _, bs, hkv, d = key_cache.shape
+    lib.orc_reshape_and_cache_fp8(_ptr(k), _ptr(v), hkv * d, hkv * d, _ptr(key_cache),
+                                  _ptr(value_cache), _ptr(sm), sm.shape[0], bs, hkv, d,
+                                  _dtype_code(dtype), float(k_scale), float(v_scale))
+
+
+def decode_fp8(q: np.ndarray, key_cache: np.ndarray, value_cache: np.ndarray,
+               k_scale: float, v_scale: float, block_tables: np.ndarray,
+               seq_lens: np.ndarray, scale: float, q_dtype, nthreads: int = 1) -> np.ndarray:
+    """fp64 paged decode attention over an E4M3 cache (elements read as
+    code * k_scale / code * v_scale); q holds uint16 bits of ``q_dtype``."""
+    lib = _load()
+    qq = np.ascontiguousarray(q, dtype=np.uint16)
+    assert key_cache.dtype == np.uint8 and value_cache.dtype == np.uint8
+    bt = np.ascontiguousarray(block_tables, dtype=np.int32)
+    sl = np.ascontiguousarray(seq_lens, dtype=np.int32)
+    B, Hq, D = qq.shape
+    _, bs, hkv, d2 = key_cache.shape
+    assert d2 == D and bt.shape[0] == B and sl.shape[0] == B
+    out = np.empty((B, Hq, D), dtype=np.float64)
+    rc = lib.orc_decode_fp8(_ptr(out), _ptr(qq), _ptr(key_cache), _ptr(value_cache),
+                            float(k_scale), float(v_scale), _ptr(bt), bt.shape[1], _ptr(sl), B,
+                            Hq, hkv, D, bs, float(scale), _dtype_code(q_dtype), int(nthreads))
+    if rc != 0:
+        raise RuntimeError("orc_decode_fp8 failed with code %d" % rc)
     return out

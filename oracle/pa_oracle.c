@@ -83,6 +83,57 @@ double orc_bf16_to_double(uint16_t b) {
   return sign ? -v : v;
 }
 
+/* ---------------------------------------------------------------------------
+ * 8-bit float, E4M3 variant of the OCP 8-bit floating point formats: 1 sign
+ * bit, 4 exponent bits (bias 7), 3 mantissa bits, no infinities, one NaN
+ * pattern per sign (exponent and mantissa all ones); the largest finite value
+ * is 448 and the smallest subnormal 2^-9.
+ * ------------------------------------------------------------------------- */
+double orc_e4m3_to_double(uint8_t c) {
+  int sign = (c >> 7) & 1;
+  int e = (c >> 3) & 0xf;
+  int m = c & 0x7;
+  double v;
+  if (e == 15 && m == 7) {
+    v = NAN;
+  } else if (e == 0) {
+    v = ldexp((double)m, -9); /* m/8 * 2^(1-7) */
+  } else {
+    v = ldexp((double)(8 + m), e - 10); /* (1 + m/8) * 2^(e-7) */
+  }
+  return sign ? -v : v;
+}
+
+/* Nearest E4M3 code to the float x, ties to the even code, finite values
+ * beyond 448 saturate to +-448; NaN gives the NaN code.  Written as a search
+ * over the 127 non-negative finite codes, which are ordered by value. */
+uint8_t orc_float_to_e4m3(float x) {
+  if (x != x) return 0x7f;
+  uint8_t sign = (x < 0.0f || (x == 0.0f && signbit(x))) ? 0x80 : 0x00;
+  double a = fabs((double)x);
+  if (a >= 448.0) return sign | 0x7e;
+  uint8_t best = 0;
+  double best_err = INFINITY;
+  for (int c = 0; c <= 0x7e; ++c) {
+    double err = fabs(orc_e4m3_to_double((uint8_t)c) - a);
+    if (err < best_err || (err == best_err && (c & 1) == 0)) {
+      best = (uint8_t)c;
+      best_err = err;
+    }
+  }
+  return sign | best;
+}
+
+/* reshape_and_cache into an fp8 cache: the code of key[t, h, d] / k_scale,
+ * the quotient taken in float (single precision), as the cache stores it. */
+void orc_reshape_and_cache_fp8(const uint16_t* key, const uint16_t* value,
+                               int64_t key_stride_t, int64_t value_stride_t,
+                               uint8_t* key_cache, uint8_t* value_cache,
+                               const int32_t* slot_mapping, int64_t num_tokens,
+                               int32_t block_size, int32_t num_kv_heads,
+                               int32_t head_dim, int32_t dtype, float k_scale,
+                               float v_scale);
+
 static double orc_decode16(uint16_t bits, int dtype) {
   return dtype == ORC_BF16 ? orc_bf16_to_double(bits) : orc_half_to_double(bits);
 }
@@ -138,6 +189,30 @@ void orc_reshape_and_cache(const uint16_t* key, const uint16_t* value,
   }
 }
 
+void orc_reshape_and_cache_fp8(const uint16_t* key, const uint16_t* value,
+                               int64_t key_stride_t, int64_t value_stride_t,
+                               uint8_t* key_cache, uint8_t* value_cache,
+                               const int32_t* slot_mapping, int64_t num_tokens,
+                               int32_t block_size, int32_t num_kv_heads,
+                               int32_t head_dim, int32_t dtype, float k_scale,
+                               float v_scale) {
+  for (int64_t t = 0; t < num_tokens; ++t) {
+    int64_t s = slot_mapping[t];
+    if (s < 0) continue;
+    int64_t block = s / block_size;
+    int64_t offset = s % block_size;
+    for (int32_t h = 0; h < num_kv_heads; ++h) {
+      int64_t dst = ((block * block_size + offset) * num_kv_heads + h) * head_dim;
+      for (int32_t d = 0; d < head_dim; ++d) {
+        float k = (float)orc_decode16(key[t * key_stride_t + (int64_t)h * head_dim + d], dtype);
+        float v = (float)orc_decode16(value[t * value_stride_t + (int64_t)h * head_dim + d], dtype);
+        key_cache[dst + d] = orc_float_to_e4m3(k / k_scale);
+        value_cache[dst + d] = orc_float_to_e4m3(v / v_scale);
+      }
+    }
+  }
+}
+
 /* ---------------------------------------------------------------------------
  * copy_blocks (copy-on-write): for every (src, dst) pair, the whole physical
  * block dst of every layer's K and V pool becomes a byte copy of block src.
@@ -179,6 +254,9 @@ typedef struct {
   const uint16_t* q;
   const uint16_t* key_cache;
   const uint16_t* value_cache;
+  const uint8_t* key_cache8;   /* fp8 cache (when not NULL, instead of the 16-bit ones) */
+  const uint8_t* value_cache8;
+  double k_scale, v_scale;
   const int32_t* block_tables;
   int64_t table_stride;
   const int32_t* seq_lens;
@@ -213,8 +291,13 @@ static int orc_decode_one(orc_decode_job* j, int32_t b) {
     for (int32_t g = 0; g < Hkv; ++g) {
       for (int32_t d = 0; d < D; ++d) {
         int64_t src = (slot * Hkv + g) * D + d;
-        Kc[(t * Hkv + g) * D + d] = orc_decode16(j->key_cache[src], j->dtype);
-        Vc[(t * Hkv + g) * D + d] = orc_decode16(j->value_cache[src], j->dtype);
+        if (j->key_cache8) {
+          Kc[(t * Hkv + g) * D + d] = orc_e4m3_to_double(j->key_cache8[src]) * j->k_scale;
+          Vc[(t * Hkv + g) * D + d] = orc_e4m3_to_double(j->value_cache8[src]) * j->v_scale;
+        } else {
+          Kc[(t * Hkv + g) * D + d] = orc_decode16(j->key_cache[src], j->dtype);
+          Vc[(t * Hkv + g) * D + d] = orc_decode16(j->value_cache[src], j->dtype);
+        }
       }
     }
   }
@@ -260,16 +343,22 @@ static void* orc_decode_worker(void* arg) {
   return NULL;
 }
 
-/* Returns 0 on success, 1 on allocation failure, 2 on a bad argument. */
-int orc_decode(double* out, const uint16_t* q, const uint16_t* key_cache,
-               const uint16_t* value_cache, const int32_t* block_tables,
-               int64_t table_stride, const int32_t* seq_lens, int32_t num_seqs,
-               int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
-               int32_t block_size, double scale, int32_t dtype,
-               int32_t nthreads) {
+/* Returns 0 on success, 1 on allocation failure, 2 on a bad argument.
+ * With key_cache8 / value_cache8 not NULL the cache holds E4M3 codes and a
+ * stored element reads as code * k_scale (keys) or code * v_scale (values);
+ * the query keeps its 16-bit type (dtype). */
+static int orc_decode_impl(double* out, const uint16_t* q, const uint16_t* key_cache,
+                           const uint16_t* value_cache, const uint8_t* key_cache8,
+                           const uint8_t* value_cache8, double k_scale, double v_scale,
+                           const int32_t* block_tables, int64_t table_stride,
+                           const int32_t* seq_lens, int32_t num_seqs, int32_t num_q_heads,
+                           int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                           double scale, int32_t dtype, int32_t nthreads) {
   if (num_kv_heads <= 0 || num_q_heads % num_kv_heads != 0 || block_size <= 0)
     return 2;
   orc_decode_job j;
+  j.key_cache8 = key_cache8; j.value_cache8 = value_cache8;
+  j.k_scale = k_scale; j.v_scale = v_scale;
   j.out = out; j.q = q; j.key_cache = key_cache; j.value_cache = value_cache;
   j.block_tables = block_tables; j.table_stride = table_stride;
   j.seq_lens = seq_lens; j.num_seqs = num_seqs; j.num_q_heads = num_q_heads;
@@ -289,4 +378,26 @@ int orc_decode(double* out, const uint16_t* q, const uint16_t* key_cache,
   }
   pthread_mutex_destroy(&j.mu);
   return j.failed ? 1 : 0;
+}
+
+int orc_decode(double* out, const uint16_t* q, const uint16_t* key_cache,
+               const uint16_t* value_cache, const int32_t* block_tables,
+               int64_t table_stride, const int32_t* seq_lens, int32_t num_seqs,
+               int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+               int32_t block_size, double scale, int32_t dtype,
+               int32_t nthreads) {
+  return orc_decode_impl(out, q, key_cache, value_cache, NULL, NULL, 1.0, 1.0,
+                         block_tables, table_stride, seq_lens, num_seqs, num_q_heads,
+                         num_kv_heads, head_dim, block_size, scale, dtype, nthreads);
+}
+
+int orc_decode_fp8(double* out, const uint16_t* q, const uint8_t* key_cache,
+                   const uint8_t* value_cache, double k_scale, double v_scale,
+                   const int32_t* block_tables, int64_t table_stride,
+                   const int32_t* seq_lens, int32_t num_seqs, int32_t num_q_heads,
+                   int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                   double scale, int32_t q_dtype, int32_t nthreads) {
+  return orc_decode_impl(out, q, NULL, NULL, key_cache, value_cache, k_scale, v_scale,
+                         block_tables, table_stride, seq_lens, num_seqs, num_q_heads,
+                         num_kv_heads, head_dim, block_size, scale, q_dtype, nthreads);
 }

@@ -306,3 +306,75 @@ def test_planted_gqa_mistake_is_caught(orc):
     wrong_q = q[:, [0, 2, 1, 3]]
     bad = orc.decode(wrong_q, kc, vc, table, np.array([L], np.int32), 0.25, "f16")[:, [0, 2, 1, 3]]
     assert np.max(np.abs(good - bad)) > 1e-3
+
+
+# --------------------------------------------------------------------------
+# fp8 (E4M3) cache pieces
+# --------------------------------------------------------------------------
+def test_e4m3_decoder_all_codes(orc):
+    codes = np.arange(256, dtype=np.uint8)
+    mine = orc.e4m3_to_double(codes)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(mine), nan) and nan.sum() == 2
+    assert np.array_equal(mine[~nan], ref[~nan])
+    assert np.nanmax(mine) == 448.0 and np.min(mine[mine > 0]) == 2.0 ** -9
+
+
+def test_e4m3_encoder_matches_library_in_range(orc):
+    rng = np.random.default_rng(0)
+    x = np.concatenate([
+        rng.standard_normal(3000).astype(np.float32) * 50,
+        rng.standard_normal(1000).astype(np.float32) * 0.01,       # subnormal range
+        orc.e4m3_to_double(np.arange(0, 0x7e, dtype=np.uint8)).astype(np.float32),  # exact codes
+        ((orc.e4m3_to_double(np.arange(0, 0x7d, dtype=np.uint8)) +
+          orc.e4m3_to_double(np.arange(1, 0x7e, dtype=np.uint8))) / 2).astype(np.float32),  # ties
+        np.array([0.0, -0.0, 447.9, -447.9, 416.0, 432.0], np.float32),
+    ])
+    x = np.concatenate([x, -x])
+    mine = orc.float_to_e4m3(x)
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(mine, ref)
+
+
+def test_e4m3_encoder_saturates(orc):
+    x = np.array([448.0, 449.0, 500.0, 1e6, np.inf, -1e6, -np.inf], np.float32)
+    assert orc.float_to_e4m3(x).tolist() == [0x7e, 0x7e, 0x7e, 0x7e, 0x7e, 0xfe, 0xfe]
+
+
+def test_fp8_write_and_decode_pins(orc):
+    """The fp8 write stores e4m3(x / scale); decode over a cache of codes equals
+    the 16-bit decode over the dequantised values (codes * scale), and a single
+    token returns its dequantised value row."""
+    rng = np.random.default_rng(4)
+    nb, bs, hkv, d, hq = 6, 4, 2, 16, 4
+    B, T = 2, 9
+    rows_k = _bits(rng.standard_normal((T, hkv, d)) * 3, "bf16")
+    rows_v = _bits(rng.standard_normal((T, hkv, d)) * 3, "bf16")
+    kc = np.zeros((nb, bs, hkv, d), np.uint8)
+    vc = np.zeros((nb, bs, hkv, d), np.uint8)
+    slots = np.array([5, 4, 6, 7, 12, 13, 14, 0, 1], np.int32)
+    orc.reshape_and_cache_fp8(rows_k, rows_v, kc, vc, slots, "bf16", 0.5, 2.0)
+    exp_k = orc.float_to_e4m3((_to_f64(rows_k, "bf16").astype(np.float32) / np.float32(0.5)))
+    assert np.array_equal(kc.reshape(nb * bs, hkv, d)[slots], exp_k)
+    exp_v = orc.float_to_e4m3((_to_f64(rows_v, "bf16").astype(np.float32) / np.float32(2.0)))
+    assert np.array_equal(vc.reshape(nb * bs, hkv, d)[slots], exp_v)
+    q = _bits(rng.standard_normal((B, hq, d)), "bf16")
+    table = np.array([[1, 3, 0], [0, 2, 1]], np.int32)
+    lens = np.array([9, 1], np.int32)
+    out = orc.decode_fp8(q, kc, vc, 0.5, 2.0, table, lens, 0.3, "bf16")
+    # same attention with the dequantised cache, through the 16-bit oracle in
+    # float64 terms: build it with torch SDPA on gathered values
+    Kd = orc.e4m3_to_double(kc) * 0.5
+    Vd = orc.e4m3_to_double(vc) * 2.0
+    Q = _to_f64(q, "bf16")
+    for b in range(B):
+        L = int(lens[b])
+        ks = np.stack([Kd[table[b, t // bs], t % bs] for t in range(L)])  # [L, hkv, d]
+        vs = np.stack([Vd[table[b, t // bs], t % bs] for t in range(L)])
+        kk = torch.from_numpy(ks).permute(1, 0, 2).repeat_interleave(hq // hkv, 0)
+        vv = torch.from_numpy(vs).permute(1, 0, 2).repeat_interleave(hq // hkv, 0)
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            torch.from_numpy(Q[b])[:, None, :], kk, vv, scale=0.3)[:, 0, :].numpy()
+        assert np.max(np.abs(out[b] - ref)) <= 1e-12
+    assert np.array_equal(out[1, 0], Vd[table[1, 0], 0, 0])
