@@ -215,7 +215,14 @@ def run_ours(args, rank, world, local_rank):
     def dev_bits(a):
         return torch.from_numpy(np.ascontiguousarray(a)).view(torch.int16).view(td).to(device)
 
-    k_cache, v_cache = dev_bits(case.k_pool), dev_bits(case.v_pool)
+    if spec.fp8:  # uint8 code pools and one-element scales
+        k_cache = torch.from_numpy(case.k_pool).to(device)
+        v_cache = torch.from_numpy(case.v_pool).to(device)
+        k_scale = torch.tensor([spec.k_scale], dtype=torch.float32, device=device)
+        v_scale = torch.tensor([spec.v_scale], dtype=torch.float32, device=device)
+    else:
+        k_cache, v_cache = dev_bits(case.k_pool), dev_bits(case.v_pool)
+        k_scale = v_scale = None
     q = dev_bits(case.q)
     new_k, new_v = dev_bits(wl["new_k"]), dev_bits(wl["new_v"])
     slots = torch.from_numpy(wl["slots"]).to(device)
@@ -236,11 +243,19 @@ def run_ours(args, rank, world, local_rank):
     def step(ev0=None, ev1=None):
         if cow is not None:
             pa.copy_blocks([k_cache], [v_cache], cow, error_flag=flag)
-        pa.reshape_and_cache(new_k, new_v, k_cache, v_cache, slots, error_flag=flag)
+        if spec.fp8:
+            pa.reshape_and_cache(new_k, new_v, k_cache, v_cache, slots, kv_cache_dtype="fp8_e4m3",
+                                 k_scale=k_scale, v_scale=v_scale, error_flag=flag)
+        else:
+            pa.reshape_and_cache(new_k, new_v, k_cache, v_cache, slots, error_flag=flag)
         if ev0 is not None:
             ev0.record(stream)
-        pa.decode_attention(out, q, k_cache, v_cache, tables, lens, max_len, scale, psize, ws,
-                            error_flag=flag)
+        if spec.fp8:
+            pa.decode_attention_fp8(out, q, k_cache, v_cache, k_scale, v_scale, tables, lens,
+                                    max_len, scale, psize, ws, error_flag=flag)
+        else:
+            pa.decode_attention(out, q, k_cache, v_cache, tables, lens, max_len, scale, psize, ws,
+                                error_flag=flag)
         if ev1 is not None:
             ev1.record(stream)
 
@@ -281,7 +296,7 @@ def run_ours(args, rank, world, local_rank):
     # ---------------- end to end: pinned host buffers through the public API
     e2e_steps = max(1, min(args.steps, args.e2e_steps))
     runner = pa.PagedDecodeStep(k_cache, v_cache, B, Hq, wl["tables"].shape[1], max_len, scale,
-                                psize)
+                                psize, query_dtype=td, k_scale=k_scale, v_scale=v_scale)
 
     def fill(dst, a, dtype=None):
         t = torch.from_numpy(np.ascontiguousarray(a))
@@ -327,12 +342,14 @@ def run_ours(args, rank, world, local_rank):
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": spec.dtype,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": spec.dtype + ("/e4m3 cache" if spec.fp8 else ""),
         "data": "synthetic (seeded N(0,1) values; lengths, placement and sharing per workload)",
         "config": {
-            "workload": "%s: B %d, Hq %d / Hkv %d, D %d, block %d, %s, lengths %s" % (
+            "workload": "%s: B %d, Hq %d / Hkv %d, D %d, block %d, %s%s, lengths %s" % (
                 spec.name, spec.num_seqs, spec.num_q_heads, spec.num_kv_heads, spec.head_dim,
-                spec.block_size, spec.dtype, describe_lengths(spec)),
+                spec.block_size, spec.dtype, ", fp8 E4M3 cache" if spec.fp8 else "",
+                describe_lengths(spec)),
             "global_batch": spec.num_seqs * world, "kv_bytes_per_step": bytes_step,
             "sum_seq_len": int(wl["lens"].sum()), "partition_size": psize,
             "num_blocks": case.num_blocks, "parallelism": "dp%d (independent batches)" % world,
@@ -402,6 +419,12 @@ def _oracle_sample(spec, wl, seqs):
     k, v = case.k_pool, case.v_pool
     threads = len(os.sched_getaffinity(0))
     t0 = time.perf_counter()
+    if spec.fp8:
+        oracle.reshape_and_cache_fp8(wl["new_k"][seqs], wl["new_v"][seqs], k, v,
+                                     wl["slots"][seqs], spec.dtype, spec.k_scale, spec.v_scale)
+        oracle.decode_fp8(case.q[seqs], k, v, spec.k_scale, spec.v_scale, wl["tables"][seqs],
+                          wl["lens"][seqs], W.scale_of(spec), spec.dtype, nthreads=threads)
+        return time.perf_counter() - t0, kv_bytes(spec, wl["lens"][seqs])
     if spec.len_dist != "shared_prefix":
         oracle.reshape_and_cache(wl["new_k"][seqs], wl["new_v"][seqs], k, v, wl["slots"][seqs])
     oracle.decode(case.q[seqs], k, v, wl["tables"][seqs], wl["lens"][seqs], W.scale_of(spec),

@@ -54,9 +54,16 @@ typedef enum {
 typedef enum { PA_F16 = 0, PA_BF16 = 1, PA_F32 = 2 } pa_dtype;
 
 /* Cache storage type of write_to_paged_cache's kv_cache_dtype ([vLLM]
- * "write_to_paged_cache: Direct In-Place Updates"); only "auto" (the cache
- * holds the model's 16-bit type) is built. */
-typedef enum { PA_KV_AUTO = 0 } pa_kv_cache_dtype;
+ * "write_to_paged_cache: Direct In-Place Updates", which passes "auto" with
+ * k_scale = v_scale = 1.0):
+ *   PA_KV_AUTO      the cache holds the model's 16-bit type;
+ *   PA_KV_FP8_E4M3  the cache holds 8-bit E4M3 codes (OCP 8-bit float, E4M3:
+ *                   bias 7, max 448, no infinities).  The pages give no
+ *                   formula; the reading built here: an element x is stored
+ *                   as e4m3(x / scale), the quotient taken in fp32, rounded to
+ *                   nearest even, saturating at +-448, and reads back as
+ *                   code * scale (per-tensor scales k_scale, v_scale). */
+typedef enum { PA_KV_AUTO = 0, PA_KV_FP8_E4M3 = 1 } pa_kv_cache_dtype;
 
 #define PA_DEVERR_BAD_BLOCK 0x1   /* block-table entry outside [0, num_blocks) */
 #define PA_DEVERR_BAD_SLOT 0x2    /* slot / block id outside the pool          */
@@ -85,10 +92,13 @@ int32_t pa_version(void);
  *  key_cache, value_cache  the pools (layout above), num_blocks blocks.
  *  slot_mapping    int32 [num_tokens], flat slot = block * block_size + offset.
  *  dtype           PA_F16 or PA_BF16 (both sides hold the same type).
- *  kv_cache_dtype  PA_KV_AUTO only; k_scale / v_scale are accepted and
- *                  ignored under AUTO (may be NULL).
- * Errors: PA_ERR_INVALID_ARG for null pointers or non-positive sizes;
- * PA_ERR_UNSUPPORTED for kv_cache_dtype != AUTO or dtype F32.  A slot at or
+ *  kv_cache_dtype  PA_KV_AUTO: the pools hold `dtype` and k_scale / v_scale
+ *                  are ignored (may be NULL).  PA_KV_FP8_E4M3: the pools hold
+ *                  uint8 codes e4m3(x / *k_scale) and e4m3(x / *v_scale);
+ *                  k_scale, v_scale are DEVICE pointers to one float each
+ *                  (required), the rows keep their 16-bit `dtype`.
+ * Errors: PA_ERR_INVALID_ARG for null pointers (scales included under fp8)
+ * or non-positive sizes; PA_ERR_UNSUPPORTED for dtype F32.  A slot at or
  * beyond num_blocks*block_size is skipped and flagged PA_DEVERR_BAD_SLOT.
  * Two tokens with the same slot: the surviving row is unspecified.
  * ------------------------------------------------------------------------- */
@@ -184,6 +194,30 @@ pa_status pa_decode_attention(void* out, pa_dtype out_dtype, const void* query,
                               int32_t partition_size, void* workspace,
                               size_t workspace_bytes,
                               int32_t* device_error_flag, pa_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * pa_decode_attention_fp8 -- pa_decode_attention over pools of E4M3 codes
+ * (written by pa_reshape_and_cache with PA_KV_FP8_E4M3).  A cached key element
+ * reads as code * (*k_scale), a value element as code * (*v_scale); k_scale
+ * and v_scale are DEVICE pointers to one float each.  query is query_dtype
+ * (PA_F16 or PA_BF16); both products run on fp16 tensor-core inputs (every
+ * E4M3 code is exactly an fp16 value; a bf16 query is rounded to fp16) with
+ * fp32 accumulation.  Built for head_dim 128.  The pool pointers must be
+ * 16-byte aligned.  Other arguments, the workspace and the errors are those
+ * of pa_decode_attention (pa_decode_workspace_bytes covers both).
+ * ------------------------------------------------------------------------- */
+pa_status pa_decode_attention_fp8(void* out, pa_dtype out_dtype, const void* query,
+                                  pa_dtype query_dtype, const void* key_cache,
+                                  const void* value_cache, const float* k_scale,
+                                  const float* v_scale, const int32_t* block_tables,
+                                  int32_t block_table_stride, const int32_t* seq_lens,
+                                  int32_t num_seqs, int32_t max_seq_len,
+                                  int32_t num_q_heads, int32_t num_kv_heads,
+                                  int32_t head_dim, int32_t num_blocks,
+                                  int32_t block_size, float scale,
+                                  int32_t partition_size, void* workspace,
+                                  size_t workspace_bytes, int32_t* device_error_flag,
+                                  pa_stream_t stream);
 
 /* ---------------------------------------------------------------------------
  * pa_decode_attention_noalloc -- pa_decode_attention for callers that cannot

@@ -24,6 +24,7 @@ parallel sampling with a shared prompt):
                 512-token partitions
   shared_prefix 32 prompts of 2047 tokens x 8 samples, each sample then
                 appending U[1, 200] tokens, bs 16, Hq 32 / Hkv 8, D 128, bf16
+  llama8b_fp8   the llama8b shape over an fp8 (E4M3) cache, scales 1/32
 """
 from __future__ import annotations
 
@@ -64,14 +65,21 @@ class Spec:
     prompt_len: int = 0
     extra_lo: int = 1
     extra_hi: int = 1
+    kv_dtype: str = "auto"           # 'auto' (16-bit pools) or 'fp8_e4m3' (code pools)
+    k_scale: float = 1.0             # fp8 pools: element = code * scale
+    v_scale: float = 1.0
 
     @property
     def group(self) -> int:
         return self.num_q_heads // self.num_kv_heads
 
     @property
+    def fp8(self) -> bool:
+        return self.kv_dtype == "fp8_e4m3"
+
+    @property
     def elem_bytes(self) -> int:
-        return 2
+        return 1 if self.fp8 else 2
 
     def replace(self, **kw) -> "Spec":
         return dataclasses.replace(self, **kw)
@@ -89,6 +97,10 @@ WORKLOADS = {
     "shared_prefix": Spec("shared_prefix", 256, 32, 8, 128, 16, "bf16", seed=1004,
                           len_dist="shared_prefix", prompts=32, samples=8,
                           prompt_len=2047, extra_lo=1, extra_hi=200),
+    # the llama8b shape over an fp8 (E4M3) cache: elements read code * 1/32
+    "llama8b_fp8": Spec("llama8b_fp8", 64, 32, 8, 128, 16, "bf16", seed=1005,
+                        len_dist="uniform", len_lo=512, len_hi=4096,
+                        kv_dtype="fp8_e4m3", k_scale=1.0 / 32, v_scale=1.0 / 32),
 }
 
 
@@ -100,8 +112,8 @@ class Case:
     num_blocks: int
     free_order: np.ndarray        # int32 [num_blocks], a permutation
     q: np.ndarray                 # uint16 [B, Hq, D]
-    k_pool: np.ndarray            # uint16 [num_blocks, bs, Hkv, D]
-    v_pool: np.ndarray            # uint16 [num_blocks, bs, Hkv, D]
+    k_pool: np.ndarray            # uint16 [num_blocks, bs, Hkv, D] (uint8 codes if fp8)
+    v_pool: np.ndarray
     new_k: np.ndarray             # uint16 [new_rows, Hkv, D]
     new_v: np.ndarray
     meta: dict = field(default_factory=dict)
@@ -154,6 +166,19 @@ def randn_bits(shape, dtype: str, g: torch.Generator, chunk: int = 1 << 26) -> n
     return out.reshape(shape)
 
 
+def randn_e4m3_codes(shape, g: torch.Generator, magnitude: float = 1.0,
+                     chunk: int = 1 << 26) -> np.ndarray:
+    """N(0, magnitude^2) float32 draws rounded to E4M3 codes (uint8) by torch's
+    float8_e4m3fn conversion, drawn in chunks: random contents for fp8 pools."""
+    n = int(np.prod(shape))
+    out = np.empty(n, dtype=np.uint8)
+    for lo in range(0, n, chunk):
+        m = min(chunk, n - lo)
+        x = torch.randn(m, generator=g, dtype=torch.float32) * magnitude
+        out[lo:lo + m] = x.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    return out.reshape(shape)
+
+
 def draw(spec: Spec) -> Case:
     g = torch.Generator().manual_seed(spec.seed)
     lens, extra = _draw_lengths(spec, g)
@@ -165,8 +190,12 @@ def draw(spec: Spec) -> Case:
     B, Hq, Hkv, D, bs = (spec.num_seqs, spec.num_q_heads, spec.num_kv_heads,
                          spec.head_dim, spec.block_size)
     q = randn_bits((B, Hq, D), spec.dtype, g)
-    k_pool = randn_bits((nb, bs, Hkv, D), spec.dtype, g)
-    v_pool = randn_bits((nb, bs, Hkv, D), spec.dtype, g)
+    if spec.fp8:  # code pools whose elements read back about N(0, 1)
+        k_pool = randn_e4m3_codes((nb, bs, Hkv, D), g, 1.0 / spec.k_scale)
+        v_pool = randn_e4m3_codes((nb, bs, Hkv, D), g, 1.0 / spec.v_scale)
+    else:
+        k_pool = randn_bits((nb, bs, Hkv, D), spec.dtype, g)
+        v_pool = randn_bits((nb, bs, Hkv, D), spec.dtype, g)
     if spec.len_dist == "shared_prefix":
         n_new = int(extra.sum())
     else:

@@ -16,6 +16,8 @@ Entry points (see the header for argument meaning, layout and errors):
   "How does copy-on-write work for parallel sampling?").
 * ``decode_attention``  -- paged decode attention with split-KV partials and a
   combine pass ("PagedAttention", "How attention reads paged memory").
+* ``decode_attention_fp8`` -- the same over E4M3 (fp8) code pools written by
+  ``reshape_and_cache(..., kv_cache_dtype="fp8_e4m3")``.
 * ``BlockManager``      -- the native host block manager (free list,
   refcounts, copy-on-write planning).
 * ``PagedDecodeStep``   -- one decode step from pinned host buffers: copies in,
@@ -77,6 +79,10 @@ def _load() -> ctypes.CDLL:
     lib.pa_decode_attention.argtypes = [p, ctypes.c_int, p, p, p, p, i32, p, i32, i32, i32, i32,
                                         i32, i32, i32, ctypes.c_float, ctypes.c_int, i32, p, sz,
                                         p, p]
+    lib.pa_decode_attention_fp8.restype = ctypes.c_int
+    lib.pa_decode_attention_fp8.argtypes = [p, ctypes.c_int, p, ctypes.c_int, p, p, p, p, p, i32,
+                                            p, i32, i32, i32, i32, i32, i32, i32, ctypes.c_float,
+                                            i32, p, sz, p, p]
     lib.pa_decode_attention_noalloc.restype = ctypes.c_int
     lib.pa_decode_attention_noalloc.argtypes = [p, ctypes.c_int, p, p, p, p, i32, p, i32, i32, i32,
                                                 i32, i32, i32, i32, ctypes.c_float, ctypes.c_int,
@@ -129,27 +135,41 @@ def _need(cond: bool, msg: str) -> None:
         raise ValueError(msg)
 
 
+_KV_CACHE_DTYPE = {"auto": 0, "fp8": 1, "fp8_e4m3": 1}
+
+
 def reshape_and_cache(key: torch.Tensor, value: torch.Tensor, key_cache: torch.Tensor,
                       value_cache: torch.Tensor, slot_mapping: torch.Tensor,
                       kv_cache_dtype: str = "auto", k_scale: Optional[torch.Tensor] = None,
                       v_scale: Optional[torch.Tensor] = None,
                       error_flag: Optional[torch.Tensor] = None,
                       stream: Optional[torch.cuda.Stream] = None) -> None:
-    """key/value [T, Hkv, D] (rows may be strided), caches [nb, bs, Hkv, D], slot_mapping int32 [T]."""
-    _need(kv_cache_dtype == "auto", "only kv_cache_dtype='auto' is built")
+    """key/value [T, Hkv, D] (rows may be strided), caches [nb, bs, Hkv, D], slot_mapping int32 [T].
+
+    kv_cache_dtype "auto": caches hold key's 16-bit type.  "fp8_e4m3": caches
+    are uint8 code pools and k_scale / v_scale are one-element float32 device
+    tensors (codes = e4m3(x / scale))."""
+    _need(kv_cache_dtype in _KV_CACHE_DTYPE, "kv_cache_dtype must be 'auto' or 'fp8_e4m3'")
+    fp8 = _KV_CACHE_DTYPE[kv_cache_dtype] == 1
     _need(key.dim() == 3 and value.shape == key.shape, "key/value must be [T, Hkv, D]")
     _need(key.stride(2) == 1 and key.stride(1) == key.shape[2] and
           value.stride(2) == 1 and value.stride(1) == value.shape[2],
           "heads and head_dim must be contiguous inside a row")
     _need(key_cache.is_contiguous() and value_cache.is_contiguous(), "caches must be contiguous")
     _need(slot_mapping.dtype == torch.int32 and slot_mapping.is_contiguous(), "slot_mapping int32")
-    _need(key.dtype == key_cache.dtype == value.dtype == value_cache.dtype, "dtype mismatch")
+    if fp8:
+        _need(key.dtype == value.dtype and key_cache.dtype == value_cache.dtype == torch.uint8,
+              "fp8 caches are uint8 code pools")
+        _need(k_scale is not None and v_scale is not None and k_scale.dtype == torch.float32 and
+              v_scale.dtype == torch.float32, "fp8 caches need float32 k_scale / v_scale")
+    else:
+        _need(key.dtype == key_cache.dtype == value.dtype == value_cache.dtype, "dtype mismatch")
     nb, bs, hkv, d = key_cache.shape
     _check(lib.pa_reshape_and_cache(
         _ptr(key), _ptr(value), key.stride(0), value.stride(0), _ptr(key_cache),
         _ptr(value_cache), _ptr(slot_mapping), key.shape[0], nb, bs, hkv, d,
-        _DTYPE_CODE[key.dtype], 0, _ptr(k_scale), _ptr(v_scale), _ptr(error_flag),
-        _stream_handle(stream)), "pa_reshape_and_cache")
+        _DTYPE_CODE[key.dtype], _KV_CACHE_DTYPE[kv_cache_dtype], _ptr(k_scale), _ptr(v_scale),
+        _ptr(error_flag), _stream_handle(stream)), "pa_reshape_and_cache")
 
 
 def copy_blocks(key_caches: Sequence[torch.Tensor], value_caches: Sequence[torch.Tensor],
@@ -211,6 +231,39 @@ def decode_attention(out: torch.Tensor, query: torch.Tensor, key_cache: torch.Te
         d, nb, bs, float(scale), _DTYPE_CODE[query.dtype], int(partition_size), _ptr(workspace),
         workspace.numel() * workspace.element_size(), _ptr(error_flag), _stream_handle(stream)),
         "pa_decode_attention")
+    return out
+
+
+def decode_attention_fp8(out: torch.Tensor, query: torch.Tensor, key_cache: torch.Tensor,
+                         value_cache: torch.Tensor, k_scale: torch.Tensor, v_scale: torch.Tensor,
+                         block_tables: torch.Tensor, seq_lens: torch.Tensor, max_seq_len: int,
+                         scale: float, partition_size: int = 0,
+                         workspace: Optional[torch.Tensor] = None,
+                         error_flag: Optional[torch.Tensor] = None,
+                         stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """Decode attention over uint8 E4M3 code pools [nb, bs, Hkv, D]; elements read
+    as code * k_scale / code * v_scale (one-element float32 device tensors)."""
+    _need(query.dim() == 3 and query.is_contiguous(), "query must be contiguous [B, Hq, D]")
+    _need(out.shape == query.shape and out.is_contiguous(), "out must be contiguous [B, Hq, D]")
+    _need(key_cache.dtype == value_cache.dtype == torch.uint8, "fp8 pools are uint8 codes")
+    _need(key_cache.is_contiguous() and value_cache.is_contiguous(), "caches must be contiguous")
+    _need(key_cache.shape == value_cache.shape, "K and V pools differ")
+    _need(k_scale.dtype == torch.float32 and v_scale.dtype == torch.float32, "float32 scales")
+    _need(block_tables.dtype == torch.int32 and block_tables.dim() == 2 and
+          block_tables.stride(1) == 1, "block_tables int32 [B, W], rows contiguous")
+    _need(seq_lens.dtype == torch.int32 and seq_lens.is_contiguous(), "seq_lens int32")
+    B, hq, d = query.shape
+    nb, bs, hkv, _ = key_cache.shape
+    if workspace is None:
+        workspace = alloc_workspace(decode_workspace_bytes(B, hq, hkv, d, bs, max_seq_len,
+                                                           partition_size), query.device)
+    _check(lib.pa_decode_attention_fp8(
+        _ptr(out), _DTYPE_CODE[out.dtype], _ptr(query), _DTYPE_CODE[query.dtype],
+        _ptr(key_cache), _ptr(value_cache), _ptr(k_scale), _ptr(v_scale), _ptr(block_tables),
+        block_tables.stride(0), _ptr(seq_lens), B, int(max_seq_len), hq, hkv, d, nb, bs,
+        float(scale), int(partition_size), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _ptr(error_flag), _stream_handle(stream)),
+        "pa_decode_attention_fp8")
     return out
 
 
@@ -325,11 +378,19 @@ class PagedDecodeStep:
     def __init__(self, key_cache: torch.Tensor, value_cache: torch.Tensor, num_seqs: int,
                  num_q_heads: int, table_width: int, max_seq_len: int, scale: float,
                  partition_size: int = 0, out_dtype: Optional[torch.dtype] = None,
-                 stream: Optional[torch.cuda.Stream] = None, use_graph: bool = True):
+                 stream: Optional[torch.cuda.Stream] = None, use_graph: bool = True,
+                 query_dtype: Optional[torch.dtype] = None,
+                 k_scale: Optional[torch.Tensor] = None, v_scale: Optional[torch.Tensor] = None):
+        """uint8 pools are fp8 (E4M3) code pools: pass query_dtype and the
+        one-element float32 device scales."""
         self.k, self.v = key_cache, value_cache
         nb, bs, hkv, d = key_cache.shape
         dev = key_cache.device
-        dt = key_cache.dtype
+        self.fp8 = key_cache.dtype == torch.uint8
+        _need(not self.fp8 or (query_dtype is not None and k_scale is not None and
+                               v_scale is not None), "fp8 pools need query_dtype and scales")
+        self.k_scale, self.v_scale = k_scale, v_scale
+        dt = query_dtype if self.fp8 else key_cache.dtype
         self.max_seq_len, self.scale, self.partition_size = max_seq_len, scale, partition_size
         self.stream = stream if stream is not None else torch.cuda.Stream(device=dev)
         self.use_graph = use_graph
@@ -366,9 +427,17 @@ class PagedDecodeStep:
     def _enqueue(self) -> None:
         dv = self.dev
         self._dev_buf.copy_(self._host_buf, non_blocking=True)
-        reshape_and_cache(dv["new_k"], dv["new_v"], self.k, self.v, dv["slots"])
-        decode_attention(self.out, dv["q"], self.k, self.v, dv["tables"], dv["lens"],
-                         self.max_seq_len, self.scale, self.partition_size, self.ws)
+        if self.fp8:
+            reshape_and_cache(dv["new_k"], dv["new_v"], self.k, self.v, dv["slots"],
+                              kv_cache_dtype="fp8_e4m3", k_scale=self.k_scale,
+                              v_scale=self.v_scale)
+            decode_attention_fp8(self.out, dv["q"], self.k, self.v, self.k_scale, self.v_scale,
+                                 dv["tables"], dv["lens"], self.max_seq_len, self.scale,
+                                 self.partition_size, self.ws)
+        else:
+            reshape_and_cache(dv["new_k"], dv["new_v"], self.k, self.v, dv["slots"])
+            decode_attention(self.out, dv["q"], self.k, self.v, dv["tables"], dv["lens"],
+                             self.max_seq_len, self.scale, self.partition_size, self.ws)
         self.host_out.copy_(self.out, non_blocking=True)
 
     def __call__(self) -> torch.Tensor:

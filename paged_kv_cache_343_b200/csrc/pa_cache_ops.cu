@@ -66,6 +66,51 @@ __global__ void __launch_bounds__(kRowThreads)
   }
 }
 
+// fp8 variant: each thread takes 8 elements (16 bytes in, 8 bytes out);
+// code = e4m3(x / scale) with the quotient in fp32.
+template <bool kBF16>
+__global__ void __launch_bounds__(kRowThreads)
+    pa_reshape_and_cache_fp8_kernel(const uint16_t* __restrict__ key,
+                                    const uint16_t* __restrict__ value, int64_t key_stride,
+                                    int64_t value_stride, uint8_t* __restrict__ key_cache,
+                                    uint8_t* __restrict__ value_cache,
+                                    const int32_t* __restrict__ slot_mapping, int32_t num_tokens,
+                                    int64_t num_slots, int32_t row_elems,
+                                    const float* __restrict__ k_scale,
+                                    const float* __restrict__ v_scale, int32_t* err) {
+  const int32_t nvec = row_elems / 8;
+  griddep_launch_dependents();
+  griddep_wait();
+  const float ks = *k_scale, vs = *v_scale;
+  for (int64_t t = blockIdx.x; t < num_tokens; t += gridDim.x) {
+    const int64_t slot = slot_mapping[t];
+    if (slot < 0) continue;
+    if (slot >= num_slots) {
+      if (threadIdx.x == 0) flag_error(err, PA_DEVERR_BAD_SLOT);
+      continue;
+    }
+    for (int32_t i = threadIdx.x; i < 2 * nvec; i += kRowThreads) {
+      const bool is_v = i >= nvec;
+      const int32_t j = is_v ? i - nvec : i;
+      const uint4 x = reinterpret_cast<const uint4*>((is_v ? value + t * value_stride
+                                                             : key + t * key_stride))[j];
+      const float s = is_v ? vs : ks;
+      const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+      uint16_t c[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float lo = __fdiv_rn(lo_to_float<kBF16>(w[q]), s);
+        const float hi = __fdiv_rn(hi_to_float<kBF16>(w[q]), s);
+        c[q] = pack_e4m3x2(lo, hi);
+      }
+      uint2 out;
+      out.x = static_cast<uint32_t>(c[0]) | (static_cast<uint32_t>(c[1]) << 16);
+      out.y = static_cast<uint32_t>(c[2]) | (static_cast<uint32_t>(c[3]) << 16);
+      reinterpret_cast<uint2*>((is_v ? value_cache : key_cache) + slot * row_elems)[j] = out;
+    }
+  }
+}
+
 struct CopyPtrs {
   uint8_t* p[kMaxCopyCaches];
 };
@@ -109,14 +154,40 @@ extern "C" pa_status pa_reshape_and_cache(const void* key, const void* value,
                                           pa_dtype dtype, pa_kv_cache_dtype kv_cache_dtype,
                                           const float* k_scale, const float* v_scale,
                                           int32_t* device_error_flag, pa_stream_t stream) {
-  (void)k_scale;
-  (void)v_scale;
   if (num_tokens < 0 || num_blocks <= 0 || block_size <= 0 || num_kv_heads <= 0 ||
       head_dim <= 0)
     return PA_ERR_INVALID_ARG;
   if (dtype != PA_F16 && dtype != PA_BF16) return PA_ERR_UNSUPPORTED;
-  if (kv_cache_dtype != PA_KV_AUTO) return PA_ERR_UNSUPPORTED;
+  if (kv_cache_dtype != PA_KV_AUTO && kv_cache_dtype != PA_KV_FP8_E4M3) return PA_ERR_UNSUPPORTED;
   if (num_tokens == 0) return PA_OK;
+  if (kv_cache_dtype == PA_KV_FP8_E4M3) {
+    if (!key || !value || !key_cache || !value_cache || !slot_mapping || !k_scale || !v_scale)
+      return PA_ERR_INVALID_ARG;
+    const int64_t row = static_cast<int64_t>(num_kv_heads) * head_dim;
+    if (row > INT32_MAX || key_stride_t < row || value_stride_t < row) return PA_ERR_INVALID_ARG;
+    // 16-byte row loads and 8-byte code stores
+    if (row % 8 != 0 || key_stride_t % 8 != 0 || value_stride_t % 8 != 0 || !aligned(key, 16) ||
+        !aligned(value, 16) || !aligned(key_cache, 8) || !aligned(value_cache, 8) ||
+        !aligned(slot_mapping, 4) || !aligned(k_scale, 4) || !aligned(v_scale, 4))
+      return PA_ERR_INVALID_ARG;
+    const int64_t num_slots = static_cast<int64_t>(num_blocks) * block_size;
+    const int grid = num_tokens < (1 << 20) ? num_tokens : (1 << 20);
+    PdlLaunch launch(reinterpret_cast<cudaStream_t>(stream), dim3(grid), dim3(kRowThreads));
+    const uint16_t* k = static_cast<const uint16_t*>(key);
+    const uint16_t* v = static_cast<const uint16_t*>(value);
+    uint8_t* kc = static_cast<uint8_t*>(key_cache);
+    uint8_t* vc = static_cast<uint8_t*>(value_cache);
+    const int32_t re = static_cast<int32_t>(row);
+    const cudaError_t e =
+        dtype == PA_BF16
+            ? launch(pa_reshape_and_cache_fp8_kernel<true>, k, v, key_stride_t, value_stride_t,
+                     kc, vc, slot_mapping, num_tokens, num_slots, re, k_scale, v_scale,
+                     device_error_flag)
+            : launch(pa_reshape_and_cache_fp8_kernel<false>, k, v, key_stride_t, value_stride_t,
+                     kc, vc, slot_mapping, num_tokens, num_slots, re, k_scale, v_scale,
+                     device_error_flag);
+    return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+  }
   if (!key || !value || !key_cache || !value_cache || !slot_mapping) return PA_ERR_INVALID_ARG;
   const int64_t row = static_cast<int64_t>(num_kv_heads) * head_dim;
   if (row > INT32_MAX || key_stride_t < row || value_stride_t < row) return PA_ERR_INVALID_ARG;

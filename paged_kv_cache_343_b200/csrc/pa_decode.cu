@@ -73,6 +73,9 @@ struct DecodeParams {
   float* part_o;           // [groups][nseg_cap][HG * group][head_dim]
   float* part_ml;          // [groups][nseg_cap][HG * group][2]  (m in log2 units, l)
   int32_t* err;
+  const float* k_scale;    // fp8 cache only: element = code * (*k_scale)
+  const float* v_scale;
+  int32_t q_bf16;          // fp8 cache only: the query is bf16 (else fp16)
 };
 
 __device__ __forceinline__ int32_t clamp_len(int32_t L, int32_t max_len) {
@@ -220,20 +223,28 @@ __global__ void __launch_bounds__(kPlanThreads) pa_plan_kernel(DecodeParams p) {
 // ---------------------------------------------------------------------------
 // main kernel
 // ---------------------------------------------------------------------------
-template <int D, int HG, bool kBF16>
+// kFP8: the pools hold 8-bit E4M3 codes.  Stages then carry the codes, and
+// each consumer warp widens its head's K and V codes into its own fp16 tiles
+// in shared memory (exact: every code is an fp16 value) before the MMAs,
+// which then run in fp16 (kBF16 must be false).
+template <int D, int HG, bool kBF16, bool kFP8>
 __global__ void __launch_bounds__((HG + 1) * 32, 1)
     pa_decode_main_kernel(const __grid_constant__ CUtensorMap tmK,
                           const __grid_constant__ CUtensorMap tmV, const DecodeParams p) {
-  constexpr int DC = D / 64;                       // 128-byte column chunks of a row
+  static_assert(!kFP8 || (D == 128 && !kBF16), "fp8 caches: head_dim 128, fp16 MMA");
+  constexpr int DC = D / 64;                       // 128-byte column chunks of a 16-bit row
+  constexpr int DCT = kFP8 ? 1 : DC;               // 128-byte rows per (token, head) in a stage
   constexpr int KSTEPS = D / 16;                   // k16 steps of S^T = K Q^T
   constexpr int MTILES = D / 16;                   // m16 tiles of O^T = V^T P^T
-  constexpr uint32_t kTileBytes = kTile * HG * D * 2;  // K (or V) bytes per stage
+  constexpr uint32_t kTileBytes = kTile * HG * D * (kFP8 ? 1 : 2);  // K (or V) bytes per stage
+  constexpr uint32_t kScratchBytes = kFP8 ? 2u * kTile * D * 2 : 0u;  // fp16 K and V, per warp
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const int NS = p.stages;
-  TileInfo* info = reinterpret_cast<TileInfo*>(smem + static_cast<size_t>(NS) * 2 * kTileBytes);
+  TileInfo* info = reinterpret_cast<TileInfo*>(smem + static_cast<size_t>(NS) * 2 * kTileBytes +
+                                               static_cast<size_t>(HG) * kScratchBytes);
   uint64_t* bars = reinterpret_cast<uint64_t*>(info + NS);
   const uint32_t smem_base = smem_u32(smem);
   const uint32_t bar_base = smem_u32(bars);
@@ -274,7 +285,7 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
     const uint64_t policy = l2_policy_evict_first();
     const int bs = p.block_size;
     const int TB = p.tok_box;
-    const uint32_t box_bytes = static_cast<uint32_t>(HG * DC * TB * 128);
+    const uint32_t box_bytes = static_cast<uint32_t>(HG * DCT * TB * 128);
     const int bpt = bs < kTile ? kTile / bs : 1;  // blocks per tile
     int b = p.start_seq[c];
     int32_t t_first = p.plan_tiles[b];
@@ -378,8 +389,8 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
                       phys[k], policy);
         } else {
           for (int hh = 0; hh < HG; ++hh) {
-            for (int dc = 0; dc < DC; ++dc) {
-              const uint32_t off = k * box_bytes + ((hh * DC + dc) * TB) * 128u;
+            for (int dc = 0; dc < DCT; ++dc) {
+              const uint32_t off = k * box_bytes + ((hh * DCT + dc) * TB) * 128u;
               tma_load_5d(kdst + off, &tmK, full_k(stage), 0, dc, hg * HG + hh, tok_off[k],
                           phys[k], policy);
               tma_load_5d(vdst + off, &tmV, full_v(stage), 0, dc, hg * HG + hh, tok_off[k],
@@ -413,7 +424,10 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
 
   // Per-lane row indices of the ldmatrix addresses (see the layout note in
   // the producer: rows of 128 bytes ordered [box][head][d-chunk][token]).
+  // With an fp8 cache the MMAs read the warp's own fp16 tiles, laid out
+  // [d-chunk][token] (one head, 16 tokens).
   auto row_of = [&](int tok, int dc) {
+    if constexpr (kFP8) return dc * kTile + tok;
     return ((tok >> tb_shift) * HG * DC + g * DC + dc) * TB + (tok & (TB - 1));
   };
   const int mi = lane >> 3, rr = lane & 7;
@@ -425,13 +439,56 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
     k_row[dc] = row_of(k_tok, dc);
     v_row[dc] = row_of(v_tok, dc);
   }
+  const uint32_t scratch_k = smem_base + static_cast<uint32_t>(NS) * 2u * kTileBytes +
+                             static_cast<uint32_t>(g) * kScratchBytes;
+  const uint32_t scratch_v = scratch_k + kScratchBytes / 2;
+  // Widens this head's 16 x D codes of a stage tile into an fp16 tile.
+  auto widen = [&](uint32_t src, uint32_t dst) {
+#pragma unroll
+    for (int it = 0; it < (kTile * (D / 16)) / 32; ++it) {
+      const int idx = it * 32 + lane;
+      const int tok = idx / (D / 16), c8 = idx % (D / 16);  // 16 codes = d 16*c8 .. +15
+      const int r8 = ((tok >> tb_shift) * HG + g) * TB + (tok & (TB - 1));
+      uint32_t w0, w1, w2, w3;
+      asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                   : "=r"(w0), "=r"(w1), "=r"(w2), "=r"(w3)
+                   : "r"(src + static_cast<uint32_t>(r8) * 128u +
+                         static_cast<uint32_t>((c8 ^ (r8 & 7)) * 16)));
+      const uint32_t h0 = e4m3x2_to_f16x2(static_cast<uint16_t>(w0 & 0xffffu));
+      const uint32_t h1 = e4m3x2_to_f16x2(static_cast<uint16_t>(w0 >> 16));
+      const uint32_t h2 = e4m3x2_to_f16x2(static_cast<uint16_t>(w1 & 0xffffu));
+      const uint32_t h3 = e4m3x2_to_f16x2(static_cast<uint16_t>(w1 >> 16));
+      const uint32_t h4 = e4m3x2_to_f16x2(static_cast<uint16_t>(w2 & 0xffffu));
+      const uint32_t h5 = e4m3x2_to_f16x2(static_cast<uint16_t>(w2 >> 16));
+      const uint32_t h6 = e4m3x2_to_f16x2(static_cast<uint16_t>(w3 & 0xffffu));
+      const uint32_t h7 = e4m3x2_to_f16x2(static_cast<uint16_t>(w3 >> 16));
+      const int row16 = (c8 >> 2) * kTile + tok;
+      const int ch = 2 * (c8 & 3);
+      const uint32_t rowa = dst + static_cast<uint32_t>(row16) * 128u;
+      asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(
+                       rowa + static_cast<uint32_t>((ch ^ (tok & 7)) * 16)),
+                   "r"(h0), "r"(h1), "r"(h2), "r"(h3)
+                   : "memory");
+      asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(
+                       rowa + static_cast<uint32_t>(((ch + 1) ^ (tok & 7)) * 16)),
+                   "r"(h4), "r"(h5), "r"(h6), "r"(h7)
+                   : "memory");
+    }
+  };
+  (void)widen;
+  (void)scratch_v;
+  float k_scale = 1.f, v_scale = 1.f;
+  if constexpr (kFP8) {
+    k_scale = *p.k_scale;
+    v_scale = *p.v_scale;
+  }
 
   uint32_t qf[KSTEPS][2];
   float acc[MTILES][4];
   float m_run[2], l_part[2];
   int stage = 0;
   uint32_t phase = 0;
-  const float sl2 = p.scale_log2;
+  const float sl2 = p.scale_log2 * k_scale;
 
   for (int64_t t = lo; t < hi; ++t) {
     if (!mbar_wait(full_k(stage), phase, p.err)) break;
@@ -444,6 +501,10 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
           const uint16_t* qp = qb + grp * D + kc * 16 + quad * 2;
           qf[kc][0] = *reinterpret_cast<const uint32_t*>(qp);
           qf[kc][1] = *reinterpret_cast<const uint32_t*>(qp + 8);
+          if (kFP8 && p.q_bf16) {  // the fp8 path multiplies in fp16
+            qf[kc][0] = bf16x2_to_f16x2(qf[kc][0]);
+            qf[kc][1] = bf16x2_to_f16x2(qf[kc][1]);
+          }
         } else {
           qf[kc][0] = 0u;
           qf[kc][1] = 0u;
@@ -457,8 +518,18 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
       m_run[0] = m_run[1] = -INFINITY;
       l_part[0] = l_part[1] = 0.f;
     }
-    const uint32_t kbase = smem_base + static_cast<uint32_t>(stage) * 2u * kTileBytes;
-    const uint32_t vbase = kbase + kTileBytes;
+    uint32_t kbase = smem_base + static_cast<uint32_t>(stage) * 2u * kTileBytes;
+    uint32_t vbase = kbase + kTileBytes;
+    if constexpr (kFP8) {
+      __syncwarp();  // the previous tile's reads of the fp16 tiles are done
+      widen(kbase, scratch_k);
+      if (!mbar_wait(full_v(stage), phase, p.err)) break;
+      widen(vbase, scratch_v);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(empty(stage));  // the codes are no longer needed
+      kbase = scratch_k;
+      vbase = scratch_v;
+    }
 
     // ---- S^T[16 tok x 8 heads] = K[16 x D] * Q^T[D x 8]
     float s[4] = {0.f, 0.f, 0.f, 0.f};
@@ -517,7 +588,7 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
     const uint32_t pc1 = movmatrix_trans(pl1);
 
     // ---- O^T[D x 8] += V^T[D x 16 tok] * P^T[16 tok x 8]
-    if (!mbar_wait(full_v(stage), phase, p.err)) break;
+    if (!kFP8 && !mbar_wait(full_v(stage), phase, p.err)) break;
     const bool partial = mask != 0xffffu;
     uint32_t z01 = 0xffffffffu, z23 = 0xffffffffu;
     if (partial) {
@@ -541,8 +612,10 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
       mma_16816<kBF16>(acc[mt], a0, a1, a2, a3, pb0, pb1);
       mma_16816<kBF16>(acc[mt], a0, a1, a2, a3, pc0, pc1);
     }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(empty(stage));
+    if constexpr (!kFP8) {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(empty(stage));
+    }
     if (++stage == NS) { stage = 0; phase ^= 1u; }
 
     if (ti.flags & kSegEnd) {
@@ -552,8 +625,8 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
         l0 += __shfl_xor_sync(0xffffffffu, l0, o);
         l1 += __shfl_xor_sync(0xffffffffu, l1, o);
       }
-      const float inv0 = l0 > 0.f ? 1.f / l0 : 0.f;
-      const float inv1 = l1 > 0.f ? 1.f / l1 : 0.f;
+      const float inv0 = l0 > 0.f ? v_scale / l0 : 0.f;
+      const float inv1 = l1 > 0.f ? v_scale / l1 : 0.f;
       const int h0 = 2 * quad, h1 = h0 + 1;
       if (ti.flags & kDirect) {
         const int64_t obase = (static_cast<int64_t>(ti.b) * p.num_q_heads + kvh * G) * D;
@@ -690,15 +763,25 @@ namespace {
 
 using MainKernel = void (*)(const CUtensorMap, const CUtensorMap, const DecodeParams);
 
-template <int D, int HG, bool BF>
+template <int D, int HG, bool BF, bool F8>
 MainKernel main_kernel_ptr() {
-  return pa_decode_main_kernel<D, HG, BF>;
+  return pa_decode_main_kernel<D, HG, BF, F8>;
 }
 
-MainKernel select_main(int D, int HG, bool bf16) {
-#define PA_SEL(d, hg)                                                      \
-  if (D == d && HG == hg) return bf16 ? main_kernel_ptr<d, hg, true>()     \
-                                      : main_kernel_ptr<d, hg, false>();
+MainKernel select_main(int D, int HG, bool bf16, bool fp8) {
+  if (fp8) {
+    if (D != 128) return nullptr;
+    switch (HG) {
+      case 1: return main_kernel_ptr<128, 1, false, true>();
+      case 2: return main_kernel_ptr<128, 2, false, true>();
+      case 4: return main_kernel_ptr<128, 4, false, true>();
+      case 8: return main_kernel_ptr<128, 8, false, true>();
+      default: return nullptr;
+    }
+  }
+#define PA_SEL(d, hg)                                                             \
+  if (D == d && HG == hg) return bf16 ? main_kernel_ptr<d, hg, true, false>()     \
+                                      : main_kernel_ptr<d, hg, false, false>();
   PA_SEL(64, 1) PA_SEL(64, 2) PA_SEL(64, 4) PA_SEL(64, 8)
   PA_SEL(128, 1) PA_SEL(128, 2) PA_SEL(128, 4) PA_SEL(128, 8)
 #undef PA_SEL
@@ -719,7 +802,8 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
 
 pa_status make_plan(int32_t num_seqs, int32_t Hq, int32_t Hkv, int32_t D, int32_t bs,
-                    int32_t max_seq_len, int32_t partition_size, bool bf16, LaunchPlan* lp) {
+                    int32_t max_seq_len, int32_t partition_size, bool bf16, bool fp8,
+                    LaunchPlan* lp) {
   if (num_seqs < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || bs <= 0 || max_seq_len < 0 ||
       partition_size < 0)
     return PA_ERR_INVALID_ARG;
@@ -732,22 +816,24 @@ pa_status make_plan(int32_t num_seqs, int32_t Hq, int32_t Hkv, int32_t D, int32_
     return PA_ERR_INVALID_ARG;
   int HG = 8;
   while (Hkv % HG != 0) HG >>= 1;
-  const int DC = D / 64;
+  if (fp8 && D != 128) return PA_ERR_UNSUPPORTED;
+  const int DCT = fp8 ? 1 : D / 64;  // 128-byte rows per (token, head) in a stage
   const int TB = bs < kTile ? bs : kTile;
-  if ((HG * DC * TB * 128) % 1024 != 0) return PA_ERR_UNSUPPORTED;
+  if ((HG * DCT * TB * 128) % 1024 != 0) return PA_ERR_UNSUPPORTED;
   lp->HG = HG;
   lp->groups = Hkv / HG;
   lp->tok_box = TB;
   lp->threads = (HG + 1) * 32;
-  const size_t tile_bytes = static_cast<size_t>(kTile) * HG * D * 2;
+  const size_t tile_bytes = static_cast<size_t>(kTile) * HG * D * (fp8 ? 1 : 2);
+  const size_t scratch = fp8 ? static_cast<size_t>(HG) * 2 * kTile * D * 2 : 0;
   const size_t budget = 200 * 1024;
-  int stages = static_cast<int>(budget / (2 * tile_bytes));
+  int stages = static_cast<int>((budget - scratch) / (2 * tile_bytes));
   if (stages > 6) stages = 6;
   if (stages < 2) return PA_ERR_UNSUPPORTED;
   lp->stages = stages;
-  lp->smem = 1024 + static_cast<size_t>(stages) * 2 * tile_bytes + stages * sizeof(TileInfo) +
-             3 * stages * sizeof(uint64_t);
-  lp->kernel = select_main(D, HG, bf16);
+  lp->smem = 1024 + static_cast<size_t>(stages) * 2 * tile_bytes + scratch +
+             stages * sizeof(TileInfo) + 3 * stages * sizeof(uint64_t);
+  lp->kernel = select_main(D, HG, bf16, fp8);
   if (lp->kernel == nullptr) return PA_ERR_UNSUPPORTED;
 
   const DeviceInfo* dev = current_device_info();
@@ -792,30 +878,45 @@ extern "C" pa_status pa_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_h
   if (bytes == nullptr) return PA_ERR_INVALID_ARG;
   LaunchPlan lp;
   const pa_status st = make_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
-                                 max_seq_len, partition_size, true, &lp);
+                                 max_seq_len, partition_size, true, false, &lp);
   if (st != PA_OK) return st;
   *bytes = lp.total;
+  // enough for the fp8-cache kernel of the same shape too
+  LaunchPlan lp8;
+  if (make_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, max_seq_len,
+                partition_size, false, true, &lp8) == PA_OK &&
+      lp8.total > *bytes)
+    *bytes = lp8.total;
   return PA_OK;
 }
 
-extern "C" pa_status pa_decode_attention(
-    void* out, pa_dtype out_dtype, const void* query, const void* key_cache,
-    const void* value_cache, const int32_t* block_tables, int32_t block_table_stride,
-    const int32_t* seq_lens, int32_t num_seqs, int32_t max_seq_len, int32_t num_q_heads,
-    int32_t num_kv_heads, int32_t head_dim, int32_t num_blocks, int32_t block_size, float scale,
-    pa_dtype kv_dtype, int32_t partition_size, void* workspace, size_t workspace_bytes,
-    int32_t* device_error_flag, pa_stream_t stream) {
+namespace {
+
+// Shared by the 16-bit and the fp8 entry points.  elem_bytes is 1 for E4M3
+// codes; then q_dtype is the query's type and k_scale / v_scale are set.
+pa_status launch_decode(void* out, pa_dtype out_dtype, const void* query, pa_dtype q_dtype,
+                        const void* key_cache, const void* value_cache, int elem_bytes,
+                        const float* k_scale, const float* v_scale,
+                        const int32_t* block_tables, int32_t block_table_stride,
+                        const int32_t* seq_lens, int32_t num_seqs, int32_t max_seq_len,
+                        int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                        int32_t num_blocks, int32_t block_size, float scale,
+                        int32_t partition_size, void* workspace, size_t workspace_bytes,
+                        int32_t* device_error_flag, pa_stream_t stream) {
   if (num_seqs < 0) return PA_ERR_INVALID_ARG;
   if (num_seqs == 0) return PA_OK;
   if (!out || !query || !key_cache || !value_cache || !block_tables || !seq_lens || !workspace)
     return PA_ERR_INVALID_ARG;
-  if (kv_dtype != PA_F16 && kv_dtype != PA_BF16) return PA_ERR_UNSUPPORTED;
+  const bool fp8 = elem_bytes == 1;
+  if (fp8 && (!k_scale || !v_scale || !aligned(k_scale, 4) || !aligned(v_scale, 4)))
+    return PA_ERR_INVALID_ARG;
+  if (q_dtype != PA_F16 && q_dtype != PA_BF16) return PA_ERR_UNSUPPORTED;
   if (out_dtype != PA_F16 && out_dtype != PA_BF16 && out_dtype != PA_F32)
     return PA_ERR_INVALID_ARG;
   if (num_blocks <= 0 || !(scale == scale)) return PA_ERR_INVALID_ARG;
   LaunchPlan lp;
   pa_status st = make_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
-                           max_seq_len, partition_size, kv_dtype == PA_BF16, &lp);
+                           max_seq_len, partition_size, !fp8 && q_dtype == PA_BF16, fp8, &lp);
   if (st != PA_OK) return st;
   const int64_t need_blocks = (static_cast<int64_t>(max_seq_len) + block_size - 1) / block_size;
   if (block_table_stride < need_blocks) return PA_ERR_INVALID_ARG;
@@ -825,26 +926,29 @@ extern "C" pa_status pa_decode_attention(
       !aligned(block_tables, 4) || !aligned(seq_lens, 4))
     return PA_ERR_INVALID_ARG;
 
-  const int HG = lp.HG, D = head_dim, DC = D / 64;
-  const uint64_t e = 2;
+  const int HG = lp.HG, D = head_dim;
+  const uint64_t e = static_cast<uint64_t>(elem_bytes);
+  const int DCT = fp8 ? 1 : D / 64;           // 128-byte rows per (token, head)
+  const uint32_t inner = fp8 ? 128u : 64u;    // elements in one 128-byte row
   CUtensorMap tmK, tmV;
   int mode = 0;
   {
-    // mode 0: dims {64 d, tokens, d-chunks, heads, blocks}, box {64, TB, DC, HG, 1}
-    const uint64_t dims0[5] = {64, (uint64_t)block_size, (uint64_t)DC, (uint64_t)num_kv_heads,
-                               (uint64_t)num_blocks};
+    // mode 0: dims {row, tokens, d-chunks, heads, blocks}, box {row, TB, DCT, HG, 1}
+    const uint64_t dims0[5] = {inner, (uint64_t)block_size, (uint64_t)DCT,
+                               (uint64_t)num_kv_heads, (uint64_t)num_blocks};
     const uint64_t str0[4] = {num_kv_heads * D * e, 128, D * e, block_size * num_kv_heads * D * e};
-    const uint32_t box0[5] = {64, (uint32_t)lp.tok_box, (uint32_t)DC, (uint32_t)HG, 1};
-    // mode 1: dims {64 d, d-chunks, heads, tokens, blocks}, box {64, 1, 1, TB, 1}
-    const uint64_t dims1[5] = {64, (uint64_t)DC, (uint64_t)num_kv_heads, (uint64_t)block_size,
-                               (uint64_t)num_blocks};
+    const uint32_t box0[5] = {inner, (uint32_t)lp.tok_box, (uint32_t)DCT, (uint32_t)HG, 1};
+    // mode 1: dims {row, d-chunks, heads, tokens, blocks}, box {row, 1, 1, TB, 1}
+    const uint64_t dims1[5] = {inner, (uint64_t)DCT, (uint64_t)num_kv_heads,
+                               (uint64_t)block_size, (uint64_t)num_blocks};
     const uint64_t str1[4] = {128, D * e, num_kv_heads * D * e, block_size * num_kv_heads * D * e};
-    const uint32_t box1[5] = {64, 1, 1, (uint32_t)lp.tok_box, 1};
-    if (get_tensor_map(&tmK, key_cache, dims0, str0, box0) &&
-        get_tensor_map(&tmV, value_cache, dims0, str0, box0)) {
+    const uint32_t box1[5] = {inner, 1, 1, (uint32_t)lp.tok_box, 1};
+    if (get_tensor_map(&tmK, key_cache, dims0, str0, box0, elem_bytes) &&
+        get_tensor_map(&tmV, value_cache, dims0, str0, box0, elem_bytes)) {
       mode = 0;
-    } else if (lp.tok_box * 128 % 1024 == 0 && get_tensor_map(&tmK, key_cache, dims1, str1, box1) &&
-               get_tensor_map(&tmV, value_cache, dims1, str1, box1)) {
+    } else if (lp.tok_box * 128 % 1024 == 0 &&
+               get_tensor_map(&tmK, key_cache, dims1, str1, box1, elem_bytes) &&
+               get_tensor_map(&tmV, value_cache, dims1, str1, box1, elem_bytes)) {
       mode = 1;
     } else {
       return PA_ERR_UNSUPPORTED;
@@ -881,6 +985,9 @@ extern "C" pa_status pa_decode_attention(
   p.part_o = reinterpret_cast<float*>(ws + lp.off_o);
   p.part_ml = reinterpret_cast<float*>(ws + lp.off_ml);
   p.err = device_error_flag;
+  p.k_scale = k_scale;
+  p.v_scale = v_scale;
+  p.q_bf16 = q_dtype == PA_BF16 ? 1 : 0;
 
   // All three launches use programmatic dependent launch: each may start while
   // its predecessor runs and waits (griddepcontrol.wait) before touching data.
@@ -895,6 +1002,37 @@ extern "C" pa_status pa_decode_attention(
   const cudaError_t e3 =
       D == 128 ? combine(pa_combine_kernel<128>, p) : combine(pa_combine_kernel<64>, p);
   return e3 == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" pa_status pa_decode_attention(
+    void* out, pa_dtype out_dtype, const void* query, const void* key_cache,
+    const void* value_cache, const int32_t* block_tables, int32_t block_table_stride,
+    const int32_t* seq_lens, int32_t num_seqs, int32_t max_seq_len, int32_t num_q_heads,
+    int32_t num_kv_heads, int32_t head_dim, int32_t num_blocks, int32_t block_size, float scale,
+    pa_dtype kv_dtype, int32_t partition_size, void* workspace, size_t workspace_bytes,
+    int32_t* device_error_flag, pa_stream_t stream) {
+  return launch_decode(out, out_dtype, query, kv_dtype, key_cache, value_cache, 2, nullptr,
+                       nullptr, block_tables, block_table_stride, seq_lens, num_seqs,
+                       max_seq_len, num_q_heads, num_kv_heads, head_dim, num_blocks, block_size,
+                       scale, partition_size, workspace, workspace_bytes, device_error_flag,
+                       stream);
+}
+
+extern "C" pa_status pa_decode_attention_fp8(
+    void* out, pa_dtype out_dtype, const void* query, pa_dtype query_dtype,
+    const void* key_cache, const void* value_cache, const float* k_scale, const float* v_scale,
+    const int32_t* block_tables, int32_t block_table_stride, const int32_t* seq_lens,
+    int32_t num_seqs, int32_t max_seq_len, int32_t num_q_heads, int32_t num_kv_heads,
+    int32_t head_dim, int32_t num_blocks, int32_t block_size, float scale,
+    int32_t partition_size, void* workspace, size_t workspace_bytes,
+    int32_t* device_error_flag, pa_stream_t stream) {
+  return launch_decode(out, out_dtype, query, query_dtype, key_cache, value_cache, 1, k_scale,
+                       v_scale, block_tables, block_table_stride, seq_lens, num_seqs,
+                       max_seq_len, num_q_heads, num_kv_heads, head_dim, num_blocks, block_size,
+                       scale, partition_size, workspace, workspace_bytes, device_error_flag,
+                       stream);
 }
 
 // ===========================================================================

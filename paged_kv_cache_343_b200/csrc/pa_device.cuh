@@ -197,6 +197,29 @@ __device__ __forceinline__ float hi_to_float(uint32_t v) {
   }
 }
 
+// Two floats to two E4M3 codes (lo in the low byte), round to nearest even,
+// finite values beyond 448 saturate.
+__device__ __forceinline__ uint16_t pack_e4m3x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// Two E4M3 codes (low byte first) to an fp16 pair; exact for every code.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t v) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(v));
+  return r;
+}
+
+// bf16 pair to fp16 pair (each value rounded to nearest even).
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t v) {
+  const float lo = __uint_as_float(v << 16), hi = __uint_as_float(v & 0xffff0000u);
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
 // 128-byte TMA swizzle: the 16-byte chunk index inside each 128-byte row is
 // XORed with the row index modulo 8 (rows counted from a 1024-byte boundary).
 __device__ __forceinline__ uint32_t swz128(uint32_t off) { return off ^ ((off >> 3) & 0x70u); }

@@ -50,10 +50,16 @@ def test_host_validation_without_gpu(pa):
     st = lib.pa_reshape_and_cache(None, None, 128, 128, None, None, None, 4, 8, 4, 2, 64, 0, 0,
                                   None, None, None, None)
     assert st == 1
-    # fp8 cache types are not built
-    st = lib.pa_reshape_and_cache(None, None, 128, 128, None, None, None, 4, 8, 4, 2, 64, 0, 1,
+    # unknown cache types are refused; fp8 without its scales is an invalid call
+    st = lib.pa_reshape_and_cache(None, None, 128, 128, None, None, None, 4, 8, 4, 2, 64, 0, 7,
                                   None, None, None, None)
     assert st == 2
+    st = lib.pa_reshape_and_cache(None, None, 128, 128, None, None, None, 4, 8, 4, 2, 64, 0, 1,
+                                  None, None, None, None)
+    assert st == 1
+    st = lib.pa_decode_attention_fp8(None, 1, None, 1, None, None, None, None, None, 1, None, 4,
+                                     16, 4, 2, 128, 8, 16, 0.1, 0, None, 0, None, None)
+    assert st == 1
     # zero work is a no-op
     assert lib.pa_decode_attention(None, 1, None, None, None, None, 1, None, 0, 16, 4, 2, 64, 8,
                                    4, 0.125, 1, 0, None, 0, None, None) == 0
