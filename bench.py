@@ -185,6 +185,26 @@ def build_workload(spec, pa):
                 cow=np.array(cow, np.int32).reshape(-1, 2), new_k=new_k, new_v=new_v)
 
 
+def kv_memory(spec, wl) -> dict:
+    """KV-cache memory held by the step's sequences ("PagedAttention": waste is
+    under one block per sequence; shared prompt blocks are held once)."""
+    bs = spec.block_size
+    lens = wl["lens"].astype(np.int64)
+    per_seq_blocks = -(-lens // bs)
+    logical_blocks = int(per_seq_blocks.sum())
+    held = set()
+    for b in range(spec.num_seqs):
+        held.update(int(x) for x in wl["tables"][b, :per_seq_blocks[b]])
+    tokens = int(lens.sum())
+    waste = per_seq_blocks * bs - lens
+    return {"block_size": bs, "tokens": tokens, "blocks_held": len(held),
+            "blocks_if_unshared": logical_blocks,
+            "occupancy": round(tokens / (logical_blocks * bs), 4),
+            "mean_waste_tokens_per_seq": round(float(waste.mean()), 2),
+            "max_waste_tokens_per_seq": int(waste.max()),
+            "sharing_saving": round(1.0 - len(held) / logical_blocks, 4)}
+
+
 def unique_kv_bytes(spec, wl) -> int:
     """KV bytes of distinct (block, offset) slots read by the step."""
     bs = spec.block_size
@@ -208,6 +228,8 @@ def run_ours(args, rank, world, local_rank):
     device = torch.device("cuda", local_rank)
     torch.cuda.set_device(device)
     spec = rank_spec(W.WORKLOADS[args.workload], rank, world)
+    if args.block_size:
+        spec = spec.replace(block_size=args.block_size)
     wl = build_workload(spec, pa)
     case = wl["case"]
     td = {"f16": torch.float16, "bf16": torch.bfloat16}[spec.dtype]
@@ -362,6 +384,7 @@ def run_ours(args, rank, world, local_rank):
                      "frac": round(achieved / peak, 4), "traffic": traffic,
                      "kernel": "pa_decode_attention (plan + main + combine launches)",
                      "peak_kind": peak_kind + " (MEASURED_PEAKS hbm_gbs, copy read+write)"},
+        "kv_memory": kv_memory(spec, wl),
         "clocks": clock_info,
         "e2e": e2e,
         "gpu_launches": launches_per_step * args.steps,
@@ -521,6 +544,8 @@ def main(argv=None):
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--ref-budget", type=float, default=90.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--block-size", type=int, default=0,
+                    help="override the workload's block size (block-size sweep)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

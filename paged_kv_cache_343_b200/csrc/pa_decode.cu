@@ -223,10 +223,17 @@ __global__ void __launch_bounds__(kPlanThreads) pa_plan_kernel(DecodeParams p) {
 // ---------------------------------------------------------------------------
 // main kernel
 // ---------------------------------------------------------------------------
-// kFP8: the pools hold 8-bit E4M3 codes.  Stages then carry the codes, and
-// each consumer warp widens its head's K and V codes into its own fp16 tiles
-// in shared memory (exact: every code is an fp16 value) before the MMAs,
-// which then run in fp16 (kBF16 must be false).
+// kFP8: the pools hold 8-bit E4M3 codes.  Stages then carry the codes; each
+// consumer lane reads exactly the code bytes of its MMA fragments from the
+// swizzled stage tile with 16-byte loads and converts them in registers to
+// fp16 (exact: every code is an fp16 value); the MMAs run in fp16 (kBF16 must
+// be false).  To make each lane's bytes contiguous, the fp8 path permutes
+//  - the k index of S^T = K Q^T: in k-step kc, lane quad q holds
+//    d = 32q + 4kc + {0,1} (k = 2q, 2q+1) and d = 32q + 4kc + {2,3}
+//    (k = 2q+8, 2q+9); the query fragments use the same map, so the dot
+//    products are unchanged;
+//  - the output rows of O^T = V^T P^T: accumulator row grp of m-tile mt is
+//    d = 16 grp + 2 mt, row grp + 8 is d = 16 grp + 2 mt + 1.
 template <int D, int HG, bool kBF16, bool kFP8>
 __global__ void __launch_bounds__((HG + 1) * 32, 1)
     pa_decode_main_kernel(const __grid_constant__ CUtensorMap tmK,
@@ -237,14 +244,12 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
   constexpr int KSTEPS = D / 16;                   // k16 steps of S^T = K Q^T
   constexpr int MTILES = D / 16;                   // m16 tiles of O^T = V^T P^T
   constexpr uint32_t kTileBytes = kTile * HG * D * (kFP8 ? 1 : 2);  // K (or V) bytes per stage
-  constexpr uint32_t kScratchBytes = kFP8 ? 2u * kTile * D * 2 : 0u;  // fp16 K and V, per warp
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const int NS = p.stages;
-  TileInfo* info = reinterpret_cast<TileInfo*>(smem + static_cast<size_t>(NS) * 2 * kTileBytes +
-                                               static_cast<size_t>(HG) * kScratchBytes);
+  TileInfo* info = reinterpret_cast<TileInfo*>(smem + static_cast<size_t>(NS) * 2 * kTileBytes);
   uint64_t* bars = reinterpret_cast<uint64_t*>(info + NS);
   const uint32_t smem_base = smem_u32(smem);
   const uint32_t bar_base = smem_u32(bars);
@@ -424,11 +429,8 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
 
   // Per-lane row indices of the ldmatrix addresses (see the layout note in
   // the producer: rows of 128 bytes ordered [box][head][d-chunk][token]).
-  // With an fp8 cache the MMAs read the warp's own fp16 tiles, laid out
-  // [d-chunk][token] (one head, 16 tokens).
   auto row_of = [&](int tok, int dc) {
-    if constexpr (kFP8) return dc * kTile + tok;
-    return ((tok >> tb_shift) * HG * DC + g * DC + dc) * TB + (tok & (TB - 1));
+    return ((tok >> tb_shift) * HG * DCT + g * DCT + dc) * TB + (tok & (TB - 1));
   };
   const int mi = lane >> 3, rr = lane & 7;
   const int k_tok = rr + 8 * (mi & 1), k_chunk = mi >> 1;   // K: non-transposed
@@ -436,47 +438,21 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
   int k_row[DC], v_row[DC];
 #pragma unroll
   for (int dc = 0; dc < DC; ++dc) {
-    k_row[dc] = row_of(k_tok, dc);
-    v_row[dc] = row_of(v_tok, dc);
+    k_row[dc] = kFP8 ? 0 : row_of(k_tok, dc);
+    v_row[dc] = kFP8 ? 0 : row_of(v_tok, dc);
   }
-  const uint32_t scratch_k = smem_base + static_cast<uint32_t>(NS) * 2u * kTileBytes +
-                             static_cast<uint32_t>(g) * kScratchBytes;
-  const uint32_t scratch_v = scratch_k + kScratchBytes / 2;
-  // Widens this head's 16 x D codes of a stage tile into an fp16 tile.
-  auto widen = [&](uint32_t src, uint32_t dst) {
+  // fp8: stage-tile rows of this lane's tokens (see kFP8 above)
+  int r8_k[2] = {0, 0}, r8_v[4] = {0, 0, 0, 0};
+  if constexpr (kFP8) {
+    r8_k[0] = row_of(grp, 0);
+    r8_k[1] = row_of(grp + 8, 0);
 #pragma unroll
-    for (int it = 0; it < (kTile * (D / 16)) / 32; ++it) {
-      const int idx = it * 32 + lane;
-      const int tok = idx / (D / 16), c8 = idx % (D / 16);  // 16 codes = d 16*c8 .. +15
-      const int r8 = ((tok >> tb_shift) * HG + g) * TB + (tok & (TB - 1));
-      uint32_t w0, w1, w2, w3;
-      asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                   : "=r"(w0), "=r"(w1), "=r"(w2), "=r"(w3)
-                   : "r"(src + static_cast<uint32_t>(r8) * 128u +
-                         static_cast<uint32_t>((c8 ^ (r8 & 7)) * 16)));
-      const uint32_t h0 = e4m3x2_to_f16x2(static_cast<uint16_t>(w0 & 0xffffu));
-      const uint32_t h1 = e4m3x2_to_f16x2(static_cast<uint16_t>(w0 >> 16));
-      const uint32_t h2 = e4m3x2_to_f16x2(static_cast<uint16_t>(w1 & 0xffffu));
-      const uint32_t h3 = e4m3x2_to_f16x2(static_cast<uint16_t>(w1 >> 16));
-      const uint32_t h4 = e4m3x2_to_f16x2(static_cast<uint16_t>(w2 & 0xffffu));
-      const uint32_t h5 = e4m3x2_to_f16x2(static_cast<uint16_t>(w2 >> 16));
-      const uint32_t h6 = e4m3x2_to_f16x2(static_cast<uint16_t>(w3 & 0xffffu));
-      const uint32_t h7 = e4m3x2_to_f16x2(static_cast<uint16_t>(w3 >> 16));
-      const int row16 = (c8 >> 2) * kTile + tok;
-      const int ch = 2 * (c8 & 3);
-      const uint32_t rowa = dst + static_cast<uint32_t>(row16) * 128u;
-      asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(
-                       rowa + static_cast<uint32_t>((ch ^ (tok & 7)) * 16)),
-                   "r"(h0), "r"(h1), "r"(h2), "r"(h3)
-                   : "memory");
-      asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(
-                       rowa + static_cast<uint32_t>(((ch + 1) ^ (tok & 7)) * 16)),
-                   "r"(h4), "r"(h5), "r"(h6), "r"(h7)
-                   : "memory");
-    }
+    for (int tt = 0; tt < 4; ++tt) r8_v[tt] = row_of(2 * quad + (tt & 1) + 8 * (tt >> 1), 0);
+  }
+  // output row of accumulator element (m-tile mt, upper = rows grp + 8)
+  auto d_of = [&](int mt, int upper) {
+    return kFP8 ? 16 * grp + 2 * mt + upper : mt * 16 + grp + 8 * upper;
   };
-  (void)widen;
-  (void)scratch_v;
   float k_scale = 1.f, v_scale = 1.f;
   if constexpr (kFP8) {
     k_scale = *p.k_scale;
@@ -498,9 +474,11 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
 #pragma unroll
       for (int kc = 0; kc < KSTEPS; ++kc) {
         if (grp < G) {
-          const uint16_t* qp = qb + grp * D + kc * 16 + quad * 2;
+          // fp8: k = 2q, 2q+1 -> d = 32q + 4kc + {0,1}; k = 2q+8, 2q+9 -> + {2,3}
+          const uint16_t* qp = kFP8 ? qb + grp * D + 32 * quad + 4 * kc
+                                    : qb + grp * D + kc * 16 + quad * 2;
           qf[kc][0] = *reinterpret_cast<const uint32_t*>(qp);
-          qf[kc][1] = *reinterpret_cast<const uint32_t*>(qp + 8);
+          qf[kc][1] = *reinterpret_cast<const uint32_t*>(qp + (kFP8 ? 2 : 8));
           if (kFP8 && p.q_bf16) {  // the fp8 path multiplies in fp16
             qf[kc][0] = bf16x2_to_f16x2(qf[kc][0]);
             qf[kc][1] = bf16x2_to_f16x2(qf[kc][1]);
@@ -518,30 +496,67 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
       m_run[0] = m_run[1] = -INFINITY;
       l_part[0] = l_part[1] = 0.f;
     }
-    uint32_t kbase = smem_base + static_cast<uint32_t>(stage) * 2u * kTileBytes;
-    uint32_t vbase = kbase + kTileBytes;
+    const uint32_t kbase = smem_base + static_cast<uint32_t>(stage) * 2u * kTileBytes;
+    const uint32_t vbase = kbase + kTileBytes;
+    // fp8: this lane's code bytes.  K: tokens grp, grp+8, d in [32q, 32q + 32)
+    // (chunks 2q, 2q+1).  V: tokens 2q, 2q+1, 2q+8, 2q+9, d in [16 grp, +16).
+    uint32_t kraw[2][8], vraw[4][4];
     if constexpr (kFP8) {
-      __syncwarp();  // the previous tile's reads of the fp16 tiles are done
-      widen(kbase, scratch_k);
+#pragma unroll
+      for (int rr2 = 0; rr2 < 2; ++rr2) {
+        const int r = r8_k[rr2];
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          const uint32_t a = kbase + static_cast<uint32_t>(r) * 128u +
+                             static_cast<uint32_t>(((2 * quad + hh) ^ (r & 7)) * 16);
+          asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                       : "=r"(kraw[rr2][4 * hh]), "=r"(kraw[rr2][4 * hh + 1]),
+                         "=r"(kraw[rr2][4 * hh + 2]), "=r"(kraw[rr2][4 * hh + 3])
+                       : "r"(a));
+        }
+      }
       if (!mbar_wait(full_v(stage), phase, p.err)) break;
-      widen(vbase, scratch_v);
+#pragma unroll
+      for (int tt = 0; tt < 4; ++tt) {
+        const int r = r8_v[tt];
+        const uint32_t a = vbase + static_cast<uint32_t>(r) * 128u +
+                           static_cast<uint32_t>((grp ^ (r & 7)) * 16);
+        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(vraw[tt][0]), "=r"(vraw[tt][1]), "=r"(vraw[tt][2]), "=r"(vraw[tt][3])
+                     : "r"(a));
+      }
+      // the codes are in registers: hand the stage back to the producer
       __syncwarp();
-      if (lane == 0) mbar_arrive(empty(stage));  // the codes are no longer needed
-      kbase = scratch_k;
-      vbase = scratch_v;
+      if (lane == 0) mbar_arrive(empty(stage));
     }
 
     // ---- S^T[16 tok x 8 heads] = K[16 x D] * Q^T[D x 8]
     float s[4] = {0.f, 0.f, 0.f, 0.f};
+    float s2[4] = {0.f, 0.f, 0.f, 0.f};  // odd k-steps: two independent MMA chains
 #pragma unroll
     for (int kc = 0; kc < KSTEPS; ++kc) {
-      const int dc = kc >> 2;
-      const int r = k_row[dc];
-      const uint32_t chunk = static_cast<uint32_t>((2 * (kc & 3) + k_chunk) ^ (r & 7));
       uint32_t a0, a1, a2, a3;
-      ldmatrix_x4(kbase + static_cast<uint32_t>(r) * 128u + chunk * 16u, a0, a1, a2, a3);
-      mma_16816<kBF16>(s, a0, a1, a2, a3, qf[kc][0], qf[kc][1]);
+      if constexpr (kFP8) {
+        a0 = e4m3x2_to_f16x2(static_cast<uint16_t>(kraw[0][kc] & 0xffffu));
+        a2 = e4m3x2_to_f16x2(static_cast<uint16_t>(kraw[0][kc] >> 16));
+        a1 = e4m3x2_to_f16x2(static_cast<uint16_t>(kraw[1][kc] & 0xffffu));
+        a3 = e4m3x2_to_f16x2(static_cast<uint16_t>(kraw[1][kc] >> 16));
+      } else {
+        const int dc = kc >> 2;
+        const int r = k_row[dc];
+        const uint32_t chunk = static_cast<uint32_t>((2 * (kc & 3) + k_chunk) ^ (r & 7));
+        ldmatrix_x4(kbase + static_cast<uint32_t>(r) * 128u + chunk * 16u, a0, a1, a2, a3);
+      }
+      if (kc & 1) {
+        mma_16816<kBF16>(s2, a0, a1, a2, a3, qf[kc][0], qf[kc][1]);
+      } else {
+        mma_16816<kBF16>(s, a0, a1, a2, a3, qf[kc][0], qf[kc][1]);
+      }
     }
+    s[0] += s2[0];
+    s[1] += s2[1];
+    s[2] += s2[2];
+    s[3] += s2[3];
     // ---- online softmax (base 2), masked by selection
     const uint32_t mask = static_cast<uint32_t>(ti.mask);
     const bool ok0 = (mask >> grp) & 1u, ok1 = (mask >> (grp + 8)) & 1u;
@@ -599,11 +614,25 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
     }
 #pragma unroll
     for (int mt = 0; mt < MTILES; ++mt) {
-      const int dc = mt >> 2;
-      const int r = v_row[dc];
-      const uint32_t chunk = static_cast<uint32_t>((2 * (mt & 3) + v_chunk) ^ (r & 7));
       uint32_t a0, a1, a2, a3;
-      ldmatrix_x4_trans(vbase + static_cast<uint32_t>(r) * 128u + chunk * 16u, a0, a1, a2, a3);
+      if constexpr (kFP8) {
+        // word mt/2 holds d = 16 grp + 2 mt + {0, 1} at bytes 2 (mt & 1) + {0, 1};
+        // pair tokens (2q, 2q+1) and (2q+8, 2q+9) byte by byte
+        const uint32_t sel = (mt & 1) ? 0x7362u : 0x5140u;
+        const int w = mt >> 1;
+        uint32_t lo, hi;
+        asm("prmt.b32 %0, %1, %2, %3;" : "=r"(lo) : "r"(vraw[0][w]), "r"(vraw[1][w]), "r"(sel));
+        asm("prmt.b32 %0, %1, %2, %3;" : "=r"(hi) : "r"(vraw[2][w]), "r"(vraw[3][w]), "r"(sel));
+        a0 = e4m3x2_to_f16x2(static_cast<uint16_t>(lo & 0xffffu));
+        a1 = e4m3x2_to_f16x2(static_cast<uint16_t>(lo >> 16));
+        a2 = e4m3x2_to_f16x2(static_cast<uint16_t>(hi & 0xffffu));
+        a3 = e4m3x2_to_f16x2(static_cast<uint16_t>(hi >> 16));
+      } else {
+        const int dc = mt >> 2;
+        const int r = v_row[dc];
+        const uint32_t chunk = static_cast<uint32_t>((2 * (mt & 3) + v_chunk) ^ (r & 7));
+        ldmatrix_x4_trans(vbase + static_cast<uint32_t>(r) * 128u + chunk * 16u, a0, a1, a2, a3);
+      }
       // masked tokens may hold anything (NaN included): zero them, never multiply
       a0 &= z01;
       a1 &= z01;
@@ -632,26 +661,26 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
         const int64_t obase = (static_cast<int64_t>(ti.b) * p.num_q_heads + kvh * G) * D;
 #pragma unroll
         for (int mt = 0; mt < MTILES; ++mt) {
-          const int d = mt * 16 + grp;
+          const int d0 = d_of(mt, 0), d1 = d_of(mt, 1);
 #pragma unroll
           for (int hh = 0; hh < 2; ++hh) {
             const int h = hh ? h1 : h0;
             if (h >= G) continue;
             const float inv = hh ? inv1 : inv0;
             const float v0 = acc[mt][hh] * inv, v1 = acc[mt][2 + hh] * inv;
-            const int64_t o = obase + static_cast<int64_t>(h) * D + d;
+            const int64_t o = obase + static_cast<int64_t>(h) * D;
             if (p.out_dtype == PA_F32) {
               float* op = static_cast<float*>(p.out);
-              op[o] = v0;
-              op[o + 8] = v1;
+              op[o + d0] = v0;
+              op[o + d1] = v1;
             } else if (p.out_dtype == PA_BF16) {
               __nv_bfloat16* op = static_cast<__nv_bfloat16*>(p.out);
-              op[o] = __float2bfloat16_rn(v0);
-              op[o + 8] = __float2bfloat16_rn(v1);
+              op[o + d0] = __float2bfloat16_rn(v0);
+              op[o + d1] = __float2bfloat16_rn(v1);
             } else {
               __half* op = static_cast<__half*>(p.out);
-              op[o] = __float2half_rn(v0);
-              op[o + 8] = __float2half_rn(v1);
+              op[o + d0] = __float2half_rn(v0);
+              op[o + d1] = __float2half_rn(v1);
             }
           }
         }
@@ -660,14 +689,14 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
         float* po = p.part_o + (sbase * HGq + g * G) * D;
 #pragma unroll
         for (int mt = 0; mt < MTILES; ++mt) {
-          const int d = mt * 16 + grp;
+          const int d0 = d_of(mt, 0), d1 = d_of(mt, 1);
           if (h0 < G) {
-            po[h0 * D + d] = acc[mt][0] * inv0;
-            po[h0 * D + d + 8] = acc[mt][2] * inv0;
+            po[h0 * D + d0] = acc[mt][0] * inv0;
+            po[h0 * D + d1] = acc[mt][2] * inv0;
           }
           if (h1 < G) {
-            po[h1 * D + d] = acc[mt][1] * inv1;
-            po[h1 * D + d + 8] = acc[mt][3] * inv1;
+            po[h1 * D + d0] = acc[mt][1] * inv1;
+            po[h1 * D + d1] = acc[mt][3] * inv1;
           }
         }
         if (grp == 0) {
@@ -825,14 +854,13 @@ pa_status make_plan(int32_t num_seqs, int32_t Hq, int32_t Hkv, int32_t D, int32_
   lp->tok_box = TB;
   lp->threads = (HG + 1) * 32;
   const size_t tile_bytes = static_cast<size_t>(kTile) * HG * D * (fp8 ? 1 : 2);
-  const size_t scratch = fp8 ? static_cast<size_t>(HG) * 2 * kTile * D * 2 : 0;
   const size_t budget = 200 * 1024;
-  int stages = static_cast<int>((budget - scratch) / (2 * tile_bytes));
+  int stages = static_cast<int>(budget / (2 * tile_bytes));
   if (stages > 6) stages = 6;
   if (stages < 2) return PA_ERR_UNSUPPORTED;
   lp->stages = stages;
-  lp->smem = 1024 + static_cast<size_t>(stages) * 2 * tile_bytes + scratch +
-             stages * sizeof(TileInfo) + 3 * stages * sizeof(uint64_t);
+  lp->smem = 1024 + static_cast<size_t>(stages) * 2 * tile_bytes + stages * sizeof(TileInfo) +
+             3 * stages * sizeof(uint64_t);
   lp->kernel = select_main(D, HG, bf16, fp8);
   if (lp->kernel == nullptr) return PA_ERR_UNSUPPORTED;
 
