@@ -69,6 +69,8 @@ typedef enum { PA_KV_AUTO = 0, PA_KV_FP8_E4M3 = 1 } pa_kv_cache_dtype;
 #define PA_DEVERR_BAD_SLOT 0x2    /* slot / block id outside the pool          */
 #define PA_DEVERR_BAD_SEQLEN 0x4  /* seq_len < 0 or > max_seq_len              */
 #define PA_DEVERR_TIMEOUT 0x8     /* a bounded pipeline wait gave up           */
+#define PA_DEVERR_BAD_SHARE 0x10  /* shared_blocks promised a block the tables
+                                     of a pack's members do not share          */
 
 /* Human-readable name of a status code (static storage). */
 const char* pa_status_string(pa_status status);
@@ -220,6 +222,59 @@ pa_status pa_decode_attention_fp8(void* out, pa_dtype out_dtype, const void* que
                                   pa_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * pa_decode_shared_prefix_workspace_bytes -- device scratch for
+ * pa_decode_attention_shared_prefix (larger than pa_decode_workspace_bytes:
+ * room for the packs' entries and eight query columns per KV head).  Same
+ * arguments and errors as pa_decode_workspace_bytes.
+ * ------------------------------------------------------------------------- */
+pa_status pa_decode_shared_prefix_workspace_bytes(int32_t num_seqs, int32_t num_q_heads,
+                                                  int32_t num_kv_heads, int32_t head_dim,
+                                                  int32_t block_size, int32_t max_seq_len,
+                                                  int32_t partition_size, size_t* bytes);
+
+/* ---------------------------------------------------------------------------
+ * pa_decode_attention_shared_prefix -- pa_decode_attention for batches whose
+ * sequences share leading blocks.  [PA] "Sharing and copy-on-write": with
+ * parallel sampling every sample's block table starts with the prompt's
+ * blocks, so pa_decode_attention reads each shared block once per sample.
+ * This entry point computes the same out[b, h, :] but reads a shared prefix
+ * once per pack of P = 8 / (num_q_heads / num_kv_heads) consecutive
+ * sequences (P = 2 for 4 query heads per KV head): the pack's queries fill the
+ * eight columns of one tensor-core product over the prefix, each sequence's
+ * own tail is attended as usual, and the combine pass merges the two
+ * softmax partials.  Packs need P >= 2 (at most 4 query heads per KV head;
+ * otherwise this is pa_decode_attention with a larger workspace).
+ *
+ *  shared_blocks  int32 [num_seqs], device: shared_blocks[b] = number of
+ *                 leading block-table entries that sequence b holds in common
+ *                 with sequence b + 1 (the same physical block ids; 0 if
+ *                 none; the last entry is ignored).  A block manager knows it
+ *                 from its fork history.  The plan packs P consecutive
+ *                 sequences b .. b+P-1 over the blocks that every pair of
+ *                 neighbours shares and that are full in every member, in
+ *                 whole 16-token tiles, when that prefix is at least 64
+ *                 tokens; sequences that do not fit a pack run alone.
+ *  workspace      at least pa_decode_shared_prefix_workspace_bytes().
+ * Other arguments, layouts and errors are those of pa_decode_attention.  On
+ * the device, a pack member whose table entry differs from the first
+ * member's within the promised prefix is flagged PA_DEVERR_BAD_SHARE (the
+ * first member's block is used for all).
+ * ------------------------------------------------------------------------- */
+pa_status pa_decode_attention_shared_prefix(void* out, pa_dtype out_dtype, const void* query,
+                                            const void* key_cache, const void* value_cache,
+                                            const int32_t* block_tables,
+                                            int32_t block_table_stride,
+                                            const int32_t* seq_lens,
+                                            const int32_t* shared_blocks, int32_t num_seqs,
+                                            int32_t max_seq_len, int32_t num_q_heads,
+                                            int32_t num_kv_heads, int32_t head_dim,
+                                            int32_t num_blocks, int32_t block_size,
+                                            float scale, pa_dtype kv_dtype,
+                                            int32_t partition_size, void* workspace,
+                                            size_t workspace_bytes,
+                                            int32_t* device_error_flag, pa_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * pa_decode_attention_noalloc -- pa_decode_attention for callers that cannot
  * allocate device memory.  The pages have no counterpart of this entry point;
  * it exists for callers such as plugins whose host framework owns every device
@@ -289,6 +344,13 @@ pa_status pa_bm_free_sequence(pa_block_manager* bm, int64_t seq);
 pa_status pa_bm_block_table(const pa_block_manager* bm, int64_t seq,
                             int32_t* out, int32_t capacity,
                             int32_t* num_blocks, int64_t* num_tokens);
+/* For the batch seqs[0 .. n-1] in that order: out[i] = number of leading
+ * table entries seqs[i] holds in common with seqs[i + 1] (same physical block
+ * ids), out[n - 1] = 0 -- the shared_blocks argument of
+ * pa_decode_attention_shared_prefix.  out is host memory of n int32.
+ * PA_ERR_NOT_FOUND if a sequence is unknown. */
+pa_status pa_bm_shared_blocks(const pa_block_manager* bm, const int64_t* seqs, int32_t n,
+                              int32_t* out);
 /* Reference count of a physical block (-1 if out of range). */
 int32_t pa_bm_refcount(const pa_block_manager* bm, int32_t block);
 int32_t pa_bm_num_free(const pa_block_manager* bm);

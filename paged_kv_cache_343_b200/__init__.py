@@ -18,8 +18,12 @@ Entry points (see the header for argument meaning, layout and errors):
   combine pass ("PagedAttention", "How attention reads paged memory").
 * ``decode_attention_fp8`` -- the same over E4M3 (fp8) code pools written by
   ``reshape_and_cache(..., kv_cache_dtype="fp8_e4m3")``.
+* ``decode_attention_shared_prefix`` -- the same result for batches whose
+  neighbouring sequences share leading blocks (parallel samples of one
+  prompt, "Sharing and copy-on-write"): a shared prefix is read once per pack
+  of sequences instead of once per sequence.
 * ``BlockManager``      -- the native host block manager (free list,
-  refcounts, copy-on-write planning).
+  refcounts, copy-on-write planning, shared-prefix counts).
 * ``PagedDecodeStep``   -- one decode step from pinned host buffers: copies in,
   the two kernels, copy out (the end-to-end call).
 """
@@ -33,8 +37,10 @@ import torch
 
 __all__ = [
     "LIB_PATH", "PagedAttnError", "reshape_and_cache", "copy_blocks", "decode_attention",
-    "decode_workspace_bytes", "BlockManager", "PagedDecodeStep", "DEVERR_BAD_BLOCK",
-    "DEVERR_BAD_SLOT", "DEVERR_BAD_SEQLEN", "DEVERR_TIMEOUT", "version",
+    "decode_workspace_bytes", "decode_attention_fp8", "decode_attention_noalloc",
+    "decode_attention_shared_prefix", "shared_prefix_workspace_bytes", "BlockManager",
+    "PagedDecodeStep", "DEVERR_BAD_BLOCK", "DEVERR_BAD_SLOT", "DEVERR_BAD_SEQLEN",
+    "DEVERR_TIMEOUT", "DEVERR_BAD_SHARE", "version",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpagedattn.so")
@@ -43,6 +49,7 @@ DEVERR_BAD_BLOCK = 0x1
 DEVERR_BAD_SLOT = 0x2
 DEVERR_BAD_SEQLEN = 0x4
 DEVERR_TIMEOUT = 0x8
+DEVERR_BAD_SHARE = 0x10
 
 _PA_F16, _PA_BF16, _PA_F32 = 0, 1, 2
 _DTYPE_CODE = {torch.float16: _PA_F16, torch.bfloat16: _PA_BF16, torch.float32: _PA_F32}
@@ -83,6 +90,14 @@ def _load() -> ctypes.CDLL:
     lib.pa_decode_attention_fp8.argtypes = [p, ctypes.c_int, p, ctypes.c_int, p, p, p, p, p, i32,
                                             p, i32, i32, i32, i32, i32, i32, i32, ctypes.c_float,
                                             i32, p, sz, p, p]
+    lib.pa_decode_shared_prefix_workspace_bytes.restype = ctypes.c_int
+    lib.pa_decode_shared_prefix_workspace_bytes.argtypes = [i32, i32, i32, i32, i32, i32, i32,
+                                                            ctypes.POINTER(sz)]
+    lib.pa_decode_attention_shared_prefix.restype = ctypes.c_int
+    lib.pa_decode_attention_shared_prefix.argtypes = [p, ctypes.c_int, p, p, p, p, i32, p, p, i32,
+                                                      i32, i32, i32, i32, i32, i32,
+                                                      ctypes.c_float, ctypes.c_int, i32, p, sz,
+                                                      p, p]
     lib.pa_decode_attention_noalloc.restype = ctypes.c_int
     lib.pa_decode_attention_noalloc.argtypes = [p, ctypes.c_int, p, p, p, p, i32, p, i32, i32, i32,
                                                 i32, i32, i32, i32, ctypes.c_float, ctypes.c_int,
@@ -104,6 +119,8 @@ def _load() -> ctypes.CDLL:
     lib.pa_bm_block_table.argtypes = [p, i64, p, i32, ctypes.POINTER(i32), ctypes.POINTER(i64)]
     lib.pa_bm_refcount.restype = i32
     lib.pa_bm_refcount.argtypes = [p, i32]
+    lib.pa_bm_shared_blocks.restype = ctypes.c_int
+    lib.pa_bm_shared_blocks.argtypes = [p, ctypes.POINTER(i64), i32, ctypes.POINTER(i32)]
     lib.pa_bm_num_free.restype = i32
     lib.pa_bm_num_free.argtypes = [p]
     return lib
@@ -200,6 +217,16 @@ def decode_workspace_bytes(num_seqs: int, num_q_heads: int, num_kv_heads: int, h
     return int(out.value)
 
 
+def shared_prefix_workspace_bytes(num_seqs: int, num_q_heads: int, num_kv_heads: int,
+                                  head_dim: int, block_size: int, max_seq_len: int,
+                                  partition_size: int = 0) -> int:
+    out = ctypes.c_size_t(0)
+    _check(lib.pa_decode_shared_prefix_workspace_bytes(
+        num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, max_seq_len, partition_size,
+        ctypes.byref(out)), "pa_decode_shared_prefix_workspace_bytes")
+    return int(out.value)
+
+
 def alloc_workspace(nbytes: int, device) -> torch.Tensor:
     """A device buffer of nbytes, 256-byte aligned (torch's allocator aligns to 512)."""
     return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
@@ -264,6 +291,43 @@ def decode_attention_fp8(out: torch.Tensor, query: torch.Tensor, key_cache: torc
         float(scale), int(partition_size), _ptr(workspace),
         workspace.numel() * workspace.element_size(), _ptr(error_flag), _stream_handle(stream)),
         "pa_decode_attention_fp8")
+    return out
+
+
+def decode_attention_shared_prefix(out: torch.Tensor, query: torch.Tensor,
+                                   key_cache: torch.Tensor, value_cache: torch.Tensor,
+                                   block_tables: torch.Tensor, seq_lens: torch.Tensor,
+                                   shared_blocks: torch.Tensor, max_seq_len: int, scale: float,
+                                   partition_size: int = 0,
+                                   workspace: Optional[torch.Tensor] = None,
+                                   error_flag: Optional[torch.Tensor] = None,
+                                   stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """decode_attention for batches whose consecutive sequences share leading
+    blocks (parallel samples of one prompt): shared_blocks int32 [B] on the
+    device, shared_blocks[b] = leading table entries b holds in common with
+    b + 1 (BlockManager.shared_blocks gives it).  Same result; a shared prefix
+    is read once per pack of 8 // (Hq / Hkv) sequences."""
+    _need(query.dim() == 3 and query.is_contiguous(), "query must be contiguous [B, Hq, D]")
+    _need(out.shape == query.shape and out.is_contiguous(), "out must be contiguous [B, Hq, D]")
+    _need(key_cache.is_contiguous() and value_cache.is_contiguous(), "caches must be contiguous")
+    _need(key_cache.shape == value_cache.shape, "K and V pools differ")
+    _need(block_tables.dtype == torch.int32 and block_tables.dim() == 2 and
+          block_tables.stride(1) == 1, "block_tables int32 [B, W], rows contiguous")
+    _need(seq_lens.dtype == torch.int32 and seq_lens.is_contiguous(), "seq_lens int32")
+    _need(shared_blocks.dtype == torch.int32 and shared_blocks.is_contiguous() and
+          shared_blocks.numel() == query.shape[0], "shared_blocks int32 [B]")
+    _need(query.dtype == key_cache.dtype == value_cache.dtype, "query and caches share a dtype")
+    B, hq, d = query.shape
+    nb, bs, hkv, _ = key_cache.shape
+    if workspace is None:
+        workspace = alloc_workspace(shared_prefix_workspace_bytes(
+            B, hq, hkv, d, bs, max_seq_len, partition_size), query.device)
+    _check(lib.pa_decode_attention_shared_prefix(
+        _ptr(out), _DTYPE_CODE[out.dtype], _ptr(query), _ptr(key_cache), _ptr(value_cache),
+        _ptr(block_tables), block_tables.stride(0), _ptr(seq_lens), _ptr(shared_blocks), B,
+        int(max_seq_len), hq, hkv, d, nb, bs, float(scale), _DTYPE_CODE[query.dtype],
+        int(partition_size), _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _ptr(error_flag), _stream_handle(stream)), "pa_decode_attention_shared_prefix")
     return out
 
 
@@ -350,6 +414,14 @@ class BlockManager:
 
     def num_free(self) -> int:
         return int(lib.pa_bm_num_free(self._h))
+
+    def shared_blocks(self, seqs: Sequence[int]) -> torch.Tensor:
+        """int32 [len(seqs)] host tensor: leading blocks seqs[i] shares with seqs[i + 1]."""
+        n = len(seqs)
+        ids = (ctypes.c_int64 * max(n, 1))(*[int(s) for s in seqs])
+        out = (ctypes.c_int32 * max(n, 1))()
+        _check(lib.pa_bm_shared_blocks(self._h, ids, n, out), "pa_bm_shared_blocks")
+        return torch.tensor(list(out)[:n], dtype=torch.int32)
 
     def tables(self, seqs: Sequence[int], width: int) -> torch.Tensor:
         """int32 [len(seqs), width] host tensor of block tables, padded with -1."""

@@ -156,6 +156,28 @@ extern "C" pa_status pa_bm_block_table(const pa_block_manager* bm, int64_t seq, 
   return PA_OK;
 }
 
+// Sequences forked from one parent share the parent's leading blocks until
+// they diverge ("Sharing and copy-on-write"); the count is read off the tables.
+extern "C" pa_status pa_bm_shared_blocks(const pa_block_manager* bm, const int64_t* seqs,
+                                         int32_t n, int32_t* out) {
+  if (bm == nullptr || n < 0 || (n > 0 && (seqs == nullptr || out == nullptr)))
+    return PA_ERR_INVALID_ARG;
+  const std::vector<int32_t>* prev = nullptr;
+  for (int32_t i = 0; i < n; ++i) {
+    auto it = bm->seqs.find(seqs[i]);
+    if (it == bm->seqs.end()) return PA_ERR_NOT_FOUND;
+    const std::vector<int32_t>& t = it->second.table;
+    if (prev != nullptr) {
+      size_t k = 0;
+      while (k < prev->size() && k < t.size() && (*prev)[k] == t[k]) ++k;
+      out[i - 1] = static_cast<int32_t>(k);
+    }
+    prev = &t;
+  }
+  if (n > 0) out[n - 1] = 0;
+  return PA_OK;
+}
+
 extern "C" int32_t pa_bm_refcount(const pa_block_manager* bm, int32_t block) {
   if (bm == nullptr || block < 0 || block >= bm->num_blocks) return -1;
   return bm->refcount[block];

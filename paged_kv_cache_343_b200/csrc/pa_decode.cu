@@ -41,13 +41,17 @@ enum : int32_t {
   kDirect = 8,    // the segment is the whole sequence: write `out` directly
 };
 
+constexpr int kMaxCols = 8;        // query columns per KV head in one MMA (its N)
+constexpr int kMinPackTiles = 4;   // shared prefixes shorter than this are not packed
+
 struct TileInfo {
-  int32_t b;       // sequence
+  int32_t b;       // sequence (the first member of a pack)
   int32_t valid;   // tokens of this tile inside the sequence (1..16)
   int32_t mask;    // bit t set: token t takes part (valid and its block id is good)
   int32_t seg;     // segment id inside this head group
   int32_t flags;
-  int32_t pad[3];
+  int32_t members;  // sequences whose queries use this tile (pack size or 1)
+  int32_t pad[2];
 };
 
 struct DecodeParams {
@@ -66,12 +70,23 @@ struct DecodeParams {
   int32_t stages;
   int32_t tok_box;         // tokens per TMA box: min(block_size, 16)
   int32_t tma_mode;        // 0: one box per block per tile, 1: one per (head, d-half)
-  int32_t* plan_tiles;     // [num_seqs + 1] tile prefix sums
-  int32_t* seg_base;       // [num_seqs + 1] segment prefix sums (partial slots)
-  int32_t* start_seq;      // [ctas_per_group] sequence holding each CTA's first tile
-  int32_t* first_k;        // [ctas_per_group] index of that tile's segment in its sequence
-  float* part_o;           // [groups][nseg_cap][HG * group][head_dim]
-  float* part_ml;          // [groups][nseg_cap][HG * group][2]  (m in log2 units, l)
+  int32_t* plan_tiles;     // [entries + 1] tile prefix sums
+  int32_t* seg_base;       // [entries + 1] segment prefix sums (partial slots)
+  int32_t* start_seq;      // [ctas_per_group] entry holding each CTA's first tile
+  int32_t* first_k;        // [ctas_per_group] index of that tile's segment in its entry
+  // shared prompts: packs of pack_size consecutive sequences whose block tables
+  // share leading blocks are attended together over that prefix ("entries"
+  // 0 .. K-1 are the packs' prefixes, K + b the rest of sequence b)
+  const int32_t* shared_blocks;  // [num_seqs] leading blocks b shares with b + 1, or null
+  int32_t pack_size;       // sequences per pack (8 / group, or 1: no packing)
+  int32_t* pack_first;     // [num_seqs] first sequence of pack k
+  int32_t* pack_tiles;     // [num_seqs] prefix tiles of pack k
+  int32_t* seq_pack;       // [num_seqs] pack of sequence b, or -1
+  int32_t* seq_pre;        // [num_seqs] tiles of b attended through its pack
+  int32_t* meta;           // [1] number of packs K (0 without packing)
+  int32_t cols;            // partial columns per KV head: pack_size * group
+  float* part_o;           // [groups][nseg_cap][HG][cols][head_dim]
+  float* part_ml;          // [groups][nseg_cap][HG][cols][2]  (m in log2 units, l)
   int32_t* err;
   const float* k_scale;    // fp8 cache only: element = code * (*k_scale)
   const float* v_scale;
@@ -85,15 +100,20 @@ __device__ __forceinline__ int32_t clamp_len(int32_t L, int32_t max_len) {
 
 // ---------------------------------------------------------------------------
 // plan (one CTA)
-//   tiles[b]    = sum_{b' < b} ceil(L_b' / 16)          (N = tiles[B] in all)
-//   segments    a sequence's tiles are cut wherever a partition starts
-//               (every tiles_per_part tiles from its first tile) or a CTA's
-//               share starts (lo(c) = floor(c N / C)); each piece is one
-//               segment, numbered 0, 1, ... within the sequence;
-//   seg_base[b] = sum_{b' < b} (segments of b'), so the partials of sequence
-//               b occupy slots seg_base[b] .. seg_base[b + 1] - 1;
-//   start_seq[c], first_k[c]: the sequence holding lo(c) and the number of
-//               that sequence's segments that start before lo(c).
+//   entries     the units of work laid end to end: first the K packs (only
+//               with shared_blocks: pack j attends sequences b_j .. b_j+P-1
+//               over their first pack_tiles[j] tiles, which they share), then
+//               every sequence b over its remaining tiles seq_pre[b] ..
+//               ceil(L_b / 16) - 1 (seq_pre[b] = 0 outside packs);
+//   tiles[e]    = sum_{e' < e} (tiles of entry e')          (N = tiles[E] in all)
+//   segments    an entry's tiles are cut wherever a partition starts (every
+//               tiles_per_part tiles from its first tile) or a CTA's share
+//               starts (lo(c) = floor(c N / C)); each piece is one segment,
+//               numbered 0, 1, ... within the entry;
+//   seg_base[e] = sum_{e' < e} (segments of e'), so the partials of entry e
+//               occupy slots seg_base[e] .. seg_base[e + 1] - 1;
+//   start_seq[c], first_k[c]: the entry holding lo(c) and the number of
+//               that entry's segments that start before lo(c).
 // ---------------------------------------------------------------------------
 constexpr int kPlanWarps = kPlanThreads / 32;
 
@@ -125,7 +145,7 @@ __device__ __forceinline__ int32_t block_exclusive_scan(int32_t v, int32_t* warp
   return before;
 }
 
-// Walks the segment starts of sequence b (tiles [t0, t1)) in order: the
+// Walks the segment starts of entry b (tiles [t0, t1)) in order: the
 // partition starts and the CTA-share starts, equal points counted once.
 // Records start_seq / first_k for every CTA whose share starts inside b and
 // returns the number of segments.
@@ -160,27 +180,74 @@ __device__ int32_t plan_sequence_segments(const DecodeParams& p, int32_t b, int6
   return count;
 }
 
-constexpr int kPlanRegChunks = 8;  // batches up to 8 x 256 sequences keep their counts in registers
+constexpr int kPlanRegChunks = 8;  // up to 8 x 256 entries keep their counts in registers
 
 __global__ void __launch_bounds__(kPlanThreads) pa_plan_kernel(DecodeParams p) {
   __shared__ int32_t warp_buf[kPlanWarps];
   const int tid = threadIdx.x;
+  const int B = p.num_seqs;
   griddep_launch_dependents();
   griddep_wait();  // seq_lens may come from the previous kernel on the stream
-  const int nchunks = (p.num_seqs + kPlanThreads - 1) / kPlanThreads;
+  // ---- packs: aligned windows b = P w .. P w + P - 1 over their shared prefix
+  int K = 0;
+  if (p.pack_size > 1) {
+    const int PK = p.pack_size;
+    const int W = B / PK;
+    for (int w0 = 0; w0 < W; w0 += kPlanThreads) {  // uniform trip count: the scan syncs
+      const int w = w0 + tid;
+      int32_t tiles = 0;
+      if (w < W) {
+        const int b0 = w * PK;
+        int64_t P = INT64_MAX;  // blocks common to all members and full in each
+        for (int m = 0; m < PK; ++m) {
+          P = min(P, static_cast<int64_t>(clamp_len(p.seq_lens[b0 + m], p.max_seq_len) /
+                                          p.block_size));
+          if (m + 1 < PK) P = min(P, static_cast<int64_t>(max(0, p.shared_blocks[b0 + m])));
+        }
+        tiles = static_cast<int32_t>(P * p.block_size / kTile);
+        if (tiles < kMinPackTiles) tiles = 0;
+      }
+      int32_t count = 0;
+      const int32_t k = K + block_exclusive_scan(tiles > 0 ? 1 : 0, warp_buf, &count);
+      if (w < W) {
+        const int b0 = w * PK;
+        if (tiles > 0) {
+          p.pack_first[k] = b0;
+          p.pack_tiles[k] = tiles;
+        }
+        for (int m = 0; m < PK; ++m) {
+          p.seq_pack[b0 + m] = tiles > 0 ? k : -1;
+          p.seq_pre[b0 + m] = tiles;
+        }
+      }
+      K += count;
+    }
+    for (int b = W * PK + tid; b < B; b += kPlanThreads) {
+      p.seq_pack[b] = -1;
+      p.seq_pre[b] = 0;
+    }
+    __syncthreads();  // the pack arrays are read back below
+  }
+  if (tid == 0) p.meta[0] = K;
+  const int E = K + B;  // entries: the packs' prefixes, then the sequences
+  const int nchunks = (E + kPlanThreads - 1) / kPlanThreads;
   const bool in_regs = nchunks <= kPlanRegChunks;
   int32_t t_reg[kPlanRegChunks], n_reg[kPlanRegChunks];
   int32_t carry = 0, total = 0;
   for (int ch = 0; ch < nchunks; ++ch) {
-    const int b = ch * kPlanThreads + tid;
+    const int e = ch * kPlanThreads + tid;
     int32_t nt = 0;
-    if (b < p.num_seqs) {
+    if (e < K) {
+      nt = p.pack_tiles[e];
+    } else if (e < E) {
+      const int b = e - K;
       const int32_t raw = p.seq_lens[b];
       if (raw < 0 || raw > p.max_seq_len) flag_error(p.err, PA_DEVERR_BAD_SEQLEN);
       nt = (clamp_len(raw, p.max_seq_len) + kTile - 1) / kTile;
+      if (p.pack_size > 1) nt -= p.seq_pre[b];
     }
     const int32_t ex = block_exclusive_scan(nt, warp_buf, &total);
-    if (b < p.num_seqs) p.plan_tiles[b] = carry + ex;
+    if (e < E) p.plan_tiles[e] = carry + ex;
 #pragma unroll
     for (int r = 0; r < kPlanRegChunks; ++r) {
       if (r == ch) {
@@ -190,14 +257,14 @@ __global__ void __launch_bounds__(kPlanThreads) pa_plan_kernel(DecodeParams p) {
     }
     carry += total;
   }
-  if (tid == 0) p.plan_tiles[p.num_seqs] = carry;
+  if (tid == 0) p.plan_tiles[E] = carry;
   if (!in_regs) __syncthreads();  // the global copy is read back below
   const int64_t N = carry, C = p.ctas_per_group;
   int32_t seg_carry = 0;
   for (int ch = 0; ch < nchunks; ++ch) {
-    const int b = ch * kPlanThreads + tid;
+    const int e = ch * kPlanThreads + tid;
     int32_t ns = 0;
-    if (b < p.num_seqs && N > 0) {
+    if (e < E && N > 0) {
       int64_t t0 = 0, t1 = 0;
       if (in_regs) {
 #pragma unroll
@@ -208,16 +275,16 @@ __global__ void __launch_bounds__(kPlanThreads) pa_plan_kernel(DecodeParams p) {
           }
         }
       } else {
-        t0 = p.plan_tiles[b];
-        t1 = p.plan_tiles[b + 1];
+        t0 = p.plan_tiles[e];
+        t1 = p.plan_tiles[e + 1];
       }
-      if (t1 > t0) ns = plan_sequence_segments(p, b, t0, t1, N, C);
+      if (t1 > t0) ns = plan_sequence_segments(p, e, t0, t1, N, C);
     }
     const int32_t ex = block_exclusive_scan(ns, warp_buf, &total);
-    if (b < p.num_seqs) p.seg_base[b] = seg_carry + ex;
+    if (e < E) p.seg_base[e] = seg_carry + ex;
     seg_carry += total;
   }
-  if (tid == 0) p.seg_base[p.num_seqs] = seg_carry;
+  if (tid == 0) p.seg_base[E] = seg_carry;
 }
 
 // ---------------------------------------------------------------------------
@@ -279,7 +346,8 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
   griddep_launch_dependents();
   griddep_wait();  // the plan (and all earlier work on the stream) is complete
 
-  const int64_t N = p.plan_tiles[B];
+  const int E = p.meta[0] + B;  // entries: packs' prefixes, then sequences
+  const int64_t N = p.plan_tiles[E];
   const int64_t lo = static_cast<int64_t>(c) * N / C;
   const int64_t hi = static_cast<int64_t>(c + 1) * N / C;
   if (lo >= hi) return;
@@ -292,41 +360,61 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
     const int TB = p.tok_box;
     const uint32_t box_bytes = static_cast<uint32_t>(HG * DCT * TB * 128);
     const int bpt = bs < kTile ? kTile / bs : 1;  // blocks per tile
-    int b = p.start_seq[c];
-    int32_t t_first = p.plan_tiles[b];
-    int32_t n_b = p.plan_tiles[b + 1] - t_first;
-    int32_t L_b = clamp_len(p.seq_lens[b], p.max_seq_len);
-    int32_t seg_b = p.seg_base[b];
-    int32_t nseg_b = p.seg_base[b + 1] - seg_b;
-    int32_t k = p.first_k[c] - 1;  // segment index inside the sequence (advanced at starts)
-    const int32_t* row = p.block_tables + static_cast<int64_t>(b) * p.table_stride;
+    const int K = E - B;
+    // the entry being walked: tiles t_first .. t_first + n_e - 1 of the line,
+    // which are tiles i0 .. i0 + n_e - 1 of sequence b (of every pack member)
+    int e = p.start_seq[c];
+    int b = 0, members = 1;
+    int32_t t_first = 0, n_e = 0, i0 = 0, L_b = 0, seg_e = 0, nseg_e = 0;
+    const int32_t* row = p.block_tables;
+    auto enter = [&](int ent) {
+      t_first = p.plan_tiles[ent];
+      n_e = p.plan_tiles[ent + 1] - t_first;
+      seg_e = p.seg_base[ent];
+      nseg_e = p.seg_base[ent + 1] - seg_e;
+      if (ent < K) {
+        b = p.pack_first[ent];
+        members = p.pack_size;
+        i0 = 0;
+        L_b = n_e * kTile;
+      } else {
+        b = ent - K;
+        members = 1;
+        i0 = p.pack_size > 1 ? p.seq_pre[b] : 0;
+        L_b = clamp_len(p.seq_lens[b], p.max_seq_len);
+      }
+      row = p.block_tables + static_cast<int64_t>(b) * p.table_stride;
+    };
+    enter(e);
+    int32_t k = p.first_k[c] - 1;  // segment index inside the entry (advanced at starts)
     int32_t i = static_cast<int32_t>(lo - t_first);
     bool new_seq = true;
     int stage = 0;
     uint32_t phase = 0;
     int64_t issued = 0;
+    // the pack's other members must hold the same block ids
+    auto check_shared = [&](int64_t idx, int32_t id) {
+      for (int m = 1; m < members; ++m)
+        if (__ldg(row + static_cast<int64_t>(m) * p.table_stride + idx) != id)
+          flag_error(p.err, PA_DEVERR_BAD_SHARE);
+    };
     for (int64_t t = lo; t < hi; ++t, ++i) {
-      while (i >= n_b) {  // next sequence that has tiles
-        ++b;
-        t_first = p.plan_tiles[b];
-        n_b = p.plan_tiles[b + 1] - t_first;
-        L_b = clamp_len(p.seq_lens[b], p.max_seq_len);
-        seg_b = p.seg_base[b];
-        nseg_b = p.seg_base[b + 1] - seg_b;
+      while (i >= n_e) {  // next entry that has tiles
+        enter(++e);
         k = -1;
-        row = p.block_tables + static_cast<int64_t>(b) * p.table_stride;
         i = 0;
         new_seq = true;
       }
       if (!mbar_wait(empty(stage), phase ^ 1u, p.err)) break;
 
-      const int32_t valid = min(kTile, L_b - i * kTile);
+      const int32_t ti_seq = i0 + i;  // tile index inside the sequence
+      const int32_t valid = min(kTile, L_b - ti_seq * kTile);
       const int32_t j = (p.tiles_per_part == INT_MAX) ? 0 : i / p.tiles_per_part;
       const int64_t part_lo = t_first + static_cast<int64_t>(j) *
                                             (p.tiles_per_part == INT_MAX ? 0 : p.tiles_per_part);
       const int64_t part_hi = (p.tiles_per_part == INT_MAX)
-                                  ? t_first + n_b
-                                  : min(static_cast<int64_t>(t_first) + n_b,
+                                  ? t_first + n_e
+                                  : min(static_cast<int64_t>(t_first) + n_e,
                                         part_lo + p.tiles_per_part);
       const int64_t seg_lo = max(part_lo, lo), seg_hi = min(part_hi, hi);
       int32_t flags = 0;
@@ -336,7 +424,7 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
         ++k;
       }
       if (t == seg_hi - 1) flags |= kSegEnd;
-      if (nseg_b == 1) flags |= kDirect;
+      if (nseg_e == 1 && members == 1 && i0 == 0) flags |= kDirect;
       new_seq = false;
 
       uint32_t mask = valid >= kTile ? 0xffffu : ((1u << valid) - 1u);
@@ -349,7 +437,9 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
         for (int k = 0; k < bpt; ++k) {
           const int tok0 = k * bs;
           if (tok0 >= valid) break;
-          const int32_t id = __ldg(row + static_cast<int64_t>(i) * bpt + k);
+          const int64_t idx = static_cast<int64_t>(ti_seq) * bpt + k;
+          const int32_t id = __ldg(row + idx);
+          if (members > 1) check_shared(idx, id);
           if (id < 0 || id >= p.num_blocks) {
             flag_error(p.err, PA_DEVERR_BAD_BLOCK);
             mask &= ~(((1u << bs) - 1u) << tok0);
@@ -362,8 +452,9 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
           bytes += box_bytes;
         }
       } else {
-        const int64_t tok = static_cast<int64_t>(i) * kTile;
+        const int64_t tok = static_cast<int64_t>(ti_seq) * kTile;
         const int32_t id = __ldg(row + tok / bs);
+        if (members > 1) check_shared(tok / bs, id);
         tok_off[0] = static_cast<int32_t>(tok % bs);
         if (id < 0 || id >= p.num_blocks) {
           flag_error(p.err, PA_DEVERR_BAD_BLOCK);
@@ -379,8 +470,9 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
       ti.b = b;
       ti.valid = valid;
       ti.mask = static_cast<int32_t>(mask);
-      ti.seg = seg_b + k;
+      ti.seg = seg_e + k;
       ti.flags = flags;
+      ti.members = members;
       mbar_arrive_expect_tx(full_k(stage), bytes);
       mbar_arrive_expect_tx(full_v(stage), bytes);
       const uint32_t kdst = smem_base + static_cast<uint32_t>(stage) * 2u * kTileBytes;
@@ -422,7 +514,6 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
   const int g = warp;                         // KV head inside the group
   const int kvh = hg * HG + g;                // KV head
   const int G = p.group;
-  const int HGq = HG * G;                     // query heads of this CTA's group
   const int quad = lane & 3, grp = lane >> 2;
   const int TB = p.tok_box;
   const int tb_shift = TB == 16 ? 4 : (TB == 8 ? 3 : 2);
@@ -470,13 +561,16 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
     if (!mbar_wait(full_k(stage), phase, p.err)) break;
     const TileInfo ti = info[stage];
     if (ti.flags & kNewSeq) {
-      const uint16_t* qb = p.query + (static_cast<int64_t>(ti.b) * p.num_q_heads + kvh * G) * D;
+      // column grp: query head grp % G of pack member grp / G (sequence b + member)
+      const int member = grp / G;
+      const uint16_t* qb =
+          p.query +
+          ((static_cast<int64_t>(ti.b) + member) * p.num_q_heads + kvh * G + (grp - member * G)) * D;
 #pragma unroll
       for (int kc = 0; kc < KSTEPS; ++kc) {
-        if (grp < G) {
+        if (grp < ti.members * G) {
           // fp8: k = 2q, 2q+1 -> d = 32q + 4kc + {0,1}; k = 2q+8, 2q+9 -> + {2,3}
-          const uint16_t* qp = kFP8 ? qb + grp * D + 32 * quad + 4 * kc
-                                    : qb + grp * D + kc * 16 + quad * 2;
+          const uint16_t* qp = kFP8 ? qb + 32 * quad + 4 * kc : qb + kc * 16 + quad * 2;
           qf[kc][0] = *reinterpret_cast<const uint32_t*>(qp);
           qf[kc][1] = *reinterpret_cast<const uint32_t*>(qp + (kFP8 ? 2 : 8));
           if (kFP8 && p.q_bf16) {  // the fp8 path multiplies in fp16
@@ -685,27 +779,28 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
           }
         }
       } else if (ti.seg < p.nseg_cap) {
-        const int64_t sbase = static_cast<int64_t>(hg) * p.nseg_cap + ti.seg;
-        float* po = p.part_o + (sbase * HGq + g * G) * D;
+        const int ncol = ti.members * G;
+        const int64_t prow = ((static_cast<int64_t>(hg) * p.nseg_cap + ti.seg) * HG + g) * p.cols;
+        float* po = p.part_o + prow * D;
 #pragma unroll
         for (int mt = 0; mt < MTILES; ++mt) {
           const int d0 = d_of(mt, 0), d1 = d_of(mt, 1);
-          if (h0 < G) {
+          if (h0 < ncol) {
             po[h0 * D + d0] = acc[mt][0] * inv0;
             po[h0 * D + d1] = acc[mt][2] * inv0;
           }
-          if (h1 < G) {
+          if (h1 < ncol) {
             po[h1 * D + d0] = acc[mt][1] * inv1;
             po[h1 * D + d1] = acc[mt][3] * inv1;
           }
         }
         if (grp == 0) {
-          float* pm = p.part_ml + (sbase * HGq + g * G) * 2;
-          if (h0 < G) {
+          float* pm = p.part_ml + prow * 2;
+          if (h0 < ncol) {
             pm[h0 * 2] = l0 > 0.f ? m_run[0] : -INFINITY;
             pm[h0 * 2 + 1] = l0;
           }
-          if (h1 < G) {
+          if (h1 < ncol) {
             pm[h1 * 2] = l1 > 0.f ? m_run[1] : -INFINITY;
             pm[h1 * 2 + 1] = l1;
           }
@@ -719,10 +814,12 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
 
 // ---------------------------------------------------------------------------
 // combine: out[b, h] = sum_k w_k o_k / sum_k w_k,  w_k = l_k 2^(m_k - M),
-// M = max_k m_k over the segments k of sequence b (slots seg_base[b] ..).
+// M = max_k m_k over the partials k of sequence b: the segments of its own
+// entry (slots seg_base[K + b] .., column h) and, when b belongs to pack j,
+// those of the pack's entry (slots seg_base[j] .., column member * G + h).
 // grid (B, ceil(Hq / kCombineWarps)), one warp per query head; the weights are
-// found with the lanes spread over segments, then the lanes (spread over
-// head_dim) stream the partial outputs with no dependence between segments.
+// found with the lanes spread over partials, then the lanes (spread over
+// head_dim) stream the partial outputs with no dependence between partials.
 // ---------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(kCombineWarps * 32) pa_combine_kernel(const DecodeParams p) {
@@ -733,19 +830,34 @@ __global__ void __launch_bounds__(kCombineWarps * 32) pa_combine_kernel(const De
   griddep_wait();  // the main kernel's partials are complete and visible
   if (qh >= p.num_q_heads) return;
   const int G = p.group, HG = p.heads_per_cta;
-  const int hg = (qh / G) / HG;
-  const int HGq = HG * G;
-  const int qloc = qh - hg * HGq;
-  const int32_t s0 = p.seg_base[b], ns = p.seg_base[b + 1] - s0;
-  if (ns == 1) return;  // the main kernel wrote this sequence directly
+  const int kvh = qh / G, h = qh - kvh * G;
+  const int hg = kvh / HG, g = kvh - hg * HG;
+  const int K = p.meta[0];
+  const int32_t s0 = p.seg_base[K + b], ns = p.seg_base[K + b + 1] - s0;
+  const int pk = p.pack_size > 1 ? p.seq_pack[b] : -1;
+  if (pk < 0 && ns == 1) return;  // the main kernel wrote this sequence directly
+  // partial k: k < ns from the sequence's entry, then the pack's
+  int32_t s1 = 0, np = 0, col1 = 0;
+  if (pk >= 0) {
+    s1 = p.seg_base[pk];
+    np = p.seg_base[pk + 1] - s1;
+    col1 = (b - p.pack_first[pk]) * G + h;
+  }
+  const int32_t nseq = (s0 + ns <= p.nseg_cap) ? ns : 0;
+  const int32_t npack = (s1 + np <= p.nseg_cap) ? np : 0;
+  const int32_t ntot = nseq + npack;
+  auto row_of = [&](int32_t k) {
+    const int32_t slot = k < nseq ? s0 + k : s1 + (k - nseq);
+    const int col = k < nseq ? h : col1;
+    return ((static_cast<int64_t>(hg) * p.nseg_cap + slot) * HG + g) * p.cols + col;
+  };
   const int64_t obase = (static_cast<int64_t>(b) * p.num_q_heads + qh) * D + lane * V;
-  const int64_t sidx0 = (static_cast<int64_t>(hg) * p.nseg_cap + s0) * HGq + qloc;
-  const int32_t nvalid = (s0 + ns <= p.nseg_cap) ? ns : 0;
 
   float M = -INFINITY;
-  for (int k = lane; k < nvalid; k += 32) {
-    const float m = p.part_ml[(sidx0 + static_cast<int64_t>(k) * HGq) * 2];
-    const float l = p.part_ml[(sidx0 + static_cast<int64_t>(k) * HGq) * 2 + 1];
+  for (int k = lane; k < ntot; k += 32) {
+    const int64_t r = row_of(k);
+    const float m = p.part_ml[r * 2];
+    const float l = p.part_ml[r * 2 + 1];
     if (l > 0.f) M = fmaxf(M, m);
   }
 #pragma unroll
@@ -755,13 +867,13 @@ __global__ void __launch_bounds__(kCombineWarps * 32) pa_combine_kernel(const De
   for (int v = 0; v < V; ++v) acc[v] = 0.f;
   float W = 0.f;
 #pragma unroll 4
-  for (int k = 0; k < nvalid; ++k) {
-    const int64_t sidx = sidx0 + static_cast<int64_t>(k) * HGq;
-    const float m = p.part_ml[sidx * 2];
-    const float l = p.part_ml[sidx * 2 + 1];
+  for (int k = 0; k < ntot; ++k) {
+    const int64_t r = row_of(k);
+    const float m = p.part_ml[r * 2];
+    const float l = p.part_ml[r * 2 + 1];
     if (!(l > 0.f)) continue;  // nothing attended in this partial: skip it, never 0 * o
     const float w = l * ex2(m - M);
-    const float* po = p.part_o + sidx * D + lane * V;
+    const float* po = p.part_o + r * D + lane * V;
     if constexpr (V == 4) {
       const float4 o4 = *reinterpret_cast<const float4*>(po);
       acc[0] += w * o4.x; acc[1] += w * o4.y; acc[2] += w * o4.z; acc[3] += w * o4.w;
@@ -820,9 +932,11 @@ MainKernel select_main(int D, int HG, bool bf16, bool fp8) {
 struct LaunchPlan {
   int HG = 0, groups = 0, stages = 0, tok_box = 0, threads = 0;
   int ctas_per_group = 0, tiles_per_part = INT_MAX, nseg_cap = 0;
+  int pack_size = 1, cols = 0;
   size_t smem = 0;
-  size_t off_tiles = 0, off_segs = 0, off_start = 0, off_firstk = 0, off_o = 0, off_ml = 0,
-         total = 0;
+  size_t off_tiles = 0, off_segs = 0, off_start = 0, off_firstk = 0, off_meta = 0,
+         off_pack_first = 0, off_pack_tiles = 0, off_seq_pack = 0, off_seq_pre = 0, off_o = 0,
+         off_ml = 0, total = 0;
   MainKernel kernel = nullptr;
 };
 
@@ -830,9 +944,11 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
 
+// shared_prefix: consecutive sequences may be packed over shared leading
+// blocks (8 / group sequences per pack); otherwise every sequence is its own entry.
 pa_status make_plan(int32_t num_seqs, int32_t Hq, int32_t Hkv, int32_t D, int32_t bs,
                     int32_t max_seq_len, int32_t partition_size, bool bf16, bool fp8,
-                    LaunchPlan* lp) {
+                    bool shared_prefix, LaunchPlan* lp) {
   if (num_seqs < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || bs <= 0 || max_seq_len < 0 ||
       partition_size < 0)
     return PA_ERR_INVALID_ARG;
@@ -879,17 +995,33 @@ pa_status make_plan(int32_t num_seqs, int32_t Hq, int32_t Hkv, int32_t D, int32_
     parts_per_seq = (max_tiles + lp->tiles_per_part - 1) / lp->tiles_per_part;
     if (parts_per_seq < 1) parts_per_seq = 1;
   }
-  const int64_t nseg = static_cast<int64_t>(num_seqs) * parts_per_seq + lp->ctas_per_group;
+  lp->pack_size = (shared_prefix && kMaxCols / G >= 2) ? kMaxCols / G : 1;
+  lp->cols = lp->pack_size * G;
+  // entries: at most num_seqs / pack_size packs, then the sequences
+  const int64_t max_packs = lp->pack_size > 1 ? num_seqs / lp->pack_size : 0;
+  const int64_t entries = static_cast<int64_t>(num_seqs) + max_packs;
+  const int64_t nseg = entries * parts_per_seq + lp->ctas_per_group;
   if (nseg > INT_MAX / 2) return PA_ERR_UNSUPPORTED;
   lp->nseg_cap = static_cast<int>(nseg);
+  auto words = [](int64_t n) { return align_up(static_cast<size_t>(n) * 4, 256); };
   lp->off_tiles = 0;
-  lp->off_segs = align_up(static_cast<size_t>(num_seqs + 1) * 4, 256);
-  lp->off_start = lp->off_segs + align_up(static_cast<size_t>(num_seqs + 1) * 4, 256);
-  lp->off_firstk = lp->off_start + align_up(static_cast<size_t>(lp->ctas_per_group) * 4, 256);
-  lp->off_o = lp->off_firstk + align_up(static_cast<size_t>(lp->ctas_per_group) * 4, 256);
-  const size_t o_bytes = static_cast<size_t>(lp->groups) * nseg * HG * G * D * sizeof(float);
+  lp->off_segs = lp->off_tiles + words(entries + 1);
+  lp->off_start = lp->off_segs + words(entries + 1);
+  lp->off_firstk = lp->off_start + words(lp->ctas_per_group);
+  lp->off_meta = lp->off_firstk + words(lp->ctas_per_group);
+  size_t off = lp->off_meta + words(1);
+  if (lp->pack_size > 1) {
+    lp->off_pack_first = off;
+    lp->off_pack_tiles = lp->off_pack_first + words(max_packs + 1);
+    lp->off_seq_pack = lp->off_pack_tiles + words(max_packs + 1);
+    lp->off_seq_pre = lp->off_seq_pack + words(num_seqs);
+    off = lp->off_seq_pre + words(num_seqs);
+  }
+  lp->off_o = off;
+  const size_t o_bytes = static_cast<size_t>(lp->groups) * nseg * HG * lp->cols * D * sizeof(float);
   lp->off_ml = lp->off_o + align_up(o_bytes, 256);
-  const size_t ml_bytes = static_cast<size_t>(lp->groups) * nseg * HG * G * 2 * sizeof(float);
+  const size_t ml_bytes =
+      static_cast<size_t>(lp->groups) * nseg * HG * lp->cols * 2 * sizeof(float);
   lp->total = lp->off_ml + align_up(ml_bytes, 256);
   return PA_OK;
 }
@@ -899,23 +1031,42 @@ pa_status make_plan(int32_t num_seqs, int32_t Hq, int32_t Hkv, int32_t D, int32_
 
 using namespace pa;
 
+namespace {
+
+// The larger of the 16-bit and the fp8-cache plans of one shape.
+pa_status workspace_bytes(int32_t num_seqs, int32_t Hq, int32_t Hkv, int32_t D, int32_t bs,
+                          int32_t max_seq_len, int32_t partition_size, bool shared_prefix,
+                          size_t* bytes) {
+  LaunchPlan lp;
+  const pa_status st = make_plan(num_seqs, Hq, Hkv, D, bs, max_seq_len, partition_size, true,
+                                 false, shared_prefix, &lp);
+  if (st != PA_OK) return st;
+  *bytes = lp.total;
+  LaunchPlan lp8;
+  if (make_plan(num_seqs, Hq, Hkv, D, bs, max_seq_len, partition_size, false, true,
+                shared_prefix, &lp8) == PA_OK &&
+      lp8.total > *bytes)
+    *bytes = lp8.total;
+  return PA_OK;
+}
+
+}  // namespace
+
 extern "C" pa_status pa_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads,
                                                int32_t num_kv_heads, int32_t head_dim,
                                                int32_t block_size, int32_t max_seq_len,
                                                int32_t partition_size, size_t* bytes) {
   if (bytes == nullptr) return PA_ERR_INVALID_ARG;
-  LaunchPlan lp;
-  const pa_status st = make_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
-                                 max_seq_len, partition_size, true, false, &lp);
-  if (st != PA_OK) return st;
-  *bytes = lp.total;
-  // enough for the fp8-cache kernel of the same shape too
-  LaunchPlan lp8;
-  if (make_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, max_seq_len,
-                partition_size, false, true, &lp8) == PA_OK &&
-      lp8.total > *bytes)
-    *bytes = lp8.total;
-  return PA_OK;
+  return workspace_bytes(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
+                         max_seq_len, partition_size, false, bytes);
+}
+
+extern "C" pa_status pa_decode_shared_prefix_workspace_bytes(
+    int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+    int32_t block_size, int32_t max_seq_len, int32_t partition_size, size_t* bytes) {
+  if (bytes == nullptr) return PA_ERR_INVALID_ARG;
+  return workspace_bytes(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
+                         max_seq_len, partition_size, true, bytes);
 }
 
 namespace {
@@ -929,8 +1080,8 @@ pa_status launch_decode(void* out, pa_dtype out_dtype, const void* query, pa_dty
                         const int32_t* seq_lens, int32_t num_seqs, int32_t max_seq_len,
                         int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
                         int32_t num_blocks, int32_t block_size, float scale,
-                        int32_t partition_size, void* workspace, size_t workspace_bytes,
-                        int32_t* device_error_flag, pa_stream_t stream) {
+                        int32_t partition_size, const int32_t* shared_blocks, void* workspace,
+                        size_t workspace_bytes, int32_t* device_error_flag, pa_stream_t stream) {
   if (num_seqs < 0) return PA_ERR_INVALID_ARG;
   if (num_seqs == 0) return PA_OK;
   if (!out || !query || !key_cache || !value_cache || !block_tables || !seq_lens || !workspace)
@@ -943,8 +1094,10 @@ pa_status launch_decode(void* out, pa_dtype out_dtype, const void* query, pa_dty
     return PA_ERR_INVALID_ARG;
   if (num_blocks <= 0 || !(scale == scale)) return PA_ERR_INVALID_ARG;
   LaunchPlan lp;
+  if (shared_blocks != nullptr && !aligned(shared_blocks, 4)) return PA_ERR_INVALID_ARG;
   pa_status st = make_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
-                           max_seq_len, partition_size, !fp8 && q_dtype == PA_BF16, fp8, &lp);
+                           max_seq_len, partition_size, !fp8 && q_dtype == PA_BF16, fp8,
+                           shared_blocks != nullptr, &lp);
   if (st != PA_OK) return st;
   const int64_t need_blocks = (static_cast<int64_t>(max_seq_len) + block_size - 1) / block_size;
   if (block_table_stride < need_blocks) return PA_ERR_INVALID_ARG;
@@ -1010,6 +1163,16 @@ pa_status launch_decode(void* out, pa_dtype out_dtype, const void* query, pa_dty
   p.seg_base = reinterpret_cast<int32_t*>(ws + lp.off_segs);
   p.start_seq = reinterpret_cast<int32_t*>(ws + lp.off_start);
   p.first_k = reinterpret_cast<int32_t*>(ws + lp.off_firstk);
+  p.meta = reinterpret_cast<int32_t*>(ws + lp.off_meta);
+  p.shared_blocks = shared_blocks;
+  p.pack_size = lp.pack_size;
+  p.cols = lp.cols;
+  if (lp.pack_size > 1) {
+    p.pack_first = reinterpret_cast<int32_t*>(ws + lp.off_pack_first);
+    p.pack_tiles = reinterpret_cast<int32_t*>(ws + lp.off_pack_tiles);
+    p.seq_pack = reinterpret_cast<int32_t*>(ws + lp.off_seq_pack);
+    p.seq_pre = reinterpret_cast<int32_t*>(ws + lp.off_seq_pre);
+  }
   p.part_o = reinterpret_cast<float*>(ws + lp.off_o);
   p.part_ml = reinterpret_cast<float*>(ws + lp.off_ml);
   p.err = device_error_flag;
@@ -1044,8 +1207,8 @@ extern "C" pa_status pa_decode_attention(
   return launch_decode(out, out_dtype, query, kv_dtype, key_cache, value_cache, 2, nullptr,
                        nullptr, block_tables, block_table_stride, seq_lens, num_seqs,
                        max_seq_len, num_q_heads, num_kv_heads, head_dim, num_blocks, block_size,
-                       scale, partition_size, workspace, workspace_bytes, device_error_flag,
-                       stream);
+                       scale, partition_size, nullptr, workspace, workspace_bytes,
+                       device_error_flag, stream);
 }
 
 extern "C" pa_status pa_decode_attention_fp8(
@@ -1059,8 +1222,24 @@ extern "C" pa_status pa_decode_attention_fp8(
   return launch_decode(out, out_dtype, query, query_dtype, key_cache, value_cache, 1, k_scale,
                        v_scale, block_tables, block_table_stride, seq_lens, num_seqs,
                        max_seq_len, num_q_heads, num_kv_heads, head_dim, num_blocks, block_size,
-                       scale, partition_size, workspace, workspace_bytes, device_error_flag,
-                       stream);
+                       scale, partition_size, nullptr, workspace, workspace_bytes,
+                       device_error_flag, stream);
+}
+
+extern "C" pa_status pa_decode_attention_shared_prefix(
+    void* out, pa_dtype out_dtype, const void* query, const void* key_cache,
+    const void* value_cache, const int32_t* block_tables, int32_t block_table_stride,
+    const int32_t* seq_lens, const int32_t* shared_blocks, int32_t num_seqs,
+    int32_t max_seq_len, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+    int32_t num_blocks, int32_t block_size, float scale, pa_dtype kv_dtype,
+    int32_t partition_size, void* workspace, size_t workspace_bytes, int32_t* device_error_flag,
+    pa_stream_t stream) {
+  if (shared_blocks == nullptr && num_seqs > 0) return PA_ERR_INVALID_ARG;
+  return launch_decode(out, out_dtype, query, kv_dtype, key_cache, value_cache, 2, nullptr,
+                       nullptr, block_tables, block_table_stride, seq_lens, num_seqs,
+                       max_seq_len, num_q_heads, num_kv_heads, head_dim, num_blocks, block_size,
+                       scale, partition_size, shared_blocks, workspace, workspace_bytes,
+                       device_error_flag, stream);
 }
 
 // ===========================================================================

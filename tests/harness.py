@@ -123,3 +123,44 @@ def bits_of(t: torch.Tensor) -> np.ndarray:
 
 def as_f64(t: torch.Tensor) -> np.ndarray:
     return t.detach().cpu().to(torch.float64).numpy()
+
+
+TOL_F32 = 1e-4
+
+
+def half_ulp(ref: np.ndarray, dtype: str) -> np.ndarray:
+    """Half a unit in the last place of the 16-bit storage type at |ref|: the
+    rounding that storing an exact result in that type may add."""
+    mant, emin = (7, -126) if dtype == "bf16" else (10, -14)
+    e = np.floor(np.log2(np.maximum(np.abs(ref), 2.0 ** emin)))
+    return 0.5 * np.exp2(e - mant)
+
+
+def stored_within(out, ref, dtype, tol_f32: float = TOL_F32) -> bool:
+    """Stored outputs: the fp32-path error plus the storage rounding."""
+    o = as_f64(out)
+    assert np.all(np.isfinite(o))
+    return bool(np.all(np.abs(o - ref) <= tol_f32 + half_ulp(ref, dtype)))
+
+
+def shared_blocks_of(tables: np.ndarray, seq_lens: np.ndarray, bs: int) -> np.ndarray:
+    """int32 [B]: leading block-table entries row b holds in common with row
+    b + 1 among the blocks each sequence uses (last entry 0)."""
+    B = tables.shape[0]
+    out = np.zeros(B, dtype=np.int32)
+    for b in range(B - 1):
+        n = min(-(-int(seq_lens[b]) // bs), -(-int(seq_lens[b + 1]) // bs))
+        eq = tables[b, :n] == tables[b + 1, :n]
+        out[b] = n if eq.all() else int(np.argmin(eq))
+    return out
+
+
+def pools_after_appends(prep: "Prepared"):
+    """The pools the decode step reads: after the copy-on-write copies and the
+    appended rows (oracle routines), else the prepared pools."""
+    k, v = prep.k_pool, prep.v_pool
+    if prep.cow_pairs is not None:
+        k, v = k.copy(), v.copy()
+        oracle.copy_blocks([k, v], prep.cow_pairs, int(np.prod(k.shape[1:])) * 2)
+        oracle.reshape_and_cache(prep.case.new_k, prep.case.new_v, k, v, prep.new_slots)
+    return k, v

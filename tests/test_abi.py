@@ -128,3 +128,32 @@ def test_native_block_manager_errors(pa):
     assert e.value.name == "PA_ERR_NOT_FOUND"
     with pytest.raises(pa.PagedAttnError):
         pa.BlockManager(3, 4, [0, 0, 1])  # not a permutation
+
+
+def test_native_shared_blocks_counts(pa):
+    """pa_bm_shared_blocks on forked sequences: the prompt's full blocks are
+    shared until a copy-on-write replaces the partial one."""
+    bm = pa.BlockManager(64, 4)
+    bm.add_sequence(0, 10)          # blocks a, b, c(partial)
+    bm.fork(0, 1)
+    bm.fork(0, 2)
+    bm.add_sequence(3, 9)
+    bm.append_slot(1)               # copy-on-write of the partial block
+    assert bm.shared_blocks([0, 1, 2, 3]).tolist() == [2, 2, 0, 0]
+    assert bm.shared_blocks([0, 2]).tolist() == [3, 0]
+    assert bm.shared_blocks([]).tolist() == []
+    with pytest.raises(pa.PagedAttnError) as e:
+        bm.shared_blocks([0, 9])
+    assert e.value.name == "PA_ERR_NOT_FOUND"
+
+
+def test_shared_prefix_host_validation(pa):
+    lib = pa.lib
+    # a null shared_blocks is an invalid call; zero work is a no-op
+    st = lib.pa_decode_attention_shared_prefix(None, 1, None, None, None, None, 1, None, None, 4,
+                                               16, 4, 2, 64, 8, 4, 0.125, 1, 0, None, 0, None,
+                                               None)
+    assert st == 1
+    assert lib.pa_decode_attention_shared_prefix(None, 1, None, None, None, None, 1, None, None,
+                                                 0, 16, 4, 2, 64, 8, 4, 0.125, 1, 0, None, 0,
+                                                 None, None) == 0

@@ -13,7 +13,7 @@ import pytest
 import torch
 
 import pa_workloads as W
-from harness import as_f64, prepare, to_dev
+from harness import as_f64, half_ulp, prepare, stored_within, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -63,19 +63,8 @@ def _maxerr(out, ref, seqs=None):
     return float(np.max(np.abs(o - ref)))
 
 
-def half_ulp(ref: np.ndarray, dtype: str) -> np.ndarray:
-    """Half a unit in the last place of the 16-bit storage type at |ref|: the
-    rounding that storing an exact result in that type may add."""
-    mant, emin = (7, -126) if dtype == "bf16" else (10, -14)
-    e = np.floor(np.log2(np.maximum(np.abs(ref), 2.0 ** emin)))
-    return 0.5 * np.exp2(e - mant)
-
-
 def _stored_within(out, ref, dtype):
-    """Stored outputs: the fp32-path error plus the storage rounding."""
-    o = as_f64(out)
-    assert np.all(np.isfinite(o))
-    return bool(np.all(np.abs(o - ref) <= TOL_F32 + half_ulp(ref, dtype)))
+    return stored_within(out, ref, dtype, TOL_F32)
 
 
 def _reduced(name):
