@@ -114,6 +114,14 @@ __device__ __forceinline__ int32_t clamp_len(int32_t L, int32_t max_len) {
 //               occupy slots seg_base[e] .. seg_base[e + 1] - 1;
 //   start_seq[c], first_k[c]: the entry holding lo(c) and the number of
 //               that entry's segments that start before lo(c).
+// Counting, with no walk over the cut points: CTA c "holds" the start lo(c)
+// when its share is not empty (lo(c) < lo(c + 1)), so every distinct start
+// is held once; it "coincides" when lo(c) is also a partition start of its
+// entry.  With SD, SDC the prefix sums over c of held and held-and-coincident,
+// and cnt(x) = min(C, ceil(x C / N)) the number of CTAs with lo(c) < x:
+//   segments(e)  = partitions(e) + SD/SDC counts over CTAs cnt(t0) .. cnt(t1);
+//   first_k[c]   = partition starts of e below lo(c) + held starts in
+//                  [cnt(t0), c) - coincident ones among them.
 // ---------------------------------------------------------------------------
 constexpr int kPlanWarps = kPlanThreads / 32;
 
@@ -145,45 +153,23 @@ __device__ __forceinline__ int32_t block_exclusive_scan(int32_t v, int32_t* warp
   return before;
 }
 
-// Walks the segment starts of entry b (tiles [t0, t1)) in order: the
-// partition starts and the CTA-share starts, equal points counted once.
-// Records start_seq / first_k for every CTA whose share starts inside b and
-// returns the number of segments.
-__device__ int32_t plan_sequence_segments(const DecodeParams& p, int32_t b, int64_t t0,
-                                          int64_t t1, int64_t N, int64_t C) {
-  const int64_t q = N / C, r = N % C;
-  int64_t c = (t0 * C + N - 1) / N;  // first CTA with lo(c) >= t0
-  int64_t lo_c = c * q + (c * r) / C;
-  int64_t rem = (c * r) % C;         // lo(c + 1) = lo(c) + q + [rem + r >= C]
-  int64_t part = t0;                 // next partition start
-  const int64_t tpp = p.tiles_per_part;
-  int32_t count = 0;
-  int64_t last = -1;
-  while (true) {
-    const int64_t cta_pt = (c < C && lo_c < t1) ? lo_c : INT64_MAX;
-    const int64_t part_pt = part < t1 ? part : INT64_MAX;
-    if (cta_pt == INT64_MAX && part_pt == INT64_MAX) break;
-    if (cta_pt <= part_pt) {
-      const int32_t idx = (cta_pt == last) ? count - 1 : count;
-      if (cta_pt != last) { ++count; last = cta_pt; }
-      p.start_seq[c] = b;
-      p.first_k[c] = idx;
-      ++c;
-      rem += r;
-      lo_c += q;
-      if (rem >= C) { rem -= C; ++lo_c; }
-    } else {
-      if (part_pt != last) { ++count; last = part_pt; }
-      part = (tpp == INT_MAX) ? INT64_MAX : part + tpp;
-    }
-  }
-  return count;
-}
+constexpr int kPlanSmemTiles = 4096;  // entries whose prefix sums are searched in shared memory
+constexpr int kPlanMaxCtas = 2048;    // CTAs per head group the plan can describe
 
-constexpr int kPlanRegChunks = 8;  // up to 8 x 256 entries keep their counts in registers
+// Largest e in [0, n) with tiles[e] <= x (tiles non-decreasing, tiles[0] = 0 <= x).
+__device__ __forceinline__ int upper_entry(const int32_t* tiles, int n, int64_t x) {
+  int lo = 0, hi = n;  // invariant: tiles[lo] <= x, answer in [lo, hi)
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (tiles[mid] <= x) lo = mid; else hi = mid;
+  }
+  return lo;
+}
 
 __global__ void __launch_bounds__(kPlanThreads) pa_plan_kernel(DecodeParams p) {
   __shared__ int32_t warp_buf[kPlanWarps];
+  __shared__ int32_t s_tiles[kPlanSmemTiles + 1];
+  __shared__ int32_t s_sd[kPlanMaxCtas + 1], s_sdc[kPlanMaxCtas + 1];
   const int tid = threadIdx.x;
   const int B = p.num_seqs;
   griddep_launch_dependents();
@@ -231,8 +217,6 @@ __global__ void __launch_bounds__(kPlanThreads) pa_plan_kernel(DecodeParams p) {
   if (tid == 0) p.meta[0] = K;
   const int E = K + B;  // entries: the packs' prefixes, then the sequences
   const int nchunks = (E + kPlanThreads - 1) / kPlanThreads;
-  const bool in_regs = nchunks <= kPlanRegChunks;
-  int32_t t_reg[kPlanRegChunks], n_reg[kPlanRegChunks];
   int32_t carry = 0, total = 0;
   for (int ch = 0; ch < nchunks; ++ch) {
     const int e = ch * kPlanThreads + tid;
@@ -248,41 +232,79 @@ __global__ void __launch_bounds__(kPlanThreads) pa_plan_kernel(DecodeParams p) {
     }
     const int32_t ex = block_exclusive_scan(nt, warp_buf, &total);
     if (e < E) p.plan_tiles[e] = carry + ex;
-#pragma unroll
-    for (int r = 0; r < kPlanRegChunks; ++r) {
-      if (r == ch) {
-        t_reg[r] = carry + ex;
-        n_reg[r] = nt;
-      }
-    }
+    if (e < E && e <= kPlanSmemTiles) s_tiles[e] = carry + ex;
     carry += total;
   }
-  if (tid == 0) p.plan_tiles[E] = carry;
-  if (!in_regs) __syncthreads();  // the global copy is read back below
-  const int64_t N = carry, C = p.ctas_per_group;
+  if (tid == 0) {
+    p.plan_tiles[E] = carry;
+    if (E <= kPlanSmemTiles) s_tiles[E] = carry;
+  }
+  __syncthreads();  // the prefix sums are read back below
+  const int64_t N = carry;
+  const int C = p.ctas_per_group;
+  const int32_t tpp = p.tiles_per_part;
+  const int32_t* tiles = E <= kPlanSmemTiles ? s_tiles : p.plan_tiles;
+  auto lo_of = [&](int64_t c) { return c * N / C; };
+  auto cnt_below = [&](int64_t x) {  // CTAs with lo(c) < x
+    return static_cast<int>(min(static_cast<int64_t>(C), (x * C + N - 1) / N));
+  };
+  // ---- CTAs: the entry holding each share's start; held / coincident flags,
+  // scanned together as held + coincident * 2^16 (C <= kPlanMaxCtas < 2^15)
+  int32_t sd_carry = 0, sdc_carry = 0;
+  int my_e = 0;  // the entry of CTA tid (one chunk of CTAs)
+  for (int c0 = 0; c0 < C; c0 += kPlanThreads) {  // uniform trip count: the scans sync
+    const int c = c0 + tid;
+    int32_t flags = 0;
+    if (c < C && N > 0) {
+      const int64_t x = lo_of(c);
+      const int e = upper_entry(tiles, E + 1, x);
+      p.start_seq[c] = e;
+      my_e = e;
+      const bool held = x < lo_of(c + 1);
+      const int64_t t0 = tiles[e];
+      const bool coin = held && (tpp == INT_MAX ? x == t0 : (x - t0) % tpp == 0);
+      flags = (held ? 1 : 0) + (coin ? 1 << 16 : 0);
+    }
+    int32_t tot = 0;
+    const int32_t ex = block_exclusive_scan(flags, warp_buf, &tot);
+    if (c < C) {
+      s_sd[c] = sd_carry + (ex & 0xffff);
+      s_sdc[c] = sdc_carry + (ex >> 16);
+    }
+    sd_carry += tot & 0xffff;
+    sdc_carry += tot >> 16;
+  }
+  if (tid == 0) {
+    s_sd[C] = sd_carry;
+    s_sdc[C] = sdc_carry;
+  }
+  __syncthreads();
+  // ---- entries: segment counts and their prefix sums
   int32_t seg_carry = 0;
   for (int ch = 0; ch < nchunks; ++ch) {
     const int e = ch * kPlanThreads + tid;
     int32_t ns = 0;
     if (e < E && N > 0) {
-      int64_t t0 = 0, t1 = 0;
-      if (in_regs) {
-#pragma unroll
-        for (int r = 0; r < kPlanRegChunks; ++r) {
-          if (r == ch) {
-            t0 = t_reg[r];
-            t1 = t0 + n_reg[r];
-          }
-        }
-      } else {
-        t0 = p.plan_tiles[e];
-        t1 = p.plan_tiles[e + 1];
+      const int64_t t0 = tiles[e], t1 = tiles[e + 1];
+      if (t1 > t0) {
+        const int a = cnt_below(t0), z = cnt_below(t1);
+        const int64_t parts = tpp == INT_MAX ? 1 : (t1 - t0 + tpp - 1) / tpp;
+        ns = static_cast<int32_t>(parts) + (s_sd[z] - s_sd[a]) - (s_sdc[z] - s_sdc[a]);
       }
-      if (t1 > t0) ns = plan_sequence_segments(p, e, t0, t1, N, C);
     }
     const int32_t ex = block_exclusive_scan(ns, warp_buf, &total);
     if (e < E) p.seg_base[e] = seg_carry + ex;
     seg_carry += total;
+  }
+  // ---- CTAs: index of the segment that starts at lo(c) inside its entry
+  for (int c = tid; c < C && N > 0; c += kPlanThreads) {
+    const int64_t x = lo_of(c);
+    if (x >= N) continue;  // no share: the main kernel returns before reading it
+    const int e = C <= kPlanThreads ? my_e : upper_entry(tiles, E + 1, x);
+    const int64_t t0 = tiles[e];
+    const int a = cnt_below(t0);
+    const int64_t pb = x == t0 ? 0 : (tpp == INT_MAX ? 1 : (x - t0 + tpp - 1) / tpp);
+    p.first_k[c] = static_cast<int32_t>(pb) + (s_sd[c] - s_sd[a]) - (s_sdc[c] - s_sdc[a]);
   }
   if (tid == 0) p.seg_base[E] = seg_carry;
 }
@@ -817,18 +839,21 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
 // M = max_k m_k over the partials k of sequence b: the segments of its own
 // entry (slots seg_base[K + b] .., column h) and, when b belongs to pack j,
 // those of the pack's entry (slots seg_base[j] .., column member * G + h).
-// grid (B, ceil(Hq / kCombineWarps)), one warp per query head; the weights are
-// found with the lanes spread over partials, then the lanes (spread over
-// head_dim) stream the partial outputs with no dependence between partials.
+// grid (B, Hq), one CTA per (sequence, query head).  Every warp finds M with
+// its lanes spread over the partials; then warp w takes partials w, w + W, ...
+// (lane j weighs one of them, all lanes stream the rows over head_dim with the
+// weight broadcast, the loads independent of one another), and the warps'
+// sums meet in shared memory.
 // ---------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(kCombineWarps * 32) pa_combine_kernel(const DecodeParams p) {
   constexpr int V = D / 32;  // floats per lane
+  __shared__ float s_acc[kCombineWarps][D];
+  __shared__ float s_w[kCombineWarps];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int b = blockIdx.x;
-  const int qh = blockIdx.y * kCombineWarps + warp;
+  const int qh = blockIdx.y;
   griddep_wait();  // the main kernel's partials are complete and visible
-  if (qh >= p.num_q_heads) return;
   const int G = p.group, HG = p.heads_per_cta;
   const int kvh = qh / G, h = qh - kvh * G;
   const int hg = kvh / HG, g = kvh - hg * HG;
@@ -836,7 +861,6 @@ __global__ void __launch_bounds__(kCombineWarps * 32) pa_combine_kernel(const De
   const int32_t s0 = p.seg_base[K + b], ns = p.seg_base[K + b + 1] - s0;
   const int pk = p.pack_size > 1 ? p.seq_pack[b] : -1;
   if (pk < 0 && ns == 1) return;  // the main kernel wrote this sequence directly
-  // partial k: k < ns from the sequence's entry, then the pack's
   int32_t s1 = 0, np = 0, col1 = 0;
   if (pk >= 0) {
     s1 = p.seg_base[pk];
@@ -846,47 +870,72 @@ __global__ void __launch_bounds__(kCombineWarps * 32) pa_combine_kernel(const De
   const int32_t nseq = (s0 + ns <= p.nseg_cap) ? ns : 0;
   const int32_t npack = (s1 + np <= p.nseg_cap) ? np : 0;
   const int32_t ntot = nseq + npack;
-  auto row_of = [&](int32_t k) {
+  auto row_of = [&](int32_t k) {  // partial k: own entry's first, then the pack's
     const int32_t slot = k < nseq ? s0 + k : s1 + (k - nseq);
     const int col = k < nseq ? h : col1;
     return ((static_cast<int64_t>(hg) * p.nseg_cap + slot) * HG + g) * p.cols + col;
   };
-  const int64_t obase = (static_cast<int64_t>(b) * p.num_q_heads + qh) * D + lane * V;
 
   float M = -INFINITY;
   for (int k = lane; k < ntot; k += 32) {
     const int64_t r = row_of(k);
-    const float m = p.part_ml[r * 2];
-    const float l = p.part_ml[r * 2 + 1];
-    if (l > 0.f) M = fmaxf(M, m);
+    if (p.part_ml[r * 2 + 1] > 0.f) M = fmaxf(M, p.part_ml[r * 2]);
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+
   float acc[V];
 #pragma unroll
   for (int v = 0; v < V; ++v) acc[v] = 0.f;
   float W = 0.f;
-#pragma unroll 4
-  for (int k = 0; k < ntot; ++k) {
-    const int64_t r = row_of(k);
-    const float m = p.part_ml[r * 2];
-    const float l = p.part_ml[r * 2 + 1];
-    if (!(l > 0.f)) continue;  // nothing attended in this partial: skip it, never 0 * o
-    const float w = l * ex2(m - M);
-    const float* po = p.part_o + r * D + lane * V;
-    if constexpr (V == 4) {
-      const float4 o4 = *reinterpret_cast<const float4*>(po);
-      acc[0] += w * o4.x; acc[1] += w * o4.y; acc[2] += w * o4.z; acc[3] += w * o4.w;
-    } else {
-      const float2 o2 = *reinterpret_cast<const float2*>(po);
-      acc[0] += w * o2.x; acc[1] += w * o2.y;
+  for (int r0 = 0; r0 < ntot; r0 += 32 * kCombineWarps) {
+    const int k = r0 + warp + lane * kCombineWarps;  // the partial this lane weighs
+    float w = 0.f;
+    if (k < ntot) {
+      const int64_t r = row_of(k);
+      const float m = p.part_ml[r * 2];
+      const float l = p.part_ml[r * 2 + 1];
+      w = l > 0.f ? l * ex2(m - M) : 0.f;  // nothing attended: weight 0, row skipped
     }
     W += w;
+    const int rem = ntot - r0 - warp;
+    const int cnt = rem <= 0 ? 0 : min(32, (rem + kCombineWarps - 1) / kCombineWarps);
+#pragma unroll 8
+    for (int j = 0; j < cnt; ++j) {
+      const float wj = __shfl_sync(0xffffffffu, w, j);
+      const float* po = p.part_o + row_of(r0 + warp + j * kCombineWarps) * D + lane * V;
+      // select, never 0 * o: a skipped row contributes nothing whatever it holds
+      if constexpr (V == 4) {
+        const float4 o4 = *reinterpret_cast<const float4*>(po);
+        acc[0] += wj > 0.f ? wj * o4.x : 0.f;
+        acc[1] += wj > 0.f ? wj * o4.y : 0.f;
+        acc[2] += wj > 0.f ? wj * o4.z : 0.f;
+        acc[3] += wj > 0.f ? wj * o4.w : 0.f;
+      } else {
+        const float2 o2 = *reinterpret_cast<const float2*>(po);
+        acc[0] += wj > 0.f ? wj * o2.x : 0.f;
+        acc[1] += wj > 0.f ? wj * o2.y : 0.f;
+      }
+    }
   }
-  const float inv = W > 0.f ? 1.f / W : 0.f;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) W += __shfl_xor_sync(0xffffffffu, W, o);
+#pragma unroll
+  for (int v = 0; v < V; ++v) s_acc[warp][lane * V + v] = acc[v];
+  if (lane == 0) s_w[warp] = W;
+  __syncthreads();
+  if (warp != 0) return;
+  float Wt = 0.f;
+#pragma unroll
+  for (int w2 = 0; w2 < kCombineWarps; ++w2) Wt += s_w[w2];
+  const float inv = Wt > 0.f ? 1.f / Wt : 0.f;
+  const int64_t obase = (static_cast<int64_t>(b) * p.num_q_heads + qh) * D + lane * V;
 #pragma unroll
   for (int v = 0; v < V; ++v) {
-    const float x = acc[v] * inv;
+    float x = 0.f;
+#pragma unroll
+    for (int w2 = 0; w2 < kCombineWarps; ++w2) x += s_acc[w2][lane * V + v];
+    x *= inv;
     if (p.out_dtype == PA_F32) {
       static_cast<float*>(p.out)[obase + v] = x;
     } else if (p.out_dtype == PA_BF16) {
@@ -987,6 +1036,7 @@ pa_status make_plan(int32_t num_seqs, int32_t Hq, int32_t Hkv, int32_t D, int32_
   if (per_sm < 1) return PA_ERR_CUDA;
   const int total_ctas = dev->num_sms * per_sm;
   lp->ctas_per_group = total_ctas / lp->groups > 0 ? total_ctas / lp->groups : 1;
+  if (lp->ctas_per_group > kPlanMaxCtas) lp->ctas_per_group = kPlanMaxCtas;
 
   const int64_t max_tiles = (static_cast<int64_t>(max_seq_len) + kTile - 1) / kTile;
   int64_t parts_per_seq = 1;
@@ -1188,8 +1238,7 @@ pa_status launch_decode(void* out, pa_dtype out_dtype, const void* query, pa_dty
   if (PdlLaunch(s, dim3(lp.ctas_per_group, lp.groups), dim3(lp.threads), lp.smem)(
           lp.kernel, tmK, tmV, p) != cudaSuccess)
     return PA_ERR_CUDA;
-  PdlLaunch combine(s, dim3(num_seqs, (num_q_heads + kCombineWarps - 1) / kCombineWarps),
-                    dim3(kCombineWarps * 32));
+  PdlLaunch combine(s, dim3(num_seqs, num_q_heads), dim3(kCombineWarps * 32));
   const cudaError_t e3 =
       D == 128 ? combine(pa_combine_kernel<128>, p) : combine(pa_combine_kernel<64>, p);
   return e3 == cudaSuccess ? PA_OK : PA_ERR_CUDA;
