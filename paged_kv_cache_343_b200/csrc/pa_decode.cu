@@ -70,6 +70,8 @@ struct DecodeParams {
   int32_t stages;
   int32_t tok_box;         // tokens per TMA box: min(block_size, 16)
   int32_t tma_mode;        // 0: one box per block per tile, 1: one per (head, d-half)
+  int32_t plan_closed;     // 1: segment bookkeeping in closed form (many cut points per
+                           //    entry); 0: walk each entry's cut points (few)
   int32_t* plan_tiles;     // [entries + 1] tile prefix sums
   int32_t* seg_base;       // [entries + 1] segment prefix sums (partial slots)
   int32_t* start_seq;      // [ctas_per_group] entry holding each CTA's first tile
@@ -114,7 +116,9 @@ __device__ __forceinline__ int32_t clamp_len(int32_t L, int32_t max_len) {
 //               occupy slots seg_base[e] .. seg_base[e + 1] - 1;
 //   start_seq[c], first_k[c]: the entry holding lo(c) and the number of
 //               that entry's segments that start before lo(c).
-// Counting, with no walk over the cut points: CTA c "holds" the start lo(c)
+// Two ways to count, chosen by the host from the expected cut points per
+// entry.  Few: each entry walks its own cut points in order.  Many (long
+// sequences, partitions), with no walk over the cut points: CTA c "holds" the start lo(c)
 // when its share is not empty (lo(c) < lo(c + 1)), so every distinct start
 // is held once; it "coincides" when lo(c) is also a partition start of its
 // entry.  With SD, SDC the prefix sums over c of held and held-and-coincident,
@@ -151,6 +155,41 @@ __device__ __forceinline__ int32_t block_exclusive_scan(int32_t v, int32_t* warp
   *total = warp_buf[kPlanWarps - 1];
   __syncthreads();  // warp_buf is reused by the next call
   return before;
+}
+
+// Walks the segment starts of entry b (tiles [t0, t1)) in order: the
+// partition starts and the CTA-share starts, equal points counted once.
+// Records start_seq / first_k for every CTA whose share starts inside b and
+// returns the number of segments.
+__device__ int32_t plan_sequence_segments(const DecodeParams& p, int32_t b, int64_t t0,
+                                          int64_t t1, int64_t N, int64_t C) {
+  const int64_t q = N / C, r = N % C;
+  int64_t c = (t0 * C + N - 1) / N;  // first CTA with lo(c) >= t0
+  int64_t lo_c = c * q + (c * r) / C;
+  int64_t rem = (c * r) % C;         // lo(c + 1) = lo(c) + q + [rem + r >= C]
+  int64_t part = t0;                 // next partition start
+  const int64_t tpp = p.tiles_per_part;
+  int32_t count = 0;
+  int64_t last = -1;
+  while (true) {
+    const int64_t cta_pt = (c < C && lo_c < t1) ? lo_c : INT64_MAX;
+    const int64_t part_pt = part < t1 ? part : INT64_MAX;
+    if (cta_pt == INT64_MAX && part_pt == INT64_MAX) break;
+    if (cta_pt <= part_pt) {
+      const int32_t idx = (cta_pt == last) ? count - 1 : count;
+      if (cta_pt != last) { ++count; last = cta_pt; }
+      p.start_seq[c] = b;
+      p.first_k[c] = idx;
+      ++c;
+      rem += r;
+      lo_c += q;
+      if (rem >= C) { rem -= C; ++lo_c; }
+    } else {
+      if (part_pt != last) { ++count; last = part_pt; }
+      part = (tpp == INT_MAX) ? INT64_MAX : part + tpp;
+    }
+  }
+  return count;
 }
 
 constexpr int kPlanSmemTiles = 4096;  // entries whose prefix sums are searched in shared memory
@@ -244,6 +283,22 @@ __global__ void __launch_bounds__(kPlanThreads) pa_plan_kernel(DecodeParams p) {
   const int C = p.ctas_per_group;
   const int32_t tpp = p.tiles_per_part;
   const int32_t* tiles = E <= kPlanSmemTiles ? s_tiles : p.plan_tiles;
+  if (!p.plan_closed) {  // few cut points per entry: walk them
+    int32_t seg_carry = 0;
+    for (int ch = 0; ch < nchunks; ++ch) {
+      const int e = ch * kPlanThreads + tid;
+      int32_t ns = 0;
+      if (e < E && N > 0) {
+        const int64_t t0 = tiles[e], t1 = tiles[e + 1];
+        if (t1 > t0) ns = plan_sequence_segments(p, e, t0, t1, N, C);
+      }
+      const int32_t ex = block_exclusive_scan(ns, warp_buf, &total);
+      if (e < E) p.seg_base[e] = seg_carry + ex;
+      seg_carry += total;
+    }
+    if (tid == 0) p.seg_base[E] = seg_carry;
+    return;
+  }
   auto lo_of = [&](int64_t c) { return c * N / C; };
   auto cnt_below = [&](int64_t x) {  // CTAs with lo(c) < x
     return static_cast<int>(min(static_cast<int64_t>(C), (x * C + N - 1) / N));
@@ -839,14 +894,96 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
 // M = max_k m_k over the partials k of sequence b: the segments of its own
 // entry (slots seg_base[K + b] .., column h) and, when b belongs to pack j,
 // those of the pack's entry (slots seg_base[j] .., column member * G + h).
-// grid (B, Hq), one CTA per (sequence, query head).  Every warp finds M with
+// grid (B, ceil(Hq / kCombineWarps)), one warp per query head; the weights are
+// found with the lanes spread over partials, then the lanes (spread over
+// head_dim) stream the partial outputs with no dependence between partials.
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(kCombineWarps * 32) pa_combine_narrow_kernel(const DecodeParams p) {
+  constexpr int V = D / 32;  // floats per lane
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int b = blockIdx.x;
+  const int qh = blockIdx.y * kCombineWarps + warp;
+  griddep_wait();  // the main kernel's partials are complete and visible
+  if (qh >= p.num_q_heads) return;
+  const int G = p.group, HG = p.heads_per_cta;
+  const int kvh = qh / G, h = qh - kvh * G;
+  const int hg = kvh / HG, g = kvh - hg * HG;
+  const int K = p.meta[0];
+  const int32_t s0 = p.seg_base[K + b], ns = p.seg_base[K + b + 1] - s0;
+  const int pk = p.pack_size > 1 ? p.seq_pack[b] : -1;
+  if (pk < 0 && ns == 1) return;  // the main kernel wrote this sequence directly
+  // partial k: k < ns from the sequence's entry, then the pack's
+  int32_t s1 = 0, np = 0, col1 = 0;
+  if (pk >= 0) {
+    s1 = p.seg_base[pk];
+    np = p.seg_base[pk + 1] - s1;
+    col1 = (b - p.pack_first[pk]) * G + h;
+  }
+  const int32_t nseq = (s0 + ns <= p.nseg_cap) ? ns : 0;
+  const int32_t npack = (s1 + np <= p.nseg_cap) ? np : 0;
+  const int32_t ntot = nseq + npack;
+  auto row_of = [&](int32_t k) {
+    const int32_t slot = k < nseq ? s0 + k : s1 + (k - nseq);
+    const int col = k < nseq ? h : col1;
+    return ((static_cast<int64_t>(hg) * p.nseg_cap + slot) * HG + g) * p.cols + col;
+  };
+  const int64_t obase = (static_cast<int64_t>(b) * p.num_q_heads + qh) * D + lane * V;
+
+  float M = -INFINITY;
+  for (int k = lane; k < ntot; k += 32) {
+    const int64_t r = row_of(k);
+    const float m = p.part_ml[r * 2];
+    const float l = p.part_ml[r * 2 + 1];
+    if (l > 0.f) M = fmaxf(M, m);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  float acc[V];
+#pragma unroll
+  for (int v = 0; v < V; ++v) acc[v] = 0.f;
+  float W = 0.f;
+#pragma unroll 4
+  for (int k = 0; k < ntot; ++k) {
+    const int64_t r = row_of(k);
+    const float m = p.part_ml[r * 2];
+    const float l = p.part_ml[r * 2 + 1];
+    if (!(l > 0.f)) continue;  // nothing attended in this partial: skip it, never 0 * o
+    const float w = l * ex2(m - M);
+    const float* po = p.part_o + r * D + lane * V;
+    if constexpr (V == 4) {
+      const float4 o4 = *reinterpret_cast<const float4*>(po);
+      acc[0] += w * o4.x; acc[1] += w * o4.y; acc[2] += w * o4.z; acc[3] += w * o4.w;
+    } else {
+      const float2 o2 = *reinterpret_cast<const float2*>(po);
+      acc[0] += w * o2.x; acc[1] += w * o2.y;
+    }
+    W += w;
+  }
+  const float inv = W > 0.f ? 1.f / W : 0.f;
+#pragma unroll
+  for (int v = 0; v < V; ++v) {
+    const float x = acc[v] * inv;
+    if (p.out_dtype == PA_F32) {
+      static_cast<float*>(p.out)[obase + v] = x;
+    } else if (p.out_dtype == PA_BF16) {
+      static_cast<__nv_bfloat16*>(p.out)[obase + v] = __float2bfloat16_rn(x);
+    } else {
+      static_cast<__half*>(p.out)[obase + v] = __float2half_rn(x);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Wide form of the combine, for many partials per sequence (long sequences,
+// partitions): grid (B, Hq), one CTA per (sequence, query head).  Every warp finds M with
 // its lanes spread over the partials; then warp w takes partials w, w + W, ...
 // (lane j weighs one of them, all lanes stream the rows over head_dim with the
 // weight broadcast, the loads independent of one another), and the warps'
 // sums meet in shared memory.
 // ---------------------------------------------------------------------------
 template <int D>
-__global__ void __launch_bounds__(kCombineWarps * 32) pa_combine_kernel(const DecodeParams p) {
+__global__ void __launch_bounds__(kCombineWarps * 32) pa_combine_wide_kernel(const DecodeParams p) {
   constexpr int V = D / 32;  // floats per lane
   __shared__ float s_acc[kCombineWarps][D];
   __shared__ float s_w[kCombineWarps];
@@ -982,6 +1119,7 @@ struct LaunchPlan {
   int HG = 0, groups = 0, stages = 0, tok_box = 0, threads = 0;
   int ctas_per_group = 0, tiles_per_part = INT_MAX, nseg_cap = 0;
   int pack_size = 1, cols = 0;
+  bool many_partials = false;  // long sequences / partitions: closed-form plan, wide combine
   size_t smem = 0;
   size_t off_tiles = 0, off_segs = 0, off_start = 0, off_firstk = 0, off_meta = 0,
          off_pack_first = 0, off_pack_tiles = 0, off_seq_pack = 0, off_seq_pre = 0, off_o = 0,
@@ -1051,6 +1189,11 @@ pa_status make_plan(int32_t num_seqs, int32_t Hq, int32_t Hkv, int32_t D, int32_
   const int64_t max_packs = lp->pack_size > 1 ? num_seqs / lp->pack_size : 0;
   const int64_t entries = static_cast<int64_t>(num_seqs) + max_packs;
   const int64_t nseg = entries * parts_per_seq + lp->ctas_per_group;
+  // partials one sequence expects: its partitions plus the CTA shares it spans
+  // when the batch's work is cut evenly
+  const int64_t expect = parts_per_seq + (lp->ctas_per_group + num_seqs - 1) /
+                                             (num_seqs > 0 ? num_seqs : 1);
+  lp->many_partials = expect > 6;
   if (nseg > INT_MAX / 2) return PA_ERR_UNSUPPORTED;
   lp->nseg_cap = static_cast<int>(nseg);
   auto words = [](int64_t n) { return align_up(static_cast<size_t>(n) * 4, 256); };
@@ -1209,6 +1352,7 @@ pa_status launch_decode(void* out, pa_dtype out_dtype, const void* query, pa_dty
   p.stages = lp.stages;
   p.tok_box = lp.tok_box;
   p.tma_mode = mode;
+  p.plan_closed = lp.many_partials ? 1 : 0;
   p.plan_tiles = reinterpret_cast<int32_t*>(ws + lp.off_tiles);
   p.seg_base = reinterpret_cast<int32_t*>(ws + lp.off_segs);
   p.start_seq = reinterpret_cast<int32_t*>(ws + lp.off_start);
@@ -1238,9 +1382,17 @@ pa_status launch_decode(void* out, pa_dtype out_dtype, const void* query, pa_dty
   if (PdlLaunch(s, dim3(lp.ctas_per_group, lp.groups), dim3(lp.threads), lp.smem)(
           lp.kernel, tmK, tmV, p) != cudaSuccess)
     return PA_ERR_CUDA;
-  PdlLaunch combine(s, dim3(num_seqs, num_q_heads), dim3(kCombineWarps * 32));
-  const cudaError_t e3 =
-      D == 128 ? combine(pa_combine_kernel<128>, p) : combine(pa_combine_kernel<64>, p);
+  cudaError_t e3;
+  if (lp.many_partials) {
+    PdlLaunch combine(s, dim3(num_seqs, num_q_heads), dim3(kCombineWarps * 32));
+    e3 = D == 128 ? combine(pa_combine_wide_kernel<128>, p)
+                  : combine(pa_combine_wide_kernel<64>, p);
+  } else {
+    PdlLaunch combine(s, dim3(num_seqs, (num_q_heads + kCombineWarps - 1) / kCombineWarps),
+                      dim3(kCombineWarps * 32));
+    e3 = D == 128 ? combine(pa_combine_narrow_kernel<128>, p)
+                  : combine(pa_combine_narrow_kernel<64>, p);
+  }
   return e3 == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 

@@ -149,6 +149,23 @@ def test_shapes(pa, orc, bs, dtype, hq, hkv, d):
     assert _stored_within(out, ref, dtype)
 
 
+@pytest.mark.parametrize("psize", [0, 64])
+def test_batch_of_64_short_sequences(pa, orc, psize):
+    """64 sequences of 1..400 tokens: without partitions the plan walks each
+    sequence's few cut points and the combine runs a warp per head; with
+    64-token partitions (about ten partials per sequence) it counts them in
+    closed form and the combine splits each head's partials across warps."""
+    spec = W.WORKLOADS["llama8b"].replace(len_lo=1, len_hi=400, seed=2001)
+    prep = prepare(spec)
+    ref = _oracle(orc, prep)
+    out = _run(pa, prep, partition_size=psize)
+    # short sequences: |out| reaches a few units, where bf16 storage alone
+    # rounds by more than 2e-3; the fp32 output carries the tight bound
+    assert _stored_within(out, ref, spec.dtype)
+    out32 = _run(pa, prep, out_dtype=torch.float32, partition_size=psize)
+    assert _maxerr(out32, ref) <= TOL_F32
+
+
 def test_empty_and_single_token_sequences(pa, orc):
     spec = W.Spec("edge", 6, 8, 2, 128, 16, "bf16", seed=5, len_dist="fixed",
                   fixed_lens=(0, 1, 16, 17, 0, 33))

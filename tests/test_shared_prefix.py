@@ -113,6 +113,12 @@ def test_group_shapes(pa, orc, hq, hkv, d, bs, dtype):
     _check(pa, orc, spec)
 
 
+def test_many_prompts(pa, orc):
+    """6 prompts x 8 samples (48 sequences): the plan walks the few cut points
+    of each entry and the combine runs a warp per head."""
+    _check(pa, orc, _spec(prompts=6, prompt_len=300, extra_hi=40))
+
+
 @pytest.mark.parametrize("psize", [16, 64, 512])
 def test_partitions(pa, orc, psize):
     _check(pa, orc, _spec(prompt_len=900, extra_hi=80), partition_size=psize)
