@@ -223,24 +223,33 @@ def unique_kv_bytes(spec, wl) -> int:
 
 
 def packed_kv_bytes(spec, wl) -> int:
-    """KV bytes the shared-prefix decode must read: each pack of 8 // group
-    neighbouring sequences (aligned windows) reads its common prefix -- whole
-    16-token tiles of blocks full in every member, at least 64 tokens -- once,
-    and every sequence its remaining tokens."""
+    """KV bytes the shared-prefix decode reads: aligned windows of
+    P = min(8, 32 // group) neighbouring sequences (else the aligned pairs
+    inside a window, or inside the shorter last window) read their common prefix -- whole 16-token tiles of blocks
+    full in every member, at least 64 tokens -- once, and every sequence its
+    remaining tokens."""
     G = spec.num_q_heads // spec.num_kv_heads
-    PK = 8 // G if 8 // G >= 2 else 1
+    P = min(8, 32 // G)
     bs = spec.block_size
     lens = wl["lens"].astype(np.int64)
     sb = wl["shared_blocks"].astype(np.int64)
+
+    def common(b0, n):
+        c = min(int(lens[b0 + m]) // bs for m in range(n))
+        c = min([c] + [max(0, int(sb[b0 + m])) for m in range(n - 1)])
+        t = c * bs // 16
+        return t if t >= 4 else 0
+
     tokens = int(lens.sum())
-    if PK > 1:
-        for w in range(spec.num_seqs // PK):
-            b0 = w * PK
-            P = min(int(lens[b0 + m]) // bs for m in range(PK))
-            P = min([P] + [max(0, int(sb[b0 + m])) for m in range(PK - 1)])
-            tiles = P * bs // 16
-            if tiles >= 4:
-                tokens -= (PK - 1) * tiles * 16
+    if P >= 2:
+        for w in range(-(-spec.num_seqs // P)):
+            n = min(P, spec.num_seqs - w * P)
+            whole = common(w * P, P) if n == P else 0
+            if whole:
+                tokens -= (P - 1) * whole * 16
+            elif P > 2:
+                for j in range(n // 2):
+                    tokens -= common(w * P + 2 * j, 2) * 16
     return tokens * 2 * spec.num_kv_heads * spec.head_dim * spec.elem_bytes
 
 
@@ -392,9 +401,9 @@ def run_ours(args, rank, world, local_rank):
     peaks, peak_kind = load_peaks()
     ms_per_step = elapsed_ms / args.steps
     value = total_bytes * args.steps / (elapsed_ms / 1e3) / 1e9
-    # the roofline counts the bytes the kernel must read: with packing, a
-    # shared prefix once per pack
-    read_bytes = packed_kv_bytes(spec, wl) if shared else bytes_step
+    # the roofline counts the bytes that must come from HBM: for shared
+    # prompts each distinct (block, slot) once, else every token's K and V
+    read_bytes = unique_kv_bytes(spec, wl) if spec.len_dist == "shared_prefix" else bytes_step
     achieved = read_bytes / (att_avg_ms / 1e3) / 1e9
     peak = float(peaks["hbm_gbs"])
     traffic = profiled_traffic() if args.workload == "llama8b" else None
@@ -431,8 +440,11 @@ def run_ours(args, rank, world, local_rank):
     if spec.len_dist == "shared_prefix":
         ub = unique_kv_bytes(spec, wl)
         line["config"]["unique_kv_bytes_per_step"] = ub
-        line["config"]["entry_point"] = ("decode_attention_shared_prefix (packs of %d)" % (
-            8 // spec.group) if shared else "decode_attention")
+        line["config"]["entry_point"] = ("decode_attention_shared_prefix (packs of up to %d)" % (
+            min(8, 32 // spec.group)) if shared else "decode_attention")
+        if shared:
+            line["config"]["packed_kv_bytes_per_step"] = packed_kv_bytes(spec, wl)
+        line["roofline"]["basis"] = "unique KV bytes (each shared block once)"
         line["unique_gbs"] = round(ub * args.steps / (elapsed_ms / 1e3) / 1e9, 2)
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(spec, wl, budget_s=args.cpu_budget)

@@ -41,7 +41,8 @@ enum : int32_t {
   kDirect = 8,    // the segment is the whole sequence: write `out` directly
 };
 
-constexpr int kMaxCols = 8;        // query columns per KV head in one MMA (its N)
+constexpr int kMaxPack = 8;        // sequences per pack
+constexpr int kMaxPackCols = 32;   // query columns per KV head of a pack (4 blocks of 8)
 constexpr int kMinPackTiles = 4;   // shared prefixes shorter than this are not packed
 
 struct TileInfo {
@@ -80,9 +81,10 @@ struct DecodeParams {
   // share leading blocks are attended together over that prefix ("entries"
   // 0 .. K-1 are the packs' prefixes, K + b the rest of sequence b)
   const int32_t* shared_blocks;  // [num_seqs] leading blocks b shares with b + 1, or null
-  int32_t pack_size;       // sequences per pack (8 / group, or 1: no packing)
-  int32_t* pack_first;     // [num_seqs] first sequence of pack k
-  int32_t* pack_tiles;     // [num_seqs] prefix tiles of pack k
+  int32_t pack_size;       // sequences per window (1: no packing)
+  int32_t* pack_first;     // [num_seqs / 2] first sequence of pack k
+  int32_t* pack_n;         // [num_seqs / 2] sequences of pack k (pack_size, or 2)
+  int32_t* pack_tiles;     // [num_seqs / 2] prefix tiles of pack k
   int32_t* seq_pack;       // [num_seqs] pack of sequence b, or -1
   int32_t* seq_pre;        // [num_seqs] tiles of b attended through its pack
   int32_t* meta;           // [1] number of packs K (0 without packing)
@@ -213,43 +215,69 @@ __global__ void __launch_bounds__(kPlanThreads) pa_plan_kernel(DecodeParams p) {
   const int B = p.num_seqs;
   griddep_launch_dependents();
   griddep_wait();  // seq_lens may come from the previous kernel on the stream
-  // ---- packs: aligned windows b = P w .. P w + P - 1 over their shared prefix
+  // ---- packs: aligned windows b = P w .. P w + P - 1 over their shared
+  // prefix; a window whose members do not all share one (or the shorter last
+  // window) falls back to the aligned pairs inside it
   int K = 0;
   if (p.pack_size > 1) {
     const int PK = p.pack_size;
-    const int W = B / PK;
+    const int W = (B + PK - 1) / PK;
+    // prefix tiles common to sequences b0 .. b0 + n - 1 (0 if under the minimum)
+    auto common_tiles = [&](int b0, int n) {
+      int64_t P = INT64_MAX;  // blocks common to all members and full in each
+      for (int m = 0; m < n; ++m) {
+        P = min(P, static_cast<int64_t>(clamp_len(p.seq_lens[b0 + m], p.max_seq_len) /
+                                        p.block_size));
+        if (m + 1 < n) P = min(P, static_cast<int64_t>(max(0, p.shared_blocks[b0 + m])));
+      }
+      const int32_t tiles = static_cast<int32_t>(P * p.block_size / kTile);
+      return tiles < kMinPackTiles ? 0 : tiles;
+    };
     for (int w0 = 0; w0 < W; w0 += kPlanThreads) {  // uniform trip count: the scan syncs
       const int w = w0 + tid;
-      int32_t tiles = 0;
+      int32_t whole = 0, npairs = 0;
+      int32_t pair_tiles[kMaxPack / 2] = {0, 0, 0, 0};
+      const int n = w < W ? min(PK, B - w * PK) : 0;  // sequences of this window
       if (w < W) {
-        const int b0 = w * PK;
-        int64_t P = INT64_MAX;  // blocks common to all members and full in each
-        for (int m = 0; m < PK; ++m) {
-          P = min(P, static_cast<int64_t>(clamp_len(p.seq_lens[b0 + m], p.max_seq_len) /
-                                          p.block_size));
-          if (m + 1 < PK) P = min(P, static_cast<int64_t>(max(0, p.shared_blocks[b0 + m])));
+        whole = n == PK ? common_tiles(w * PK, PK) : 0;
+        if (whole == 0 && PK > 2) {
+          for (int j = 0; j < n / 2; ++j) {
+            pair_tiles[j] = common_tiles(w * PK + 2 * j, 2);
+            if (pair_tiles[j] > 0) ++npairs;
+          }
         }
-        tiles = static_cast<int32_t>(P * p.block_size / kTile);
-        if (tiles < kMinPackTiles) tiles = 0;
       }
+      const int32_t mine = whole > 0 ? 1 : npairs;
       int32_t count = 0;
-      const int32_t k = K + block_exclusive_scan(tiles > 0 ? 1 : 0, warp_buf, &count);
+      int32_t k = K + block_exclusive_scan(mine, warp_buf, &count);
       if (w < W) {
         const int b0 = w * PK;
-        if (tiles > 0) {
-          p.pack_first[k] = b0;
-          p.pack_tiles[k] = tiles;
+        for (int m = 0; m < n; ++m) {
+          p.seq_pack[b0 + m] = -1;
+          p.seq_pre[b0 + m] = 0;
         }
-        for (int m = 0; m < PK; ++m) {
-          p.seq_pack[b0 + m] = tiles > 0 ? k : -1;
-          p.seq_pre[b0 + m] = tiles;
+        if (whole > 0) {
+          p.pack_first[k] = b0;
+          p.pack_n[k] = PK;
+          p.pack_tiles[k] = whole;
+          for (int m = 0; m < PK; ++m) {
+            p.seq_pack[b0 + m] = k;
+            p.seq_pre[b0 + m] = whole;
+          }
+        } else {
+          for (int j = 0; j < n / 2; ++j) {
+            if (pair_tiles[j] == 0) continue;
+            const int bp = b0 + 2 * j;
+            p.pack_first[k] = bp;
+            p.pack_n[k] = 2;
+            p.pack_tiles[k] = pair_tiles[j];
+            p.seq_pack[bp] = p.seq_pack[bp + 1] = k;
+            p.seq_pre[bp] = p.seq_pre[bp + 1] = pair_tiles[j];
+            ++k;
+          }
         }
       }
       K += count;
-    }
-    for (int b = W * PK + tid; b < B; b += kPlanThreads) {
-      p.seq_pack[b] = -1;
-      p.seq_pre[b] = 0;
     }
     __syncthreads();  // the pack arrays are read back below
   }
@@ -378,11 +406,20 @@ __global__ void __launch_bounds__(kPlanThreads) pa_plan_kernel(DecodeParams p) {
 //    products are unchanged;
 //  - the output rows of O^T = V^T P^T: accumulator row grp of m-tile mt is
 //    d = 16 grp + 2 mt, row grp + 8 is d = 16 grp + 2 mt + 1.
-template <int D, int HG, bool kBF16, bool kFP8>
-__global__ void __launch_bounds__((HG + 1) * 32, 1)
+//
+// Query columns.  Each consumer warp owns NB blocks of 8 query columns of one
+// KV head (the N of its MMAs); CG warps share a KV head, so a head has
+// 8 NB CG columns.  Column c of a tile is query head c % G of sequence
+// b + c / G: a sequence's own tiles use the first G columns, a pack's tiles
+// one column per (member, head).
+template <int D, int HG, int NB, int CG, bool kBF16, bool kFP8>
+__global__ void __launch_bounds__((HG * CG + 1) * 32, 1)
     pa_decode_main_kernel(const __grid_constant__ CUtensorMap tmK,
                           const __grid_constant__ CUtensorMap tmV, const DecodeParams p) {
   static_assert(!kFP8 || (D == 128 && !kBF16), "fp8 caches: head_dim 128, fp16 MMA");
+  static_assert(!kFP8 || (NB == 1 && CG == 1), "fp8 caches: one column block per head");
+  static_assert(NB == 1 || NB == 2, "one or two column blocks per warp");
+  constexpr int NW = HG * CG;                      // consumer warps
   constexpr int DC = D / 64;                       // 128-byte column chunks of a 16-bit row
   constexpr int DCT = kFP8 ? 1 : DC;               // 128-byte rows per (token, head) in a stage
   constexpr int KSTEPS = D / 16;                   // k16 steps of S^T = K Q^T
@@ -411,11 +448,11 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
     for (int s = 0; s < NS; ++s) {
       mbar_init(full_k(s), 1);
       mbar_init(full_v(s), 1);
-      mbar_init(empty(s), HG);
+      mbar_init(empty(s), NW);
     }
     fence_mbar_init();
   }
-  if (warp == HG && lane == 0) {
+  if (warp == NW && lane == 0) {
     prefetch_tmap(&tmK);
     prefetch_tmap(&tmV);
   }
@@ -429,7 +466,7 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
   const int64_t hi = static_cast<int64_t>(c + 1) * N / C;
   if (lo >= hi) return;
 
-  if (warp == HG) {
+  if (warp == NW) {
     // ======================= producer =======================
     if (lane != 0) return;
     const uint64_t policy = l2_policy_evict_first();
@@ -451,7 +488,7 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
       nseg_e = p.seg_base[ent + 1] - seg_e;
       if (ent < K) {
         b = p.pack_first[ent];
-        members = p.pack_size;
+        members = p.pack_n[ent];
         i0 = 0;
         L_b = n_e * kTile;
       } else {
@@ -587,9 +624,10 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
     return;
   }
 
-  // ======================= consumers: one warp per KV head =======================
-  const int g = warp;                         // KV head inside the group
+  // ================ consumers: CG warps per KV head, NB column blocks each ================
+  const int g = warp / CG;                    // KV head inside the group
   const int kvh = hg * HG + g;                // KV head
+  const int col0 = 8 * NB * (warp - g * CG);  // first query column of this warp
   const int G = p.group;
   const int quad = lane & 3, grp = lane >> 2;
   const int TB = p.tok_box;
@@ -627,9 +665,9 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
     v_scale = *p.v_scale;
   }
 
-  uint32_t qf[KSTEPS][2];
-  float acc[MTILES][4];
-  float m_run[2], l_part[2];
+  uint32_t qf[NB][KSTEPS][2];
+  float acc[NB][MTILES][4];
+  float m_run[NB][2], l_part[NB][2];
   int stage = 0;
   uint32_t phase = 0;
   const float sl2 = p.scale_log2 * k_scale;
@@ -637,36 +675,56 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
   for (int64_t t = lo; t < hi; ++t) {
     if (!mbar_wait(full_k(stage), phase, p.err)) break;
     const TileInfo ti = info[stage];
+    const int ncol = ti.members * G;  // query columns of this tile, per KV head
+    if (CG > 1 && col0 >= ncol) {
+      // No column of this warp takes part (a sequence's own tiles fill only
+      // the first G columns).  A warp of column group 0 always does and waits
+      // for the whole stage, so the stage can be handed back at once.
+      __syncwarp();
+      if (lane == 0) mbar_arrive(empty(stage));
+      if (++stage == NS) { stage = 0; phase ^= 1u; }
+      continue;
+    }
     if (ti.flags & kNewSeq) {
-      // column grp: query head grp % G of pack member grp / G (sequence b + member)
-      const int member = grp / G;
-      const uint16_t* qb =
-          p.query +
-          ((static_cast<int64_t>(ti.b) + member) * p.num_q_heads + kvh * G + (grp - member * G)) * D;
 #pragma unroll
-      for (int kc = 0; kc < KSTEPS; ++kc) {
-        if (grp < ti.members * G) {
-          // fp8: k = 2q, 2q+1 -> d = 32q + 4kc + {0,1}; k = 2q+8, 2q+9 -> + {2,3}
-          const uint16_t* qp = kFP8 ? qb + 32 * quad + 4 * kc : qb + kc * 16 + quad * 2;
-          qf[kc][0] = *reinterpret_cast<const uint32_t*>(qp);
-          qf[kc][1] = *reinterpret_cast<const uint32_t*>(qp + (kFP8 ? 2 : 8));
-          if (kFP8 && p.q_bf16) {  // the fp8 path multiplies in fp16
-            qf[kc][0] = bf16x2_to_f16x2(qf[kc][0]);
-            qf[kc][1] = bf16x2_to_f16x2(qf[kc][1]);
+      for (int nb = 0; nb < NB; ++nb) {
+        // column c: query head c % G of pack member c / G (sequence b + member)
+        const int col = col0 + 8 * nb + grp;
+        const int member = col / G;
+        const uint16_t* qb =
+            p.query +
+            ((static_cast<int64_t>(ti.b) + member) * p.num_q_heads + kvh * G + (col - member * G)) *
+                D;
+#pragma unroll
+        for (int kc = 0; kc < KSTEPS; ++kc) {
+          if (col < ncol) {
+            // fp8: k = 2q, 2q+1 -> d = 32q + 4kc + {0,1}; k = 2q+8, 2q+9 -> + {2,3}
+            const uint16_t* qp = kFP8 ? qb + 32 * quad + 4 * kc : qb + kc * 16 + quad * 2;
+            qf[nb][kc][0] = *reinterpret_cast<const uint32_t*>(qp);
+            qf[nb][kc][1] = *reinterpret_cast<const uint32_t*>(qp + (kFP8 ? 2 : 8));
+            if (kFP8 && p.q_bf16) {  // the fp8 path multiplies in fp16
+              qf[nb][kc][0] = bf16x2_to_f16x2(qf[nb][kc][0]);
+              qf[nb][kc][1] = bf16x2_to_f16x2(qf[nb][kc][1]);
+            }
+          } else {
+            qf[nb][kc][0] = 0u;
+            qf[nb][kc][1] = 0u;
           }
-        } else {
-          qf[kc][0] = 0u;
-          qf[kc][1] = 0u;
         }
       }
     }
     if (ti.flags & kSegStart) {
 #pragma unroll
-      for (int mt = 0; mt < MTILES; ++mt)
-        acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
-      m_run[0] = m_run[1] = -INFINITY;
-      l_part[0] = l_part[1] = 0.f;
+      for (int nb = 0; nb < NB; ++nb) {
+#pragma unroll
+        for (int mt = 0; mt < MTILES; ++mt)
+          acc[nb][mt][0] = acc[nb][mt][1] = acc[nb][mt][2] = acc[nb][mt][3] = 0.f;
+        m_run[nb][0] = m_run[nb][1] = -INFINITY;
+        l_part[nb][0] = l_part[nb][1] = 0.f;
+      }
     }
+    // n8 blocks of this warp with at least one column (warp-uniform)
+    const bool act1 = NB > 1 && col0 + 8 < ncol;
     const uint32_t kbase = smem_base + static_cast<uint32_t>(stage) * 2u * kTileBytes;
     const uint32_t vbase = kbase + kTileBytes;
     // fp8: this lane's code bytes.  K: tokens grp, grp+8, d in [32q, 32q + 32)
@@ -701,9 +759,11 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
       if (lane == 0) mbar_arrive(empty(stage));
     }
 
-    // ---- S^T[16 tok x 8 heads] = K[16 x D] * Q^T[D x 8]
-    float s[4] = {0.f, 0.f, 0.f, 0.f};
-    float s2[4] = {0.f, 0.f, 0.f, 0.f};  // odd k-steps: two independent MMA chains
+    // ---- S^T[16 tok x 8 columns] = K[16 x D] * Q^T[D x 8], per n8 block
+    float s[NB][4];
+    float s2[4] = {0.f, 0.f, 0.f, 0.f};  // one block: odd k-steps form a second chain
+#pragma unroll
+    for (int nb = 0; nb < NB; ++nb) s[nb][0] = s[nb][1] = s[nb][2] = s[nb][3] = 0.f;
 #pragma unroll
     for (int kc = 0; kc < KSTEPS; ++kc) {
       uint32_t a0, a1, a2, a3;
@@ -718,62 +778,77 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
         const uint32_t chunk = static_cast<uint32_t>((2 * (kc & 3) + k_chunk) ^ (r & 7));
         ldmatrix_x4(kbase + static_cast<uint32_t>(r) * 128u + chunk * 16u, a0, a1, a2, a3);
       }
-      if (kc & 1) {
-        mma_16816<kBF16>(s2, a0, a1, a2, a3, qf[kc][0], qf[kc][1]);
+      if constexpr (NB == 1) {
+        if (kc & 1) {
+          mma_16816<kBF16>(s2, a0, a1, a2, a3, qf[0][kc][0], qf[0][kc][1]);
+        } else {
+          mma_16816<kBF16>(s[0], a0, a1, a2, a3, qf[0][kc][0], qf[0][kc][1]);
+        }
       } else {
-        mma_16816<kBF16>(s, a0, a1, a2, a3, qf[kc][0], qf[kc][1]);
+        mma_16816<kBF16>(s[0], a0, a1, a2, a3, qf[0][kc][0], qf[0][kc][1]);
+        if (act1) mma_16816<kBF16>(s[1], a0, a1, a2, a3, qf[1][kc][0], qf[1][kc][1]);
       }
     }
-    s[0] += s2[0];
-    s[1] += s2[1];
-    s[2] += s2[2];
-    s[3] += s2[3];
-    // ---- online softmax (base 2), masked by selection
+    if constexpr (NB == 1) {
+      s[0][0] += s2[0];
+      s[0][1] += s2[1];
+      s[0][2] += s2[2];
+      s[0][3] += s2[3];
+    }
+    // ---- online softmax (base 2), masked by selection, per n8 block
     const uint32_t mask = static_cast<uint32_t>(ti.mask);
     const bool ok0 = (mask >> grp) & 1u, ok1 = (mask >> (grp + 8)) & 1u;
-    s[0] = ok0 ? s[0] * sl2 : -INFINITY;
-    s[1] = ok0 ? s[1] * sl2 : -INFINITY;
-    s[2] = ok1 ? s[2] * sl2 : -INFINITY;
-    s[3] = ok1 ? s[3] * sl2 : -INFINITY;
-    float mx0 = fmaxf(s[0], s[2]), mx1 = fmaxf(s[1], s[3]);
+    uint32_t pb0[NB], pb1[NB], pc0[NB], pc1[NB];
 #pragma unroll
-    for (int o = 4; o < 32; o <<= 1) {
-      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
-      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
-    }
-    const float mn0 = fmaxf(m_run[0], mx0), mn1 = fmaxf(m_run[1], mx1);
-    const float alpha0 = (mn0 == m_run[0]) ? 1.f : ex2(m_run[0] - mn0);
-    const float alpha1 = (mn1 == m_run[1]) ? 1.f : ex2(m_run[1] - mn1);
-    m_run[0] = mn0;
-    m_run[1] = mn1;
-    const float p0 = (s[0] == -INFINITY) ? 0.f : ex2(s[0] - mn0);
-    const float p1 = (s[1] == -INFINITY) ? 0.f : ex2(s[1] - mn1);
-    const float p2 = (s[2] == -INFINITY) ? 0.f : ex2(s[2] - mn0);
-    const float p3 = (s[3] == -INFINITY) ? 0.f : ex2(s[3] - mn1);
-    // P in two 16-bit halves, P = hi + lo, so the P.V product keeps about
-    // 16 significant bits of every weight instead of the storage type's 8 or 11.
-    const uint32_t pt0 = pack2<kBF16>(p0, p1);  // P^T row grp     (heads 2q, 2q+1)
-    const uint32_t pt1 = pack2<kBF16>(p2, p3);  // P^T row grp + 8
-    const uint32_t pl0 = pack2<kBF16>(p0 - lo_to_float<kBF16>(pt0), p1 - hi_to_float<kBF16>(pt0));
-    const uint32_t pl1 = pack2<kBF16>(p2 - lo_to_float<kBF16>(pt1), p3 - hi_to_float<kBF16>(pt1));
-    l_part[0] = l_part[0] * alpha0 + (p0 + p2);
-    l_part[1] = l_part[1] * alpha1 + (p1 + p3);
-    if (__any_sync(0xffffffffu, alpha0 != 1.f || alpha1 != 1.f)) {
+    for (int nb = 0; nb < NB; ++nb) {
+      if (nb == 1 && !act1) continue;
+      float* sv = s[nb];
+      sv[0] = ok0 ? sv[0] * sl2 : -INFINITY;
+      sv[1] = ok0 ? sv[1] * sl2 : -INFINITY;
+      sv[2] = ok1 ? sv[2] * sl2 : -INFINITY;
+      sv[3] = ok1 ? sv[3] * sl2 : -INFINITY;
+      float mx0 = fmaxf(sv[0], sv[2]), mx1 = fmaxf(sv[1], sv[3]);
 #pragma unroll
-      for (int mt = 0; mt < MTILES; ++mt) {
-        acc[mt][0] *= alpha0;
-        acc[mt][1] *= alpha1;
-        acc[mt][2] *= alpha0;
-        acc[mt][3] *= alpha1;
+      for (int o = 4; o < 32; o <<= 1) {
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
       }
+      const float mn0 = fmaxf(m_run[nb][0], mx0), mn1 = fmaxf(m_run[nb][1], mx1);
+      const float alpha0 = (mn0 == m_run[nb][0]) ? 1.f : ex2(m_run[nb][0] - mn0);
+      const float alpha1 = (mn1 == m_run[nb][1]) ? 1.f : ex2(m_run[nb][1] - mn1);
+      m_run[nb][0] = mn0;
+      m_run[nb][1] = mn1;
+      const float p0 = (sv[0] == -INFINITY) ? 0.f : ex2(sv[0] - mn0);
+      const float p1 = (sv[1] == -INFINITY) ? 0.f : ex2(sv[1] - mn1);
+      const float p2 = (sv[2] == -INFINITY) ? 0.f : ex2(sv[2] - mn0);
+      const float p3 = (sv[3] == -INFINITY) ? 0.f : ex2(sv[3] - mn1);
+      // P in two 16-bit halves, P = hi + lo, so the P.V product keeps about
+      // 16 significant bits of every weight instead of the storage type's 8 or 11.
+      const uint32_t pt0 = pack2<kBF16>(p0, p1);  // P^T row grp     (columns 2q, 2q+1)
+      const uint32_t pt1 = pack2<kBF16>(p2, p3);  // P^T row grp + 8
+      const uint32_t pl0 =
+          pack2<kBF16>(p0 - lo_to_float<kBF16>(pt0), p1 - hi_to_float<kBF16>(pt0));
+      const uint32_t pl1 =
+          pack2<kBF16>(p2 - lo_to_float<kBF16>(pt1), p3 - hi_to_float<kBF16>(pt1));
+      l_part[nb][0] = l_part[nb][0] * alpha0 + (p0 + p2);
+      l_part[nb][1] = l_part[nb][1] * alpha1 + (p1 + p3);
+      if (__any_sync(0xffffffffu, alpha0 != 1.f || alpha1 != 1.f)) {
+#pragma unroll
+        for (int mt = 0; mt < MTILES; ++mt) {
+          acc[nb][mt][0] *= alpha0;
+          acc[nb][mt][1] *= alpha1;
+          acc[nb][mt][2] *= alpha0;
+          acc[nb][mt][3] *= alpha1;
+        }
+      }
+      // P^T as the B operand (k = token, n = column): transpose the 8x8 halves
+      pb0[nb] = movmatrix_trans(pt0);
+      pb1[nb] = movmatrix_trans(pt1);
+      pc0[nb] = movmatrix_trans(pl0);
+      pc1[nb] = movmatrix_trans(pl1);
     }
-    // P^T as the B operand (k = token, n = head): transpose the 8x8 halves
-    const uint32_t pb0 = movmatrix_trans(pt0);
-    const uint32_t pb1 = movmatrix_trans(pt1);
-    const uint32_t pc0 = movmatrix_trans(pl0);
-    const uint32_t pc1 = movmatrix_trans(pl1);
 
-    // ---- O^T[D x 8] += V^T[D x 16 tok] * P^T[16 tok x 8]
+    // ---- O^T[D x 8] += V^T[D x 16 tok] * P^T[16 tok x 8], per n8 block
     if (!kFP8 && !mbar_wait(full_v(stage), phase, p.err)) break;
     const bool partial = mask != 0xffffu;
     uint32_t z01 = 0xffffffffu, z23 = 0xffffffffu;
@@ -809,8 +884,14 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
       a1 &= z01;
       a2 &= z23;
       a3 &= z23;
-      mma_16816<kBF16>(acc[mt], a0, a1, a2, a3, pb0, pb1);
-      mma_16816<kBF16>(acc[mt], a0, a1, a2, a3, pc0, pc1);
+      mma_16816<kBF16>(acc[0][mt], a0, a1, a2, a3, pb0[0], pb1[0]);
+      mma_16816<kBF16>(acc[0][mt], a0, a1, a2, a3, pc0[0], pc1[0]);
+      if constexpr (NB > 1) {
+        if (act1) {
+          mma_16816<kBF16>(acc[1][mt], a0, a1, a2, a3, pb0[1], pb1[1]);
+          mma_16816<kBF16>(acc[1][mt], a0, a1, a2, a3, pc0[1], pc1[1]);
+        }
+      }
     }
     if constexpr (!kFP8) {
       __syncwarp();
@@ -819,71 +900,76 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
     if (++stage == NS) { stage = 0; phase ^= 1u; }
 
     if (ti.flags & kSegEnd) {
-      float l0 = l_part[0], l1 = l_part[1];
 #pragma unroll
-      for (int o = 4; o < 32; o <<= 1) {
-        l0 += __shfl_xor_sync(0xffffffffu, l0, o);
-        l1 += __shfl_xor_sync(0xffffffffu, l1, o);
-      }
-      const float inv0 = l0 > 0.f ? v_scale / l0 : 0.f;
-      const float inv1 = l1 > 0.f ? v_scale / l1 : 0.f;
-      const int h0 = 2 * quad, h1 = h0 + 1;
-      if (ti.flags & kDirect) {
-        const int64_t obase = (static_cast<int64_t>(ti.b) * p.num_q_heads + kvh * G) * D;
+      for (int nb = 0; nb < NB; ++nb) {
+        if (nb == 1 && !act1) continue;
+        const int cb = col0 + 8 * nb;  // first column of the block
+        float l0 = l_part[nb][0], l1 = l_part[nb][1];
 #pragma unroll
-        for (int mt = 0; mt < MTILES; ++mt) {
-          const int d0 = d_of(mt, 0), d1 = d_of(mt, 1);
+        for (int o = 4; o < 32; o <<= 1) {
+          l0 += __shfl_xor_sync(0xffffffffu, l0, o);
+          l1 += __shfl_xor_sync(0xffffffffu, l1, o);
+        }
+        const float inv0 = l0 > 0.f ? v_scale / l0 : 0.f;
+        const float inv1 = l1 > 0.f ? v_scale / l1 : 0.f;
+        const int h0 = cb + 2 * quad, h1 = h0 + 1;  // this lane's two columns
+        if (ti.flags & kDirect) {  // one sequence: columns are its query heads
+          const int64_t obase = (static_cast<int64_t>(ti.b) * p.num_q_heads + kvh * G) * D;
 #pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-            const int h = hh ? h1 : h0;
-            if (h >= G) continue;
-            const float inv = hh ? inv1 : inv0;
-            const float v0 = acc[mt][hh] * inv, v1 = acc[mt][2 + hh] * inv;
-            const int64_t o = obase + static_cast<int64_t>(h) * D;
-            if (p.out_dtype == PA_F32) {
-              float* op = static_cast<float*>(p.out);
-              op[o + d0] = v0;
-              op[o + d1] = v1;
-            } else if (p.out_dtype == PA_BF16) {
-              __nv_bfloat16* op = static_cast<__nv_bfloat16*>(p.out);
-              op[o + d0] = __float2bfloat16_rn(v0);
-              op[o + d1] = __float2bfloat16_rn(v1);
-            } else {
-              __half* op = static_cast<__half*>(p.out);
-              op[o + d0] = __float2half_rn(v0);
-              op[o + d1] = __float2half_rn(v1);
+          for (int mt = 0; mt < MTILES; ++mt) {
+            const int d0 = d_of(mt, 0), d1 = d_of(mt, 1);
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+              const int h = hh ? h1 : h0;
+              if (h >= G) continue;
+              const float inv = hh ? inv1 : inv0;
+              const float v0 = acc[nb][mt][hh] * inv, v1 = acc[nb][mt][2 + hh] * inv;
+              const int64_t o = obase + static_cast<int64_t>(h) * D;
+              if (p.out_dtype == PA_F32) {
+                float* op = static_cast<float*>(p.out);
+                op[o + d0] = v0;
+                op[o + d1] = v1;
+              } else if (p.out_dtype == PA_BF16) {
+                __nv_bfloat16* op = static_cast<__nv_bfloat16*>(p.out);
+                op[o + d0] = __float2bfloat16_rn(v0);
+                op[o + d1] = __float2bfloat16_rn(v1);
+              } else {
+                __half* op = static_cast<__half*>(p.out);
+                op[o + d0] = __float2half_rn(v0);
+                op[o + d1] = __float2half_rn(v1);
+              }
             }
           }
-        }
-      } else if (ti.seg < p.nseg_cap) {
-        const int ncol = ti.members * G;
-        const int64_t prow = ((static_cast<int64_t>(hg) * p.nseg_cap + ti.seg) * HG + g) * p.cols;
-        float* po = p.part_o + prow * D;
+        } else if (ti.seg < p.nseg_cap) {
+          const int64_t prow =
+              ((static_cast<int64_t>(hg) * p.nseg_cap + ti.seg) * HG + g) * p.cols;
+          float* po = p.part_o + prow * D;
 #pragma unroll
-        for (int mt = 0; mt < MTILES; ++mt) {
-          const int d0 = d_of(mt, 0), d1 = d_of(mt, 1);
-          if (h0 < ncol) {
-            po[h0 * D + d0] = acc[mt][0] * inv0;
-            po[h0 * D + d1] = acc[mt][2] * inv0;
+          for (int mt = 0; mt < MTILES; ++mt) {
+            const int d0 = d_of(mt, 0), d1 = d_of(mt, 1);
+            if (h0 < ncol) {
+              po[h0 * D + d0] = acc[nb][mt][0] * inv0;
+              po[h0 * D + d1] = acc[nb][mt][2] * inv0;
+            }
+            if (h1 < ncol) {
+              po[h1 * D + d0] = acc[nb][mt][1] * inv1;
+              po[h1 * D + d1] = acc[nb][mt][3] * inv1;
+            }
           }
-          if (h1 < ncol) {
-            po[h1 * D + d0] = acc[mt][1] * inv1;
-            po[h1 * D + d1] = acc[mt][3] * inv1;
+          if (grp == 0) {
+            float* pm = p.part_ml + prow * 2;
+            if (h0 < ncol) {
+              pm[h0 * 2] = l0 > 0.f ? m_run[nb][0] : -INFINITY;
+              pm[h0 * 2 + 1] = l0;
+            }
+            if (h1 < ncol) {
+              pm[h1 * 2] = l1 > 0.f ? m_run[nb][1] : -INFINITY;
+              pm[h1 * 2 + 1] = l1;
+            }
           }
+        } else {
+          flag_error(p.err, PA_DEVERR_BAD_SEQLEN);
         }
-        if (grp == 0) {
-          float* pm = p.part_ml + prow * 2;
-          if (h0 < ncol) {
-            pm[h0 * 2] = l0 > 0.f ? m_run[0] : -INFINITY;
-            pm[h0 * 2 + 1] = l0;
-          }
-          if (h1 < ncol) {
-            pm[h1 * 2] = l1 > 0.f ? m_run[1] : -INFINITY;
-            pm[h1 * 2 + 1] = l1;
-          }
-        }
-      } else {
-        flag_error(p.err, PA_DEVERR_BAD_SEQLEN);
       }
     }
   }
@@ -1090,27 +1176,35 @@ namespace {
 
 using MainKernel = void (*)(const CUtensorMap, const CUtensorMap, const DecodeParams);
 
-template <int D, int HG, bool BF, bool F8>
+template <int D, int HG, int NB, int CG, bool BF, bool F8>
 MainKernel main_kernel_ptr() {
-  return pa_decode_main_kernel<D, HG, BF, F8>;
+  return pa_decode_main_kernel<D, HG, NB, CG, BF, F8>;
 }
 
-MainKernel select_main(int D, int HG, bool bf16, bool fp8) {
+// Built: every (head_dim, heads per CTA) with one 8-column block per head;
+// 16-bit caches also with 16 columns per warp (NB 2) and with two warps of
+// 16 columns per head (NB 2, CG 2, at most 4 heads per CTA).
+MainKernel select_main(int D, int HG, int NB, int CG, bool bf16, bool fp8) {
   if (fp8) {
-    if (D != 128) return nullptr;
+    if (D != 128 || NB != 1 || CG != 1) return nullptr;
     switch (HG) {
-      case 1: return main_kernel_ptr<128, 1, false, true>();
-      case 2: return main_kernel_ptr<128, 2, false, true>();
-      case 4: return main_kernel_ptr<128, 4, false, true>();
-      case 8: return main_kernel_ptr<128, 8, false, true>();
+      case 1: return main_kernel_ptr<128, 1, 1, 1, false, true>();
+      case 2: return main_kernel_ptr<128, 2, 1, 1, false, true>();
+      case 4: return main_kernel_ptr<128, 4, 1, 1, false, true>();
+      case 8: return main_kernel_ptr<128, 8, 1, 1, false, true>();
       default: return nullptr;
     }
   }
-#define PA_SEL(d, hg)                                                             \
-  if (D == d && HG == hg) return bf16 ? main_kernel_ptr<d, hg, true, false>()     \
-                                      : main_kernel_ptr<d, hg, false, false>();
-  PA_SEL(64, 1) PA_SEL(64, 2) PA_SEL(64, 4) PA_SEL(64, 8)
-  PA_SEL(128, 1) PA_SEL(128, 2) PA_SEL(128, 4) PA_SEL(128, 8)
+#define PA_SEL(d, hg, nb, cg)                                                         \
+  if (D == d && HG == hg && NB == nb && CG == cg)                                     \
+    return bf16 ? main_kernel_ptr<d, hg, nb, cg, true, false>()                       \
+                : main_kernel_ptr<d, hg, nb, cg, false, false>();
+  PA_SEL(64, 1, 1, 1) PA_SEL(64, 2, 1, 1) PA_SEL(64, 4, 1, 1) PA_SEL(64, 8, 1, 1)
+  PA_SEL(128, 1, 1, 1) PA_SEL(128, 2, 1, 1) PA_SEL(128, 4, 1, 1) PA_SEL(128, 8, 1, 1)
+  PA_SEL(64, 1, 2, 1) PA_SEL(64, 2, 2, 1) PA_SEL(64, 4, 2, 1) PA_SEL(64, 8, 2, 1)
+  PA_SEL(128, 1, 2, 1) PA_SEL(128, 2, 2, 1) PA_SEL(128, 4, 2, 1) PA_SEL(128, 8, 2, 1)
+  PA_SEL(64, 1, 2, 2) PA_SEL(64, 2, 2, 2) PA_SEL(64, 4, 2, 2)
+  PA_SEL(128, 1, 2, 2) PA_SEL(128, 2, 2, 2) PA_SEL(128, 4, 2, 2)
 #undef PA_SEL
   return nullptr;
 }
@@ -1118,12 +1212,12 @@ MainKernel select_main(int D, int HG, bool bf16, bool fp8) {
 struct LaunchPlan {
   int HG = 0, groups = 0, stages = 0, tok_box = 0, threads = 0;
   int ctas_per_group = 0, tiles_per_part = INT_MAX, nseg_cap = 0;
-  int pack_size = 1, cols = 0;
+  int pack_size = 1, cols = 0, nb = 1, cg = 1;
   bool many_partials = false;  // long sequences / partitions: closed-form plan, wide combine
   size_t smem = 0;
   size_t off_tiles = 0, off_segs = 0, off_start = 0, off_firstk = 0, off_meta = 0,
-         off_pack_first = 0, off_pack_tiles = 0, off_seq_pack = 0, off_seq_pre = 0, off_o = 0,
-         off_ml = 0, total = 0;
+         off_pack_first = 0, off_pack_n = 0, off_pack_tiles = 0, off_seq_pack = 0,
+         off_seq_pre = 0, off_o = 0, off_ml = 0, total = 0;
   MainKernel kernel = nullptr;
 };
 
@@ -1132,7 +1226,10 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
 
 // shared_prefix: consecutive sequences may be packed over shared leading
-// blocks (8 / group sequences per pack); otherwise every sequence is its own entry.
+// blocks, min(8, 32 / group) sequences per pack, whose group-many query heads
+// each take a column: 16 columns per consumer warp, two warps per KV head when
+// more than 16 are needed.  Otherwise every sequence is its own entry and a
+// warp holds one KV head's group columns.
 pa_status make_plan(int32_t num_seqs, int32_t Hq, int32_t Hkv, int32_t D, int32_t bs,
                     int32_t max_seq_len, int32_t partition_size, bool bf16, bool fp8,
                     bool shared_prefix, LaunchPlan* lp) {
@@ -1146,7 +1243,15 @@ pa_status make_plan(int32_t num_seqs, int32_t Hq, int32_t Hkv, int32_t D, int32_
   if (G > 8) return PA_ERR_UNSUPPORTED;
   if (partition_size > 0 && (partition_size % kTile != 0 || partition_size % bs != 0))
     return PA_ERR_INVALID_ARG;
-  int HG = 8;
+  int P = 1, NB = 1, CG = 1;
+  if (shared_prefix && !fp8) {
+    P = kMaxPackCols / G < kMaxPack ? kMaxPackCols / G : kMaxPack;
+    if (P < 2) P = 1;
+    const int need = P * G;  // columns of a whole pack
+    NB = need > 8 ? 2 : 1;
+    CG = (need + 8 * NB - 1) / (8 * NB);
+  }
+  int HG = 8 / CG;
   while (Hkv % HG != 0) HG >>= 1;
   if (fp8 && D != 128) return PA_ERR_UNSUPPORTED;
   const int DCT = fp8 ? 1 : D / 64;  // 128-byte rows per (token, head) in a stage
@@ -1155,7 +1260,9 @@ pa_status make_plan(int32_t num_seqs, int32_t Hq, int32_t Hkv, int32_t D, int32_
   lp->HG = HG;
   lp->groups = Hkv / HG;
   lp->tok_box = TB;
-  lp->threads = (HG + 1) * 32;
+  lp->threads = (HG * CG + 1) * 32;
+  lp->nb = NB;
+  lp->cg = CG;
   const size_t tile_bytes = static_cast<size_t>(kTile) * HG * D * (fp8 ? 1 : 2);
   const size_t budget = 200 * 1024;
   int stages = static_cast<int>(budget / (2 * tile_bytes));
@@ -1164,7 +1271,7 @@ pa_status make_plan(int32_t num_seqs, int32_t Hq, int32_t Hkv, int32_t D, int32_
   lp->stages = stages;
   lp->smem = 1024 + static_cast<size_t>(stages) * 2 * tile_bytes + stages * sizeof(TileInfo) +
              3 * stages * sizeof(uint64_t);
-  lp->kernel = select_main(D, HG, bf16, fp8);
+  lp->kernel = select_main(D, HG, NB, CG, bf16, fp8);
   if (lp->kernel == nullptr) return PA_ERR_UNSUPPORTED;
 
   const DeviceInfo* dev = current_device_info();
@@ -1183,10 +1290,10 @@ pa_status make_plan(int32_t num_seqs, int32_t Hq, int32_t Hkv, int32_t D, int32_
     parts_per_seq = (max_tiles + lp->tiles_per_part - 1) / lp->tiles_per_part;
     if (parts_per_seq < 1) parts_per_seq = 1;
   }
-  lp->pack_size = (shared_prefix && kMaxCols / G >= 2) ? kMaxCols / G : 1;
-  lp->cols = lp->pack_size * G;
-  // entries: at most num_seqs / pack_size packs, then the sequences
-  const int64_t max_packs = lp->pack_size > 1 ? num_seqs / lp->pack_size : 0;
+  lp->pack_size = P;
+  lp->cols = P > 1 ? 8 * NB * CG : G;
+  // entries: at most num_seqs / 2 packs (pairs), then the sequences
+  const int64_t max_packs = P > 1 ? num_seqs / 2 : 0;
   const int64_t entries = static_cast<int64_t>(num_seqs) + max_packs;
   const int64_t nseg = entries * parts_per_seq + lp->ctas_per_group;
   // partials one sequence expects: its partitions plus the CTA shares it spans
@@ -1205,7 +1312,8 @@ pa_status make_plan(int32_t num_seqs, int32_t Hq, int32_t Hkv, int32_t D, int32_
   size_t off = lp->off_meta + words(1);
   if (lp->pack_size > 1) {
     lp->off_pack_first = off;
-    lp->off_pack_tiles = lp->off_pack_first + words(max_packs + 1);
+    lp->off_pack_n = lp->off_pack_first + words(max_packs + 1);
+    lp->off_pack_tiles = lp->off_pack_n + words(max_packs + 1);
     lp->off_seq_pack = lp->off_pack_tiles + words(max_packs + 1);
     lp->off_seq_pre = lp->off_seq_pack + words(num_seqs);
     off = lp->off_seq_pre + words(num_seqs);
@@ -1363,6 +1471,7 @@ pa_status launch_decode(void* out, pa_dtype out_dtype, const void* query, pa_dty
   p.cols = lp.cols;
   if (lp.pack_size > 1) {
     p.pack_first = reinterpret_cast<int32_t*>(ws + lp.off_pack_first);
+    p.pack_n = reinterpret_cast<int32_t*>(ws + lp.off_pack_n);
     p.pack_tiles = reinterpret_cast<int32_t*>(ws + lp.off_pack_tiles);
     p.seq_pack = reinterpret_cast<int32_t*>(ws + lp.off_seq_pack);
     p.seq_pre = reinterpret_cast<int32_t*>(ws + lp.off_seq_pre);

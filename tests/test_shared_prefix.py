@@ -140,14 +140,18 @@ def test_short_prompt_is_not_packed(pa, orc):
            expect_packs=False)
 
 
-def test_no_sharing_is_bitwise_the_plain_path(pa, orc):
-    """shared_blocks all 0: no packs, the same tiles and partials as
-    decode_attention, so the same bits."""
+def test_no_sharing_matches_the_plain_path(pa, orc):
+    """shared_blocks all 0: no packs, every sequence attended alone.  The
+    entry point runs its own launch shape (fewer heads per CTA, wider warps),
+    so the partials are cut elsewhere: equal to the plain path and the oracle
+    within the fp32 bound, not bit for bit."""
     prep = prepare(_spec(prompt_len=600, extra_hi=50))
     k, v, sb = _inputs(prep)
-    out_a = _run_shared(pa, prep, k, v, np.zeros_like(sb))
-    out_b = _run_plain(pa, prep, k, v)
-    assert torch.equal(out_a.view(torch.int16), out_b.view(torch.int16))
+    ref = _ref(orc, prep, k, v)
+    a = as_f64(_run_shared(pa, prep, k, v, np.zeros_like(sb), out_dtype=torch.float32))
+    b = as_f64(_run_plain(pa, prep, k, v, out_dtype=torch.float32))
+    assert float(np.max(np.abs(a - ref))) <= TOL_F32
+    assert float(np.max(np.abs(a - b))) <= 2 * TOL_F32
 
 
 def test_packed_matches_plain_path(pa, orc):
