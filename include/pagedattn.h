@@ -65,6 +65,28 @@ typedef enum { PA_F16 = 0, PA_BF16 = 1, PA_F32 = 2 } pa_dtype;
  *                   code * scale (per-tensor scales k_scale, v_scale). */
 typedef enum { PA_KV_AUTO = 0, PA_KV_FP8_E4M3 = 1 } pa_kv_cache_dtype;
 
+/* Element strides of a KV pool whose head_dim elements are contiguous: element
+ * (block, token, head, d) sits at
+ *     base + block * block_stride + token * token_stride + head * head_stride + d
+ * (in elements of the pool's type).  The *_strided entry points take one for
+ * the K and V pools alike; the others assume the contiguous layout
+ *     {block_size * num_kv_heads * head_dim, num_kv_heads * head_dim, head_dim}.
+ * Examples ([vLLM] "Code Example" / "split_kv_cache": views of one tensor
+ * without copies):
+ *   - K and V halves of a combined (2, num_blocks, bs, Hkv, D) tensor: the
+ *     contiguous strides;
+ *   - K and V halves of a per-block interleaved (num_blocks, 2, bs, Hkv, D)
+ *     tensor: {2 * bs * Hkv * D, Hkv * D, D};
+ *   - a head-major (num_blocks, Hkv, bs, D) pool: {Hkv * bs * D, D, bs * D}.
+ * Rows of different (block, token, head) must not overlap.  The decode kernels
+ * load tiles with TMA: there every stride times the element size must be a
+ * multiple of 16 bytes. */
+typedef struct pa_cache_strides {
+  int64_t block_stride;
+  int64_t token_stride;
+  int64_t head_stride;
+} pa_cache_strides;
+
 #define PA_DEVERR_BAD_BLOCK 0x1   /* block-table entry outside [0, num_blocks) */
 #define PA_DEVERR_BAD_SLOT 0x2    /* slot / block id outside the pool          */
 #define PA_DEVERR_BAD_SEQLEN 0x4  /* seq_len < 0 or > max_seq_len              */
@@ -115,6 +137,24 @@ pa_status pa_reshape_and_cache(const void* key, const void* value,
                                int32_t* device_error_flag, pa_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * pa_reshape_and_cache_strided -- pa_reshape_and_cache into pools of any
+ * layout described by *cache_strides (host pointer; see pa_cache_strides).
+ * Same arguments, meaning and errors otherwise; also PA_ERR_INVALID_ARG for a
+ * null or non-positive stride, and under PA_KV_FP8_E4M3 for strides or
+ * head_dim that are not multiples of 8.
+ * ------------------------------------------------------------------------- */
+pa_status pa_reshape_and_cache_strided(const void* key, const void* value,
+                                       int64_t key_stride_t, int64_t value_stride_t,
+                                       void* key_cache, void* value_cache,
+                                       const pa_cache_strides* cache_strides,
+                                       const int32_t* slot_mapping, int32_t num_tokens,
+                                       int32_t num_blocks, int32_t block_size,
+                                       int32_t num_kv_heads, int32_t head_dim,
+                                       pa_dtype dtype, pa_kv_cache_dtype kv_cache_dtype,
+                                       const float* k_scale, const float* v_scale,
+                                       int32_t* device_error_flag, pa_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * pa_copy_blocks -- copy-on-write, [PA] "Sharing and copy-on-write" and "How
  * does copy-on-write work for parallel sampling?" ([KV] "Shared prompts and
  * continuous batching").
@@ -137,6 +177,21 @@ pa_status pa_copy_blocks(void* const* key_caches, void* const* value_caches,
                          int32_t num_pairs, int32_t num_blocks,
                          int64_t block_bytes, int32_t* device_error_flag,
                          pa_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * pa_copy_blocks_strided -- pa_copy_blocks for pools laid out by
+ * *cache_strides (host pointer; every pool listed shares it): block dst gets
+ * the block_size x num_kv_heads rows of head_dim elements of block src
+ * (elem_bytes 2 for 16-bit pools, 1 for E4M3 codes).  Bytes between rows are
+ * not touched.  PA_ERR_INVALID_ARG also when a row or a stride is not a
+ * multiple of 16 bytes or a pool pointer is not 16-byte aligned.
+ * ------------------------------------------------------------------------- */
+pa_status pa_copy_blocks_strided(void* const* key_caches, void* const* value_caches,
+                                 int32_t num_layers, const pa_cache_strides* cache_strides,
+                                 const int32_t* block_mapping, int32_t num_pairs,
+                                 int32_t num_blocks, int32_t block_size,
+                                 int32_t num_kv_heads, int32_t head_dim, int32_t elem_bytes,
+                                 int32_t* device_error_flag, pa_stream_t stream);
 
 /* ---------------------------------------------------------------------------
  * pa_decode_workspace_bytes -- device scratch that pa_decode_attention needs
@@ -220,6 +275,32 @@ pa_status pa_decode_attention_fp8(void* out, pa_dtype out_dtype, const void* que
                                   int32_t partition_size, void* workspace,
                                   size_t workspace_bytes, int32_t* device_error_flag,
                                   pa_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * pa_decode_attention_strided -- pa_decode_attention / pa_decode_attention_fp8
+ * over pools of any layout described by *cache_strides (host pointer; see
+ * pa_cache_strides), for example the K and V halves of one interleaved
+ * tensor, with no copy.  kv_cache_dtype PA_KV_AUTO: the pools hold
+ * query_dtype and k_scale / v_scale are ignored; PA_KV_FP8_E4M3: the pools
+ * hold E4M3 codes read as code * (*k_scale), code * (*v_scale) (device
+ * pointers), head_dim 128.  Workspace: pa_decode_workspace_bytes.  Other
+ * arguments and errors are those of pa_decode_attention; also
+ * PA_ERR_INVALID_ARG for a null or non-positive stride or one whose byte
+ * size is not a multiple of 16.
+ * ------------------------------------------------------------------------- */
+pa_status pa_decode_attention_strided(void* out, pa_dtype out_dtype, const void* query,
+                                      pa_dtype query_dtype, const void* key_cache,
+                                      const void* value_cache,
+                                      const pa_cache_strides* cache_strides,
+                                      pa_kv_cache_dtype kv_cache_dtype, const float* k_scale,
+                                      const float* v_scale, const int32_t* block_tables,
+                                      int32_t block_table_stride, const int32_t* seq_lens,
+                                      int32_t num_seqs, int32_t max_seq_len,
+                                      int32_t num_q_heads, int32_t num_kv_heads,
+                                      int32_t head_dim, int32_t num_blocks,
+                                      int32_t block_size, float scale, int32_t partition_size,
+                                      void* workspace, size_t workspace_bytes,
+                                      int32_t* device_error_flag, pa_stream_t stream);
 
 /* ---------------------------------------------------------------------------
  * pa_decode_shared_prefix_workspace_bytes -- device scratch for

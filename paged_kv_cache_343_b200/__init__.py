@@ -40,7 +40,7 @@ __all__ = [
     "decode_workspace_bytes", "decode_attention_fp8", "decode_attention_noalloc",
     "decode_attention_shared_prefix", "shared_prefix_workspace_bytes", "BlockManager",
     "PagedDecodeStep", "DEVERR_BAD_BLOCK", "DEVERR_BAD_SLOT", "DEVERR_BAD_SEQLEN",
-    "DEVERR_TIMEOUT", "DEVERR_BAD_SHARE", "version",
+    "DEVERR_TIMEOUT", "DEVERR_BAD_SHARE", "CacheStrides", "version",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpagedattn.so")
@@ -64,6 +64,22 @@ class PagedAttnError(RuntimeError):
         self.name = name
 
 
+class CacheStrides(ctypes.Structure):
+    """pa_cache_strides: element strides of a pool whose head_dim is contiguous."""
+    _fields_ = [("block_stride", ctypes.c_int64), ("token_stride", ctypes.c_int64),
+                ("head_stride", ctypes.c_int64)]
+
+
+def _pool_strides(cache: torch.Tensor) -> Optional[CacheStrides]:
+    """None for a contiguous [nb, bs, Hkv, D] pool, else its strides (head_dim
+    must be contiguous)."""
+    _need(cache.dim() == 4 and cache.stride(3) == 1, "pools are [nb, bs, Hkv, D] views "
+          "with head_dim contiguous")
+    if cache.is_contiguous():
+        return None
+    return CacheStrides(cache.stride(0), cache.stride(1), cache.stride(2))
+
+
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError("libpagedattn.so is missing at %s; build it with "
@@ -79,6 +95,18 @@ def _load() -> ctypes.CDLL:
                                          ctypes.c_int, ctypes.c_int, p, p, p, p]
     lib.pa_copy_blocks.restype = ctypes.c_int
     lib.pa_copy_blocks.argtypes = [p, p, i32, p, i32, i32, i64, p, p]
+    lib.pa_reshape_and_cache_strided.restype = ctypes.c_int
+    lib.pa_reshape_and_cache_strided.argtypes = [p, p, i64, i64, p, p, ctypes.POINTER(CacheStrides),
+                                                 p, i32, i32, i32, i32, i32, ctypes.c_int,
+                                                 ctypes.c_int, p, p, p, p]
+    lib.pa_copy_blocks_strided.restype = ctypes.c_int
+    lib.pa_copy_blocks_strided.argtypes = [p, p, i32, ctypes.POINTER(CacheStrides), p, i32, i32,
+                                           i32, i32, i32, i32, p, p]
+    lib.pa_decode_attention_strided.restype = ctypes.c_int
+    lib.pa_decode_attention_strided.argtypes = [p, ctypes.c_int, p, ctypes.c_int, p, p,
+                                                ctypes.POINTER(CacheStrides), ctypes.c_int, p, p,
+                                                p, i32, p, i32, i32, i32, i32, i32, i32, i32,
+                                                ctypes.c_float, i32, p, sz, p, p]
     lib.pa_decode_workspace_bytes.restype = ctypes.c_int
     lib.pa_decode_workspace_bytes.argtypes = [i32, i32, i32, i32, i32, i32, i32,
                                               ctypes.POINTER(sz)]
@@ -172,7 +200,9 @@ def reshape_and_cache(key: torch.Tensor, value: torch.Tensor, key_cache: torch.T
     _need(key.stride(2) == 1 and key.stride(1) == key.shape[2] and
           value.stride(2) == 1 and value.stride(1) == value.shape[2],
           "heads and head_dim must be contiguous inside a row")
-    _need(key_cache.is_contiguous() and value_cache.is_contiguous(), "caches must be contiguous")
+    _need(key_cache.shape == value_cache.shape and key_cache.stride() == value_cache.stride(),
+          "K and V pools share shape and strides")
+    strides = _pool_strides(key_cache)
     _need(slot_mapping.dtype == torch.int32 and slot_mapping.is_contiguous(), "slot_mapping int32")
     if fp8:
         _need(key.dtype == value.dtype and key_cache.dtype == value_cache.dtype == torch.uint8,
@@ -182,11 +212,19 @@ def reshape_and_cache(key: torch.Tensor, value: torch.Tensor, key_cache: torch.T
     else:
         _need(key.dtype == key_cache.dtype == value.dtype == value_cache.dtype, "dtype mismatch")
     nb, bs, hkv, d = key_cache.shape
-    _check(lib.pa_reshape_and_cache(
-        _ptr(key), _ptr(value), key.stride(0), value.stride(0), _ptr(key_cache),
-        _ptr(value_cache), _ptr(slot_mapping), key.shape[0], nb, bs, hkv, d,
-        _DTYPE_CODE[key.dtype], _KV_CACHE_DTYPE[kv_cache_dtype], _ptr(k_scale), _ptr(v_scale),
-        _ptr(error_flag), _stream_handle(stream)), "pa_reshape_and_cache")
+    if strides is None:
+        _check(lib.pa_reshape_and_cache(
+            _ptr(key), _ptr(value), key.stride(0), value.stride(0), _ptr(key_cache),
+            _ptr(value_cache), _ptr(slot_mapping), key.shape[0], nb, bs, hkv, d,
+            _DTYPE_CODE[key.dtype], _KV_CACHE_DTYPE[kv_cache_dtype], _ptr(k_scale),
+            _ptr(v_scale), _ptr(error_flag), _stream_handle(stream)), "pa_reshape_and_cache")
+    else:
+        _check(lib.pa_reshape_and_cache_strided(
+            _ptr(key), _ptr(value), key.stride(0), value.stride(0), _ptr(key_cache),
+            _ptr(value_cache), ctypes.byref(strides), _ptr(slot_mapping), key.shape[0], nb, bs,
+            hkv, d, _DTYPE_CODE[key.dtype], _KV_CACHE_DTYPE[kv_cache_dtype], _ptr(k_scale),
+            _ptr(v_scale), _ptr(error_flag), _stream_handle(stream)),
+            "pa_reshape_and_cache_strided")
 
 
 def copy_blocks(key_caches: Sequence[torch.Tensor], value_caches: Sequence[torch.Tensor],
@@ -198,14 +236,23 @@ def copy_blocks(key_caches: Sequence[torch.Tensor], value_caches: Sequence[torch
     k0 = key_caches[0]
     block_bytes = k0[0].numel() * k0.element_size()
     for c in list(key_caches) + list(value_caches):
-        _need(c.is_contiguous() and c.shape == k0.shape and c.dtype == k0.dtype, "pool shapes differ")
+        _need(c.shape == k0.shape and c.dtype == k0.dtype and c.stride() == k0.stride(),
+              "pool shapes, types and strides differ")
+    strides = _pool_strides(k0)
     n = len(key_caches)
     karr = (ctypes.c_void_p * n)(*[c.data_ptr() for c in key_caches])
     varr = (ctypes.c_void_p * n)(*[c.data_ptr() for c in value_caches])
-    _check(lib.pa_copy_blocks(ctypes.cast(karr, ctypes.c_void_p), ctypes.cast(varr, ctypes.c_void_p),
-                              n, _ptr(block_mapping), block_mapping.numel() // 2, k0.shape[0],
-                              block_bytes, _ptr(error_flag), _stream_handle(stream)),
-           "pa_copy_blocks")
+    kp, vp = ctypes.cast(karr, ctypes.c_void_p), ctypes.cast(varr, ctypes.c_void_p)
+    if strides is None:
+        _check(lib.pa_copy_blocks(kp, vp, n, _ptr(block_mapping), block_mapping.numel() // 2,
+                                  k0.shape[0], block_bytes, _ptr(error_flag),
+                                  _stream_handle(stream)), "pa_copy_blocks")
+    else:
+        nb, bs, hkv, d = k0.shape
+        _check(lib.pa_copy_blocks_strided(kp, vp, n, ctypes.byref(strides), _ptr(block_mapping),
+                                          block_mapping.numel() // 2, nb, bs, hkv, d,
+                                          k0.element_size(), _ptr(error_flag),
+                                          _stream_handle(stream)), "pa_copy_blocks_strided")
 
 
 def decode_workspace_bytes(num_seqs: int, num_q_heads: int, num_kv_heads: int, head_dim: int,
@@ -238,11 +285,14 @@ def decode_attention(out: torch.Tensor, query: torch.Tensor, key_cache: torch.Te
                      partition_size: int = 0, workspace: Optional[torch.Tensor] = None,
                      error_flag: Optional[torch.Tensor] = None,
                      stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
-    """out/query [B, Hq, D]; caches [nb, bs, Hkv, D]; block_tables int32 [B, W]; seq_lens int32 [B]."""
+    """out/query [B, Hq, D]; caches [nb, bs, Hkv, D] (any strided view with head_dim
+    contiguous, e.g. the K and V halves of one interleaved tensor); block_tables
+    int32 [B, W]; seq_lens int32 [B]."""
     _need(query.dim() == 3 and query.is_contiguous(), "query must be contiguous [B, Hq, D]")
     _need(out.shape == query.shape and out.is_contiguous(), "out must be contiguous [B, Hq, D]")
-    _need(key_cache.is_contiguous() and value_cache.is_contiguous(), "caches must be contiguous")
-    _need(key_cache.shape == value_cache.shape, "K and V pools differ")
+    _need(key_cache.shape == value_cache.shape and key_cache.stride() == value_cache.stride(),
+          "K and V pools share shape and strides")
+    strides = _pool_strides(key_cache)
     _need(block_tables.dtype == torch.int32 and block_tables.dim() == 2 and
           block_tables.stride(1) == 1, "block_tables int32 [B, W], rows contiguous")
     _need(seq_lens.dtype == torch.int32 and seq_lens.is_contiguous(), "seq_lens int32")
@@ -252,12 +302,21 @@ def decode_attention(out: torch.Tensor, query: torch.Tensor, key_cache: torch.Te
     if workspace is None:
         workspace = alloc_workspace(decode_workspace_bytes(B, hq, hkv, d, bs, max_seq_len,
                                                            partition_size), query.device)
-    _check(lib.pa_decode_attention(
-        _ptr(out), _DTYPE_CODE[out.dtype], _ptr(query), _ptr(key_cache), _ptr(value_cache),
-        _ptr(block_tables), block_tables.stride(0), _ptr(seq_lens), B, int(max_seq_len), hq, hkv,
-        d, nb, bs, float(scale), _DTYPE_CODE[query.dtype], int(partition_size), _ptr(workspace),
-        workspace.numel() * workspace.element_size(), _ptr(error_flag), _stream_handle(stream)),
-        "pa_decode_attention")
+    wsb = workspace.numel() * workspace.element_size()
+    if strides is None:
+        _check(lib.pa_decode_attention(
+            _ptr(out), _DTYPE_CODE[out.dtype], _ptr(query), _ptr(key_cache), _ptr(value_cache),
+            _ptr(block_tables), block_tables.stride(0), _ptr(seq_lens), B, int(max_seq_len), hq,
+            hkv, d, nb, bs, float(scale), _DTYPE_CODE[query.dtype], int(partition_size),
+            _ptr(workspace), wsb, _ptr(error_flag), _stream_handle(stream)),
+            "pa_decode_attention")
+    else:
+        _check(lib.pa_decode_attention_strided(
+            _ptr(out), _DTYPE_CODE[out.dtype], _ptr(query), _DTYPE_CODE[query.dtype],
+            _ptr(key_cache), _ptr(value_cache), ctypes.byref(strides), 0, None, None,
+            _ptr(block_tables), block_tables.stride(0), _ptr(seq_lens), B, int(max_seq_len), hq,
+            hkv, d, nb, bs, float(scale), int(partition_size), _ptr(workspace), wsb,
+            _ptr(error_flag), _stream_handle(stream)), "pa_decode_attention_strided")
     return out
 
 
@@ -273,8 +332,9 @@ def decode_attention_fp8(out: torch.Tensor, query: torch.Tensor, key_cache: torc
     _need(query.dim() == 3 and query.is_contiguous(), "query must be contiguous [B, Hq, D]")
     _need(out.shape == query.shape and out.is_contiguous(), "out must be contiguous [B, Hq, D]")
     _need(key_cache.dtype == value_cache.dtype == torch.uint8, "fp8 pools are uint8 codes")
-    _need(key_cache.is_contiguous() and value_cache.is_contiguous(), "caches must be contiguous")
-    _need(key_cache.shape == value_cache.shape, "K and V pools differ")
+    _need(key_cache.shape == value_cache.shape and key_cache.stride() == value_cache.stride(),
+          "K and V pools share shape and strides")
+    strides = _pool_strides(key_cache)
     _need(k_scale.dtype == torch.float32 and v_scale.dtype == torch.float32, "float32 scales")
     _need(block_tables.dtype == torch.int32 and block_tables.dim() == 2 and
           block_tables.stride(1) == 1, "block_tables int32 [B, W], rows contiguous")
@@ -284,13 +344,22 @@ def decode_attention_fp8(out: torch.Tensor, query: torch.Tensor, key_cache: torc
     if workspace is None:
         workspace = alloc_workspace(decode_workspace_bytes(B, hq, hkv, d, bs, max_seq_len,
                                                            partition_size), query.device)
-    _check(lib.pa_decode_attention_fp8(
-        _ptr(out), _DTYPE_CODE[out.dtype], _ptr(query), _DTYPE_CODE[query.dtype],
-        _ptr(key_cache), _ptr(value_cache), _ptr(k_scale), _ptr(v_scale), _ptr(block_tables),
-        block_tables.stride(0), _ptr(seq_lens), B, int(max_seq_len), hq, hkv, d, nb, bs,
-        float(scale), int(partition_size), _ptr(workspace),
-        workspace.numel() * workspace.element_size(), _ptr(error_flag), _stream_handle(stream)),
-        "pa_decode_attention_fp8")
+    wsb = workspace.numel() * workspace.element_size()
+    if strides is None:
+        _check(lib.pa_decode_attention_fp8(
+            _ptr(out), _DTYPE_CODE[out.dtype], _ptr(query), _DTYPE_CODE[query.dtype],
+            _ptr(key_cache), _ptr(value_cache), _ptr(k_scale), _ptr(v_scale), _ptr(block_tables),
+            block_tables.stride(0), _ptr(seq_lens), B, int(max_seq_len), hq, hkv, d, nb, bs,
+            float(scale), int(partition_size), _ptr(workspace), wsb, _ptr(error_flag),
+            _stream_handle(stream)), "pa_decode_attention_fp8")
+    else:
+        _check(lib.pa_decode_attention_strided(
+            _ptr(out), _DTYPE_CODE[out.dtype], _ptr(query), _DTYPE_CODE[query.dtype],
+            _ptr(key_cache), _ptr(value_cache), ctypes.byref(strides), 1, _ptr(k_scale),
+            _ptr(v_scale), _ptr(block_tables), block_tables.stride(0), _ptr(seq_lens), B,
+            int(max_seq_len), hq, hkv, d, nb, bs, float(scale), int(partition_size),
+            _ptr(workspace), wsb, _ptr(error_flag), _stream_handle(stream)),
+            "pa_decode_attention_strided")
     return out
 
 

@@ -1382,7 +1382,8 @@ pa_status launch_decode(void* out, pa_dtype out_dtype, const void* query, pa_dty
                         int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
                         int32_t num_blocks, int32_t block_size, float scale,
                         int32_t partition_size, const int32_t* shared_blocks, void* workspace,
-                        size_t workspace_bytes, int32_t* device_error_flag, pa_stream_t stream) {
+                        size_t workspace_bytes, int32_t* device_error_flag, pa_stream_t stream,
+                        const pa_cache_strides* cache_strides = nullptr) {
   if (num_seqs < 0) return PA_ERR_INVALID_ARG;
   if (num_seqs == 0) return PA_OK;
   if (!out || !query || !key_cache || !value_cache || !block_tables || !seq_lens || !workspace)
@@ -1410,6 +1411,18 @@ pa_status launch_decode(void* out, pa_dtype out_dtype, const void* query, pa_dty
 
   const int HG = lp.HG, D = head_dim;
   const uint64_t e = static_cast<uint64_t>(elem_bytes);
+  // pool strides in bytes (token, head, block); head_dim elements contiguous
+  uint64_t tok_b = static_cast<uint64_t>(num_kv_heads) * D * e, head_b = D * e,
+           blk_b = static_cast<uint64_t>(block_size) * num_kv_heads * D * e;
+  if (cache_strides != nullptr) {
+    if (cache_strides->block_stride <= 0 || cache_strides->token_stride <= 0 ||
+        cache_strides->head_stride <= 0)
+      return PA_ERR_INVALID_ARG;
+    tok_b = static_cast<uint64_t>(cache_strides->token_stride) * e;
+    head_b = static_cast<uint64_t>(cache_strides->head_stride) * e;
+    blk_b = static_cast<uint64_t>(cache_strides->block_stride) * e;
+    if (tok_b % 16 != 0 || head_b % 16 != 0 || blk_b % 16 != 0) return PA_ERR_INVALID_ARG;
+  }
   const int DCT = fp8 ? 1 : D / 64;           // 128-byte rows per (token, head)
   const uint32_t inner = fp8 ? 128u : 64u;    // elements in one 128-byte row
   CUtensorMap tmK, tmV;
@@ -1418,12 +1431,12 @@ pa_status launch_decode(void* out, pa_dtype out_dtype, const void* query, pa_dty
     // mode 0: dims {row, tokens, d-chunks, heads, blocks}, box {row, TB, DCT, HG, 1}
     const uint64_t dims0[5] = {inner, (uint64_t)block_size, (uint64_t)DCT,
                                (uint64_t)num_kv_heads, (uint64_t)num_blocks};
-    const uint64_t str0[4] = {num_kv_heads * D * e, 128, D * e, block_size * num_kv_heads * D * e};
+    const uint64_t str0[4] = {tok_b, 128, head_b, blk_b};
     const uint32_t box0[5] = {inner, (uint32_t)lp.tok_box, (uint32_t)DCT, (uint32_t)HG, 1};
     // mode 1: dims {row, d-chunks, heads, tokens, blocks}, box {row, 1, 1, TB, 1}
     const uint64_t dims1[5] = {inner, (uint64_t)DCT, (uint64_t)num_kv_heads,
                                (uint64_t)block_size, (uint64_t)num_blocks};
-    const uint64_t str1[4] = {128, D * e, num_kv_heads * D * e, block_size * num_kv_heads * D * e};
+    const uint64_t str1[4] = {128, head_b, tok_b, blk_b};
     const uint32_t box1[5] = {inner, 1, 1, (uint32_t)lp.tok_box, 1};
     if (get_tensor_map(&tmK, key_cache, dims0, str0, box0, elem_bytes) &&
         get_tensor_map(&tmV, value_cache, dims0, str0, box0, elem_bytes)) {
@@ -1534,6 +1547,26 @@ extern "C" pa_status pa_decode_attention_fp8(
                        max_seq_len, num_q_heads, num_kv_heads, head_dim, num_blocks, block_size,
                        scale, partition_size, nullptr, workspace, workspace_bytes,
                        device_error_flag, stream);
+}
+
+extern "C" pa_status pa_decode_attention_strided(
+    void* out, pa_dtype out_dtype, const void* query, pa_dtype query_dtype,
+    const void* key_cache, const void* value_cache, const pa_cache_strides* cache_strides,
+    pa_kv_cache_dtype kv_cache_dtype, const float* k_scale, const float* v_scale,
+    const int32_t* block_tables, int32_t block_table_stride, const int32_t* seq_lens,
+    int32_t num_seqs, int32_t max_seq_len, int32_t num_q_heads, int32_t num_kv_heads,
+    int32_t head_dim, int32_t num_blocks, int32_t block_size, float scale,
+    int32_t partition_size, void* workspace, size_t workspace_bytes,
+    int32_t* device_error_flag, pa_stream_t stream) {
+  if (cache_strides == nullptr) return PA_ERR_INVALID_ARG;
+  if (kv_cache_dtype != PA_KV_AUTO && kv_cache_dtype != PA_KV_FP8_E4M3) return PA_ERR_UNSUPPORTED;
+  const bool fp8 = kv_cache_dtype == PA_KV_FP8_E4M3;
+  return launch_decode(out, out_dtype, query, query_dtype, key_cache, value_cache, fp8 ? 1 : 2,
+                       fp8 ? k_scale : nullptr, fp8 ? v_scale : nullptr, block_tables,
+                       block_table_stride, seq_lens, num_seqs, max_seq_len, num_q_heads,
+                       num_kv_heads, head_dim, num_blocks, block_size, scale, partition_size,
+                       nullptr, workspace, workspace_bytes, device_error_flag, stream,
+                       cache_strides);
 }
 
 extern "C" pa_status pa_decode_attention_shared_prefix(

@@ -164,3 +164,18 @@ def pools_after_appends(prep: "Prepared"):
         oracle.copy_blocks([k, v], prep.cow_pairs, int(np.prod(k.shape[1:])) * 2)
         oracle.reshape_and_cache(prep.case.new_k, prep.case.new_v, k, v, prep.new_slots)
     return k, v
+
+
+def fp8_case(seed, B=6, lo=200, hi=1300, q_dtype="bf16", bs=16, hq=32, hkv=8, ks=0.05, vs=0.04):
+    spec = W.Spec("fp8", B, hq, hkv, 128, bs, q_dtype, seed=seed, len_dist="uniform",
+                  len_lo=lo, len_hi=hi)
+    prep = prepare(spec, poison=False)
+    g = torch.Generator().manual_seed(seed + 1)
+    nb = prep.case.num_blocks
+    # codes of N(0,1) / scale, so elements read back about N(0,1)
+    kc = W.randn_e4m3_codes((nb, bs, hkv, 128), g, 1.0 / ks)
+    vc = W.randn_e4m3_codes((nb, bs, hkv, 128), g, 1.0 / vs)
+    used = used_slot_mask(prep.tables, prep.seq_lens, nb, bs)
+    kc[~used] = 0x7F
+    vc[~used] = 0x7F
+    return spec, prep, kc, vc

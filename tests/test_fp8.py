@@ -9,7 +9,7 @@ import pytest
 import torch
 
 import pa_workloads as W
-from harness import TORCH_DTYPE, prepare, to_dev
+from harness import fp8_case, TORCH_DTYPE, prepare, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -61,20 +61,8 @@ def test_fp8_reshape_codes_bit_exact(pa, orc, dtype):
     assert (ek.reshape(-1, hkv, d)[slots[:3][slots[:3] >= 0]] & 0x7F == 0x7E).any()  # saturated
 
 
-def _fp8_case(seed, B=6, lo=200, hi=1300, q_dtype="bf16", bs=16, hq=32, hkv=8, ks=0.05, vs=0.04):
-    spec = W.Spec("fp8", B, hq, hkv, 128, bs, q_dtype, seed=seed, len_dist="uniform",
-                  len_lo=lo, len_hi=hi)
-    prep = prepare(spec, poison=False)
-    g = torch.Generator().manual_seed(seed + 1)
-    nb = prep.case.num_blocks
-    # codes of N(0,1) / scale, so elements read back about N(0,1)
-    kc = W.randn_e4m3_codes((nb, bs, hkv, 128), g, 1.0 / ks)
-    vc = W.randn_e4m3_codes((nb, bs, hkv, 128), g, 1.0 / vs)
-    from harness import used_slot_mask
-    used = used_slot_mask(prep.tables, prep.seq_lens, nb, bs)
-    kc[~used] = NAN_E4M3
-    vc[~used] = NAN_E4M3
-    return spec, prep, kc, vc
+def _fp8_case(seed, **kw):
+    return fp8_case(seed, **kw)
 
 
 @pytest.mark.parametrize("q_dtype,psize", [("bf16", 0), ("f16", 0), ("bf16", 512)])
