@@ -86,6 +86,9 @@ def _load():
         lib.orc_decode_fp8.restype = ctypes.c_int
         lib.orc_decode_fp8.argtypes = [p, p, p, p, ctypes.c_double, ctypes.c_double, p, i64, p,
                                        i32, i32, i32, i32, i32, ctypes.c_double, i32, i32]
+        lib.orc_decode_multi.restype = ctypes.c_int
+        lib.orc_decode_multi.argtypes = [p, p, p, p, p, p, i64, p, i32, i32, i32, i32, i32,
+                                         ctypes.c_double, i32, i32]
         lib.orc_decode.restype = ctypes.c_int
         lib.orc_decode.argtypes = [p, p, p, p, p, i64, p, i32, i32, i32, i32,
                                    i32, ctypes.c_double, i32, i32]
@@ -177,6 +180,32 @@ def decode(q: np.ndarray, key_cache: np.ndarray, value_cache: np.ndarray,
                         float(scale), _dtype_code(dtype), int(nthreads))
     if rc != 0:
         raise RuntimeError("orc_decode failed with code %d" % rc)
+    return out
+
+
+def decode_multi(q: np.ndarray, q_start: np.ndarray, key_cache: np.ndarray,
+                 value_cache: np.ndarray, block_tables: np.ndarray, seq_lens: np.ndarray,
+                 scale: float, dtype, nthreads: int = 1) -> np.ndarray:
+    """fp64 multi-query paged attention: sequence b owns query rows
+    q_start[b] .. q_start[b+1]-1 of q [T, Hq, D] (its last tokens); query i of
+    its n attends the first seq_lens[b] - n + i + 1 tokens.  Returns float64
+    [T, Hq, D]."""
+    lib = _load()
+    qq = np.ascontiguousarray(q, dtype=np.uint16)
+    qs = np.ascontiguousarray(q_start, dtype=np.int32)
+    assert key_cache.flags.c_contiguous and value_cache.flags.c_contiguous
+    bt = np.ascontiguousarray(block_tables, dtype=np.int32)
+    sl = np.ascontiguousarray(seq_lens, dtype=np.int32)
+    T, Hq, D = qq.shape
+    B = sl.shape[0]
+    _, bs, hkv, d2 = key_cache.shape
+    assert d2 == D and bt.shape[0] == B and qs.shape[0] == B + 1 and int(qs[-1]) == T
+    out = np.empty((T, Hq, D), dtype=np.float64)
+    rc = lib.orc_decode_multi(_ptr(out), _ptr(qq), _ptr(qs), _ptr(key_cache), _ptr(value_cache),
+                              _ptr(bt), bt.shape[1], _ptr(sl), B, Hq, hkv, D, bs, float(scale),
+                              _dtype_code(dtype), int(nthreads))
+    if rc != 0:
+        raise RuntimeError("orc_decode_multi failed with code %d" % rc)
     return out
 
 

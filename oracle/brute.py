@@ -56,3 +56,46 @@ def decode_attention(q, key_cache, value_cache, block_tables, seq_lens, scale, d
                          for d in range(D)])
         out.append(rows)
     return out
+
+
+def decode_attention_multi(q, q_start, key_cache, value_cache, block_tables, seq_lens, scale,
+                           dtype):
+    """Several query tokens per sequence: q rows q_start[b] .. q_start[b+1]-1
+    are sequence b's last n tokens; query i of them attends tokens
+    0 .. seq_lens[b] - n + i (itself and everything before it).  Returns
+    [T][Hq][D] Python floats; a query that attends nothing yields zeros."""
+    T = len(q)
+    Hq = len(q[0])
+    D = len(q[0][0])
+    bs = len(key_cache[0])
+    Hkv = len(key_cache[0][0])
+    group = Hq // Hkv
+    out = [None] * T
+    for b in range(len(seq_lens)):
+        L = int(seq_lens[b])
+        r0, r1 = int(q_start[b]), int(q_start[b + 1])
+        n = r1 - r0
+        for i in range(n):
+            r = r0 + i
+            last = min(L - n + i, L - 1)  # the last position this query sees
+            rows = []
+            for h in range(Hq):
+                if last < 0:
+                    rows.append([0.0] * D)
+                    continue
+                g = h // group
+                qv = [decode16(x, dtype) for x in q[r][h]]
+                s, vals = [], []
+                for t in range(last + 1):
+                    blk = int(block_tables[b][t // bs])
+                    off = t % bs
+                    k = [decode16(x, dtype) for x in key_cache[blk][off][g]]
+                    vals.append([decode16(x, dtype) for x in value_cache[blk][off][g]])
+                    s.append(scale * math.fsum(qv[d] * k[d] for d in range(D)))
+                m = max(s)
+                p = [math.exp(x - m) for x in s]
+                den = math.fsum(p)
+                rows.append([math.fsum(p[t] * vals[t][d] for t in range(len(p))) / den
+                             for d in range(D)])
+            out[r] = rows
+    return out

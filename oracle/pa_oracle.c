@@ -30,6 +30,13 @@
  *                         softmax(scale * q K^T) V in double precision (the
  *                         exact quantity that an online softmax reaches up to
  *                         rounding order).
+ *   orc_decode_multi      the same walk for several query tokens of one
+ *                         sequence ("PagedAttention", "Sharing and
+ *                         copy-on-write": a child request recomputes the
+ *                         tokens of its partial last block over the shared
+ *                         prompt blocks).  The causal rule is the decoder's,
+ *                         not the pages': query token i of the last n attends
+ *                         the first L - n + i + 1 tokens.
  *
  * Pool layout (one tensor for K, one for V):
  *   [num_blocks, block_size, num_kv_heads, head_dim]  -- "PagedAttention",
@@ -260,6 +267,7 @@ typedef struct {
   const int32_t* block_tables;
   int64_t table_stride;
   const int32_t* seq_lens;
+  const int32_t* q_start;      /* multi-query: rows q_start[b] .. q_start[b+1]-1, else NULL */
   int32_t num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, dtype;
   double scale;
   int32_t next_seq; /* work counter, guarded by mu */
@@ -272,9 +280,10 @@ static int orc_decode_one(orc_decode_job* j, int32_t b) {
   const int32_t bs = j->block_size;
   const int32_t group = Hq / Hkv;
   const int64_t L = j->seq_lens[b];
-  double* outb = j->out + (int64_t)b * Hq * D;
-  if (L <= 0) {
-    for (int64_t i = 0; i < (int64_t)Hq * D; ++i) outb[i] = 0.0;
+  if (L <= 0) {  /* every query row of the sequence attends to nothing */
+    const int64_t r0 = j->q_start ? j->q_start[b] : b;
+    const int64_t nq = j->q_start ? (int64_t)j->q_start[b + 1] - j->q_start[b] : 1;
+    for (int64_t i = 0; i < nq * Hq * D; ++i) j->out[r0 * Hq * D + i] = 0.0;
     return 0;
   }
   const int32_t* row = j->block_tables + (int64_t)b * j->table_stride;
@@ -301,26 +310,41 @@ static int orc_decode_one(orc_decode_job* j, int32_t b) {
       }
     }
   }
-  for (int32_t h = 0; h < Hq; ++h) {
-    const int32_t g = h / group;
-    const uint16_t* qh = j->q + ((int64_t)b * Hq + h) * D;
-    double m = -INFINITY;
-    for (int64_t t = 0; t < L; ++t) {
-      double dot = 0.0;
-      for (int32_t d = 0; d < D; ++d)
-        dot += orc_decode16(qh[d], j->dtype) * Kc[(t * Hkv + g) * D + d];
-      s[t] = j->scale * dot;
-      if (s[t] > m) m = s[t];
+  /* query rows of this sequence: one (row b) or q_start[b] .. q_start[b+1]-1;
+   * query i of n attends the first L - n + i + 1 tokens (its own position and
+   * everything before it) */
+  const int64_t r0 = j->q_start ? j->q_start[b] : b;
+  const int64_t nq = j->q_start ? (int64_t)j->q_start[b + 1] - j->q_start[b] : 1;
+  for (int64_t i = 0; i < nq; ++i) {
+    const int64_t r = r0 + i;
+    int64_t n = j->q_start ? L - nq + i + 1 : L;
+    if (n > L) n = L;
+    double* outr = j->out + r * Hq * D;
+    if (n <= 0) {
+      for (int64_t e = 0; e < (int64_t)Hq * D; ++e) outr[e] = 0.0;
+      continue;
     }
-    double denom = 0.0;
-    for (int64_t t = 0; t < L; ++t) {
-      s[t] = exp(s[t] - m);
-      denom += s[t];
-    }
-    for (int32_t d = 0; d < D; ++d) {
-      double acc = 0.0;
-      for (int64_t t = 0; t < L; ++t) acc += s[t] * Vc[(t * Hkv + g) * D + d];
-      outb[(int64_t)h * D + d] = acc / denom;
+    for (int32_t h = 0; h < Hq; ++h) {
+      const int32_t g = h / group;
+      const uint16_t* qh = j->q + (r * Hq + h) * D;
+      double m = -INFINITY;
+      for (int64_t t = 0; t < n; ++t) {
+        double dot = 0.0;
+        for (int32_t d = 0; d < D; ++d)
+          dot += orc_decode16(qh[d], j->dtype) * Kc[(t * Hkv + g) * D + d];
+        s[t] = j->scale * dot;
+        if (s[t] > m) m = s[t];
+      }
+      double denom = 0.0;
+      for (int64_t t = 0; t < n; ++t) {
+        s[t] = exp(s[t] - m);
+        denom += s[t];
+      }
+      for (int32_t d = 0; d < D; ++d) {
+        double acc = 0.0;
+        for (int64_t t = 0; t < n; ++t) acc += s[t] * Vc[(t * Hkv + g) * D + d];
+        outr[(int64_t)h * D + d] = acc / denom;
+      }
     }
   }
   free(Kc); free(Vc); free(s);
@@ -347,7 +371,8 @@ static void* orc_decode_worker(void* arg) {
  * With key_cache8 / value_cache8 not NULL the cache holds E4M3 codes and a
  * stored element reads as code * k_scale (keys) or code * v_scale (values);
  * the query keeps its 16-bit type (dtype). */
-static int orc_decode_impl(double* out, const uint16_t* q, const uint16_t* key_cache,
+static int orc_decode_impl(double* out, const uint16_t* q, const int32_t* q_start,
+                           const uint16_t* key_cache,
                            const uint16_t* value_cache, const uint8_t* key_cache8,
                            const uint8_t* value_cache8, double k_scale, double v_scale,
                            const int32_t* block_tables, int64_t table_stride,
@@ -361,7 +386,8 @@ static int orc_decode_impl(double* out, const uint16_t* q, const uint16_t* key_c
   j.k_scale = k_scale; j.v_scale = v_scale;
   j.out = out; j.q = q; j.key_cache = key_cache; j.value_cache = value_cache;
   j.block_tables = block_tables; j.table_stride = table_stride;
-  j.seq_lens = seq_lens; j.num_seqs = num_seqs; j.num_q_heads = num_q_heads;
+  j.seq_lens = seq_lens; j.q_start = q_start;
+  j.num_seqs = num_seqs; j.num_q_heads = num_q_heads;
   j.num_kv_heads = num_kv_heads; j.head_dim = head_dim;
   j.block_size = block_size; j.dtype = dtype; j.scale = scale;
   j.next_seq = 0; j.failed = 0;
@@ -386,7 +412,7 @@ int orc_decode(double* out, const uint16_t* q, const uint16_t* key_cache,
                int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
                int32_t block_size, double scale, int32_t dtype,
                int32_t nthreads) {
-  return orc_decode_impl(out, q, key_cache, value_cache, NULL, NULL, 1.0, 1.0,
+  return orc_decode_impl(out, q, NULL, key_cache, value_cache, NULL, NULL, 1.0, 1.0,
                          block_tables, table_stride, seq_lens, num_seqs, num_q_heads,
                          num_kv_heads, head_dim, block_size, scale, dtype, nthreads);
 }
@@ -397,7 +423,26 @@ int orc_decode_fp8(double* out, const uint16_t* q, const uint8_t* key_cache,
                    const int32_t* seq_lens, int32_t num_seqs, int32_t num_q_heads,
                    int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
                    double scale, int32_t q_dtype, int32_t nthreads) {
-  return orc_decode_impl(out, q, NULL, NULL, key_cache, value_cache, k_scale, v_scale,
+  return orc_decode_impl(out, q, NULL, NULL, NULL, key_cache, value_cache, k_scale, v_scale,
                          block_tables, table_stride, seq_lens, num_seqs, num_q_heads,
                          num_kv_heads, head_dim, block_size, scale, q_dtype, nthreads);
+}
+
+/* Multi-query paged attention (several new tokens per sequence, as in a chunk
+ * of prefill or the verification of speculated tokens): sequence b owns query
+ * rows q_start[b] .. q_start[b+1]-1 of q [T, Hq, D] (its last n = q_len tokens,
+ * whose K and V are already in the cache), and query i of them attends, like
+ * any token of a causal decoder, to the tokens at positions 0 .. L_b - n + i.
+ * out is double [T, Hq, D].  A query that would attend nothing (q_len > L_b)
+ * gets zeros.  Same pools and readings as orc_decode. */
+int orc_decode_multi(double* out, const uint16_t* q, const int32_t* q_start,
+                     const uint16_t* key_cache, const uint16_t* value_cache,
+                     const int32_t* block_tables, int64_t table_stride,
+                     const int32_t* seq_lens, int32_t num_seqs, int32_t num_q_heads,
+                     int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                     double scale, int32_t dtype, int32_t nthreads) {
+  if (!q_start) return 2;
+  return orc_decode_impl(out, q, q_start, key_cache, value_cache, NULL, NULL, 1.0, 1.0,
+                         block_tables, table_stride, seq_lens, num_seqs, num_q_heads,
+                         num_kv_heads, head_dim, block_size, scale, dtype, nthreads);
 }

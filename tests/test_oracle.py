@@ -309,6 +309,105 @@ def test_planted_gqa_mistake_is_caught(orc):
 
 
 # --------------------------------------------------------------------------
+# several query tokens per sequence (causal over the paged tokens)
+# --------------------------------------------------------------------------
+def _multi_case(seed, lens, qlens, hq=4, hkv=2, d=16, bs=4, dtype="f16"):
+    rng = np.random.default_rng(seed)
+    B = len(lens)
+    nblk = [-(-L // bs) for L in lens]
+    nb = sum(nblk) + 3
+    kc = _bits(rng.standard_normal((nb, bs, hkv, d)), dtype)
+    vc = _bits(rng.standard_normal((nb, bs, hkv, d)), dtype)
+    qs = np.concatenate([[0], np.cumsum(qlens)]).astype(np.int32)
+    q = _bits(rng.standard_normal((int(qs[-1]), hq, d)), dtype)
+    perm = rng.permutation(nb).astype(np.int32)
+    table = np.full((B, max(nblk) + 1), -1, np.int32)
+    k = 0
+    for b in range(B):
+        table[b, :nblk[b]] = perm[k:k + nblk[b]]
+        k += nblk[b]
+    return q, qs, kc, vc, table, np.array(lens, np.int32)
+
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+def test_multi_query_vs_brute(orc, dtype):
+    q, qs, kc, vc, table, lens = _multi_case(5, (9, 14, 3, 6), (3, 5, 3, 1), dtype=dtype)
+    out = orc.decode_multi(q, qs, kc, vc, table, lens, 0.3, dtype)
+    ref = np.array(brute.decode_attention_multi(q.tolist(), qs.tolist(), kc.tolist(), vc.tolist(),
+                                                table.tolist(), lens.tolist(), 0.3, dtype))
+    assert np.max(np.abs(out - ref)) <= 1e-12
+
+
+def test_multi_query_identity_table_vs_torch_sdpa(orc):
+    """With the block table 0, 1, 2, ... the pool is a contiguous sequence, and
+    the n new tokens are the last n queries of causal attention: torch's
+    float64 scaled_dot_product_attention with the matching boolean mask (query
+    i of n sees key positions <= L - n + i)."""
+    rng = np.random.default_rng(9)
+    hq, hkv, d, bs, L, n = 8, 2, 32, 8, 41, 6
+    nblk = -(-L // bs)
+    kc = _bits(rng.standard_normal((nblk, bs, hkv, d)), "bf16")
+    vc = _bits(rng.standard_normal((nblk, bs, hkv, d)), "bf16")
+    q = _bits(rng.standard_normal((n, hq, d)), "bf16")
+    table = np.arange(nblk, dtype=np.int32)[None]
+    scale = 1.0 / math.sqrt(d)
+    out = orc.decode_multi(q, np.array([0, n], np.int32), kc, vc, table,
+                           np.array([L], np.int32), scale, "bf16")
+    K = torch.from_numpy(_to_f64(kc, "bf16")).reshape(nblk * bs, hkv, d)[:L]
+    V = torch.from_numpy(_to_f64(vc, "bf16")).reshape(nblk * bs, hkv, d)[:L]
+    Q = torch.from_numpy(_to_f64(q, "bf16")).permute(1, 0, 2)            # [Hq, n, d]
+    kb = K.permute(1, 0, 2).repeat_interleave(hq // hkv, dim=0)          # [Hq, L, d]
+    vb = V.permute(1, 0, 2).repeat_interleave(hq // hkv, dim=0)
+    pos = torch.arange(L)[None, :]
+    allowed = pos <= (L - n + torch.arange(n))[:, None]                  # [n, L]
+    ref = torch.nn.functional.scaled_dot_product_attention(Q, kb, vb, attn_mask=allowed,
+                                                           scale=scale)
+    assert np.max(np.abs(out - ref.permute(1, 0, 2).numpy())) <= 1e-12
+
+
+def test_multi_query_single_token_is_decode(orc):
+    """One query token per sequence is the decode step (every token seen)."""
+    q, qs, kc, vc, table, lens = _multi_case(6, (9, 14, 1, 6), (1, 1, 1, 1))
+    a = orc.decode_multi(q, qs, kc, vc, table, lens, 0.3, "f16")
+    b = orc.decode(q, kc, vc, table, lens, 0.3, "f16")
+    assert np.array_equal(a, b)
+
+
+def test_multi_query_last_token_sees_everything(orc):
+    """The last of a sequence's new tokens attends the whole sequence: its row
+    equals the one-token decode of that sequence; the first new token equals
+    the decode of the sequence cut just after it."""
+    q, qs, kc, vc, table, lens = _multi_case(7, (12, 20), (4, 6))
+    out = orc.decode_multi(q, qs, kc, vc, table, lens, 0.3, "f16")
+    last = qs[1:] - 1
+    full = orc.decode(q[last], kc, vc, table, lens, 0.3, "f16")
+    assert np.max(np.abs(out[last] - full)) <= 1e-15
+    first = qs[:-1]
+    cut = lens - (qs[1:] - qs[:-1]) + 1
+    part = orc.decode(q[first], kc, vc, table, cut, 0.3, "f16")
+    assert np.max(np.abs(out[first] - part)) <= 1e-15
+
+
+def test_planted_causal_off_by_one_is_caught(orc):
+    """A plausible slip in the causal limit (query i seeing one token more or
+    one less) disagrees with the masked library attention: emulated by
+    handing the oracle one more (or one fewer) token than the sequence has."""
+    q, qs, kc, vc, table, lens = _multi_case(8, (11,), (4,), hq=2, hkv=2)
+    good = orc.decode_multi(q, qs, kc, vc, table, lens, 0.5, "f16")
+    for delta in (-1, 1):
+        bad = orc.decode_multi(q, qs, kc, vc, table, lens + delta, 0.5, "f16")
+        assert np.max(np.abs(good - bad)) > 1e-3
+
+
+def test_multi_query_more_queries_than_tokens(orc):
+    """q_len > seq_len: the leading queries see nothing and give zeros."""
+    q, qs, kc, vc, table, lens = _multi_case(4, (3,), (5,))
+    out = orc.decode_multi(q, qs, kc, vc, table, lens, 0.3, "f16")
+    assert np.all(out[:2] == 0.0)
+    assert np.all(np.abs(out[2:]).sum(axis=(1, 2)) > 0)
+
+
+# --------------------------------------------------------------------------
 # fp8 (E4M3) cache pieces
 # --------------------------------------------------------------------------
 def test_e4m3_decoder_all_codes(orc):
