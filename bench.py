@@ -172,18 +172,44 @@ def build_workload(spec, pa):
                     cow.append(c)
         new_k, new_v = case.new_k, case.new_v
     else:
-        slots = []
-        for b in range(B):
-            bm.add_sequence(b, int(lens[b]) - 1)
-            slots.append(bm.append_slot(b)[0])
-        g = torch.Generator().manual_seed(spec.seed + 7)
-        new_k = W.randn_bits((B, spec.num_kv_heads, spec.head_dim), spec.dtype, g)
-        new_v = W.randn_bits((B, spec.num_kv_heads, spec.head_dim), spec.dtype, g)
+        slots, new_k, new_v = _append_new_tokens(spec, bm, lens)
     width = max(len(bm.block_table(b)) for b in range(B))
     tables = bm.tables(list(range(B)), width).numpy()
-    return dict(case=case, lens=lens, tables=tables, slots=np.array(slots, np.int32),
-                cow=np.array(cow, np.int32).reshape(-1, 2), new_k=new_k, new_v=new_v,
-                shared_blocks=bm.shared_blocks(list(range(B))).numpy())
+    wl = dict(case=case, lens=lens, tables=tables, slots=np.array(slots, np.int32),
+              cow=np.array(cow, np.int32).reshape(-1, 2), new_k=new_k, new_v=new_v,
+              shared_blocks=bm.shared_blocks(list(range(B))).numpy())
+    _add_queries(spec, wl)
+    return wl
+
+
+def _append_new_tokens(spec, bm, lens):
+    """Every sequence holds seq_len - q_len tokens and the step appends its
+    q_len current tokens (positions seq_len - q_len .. seq_len - 1), which the
+    attention then reads.  Returns (slots, new K rows, new V rows)."""
+    B, q = spec.num_seqs, spec.q_len
+    slots = []
+    for b in range(B):
+        bm.add_sequence(b, int(lens[b]) - q)
+        for _ in range(q):
+            slots.append(bm.append_slot(b)[0])
+    g = torch.Generator().manual_seed(spec.seed + 7)
+    new_k = W.randn_bits((B * q, spec.num_kv_heads, spec.head_dim), spec.dtype, g)
+    new_v = W.randn_bits((B * q, spec.num_kv_heads, spec.head_dim), spec.dtype, g)
+    return slots, new_k, new_v
+
+
+def _add_queries(spec, wl):
+    """Query rows: the workload's [B, Hq, D] draw, or with q_len > 1 the
+    [B * q_len, Hq, D] rows of every sequence's new tokens (sequence b owns rows
+    b q_len .. b q_len + q_len - 1)."""
+    B, q = spec.num_seqs, spec.q_len
+    if q == 1:
+        wl["q"] = wl["case"].q
+        wl["q_start"] = None
+        return
+    g = torch.Generator().manual_seed(spec.seed + 11)
+    wl["q"] = W.randn_bits((B * q, spec.num_q_heads, spec.head_dim), spec.dtype, g)
+    wl["q_start"] = (np.arange(B + 1) * q).astype(np.int32)
 
 
 def kv_memory(spec, wl) -> dict:
@@ -277,14 +303,16 @@ def run_ours(args, rank, world, local_rank):
     else:
         k_cache, v_cache = dev_bits(case.k_pool), dev_bits(case.v_pool)
         k_scale = v_scale = None
-    q = dev_bits(case.q)
+    q = dev_bits(wl["q"])
+    multi = spec.q_len > 1
+    q_start = torch.from_numpy(wl["q_start"]).to(device) if multi else None
     new_k, new_v = dev_bits(wl["new_k"]), dev_bits(wl["new_v"])
     slots = torch.from_numpy(wl["slots"]).to(device)
     tables = torch.from_numpy(wl["tables"]).to(device)
     lens = torch.from_numpy(wl["lens"]).to(device)
     cow = torch.from_numpy(wl["cow"]).to(device) if wl["cow"].size else None
     out = torch.empty_like(q)
-    B, Hq, D = q.shape
+    B, Hq, D = spec.num_seqs, spec.num_q_heads, spec.head_dim
     max_len = int(wl["lens"].max())
     psize = spec.partition_size
     # parallel samples: read each shared prompt block once per pack of sequences
@@ -293,6 +321,10 @@ def run_ours(args, rank, world, local_rank):
         shared_blocks = torch.from_numpy(wl["shared_blocks"]).to(device)
         ws = pa.alloc_workspace(pa.shared_prefix_workspace_bytes(
             B, Hq, spec.num_kv_heads, D, spec.block_size, max_len, psize), device)
+    elif multi:
+        ws = pa.alloc_workspace(pa.multi_query_workspace_bytes(
+            B, q.shape[0], spec.q_len, Hq, spec.num_kv_heads, D, spec.block_size, max_len,
+            psize), device)
     else:
         ws = pa.alloc_workspace(pa.decode_workspace_bytes(
             B, Hq, spec.num_kv_heads, D, spec.block_size, max_len, psize), device)
@@ -318,6 +350,10 @@ def run_ours(args, rank, world, local_rank):
             pa.decode_attention_shared_prefix(out, q, k_cache, v_cache, tables, lens,
                                               shared_blocks, max_len, scale, psize, ws,
                                               error_flag=flag)
+        elif multi:
+            pa.decode_attention_multi_query(out, q, q_start, k_cache, v_cache, tables, lens,
+                                            max_len, spec.q_len, scale, psize, ws,
+                                            error_flag=flag)
         else:
             pa.decode_attention(out, q, k_cache, v_cache, tables, lens, max_len, scale, psize, ws,
                                 error_flag=flag)
@@ -367,7 +403,7 @@ def run_ours(args, rank, world, local_rank):
         t = torch.from_numpy(np.ascontiguousarray(a))
         dst.copy_(t.view(torch.int16).view(dtype) if dtype is not None else t)
 
-    e2e_ok = wl["slots"].shape[0] == B and cow is None
+    e2e_ok = wl["slots"].shape[0] == B and cow is None and not multi
     e2e = None
     if e2e_ok:
         h = runner.host
@@ -423,12 +459,13 @@ def run_ours(args, rank, world, local_rank):
             "num_blocks": case.num_blocks, "parallelism": "dp%d (independent batches)" % world,
             "l2": "no flush: each step reads %.0f MB of KV, more than the 126 MB L2" % (bytes_step / 1e6),
         },
-        "decode_tokens_per_s": round(spec.num_seqs * world / (ms_per_step / 1e3), 1),
+        "decode_tokens_per_s": round(spec.num_seqs * spec.q_len * world / (ms_per_step / 1e3), 1),
         "attention_gbs": round(achieved, 2),
         "pct_of_8tbs": round(100.0 * value / 8000.0, 2),
         "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": traffic,
                      "kernel": ("pa_decode_attention_shared_prefix" if shared else
+                                "pa_decode_attention_multi_query" if multi else
                                 "pa_decode_attention") + " (plan + main + combine launches)",
                      "bytes_per_launch": read_bytes,
                      "peak_kind": peak_kind + " (MEASURED_PEAKS hbm_gbs, copy read+write)"},
@@ -452,6 +489,9 @@ def run_ours(args, rank, world, local_rank):
 
 
 def describe_lengths(spec):
+    if spec.q_len > 1:
+        return "%s, %d new tokens per sequence attending causally" % (
+            describe_lengths(spec.replace(q_len=1)), spec.q_len)
     if spec.len_dist == "uniform":
         return "U[%d, %d]" % (spec.len_lo, spec.len_hi)
     if spec.len_dist == "lognormal":
@@ -501,6 +541,14 @@ def _oracle_sample(spec, wl, seqs):
         oracle.decode_fp8(case.q[seqs], k, v, spec.k_scale, spec.v_scale, wl["tables"][seqs],
                           wl["lens"][seqs], W.scale_of(spec), spec.dtype, nthreads=threads)
         return time.perf_counter() - t0, kv_bytes(spec, wl["lens"][seqs])
+    if spec.q_len > 1:  # each sequence's q_len new rows, then its q_len queries
+        q = spec.q_len
+        rows = (seqs[:, None] * q + np.arange(q)[None, :]).reshape(-1)
+        oracle.reshape_and_cache(wl["new_k"][rows], wl["new_v"][rows], k, v, wl["slots"][rows])
+        oracle.decode_multi(wl["q"][rows], (np.arange(len(seqs) + 1) * q).astype(np.int32), k, v,
+                            wl["tables"][seqs], wl["lens"][seqs], W.scale_of(spec), spec.dtype,
+                            nthreads=threads)
+        return time.perf_counter() - t0, kv_bytes(spec, wl["lens"][seqs])
     if spec.len_dist != "shared_prefix":
         oracle.reshape_and_cache(wl["new_k"][seqs], wl["new_v"][seqs], k, v, wl["slots"][seqs])
     oracle.decode(case.q[seqs], k, v, wl["tables"][seqs], wl["lens"][seqs], W.scale_of(spec),
@@ -539,13 +587,7 @@ def run_reference(args, rank, world):
     case = W.draw(spec)
     bm = RefBlockManager(case.num_blocks, spec.block_size, case.free_order)
     lens = case.seq_lens.astype(np.int32)
-    slots = []
-    for b in range(spec.num_seqs):
-        bm.add_sequence(b, int(lens[b]) - 1)
-        slots.append(bm.append_slot(b)[0])
-    g = torch.Generator().manual_seed(spec.seed + 7)
-    new_k = W.randn_bits((spec.num_seqs, spec.num_kv_heads, spec.head_dim), spec.dtype, g)
-    new_v = W.randn_bits((spec.num_seqs, spec.num_kv_heads, spec.head_dim), spec.dtype, g)
+    slots, new_k, new_v = _append_new_tokens(spec, bm, lens)
     width = max(len(bm.block_table(b)) for b in range(spec.num_seqs))
     tables = np.full((spec.num_seqs, width), -1, np.int32)
     for b in range(spec.num_seqs):
@@ -553,6 +595,7 @@ def run_reference(args, rank, world):
         tables[b, :len(t)] = t
     wl = dict(case=case, lens=lens, tables=tables, slots=np.array(slots, np.int32),
               new_k=new_k, new_v=new_v)
+    _add_queries(spec, wl)
     # size each step so warm-up + timed steps take about args.ref_budget seconds
     B = spec.num_seqs
     t1, _ = _oracle_sample(spec, wl, np.arange(1))

@@ -303,6 +303,60 @@ pa_status pa_decode_attention_strided(void* out, pa_dtype out_dtype, const void*
                                       int32_t* device_error_flag, pa_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * pa_decode_multi_query_workspace_bytes -- device scratch for
+ * pa_decode_attention_multi_query: num_query_rows query rows in all, at most
+ * max_q_len of them per sequence.  Other arguments as in
+ * pa_decode_workspace_bytes.
+ * ------------------------------------------------------------------------- */
+pa_status pa_decode_multi_query_workspace_bytes(int32_t num_seqs, int32_t num_query_rows,
+                                                int32_t max_q_len, int32_t num_q_heads,
+                                                int32_t num_kv_heads, int32_t head_dim,
+                                                int32_t block_size, int32_t max_seq_len,
+                                                int32_t partition_size, size_t* bytes);
+
+/* ---------------------------------------------------------------------------
+ * pa_decode_attention_multi_query -- paged attention for several new tokens
+ * of each sequence at once.  [PA] "Sharing and copy-on-write": a child
+ * request recomputes the tokens of its partial last block over the shared
+ * prompt blocks -- several query tokens of one sequence attending the paged
+ * cache; the same call serves verifying speculated tokens and small chunks of
+ * prefill.  The causal rule is the decoder's (the pages do not state it):
+ * sequence b owns query rows q_start[b] .. q_start[b+1]-1 (its last
+ * n_b = q_start[b+1] - q_start[b] tokens, whose K and V are already in the
+ * pool, e.g. written by pa_reshape_and_cache), and query i of them attends
+ * the tokens at positions 0 .. seq_lens[b] - n_b + i:
+ *
+ *   out[r, h, :] = sum_{t <= L_b - n_b + i} softmax_t(scale <query[r, h, :], K_b[t]>) V_b[t]
+ *
+ *  out, query      [num_query_rows, num_q_heads, head_dim], contiguous; out in
+ *                  out_dtype (F16, BF16, F32), query in kv_dtype.
+ *  q_start         int32 [num_seqs + 1], device, non-decreasing, q_start[0] >= 0,
+ *                  q_start[num_seqs] <= num_query_rows.  Rows outside every
+ *                  sequence's range are not written.
+ *  max_q_len       host-side bound of q_start[b+1] - q_start[b] (>= 1): a
+ *                  launch covers up to 32 / (num_q_heads / num_kv_heads)
+ *                  query tokens of a sequence at once; longer runs are cut
+ *                  into chunks that each read the sequence's tokens again.
+ *  workspace       at least pa_decode_multi_query_workspace_bytes().
+ * A query that would attend nothing (n_b > seq_lens[b]) gets zeros.  Other
+ * arguments, layouts and errors are those of pa_decode_attention; on the
+ * device, ranges of q_start that are negative or leave [0, num_query_rows)
+ * are flagged PA_DEVERR_BAD_SEQLEN and skipped.
+ * ------------------------------------------------------------------------- */
+pa_status pa_decode_attention_multi_query(void* out, pa_dtype out_dtype, const void* query,
+                                          const int32_t* q_start, int32_t num_query_rows,
+                                          int32_t max_q_len, const void* key_cache,
+                                          const void* value_cache, const int32_t* block_tables,
+                                          int32_t block_table_stride, const int32_t* seq_lens,
+                                          int32_t num_seqs, int32_t max_seq_len,
+                                          int32_t num_q_heads, int32_t num_kv_heads,
+                                          int32_t head_dim, int32_t num_blocks,
+                                          int32_t block_size, float scale, pa_dtype kv_dtype,
+                                          int32_t partition_size, void* workspace,
+                                          size_t workspace_bytes, int32_t* device_error_flag,
+                                          pa_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * pa_decode_shared_prefix_workspace_bytes -- device scratch for
  * pa_decode_attention_shared_prefix (larger than pa_decode_workspace_bytes:
  * room for the packs' entries and eight query columns per KV head).  Same

@@ -25,6 +25,8 @@ parallel sampling with a shared prompt):
   shared_prefix 32 prompts of 2047 tokens x 8 samples, each sample then
                 appending U[1, 200] tokens, bs 16, Hq 32 / Hkv 8, D 128, bf16
   llama8b_fp8   the llama8b shape over an fp8 (E4M3) cache, scales 1/32
+  llama8b_mq4   the llama8b shape with 4 new tokens per sequence attending
+                together (causal), as when speculated tokens are verified
 """
 from __future__ import annotations
 
@@ -68,6 +70,7 @@ class Spec:
     kv_dtype: str = "auto"           # 'auto' (16-bit pools) or 'fp8_e4m3' (code pools)
     k_scale: float = 1.0             # fp8 pools: element = code * scale
     v_scale: float = 1.0
+    q_len: int = 1                   # new tokens per sequence attending at once
 
     @property
     def group(self) -> int:
@@ -101,6 +104,9 @@ WORKLOADS = {
     "llama8b_fp8": Spec("llama8b_fp8", 64, 32, 8, 128, 16, "bf16", seed=1005,
                         len_dist="uniform", len_lo=512, len_hi=4096,
                         kv_dtype="fp8_e4m3", k_scale=1.0 / 32, v_scale=1.0 / 32),
+    # the llama8b shape, 4 new tokens per sequence
+    "llama8b_mq4": Spec("llama8b_mq4", 64, 32, 8, 128, 16, "bf16", seed=1006,
+                        len_dist="uniform", len_lo=512, len_hi=4096, q_len=4),
 }
 
 

@@ -22,6 +22,9 @@ Entry points (see the header for argument meaning, layout and errors):
   neighbouring sequences share leading blocks (parallel samples of one
   prompt, "Sharing and copy-on-write"): a shared prefix is read once per pack
   of sequences instead of once per sequence.
+* ``decode_attention_multi_query`` -- several new tokens per sequence (a
+  recomputed partial block, verified speculated tokens), each attending the
+  paged cache causally.
 * ``BlockManager``      -- the native host block manager (free list,
   refcounts, copy-on-write planning, shared-prefix counts).
 * ``PagedDecodeStep``   -- one decode step from pinned host buffers: copies in,
@@ -38,7 +41,8 @@ import torch
 __all__ = [
     "LIB_PATH", "PagedAttnError", "reshape_and_cache", "copy_blocks", "decode_attention",
     "decode_workspace_bytes", "decode_attention_fp8", "decode_attention_noalloc",
-    "decode_attention_shared_prefix", "shared_prefix_workspace_bytes", "BlockManager",
+    "decode_attention_shared_prefix", "shared_prefix_workspace_bytes",
+    "decode_attention_multi_query", "multi_query_workspace_bytes", "BlockManager",
     "PagedDecodeStep", "DEVERR_BAD_BLOCK", "DEVERR_BAD_SLOT", "DEVERR_BAD_SEQLEN",
     "DEVERR_TIMEOUT", "DEVERR_BAD_SHARE", "CacheStrides", "version",
 ]
@@ -126,6 +130,14 @@ def _load() -> ctypes.CDLL:
                                                       i32, i32, i32, i32, i32, i32,
                                                       ctypes.c_float, ctypes.c_int, i32, p, sz,
                                                       p, p]
+    lib.pa_decode_multi_query_workspace_bytes.restype = ctypes.c_int
+    lib.pa_decode_multi_query_workspace_bytes.argtypes = [i32, i32, i32, i32, i32, i32, i32, i32,
+                                                          i32, ctypes.POINTER(sz)]
+    lib.pa_decode_attention_multi_query.restype = ctypes.c_int
+    lib.pa_decode_attention_multi_query.argtypes = [p, ctypes.c_int, p, p, i32, i32, p, p, p, i32,
+                                                    p, i32, i32, i32, i32, i32, i32, i32,
+                                                    ctypes.c_float, ctypes.c_int, i32, p, sz, p,
+                                                    p]
     lib.pa_decode_attention_noalloc.restype = ctypes.c_int
     lib.pa_decode_attention_noalloc.argtypes = [p, ctypes.c_int, p, p, p, p, i32, p, i32, i32, i32,
                                                 i32, i32, i32, i32, ctypes.c_float, ctypes.c_int,
@@ -397,6 +409,55 @@ def decode_attention_shared_prefix(out: torch.Tensor, query: torch.Tensor,
         int(max_seq_len), hq, hkv, d, nb, bs, float(scale), _DTYPE_CODE[query.dtype],
         int(partition_size), _ptr(workspace), workspace.numel() * workspace.element_size(),
         _ptr(error_flag), _stream_handle(stream)), "pa_decode_attention_shared_prefix")
+    return out
+
+
+def multi_query_workspace_bytes(num_seqs: int, num_query_rows: int, max_q_len: int,
+                                num_q_heads: int, num_kv_heads: int, head_dim: int,
+                                block_size: int, max_seq_len: int,
+                                partition_size: int = 0) -> int:
+    out = ctypes.c_size_t(0)
+    _check(lib.pa_decode_multi_query_workspace_bytes(
+        num_seqs, num_query_rows, max_q_len, num_q_heads, num_kv_heads, head_dim, block_size,
+        max_seq_len, partition_size, ctypes.byref(out)), "pa_decode_multi_query_workspace_bytes")
+    return int(out.value)
+
+
+def decode_attention_multi_query(out: torch.Tensor, query: torch.Tensor, q_start: torch.Tensor,
+                                 key_cache: torch.Tensor, value_cache: torch.Tensor,
+                                 block_tables: torch.Tensor, seq_lens: torch.Tensor,
+                                 max_seq_len: int, max_q_len: int, scale: float,
+                                 partition_size: int = 0,
+                                 workspace: Optional[torch.Tensor] = None,
+                                 error_flag: Optional[torch.Tensor] = None,
+                                 stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """Several new tokens per sequence: query/out [T, Hq, D]; q_start int32 [B + 1]
+    on the device (sequence b owns rows q_start[b] .. q_start[b+1]-1, its last
+    tokens, already in the cache); query i of a sequence's n attends positions
+    0 .. seq_len - n + i.  max_q_len bounds n (host side)."""
+    _need(query.dim() == 3 and query.is_contiguous(), "query must be contiguous [T, Hq, D]")
+    _need(out.shape == query.shape and out.is_contiguous(), "out must be contiguous [T, Hq, D]")
+    _need(key_cache.is_contiguous() and value_cache.is_contiguous(), "caches must be contiguous")
+    _need(key_cache.shape == value_cache.shape, "K and V pools differ")
+    _need(block_tables.dtype == torch.int32 and block_tables.dim() == 2 and
+          block_tables.stride(1) == 1, "block_tables int32 [B, W], rows contiguous")
+    _need(seq_lens.dtype == torch.int32 and seq_lens.is_contiguous(), "seq_lens int32")
+    _need(q_start.dtype == torch.int32 and q_start.is_contiguous() and
+          q_start.numel() == seq_lens.numel() + 1, "q_start int32 [B + 1]")
+    _need(query.dtype == key_cache.dtype == value_cache.dtype, "query and caches share a dtype")
+    T, hq, d = query.shape
+    B = seq_lens.numel()
+    nb, bs, hkv, _ = key_cache.shape
+    if workspace is None:
+        workspace = alloc_workspace(multi_query_workspace_bytes(
+            B, T, int(max_q_len), hq, hkv, d, bs, int(max_seq_len), partition_size), query.device)
+    _check(lib.pa_decode_attention_multi_query(
+        _ptr(out), _DTYPE_CODE[out.dtype], _ptr(query), _ptr(q_start), T, int(max_q_len),
+        _ptr(key_cache), _ptr(value_cache), _ptr(block_tables), block_tables.stride(0),
+        _ptr(seq_lens), B, int(max_seq_len), hq, hkv, d, nb, bs, float(scale),
+        _DTYPE_CODE[query.dtype], int(partition_size), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _ptr(error_flag), _stream_handle(stream)),
+        "pa_decode_attention_multi_query")
     return out
 
 

@@ -39,6 +39,7 @@ enum : int32_t {
   kSegStart = 2,  // reset the online-softmax state
   kSegEnd = 4,    // finalise and write the segment
   kDirect = 8,    // the segment is the whole sequence: write `out` directly
+  kCausal = 16,   // several query tokens of one sequence: column c sees rows <= rel + c / G
 };
 
 constexpr int kMaxPack = 8;        // sequences per pack
@@ -51,8 +52,9 @@ struct TileInfo {
   int32_t mask;    // bit t set: token t takes part (valid and its block id is good)
   int32_t seg;     // segment id inside this head group
   int32_t flags;
-  int32_t members;  // sequences whose queries use this tile (pack size or 1)
-  int32_t pad[2];
+  int32_t members;  // query rows using this tile: pack members, query tokens, or 1
+  int32_t qrow0;    // query row of column 0 (column c: row qrow0 + c / G, head c % G)
+  int32_t rel;      // kCausal: last visible tile row of column 0 (may be < 0 or > 15)
 };
 
 struct DecodeParams {
@@ -63,6 +65,7 @@ struct DecodeParams {
   int64_t table_stride;
   int32_t out_dtype;
   int32_t num_seqs, max_seq_len, num_q_heads, group, num_blocks, block_size;
+  int32_t num_rows;        // query (and output) rows: num_seqs, or the multi-query rows
   int32_t tiles_per_part;  // partition length in tiles (INT_MAX: no partitions)
   float scale_log2;        // scale * log2(e)
   int32_t ctas_per_group;  // CTAs sharing one head group's tiles
@@ -87,7 +90,16 @@ struct DecodeParams {
   int32_t* pack_tiles;     // [num_seqs / 2] prefix tiles of pack k
   int32_t* seq_pack;       // [num_seqs] pack of sequence b, or -1
   int32_t* seq_pre;        // [num_seqs] tiles of b attended through its pack
-  int32_t* meta;           // [1] number of packs K (0 without packing)
+  int32_t* meta;           // [2] number of packs K (0 without packing), number of entries E
+  // several query tokens per sequence ("multi-query"): entries are chunks of
+  // at most q_per_entry query tokens of one sequence
+  const int32_t* q_start;  // [num_seqs + 1] query rows of sequence b, or null
+  int32_t q_per_entry;
+  int32_t* ent_b;          // [rows] sequence of entry e
+  int32_t* ent_q0;         // [rows] first query row of entry e
+  int32_t* ent_nq;         // [rows] query rows of entry e
+  int32_t* ent_tok;        // [rows] tokens entry e reads: one past its last query's position
+  int32_t* q_entry;        // [rows] entry of query row r
   int32_t cols;            // partial columns per KV head: pack_size * group
   float* part_o;           // [groups][nseg_cap][HG][cols][head_dim]
   float* part_ml;          // [groups][nseg_cap][HG][cols][2]  (m in log2 units, l)
@@ -215,6 +227,51 @@ __global__ void __launch_bounds__(kPlanThreads) pa_plan_kernel(DecodeParams p) {
   const int B = p.num_seqs;
   griddep_launch_dependents();
   griddep_wait();  // seq_lens may come from the previous kernel on the stream
+  int E = 0;       // entries
+  const bool multi = p.q_start != nullptr;
+  if (multi) {
+    // ---- several query tokens per sequence: entry = a chunk of at most
+    // q_per_entry consecutive query rows of one sequence; it reads the tokens
+    // up to its last query's position
+    const int Qc = p.q_per_entry;
+    for (int r = tid; r < p.num_rows; r += kPlanThreads) p.q_entry[r] = -1;
+    __syncthreads();
+    int32_t ecarry = 0;
+    for (int b0 = 0; b0 < B; b0 += kPlanThreads) {  // uniform trip count: the scan syncs
+      const int b = b0 + tid;
+      int32_t nch = 0, qlen = 0, L = 0, q0 = 0;
+      if (b < B) {
+        q0 = p.q_start[b];
+        qlen = p.q_start[b + 1] - q0;
+        const int32_t raw = p.seq_lens[b];
+        if (raw < 0 || raw > p.max_seq_len || qlen < 0 || q0 < 0 ||
+            static_cast<int64_t>(q0) + qlen > p.num_rows) {
+          flag_error(p.err, PA_DEVERR_BAD_SEQLEN);
+          qlen = (qlen < 0 || q0 < 0 || static_cast<int64_t>(q0) + qlen > p.num_rows) ? 0 : qlen;
+        }
+        L = clamp_len(raw, p.max_seq_len);
+        nch = (qlen + Qc - 1) / Qc;
+      }
+      int32_t tot = 0;
+      const int32_t eb = ecarry + block_exclusive_scan(nch, warp_buf, &tot);
+      for (int j = 0; j < nch; ++j) {
+        const int e = eb + j;
+        if (e >= p.num_rows) {  // overlapping query ranges: more chunks than rows
+          flag_error(p.err, PA_DEVERR_BAD_SEQLEN);
+          break;
+        }
+        const int32_t nq = min(Qc, qlen - j * Qc);
+        p.ent_b[e] = b;
+        p.ent_q0[e] = q0 + j * Qc;
+        p.ent_nq[e] = nq;
+        p.ent_tok[e] = max(0, min(L, L - qlen + j * Qc + nq));
+        for (int r = 0; r < nq; ++r) p.q_entry[q0 + j * Qc + r] = e;
+      }
+      ecarry += tot;
+    }
+    E = min(ecarry, p.num_rows);
+    __syncthreads();  // the entries are read back below
+  }
   // ---- packs: aligned windows b = P w .. P w + P - 1 over their shared
   // prefix; a window whose members do not all share one (or the shorter last
   // window) falls back to the aligned pairs inside it
@@ -281,14 +338,19 @@ __global__ void __launch_bounds__(kPlanThreads) pa_plan_kernel(DecodeParams p) {
     }
     __syncthreads();  // the pack arrays are read back below
   }
-  if (tid == 0) p.meta[0] = K;
-  const int E = K + B;  // entries: the packs' prefixes, then the sequences
+  if (!multi) E = K + B;  // entries: the packs' prefixes, then the sequences
+  if (tid == 0) {
+    p.meta[0] = K;
+    p.meta[1] = E;
+  }
   const int nchunks = (E + kPlanThreads - 1) / kPlanThreads;
   int32_t carry = 0, total = 0;
   for (int ch = 0; ch < nchunks; ++ch) {
     const int e = ch * kPlanThreads + tid;
     int32_t nt = 0;
-    if (e < K) {
+    if (multi) {
+      if (e < E) nt = (p.ent_tok[e] + kTile - 1) / kTile;
+    } else if (e < K) {
       nt = p.pack_tiles[e];
     } else if (e < E) {
       const int b = e - K;
@@ -460,7 +522,7 @@ __global__ void __launch_bounds__((HG * CG + 1) * 32, 1)
   griddep_launch_dependents();
   griddep_wait();  // the plan (and all earlier work on the stream) is complete
 
-  const int E = p.meta[0] + B;  // entries: packs' prefixes, then sequences
+  const int E = p.meta[1];  // entries: packs' prefixes then sequences, or query chunks
   const int64_t N = p.plan_tiles[E];
   const int64_t lo = static_cast<int64_t>(c) * N / C;
   const int64_t hi = static_cast<int64_t>(c + 1) * N / C;
@@ -474,28 +536,41 @@ __global__ void __launch_bounds__((HG * CG + 1) * 32, 1)
     const int TB = p.tok_box;
     const uint32_t box_bytes = static_cast<uint32_t>(HG * DCT * TB * 128);
     const int bpt = bs < kTile ? kTile / bs : 1;  // blocks per tile
-    const int K = E - B;
+    const int K = p.meta[0];
     // the entry being walked: tiles t_first .. t_first + n_e - 1 of the line,
     // which are tiles i0 .. i0 + n_e - 1 of sequence b (of every pack member)
     int e = p.start_seq[c];
     int b = 0, members = 1;
     int32_t t_first = 0, n_e = 0, i0 = 0, L_b = 0, seg_e = 0, nseg_e = 0;
+    int32_t qrow0 = 0, lim0 = 0;  // first query row; causal: position of query 0
+    bool pack = false;
     const int32_t* row = p.block_tables;
     auto enter = [&](int ent) {
       t_first = p.plan_tiles[ent];
       n_e = p.plan_tiles[ent + 1] - t_first;
       seg_e = p.seg_base[ent];
       nseg_e = p.seg_base[ent + 1] - seg_e;
-      if (ent < K) {
+      pack = false;
+      if (p.q_start != nullptr) {
+        b = p.ent_b[ent];
+        members = p.ent_nq[ent];
+        i0 = 0;
+        L_b = p.ent_tok[ent];
+        qrow0 = p.ent_q0[ent];
+        lim0 = L_b - members;
+      } else if (ent < K) {
         b = p.pack_first[ent];
         members = p.pack_n[ent];
         i0 = 0;
         L_b = n_e * kTile;
+        qrow0 = b;
+        pack = true;
       } else {
         b = ent - K;
         members = 1;
         i0 = p.pack_size > 1 ? p.seq_pre[b] : 0;
         L_b = clamp_len(p.seq_lens[b], p.max_seq_len);
+        qrow0 = b;
       }
       row = p.block_tables + static_cast<int64_t>(b) * p.table_stride;
     };
@@ -538,7 +613,9 @@ __global__ void __launch_bounds__((HG * CG + 1) * 32, 1)
         ++k;
       }
       if (t == seg_hi - 1) flags |= kSegEnd;
-      if (nseg_e == 1 && members == 1 && i0 == 0) flags |= kDirect;
+      // one segment holds the whole attention of every query row of the entry
+      if (nseg_e == 1 && !pack && i0 == 0) flags |= kDirect;
+      if (p.q_start != nullptr) flags |= kCausal;
       new_seq = false;
 
       uint32_t mask = valid >= kTile ? 0xffffu : ((1u << valid) - 1u);
@@ -553,7 +630,7 @@ __global__ void __launch_bounds__((HG * CG + 1) * 32, 1)
           if (tok0 >= valid) break;
           const int64_t idx = static_cast<int64_t>(ti_seq) * bpt + k;
           const int32_t id = __ldg(row + idx);
-          if (members > 1) check_shared(idx, id);
+          if (pack) check_shared(idx, id);
           if (id < 0 || id >= p.num_blocks) {
             flag_error(p.err, PA_DEVERR_BAD_BLOCK);
             mask &= ~(((1u << bs) - 1u) << tok0);
@@ -568,7 +645,7 @@ __global__ void __launch_bounds__((HG * CG + 1) * 32, 1)
       } else {
         const int64_t tok = static_cast<int64_t>(ti_seq) * kTile;
         const int32_t id = __ldg(row + tok / bs);
-        if (members > 1) check_shared(tok / bs, id);
+        if (pack) check_shared(tok / bs, id);
         tok_off[0] = static_cast<int32_t>(tok % bs);
         if (id < 0 || id >= p.num_blocks) {
           flag_error(p.err, PA_DEVERR_BAD_BLOCK);
@@ -587,6 +664,8 @@ __global__ void __launch_bounds__((HG * CG + 1) * 32, 1)
       ti.seg = seg_e + k;
       ti.flags = flags;
       ti.members = members;
+      ti.qrow0 = qrow0;
+      ti.rel = lim0 - ti_seq * kTile;
       mbar_arrive_expect_tx(full_k(stage), bytes);
       mbar_arrive_expect_tx(full_v(stage), bytes);
       const uint32_t kdst = smem_base + static_cast<uint32_t>(stage) * 2u * kTileBytes;
@@ -688,12 +767,14 @@ __global__ void __launch_bounds__((HG * CG + 1) * 32, 1)
     if (ti.flags & kNewSeq) {
 #pragma unroll
       for (int nb = 0; nb < NB; ++nb) {
-        // column c: query head c % G of pack member c / G (sequence b + member)
+        // column c: query head c % G of query row qrow0 + c / G (a pack
+        // member, or one of a sequence's query tokens)
         const int col = col0 + 8 * nb + grp;
         const int member = col / G;
         const uint16_t* qb =
             p.query +
-            ((static_cast<int64_t>(ti.b) + member) * p.num_q_heads + kvh * G + (col - member * G)) *
+            ((static_cast<int64_t>(ti.qrow0) + member) * p.num_q_heads + kvh * G +
+             (col - member * G)) *
                 D;
 #pragma unroll
         for (int kc = 0; kc < KSTEPS; ++kc) {
@@ -798,15 +879,25 @@ __global__ void __launch_bounds__((HG * CG + 1) * 32, 1)
     // ---- online softmax (base 2), masked by selection, per n8 block
     const uint32_t mask = static_cast<uint32_t>(ti.mask);
     const bool ok0 = (mask >> grp) & 1u, ok1 = (mask >> (grp + 8)) & 1u;
+    const bool causal = (ti.flags & kCausal) != 0;
     uint32_t pb0[NB], pb1[NB], pc0[NB], pc1[NB];
 #pragma unroll
     for (int nb = 0; nb < NB; ++nb) {
       if (nb == 1 && !act1) continue;
       float* sv = s[nb];
-      sv[0] = ok0 ? sv[0] * sl2 : -INFINITY;
-      sv[1] = ok0 ? sv[1] * sl2 : -INFINITY;
-      sv[2] = ok1 ? sv[2] * sl2 : -INFINITY;
-      sv[3] = ok1 ? sv[3] * sl2 : -INFINITY;
+      bool okA0 = ok0, okB0 = ok0, okA1 = ok1, okB1 = ok1;
+      if (causal) {  // columns 2q, 2q+1 see tile rows up to rel + column / G
+        const int cA = col0 + 8 * nb + 2 * quad;
+        const int limA = ti.rel + cA / G, limB = ti.rel + (cA + 1) / G;
+        okA0 = okA0 && grp <= limA;
+        okB0 = okB0 && grp <= limB;
+        okA1 = okA1 && grp + 8 <= limA;
+        okB1 = okB1 && grp + 8 <= limB;
+      }
+      sv[0] = okA0 ? sv[0] * sl2 : -INFINITY;
+      sv[1] = okB0 ? sv[1] * sl2 : -INFINITY;
+      sv[2] = okA1 ? sv[2] * sl2 : -INFINITY;
+      sv[3] = okB1 ? sv[3] * sl2 : -INFINITY;
       float mx0 = fmaxf(sv[0], sv[2]), mx1 = fmaxf(sv[1], sv[3]);
 #pragma unroll
       for (int o = 4; o < 32; o <<= 1) {
@@ -913,18 +1004,20 @@ __global__ void __launch_bounds__((HG * CG + 1) * 32, 1)
         const float inv0 = l0 > 0.f ? v_scale / l0 : 0.f;
         const float inv1 = l1 > 0.f ? v_scale / l1 : 0.f;
         const int h0 = cb + 2 * quad, h1 = h0 + 1;  // this lane's two columns
-        if (ti.flags & kDirect) {  // one sequence: columns are its query heads
-          const int64_t obase = (static_cast<int64_t>(ti.b) * p.num_q_heads + kvh * G) * D;
+        if (ti.flags & kDirect) {  // the whole attention of the entry's rows
 #pragma unroll
           for (int mt = 0; mt < MTILES; ++mt) {
             const int d0 = d_of(mt, 0), d1 = d_of(mt, 1);
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
-              const int h = hh ? h1 : h0;
-              if (h >= G) continue;
+              const int h = hh ? h1 : h0;  // column: row qrow0 + h / G, head h % G
+              if (h >= ncol) continue;
               const float inv = hh ? inv1 : inv0;
               const float v0 = acc[nb][mt][hh] * inv, v1 = acc[nb][mt][2 + hh] * inv;
-              const int64_t o = obase + static_cast<int64_t>(h) * D;
+              const int r = h / G;
+              const int64_t o =
+                  ((static_cast<int64_t>(ti.qrow0) + r) * p.num_q_heads + kvh * G + (h - r * G)) *
+                  D;
               if (p.out_dtype == PA_F32) {
                 float* op = static_cast<float*>(p.out);
                 op[o + d0] = v0;
@@ -984,6 +1077,43 @@ __global__ void __launch_bounds__((HG * CG + 1) * 32, 1)
 // found with the lanes spread over partials, then the lanes (spread over
 // head_dim) stream the partial outputs with no dependence between partials.
 // ---------------------------------------------------------------------------
+// The partials of output row r, query head h (h inside its KV head's group):
+// those of its own entry (slots s0 .., column col0) and, for a pack member,
+// those of the pack's entry (slots s1 .., column col1).  direct: the main
+// kernel wrote the row itself.  valid: the row belongs to an entry.
+struct RowParts {
+  int32_t s0, ns, col0, s1, np, col1;
+  bool direct, valid;
+};
+
+__device__ __forceinline__ RowParts row_parts(const DecodeParams& p, int r, int h) {
+  RowParts q;
+  q.s1 = q.np = q.col1 = 0;
+  q.valid = true;
+  if (p.q_start != nullptr) {  // query chunks: row r is column (r - first row) * G + h
+    const int e = p.q_entry[r];
+    q.valid = e >= 0 && e < p.meta[1];
+    const int ee = q.valid ? e : 0;
+    q.s0 = p.seg_base[ee];
+    q.ns = p.seg_base[ee + 1] - q.s0;
+    q.col0 = (r - p.ent_q0[ee]) * p.group + h;
+    q.direct = q.ns == 1;
+    return q;
+  }
+  const int K = p.meta[0];
+  q.s0 = p.seg_base[K + r];
+  q.ns = p.seg_base[K + r + 1] - q.s0;
+  q.col0 = h;
+  const int pk = p.pack_size > 1 ? p.seq_pack[r] : -1;
+  q.direct = pk < 0 && q.ns == 1;
+  if (pk >= 0) {
+    q.s1 = p.seg_base[pk];
+    q.np = p.seg_base[pk + 1] - q.s1;
+    q.col1 = (r - p.pack_first[pk]) * p.group + h;
+  }
+  return q;
+}
+
 template <int D>
 __global__ void __launch_bounds__(kCombineWarps * 32) pa_combine_narrow_kernel(const DecodeParams p) {
   constexpr int V = D / 32;  // floats per lane
@@ -995,23 +1125,15 @@ __global__ void __launch_bounds__(kCombineWarps * 32) pa_combine_narrow_kernel(c
   const int G = p.group, HG = p.heads_per_cta;
   const int kvh = qh / G, h = qh - kvh * G;
   const int hg = kvh / HG, g = kvh - hg * HG;
-  const int K = p.meta[0];
-  const int32_t s0 = p.seg_base[K + b], ns = p.seg_base[K + b + 1] - s0;
-  const int pk = p.pack_size > 1 ? p.seq_pack[b] : -1;
-  if (pk < 0 && ns == 1) return;  // the main kernel wrote this sequence directly
-  // partial k: k < ns from the sequence's entry, then the pack's
-  int32_t s1 = 0, np = 0, col1 = 0;
-  if (pk >= 0) {
-    s1 = p.seg_base[pk];
-    np = p.seg_base[pk + 1] - s1;
-    col1 = (b - p.pack_first[pk]) * G + h;
-  }
-  const int32_t nseq = (s0 + ns <= p.nseg_cap) ? ns : 0;
-  const int32_t npack = (s1 + np <= p.nseg_cap) ? np : 0;
+  const RowParts rp = row_parts(p, b, h);
+  if (rp.direct || !rp.valid) return;  // written by the main kernel (or no entry)
+  // partial k: k < ns from the row's own entry, then the pack's
+  const int32_t nseq = (rp.s0 + rp.ns <= p.nseg_cap) ? rp.ns : 0;
+  const int32_t npack = (rp.s1 + rp.np <= p.nseg_cap) ? rp.np : 0;
   const int32_t ntot = nseq + npack;
   auto row_of = [&](int32_t k) {
-    const int32_t slot = k < nseq ? s0 + k : s1 + (k - nseq);
-    const int col = k < nseq ? h : col1;
+    const int32_t slot = k < nseq ? rp.s0 + k : rp.s1 + (k - nseq);
+    const int col = k < nseq ? rp.col0 : rp.col1;
     return ((static_cast<int64_t>(hg) * p.nseg_cap + slot) * HG + g) * p.cols + col;
   };
   const int64_t obase = (static_cast<int64_t>(b) * p.num_q_heads + qh) * D + lane * V;
@@ -1080,22 +1202,14 @@ __global__ void __launch_bounds__(kCombineWarps * 32) pa_combine_wide_kernel(con
   const int G = p.group, HG = p.heads_per_cta;
   const int kvh = qh / G, h = qh - kvh * G;
   const int hg = kvh / HG, g = kvh - hg * HG;
-  const int K = p.meta[0];
-  const int32_t s0 = p.seg_base[K + b], ns = p.seg_base[K + b + 1] - s0;
-  const int pk = p.pack_size > 1 ? p.seq_pack[b] : -1;
-  if (pk < 0 && ns == 1) return;  // the main kernel wrote this sequence directly
-  int32_t s1 = 0, np = 0, col1 = 0;
-  if (pk >= 0) {
-    s1 = p.seg_base[pk];
-    np = p.seg_base[pk + 1] - s1;
-    col1 = (b - p.pack_first[pk]) * G + h;
-  }
-  const int32_t nseq = (s0 + ns <= p.nseg_cap) ? ns : 0;
-  const int32_t npack = (s1 + np <= p.nseg_cap) ? np : 0;
+  const RowParts rp = row_parts(p, b, h);
+  if (rp.direct || !rp.valid) return;  // written by the main kernel (or no entry)
+  const int32_t nseq = (rp.s0 + rp.ns <= p.nseg_cap) ? rp.ns : 0;
+  const int32_t npack = (rp.s1 + rp.np <= p.nseg_cap) ? rp.np : 0;
   const int32_t ntot = nseq + npack;
   auto row_of = [&](int32_t k) {  // partial k: own entry's first, then the pack's
-    const int32_t slot = k < nseq ? s0 + k : s1 + (k - nseq);
-    const int col = k < nseq ? h : col1;
+    const int32_t slot = k < nseq ? rp.s0 + k : rp.s1 + (k - nseq);
+    const int col = k < nseq ? rp.col0 : rp.col1;
     return ((static_cast<int64_t>(hg) * p.nseg_cap + slot) * HG + g) * p.cols + col;
   };
 
@@ -1212,12 +1326,13 @@ MainKernel select_main(int D, int HG, int NB, int CG, bool bf16, bool fp8) {
 struct LaunchPlan {
   int HG = 0, groups = 0, stages = 0, tok_box = 0, threads = 0;
   int ctas_per_group = 0, tiles_per_part = INT_MAX, nseg_cap = 0;
-  int pack_size = 1, cols = 0, nb = 1, cg = 1;
+  int pack_size = 1, cols = 0, nb = 1, cg = 1, q_per_entry = 0;
+  int64_t rows = 0;  // output rows
   bool many_partials = false;  // long sequences / partitions: closed-form plan, wide combine
   size_t smem = 0;
   size_t off_tiles = 0, off_segs = 0, off_start = 0, off_firstk = 0, off_meta = 0,
          off_pack_first = 0, off_pack_n = 0, off_pack_tiles = 0, off_seq_pack = 0,
-         off_seq_pre = 0, off_o = 0, off_ml = 0, total = 0;
+         off_seq_pre = 0, off_ent = 0, off_o = 0, off_ml = 0, total = 0;
   MainKernel kernel = nullptr;
 };
 
@@ -1230,9 +1345,13 @@ bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
 // each take a column: 16 columns per consumer warp, two warps per KV head when
 // more than 16 are needed.  Otherwise every sequence is its own entry and a
 // warp holds one KV head's group columns.
+// max_q_len > 0: several query tokens per sequence (num_rows query rows in
+// all): entries are chunks of up to min(max_q_len, 32 / group) of them, whose
+// group-many heads each take a column.
 pa_status make_plan(int32_t num_seqs, int32_t Hq, int32_t Hkv, int32_t D, int32_t bs,
                     int32_t max_seq_len, int32_t partition_size, bool bf16, bool fp8,
-                    bool shared_prefix, LaunchPlan* lp) {
+                    bool shared_prefix, LaunchPlan* lp, int32_t max_q_len = 0,
+                    int64_t num_rows = 0) {
   if (num_seqs < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || bs <= 0 || max_seq_len < 0 ||
       partition_size < 0)
     return PA_ERR_INVALID_ARG;
@@ -1243,8 +1362,15 @@ pa_status make_plan(int32_t num_seqs, int32_t Hq, int32_t Hkv, int32_t D, int32_
   if (G > 8) return PA_ERR_UNSUPPORTED;
   if (partition_size > 0 && (partition_size % kTile != 0 || partition_size % bs != 0))
     return PA_ERR_INVALID_ARG;
-  int P = 1, NB = 1, CG = 1;
-  if (shared_prefix && !fp8) {
+  int P = 1, NB = 1, CG = 1, Qc = 0;
+  if (max_q_len < 0 || num_rows < 0 || num_rows > INT_MAX / 2) return PA_ERR_INVALID_ARG;
+  if (max_q_len > 0) {
+    if (fp8 || shared_prefix) return PA_ERR_UNSUPPORTED;
+    Qc = kMaxPackCols / G < max_q_len ? kMaxPackCols / G : max_q_len;
+    const int need = Qc * G;  // columns of a whole chunk
+    NB = need > 8 ? 2 : 1;
+    CG = (need + 8 * NB - 1) / (8 * NB);
+  } else if (shared_prefix && !fp8) {
     P = kMaxPackCols / G < kMaxPack ? kMaxPackCols / G : kMaxPack;
     if (P < 2) P = 1;
     const int need = P * G;  // columns of a whole pack
@@ -1291,15 +1417,19 @@ pa_status make_plan(int32_t num_seqs, int32_t Hq, int32_t Hkv, int32_t D, int32_
     if (parts_per_seq < 1) parts_per_seq = 1;
   }
   lp->pack_size = P;
-  lp->cols = P > 1 ? 8 * NB * CG : G;
-  // entries: at most num_seqs / 2 packs (pairs), then the sequences
+  lp->q_per_entry = Qc;
+  lp->rows = Qc > 0 ? num_rows : num_seqs;
+  lp->cols = (P > 1 || Qc > 0) ? 8 * NB * CG : G;
+  // entries: at most num_seqs / 2 packs (pairs), then the sequences; or at
+  // most one chunk per query row
   const int64_t max_packs = P > 1 ? num_seqs / 2 : 0;
-  const int64_t entries = static_cast<int64_t>(num_seqs) + max_packs;
+  const int64_t entries = Qc > 0 ? num_rows : static_cast<int64_t>(num_seqs) + max_packs;
   const int64_t nseg = entries * parts_per_seq + lp->ctas_per_group;
   // partials one sequence expects: its partitions plus the CTA shares it spans
   // when the batch's work is cut evenly
-  const int64_t expect = parts_per_seq + (lp->ctas_per_group + num_seqs - 1) /
-                                             (num_seqs > 0 ? num_seqs : 1);
+  const int64_t units = Qc > 0 ? (num_rows + Qc - 1) / Qc : num_seqs;  // entries, roughly
+  const int64_t expect = parts_per_seq + (lp->ctas_per_group + units - 1) /
+                                             (units > 0 ? units : 1);
   lp->many_partials = expect > 6;
   if (nseg > INT_MAX / 2) return PA_ERR_UNSUPPORTED;
   lp->nseg_cap = static_cast<int>(nseg);
@@ -1309,7 +1439,7 @@ pa_status make_plan(int32_t num_seqs, int32_t Hq, int32_t Hkv, int32_t D, int32_
   lp->off_start = lp->off_segs + words(entries + 1);
   lp->off_firstk = lp->off_start + words(lp->ctas_per_group);
   lp->off_meta = lp->off_firstk + words(lp->ctas_per_group);
-  size_t off = lp->off_meta + words(1);
+  size_t off = lp->off_meta + words(2);
   if (lp->pack_size > 1) {
     lp->off_pack_first = off;
     lp->off_pack_n = lp->off_pack_first + words(max_packs + 1);
@@ -1317,6 +1447,10 @@ pa_status make_plan(int32_t num_seqs, int32_t Hq, int32_t Hkv, int32_t D, int32_
     lp->off_seq_pack = lp->off_pack_tiles + words(max_packs + 1);
     lp->off_seq_pre = lp->off_seq_pack + words(num_seqs);
     off = lp->off_seq_pre + words(num_seqs);
+  }
+  if (Qc > 0) {  // ent_b, ent_q0, ent_nq, ent_tok, q_entry: one row each
+    lp->off_ent = off;
+    off = lp->off_ent + 5 * words(num_rows);
   }
   lp->off_o = off;
   const size_t o_bytes = static_cast<size_t>(lp->groups) * nseg * HG * lp->cols * D * sizeof(float);
@@ -1337,14 +1471,15 @@ namespace {
 // The larger of the 16-bit and the fp8-cache plans of one shape.
 pa_status workspace_bytes(int32_t num_seqs, int32_t Hq, int32_t Hkv, int32_t D, int32_t bs,
                           int32_t max_seq_len, int32_t partition_size, bool shared_prefix,
-                          size_t* bytes) {
+                          size_t* bytes, int32_t max_q_len = 0, int64_t num_rows = 0) {
   LaunchPlan lp;
   const pa_status st = make_plan(num_seqs, Hq, Hkv, D, bs, max_seq_len, partition_size, true,
-                                 false, shared_prefix, &lp);
+                                 false, shared_prefix, &lp, max_q_len, num_rows);
   if (st != PA_OK) return st;
   *bytes = lp.total;
   LaunchPlan lp8;
-  if (make_plan(num_seqs, Hq, Hkv, D, bs, max_seq_len, partition_size, false, true,
+  if (max_q_len == 0 &&
+      make_plan(num_seqs, Hq, Hkv, D, bs, max_seq_len, partition_size, false, true,
                 shared_prefix, &lp8) == PA_OK &&
       lp8.total > *bytes)
     *bytes = lp8.total;
@@ -1360,6 +1495,15 @@ extern "C" pa_status pa_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_h
   if (bytes == nullptr) return PA_ERR_INVALID_ARG;
   return workspace_bytes(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
                          max_seq_len, partition_size, false, bytes);
+}
+
+extern "C" pa_status pa_decode_multi_query_workspace_bytes(
+    int32_t num_seqs, int32_t num_query_rows, int32_t max_q_len, int32_t num_q_heads,
+    int32_t num_kv_heads, int32_t head_dim, int32_t block_size, int32_t max_seq_len,
+    int32_t partition_size, size_t* bytes) {
+  if (bytes == nullptr || max_q_len <= 0 || num_query_rows < 0) return PA_ERR_INVALID_ARG;
+  return workspace_bytes(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
+                         max_seq_len, partition_size, false, bytes, max_q_len, num_query_rows);
 }
 
 extern "C" pa_status pa_decode_shared_prefix_workspace_bytes(
@@ -1383,9 +1527,12 @@ pa_status launch_decode(void* out, pa_dtype out_dtype, const void* query, pa_dty
                         int32_t num_blocks, int32_t block_size, float scale,
                         int32_t partition_size, const int32_t* shared_blocks, void* workspace,
                         size_t workspace_bytes, int32_t* device_error_flag, pa_stream_t stream,
-                        const pa_cache_strides* cache_strides = nullptr) {
-  if (num_seqs < 0) return PA_ERR_INVALID_ARG;
-  if (num_seqs == 0) return PA_OK;
+                        const pa_cache_strides* cache_strides = nullptr,
+                        const int32_t* q_start = nullptr, int32_t num_rows = 0,
+                        int32_t max_q_len = 0) {
+  if (num_seqs < 0 || num_rows < 0) return PA_ERR_INVALID_ARG;
+  if (num_seqs == 0 || (q_start != nullptr && num_rows == 0)) return PA_OK;
+  if (q_start != nullptr && (max_q_len <= 0 || !aligned(q_start, 4))) return PA_ERR_INVALID_ARG;
   if (!out || !query || !key_cache || !value_cache || !block_tables || !seq_lens || !workspace)
     return PA_ERR_INVALID_ARG;
   const bool fp8 = elem_bytes == 1;
@@ -1399,7 +1546,8 @@ pa_status launch_decode(void* out, pa_dtype out_dtype, const void* query, pa_dty
   if (shared_blocks != nullptr && !aligned(shared_blocks, 4)) return PA_ERR_INVALID_ARG;
   pa_status st = make_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
                            max_seq_len, partition_size, !fp8 && q_dtype == PA_BF16, fp8,
-                           shared_blocks != nullptr, &lp);
+                           shared_blocks != nullptr, &lp, q_start != nullptr ? max_q_len : 0,
+                           num_rows);
   if (st != PA_OK) return st;
   const int64_t need_blocks = (static_cast<int64_t>(max_seq_len) + block_size - 1) / block_size;
   if (block_table_stride < need_blocks) return PA_ERR_INVALID_ARG;
@@ -1460,6 +1608,7 @@ pa_status launch_decode(void* out, pa_dtype out_dtype, const void* query, pa_dty
   p.table_stride = block_table_stride;
   p.out_dtype = out_dtype;
   p.num_seqs = num_seqs;
+  p.num_rows = static_cast<int32_t>(lp.rows);
   p.max_seq_len = max_seq_len;
   p.num_q_heads = num_q_heads;
   p.group = num_q_heads / num_kv_heads;
@@ -1479,6 +1628,16 @@ pa_status launch_decode(void* out, pa_dtype out_dtype, const void* query, pa_dty
   p.start_seq = reinterpret_cast<int32_t*>(ws + lp.off_start);
   p.first_k = reinterpret_cast<int32_t*>(ws + lp.off_firstk);
   p.meta = reinterpret_cast<int32_t*>(ws + lp.off_meta);
+  if (q_start != nullptr) {
+    p.q_start = q_start;
+    p.q_per_entry = lp.q_per_entry;
+    const size_t w = align_up(static_cast<size_t>(lp.rows) * 4, 256);
+    p.ent_b = reinterpret_cast<int32_t*>(ws + lp.off_ent);
+    p.ent_q0 = reinterpret_cast<int32_t*>(ws + lp.off_ent + w);
+    p.ent_nq = reinterpret_cast<int32_t*>(ws + lp.off_ent + 2 * w);
+    p.ent_tok = reinterpret_cast<int32_t*>(ws + lp.off_ent + 3 * w);
+    p.q_entry = reinterpret_cast<int32_t*>(ws + lp.off_ent + 4 * w);
+  }
   p.shared_blocks = shared_blocks;
   p.pack_size = lp.pack_size;
   p.cols = lp.cols;
@@ -1506,11 +1665,13 @@ pa_status launch_decode(void* out, pa_dtype out_dtype, const void* query, pa_dty
     return PA_ERR_CUDA;
   cudaError_t e3;
   if (lp.many_partials) {
-    PdlLaunch combine(s, dim3(num_seqs, num_q_heads), dim3(kCombineWarps * 32));
+    PdlLaunch combine(s, dim3(static_cast<unsigned>(lp.rows), num_q_heads),
+                      dim3(kCombineWarps * 32));
     e3 = D == 128 ? combine(pa_combine_wide_kernel<128>, p)
                   : combine(pa_combine_wide_kernel<64>, p);
   } else {
-    PdlLaunch combine(s, dim3(num_seqs, (num_q_heads + kCombineWarps - 1) / kCombineWarps),
+    PdlLaunch combine(s, dim3(static_cast<unsigned>(lp.rows),
+                           (num_q_heads + kCombineWarps - 1) / kCombineWarps),
                       dim3(kCombineWarps * 32));
     e3 = D == 128 ? combine(pa_combine_narrow_kernel<128>, p)
                   : combine(pa_combine_narrow_kernel<64>, p);
@@ -1567,6 +1728,22 @@ extern "C" pa_status pa_decode_attention_strided(
                        num_kv_heads, head_dim, num_blocks, block_size, scale, partition_size,
                        nullptr, workspace, workspace_bytes, device_error_flag, stream,
                        cache_strides);
+}
+
+extern "C" pa_status pa_decode_attention_multi_query(
+    void* out, pa_dtype out_dtype, const void* query, const int32_t* q_start,
+    int32_t num_query_rows, int32_t max_q_len, const void* key_cache, const void* value_cache,
+    const int32_t* block_tables, int32_t block_table_stride, const int32_t* seq_lens,
+    int32_t num_seqs, int32_t max_seq_len, int32_t num_q_heads, int32_t num_kv_heads,
+    int32_t head_dim, int32_t num_blocks, int32_t block_size, float scale, pa_dtype kv_dtype,
+    int32_t partition_size, void* workspace, size_t workspace_bytes,
+    int32_t* device_error_flag, pa_stream_t stream) {
+  if (q_start == nullptr && num_seqs > 0) return PA_ERR_INVALID_ARG;
+  return launch_decode(out, out_dtype, query, kv_dtype, key_cache, value_cache, 2, nullptr,
+                       nullptr, block_tables, block_table_stride, seq_lens, num_seqs,
+                       max_seq_len, num_q_heads, num_kv_heads, head_dim, num_blocks, block_size,
+                       scale, partition_size, nullptr, workspace, workspace_bytes,
+                       device_error_flag, stream, nullptr, q_start, num_query_rows, max_q_len);
 }
 
 extern "C" pa_status pa_decode_attention_shared_prefix(
