@@ -209,6 +209,8 @@ def reshape_and_cache(key: torch.Tensor, value: torch.Tensor, key_cache: torch.T
     _need(kv_cache_dtype in _KV_CACHE_DTYPE, "kv_cache_dtype must be 'auto' or 'fp8_e4m3'")
     fp8 = _KV_CACHE_DTYPE[kv_cache_dtype] == 1
     _need(key.dim() == 3 and value.shape == key.shape, "key/value must be [T, Hkv, D]")
+    _need(key_cache.dim() == 4 and tuple(key.shape[1:]) == tuple(key_cache.shape[2:]),
+          "key/value rows [Hkv, D] must match the pools' [.., Hkv, D]")
     _need(key.stride(2) == 1 and key.stride(1) == key.shape[2] and
           value.stride(2) == 1 and value.stride(1) == value.shape[2],
           "heads and head_dim must be contiguous inside a row")
@@ -311,6 +313,7 @@ def decode_attention(out: torch.Tensor, query: torch.Tensor, key_cache: torch.Te
     _need(query.dtype == key_cache.dtype == value_cache.dtype, "query and caches share a dtype")
     B, hq, d = query.shape
     nb, bs, hkv, _ = key_cache.shape
+    _need(key_cache.shape[3] == d, "query and pools must share head_dim")
     if workspace is None:
         workspace = alloc_workspace(decode_workspace_bytes(B, hq, hkv, d, bs, max_seq_len,
                                                            partition_size), query.device)
@@ -353,6 +356,7 @@ def decode_attention_fp8(out: torch.Tensor, query: torch.Tensor, key_cache: torc
     _need(seq_lens.dtype == torch.int32 and seq_lens.is_contiguous(), "seq_lens int32")
     B, hq, d = query.shape
     nb, bs, hkv, _ = key_cache.shape
+    _need(key_cache.shape[3] == d, "query and pools must share head_dim")
     if workspace is None:
         workspace = alloc_workspace(decode_workspace_bytes(B, hq, hkv, d, bs, max_seq_len,
                                                            partition_size), query.device)
@@ -400,6 +404,7 @@ def decode_attention_shared_prefix(out: torch.Tensor, query: torch.Tensor,
     _need(query.dtype == key_cache.dtype == value_cache.dtype, "query and caches share a dtype")
     B, hq, d = query.shape
     nb, bs, hkv, _ = key_cache.shape
+    _need(key_cache.shape[3] == d, "query and pools must share head_dim")
     if workspace is None:
         workspace = alloc_workspace(shared_prefix_workspace_bytes(
             B, hq, hkv, d, bs, max_seq_len, partition_size), query.device)
@@ -448,6 +453,7 @@ def decode_attention_multi_query(out: torch.Tensor, query: torch.Tensor, q_start
     T, hq, d = query.shape
     B = seq_lens.numel()
     nb, bs, hkv, _ = key_cache.shape
+    _need(key_cache.shape[3] == d, "query and pools must share head_dim")
     if workspace is None:
         workspace = alloc_workspace(multi_query_workspace_bytes(
             B, T, int(max_q_len), hq, hkv, d, bs, int(max_seq_len), partition_size), query.device)
@@ -477,6 +483,7 @@ def decode_attention_noalloc(out: torch.Tensor, query: torch.Tensor, key_cache: 
     array and race; the first call on a device should precede stream capture."""
     B, hq, d = query.shape
     nb, bs, hkv, _ = key_cache.shape
+    _need(key_cache.shape[3] == d, "query and pools must share head_dim")
     _check(lib.pa_decode_attention_noalloc(
         _ptr(out), _DTYPE_CODE[out.dtype], _ptr(query), _ptr(key_cache), _ptr(value_cache),
         _ptr(block_tables), block_tables.stride(0), _ptr(seq_lens), B, int(max_seq_len), hq, hkv,

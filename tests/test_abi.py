@@ -157,3 +157,21 @@ def test_shared_prefix_host_validation(pa):
     assert lib.pa_decode_attention_shared_prefix(None, 1, None, None, None, None, 1, None, None,
                                                  0, 16, 4, 2, 64, 8, 4, 0.125, 1, 0, None, 0,
                                                  None, None) == 0
+
+
+def test_binding_refuses_mismatched_head_dim(pa):
+    """Pools whose head_dim differs from the query's are refused before any
+    pointer reaches the library (the C entry points take head_dim from one
+    side only)."""
+    import torch
+    q = torch.zeros(2, 8, 128, dtype=torch.bfloat16)
+    k = torch.zeros(4, 16, 2, 64, dtype=torch.bfloat16)
+    tables = torch.zeros(2, 8, dtype=torch.int32)
+    lens = torch.ones(2, dtype=torch.int32)
+    for fn in (pa.decode_attention, pa.decode_attention_noalloc):
+        with pytest.raises(ValueError):
+            fn(torch.empty_like(q), q, k, k, tables, lens, 16, 0.1)
+    with pytest.raises(ValueError):
+        pa.reshape_and_cache(torch.zeros(3, 2, 128, dtype=torch.bfloat16),
+                             torch.zeros(3, 2, 128, dtype=torch.bfloat16), k, k,
+                             torch.zeros(3, dtype=torch.int32))
