@@ -587,74 +587,84 @@ __global__ void __launch_bounds__((HG * CG + 1) * 32, 1)
         if (__ldg(row + static_cast<int64_t>(m) * p.table_stride + idx) != id)
           flag_error(p.err, PA_DEVERR_BAD_SHARE);
     };
+    // Tile index inside its partition: segments start at the CTA's first
+    // tile, at an entry's first tile and at every partition start, and end
+    // before the next start or at the CTA's last tile.
+    const int32_t tpp = p.tiles_per_part;
+    int32_t ip = tpp == INT_MAX ? i : i % tpp;
     for (int64_t t = lo; t < hi; ++t, ++i) {
       while (i >= n_e) {  // next entry that has tiles
         enter(++e);
         k = -1;
         i = 0;
+        ip = 0;
         new_seq = true;
       }
-      if (!mbar_wait(empty(stage), phase ^ 1u, p.err)) break;
-
       const int32_t ti_seq = i0 + i;  // tile index inside the sequence
       const int32_t valid = min(kTile, L_b - ti_seq * kTile);
-      const int32_t j = (p.tiles_per_part == INT_MAX) ? 0 : i / p.tiles_per_part;
-      const int64_t part_lo = t_first + static_cast<int64_t>(j) *
-                                            (p.tiles_per_part == INT_MAX ? 0 : p.tiles_per_part);
-      const int64_t part_hi = (p.tiles_per_part == INT_MAX)
-                                  ? t_first + n_e
-                                  : min(static_cast<int64_t>(t_first) + n_e,
-                                        part_lo + p.tiles_per_part);
-      const int64_t seg_lo = max(part_lo, lo), seg_hi = min(part_hi, hi);
-      int32_t flags = 0;
-      if (new_seq) flags |= kNewSeq;
-      if (t == seg_lo) {
+      int32_t flags = new_seq ? kNewSeq : 0;
+      if (t == lo || ip == 0) {
         flags |= kSegStart;
         ++k;
       }
-      if (t == seg_hi - 1) flags |= kSegEnd;
+      if (t == hi - 1 || i == n_e - 1 || ip == tpp - 1) flags |= kSegEnd;
       // one segment holds the whole attention of every query row of the entry
       if (nseg_e == 1 && !pack && i0 == 0) flags |= kDirect;
       if (p.q_start != nullptr) flags |= kCausal;
       new_seq = false;
-
+      if (++ip == tpp) ip = 0;
       uint32_t mask = valid >= kTile ? 0xffffu : ((1u << valid) - 1u);
-      // block-table lookups first, so the expected byte count is known
-      int32_t phys[kTile / 4];
-      int32_t tok_off[kTile / 4];
-      int nbox = 0;
-      uint32_t bytes = 0;
-      if (bs <= kTile) {
-        for (int k = 0; k < bpt; ++k) {
-          const int tok0 = k * bs;
-          if (tok0 >= valid) break;
-          const int64_t idx = static_cast<int64_t>(ti_seq) * bpt + k;
-          const int32_t id = __ldg(row + idx);
-          if (pack) check_shared(idx, id);
-          if (id < 0 || id >= p.num_blocks) {
-            flag_error(p.err, PA_DEVERR_BAD_BLOCK);
-            mask &= ~(((1u << bs) - 1u) << tok0);
-            phys[k] = -1;
-            continue;
+      // the first block id is loaded before the wait for a free stage
+      const int64_t idx0 = bs <= kTile ? static_cast<int64_t>(ti_seq) * bpt
+                                       : static_cast<int64_t>(ti_seq) * kTile / bs;
+      const int32_t id0 = __ldg(row + idx0);
+
+      if (!mbar_wait(empty(stage), phase ^ 1u, p.err)) break;
+      const uint32_t kdst = smem_base + static_cast<uint32_t>(stage) * 2u * kTileBytes;
+      const uint32_t vdst = kdst + kTileBytes;
+      // one box per block of the tile; each copy's bytes are announced on the
+      // stage's barriers just before it is issued
+      auto issue = [&](uint32_t off, int32_t tok_off, int32_t id) {
+        mbar_expect_tx(full_k(stage), box_bytes);
+        mbar_expect_tx(full_v(stage), box_bytes);
+        if (p.tma_mode == 0) {
+          tma_load_5d(kdst + off, &tmK, full_k(stage), 0, tok_off, 0, hg * HG, id, policy);
+          tma_load_5d(vdst + off, &tmV, full_v(stage), 0, tok_off, 0, hg * HG, id, policy);
+        } else {
+          for (int hh = 0; hh < HG; ++hh) {
+            for (int dc = 0; dc < DCT; ++dc) {
+              const uint32_t o2 = off + ((hh * DCT + dc) * TB) * 128u;
+              tma_load_5d(kdst + o2, &tmK, full_k(stage), 0, dc, hg * HG + hh, tok_off, id,
+                          policy);
+              tma_load_5d(vdst + o2, &tmV, full_v(stage), 0, dc, hg * HG + hh, tok_off, id,
+                          policy);
+            }
           }
-          phys[k] = id;
-          tok_off[k] = 0;
-          nbox = k + 1;
-          bytes += box_bytes;
+        }
+      };
+      if (bs <= kTile) {
+#pragma unroll
+        for (int kk = 0; kk < kTile / 4; ++kk) {  // at most 4 blocks: block_size >= 4
+          const int tok0 = kk * bs;
+          if (kk < bpt && tok0 < valid) {
+            const int64_t idx = idx0 + kk;
+            const int32_t id = kk == 0 ? id0 : __ldg(row + idx);
+            if (pack) check_shared(idx, id);
+            if (id < 0 || id >= p.num_blocks) {
+              flag_error(p.err, PA_DEVERR_BAD_BLOCK);
+              mask &= ~(((1u << bs) - 1u) << tok0);
+            } else {
+              issue(static_cast<uint32_t>(kk) * box_bytes, 0, id);
+            }
+          }
         }
       } else {
-        const int64_t tok = static_cast<int64_t>(ti_seq) * kTile;
-        const int32_t id = __ldg(row + tok / bs);
-        if (pack) check_shared(tok / bs, id);
-        tok_off[0] = static_cast<int32_t>(tok % bs);
-        if (id < 0 || id >= p.num_blocks) {
+        if (pack) check_shared(idx0, id0);
+        if (id0 < 0 || id0 >= p.num_blocks) {
           flag_error(p.err, PA_DEVERR_BAD_BLOCK);
           mask = 0;
-          phys[0] = -1;
         } else {
-          phys[0] = id;
-          nbox = 1;
-          bytes = box_bytes;
+          issue(0, static_cast<int32_t>((static_cast<int64_t>(ti_seq) * kTile) % bs), id0);
         }
       }
       TileInfo& ti = info[stage];
@@ -665,30 +675,10 @@ __global__ void __launch_bounds__((HG * CG + 1) * 32, 1)
       ti.flags = flags;
       ti.members = members;
       ti.qrow0 = qrow0;
-      ti.rel = lim0 - ti_seq * kTile;
-      mbar_arrive_expect_tx(full_k(stage), bytes);
-      mbar_arrive_expect_tx(full_v(stage), bytes);
-      const uint32_t kdst = smem_base + static_cast<uint32_t>(stage) * 2u * kTileBytes;
-      const uint32_t vdst = kdst + kTileBytes;
-      for (int k = 0; k < nbox; ++k) {
-        if (phys[k] < 0) continue;
-        if (p.tma_mode == 0) {
-          tma_load_5d(kdst + k * box_bytes, &tmK, full_k(stage), 0, tok_off[k], 0, hg * HG,
-                      phys[k], policy);
-          tma_load_5d(vdst + k * box_bytes, &tmV, full_v(stage), 0, tok_off[k], 0, hg * HG,
-                      phys[k], policy);
-        } else {
-          for (int hh = 0; hh < HG; ++hh) {
-            for (int dc = 0; dc < DCT; ++dc) {
-              const uint32_t off = k * box_bytes + ((hh * DCT + dc) * TB) * 128u;
-              tma_load_5d(kdst + off, &tmK, full_k(stage), 0, dc, hg * HG + hh, tok_off[k],
-                          phys[k], policy);
-              tma_load_5d(vdst + off, &tmV, full_v(stage), 0, dc, hg * HG + hh, tok_off[k],
-                          phys[k], policy);
-            }
-          }
-        }
-      }
+      ti.rel = (flags & kCausal) ? lim0 - ti_seq * kTile : kTile;  // kTile: every row visible
+      // the one arrival of the phase: it completes once the announced bytes land
+      mbar_arrive(full_k(stage));
+      mbar_arrive(full_v(stage));
       ++issued;
       if (++stage == NS) { stage = 0; phase ^= 1u; }
     }
@@ -744,6 +734,13 @@ __global__ void __launch_bounds__((HG * CG + 1) * 32, 1)
     v_scale = *p.v_scale;
   }
 
+  // query row offset (column / G) of this lane's two accumulator columns
+  int cdiv[NB][2];
+#pragma unroll
+  for (int nb = 0; nb < NB; ++nb) {
+    cdiv[nb][0] = (col0 + 8 * nb + 2 * quad) / G;
+    cdiv[nb][1] = (col0 + 8 * nb + 2 * quad + 1) / G;
+  }
   uint32_t qf[NB][KSTEPS][2];
   float acc[NB][MTILES][4];
   float m_run[NB][2], l_part[NB][2];
@@ -804,8 +801,10 @@ __global__ void __launch_bounds__((HG * CG + 1) * 32, 1)
         l_part[nb][0] = l_part[nb][1] = 0.f;
       }
     }
-    // n8 blocks of this warp with at least one column (warp-uniform)
-    const bool act1 = NB > 1 && col0 + 8 < ncol;
+    // Both n8 blocks always run: a block whose columns are all beyond ncol
+    // works on zero queries and writes nothing.  A runtime test here splits
+    // the unrolled MMA loops and costs more than the work it saves.
+    constexpr bool act1 = NB > 1;
     const uint32_t kbase = smem_base + static_cast<uint32_t>(stage) * 2u * kTileBytes;
     const uint32_t vbase = kbase + kTileBytes;
     // fp8: this lane's code bytes.  K: tokens grp, grp+8, d in [32q, 32q + 32)
@@ -879,21 +878,16 @@ __global__ void __launch_bounds__((HG * CG + 1) * 32, 1)
     // ---- online softmax (base 2), masked by selection, per n8 block
     const uint32_t mask = static_cast<uint32_t>(ti.mask);
     const bool ok0 = (mask >> grp) & 1u, ok1 = (mask >> (grp + 8)) & 1u;
-    const bool causal = (ti.flags & kCausal) != 0;
     uint32_t pb0[NB], pb1[NB], pc0[NB], pc1[NB];
 #pragma unroll
     for (int nb = 0; nb < NB; ++nb) {
       if (nb == 1 && !act1) continue;
       float* sv = s[nb];
-      bool okA0 = ok0, okB0 = ok0, okA1 = ok1, okB1 = ok1;
-      if (causal) {  // columns 2q, 2q+1 see tile rows up to rel + column / G
-        const int cA = col0 + 8 * nb + 2 * quad;
-        const int limA = ti.rel + cA / G, limB = ti.rel + (cA + 1) / G;
-        okA0 = okA0 && grp <= limA;
-        okB0 = okB0 && grp <= limB;
-        okA1 = okA1 && grp + 8 <= limA;
-        okB1 = okB1 && grp + 8 <= limB;
-      }
+      // columns 2q, 2q+1 see tile rows up to rel + column / G (rel = 16 when
+      // every row is visible)
+      const int limA = ti.rel + cdiv[nb][0], limB = ti.rel + cdiv[nb][1];
+      const bool okA0 = ok0 && grp <= limA, okB0 = ok0 && grp <= limB;
+      const bool okA1 = ok1 && grp + 8 <= limA, okB1 = ok1 && grp + 8 <= limB;
       sv[0] = okA0 ? sv[0] * sl2 : -INFINITY;
       sv[1] = okB0 ? sv[1] * sl2 : -INFINITY;
       sv[2] = okA1 ? sv[2] * sl2 : -INFINITY;
