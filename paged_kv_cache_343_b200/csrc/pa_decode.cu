@@ -522,7 +522,9 @@ __global__ void __launch_bounds__((HG * CG + 1) * 32, 1)
   griddep_launch_dependents();
   griddep_wait();  // the plan (and all earlier work on the stream) is complete
 
-  const int E = p.meta[1];  // entries: packs' prefixes then sequences, or query chunks
+  // entries: packs' prefixes then sequences, or query chunks (plain: the B sequences)
+  const bool plain = p.pack_size == 1 && p.q_start == nullptr;
+  const int E = plain ? B : p.meta[1];
   const int64_t N = p.plan_tiles[E];
   const int64_t lo = static_cast<int64_t>(c) * N / C;
   const int64_t hi = static_cast<int64_t>(c + 1) * N / C;
@@ -536,7 +538,7 @@ __global__ void __launch_bounds__((HG * CG + 1) * 32, 1)
     const int TB = p.tok_box;
     const uint32_t box_bytes = static_cast<uint32_t>(HG * DCT * TB * 128);
     const int bpt = bs < kTile ? kTile / bs : 1;  // blocks per tile
-    const int K = p.meta[0];
+    const int K = plain ? 0 : p.meta[0];
     // the entry being walked: tiles t_first .. t_first + n_e - 1 of the line,
     // which are tiles i0 .. i0 + n_e - 1 of sequence b (of every pack member)
     int e = p.start_seq[c];
@@ -1094,7 +1096,7 @@ __device__ __forceinline__ RowParts row_parts(const DecodeParams& p, int r, int 
     q.direct = q.ns == 1;
     return q;
   }
-  const int K = p.meta[0];
+  const int K = p.pack_size > 1 ? p.meta[0] : 0;
   q.s0 = p.seg_base[K + r];
   q.ns = p.seg_base[K + r + 1] - q.s0;
   q.col0 = h;
