@@ -568,7 +568,7 @@ def cpu_baseline(spec, wl, budget_s=20.0):
         total_t += t
         total_b += b
         n += 1
-        if total_t + t > budget_s or n >= 5:
+        if total_t + t > budget_s or n >= 40:
             break
     return {"value": round(total_b / total_t / 1e9, 4), "unit": "GB/s", "cores": threads,
             "kind": "oracle",
