@@ -123,3 +123,30 @@ def test_fp8_write_then_attend(pa, orc):
         torch.cuda.synchronize()
         assert np.array_equal(dk.cpu().numpy(), ek)
         assert float(np.max(np.abs(out.double().cpu().numpy() - ref))) <= TOL_F32
+
+
+@pytest.mark.slow
+def test_full_size_fp8_workload(pa, orc):
+    """The benchmark's E4M3 workload (llama8b shape) in its launch
+    configuration, on 16 sampled sequences; NaN codes outside the tokens."""
+    from harness import used_slot_mask
+    spec = W.WORKLOADS["llama8b_fp8"]
+    prep = prepare(spec, poison=False)
+    kc, vc = prep.k_pool.copy(), prep.v_pool.copy()
+    used = used_slot_mask(prep.tables, prep.seq_lens, prep.case.num_blocks, spec.block_size)
+    kc[~used] = NAN_E4M3
+    vc[~used] = NAN_E4M3
+    q = to_dev(prep.case.q, spec.dtype)
+    ks, vs = _scales(spec.k_scale, spec.v_scale)
+    out = torch.empty(q.shape, dtype=torch.float32, device="cuda")
+    pa.decode_attention_fp8(out, q, _codes_dev(kc), _codes_dev(vc), ks, vs, to_dev(prep.tables),
+                            to_dev(prep.seq_lens), int(prep.seq_lens.max()), W.scale_of(spec))
+    torch.cuda.synchronize()
+    o = out.double().cpu().numpy()
+    assert np.all(np.isfinite(o))
+    rng = np.random.default_rng(2)
+    seqs = np.sort(rng.choice(spec.num_seqs, size=16, replace=False))
+    ref = orc.decode_fp8(prep.case.q[seqs], kc, vc, spec.k_scale, spec.v_scale,
+                         prep.tables[seqs], prep.seq_lens[seqs], W.scale_of(spec), spec.dtype,
+                         nthreads=8)
+    assert float(np.max(np.abs(o[seqs] - ref))) <= TOL_F32

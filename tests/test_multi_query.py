@@ -129,3 +129,24 @@ def test_bad_query_ranges_are_flagged(pa):
     torch.cuda.synchronize()
     assert int(flag.item()) & pa.DEVERR_BAD_SEQLEN
     assert torch.count_nonzero(guard).item() == 0
+
+
+@pytest.mark.slow
+def test_full_size_four_new_tokens(pa, orc):
+    """The benchmark's multi-query workload (llama8b shape, 4 new tokens per
+    sequence) in its launch configuration, on 16 sampled sequences."""
+    spec = W.WORKLOADS["llama8b_mq4"]
+    prep = prepare(spec.replace(q_len=1))  # pools, tables and lengths of the shape
+    g = torch.Generator().manual_seed(spec.seed + 11)
+    qlens = np.full(spec.num_seqs, spec.q_len, np.int32)
+    qs = np.concatenate([[0], np.cumsum(qlens)]).astype(np.int32)
+    q = W.randn_bits((int(qs[-1]), spec.num_q_heads, spec.head_dim), spec.dtype, g)
+    out = as_f64(_run(pa, spec, prep, q, qs, spec.q_len, torch.float32))
+    assert np.all(np.isfinite(out))
+    rng = np.random.default_rng(1)
+    seqs = np.sort(rng.choice(spec.num_seqs, size=16, replace=False))
+    rows = (seqs[:, None] * spec.q_len + np.arange(spec.q_len)[None, :]).reshape(-1)
+    sub_qs = (np.arange(len(seqs) + 1) * spec.q_len).astype(np.int32)
+    ref = orc.decode_multi(q[rows], sub_qs, prep.k_pool, prep.v_pool, prep.tables[seqs],
+                           prep.seq_lens[seqs], W.scale_of(spec), spec.dtype, nthreads=8)
+    assert float(np.max(np.abs(out[rows] - ref))) <= TOL_F32
