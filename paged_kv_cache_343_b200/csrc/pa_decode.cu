@@ -881,9 +881,11 @@ __global__ void __launch_bounds__((HG * CG + 1) * 32, 1)
     const uint32_t mask = static_cast<uint32_t>(ti.mask);
     const bool ok0 = (mask >> grp) & 1u, ok1 = (mask >> (grp + 8)) & 1u;
     uint32_t pb0[NB], pb1[NB], pc0[NB], pc1[NB];
+    // The blocks' steps run side by side (their max reductions, exponentials
+    // and transposes are independent), so their latencies overlap.
+    float mx0[NB], mx1[NB];
 #pragma unroll
     for (int nb = 0; nb < NB; ++nb) {
-      if (nb == 1 && !act1) continue;
       float* sv = s[nb];
       // columns 2q, 2q+1 see tile rows up to rel + column / G (rel = 16 when
       // every row is visible)
@@ -894,15 +896,26 @@ __global__ void __launch_bounds__((HG * CG + 1) * 32, 1)
       sv[1] = okB0 ? sv[1] * sl2 : -INFINITY;
       sv[2] = okA1 ? sv[2] * sl2 : -INFINITY;
       sv[3] = okB1 ? sv[3] * sl2 : -INFINITY;
-      float mx0 = fmaxf(sv[0], sv[2]), mx1 = fmaxf(sv[1], sv[3]);
+      mx0[nb] = fmaxf(sv[0], sv[2]);
+      mx1[nb] = fmaxf(sv[1], sv[3]);
+    }
 #pragma unroll
-      for (int o = 4; o < 32; o <<= 1) {
-        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+    for (int o = 4; o < 32; o <<= 1) {
+#pragma unroll
+      for (int nb = 0; nb < NB; ++nb) {
+        mx0[nb] = fmaxf(mx0[nb], __shfl_xor_sync(0xffffffffu, mx0[nb], o));
+        mx1[nb] = fmaxf(mx1[nb], __shfl_xor_sync(0xffffffffu, mx1[nb], o));
       }
-      const float mn0 = fmaxf(m_run[nb][0], mx0), mn1 = fmaxf(m_run[nb][1], mx1);
-      const float alpha0 = (mn0 == m_run[nb][0]) ? 1.f : ex2(m_run[nb][0] - mn0);
-      const float alpha1 = (mn1 == m_run[nb][1]) ? 1.f : ex2(m_run[nb][1] - mn1);
+    }
+    float alpha0[NB], alpha1[NB];
+    bool rescale = false;
+#pragma unroll
+    for (int nb = 0; nb < NB; ++nb) {
+      const float* sv = s[nb];
+      const float mn0 = fmaxf(m_run[nb][0], mx0[nb]), mn1 = fmaxf(m_run[nb][1], mx1[nb]);
+      alpha0[nb] = (mn0 == m_run[nb][0]) ? 1.f : ex2(m_run[nb][0] - mn0);
+      alpha1[nb] = (mn1 == m_run[nb][1]) ? 1.f : ex2(m_run[nb][1] - mn1);
+      rescale = rescale || alpha0[nb] != 1.f || alpha1[nb] != 1.f;
       m_run[nb][0] = mn0;
       m_run[nb][1] = mn1;
       const float p0 = (sv[0] == -INFINITY) ? 0.f : ex2(sv[0] - mn0);
@@ -917,22 +930,25 @@ __global__ void __launch_bounds__((HG * CG + 1) * 32, 1)
           pack2<kBF16>(p0 - lo_to_float<kBF16>(pt0), p1 - hi_to_float<kBF16>(pt0));
       const uint32_t pl1 =
           pack2<kBF16>(p2 - lo_to_float<kBF16>(pt1), p3 - hi_to_float<kBF16>(pt1));
-      l_part[nb][0] = l_part[nb][0] * alpha0 + (p0 + p2);
-      l_part[nb][1] = l_part[nb][1] * alpha1 + (p1 + p3);
-      if (__any_sync(0xffffffffu, alpha0 != 1.f || alpha1 != 1.f)) {
-#pragma unroll
-        for (int mt = 0; mt < MTILES; ++mt) {
-          acc[nb][mt][0] *= alpha0;
-          acc[nb][mt][1] *= alpha1;
-          acc[nb][mt][2] *= alpha0;
-          acc[nb][mt][3] *= alpha1;
-        }
-      }
+      l_part[nb][0] = l_part[nb][0] * alpha0[nb] + (p0 + p2);
+      l_part[nb][1] = l_part[nb][1] * alpha1[nb] + (p1 + p3);
       // P^T as the B operand (k = token, n = column): transpose the 8x8 halves
       pb0[nb] = movmatrix_trans(pt0);
       pb1[nb] = movmatrix_trans(pt1);
       pc0[nb] = movmatrix_trans(pl0);
       pc1[nb] = movmatrix_trans(pl1);
+    }
+    if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll
+      for (int nb = 0; nb < NB; ++nb) {
+#pragma unroll
+        for (int mt = 0; mt < MTILES; ++mt) {
+          acc[nb][mt][0] *= alpha0[nb];
+          acc[nb][mt][1] *= alpha1[nb];
+          acc[nb][mt][2] *= alpha0[nb];
+          acc[nb][mt][3] *= alpha1[nb];
+        }
+      }
     }
 
     // ---- O^T[D x 8] += V^T[D x 16 tok] * P^T[16 tok x 8], per n8 block
