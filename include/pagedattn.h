@@ -373,22 +373,23 @@ pa_status pa_decode_shared_prefix_workspace_bytes(int32_t num_seqs, int32_t num_
  * parallel sampling every sample's block table starts with the prompt's
  * blocks, so pa_decode_attention reads each shared block once per sample.
  * This entry point computes the same out[b, h, :] but reads a shared prefix
- * once per pack of P = 8 / (num_q_heads / num_kv_heads) consecutive
- * sequences (P = 2 for 4 query heads per KV head): the pack's queries fill the
- * eight columns of one tensor-core product over the prefix, each sequence's
- * own tail is attended as usual, and the combine pass merges the two
- * softmax partials.  Packs need P >= 2 (at most 4 query heads per KV head;
- * otherwise this is pa_decode_attention with a larger workspace).
+ * once per pack of up to P = min(8, 32 / (num_q_heads / num_kv_heads))
+ * consecutive sequences (P = 8 for 4 query heads per KV head): the pack's
+ * queries fill up to 32 columns of the tensor-core products over the prefix
+ * (one column per member and query head), each sequence's own tail is attended
+ * as usual, and the combine pass merges the two softmax partials.
  *
  *  shared_blocks  int32 [num_seqs], device: shared_blocks[b] = number of
  *                 leading block-table entries that sequence b holds in common
  *                 with sequence b + 1 (the same physical block ids; 0 if
  *                 none; the last entry is ignored).  A block manager knows it
- *                 from its fork history.  The plan packs P consecutive
- *                 sequences b .. b+P-1 over the blocks that every pair of
- *                 neighbours shares and that are full in every member, in
- *                 whole 16-token tiles, when that prefix is at least 64
- *                 tokens; sequences that do not fit a pack run alone.
+ *                 from its fork history.  The plan takes aligned windows of P
+ *                 sequences (b = P w .. P w + P - 1) and packs a window over
+ *                 the blocks that every pair of neighbours shares and that are
+ *                 full in every member, in whole 16-token tiles, when that
+ *                 prefix is at least 64 tokens; a window that does not share
+ *                 one (and the shorter last window) falls back to the aligned
+ *                 pairs inside it; sequences outside every pack run alone.
  *  workspace      at least pa_decode_shared_prefix_workspace_bytes().
  * Other arguments, layouts and errors are those of pa_decode_attention.  On
  * the device, a pack member whose table entry differs from the first

@@ -391,7 +391,7 @@ def decode_attention_shared_prefix(out: torch.Tensor, query: torch.Tensor,
     blocks (parallel samples of one prompt): shared_blocks int32 [B] on the
     device, shared_blocks[b] = leading table entries b holds in common with
     b + 1 (BlockManager.shared_blocks gives it).  Same result; a shared prefix
-    is read once per pack of 8 // (Hq / Hkv) sequences."""
+    is read once per pack of up to min(8, 32 // (Hq / Hkv)) sequences."""
     _need(query.dim() == 3 and query.is_contiguous(), "query must be contiguous [B, Hq, D]")
     _need(out.shape == query.shape and out.is_contiguous(), "out must be contiguous [B, Hq, D]")
     _need(key_cache.is_contiguous() and value_cache.is_contiguous(), "caches must be contiguous")

@@ -4,19 +4,24 @@
 // pool and run attention over them with an online softmax).
 //
 // Three launches per call, all on the caller's stream:
-//   1. plan     (1 CTA)   per-sequence prefix sums of 16-token tiles and of
-//                         partitions, written to the workspace;
+//   1. plan     (1 CTA)   the units of work ("entries": sequences, packs of
+//                         sequences over a shared prompt, or chunks of a
+//                         sequence's query tokens), prefix sums of their
+//                         16-token tiles and the segment bookkeeping, written
+//                         to the workspace;
 //   2. main     (1 CTA per SM and head group, persistent)  the batch's tiles
 //                         laid end to end are cut into equal shares, one per
 //                         CTA; a producer warp streams each tile's K and V
 //                         from the pool into shared memory with 5-D TMA loads
-//                         (one block-table lookup per block), and one consumer
-//                         warp per KV head computes S^T = K Q^T and
-//                         O^T += V^T P^T on the tensor cores (grouped query
-//                         heads packed into the MMA's N dimension) with an
-//                         fp32 online softmax;
-//   3. combine            merges the (o, m, l) partials of every sequence
-//                         whose tiles were split across CTAs or partitions.
+//                         (one block-table lookup per block), and consumer
+//                         warps (one to two per KV head) compute S^T = K Q^T
+//                         and O^T += V^T P^T on the tensor cores, the query
+//                         heads of a KV head (and the query rows of an entry)
+//                         packed into the MMA's N dimension, with an fp32
+//                         online softmax;
+//   3. combine            merges the (o, m, l) partials of every output row
+//                         whose tiles were split across CTAs, partitions or
+//                         a pack and the sequence's own tail.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
