@@ -451,8 +451,8 @@ pa_status pa_decode_attention_noalloc(void* out, pa_dtype out_dtype, const void*
 /* ---------------------------------------------------------------------------
  * Host block manager -- [PA] "The idea: page the KV cache" (allocate a block
  * when the previous one is full, from a free list, from anywhere in memory),
- * "Sharing and copy-on-write" (per-block reference counts; full blocks are
- * never written again) and "How does copy-on-write work for parallel
+ * "Sharing and copy-on-write" (per-block reference counts; a filled block is
+ * not written again) and "How does copy-on-write work for parallel
  * sampling?" (allocate, copy, decrement, write into the copy).
  *
  * Host-only, not thread-safe (one manager per scheduler thread).  Block ids

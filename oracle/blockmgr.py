@@ -3,16 +3,17 @@
 A plain restatement of the host-side bookkeeping on the "PagedAttention" page
 (shubhamtatvamasi):
 
-* "The idea: page the KV cache" (table row "Allocate a page on first touch")
-  and the five-request figure: a sequence gets a new physical block from the
-  free list only when its previous block is full; blocks come from anywhere.
+* "The idea: page the KV cache" (the OS analogy table and the five-request
+  figure): a sequence gets a new physical block from the free list only when
+  its previous block is full; blocks come from anywhere.
 * "Sharing and copy-on-write": two sequences may point at the same physical
-  block; every block keeps a reference count; full blocks are never written
-  again, so only a shared, partially filled last block is ever copied.
+  block; every block keeps a reference count; a block that has filled up is
+  not written again, so only a shared, partially filled last block is copied.
 * "How does copy-on-write work for parallel sampling?": all samples' tables
   point at the prompt's blocks with refcount = number of users; a sample that
-  must append into a shared partial block allocates a new block, copies the
-  existing tokens, decrements the old block's count and writes into the copy.
+  must append into a shared partial block takes a new block, has the tokens
+  already there copied into it, drops its count on the old block and writes
+  into the copy.
 
 Free-list order is part of the input: ``free_order`` lists the physical ids in
 the order they are handed out (front first); a freed block goes to the back.
@@ -73,7 +74,7 @@ class RefBlockManager:
         bs = self.block_size
         cow = None
         if pos % bs == 0:
-            # previous block full (or no block yet): allocate on first touch
+            # previous block full (or no block yet): take a fresh block now
             table.append(self._alloc())
         else:
             last = table[-1]

@@ -3,10 +3,10 @@
 //
 // Rules from "PagedAttention" (shubhamtatvamasi.com):
 //  - "The idea: page the KV cache": a sequence gets a new physical block only
-//    when its previous block is full ("allocate a page on first touch"), from a
-//    free list, from anywhere in memory;
+//    when its previous block is full (the OS analogy: a page is allocated when
+//    first used), from a free list, from anywhere in memory;
 //  - "Sharing and copy-on-write": tables may point at the same physical block;
-//    each block keeps a reference count; full blocks are never written again;
+//    each block keeps a reference count; a filled block is not written again;
 //  - "How does copy-on-write work for parallel sampling?": a sequence that must
 //    append into a shared, partially filled block allocates a new block, has
 //    the old contents copied into it, decrements the old block's count and
