@@ -333,7 +333,7 @@ def run_ours(args, rank, world, local_rank):
     stream = torch.cuda.current_stream(device)
     launches_per_step = 1 + 3 + (1 if cow is not None else 0)
 
-    def step(ev0=None, ev1=None):
+    def step():
         if cow is not None:
             pa.copy_blocks([k_cache], [v_cache], cow, error_flag=flag)
         if spec.fp8:
@@ -341,8 +341,9 @@ def run_ours(args, rank, world, local_rank):
                                  k_scale=k_scale, v_scale=v_scale, error_flag=flag)
         else:
             pa.reshape_and_cache(new_k, new_v, k_cache, v_cache, slots, error_flag=flag)
-        if ev0 is not None:
-            ev0.record(stream)
+        attention()
+
+    def attention():
         if spec.fp8:
             pa.decode_attention_fp8(out, q, k_cache, v_cache, k_scale, v_scale, tables, lens,
                                     max_len, scale, psize, ws, error_flag=flag)
@@ -357,8 +358,6 @@ def run_ours(args, rank, world, local_rank):
         else:
             pa.decode_attention(out, q, k_cache, v_cache, tables, lens, max_len, scale, psize, ws,
                                 error_flag=flag)
-        if ev1 is not None:
-            ev1.record(stream)
 
     bytes_step = kv_bytes(spec, wl["lens"])
     clocks = ClockSampler(local_rank if "CUDA_VISIBLE_DEVICES" not in os.environ
@@ -371,33 +370,66 @@ def run_ours(args, rank, world, local_rank):
     if int(flag.item()) != 0:
         raise RuntimeError("device error flag %#x during warm-up" % int(flag.item()))
 
-    ev_att = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-              for _ in range(args.steps)]
+    # The timed steps replay one captured step (its kernels chained by
+    # programmatic dependent launch, no host launch cost); --no-graph launches
+    # them one by one instead.
+    run_stream = stream
+    graph = None
+    if not args.no_graph:
+        run_stream = torch.cuda.Stream(device=device)
+        run_stream.wait_stream(stream)
+        with torch.cuda.stream(run_stream):
+            step()
+        run_stream.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=run_stream, capture_error_mode="thread_local"):
+            step()
+        torch.cuda.synchronize()
+        for _ in range(3):  # warm-up replays
+            with torch.cuda.stream(run_stream):
+                graph.replay()
+        torch.cuda.synchronize()
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
     wall0 = time.time()
-    t_start.record(stream)
-    for i in range(args.steps):
-        step(*ev_att[i])
-    t_end.record(stream)
+    with torch.cuda.stream(run_stream):
+        t_start.record(run_stream)
+        for i in range(args.steps):
+            if graph is not None:
+                graph.replay()
+            else:
+                step()
+        t_end.record(run_stream)
     torch.cuda.synchronize()
     wall1 = time.time()
     if world > 1:
         torch.distributed.barrier()
+    elapsed_ms = t_start.elapsed_time(t_end)
+    # The attention call alone, for the roofline: its average duration over
+    # att_steps calls launched back to back on its stream between two events
+    # (an event between the calls of one chain would break the programmatic
+    # dependent launch that overlaps them).
+    att_steps = min(args.steps, 500)
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    a0.record(stream)
+    for _ in range(att_steps):
+        attention()
+    a1.record(stream)
+    torch.cuda.synchronize()
     clock_info = clocks.summary(wall0, wall1)
     clocks.stop()
-    elapsed_ms = t_start.elapsed_time(t_end)
-    att_ms = [a.elapsed_time(b) for a, b in ev_att]
-    att_avg_ms = sum(att_ms) / len(att_ms)
+    att_avg_ms = a0.elapsed_time(a1) / att_steps
     if int(flag.item()) != 0:
         raise RuntimeError("device error flag %#x in the timed region" % int(flag.item()))
 
     # ---------------- end to end: pinned host buffers through the public API
     e2e_steps = max(1, min(args.steps, args.e2e_steps))
     runner = pa.PagedDecodeStep(k_cache, v_cache, B, Hq, wl["tables"].shape[1], max_len, scale,
-                                psize, query_dtype=td, k_scale=k_scale, v_scale=v_scale)
+                                psize, query_dtype=td, k_scale=k_scale, v_scale=v_scale,
+                                slots=2)
 
     def fill(dst, a, dtype=None):
         t = torch.from_numpy(np.ascontiguousarray(a))
@@ -406,28 +438,37 @@ def run_ours(args, rank, world, local_rank):
     e2e_ok = wl["slots"].shape[0] == B and cow is None and not multi
     e2e = None
     if e2e_ok:
-        h = runner.host
-        fill(h["q"], case.q, td)
-        fill(h["new_k"], wl["new_k"], td)
-        fill(h["new_v"], wl["new_v"], td)
-        fill(h["slots"], wl["slots"])
-        fill(h["tables"], wl["tables"])
-        fill(h["lens"], wl["lens"])
-        for _ in range(3):
-            runner()
+        for sl in range(2):
+            h = runner.slot_host(sl)
+            fill(h["q"], case.q, td)
+            fill(h["new_k"], wl["new_k"], td)
+            fill(h["new_v"], wl["new_v"], td)
+            fill(h["slots"], wl["slots"])
+            fill(h["tables"], wl["tables"])
+            fill(h["lens"], wl["lens"])
+        for i in range(4):  # warm-up; captures each slot's kernels in a graph
+            runner.submit(i % 2)
+            runner.wait(i % 2)
         if world > 1:
             torch.distributed.barrier()
+        # every step copies its inputs in and its output out; step i + 1 is
+        # submitted before the host waits for step i, as a serving loop does
         t0 = time.perf_counter()
-        for _ in range(e2e_steps):
-            runner()
+        runner.submit(0)
+        for i in range(1, e2e_steps):
+            runner.submit(i % 2)
+            runner.wait((i - 1) % 2)
+        runner.wait((e2e_steps - 1) % 2)
         e2e_s = time.perf_counter() - t0
         e2e_s = max_over_ranks(e2e_s, world, device)
         e2e = {"value": round(bytes_step * e2e_steps * world / e2e_s / 1e9, 2), "unit": "GB/s",
                "h2d_bytes_per_step": runner.h2d_bytes(), "d2h_bytes_per_step": runner.d2h_bytes(),
                "steps": e2e_steps, "ms_per_step": round(e2e_s * 1e3 / e2e_steps, 4),
-               "how": "PagedDecodeStep: one pinned H2D copy of the step's inputs, "
-                      "reshape_and_cache + decode_attention, one D2H copy of the output, "
-                      "stream synchronise; replayed as a CUDA graph"}
+               "how": "PagedDecodeStep with two slots: per step one pinned H2D copy of "
+                      "the step's inputs, reshape_and_cache + decode_attention (a CUDA "
+                      "graph per slot), one D2H copy of the output into pinned memory; "
+                      "step i + 1 is submitted before the host waits for step i's output, "
+                      "so one step's copies overlap another's kernels"}
 
     elapsed_ms = max_over_ranks(elapsed_ms, world, device)
     att_avg_ms = max_over_ranks(att_avg_ms, world, device)
@@ -458,6 +499,8 @@ def run_ours(args, rank, world, local_rank):
             "sum_seq_len": int(wl["lens"].sum()), "partition_size": psize,
             "num_blocks": case.num_blocks, "parallelism": "dp%d (independent batches)" % world,
             "l2": "no flush: each step reads %.0f MB of KV, more than the 126 MB L2" % (bytes_step / 1e6),
+            "timed_as": ("a CUDA graph of one step, replayed %d times" % args.steps
+                         if graph is not None else "%d steps launched one by one" % args.steps),
         },
         "decode_tokens_per_s": round(spec.num_seqs * spec.q_len * world / (ms_per_step / 1e3), 1),
         "attention_gbs": round(achieved, 2),
@@ -640,6 +683,8 @@ def main(argv=None):
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--ref-budget", type=float, default=90.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="launch the timed steps one by one instead of replaying a graph")
     ap.add_argument("--no-shared-prefix", action="store_true",
                     help="shared_prefix workload: use the plain decode entry point")
     ap.add_argument("--block-size", type=int, default=0,

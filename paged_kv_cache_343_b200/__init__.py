@@ -572,15 +572,25 @@ class BlockManager:
 class PagedDecodeStep:
     """One decode step driven from pinned host memory (the end-to-end call).
 
-    Holds, for a fixed batch shape, one pinned host staging buffer and a device
-    buffer of the same layout.  The caller writes the step's inputs into the
+    Holds, for a fixed batch shape, pinned host staging buffers and device
+    buffers of the same layout.  The caller writes the step's inputs into the
     views of ``host`` (``q``, ``new_k``, ``new_v``, ``slots``, ``tables``,
     ``lens``); a call copies the whole staging buffer host->device in one copy,
     writes the new rows into the pools with reshape_and_cache, runs
     decode_attention, copies the output into the pinned ``host_out`` in one copy
     and waits for the stream.  With ``use_graph`` (default) the first call runs
     eagerly and captures the step (copies and kernels) into a CUDA graph that
-    later calls replay."""
+    later calls replay.
+
+    Pipelined use (``slots`` >= 2): slot s has its own staging buffers
+    (``slot_host(s)``, slot 0 being ``host``) and output (``slot_out(s)``);
+    ``submit(s)`` enqueues the slot's host->device copy on a copy stream, the
+    kernels on the compute stream and the device->host copy of the output on a
+    second copy stream, ordered by events, and returns at once; ``wait(s)``
+    returns the slot's pinned output once it has arrived.  A serving loop
+    submits step i + 1 before it waits for step i, so the copies of one step
+    overlap the kernels of another.  A slot's inputs may be rewritten once its
+    previous ``submit`` has been waited for."""
 
     _ALIGN = 256
 
@@ -589,9 +599,11 @@ class PagedDecodeStep:
                  partition_size: int = 0, out_dtype: Optional[torch.dtype] = None,
                  stream: Optional[torch.cuda.Stream] = None, use_graph: bool = True,
                  query_dtype: Optional[torch.dtype] = None,
-                 k_scale: Optional[torch.Tensor] = None, v_scale: Optional[torch.Tensor] = None):
+                 k_scale: Optional[torch.Tensor] = None, v_scale: Optional[torch.Tensor] = None,
+                 slots: int = 1):
         """uint8 pools are fp8 (E4M3) code pools: pass query_dtype and the
         one-element float32 device scales."""
+        _need(slots >= 1, "at least one slot")
         self.k, self.v = key_cache, value_cache
         nb, bs, hkv, d = key_cache.shape
         dev = key_cache.device
@@ -614,18 +626,33 @@ class PagedDecodeStep:
             layout.append((name, shape, dtype, off, nbytes))
             off += -(-nbytes // self._ALIGN) * self._ALIGN
         self._nbytes = off
-        self._host_buf = torch.empty(off, dtype=torch.uint8).pin_memory()
-        self._dev_buf = torch.empty(off, dtype=torch.uint8, device=dev)
 
         def views(buf):
             return {name: buf[o:o + n].view(dtype).view(shape) for name, shape, dtype, o, n in layout}
 
-        self.host = views(self._host_buf)
-        self.dev = views(self._dev_buf)
-        self.out = torch.empty((num_seqs, num_q_heads, d), dtype=out_dtype or dt, device=dev)
-        self.host_out = torch.empty(self.out.shape, dtype=self.out.dtype).pin_memory()
+        out_shape = (num_seqs, num_q_heads, d)
+        self._host_bufs = [torch.empty(off, dtype=torch.uint8).pin_memory() for _ in range(slots)]
+        self._dev_bufs = [torch.empty(off, dtype=torch.uint8, device=dev) for _ in range(slots)]
+        self._hosts = [views(b) for b in self._host_bufs]
+        self._devs = [views(b) for b in self._dev_bufs]
+        self._outs = [torch.empty(out_shape, dtype=out_dtype or dt, device=dev)
+                      for _ in range(slots)]
+        self._host_outs = [torch.empty(out_shape, dtype=out_dtype or dt).pin_memory()
+                           for _ in range(slots)]
+        # slot 0 is also the sequential call's buffers
+        self._host_buf, self._dev_buf = self._host_bufs[0], self._dev_bufs[0]
+        self.host, self.dev = self._hosts[0], self._devs[0]
+        self.out, self.host_out = self._outs[0], self._host_outs[0]
         self.ws = alloc_workspace(decode_workspace_bytes(num_seqs, num_q_heads, hkv, d, bs,
                                                          max_seq_len, partition_size), dev)
+        # pipelined use: copy streams, per-slot events and compute graphs
+        self._copy_in = torch.cuda.Stream(device=dev)
+        self._copy_out = torch.cuda.Stream(device=dev)
+        self._ev_in = [torch.cuda.Event() for _ in range(slots)]
+        self._ev_comp = [torch.cuda.Event() for _ in range(slots)]
+        self._ev_out = [torch.cuda.Event() for _ in range(slots)]
+        self._slot_graphs = [None] * slots
+        self._pending = [False] * slots
 
     def h2d_bytes(self) -> int:
         return self._nbytes
@@ -633,20 +660,29 @@ class PagedDecodeStep:
     def d2h_bytes(self) -> int:
         return self.out.numel() * self.out.element_size()
 
-    def _enqueue(self) -> None:
-        dv = self.dev
-        self._dev_buf.copy_(self._host_buf, non_blocking=True)
+    def slot_host(self, slot: int) -> dict:
+        """Pinned input views of a slot (write them before ``submit(slot)``)."""
+        return self._hosts[slot]
+
+    def slot_out(self, slot: int) -> torch.Tensor:
+        return self._host_outs[slot]
+
+    def _kernels(self, dv, out) -> None:
         if self.fp8:
             reshape_and_cache(dv["new_k"], dv["new_v"], self.k, self.v, dv["slots"],
                               kv_cache_dtype="fp8_e4m3", k_scale=self.k_scale,
                               v_scale=self.v_scale)
-            decode_attention_fp8(self.out, dv["q"], self.k, self.v, self.k_scale, self.v_scale,
+            decode_attention_fp8(out, dv["q"], self.k, self.v, self.k_scale, self.v_scale,
                                  dv["tables"], dv["lens"], self.max_seq_len, self.scale,
                                  self.partition_size, self.ws)
         else:
             reshape_and_cache(dv["new_k"], dv["new_v"], self.k, self.v, dv["slots"])
-            decode_attention(self.out, dv["q"], self.k, self.v, dv["tables"], dv["lens"],
+            decode_attention(out, dv["q"], self.k, self.v, dv["tables"], dv["lens"],
                              self.max_seq_len, self.scale, self.partition_size, self.ws)
+
+    def _enqueue(self) -> None:
+        self._dev_buf.copy_(self._host_buf, non_blocking=True)
+        self._kernels(self.dev, self.out)
         self.host_out.copy_(self.out, non_blocking=True)
 
     def __call__(self) -> torch.Tensor:
@@ -664,3 +700,39 @@ class PagedDecodeStep:
                 self._enqueue()
             self.graph = g
         return self.host_out
+
+    def submit(self, slot: int) -> None:
+        """Enqueue one step on a slot: copy in, kernels, copy out; no wait."""
+        _need(not self._pending[slot], "wait for the slot's previous step first")
+        cs, ci, co = self.stream, self._copy_in, self._copy_out
+        # the slot's device inputs are free once its previous kernels finished
+        ci.wait_event(self._ev_comp[slot])
+        with torch.cuda.stream(ci):
+            self._dev_bufs[slot].copy_(self._host_bufs[slot], non_blocking=True)
+            self._ev_in[slot].record(ci)
+        cs.wait_event(self._ev_in[slot])
+        g = self._slot_graphs[slot]
+        if g is not None:
+            with torch.cuda.stream(cs):
+                g.replay()
+        else:
+            with torch.cuda.stream(cs):
+                self._kernels(self._devs[slot], self._outs[slot])
+            if self.use_graph:
+                cs.synchronize()
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=cs, capture_error_mode="thread_local"):
+                    self._kernels(self._devs[slot], self._outs[slot])
+                self._slot_graphs[slot] = g
+        self._ev_comp[slot].record(cs)
+        co.wait_event(self._ev_comp[slot])
+        with torch.cuda.stream(co):
+            self._host_outs[slot].copy_(self._outs[slot], non_blocking=True)
+            self._ev_out[slot].record(co)
+        self._pending[slot] = True
+
+    def wait(self, slot: int) -> torch.Tensor:
+        """The slot's pinned output, once its device->host copy has landed."""
+        self._ev_out[slot].synchronize()
+        self._pending[slot] = False
+        return self._host_outs[slot]

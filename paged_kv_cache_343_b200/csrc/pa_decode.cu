@@ -1137,6 +1137,9 @@ __global__ void __launch_bounds__(kCombineWarps * 32) pa_combine_narrow_kernel(c
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int b = blockIdx.x;
   const int qh = blockIdx.y * kCombineWarps + warp;
+  // the next launch on the stream may start its prologue now; it waits for
+  // this grid before touching data
+  griddep_launch_dependents();
   griddep_wait();  // the main kernel's partials are complete and visible
   if (qh >= p.num_q_heads) return;
   const int G = p.group, HG = p.heads_per_cta;
@@ -1215,6 +1218,9 @@ __global__ void __launch_bounds__(kCombineWarps * 32) pa_combine_wide_kernel(con
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int b = blockIdx.x;
   const int qh = blockIdx.y;
+  // the next launch on the stream may start its prologue now; it waits for
+  // this grid before touching data
+  griddep_launch_dependents();
   griddep_wait();  // the main kernel's partials are complete and visible
   const int G = p.group, HG = p.heads_per_cta;
   const int kvh = qh / G, h = qh - kvh * G;

@@ -368,3 +368,53 @@ def test_end_to_end_step_from_host_buffers(pa, orc, use_graph):
         orc.reshape_and_cache(nk, nv, k_ref, v_ref, slots)
         ref = orc.decode(q, k_ref, v_ref, tables, lens, W.scale_of(s), s.dtype, nthreads=4)
         assert np.max(np.abs(out.double().numpy() - ref)) <= TOL_STORED
+
+
+def test_end_to_end_pipelined_slots(pa, orc):
+    """PagedDecodeStep with two slots: the host fills one slot while the other
+    step is in flight (submit step i + 1, then wait for step i); every step
+    appends one token per sequence, and each output matches the oracle on the
+    pools as they stand after that step's writes."""
+    spec = W.WORKLOADS["llama8b"].replace(num_seqs=5, len_lo=40, len_hi=600, seed=42)
+    prep = prepare(spec)
+    s = prep.case.spec
+    B = s.num_seqs
+    bm = prep.extra["bm"]
+    dk, dv = to_dev(prep.k_pool, s.dtype), to_dev(prep.v_pool, s.dtype)
+    k_ref, v_ref = prep.k_pool.copy(), prep.v_pool.copy()
+    width = prep.tables.shape[1] + 4
+    step = pa.PagedDecodeStep(dk, dv, B, s.num_q_heads, width, int(prep.seq_lens.max()) + 8,
+                              W.scale_of(s), slots=2)
+    td = {"bf16": torch.bfloat16, "f16": torch.float16}[s.dtype]
+    g = torch.Generator().manual_seed(5)
+    refs = {}
+
+    def fill(slot, it):
+        slots = np.array([bm.append_slot(b)[0] for b in range(B)], np.int32)
+        lens = np.array([bm.lengths[b] for b in range(B)], np.int32)
+        tables = np.full((B, width), -1, np.int32)
+        for b in range(B):
+            t = bm.block_table(b)
+            tables[b, :len(t)] = t
+        q = W.randn_bits((B, s.num_q_heads, s.head_dim), s.dtype, g)
+        nk = W.randn_bits((B, s.num_kv_heads, s.head_dim), s.dtype, g)
+        nv = W.randn_bits((B, s.num_kv_heads, s.head_dim), s.dtype, g)
+        h = step.slot_host(slot)
+        for name, src in (("q", q), ("new_k", nk), ("new_v", nv)):
+            h[name].copy_(torch.from_numpy(src).view(torch.int16).view(td))
+        h["slots"].copy_(torch.from_numpy(slots))
+        h["tables"].copy_(torch.from_numpy(tables))
+        h["lens"].copy_(torch.from_numpy(lens))
+        orc.reshape_and_cache(nk, nv, k_ref, v_ref, slots)
+        refs[it] = orc.decode(q, k_ref, v_ref, tables, lens, W.scale_of(s), s.dtype, nthreads=4)
+
+    steps = 5
+    fill(0, 0)
+    step.submit(0)
+    for it in range(1, steps):
+        fill(it % 2, it)
+        step.submit(it % 2)
+        out = step.wait((it - 1) % 2)
+        assert np.max(np.abs(out.double().numpy() - refs[it - 1])) <= TOL_STORED
+    out = step.wait((steps - 1) % 2)
+    assert np.max(np.abs(out.double().numpy() - refs[steps - 1])) <= TOL_STORED
