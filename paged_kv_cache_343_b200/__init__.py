@@ -6,7 +6,7 @@ torch tensors into pointers, sizes and the current CUDA stream, calls the C
 entry point of the same name and raises on a non-OK status.  Every step of
 the hot path runs in the library's kernels; there is no fallback.  Importing
 this package fails loudly if the library has not been built
-(``python -m paged_kv_cache_343_b200.build``).
+(``python paged_kv_cache_343_b200/build.py``).
 
 Entry points (see the header for argument meaning, layout and errors):
 
@@ -87,7 +87,7 @@ def _pool_strides(cache: torch.Tensor) -> Optional[CacheStrides]:
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError("libpagedattn.so is missing at %s; build it with "
-                          "`python -m paged_kv_cache_343_b200.build`" % LIB_PATH)
+                          "`python paged_kv_cache_343_b200/build.py`" % LIB_PATH)
     lib = ctypes.CDLL(LIB_PATH)
     i32, i64, p, sz = ctypes.c_int32, ctypes.c_int64, ctypes.c_void_p, ctypes.c_size_t
     lib.pa_status_string.restype = ctypes.c_char_p

@@ -1,6 +1,9 @@
 """Builds libpagedattn.so (the C-ABI library) in-tree with nvcc for sm_100a.
 
-    python -m paged_kv_cache_343_b200.build [--force] [--verbose]
+    python paged_kv_cache_343_b200/build.py [--force] [--verbose]
+
+Run it by path: importing it through the package would load the package,
+which refuses to import without the library.
 
 Sources: csrc/*.cu and csrc/*.cpp.  Objects go to _build/ (git-ignored); the
 shared library lands next to this file so the Python binding finds it.

@@ -14,8 +14,12 @@ HEADER = os.path.join(ROOT, "include", "pagedattn.h")
 
 @pytest.fixture(scope="module")
 def pa():
-    from paged_kv_cache_343_b200 import build
-    build.build()
+    import importlib.util
+    path = os.path.join(ROOT, "paged_kv_cache_343_b200", "build.py")
+    spec = importlib.util.spec_from_file_location("_pa_build", path)
+    builder = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(builder)
+    builder.build()  # compiles the library if missing, before the package loads it
     import paged_kv_cache_343_b200 as pa
     return pa
 
