@@ -280,6 +280,54 @@ def packed_kv_bytes(spec, wl) -> int:
 
 
 # --------------------------------------------------------------------------- our arm
+def read_ceiling(device, stream):
+    """The read-bandwidth ceiling measured in the same run: the library's read
+    stream over 1 GiB (eight times the L2), the best of 2, 4 and 8 CTAs per SM,
+    ten passes each between two events after three untimed ones."""
+    sms = torch.cuda.get_device_properties(device).multi_processor_count
+    buf = torch.ones(1 << 28, dtype=torch.int32, device=device)
+    nbytes = buf.numel() * buf.element_size()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    best, best_per_sm = 0.0, 0
+    for per_sm in (2, 4, 8):
+        sink = torch.empty(sms * per_sm, dtype=torch.int32, device=device)
+        for _ in range(3):
+            pa.stream_read(buf, sink, stream)
+        e0.record(stream)
+        for _ in range(10):
+            pa.stream_read(buf, sink, stream)
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        gbs = 10 * nbytes / (e0.elapsed_time(e1) / 1e3) / 1e9
+        if gbs > best:
+            best, best_per_sm = gbs, per_sm
+    del buf
+    return {"gbs": round(best, 1), "bytes": nbytes,
+            "how": "pa_stream_read: 16-byte loads, %d CTAs of 512 threads per SM, 1 GiB read "
+                   "10 times" % best_per_sm}
+
+
+def latency_distribution(attention, read_bytes, device, stream, runs=100):
+    """One attention call per run, the L2 flushed before each (a write of twice
+    its size), timed alone between two events: median, p10 and p90."""
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    flush = torch.empty(max(1, 2 * l2 // 4), dtype=torch.int32, device=device)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(runs)]
+    with torch.cuda.stream(stream):
+        for a, b in ev:
+            flush.zero_()
+            a.record(stream)
+            attention()
+            b.record(stream)
+    torch.cuda.synchronize(device)
+    us = np.array(sorted(a.elapsed_time(b) * 1e3 for a, b in ev))
+    p10, med, p90 = (float(np.percentile(us, q)) for q in (10, 50, 90))
+    return {"runs": runs, "l2": "flushed before each run (%d MB written)" % (2 * l2 // 2**20),
+            "median_us": round(med, 2), "p10_us": round(p10, 2), "p90_us": round(p90, 2),
+            "gbs_at_median": round(read_bytes / (med / 1e6) / 1e9, 2)}
+
+
 def run_ours(args, rank, world, local_rank):
     import paged_kv_cache_343_b200 as pa
 
@@ -422,6 +470,9 @@ def run_ours(args, rank, world, local_rank):
     clock_info = clocks.summary(wall0, wall1)
     clocks.stop()
     att_avg_ms = a0.elapsed_time(a1) / att_steps
+    read_bytes = unique_kv_bytes(spec, wl) if spec.len_dist == "shared_prefix" else bytes_step
+    latency = latency_distribution(attention, read_bytes, device, stream)
+    ceiling = read_ceiling(device, stream)
     if int(flag.item()) != 0:
         raise RuntimeError("device error flag %#x in the timed region" % int(flag.item()))
 
@@ -480,7 +531,6 @@ def run_ours(args, rank, world, local_rank):
     value = total_bytes * args.steps / (elapsed_ms / 1e3) / 1e9
     # the roofline counts the bytes that must come from HBM: for shared
     # prompts each distinct (block, slot) once, else every token's K and V
-    read_bytes = unique_kv_bytes(spec, wl) if spec.len_dist == "shared_prefix" else bytes_step
     achieved = read_bytes / (att_avg_ms / 1e3) / 1e9
     peak = float(peaks["hbm_gbs"])
     traffic = profiled_traffic() if args.workload == "llama8b" else None
@@ -512,6 +562,8 @@ def run_ours(args, rank, world, local_rank):
                                 "pa_decode_attention") + " (plan + main + combine launches)",
                      "bytes_per_launch": read_bytes,
                      "peak_kind": peak_kind + " (MEASURED_PEAKS hbm_gbs, copy read+write)"},
+        "attention_latency": latency,
+        "read_ceiling": dict(ceiling, frac=round(achieved / ceiling["gbs"], 4)),
         "kv_memory": kv_memory(spec, wl),
         "clocks": clock_info,
         "e2e": e2e,

@@ -449,6 +449,22 @@ pa_status pa_decode_attention_noalloc(void* out, pa_dtype out_dtype, const void*
                                       int32_t* device_error_flag, pa_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * Read-bandwidth ceiling -- a measurement aid, not a step of the method.
+ * Decode is limited by reading the cache from memory ([KV] opening section),
+ * so its kernels are held against the rate at which this GPU streams reads.
+ *
+ * Reads `bytes` bytes of the device buffer `buf` once (16-byte loads,
+ * grid-stride, num_ctas CTAs of 512 threads) and writes to sink[c] (device,
+ * num_ctas uint32) the XOR of the 32-bit words CTA c read, so that the XOR
+ * of sink[0 .. num_ctas) equals the XOR of every word of the buffer.
+ * PA_ERR_INVALID_ARG: bytes < 0 or not a multiple of 16, buf not 16-byte
+ * aligned (when bytes > 0), sink NULL or not 4-byte aligned, num_ctas
+ * outside [1, 65535].  PA_ERR_CUDA: the launch failed.
+ * ------------------------------------------------------------------------- */
+pa_status pa_stream_read(const void* buf, int64_t bytes, uint32_t* sink, int32_t num_ctas,
+                         pa_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * Host block manager -- [PA] "The idea: page the KV cache" (allocate a block
  * when the previous one is full, from a free list, from anywhere in memory),
  * "Sharing and copy-on-write" (per-block reference counts; a filled block is

@@ -44,7 +44,7 @@ __all__ = [
     "decode_attention_shared_prefix", "shared_prefix_workspace_bytes",
     "decode_attention_multi_query", "multi_query_workspace_bytes", "BlockManager",
     "PagedDecodeStep", "DEVERR_BAD_BLOCK", "DEVERR_BAD_SLOT", "DEVERR_BAD_SEQLEN",
-    "DEVERR_TIMEOUT", "DEVERR_BAD_SHARE", "CacheStrides", "version",
+    "DEVERR_TIMEOUT", "DEVERR_BAD_SHARE", "CacheStrides", "version", "stream_read",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpagedattn.so")
@@ -142,6 +142,8 @@ def _load() -> ctypes.CDLL:
     lib.pa_decode_attention_noalloc.argtypes = [p, ctypes.c_int, p, p, p, p, i32, p, i32, i32, i32,
                                                 i32, i32, i32, i32, ctypes.c_float, ctypes.c_int,
                                                 i32, p, p]
+    lib.pa_stream_read.restype = ctypes.c_int
+    lib.pa_stream_read.argtypes = [p, i64, p, i32, p]
     lib.pa_bm_create.restype = ctypes.c_int
     lib.pa_bm_create.argtypes = [i32, i32, p, ctypes.POINTER(p)]
     lib.pa_bm_destroy.restype = None
@@ -490,6 +492,20 @@ def decode_attention_noalloc(out: torch.Tensor, query: torch.Tensor, key_cache: 
         d, nb, bs, float(scale), _DTYPE_CODE[query.dtype], int(partition_size),
         _ptr(error_flag), _stream_handle(stream)), "pa_decode_attention_noalloc")
     return out
+
+
+def stream_read(buf: torch.Tensor, sink: torch.Tensor,
+                stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """Read every byte of the contiguous device tensor `buf` once (a
+    measurement of the read-bandwidth ceiling, not a step of the method);
+    sink (int32 or uint32, one entry per CTA) gets each CTA's XOR of the
+    32-bit words it read."""
+    _need(buf.is_cuda and buf.is_contiguous(), "buf must be a contiguous device tensor")
+    _need(sink.is_cuda and sink.is_contiguous() and sink.element_size() == 4,
+          "sink must be a contiguous 32-bit device tensor")
+    _check(lib.pa_stream_read(_ptr(buf), buf.numel() * buf.element_size(), _ptr(sink),
+                              sink.numel(), _stream_handle(stream)), "pa_stream_read")
+    return sink
 
 
 class BlockManager:

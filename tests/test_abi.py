@@ -70,6 +70,14 @@ def test_host_validation_without_gpu(pa):
     assert lib.pa_copy_blocks(None, None, 1, None, 0, 8, 1024, None, None) == 0
     # bad sizes
     assert lib.pa_copy_blocks(None, None, 1, None, 3, 0, 1024, None, None) == 1
+    # the read-bandwidth stream: ragged sizes, unaligned buffers, no sink, bad grids
+    fake = 1 << 20  # a 16-byte aligned address that is never dereferenced
+    assert lib.pa_stream_read(fake, 100, fake, 4, None) == 1
+    assert lib.pa_stream_read(fake + 8, 1024, fake, 4, None) == 1
+    assert lib.pa_stream_read(fake, 1024, None, 4, None) == 1
+    assert lib.pa_stream_read(fake, 1024, fake, 0, None) == 1
+    assert lib.pa_stream_read(fake, 1024, fake, 65536, None) == 1
+    assert lib.pa_stream_read(fake, -16, fake, 4, None) == 1
 
 
 def test_workspace_shape_checks_without_gpu(pa):
