@@ -1,14 +1,16 @@
 // pa_measure.cu -- a read-only HBM stream, the ceiling the decode kernels are
-// held against.  Decode reads each K/V byte once and writes almost nothing
-// ("vAttention: Dynamic Memory Management ...", the decode phase is bound by
-// memory bandwidth), so its roofline is the rate at which this GPU can read,
-// which a copy benchmark (half reads, half writes) does not show directly.
+// held against.  Decode reads each K/V byte once and writes almost nothing,
+// and reading the growing cache is what limits it ("KV cache and
+// PagedAttention: how vLLM uses GPU memory more efficiently", opening
+// section), so its roofline is the rate at which this GPU can read, which a
+// copy benchmark (half reads, half writes) does not show directly.
 //
-// Each thread streams 16-byte words with a grid-stride loop, four loads in
-// flight, and folds them into an XOR; each CTA writes the XOR of everything
-// it read, so nothing can be optimised away and the caller can check that
-// every word was read exactly once (the XOR of the sink equals the XOR of
-// the buffer).
+// Each thread streams 16-byte words with a grid-stride loop, so the loads in
+// flight at any moment cover one contiguous window of the buffer (spreading
+// each thread's loads over several windows measured slower), and folds them
+// into an XOR; each CTA writes the XOR of everything it read, so nothing can
+// be optimised away and the caller can check that every word was read
+// exactly once (the XOR of the sink equals the XOR of the buffer).
 #include <cuda_runtime.h>
 
 #include "pa_device.cuh"
@@ -23,16 +25,10 @@ __device__ __forceinline__ uint32_t fold(const uint4 v) { return v.x ^ v.y ^ v.z
 __global__ void __launch_bounds__(kStreamThreads)
     pa_stream_read_kernel(const uint4* __restrict__ buf, int64_t n16, uint32_t* __restrict__ sink) {
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   uint32_t acc = 0;
-  for (; i + 3 * stride < n16; i += 4 * stride) {
-    const uint4 a = __ldcs(buf + i);
-    const uint4 b = __ldcs(buf + i + stride);
-    const uint4 c = __ldcs(buf + i + 2 * stride);
-    const uint4 d = __ldcs(buf + i + 3 * stride);
-    acc ^= fold(a) ^ fold(b) ^ fold(c) ^ fold(d);
-  }
-  for (; i < n16; i += stride) acc ^= fold(__ldcs(buf + i));
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n16;
+       i += stride)
+    acc ^= fold(__ldcs(buf + i));
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) acc ^= __shfl_xor_sync(0xffffffffu, acc, o);
   __shared__ uint32_t s_warp[kStreamThreads / 32];

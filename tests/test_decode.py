@@ -249,6 +249,22 @@ def test_seq_len_above_max_is_flagged(pa):
 
 # --------------------------------------------------------------------------
 # full sizes, in the launch configuration the benchmark times
+@pytest.mark.parametrize("psize", [0, 16])
+def test_more_sequences_than_the_plans_shared_table(pa, orc, psize):
+    """4500 short sequences: more than the 4096 entries whose tile prefix sums
+    the plan keeps in shared memory, so the plan and the CTAs locate tiles
+    through the prefix sums in the workspace; with 16-token partitions every
+    tile is its own partial."""
+    spec = W.Spec("many", 4500, 8, 2, 64, 16, "bf16", seed=91, len_dist="uniform", len_lo=1,
+                  len_hi=40)
+    prep = prepare(spec)
+    ref = _oracle(orc, prep)
+    flag = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out32 = _run(pa, prep, out_dtype=torch.float32, partition_size=psize, flag=flag)
+    assert _maxerr(out32, ref) <= TOL_F32
+    assert int(flag.item()) == 0
+
+
 # --------------------------------------------------------------------------
 @pytest.mark.slow
 @pytest.mark.parametrize("name", ["llama8b", "longtail", "longctx", "shared_prefix"])

@@ -86,6 +86,17 @@ def test_multi_query_many_sequences(pa, orc):
     _check(pa, orc, spec, prep, q, qs, m)
 
 
+def test_multi_query_more_chunks_than_the_plans_shared_table(pa, orc):
+    """3000 sequences of 1..8 new tokens at group 8 (chunks of 4 query rows):
+    about 4500 entries, more than the 4096 whose prefix sums the plan keeps in
+    shared memory."""
+    spec, prep, q, qs, m = _case(hq=16, hkv=2, d=64, bs=16, B=3000, lo=1, hi=60, qmax=8,
+                                 seed=3007)
+    qlens = np.diff(qs)
+    assert int(np.sum((qlens + 3) // 4)) > 4096
+    _check(pa, orc, spec, prep, q, qs, m)
+
+
 def test_multi_query_edges(pa, orc):
     """No new token for one sequence, more new tokens than the sequence holds
     for another (its first queries see nothing: zeros), a single token."""
