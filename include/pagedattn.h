@@ -503,6 +503,40 @@ pa_status pa_bm_block_table(const pa_block_manager* bm, int64_t seq,
  * PA_ERR_NOT_FOUND if a sequence is unknown. */
 pa_status pa_bm_shared_blocks(const pa_block_manager* bm, const int64_t* seqs, int32_t n,
                               int32_t* out);
+/* One decode step's appends for a batch: for i = 0 .. n-1 in order, reserve
+ * the slot of seqs[i]'s next token (as pa_bm_append_slot).  Host outputs:
+ * slot_mapping[i] (int32, n entries: the slot_mapping of
+ * pa_reshape_and_cache), cow_pairs (int32 [n, 2], (src, dst) of each
+ * copy-on-write in order: the block_mapping of pa_copy_blocks, at most one
+ * per sequence) and *num_cow (pairs written).  All or nothing: if the free
+ * list cannot cover the batch, PA_ERR_OUT_OF_BLOCKS and no state changes.
+ * PA_ERR_NOT_FOUND: an unknown sequence; PA_ERR_INVALID_ARG: a sequence
+ * listed twice, a NULL output; PA_ERR_UNSUPPORTED: slots would not fit in
+ * int32 (num_blocks * block_size > 2^31). */
+pa_status pa_bm_append_slots(pa_block_manager* bm, const int64_t* seqs, int32_t n,
+                             int32_t* slot_mapping, int32_t* cow_pairs, int32_t* num_cow);
+/* The decode metadata for the batch seqs[0 .. n-1]: tables (host int32,
+ * row i at tables + i * width) gets seqs[i]'s block table padded with -1 and
+ * seq_lens[i] (optional, host int32) its length.  Nothing is written on an
+ * error: PA_ERR_NOT_FOUND (unknown sequence), PA_ERR_INVALID_ARG (a table
+ * longer than width, a length above INT32_MAX, NULL tables with width > 0). */
+pa_status pa_bm_fill_tables(const pa_block_manager* bm, const int64_t* seqs, int32_t n,
+                            int32_t* tables, int32_t width, int32_t* seq_lens);
+/* Memory held by the manager's sequences ([PA] "The idea: page the KV cache":
+ * only a last block can be partly empty; "Sharing and copy-on-write": a
+ * shared block is held once). */
+typedef struct pa_bm_stats_t {
+  int64_t num_blocks;        /* pool size */
+  int64_t free_blocks;       /* on the free list */
+  int64_t held_blocks;       /* reference count > 0 */
+  int64_t logical_blocks;    /* sum of the table lengths (blocks held without sharing) */
+  int64_t num_seqs;
+  int64_t tokens;            /* sum of the sequence lengths */
+  int64_t stored_slots;      /* held slots where some sequence holding the block has a token */
+  int64_t waste_slots;       /* held_blocks * block_size - stored_slots */
+  int64_t max_waste_per_seq; /* max over sequences of table slots - tokens (< block_size) */
+} pa_bm_stats_t;
+pa_status pa_bm_stats(const pa_block_manager* bm, pa_bm_stats_t* out);
 /* Reference count of a physical block (-1 if out of range). */
 int32_t pa_bm_refcount(const pa_block_manager* bm, int32_t block);
 int32_t pa_bm_num_free(const pa_block_manager* bm);

@@ -74,6 +74,13 @@ class CacheStrides(ctypes.Structure):
                 ("head_stride", ctypes.c_int64)]
 
 
+class BmStats(ctypes.Structure):
+    """pa_bm_stats_t: memory held by a block manager's sequences."""
+    _fields_ = [(name, ctypes.c_int64) for name in (
+        "num_blocks", "free_blocks", "held_blocks", "logical_blocks", "num_seqs", "tokens",
+        "stored_slots", "waste_slots", "max_waste_per_seq")]
+
+
 def _pool_strides(cache: torch.Tensor) -> Optional[CacheStrides]:
     """None for a contiguous [nb, bs, Hkv, D] pool, else its strides (head_dim
     must be contiguous)."""
@@ -165,6 +172,13 @@ def _load() -> ctypes.CDLL:
     lib.pa_bm_shared_blocks.argtypes = [p, ctypes.POINTER(i64), i32, ctypes.POINTER(i32)]
     lib.pa_bm_num_free.restype = i32
     lib.pa_bm_num_free.argtypes = [p]
+    lib.pa_bm_append_slots.restype = ctypes.c_int
+    lib.pa_bm_append_slots.argtypes = [p, ctypes.POINTER(i64), i32, ctypes.POINTER(i32),
+                                       ctypes.POINTER(i32), ctypes.POINTER(i32)]
+    lib.pa_bm_fill_tables.restype = ctypes.c_int
+    lib.pa_bm_fill_tables.argtypes = [p, ctypes.POINTER(i64), i32, p, i32, p]
+    lib.pa_bm_stats.restype = ctypes.c_int
+    lib.pa_bm_stats.argtypes = [p, ctypes.POINTER(BmStats)]
     return lib
 
 
@@ -522,11 +536,13 @@ class BlockManager:
         else:
             _check(lib.pa_bm_create(num_blocks, block_size, None, ctypes.byref(h)), "pa_bm_create")
         self._h = h
+        # held here: at interpreter exit the module's globals may be gone first
+        self._destroy = lib.pa_bm_destroy
 
     def __del__(self):
         h = getattr(self, "_h", None)
         if h is not None and h.value:
-            lib.pa_bm_destroy(h)
+            self._destroy(h)
             self._h = None
 
     def add_sequence(self, seq: int, num_tokens: int) -> None:
@@ -578,11 +594,45 @@ class BlockManager:
 
     def tables(self, seqs: Sequence[int], width: int) -> torch.Tensor:
         """int32 [len(seqs), width] host tensor of block tables, padded with -1."""
-        t = torch.full((len(seqs), width), -1, dtype=torch.int32)
-        for i, s in enumerate(seqs):
-            row = self.block_table(s)
-            t[i, :len(row)] = torch.tensor(row, dtype=torch.int32)
-        return t
+        return self.fill_tables(seqs, width)[0]
+
+    def fill_tables(self, seqs: Sequence[int], width: int):
+        """(tables int32 [n, width] padded with -1, seq_lens int32 [n]): the
+        decode kernels' metadata for the batch, as host tensors."""
+        n = len(seqs)
+        ids = (ctypes.c_int64 * max(n, 1))(*[int(x) for x in seqs])
+        tables = torch.empty((n, width), dtype=torch.int32)
+        lens = torch.empty((n,), dtype=torch.int32)
+        _check(lib.pa_bm_fill_tables(self._h, ids, n, tables.data_ptr() if tables.numel() else None,
+                                     width, lens.data_ptr() if n else None),
+               "pa_bm_fill_tables")
+        return tables, lens
+
+    def append_slots(self, seqs: Sequence[int]):
+        """One new token for each of seqs, in order, all or nothing: (slot_mapping
+        int32 [n], copy-on-write pairs int32 [k, 2]) as host tensors."""
+        n = len(seqs)
+        ids = (ctypes.c_int64 * max(n, 1))(*[int(x) for x in seqs])
+        slots = (ctypes.c_int32 * max(n, 1))()
+        pairs = (ctypes.c_int32 * max(2 * n, 2))()
+        ncow = ctypes.c_int32()
+        _check(lib.pa_bm_append_slots(self._h, ids, n, slots, pairs, ctypes.byref(ncow)),
+               "pa_bm_append_slots")
+        k = ncow.value
+        return (torch.tensor(list(slots)[:n], dtype=torch.int32),
+                torch.tensor(list(pairs)[:2 * k], dtype=torch.int32).reshape(k, 2))
+
+    def stats(self) -> dict:
+        """Memory the sequences hold (pa_bm_stats), plus occupancy = stored
+        slots / held slots and the saving of sharing = 1 - held / logical."""
+        st = BmStats()
+        _check(lib.pa_bm_stats(self._h, ctypes.byref(st)), "pa_bm_stats")
+        d = {name: int(getattr(st, name)) for name, _ in BmStats._fields_}
+        held_slots = d["held_blocks"] * self.block_size
+        d["occupancy"] = d["stored_slots"] / held_slots if held_slots else 1.0
+        d["sharing_saving"] = (1.0 - d["held_blocks"] / d["logical_blocks"]
+                               if d["logical_blocks"] else 0.0)
+        return d
 
 
 class PagedDecodeStep:

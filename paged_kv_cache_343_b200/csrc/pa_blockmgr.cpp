@@ -13,6 +13,8 @@
 //    writes into the copy.
 // The copy itself is the device's job (pa_copy_blocks); this manager returns
 // the (src, dst) pair.
+#include <algorithm>
+#include <climits>
 #include <cstdint>
 #include <deque>
 #include <new>
@@ -185,4 +187,122 @@ extern "C" int32_t pa_bm_refcount(const pa_block_manager* bm, int32_t block) {
 
 extern "C" int32_t pa_bm_num_free(const pa_block_manager* bm) {
   return bm == nullptr ? -1 : static_cast<int32_t>(bm->free_list.size());
+}
+
+// One step's appends for a batch: the slot of every listed sequence's next
+// token and the copy-on-write pairs, in order, as pa_bm_append_slot would give
+// them one by one.  The blocks the batch needs are counted first, replaying
+// the reference counts the earlier appends of the batch change (a shared
+// partial block copied for one sequence may be written in place by the last
+// one still holding it), so that a batch that does not fit changes nothing.
+extern "C" pa_status pa_bm_append_slots(pa_block_manager* bm, const int64_t* seqs, int32_t n,
+                                        int32_t* slot_mapping, int32_t* cow_pairs,
+                                        int32_t* num_cow) {
+  if (bm == nullptr || n < 0 || num_cow == nullptr ||
+      (n > 0 && (seqs == nullptr || slot_mapping == nullptr || cow_pairs == nullptr)))
+    return PA_ERR_INVALID_ARG;
+  *num_cow = 0;
+  const int32_t bs = bm->block_size;
+  if (static_cast<int64_t>(bm->num_blocks) * bs - 1 > INT32_MAX) return PA_ERR_UNSUPPORTED;
+  std::vector<pa_block_manager::Seq*> rows(static_cast<size_t>(n));
+  std::unordered_map<int64_t, int32_t> seen;
+  for (int32_t i = 0; i < n; ++i) {
+    auto it = bm->seqs.find(seqs[i]);
+    if (it == bm->seqs.end()) return PA_ERR_NOT_FOUND;
+    if (!seen.emplace(seqs[i], i).second) return PA_ERR_INVALID_ARG;  // one token each
+    rows[i] = &it->second;
+  }
+  // dry run: blocks taken from the free list
+  std::unordered_map<int32_t, int32_t> drop;  // refcount decrements so far, per block
+  int64_t need = 0;
+  for (int32_t i = 0; i < n; ++i) {
+    const pa_block_manager::Seq& s = *rows[i];
+    if (s.tokens % bs == 0) {
+      ++need;
+    } else {
+      const int32_t last = s.table.back();
+      if (bm->refcount[last] - drop[last] > 1) {
+        ++need;
+        ++drop[last];
+      }
+    }
+  }
+  if (need > static_cast<int64_t>(bm->free_list.size())) return PA_ERR_OUT_OF_BLOCKS;
+  for (int32_t i = 0; i < n; ++i) {
+    int64_t slot;
+    int32_t src, dst;
+    const pa_status st = pa_bm_append_slot(bm, seqs[i], &slot, &src, &dst);
+    if (st != PA_OK) return st;  // not reached: the dry run found every block
+    slot_mapping[i] = static_cast<int32_t>(slot);
+    if (src >= 0) {
+      cow_pairs[2 * *num_cow] = src;
+      cow_pairs[2 * *num_cow + 1] = dst;
+      ++*num_cow;
+    }
+  }
+  return PA_OK;
+}
+
+// The decode kernels' metadata for a batch: row i of `tables` (row stride
+// `width`) is the block table of seqs[i] padded with -1, seq_lens[i] its
+// length.  Nothing is written if a sequence is unknown, holds more than
+// `width` blocks or more than INT32_MAX tokens.
+extern "C" pa_status pa_bm_fill_tables(const pa_block_manager* bm, const int64_t* seqs,
+                                       int32_t n, int32_t* tables, int32_t width,
+                                       int32_t* seq_lens) {
+  if (bm == nullptr || n < 0 || width < 0 ||
+      (n > 0 && (seqs == nullptr || (width > 0 && tables == nullptr))))
+    return PA_ERR_INVALID_ARG;
+  std::vector<const pa_block_manager::Seq*> rows(static_cast<size_t>(n));
+  for (int32_t i = 0; i < n; ++i) {
+    auto it = bm->seqs.find(seqs[i]);
+    if (it == bm->seqs.end()) return PA_ERR_NOT_FOUND;
+    if (it->second.table.size() > static_cast<size_t>(width) || it->second.tokens > INT32_MAX)
+      return PA_ERR_INVALID_ARG;
+    rows[i] = &it->second;
+  }
+  for (int32_t i = 0; i < n; ++i) {
+    const std::vector<int32_t>& t = rows[i]->table;
+    int32_t* row = tables + static_cast<int64_t>(i) * width;
+    std::copy(t.begin(), t.end(), row);
+    std::fill(row + t.size(), row + width, -1);
+    if (seq_lens) seq_lens[i] = static_cast<int32_t>(rows[i]->tokens);
+  }
+  return PA_OK;
+}
+
+// Memory the sequences hold ("PagedAttention", "The idea: page the KV cache":
+// only a sequence's last block can be partly empty, so waste stays under one
+// block per sequence; "Sharing and copy-on-write": a shared block is held
+// once).  A slot counts as stored when some sequence holding the block has a
+// token there.
+extern "C" pa_status pa_bm_stats(const pa_block_manager* bm, pa_bm_stats_t* out) {
+  if (bm == nullptr || out == nullptr) return PA_ERR_INVALID_ARG;
+  const int64_t bs = bm->block_size;
+  std::vector<int32_t> fill(static_cast<size_t>(bm->num_blocks), 0);  // max tokens per block
+  pa_bm_stats_t st = {};
+  st.num_blocks = bm->num_blocks;
+  st.free_blocks = static_cast<int64_t>(bm->free_list.size());
+  st.num_seqs = static_cast<int64_t>(bm->seqs.size());
+  for (const auto& kv : bm->seqs) {
+    const pa_block_manager::Seq& s = kv.second;
+    const int64_t nb = static_cast<int64_t>(s.table.size());
+    st.logical_blocks += nb;
+    st.tokens += s.tokens;
+    st.max_waste_per_seq = std::max(st.max_waste_per_seq, nb * bs - s.tokens);
+    for (int64_t i = 0; i < nb; ++i) {
+      const int32_t f = static_cast<int32_t>(std::min<int64_t>(bs, s.tokens - i * bs));
+      int32_t& m = fill[static_cast<size_t>(s.table[static_cast<size_t>(i)])];
+      m = std::max(m, f);
+    }
+  }
+  for (int32_t b = 0; b < bm->num_blocks; ++b) {
+    if (bm->refcount[b] > 0) {
+      ++st.held_blocks;
+      st.stored_slots += fill[static_cast<size_t>(b)];
+    }
+  }
+  st.waste_slots = st.held_blocks * bs - st.stored_slots;
+  *out = st;
+  return PA_OK;
 }

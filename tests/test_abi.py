@@ -187,3 +187,140 @@ def test_binding_refuses_mismatched_head_dim(pa):
         pa.reshape_and_cache(torch.zeros(3, 2, 128, dtype=torch.bfloat16),
                              torch.zeros(3, 2, 128, dtype=torch.bfloat16), k, k,
                              torch.zeros(3, dtype=torch.int32))
+
+
+def _sampling_trace(bm, seed, prompts=3, samples=4, prompt_len=10):
+    """Prompts forked into samples (parallel sampling), as both managers see it."""
+    sid = 0
+    for _ in range(prompts):
+        bm.add_sequence(sid, prompt_len + seed)
+        for s in range(1, samples):
+            bm.fork(sid, sid + s)
+        sid += samples
+    return list(range(sid))
+
+
+@pytest.mark.parametrize("seed", [0, 1, 3])
+def test_native_append_slots_matches_one_by_one(pa, seed):
+    """pa_bm_append_slots over a batch gives the slots and copy-on-write pairs
+    of pa_bm_append_slot called in the same order, and of the reference
+    manager, step after step (block boundaries and copies included)."""
+    from oracle.blockmgr import RefBlockManager
+    rng = np.random.default_rng(seed)
+    order = rng.permutation(96).astype(np.int32)
+    batch_bm, one_bm, ref = (pa.BlockManager(96, 4, order), pa.BlockManager(96, 4, order),
+                             RefBlockManager(96, 4, order))
+    seqs = [_sampling_trace(m, seed) for m in (batch_bm, one_bm, ref)][0]
+    for step in range(7):
+        batch = [int(x) for x in rng.permutation(seqs)[:int(rng.integers(1, len(seqs) + 1))]]
+        slots, pairs = batch_bm.append_slots(batch)
+        want_slots, want_pairs = [], []
+        for s in batch:
+            slot, cow = one_bm.append_slot(s)
+            rslot, rcow = ref.append_slot(s)
+            assert (slot, cow) == (rslot, rcow)
+            want_slots.append(slot)
+            if cow is not None:
+                want_pairs.append(cow)
+        assert slots.tolist() == want_slots
+        assert [tuple(p) for p in pairs.tolist()] == want_pairs
+        for s in seqs:
+            assert batch_bm.block_table(s) == ref.block_table(s)
+        ref.check_invariants()
+    assert [batch_bm.refcount(i) for i in range(96)] == [ref.refcount[i] for i in range(96)]
+
+
+def test_native_append_slots_all_or_nothing(pa):
+    """A batch the free list cannot cover fails with PA_ERR_OUT_OF_BLOCKS and
+    changes nothing; an unknown or repeated sequence is refused up front."""
+    bm = pa.BlockManager(5, 4)
+    bm.add_sequence(0, 6)          # blocks 0, 1 (2 of 4 slots used in 1)
+    bm.fork(0, 1)
+    bm.fork(0, 2)                  # block 1 shared three ways, partially filled
+    bm.add_sequence(3, 4)          # block 2, full
+    # seq 0 and seq 1 each copy the shared block, seq 3 needs a new block:
+    # three blocks, two free
+    before = ([bm.block_table(s) for s in range(4)], [bm.refcount(i) for i in range(5)],
+              bm.num_free())
+    with pytest.raises(pa.PagedAttnError) as e:
+        bm.append_slots([0, 1, 3])
+    assert e.value.name == "PA_ERR_OUT_OF_BLOCKS"
+    assert ([bm.block_table(s) for s in range(4)], [bm.refcount(i) for i in range(5)],
+            bm.num_free()) == before
+    # the last holder writes in place: seqs 0, 1 copy, seq 2 does not
+    slots, pairs = bm.append_slots([0, 1, 2])
+    assert pairs.tolist() == [[1, 3], [1, 4]]
+    assert slots.tolist() == [3 * 4 + 2, 4 * 4 + 2, 1 * 4 + 2]
+    assert bm.num_free() == 0
+    for bad, name in (([7], "PA_ERR_NOT_FOUND"), ([0, 0], "PA_ERR_INVALID_ARG")):
+        with pytest.raises(pa.PagedAttnError) as e:
+            bm.append_slots(bad)
+        assert e.value.name == name
+    assert bm.append_slots([])[0].numel() == 0
+
+
+def test_native_fill_tables(pa):
+    bm = pa.BlockManager(32, 4, np.arange(31, -1, -1).astype(np.int32))
+    bm.add_sequence(5, 9)
+    bm.add_sequence(9, 0)
+    bm.add_sequence(2, 4)
+    tables, lens = bm.fill_tables([9, 5, 2], 4)
+    assert tables.tolist() == [[-1, -1, -1, -1], [31, 30, 29, -1], [28, -1, -1, -1]]
+    assert lens.tolist() == [0, 9, 4]
+    with pytest.raises(pa.PagedAttnError) as e:
+        bm.fill_tables([5], 2)      # three blocks do not fit in two columns
+    assert e.value.name == "PA_ERR_INVALID_ARG"
+    with pytest.raises(pa.PagedAttnError) as e:
+        bm.fill_tables([5, 4], 4)
+    assert e.value.name == "PA_ERR_NOT_FOUND"
+
+
+def test_native_stats_by_hand(pa):
+    """Counted by hand: block size 4, a 6-token prompt forked twice, then one
+    token for each of the three sequences (two copy the shared partial block)."""
+    bm = pa.BlockManager(16, 4)
+    bm.add_sequence(0, 6)
+    bm.fork(0, 1)
+    bm.fork(0, 2)
+    st = bm.stats()
+    assert (st["held_blocks"], st["logical_blocks"], st["tokens"]) == (2, 6, 18)
+    assert (st["stored_slots"], st["waste_slots"], st["max_waste_per_seq"]) == (6, 2, 2)
+    bm.append_slots([0, 1, 2])
+    st = bm.stats()
+    # blocks: 0 shared (4 tokens), 1 (seq 2, 3 tokens), 2 and 3 (copies, 3 each)
+    assert (st["held_blocks"], st["free_blocks"], st["logical_blocks"]) == (4, 12, 6)
+    assert (st["tokens"], st["stored_slots"], st["waste_slots"]) == (21, 13, 3)
+    assert st["max_waste_per_seq"] == 1 and st["num_seqs"] == 3
+    assert abs(st["occupancy"] - 13 / 16) < 1e-12
+    assert abs(st["sharing_saving"] - (1 - 4 / 6)) < 1e-12
+
+
+def test_native_stats_agree_with_the_bench_accounting(pa):
+    """On a parallel-sampling workload the native counts equal the benchmark's
+    own count from the tables (blocks held once, blocks without sharing,
+    tokens, largest waste per sequence)."""
+    import bench
+    import pa_workloads as W
+    spec = W.WORKLOADS["shared_prefix"].replace(prompts=4, num_seqs=32, seed=5)
+    case = W.draw(spec)
+    bm = pa.BlockManager(case.num_blocks, spec.block_size, case.free_order)
+    sid = 0
+    for _ in range(spec.prompts):
+        bm.add_sequence(sid, spec.prompt_len)
+        for s in range(1, spec.samples):
+            bm.fork(sid, sid + s)
+        sid += spec.samples
+    for _ in range(int(case.extra_tokens.max())):
+        live = [b for b in range(spec.num_seqs)
+                if bm.seq_len(b) < spec.prompt_len + int(case.extra_tokens[b])]
+        bm.append_slots(live)
+    seqs = list(range(spec.num_seqs))
+    width = max(len(bm.block_table(b)) for b in seqs)
+    tables, lens = bm.fill_tables(seqs, width)
+    mem = bench.kv_memory(spec, {"lens": lens.numpy(), "tables": tables.numpy()})
+    st = bm.stats()
+    assert st["held_blocks"] == mem["blocks_held"]
+    assert st["logical_blocks"] == mem["blocks_if_unshared"]
+    assert st["tokens"] == mem["tokens"]
+    assert st["max_waste_per_seq"] == mem["max_waste_tokens_per_seq"]
+    assert abs(st["sharing_saving"] - mem["sharing_saving"]) < 1e-4
