@@ -177,7 +177,7 @@ def build_workload(spec, pa):
     tables = bm.tables(list(range(B)), width).numpy()
     wl = dict(case=case, lens=lens, tables=tables, slots=np.array(slots, np.int32),
               cow=np.array(cow, np.int32).reshape(-1, 2), new_k=new_k, new_v=new_v,
-              shared_blocks=bm.shared_blocks(list(range(B))).numpy())
+              shared_blocks=bm.shared_blocks(list(range(B))).numpy(), bm_stats=bm.stats())
     _add_queries(spec, wl)
     return wl
 
@@ -566,7 +566,9 @@ def run_ours(args, rank, world, local_rank):
                      "peak_kind": peak_kind + " (MEASURED_PEAKS hbm_gbs, copy read+write)"},
         "attention_latency": latency,
         "read_ceiling": dict(ceiling, frac=round(achieved / ceiling["gbs"], 4)),
-        "kv_memory": kv_memory(spec, wl),
+        "kv_memory": dict(kv_memory(spec, wl), block_manager={
+            k: wl["bm_stats"][k] for k in ("held_blocks", "free_blocks", "stored_slots",
+                                           "waste_slots", "max_waste_per_seq")}),
         "clocks": clock_info,
         "e2e": e2e,
         "gpu_launches": launches_per_step * args.steps,
