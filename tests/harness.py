@@ -3,9 +3,7 @@ device copies.  Block tables and slots here come from the oracle's reference
 block manager (oracle/blockmgr.py), never from the product."""
 from __future__ import annotations
 
-import math
 from dataclasses import dataclass, field
-from typing import List, Optional, Tuple
 
 import numpy as np
 import torch

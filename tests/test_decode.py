@@ -5,7 +5,6 @@ max-abs of the oracle (fp16/bf16 storage, fp32 accumulation); the fp32-output
 mode, which removes the final storage rounding, must be within 1e-4.  Pools are
 NaN-poisoned in every slot that holds no token, so any read past a sequence's
 end or of a block outside its table shows up as NaN."""
-import math
 import os
 
 import numpy as np
@@ -13,7 +12,7 @@ import pytest
 import torch
 
 import pa_workloads as W
-from harness import as_f64, half_ulp, prepare, stored_within, to_dev
+from harness import as_f64, prepare, stored_within, to_dev
 
 pytestmark = pytest.mark.gpu
 
