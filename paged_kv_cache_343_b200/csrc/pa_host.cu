@@ -179,4 +179,4 @@ extern "C" const char* pa_status_string(pa_status status) {
   return "PA_ERR_UNKNOWN";
 }
 
-extern "C" int32_t pa_version(void) { return 100; }
+extern "C" int32_t pa_version(void) { return 200; }
