@@ -208,6 +208,12 @@ def _need(cond: bool, msg: str) -> None:
         raise ValueError(msg)
 
 
+def _dtype_code(dtype: torch.dtype) -> int:
+    _need(dtype in _DTYPE_CODE, "unsupported dtype %s: float16 or bfloat16 (float32 for outputs)"
+          % dtype)
+    return _DTYPE_CODE[dtype]
+
+
 _KV_CACHE_DTYPE = {"auto": 0, "fp8": 1, "fp8_e4m3": 1}
 
 
@@ -246,13 +252,13 @@ def reshape_and_cache(key: torch.Tensor, value: torch.Tensor, key_cache: torch.T
         _check(lib.pa_reshape_and_cache(
             _ptr(key), _ptr(value), key.stride(0), value.stride(0), _ptr(key_cache),
             _ptr(value_cache), _ptr(slot_mapping), key.shape[0], nb, bs, hkv, d,
-            _DTYPE_CODE[key.dtype], _KV_CACHE_DTYPE[kv_cache_dtype], _ptr(k_scale),
+            _dtype_code(key.dtype), _KV_CACHE_DTYPE[kv_cache_dtype], _ptr(k_scale),
             _ptr(v_scale), _ptr(error_flag), _stream_handle(stream)), "pa_reshape_and_cache")
     else:
         _check(lib.pa_reshape_and_cache_strided(
             _ptr(key), _ptr(value), key.stride(0), value.stride(0), _ptr(key_cache),
             _ptr(value_cache), ctypes.byref(strides), _ptr(slot_mapping), key.shape[0], nb, bs,
-            hkv, d, _DTYPE_CODE[key.dtype], _KV_CACHE_DTYPE[kv_cache_dtype], _ptr(k_scale),
+            hkv, d, _dtype_code(key.dtype), _KV_CACHE_DTYPE[kv_cache_dtype], _ptr(k_scale),
             _ptr(v_scale), _ptr(error_flag), _stream_handle(stream)),
             "pa_reshape_and_cache_strided")
 
@@ -330,20 +336,21 @@ def decode_attention(out: torch.Tensor, query: torch.Tensor, key_cache: torch.Te
     B, hq, d = query.shape
     nb, bs, hkv, _ = key_cache.shape
     _need(key_cache.shape[3] == d, "query and pools must share head_dim")
+    _dtype_code(out.dtype), _dtype_code(query.dtype)  # refused before any library call
     if workspace is None:
         workspace = alloc_workspace(decode_workspace_bytes(B, hq, hkv, d, bs, max_seq_len,
                                                            partition_size), query.device)
     wsb = workspace.numel() * workspace.element_size()
     if strides is None:
         _check(lib.pa_decode_attention(
-            _ptr(out), _DTYPE_CODE[out.dtype], _ptr(query), _ptr(key_cache), _ptr(value_cache),
+            _ptr(out), _dtype_code(out.dtype), _ptr(query), _ptr(key_cache), _ptr(value_cache),
             _ptr(block_tables), block_tables.stride(0), _ptr(seq_lens), B, int(max_seq_len), hq,
-            hkv, d, nb, bs, float(scale), _DTYPE_CODE[query.dtype], int(partition_size),
+            hkv, d, nb, bs, float(scale), _dtype_code(query.dtype), int(partition_size),
             _ptr(workspace), wsb, _ptr(error_flag), _stream_handle(stream)),
             "pa_decode_attention")
     else:
         _check(lib.pa_decode_attention_strided(
-            _ptr(out), _DTYPE_CODE[out.dtype], _ptr(query), _DTYPE_CODE[query.dtype],
+            _ptr(out), _dtype_code(out.dtype), _ptr(query), _dtype_code(query.dtype),
             _ptr(key_cache), _ptr(value_cache), ctypes.byref(strides), 0, None, None,
             _ptr(block_tables), block_tables.stride(0), _ptr(seq_lens), B, int(max_seq_len), hq,
             hkv, d, nb, bs, float(scale), int(partition_size), _ptr(workspace), wsb,
@@ -373,20 +380,21 @@ def decode_attention_fp8(out: torch.Tensor, query: torch.Tensor, key_cache: torc
     B, hq, d = query.shape
     nb, bs, hkv, _ = key_cache.shape
     _need(key_cache.shape[3] == d, "query and pools must share head_dim")
+    _dtype_code(out.dtype), _dtype_code(query.dtype)  # refused before any library call
     if workspace is None:
         workspace = alloc_workspace(decode_workspace_bytes(B, hq, hkv, d, bs, max_seq_len,
                                                            partition_size), query.device)
     wsb = workspace.numel() * workspace.element_size()
     if strides is None:
         _check(lib.pa_decode_attention_fp8(
-            _ptr(out), _DTYPE_CODE[out.dtype], _ptr(query), _DTYPE_CODE[query.dtype],
+            _ptr(out), _dtype_code(out.dtype), _ptr(query), _dtype_code(query.dtype),
             _ptr(key_cache), _ptr(value_cache), _ptr(k_scale), _ptr(v_scale), _ptr(block_tables),
             block_tables.stride(0), _ptr(seq_lens), B, int(max_seq_len), hq, hkv, d, nb, bs,
             float(scale), int(partition_size), _ptr(workspace), wsb, _ptr(error_flag),
             _stream_handle(stream)), "pa_decode_attention_fp8")
     else:
         _check(lib.pa_decode_attention_strided(
-            _ptr(out), _DTYPE_CODE[out.dtype], _ptr(query), _DTYPE_CODE[query.dtype],
+            _ptr(out), _dtype_code(out.dtype), _ptr(query), _dtype_code(query.dtype),
             _ptr(key_cache), _ptr(value_cache), ctypes.byref(strides), 1, _ptr(k_scale),
             _ptr(v_scale), _ptr(block_tables), block_tables.stride(0), _ptr(seq_lens), B,
             int(max_seq_len), hq, hkv, d, nb, bs, float(scale), int(partition_size),
@@ -421,13 +429,14 @@ def decode_attention_shared_prefix(out: torch.Tensor, query: torch.Tensor,
     B, hq, d = query.shape
     nb, bs, hkv, _ = key_cache.shape
     _need(key_cache.shape[3] == d, "query and pools must share head_dim")
+    _dtype_code(out.dtype), _dtype_code(query.dtype)  # refused before any library call
     if workspace is None:
         workspace = alloc_workspace(shared_prefix_workspace_bytes(
             B, hq, hkv, d, bs, max_seq_len, partition_size), query.device)
     _check(lib.pa_decode_attention_shared_prefix(
-        _ptr(out), _DTYPE_CODE[out.dtype], _ptr(query), _ptr(key_cache), _ptr(value_cache),
+        _ptr(out), _dtype_code(out.dtype), _ptr(query), _ptr(key_cache), _ptr(value_cache),
         _ptr(block_tables), block_tables.stride(0), _ptr(seq_lens), _ptr(shared_blocks), B,
-        int(max_seq_len), hq, hkv, d, nb, bs, float(scale), _DTYPE_CODE[query.dtype],
+        int(max_seq_len), hq, hkv, d, nb, bs, float(scale), _dtype_code(query.dtype),
         int(partition_size), _ptr(workspace), workspace.numel() * workspace.element_size(),
         _ptr(error_flag), _stream_handle(stream)), "pa_decode_attention_shared_prefix")
     return out
@@ -470,14 +479,15 @@ def decode_attention_multi_query(out: torch.Tensor, query: torch.Tensor, q_start
     B = seq_lens.numel()
     nb, bs, hkv, _ = key_cache.shape
     _need(key_cache.shape[3] == d, "query and pools must share head_dim")
+    _dtype_code(out.dtype), _dtype_code(query.dtype)  # refused before any library call
     if workspace is None:
         workspace = alloc_workspace(multi_query_workspace_bytes(
             B, T, int(max_q_len), hq, hkv, d, bs, int(max_seq_len), partition_size), query.device)
     _check(lib.pa_decode_attention_multi_query(
-        _ptr(out), _DTYPE_CODE[out.dtype], _ptr(query), _ptr(q_start), T, int(max_q_len),
+        _ptr(out), _dtype_code(out.dtype), _ptr(query), _ptr(q_start), T, int(max_q_len),
         _ptr(key_cache), _ptr(value_cache), _ptr(block_tables), block_tables.stride(0),
         _ptr(seq_lens), B, int(max_seq_len), hq, hkv, d, nb, bs, float(scale),
-        _DTYPE_CODE[query.dtype], int(partition_size), _ptr(workspace),
+        _dtype_code(query.dtype), int(partition_size), _ptr(workspace),
         workspace.numel() * workspace.element_size(), _ptr(error_flag), _stream_handle(stream)),
         "pa_decode_attention_multi_query")
     return out
@@ -501,9 +511,9 @@ def decode_attention_noalloc(out: torch.Tensor, query: torch.Tensor, key_cache: 
     nb, bs, hkv, _ = key_cache.shape
     _need(key_cache.shape[3] == d, "query and pools must share head_dim")
     _check(lib.pa_decode_attention_noalloc(
-        _ptr(out), _DTYPE_CODE[out.dtype], _ptr(query), _ptr(key_cache), _ptr(value_cache),
+        _ptr(out), _dtype_code(out.dtype), _ptr(query), _ptr(key_cache), _ptr(value_cache),
         _ptr(block_tables), block_tables.stride(0), _ptr(seq_lens), B, int(max_seq_len), hq, hkv,
-        d, nb, bs, float(scale), _DTYPE_CODE[query.dtype], int(partition_size),
+        d, nb, bs, float(scale), _dtype_code(query.dtype), int(partition_size),
         _ptr(error_flag), _stream_handle(stream)), "pa_decode_attention_noalloc")
     return out
 

@@ -189,6 +189,23 @@ def test_binding_refuses_mismatched_head_dim(pa):
                              torch.zeros(3, dtype=torch.int32))
 
 
+def test_binding_refuses_unsupported_dtypes(pa):
+    """An output or query type the library has no code for is a ValueError
+    raised by the binding, before any call into the library."""
+    import torch
+    q = torch.zeros(2, 8, 64, dtype=torch.bfloat16)
+    k = torch.zeros(4, 16, 2, 64, dtype=torch.bfloat16)
+    tables = torch.zeros(2, 8, dtype=torch.int32)
+    lens = torch.ones(2, dtype=torch.int32)
+    with pytest.raises(ValueError, match="unsupported dtype"):
+        pa.decode_attention(torch.empty(q.shape, dtype=torch.float64), q, k, k, tables, lens,
+                            16, 0.1)
+    q64 = q.double()
+    with pytest.raises(ValueError):
+        pa.decode_attention(torch.empty_like(q64), q64, k.double(), k.double(), tables, lens,
+                            16, 0.1)
+
+
 def _sampling_trace(bm, seed, prompts=3, samples=4, prompt_len=10):
     """Prompts forked into samples (parallel sampling), as both managers see it."""
     sid = 0
