@@ -515,6 +515,18 @@ pa_status pa_bm_shared_blocks(const pa_block_manager* bm, const int64_t* seqs, i
  * int32 (num_blocks * block_size > 2^31). */
 pa_status pa_bm_append_slots(pa_block_manager* bm, const int64_t* seqs, int32_t n,
                              int32_t* slot_mapping, int32_t* cow_pairs, int32_t* num_cow);
+/* Several new tokens per sequence (the multi-query decode's inputs): for
+ * i = 0 .. n-1 in order, reserve the slots of counts[i] >= 0 consecutive new
+ * tokens of seqs[i].  Host outputs: slot_mapping (int32, sum(counts)
+ * entries; may be NULL when the sum is 0), q_start (int32, n + 1 entries:
+ * sequence i's tokens are rows q_start[i] .. q_start[i+1]-1 of the new rows
+ * and of the queries), cow_pairs (int32 [n, 2]; a sequence copies a shared
+ * partial last block at most once, on its first new token) and *num_cow.
+ * All or nothing and the same errors as pa_bm_append_slots; a negative count
+ * is PA_ERR_INVALID_ARG. */
+pa_status pa_bm_append_tokens(pa_block_manager* bm, const int64_t* seqs, int32_t n,
+                              const int32_t* counts, int32_t* slot_mapping, int32_t* q_start,
+                              int32_t* cow_pairs, int32_t* num_cow);
 /* The decode metadata for the batch seqs[0 .. n-1]: tables (host int32,
  * row i at tables + i * width) gets seqs[i]'s block table padded with -1 and
  * seq_lens[i] (optional, host int32) its length.  Nothing is written on an

@@ -175,6 +175,10 @@ def _load() -> ctypes.CDLL:
     lib.pa_bm_append_slots.restype = ctypes.c_int
     lib.pa_bm_append_slots.argtypes = [p, ctypes.POINTER(i64), i32, ctypes.POINTER(i32),
                                        ctypes.POINTER(i32), ctypes.POINTER(i32)]
+    lib.pa_bm_append_tokens.restype = ctypes.c_int
+    lib.pa_bm_append_tokens.argtypes = [p, ctypes.POINTER(i64), i32, ctypes.POINTER(i32),
+                                        ctypes.POINTER(i32), ctypes.POINTER(i32),
+                                        ctypes.POINTER(i32), ctypes.POINTER(i32)]
     lib.pa_bm_fill_tables.restype = ctypes.c_int
     lib.pa_bm_fill_tables.argtypes = [p, ctypes.POINTER(i64), i32, p, i32, p]
     lib.pa_bm_stats.restype = ctypes.c_int
@@ -630,6 +634,27 @@ class BlockManager:
                "pa_bm_append_slots")
         k = ncow.value
         return (torch.tensor(list(slots)[:n], dtype=torch.int32),
+                torch.tensor(list(pairs)[:2 * k], dtype=torch.int32).reshape(k, 2))
+
+    def append_tokens(self, seqs: Sequence[int], counts: Sequence[int]):
+        """counts[i] new tokens for each seqs[i], in order, all or nothing:
+        (slot_mapping int32 [sum(counts)], q_start int32 [n + 1],
+        copy-on-write pairs int32 [k, 2]) as host tensors -- the inputs of
+        reshape_and_cache and decode_attention_multi_query."""
+        n = len(seqs)
+        _need(len(counts) == n, "one count per sequence")
+        ids = (ctypes.c_int64 * max(n, 1))(*[int(x) for x in seqs])
+        cnt = (ctypes.c_int32 * max(n, 1))(*[int(x) for x in counts])
+        total = sum(int(x) for x in counts)
+        slots = (ctypes.c_int32 * max(total, 1))()
+        qs = (ctypes.c_int32 * (n + 1))()
+        pairs = (ctypes.c_int32 * max(2 * n, 2))()
+        ncow = ctypes.c_int32()
+        _check(lib.pa_bm_append_tokens(self._h, ids, n, cnt, slots, qs, pairs, ctypes.byref(ncow)),
+               "pa_bm_append_tokens")
+        k = ncow.value
+        return (torch.tensor(list(slots)[:total], dtype=torch.int32),
+                torch.tensor(list(qs)[:n + 1] if n else [0], dtype=torch.int32),
                 torch.tensor(list(pairs)[:2 * k], dtype=torch.int32).reshape(k, 2))
 
     def stats(self) -> dict:

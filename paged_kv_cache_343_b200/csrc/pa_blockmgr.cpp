@@ -243,6 +243,72 @@ extern "C" pa_status pa_bm_append_slots(pa_block_manager* bm, const int64_t* seq
   return PA_OK;
 }
 
+// Several new tokens per sequence (chunked prefill, speculative tokens): the
+// slots of counts[i] consecutive tokens of seqs[i], for i in order, laid out
+// as the query rows of pa_decode_attention_multi_query (sequence i's tokens
+// at rows q_start[i] .. q_start[i + 1] - 1).  A sequence copies a shared
+// partial last block at most once, on its first new token.  All or nothing,
+// as pa_bm_append_slots.
+extern "C" pa_status pa_bm_append_tokens(pa_block_manager* bm, const int64_t* seqs, int32_t n,
+                                         const int32_t* counts, int32_t* slot_mapping,
+                                         int32_t* q_start, int32_t* cow_pairs,
+                                         int32_t* num_cow) {
+  if (bm == nullptr || n < 0 || num_cow == nullptr ||
+      (n > 0 && (seqs == nullptr || counts == nullptr || q_start == nullptr ||
+                 cow_pairs == nullptr)))
+    return PA_ERR_INVALID_ARG;
+  *num_cow = 0;
+  const int32_t bs = bm->block_size;
+  if (static_cast<int64_t>(bm->num_blocks) * bs - 1 > INT32_MAX) return PA_ERR_UNSUPPORTED;
+  std::vector<pa_block_manager::Seq*> rows(static_cast<size_t>(n));
+  std::unordered_map<int64_t, int32_t> seen;
+  int64_t total = 0;
+  for (int32_t i = 0; i < n; ++i) {
+    auto it = bm->seqs.find(seqs[i]);
+    if (it == bm->seqs.end()) return PA_ERR_NOT_FOUND;
+    if (counts[i] < 0 || !seen.emplace(seqs[i], i).second) return PA_ERR_INVALID_ARG;
+    rows[i] = &it->second;
+    total += counts[i];
+  }
+  if (total > INT32_MAX) return PA_ERR_INVALID_ARG;
+  if (total > 0 && slot_mapping == nullptr) return PA_ERR_INVALID_ARG;
+  // dry run: a copy for a shared partial block, then a block per boundary
+  std::unordered_map<int32_t, int32_t> drop;
+  int64_t need = 0;
+  for (int32_t i = 0; i < n; ++i) {
+    const pa_block_manager::Seq& s = *rows[i];
+    if (counts[i] == 0) continue;
+    if (s.tokens % bs != 0) {
+      const int32_t last = s.table.back();
+      if (bm->refcount[last] - drop[last] > 1) {
+        ++need;
+        ++drop[last];
+      }
+    }
+    const int64_t first = s.tokens, end = s.tokens + counts[i];
+    need += (end + bs - 1) / bs - (first + bs - 1) / bs;  // blocks started by the new tokens
+  }
+  if (need > static_cast<int64_t>(bm->free_list.size())) return PA_ERR_OUT_OF_BLOCKS;
+  int32_t row = 0;
+  for (int32_t i = 0; i < n; ++i) {
+    q_start[i] = row;
+    for (int32_t j = 0; j < counts[i]; ++j) {
+      int64_t slot;
+      int32_t src, dst;
+      const pa_status st = pa_bm_append_slot(bm, seqs[i], &slot, &src, &dst);
+      if (st != PA_OK) return st;  // not reached: the dry run found every block
+      slot_mapping[row++] = static_cast<int32_t>(slot);
+      if (src >= 0) {
+        cow_pairs[2 * *num_cow] = src;
+        cow_pairs[2 * *num_cow + 1] = dst;
+        ++*num_cow;
+      }
+    }
+  }
+  if (n > 0) q_start[n] = row;
+  return PA_OK;
+}
+
 // The decode kernels' metadata for a batch: row i of `tables` (row stride
 // `width`) is the block table of seqs[i] padded with -1, seq_lens[i] its
 // length.  Nothing is written if a sequence is unknown, holds more than

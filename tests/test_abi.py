@@ -341,3 +341,53 @@ def test_native_stats_agree_with_the_bench_accounting(pa):
     assert st["tokens"] == mem["tokens"]
     assert st["max_waste_per_seq"] == mem["max_waste_tokens_per_seq"]
     assert abs(st["sharing_saving"] - mem["sharing_saving"]) < 1e-4
+
+
+@pytest.mark.parametrize("seed", [0, 2])
+def test_native_append_tokens_matches_the_reference_manager(pa, seed):
+    """pa_bm_append_tokens: counts[i] tokens of seqs[i] in order give the
+    slots and copies of the reference manager appending them one by one, and
+    q_start is the running sum of the counts (zero counts included)."""
+    from oracle.blockmgr import RefBlockManager
+    rng = np.random.default_rng(10 + seed)
+    order = rng.permutation(160).astype(np.int32)
+    nat, ref = pa.BlockManager(160, 4, order), RefBlockManager(160, 4, order)
+    seqs = [_sampling_trace(m, seed, prompts=2, samples=3, prompt_len=9) for m in (nat, ref)][0]
+    for step in range(5):
+        batch = [int(x) for x in rng.permutation(seqs)]
+        counts = [int(c) for c in rng.integers(0, 6, len(batch))]
+        slots, q_start, pairs = nat.append_tokens(batch, counts)
+        want_slots, want_pairs = [], []
+        for s, c in zip(batch, counts):
+            for _ in range(c):
+                slot, cow = ref.append_slot(s)
+                want_slots.append(slot)
+                if cow is not None:
+                    want_pairs.append(cow)
+        assert slots.tolist() == want_slots
+        assert [tuple(p) for p in pairs.tolist()] == want_pairs
+        assert q_start.tolist() == [0] + list(np.cumsum(counts))
+        for s in seqs:
+            assert nat.block_table(s) == ref.block_table(s)
+        ref.check_invariants()
+
+
+def test_native_append_tokens_all_or_nothing(pa):
+    bm = pa.BlockManager(4, 4)
+    bm.add_sequence(0, 6)           # blocks 0, 1
+    bm.fork(0, 1)                   # block 1 shared and partial
+    before = ([bm.block_table(s) for s in range(2)], bm.num_free())
+    # seq 0: a copy of block 1 plus one new block for positions 8..9 -> 2;
+    # seq 1: then the last holder of block 1, writes in place, and needs a new
+    # block for positions 8..11 -> 1; three blocks, two free
+    with pytest.raises(pa.PagedAttnError) as e:
+        bm.append_tokens([0, 1], [4, 6])
+    assert e.value.name == "PA_ERR_OUT_OF_BLOCKS"
+    assert ([bm.block_table(s) for s in range(2)], bm.num_free()) == before
+    with pytest.raises(pa.PagedAttnError) as e:
+        bm.append_tokens([0], [-1])
+    assert e.value.name == "PA_ERR_INVALID_ARG"
+    slots, q_start, pairs = bm.append_tokens([0, 1], [4, 2])
+    assert q_start.tolist() == [0, 4, 6] and pairs.tolist() == [[1, 2]]
+    assert slots.tolist() == [2 * 4 + 2, 2 * 4 + 3, 3 * 4 + 0, 3 * 4 + 1, 1 * 4 + 2, 1 * 4 + 3]
+    assert bm.num_free() == 0
