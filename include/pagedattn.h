@@ -527,6 +527,12 @@ pa_status pa_bm_append_slots(pa_block_manager* bm, const int64_t* seqs, int32_t 
 pa_status pa_bm_append_tokens(pa_block_manager* bm, const int64_t* seqs, int32_t n,
                               const int32_t* counts, int32_t* slot_mapping, int32_t* q_start,
                               int32_t* cow_pairs, int32_t* num_cow);
+/* Capacity check for a scheduler: *need gets the free blocks that
+ * pa_bm_append_tokens(seqs, counts) (counts NULL: one token each, as
+ * pa_bm_append_slots) would take -- copies of shared partial blocks plus new
+ * blocks -- without changing any state.  Errors as pa_bm_append_tokens. */
+pa_status pa_bm_blocks_needed(const pa_block_manager* bm, const int64_t* seqs, int32_t n,
+                              const int32_t* counts, int64_t* need);
 /* The decode metadata for the batch seqs[0 .. n-1]: tables (host int32,
  * row i at tables + i * width) gets seqs[i]'s block table padded with -1 and
  * seq_lens[i] (optional, host int32) its length.  Nothing is written on an

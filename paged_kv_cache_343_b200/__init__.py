@@ -179,6 +179,8 @@ def _load() -> ctypes.CDLL:
     lib.pa_bm_append_tokens.argtypes = [p, ctypes.POINTER(i64), i32, ctypes.POINTER(i32),
                                         ctypes.POINTER(i32), ctypes.POINTER(i32),
                                         ctypes.POINTER(i32), ctypes.POINTER(i32)]
+    lib.pa_bm_blocks_needed.restype = ctypes.c_int
+    lib.pa_bm_blocks_needed.argtypes = [p, ctypes.POINTER(i64), i32, p, ctypes.POINTER(i64)]
     lib.pa_bm_fill_tables.restype = ctypes.c_int
     lib.pa_bm_fill_tables.argtypes = [p, ctypes.POINTER(i64), i32, p, i32, p]
     lib.pa_bm_stats.restype = ctypes.c_int
@@ -656,6 +658,20 @@ class BlockManager:
         return (torch.tensor(list(slots)[:total], dtype=torch.int32),
                 torch.tensor(list(qs)[:n + 1] if n else [0], dtype=torch.int32),
                 torch.tensor(list(pairs)[:2 * k], dtype=torch.int32).reshape(k, 2))
+
+    def blocks_needed(self, seqs: Sequence[int], counts: Optional[Sequence[int]] = None) -> int:
+        """Free blocks append_tokens(seqs, counts) (or append_slots(seqs) when
+        counts is None) would take, with no change to any table."""
+        n = len(seqs)
+        ids = (ctypes.c_int64 * max(n, 1))(*[int(x) for x in seqs])
+        cnt = None
+        if counts is not None:
+            _need(len(counts) == n, "one count per sequence")
+            cnt = (ctypes.c_int32 * max(n, 1))(*[int(x) for x in counts])
+        need = ctypes.c_int64()
+        _check(lib.pa_bm_blocks_needed(self._h, ids, n, cnt, ctypes.byref(need)),
+               "pa_bm_blocks_needed")
+        return int(need.value)
 
     def stats(self) -> dict:
         """Memory the sequences hold (pa_bm_stats), plus occupancy = stored

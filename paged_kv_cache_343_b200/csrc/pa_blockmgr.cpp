@@ -189,115 +189,65 @@ extern "C" int32_t pa_bm_num_free(const pa_block_manager* bm) {
   return bm == nullptr ? -1 : static_cast<int32_t>(bm->free_list.size());
 }
 
-// One step's appends for a batch: the slot of every listed sequence's next
-// token and the copy-on-write pairs, in order, as pa_bm_append_slot would give
-// them one by one.  The blocks the batch needs are counted first, replaying
-// the reference counts the earlier appends of the batch change (a shared
-// partial block copied for one sequence may be written in place by the last
-// one still holding it), so that a batch that does not fit changes nothing.
-extern "C" pa_status pa_bm_append_slots(pa_block_manager* bm, const int64_t* seqs, int32_t n,
-                                        int32_t* slot_mapping, int32_t* cow_pairs,
-                                        int32_t* num_cow) {
-  if (bm == nullptr || n < 0 || num_cow == nullptr ||
-      (n > 0 && (seqs == nullptr || slot_mapping == nullptr || cow_pairs == nullptr)))
-    return PA_ERR_INVALID_ARG;
-  *num_cow = 0;
-  const int32_t bs = bm->block_size;
-  if (static_cast<int64_t>(bm->num_blocks) * bs - 1 > INT32_MAX) return PA_ERR_UNSUPPORTED;
-  std::vector<pa_block_manager::Seq*> rows(static_cast<size_t>(n));
+namespace {
+
+// The sequences of a batch, checked: known, listed once, counts >= 0 (NULL
+// counts = one token each).  *total gets the sum of the counts.
+pa_status batch_rows(pa_block_manager* bm, const int64_t* seqs, int32_t n, const int32_t* counts,
+                     std::vector<pa_block_manager::Seq*>* rows, int64_t* total) {
+  rows->assign(static_cast<size_t>(n), nullptr);
   std::unordered_map<int64_t, int32_t> seen;
+  *total = 0;
   for (int32_t i = 0; i < n; ++i) {
     auto it = bm->seqs.find(seqs[i]);
     if (it == bm->seqs.end()) return PA_ERR_NOT_FOUND;
-    if (!seen.emplace(seqs[i], i).second) return PA_ERR_INVALID_ARG;  // one token each
-    rows[i] = &it->second;
-  }
-  // dry run: blocks taken from the free list
-  std::unordered_map<int32_t, int32_t> drop;  // refcount decrements so far, per block
-  int64_t need = 0;
-  for (int32_t i = 0; i < n; ++i) {
-    const pa_block_manager::Seq& s = *rows[i];
-    if (s.tokens % bs == 0) {
-      ++need;
-    } else {
-      const int32_t last = s.table.back();
-      if (bm->refcount[last] - drop[last] > 1) {
-        ++need;
-        ++drop[last];
-      }
-    }
-  }
-  if (need > static_cast<int64_t>(bm->free_list.size())) return PA_ERR_OUT_OF_BLOCKS;
-  for (int32_t i = 0; i < n; ++i) {
-    int64_t slot;
-    int32_t src, dst;
-    const pa_status st = pa_bm_append_slot(bm, seqs[i], &slot, &src, &dst);
-    if (st != PA_OK) return st;  // not reached: the dry run found every block
-    slot_mapping[i] = static_cast<int32_t>(slot);
-    if (src >= 0) {
-      cow_pairs[2 * *num_cow] = src;
-      cow_pairs[2 * *num_cow + 1] = dst;
-      ++*num_cow;
-    }
+    const int32_t c = counts ? counts[i] : 1;
+    if (c < 0 || !seen.emplace(seqs[i], i).second) return PA_ERR_INVALID_ARG;
+    (*rows)[static_cast<size_t>(i)] = &it->second;
+    *total += c;
   }
   return PA_OK;
 }
 
-// Several new tokens per sequence (chunked prefill, speculative tokens): the
-// slots of counts[i] consecutive tokens of seqs[i], for i in order, laid out
-// as the query rows of pa_decode_attention_multi_query (sequence i's tokens
-// at rows q_start[i] .. q_start[i + 1] - 1).  A sequence copies a shared
-// partial last block at most once, on its first new token.  All or nothing,
-// as pa_bm_append_slots.
-extern "C" pa_status pa_bm_append_tokens(pa_block_manager* bm, const int64_t* seqs, int32_t n,
-                                         const int32_t* counts, int32_t* slot_mapping,
-                                         int32_t* q_start, int32_t* cow_pairs,
-                                         int32_t* num_cow) {
-  if (bm == nullptr || n < 0 || num_cow == nullptr ||
-      (n > 0 && (seqs == nullptr || counts == nullptr || q_start == nullptr ||
-                 cow_pairs == nullptr)))
-    return PA_ERR_INVALID_ARG;
-  *num_cow = 0;
-  const int32_t bs = bm->block_size;
-  if (static_cast<int64_t>(bm->num_blocks) * bs - 1 > INT32_MAX) return PA_ERR_UNSUPPORTED;
-  std::vector<pa_block_manager::Seq*> rows(static_cast<size_t>(n));
-  std::unordered_map<int64_t, int32_t> seen;
-  int64_t total = 0;
-  for (int32_t i = 0; i < n; ++i) {
-    auto it = bm->seqs.find(seqs[i]);
-    if (it == bm->seqs.end()) return PA_ERR_NOT_FOUND;
-    if (counts[i] < 0 || !seen.emplace(seqs[i], i).second) return PA_ERR_INVALID_ARG;
-    rows[i] = &it->second;
-    total += counts[i];
-  }
-  if (total > INT32_MAX) return PA_ERR_INVALID_ARG;
-  if (total > 0 && slot_mapping == nullptr) return PA_ERR_INVALID_ARG;
-  // dry run: a copy for a shared partial block, then a block per boundary
+// Blocks the free list must give for the batch's appends, without changing
+// anything: for each sequence in order, a copy when its first new token falls
+// into a partial last block that some other sequence still holds (replaying
+// the reference counts the earlier copies of the batch release: the last
+// holder writes in place), then one block per block boundary its new tokens
+// start.
+int64_t blocks_needed(const pa_block_manager* bm,
+                      const std::vector<pa_block_manager::Seq*>& rows, const int32_t* counts) {
+  const int64_t bs = bm->block_size;
   std::unordered_map<int32_t, int32_t> drop;
   int64_t need = 0;
-  for (int32_t i = 0; i < n; ++i) {
+  for (size_t i = 0; i < rows.size(); ++i) {
+    const int32_t c = counts ? counts[i] : 1;
+    if (c == 0) continue;
     const pa_block_manager::Seq& s = *rows[i];
-    if (counts[i] == 0) continue;
     if (s.tokens % bs != 0) {
       const int32_t last = s.table.back();
-      if (bm->refcount[last] - drop[last] > 1) {
+      if (bm->refcount[static_cast<size_t>(last)] - drop[last] > 1) {
         ++need;
         ++drop[last];
       }
     }
-    const int64_t first = s.tokens, end = s.tokens + counts[i];
-    need += (end + bs - 1) / bs - (first + bs - 1) / bs;  // blocks started by the new tokens
+    need += (s.tokens + c + bs - 1) / bs - (s.tokens + bs - 1) / bs;
   }
-  if (need > static_cast<int64_t>(bm->free_list.size())) return PA_ERR_OUT_OF_BLOCKS;
+  return need;
+}
+
+// The appends themselves, after the checks and the dry run.
+void append_batch(pa_block_manager* bm, const int64_t* seqs, int32_t n, const int32_t* counts,
+                  int32_t* slot_mapping, int32_t* q_start, int32_t* cow_pairs, int32_t* num_cow) {
   int32_t row = 0;
   for (int32_t i = 0; i < n; ++i) {
-    q_start[i] = row;
-    for (int32_t j = 0; j < counts[i]; ++j) {
+    if (q_start) q_start[i] = row;
+    const int32_t c = counts ? counts[i] : 1;
+    for (int32_t j = 0; j < c; ++j) {
       int64_t slot;
       int32_t src, dst;
-      const pa_status st = pa_bm_append_slot(bm, seqs[i], &slot, &src, &dst);
-      if (st != PA_OK) return st;  // not reached: the dry run found every block
-      slot_mapping[row++] = static_cast<int32_t>(slot);
+      pa_bm_append_slot(bm, seqs[i], &slot, &src, &dst);  // cannot fail: the dry run
+      slot_mapping[row++] = static_cast<int32_t>(slot);  // found every block
       if (src >= 0) {
         cow_pairs[2 * *num_cow] = src;
         cow_pairs[2 * *num_cow + 1] = dst;
@@ -305,7 +255,65 @@ extern "C" pa_status pa_bm_append_tokens(pa_block_manager* bm, const int64_t* se
       }
     }
   }
-  if (n > 0) q_start[n] = row;
+  if (q_start && n > 0) q_start[n] = row;
+}
+
+pa_status append_checked(pa_block_manager* bm, const int64_t* seqs, int32_t n,
+                         const int32_t* counts, int32_t* slot_mapping, int32_t* q_start,
+                         int32_t* cow_pairs, int32_t* num_cow) {
+  if (bm == nullptr || n < 0 || num_cow == nullptr ||
+      (n > 0 && (seqs == nullptr || cow_pairs == nullptr)))
+    return PA_ERR_INVALID_ARG;
+  *num_cow = 0;
+  if (static_cast<int64_t>(bm->num_blocks) * bm->block_size - 1 > INT32_MAX)
+    return PA_ERR_UNSUPPORTED;
+  std::vector<pa_block_manager::Seq*> rows;
+  int64_t total = 0;
+  const pa_status st = batch_rows(bm, seqs, n, counts, &rows, &total);
+  if (st != PA_OK) return st;
+  if (total > INT32_MAX || (total > 0 && slot_mapping == nullptr)) return PA_ERR_INVALID_ARG;
+  if (blocks_needed(bm, rows, counts) > static_cast<int64_t>(bm->free_list.size()))
+    return PA_ERR_OUT_OF_BLOCKS;
+  append_batch(bm, seqs, n, counts, slot_mapping, q_start, cow_pairs, num_cow);
+  return PA_OK;
+}
+
+}  // namespace
+
+// One step's appends for a batch: the slot of every listed sequence's next
+// token and the copy-on-write pairs, in order, as pa_bm_append_slot would give
+// them one by one; a batch that does not fit changes nothing.
+extern "C" pa_status pa_bm_append_slots(pa_block_manager* bm, const int64_t* seqs, int32_t n,
+                                        int32_t* slot_mapping, int32_t* cow_pairs,
+                                        int32_t* num_cow) {
+  return append_checked(bm, seqs, n, nullptr, slot_mapping, nullptr, cow_pairs, num_cow);
+}
+
+// Several new tokens per sequence (chunked prefill, speculative tokens): the
+// slots of counts[i] consecutive tokens of seqs[i], for i in order, laid out
+// as the query rows of pa_decode_attention_multi_query (sequence i's tokens
+// at rows q_start[i] .. q_start[i + 1] - 1).  A sequence copies a shared
+// partial last block at most once, on its first new token.
+extern "C" pa_status pa_bm_append_tokens(pa_block_manager* bm, const int64_t* seqs, int32_t n,
+                                         const int32_t* counts, int32_t* slot_mapping,
+                                         int32_t* q_start, int32_t* cow_pairs,
+                                         int32_t* num_cow) {
+  if (n > 0 && (counts == nullptr || q_start == nullptr)) return PA_ERR_INVALID_ARG;
+  return append_checked(bm, seqs, n, counts, slot_mapping, q_start, cow_pairs, num_cow);
+}
+
+// What a scheduler asks before it admits a batch: the free blocks the appends
+// would take (0 .. ), with no change to any table.
+extern "C" pa_status pa_bm_blocks_needed(const pa_block_manager* bm, const int64_t* seqs,
+                                         int32_t n, const int32_t* counts, int64_t* need) {
+  if (bm == nullptr || n < 0 || need == nullptr || (n > 0 && seqs == nullptr))
+    return PA_ERR_INVALID_ARG;
+  std::vector<pa_block_manager::Seq*> rows;
+  int64_t total = 0;
+  const pa_status st =
+      batch_rows(const_cast<pa_block_manager*>(bm), seqs, n, counts, &rows, &total);
+  if (st != PA_OK) return st;
+  *need = blocks_needed(bm, rows, counts);
   return PA_OK;
 }
 

@@ -391,3 +391,28 @@ def test_native_append_tokens_all_or_nothing(pa):
     assert q_start.tolist() == [0, 4, 6] and pairs.tolist() == [[1, 2]]
     assert slots.tolist() == [2 * 4 + 2, 2 * 4 + 3, 3 * 4 + 0, 3 * 4 + 1, 1 * 4 + 2, 1 * 4 + 3]
     assert bm.num_free() == 0
+
+
+def test_native_blocks_needed_predicts_the_appends(pa):
+    """pa_bm_blocks_needed changes nothing and equals the free blocks the
+    following append call takes, copies of shared partial blocks included."""
+    rng = np.random.default_rng(4)
+    bm = pa.BlockManager(400, 4, rng.permutation(400).astype(np.int32))
+    seqs = _sampling_trace(bm, 1, prompts=3, samples=4, prompt_len=9)
+    for step in range(6):
+        batch = [int(x) for x in rng.permutation(seqs)]
+        if step % 2:
+            counts = [int(c) for c in rng.integers(0, 7, len(batch))]
+            tables = [bm.block_table(s) for s in seqs]
+            need = bm.blocks_needed(batch, counts)
+            assert [bm.block_table(s) for s in seqs] == tables
+            free = bm.num_free()
+            bm.append_tokens(batch, counts)
+        else:
+            need = bm.blocks_needed(batch)
+            free = bm.num_free()
+            bm.append_slots(batch)
+        assert free - bm.num_free() == need
+    with pytest.raises(pa.PagedAttnError) as e:
+        bm.blocks_needed([0, 0])
+    assert e.value.name == "PA_ERR_INVALID_ARG"
