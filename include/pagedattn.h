@@ -483,6 +483,23 @@ pa_status pa_bm_create(int32_t num_blocks, int32_t block_size,
 void pa_bm_destroy(pa_block_manager* bm);
 /* A new sequence that already holds num_tokens tokens: ceil(n / bs) blocks. */
 pa_status pa_bm_add_sequence(pa_block_manager* bm, int64_t seq, int64_t num_tokens);
+/* Prefix caching ([PA] "Sharing and copy-on-write": requests with the same
+ * system prompt share blocks; full blocks are never written again).  A new
+ * sequence whose num_tokens prompt tokens are token_ids (host int32): its
+ * leading FULL blocks whose tokens -- and every token before them -- match
+ * a block still held in the manager are shared (refcount + 1) and
+ * *cached_tokens gets how many tokens they hold (a multiple of block_size);
+ * the other blocks are allocated and its new full blocks are entered in the
+ * cache (a partial last block never is).  Rows of tokens cached_tokens ..
+ * num_tokens - 1 are the caller's to write (pa_reshape_and_cache) before any
+ * attention reads them; the multi-query decode attends the uncached tokens
+ * over the shared ones.  Matches compare token ids exactly.  A cache entry
+ * lives while its block is held; blocks that return to the free list leave
+ * the cache.  All or nothing (PA_ERR_OUT_OF_BLOCKS changes nothing);
+ * PA_ERR_INVALID_ARG for a known seq id or NULL pointers. */
+pa_status pa_bm_add_sequence_with_prefix(pa_block_manager* bm, int64_t seq,
+                                         const int32_t* token_ids, int64_t num_tokens,
+                                         int64_t* cached_tokens);
 /* child shares all of parent's blocks (each refcount + 1). */
 pa_status pa_bm_fork(pa_block_manager* bm, int64_t parent, int64_t child);
 /* Reserve the slot of seq's next token.  *slot gets the flat slot; if the
@@ -553,6 +570,7 @@ typedef struct pa_bm_stats_t {
   int64_t stored_slots;      /* held slots where some sequence holding the block has a token */
   int64_t waste_slots;       /* held_blocks * block_size - stored_slots */
   int64_t max_waste_per_seq; /* max over sequences of table slots - tokens (< block_size) */
+  int64_t cached_blocks;     /* full blocks in the prefix cache */
 } pa_bm_stats_t;
 pa_status pa_bm_stats(const pa_block_manager* bm, pa_bm_stats_t* out);
 /* Reference count of a physical block (-1 if out of range). */

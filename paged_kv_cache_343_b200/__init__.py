@@ -78,7 +78,7 @@ class BmStats(ctypes.Structure):
     """pa_bm_stats_t: memory held by a block manager's sequences."""
     _fields_ = [(name, ctypes.c_int64) for name in (
         "num_blocks", "free_blocks", "held_blocks", "logical_blocks", "num_seqs", "tokens",
-        "stored_slots", "waste_slots", "max_waste_per_seq")]
+        "stored_slots", "waste_slots", "max_waste_per_seq", "cached_blocks")]
 
 
 def _pool_strides(cache: torch.Tensor) -> Optional[CacheStrides]:
@@ -157,6 +157,9 @@ def _load() -> ctypes.CDLL:
     lib.pa_bm_destroy.argtypes = [p]
     lib.pa_bm_add_sequence.restype = ctypes.c_int
     lib.pa_bm_add_sequence.argtypes = [p, i64, i64]
+    lib.pa_bm_add_sequence_with_prefix.restype = ctypes.c_int
+    lib.pa_bm_add_sequence_with_prefix.argtypes = [p, i64, ctypes.POINTER(i32), i64,
+                                                   ctypes.POINTER(i64)]
     lib.pa_bm_fork.restype = ctypes.c_int
     lib.pa_bm_fork.argtypes = [p, i64, i64]
     lib.pa_bm_append_slot.restype = ctypes.c_int
@@ -563,6 +566,17 @@ class BlockManager:
 
     def add_sequence(self, seq: int, num_tokens: int) -> None:
         _check(lib.pa_bm_add_sequence(self._h, seq, num_tokens), "pa_bm_add_sequence")
+
+    def add_sequence_with_prefix(self, seq: int, token_ids: Sequence[int]) -> int:
+        """A new request with its prompt's token ids: shares the leading full
+        blocks the prefix cache holds for the same tokens and returns how many
+        tokens those hold (their rows are already in the pool)."""
+        n = len(token_ids)
+        toks = (ctypes.c_int32 * max(n, 1))(*[int(t) for t in token_ids])
+        cached = ctypes.c_int64()
+        _check(lib.pa_bm_add_sequence_with_prefix(self._h, seq, toks, n, ctypes.byref(cached)),
+               "pa_bm_add_sequence_with_prefix")
+        return int(cached.value)
 
     def fork(self, parent: int, child: int) -> None:
         _check(lib.pa_bm_fork(self._h, parent, child), "pa_bm_fork")

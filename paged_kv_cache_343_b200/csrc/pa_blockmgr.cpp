@@ -13,6 +13,15 @@
 //    writes into the copy.
 // The copy itself is the device's job (pa_copy_blocks); this manager returns
 // the (src, dst) pair.
+//
+// Prefix caching ("Sharing and copy-on-write": requests with the same system
+// prompt share blocks; full blocks are never written again, so they can be
+// shared for as long as they live): a full block added with its token ids is
+// entered in an index under (the physical block before it, its tokens); a
+// later request whose prompt starts with the same tokens finds its leading
+// full blocks there and shares them.  The match is exact (the tokens are
+// compared, not only hashed) and chained (a block matches only after its
+// predecessor did).  An entry lives as long as its block is held.
 #include <algorithm>
 #include <climits>
 #include <cstdint>
@@ -33,6 +42,63 @@ struct pa_block_manager {
     int64_t tokens = 0;
   };
   std::unordered_map<int64_t, Seq> seqs;
+  // prefix cache: entry of a physical block (valid while the block is held)
+  struct Cached {
+    bool valid = false;
+    uint64_t key = 0;
+    int32_t parent = -1;          // the physical block before it in its table
+    std::vector<int32_t> tokens;  // its block_size token ids
+  };
+  std::vector<Cached> cached;
+  std::unordered_multimap<uint64_t, int32_t> prefix_index;  // key -> block
+  int64_t num_cached = 0;
+
+  static uint64_t key_of(int32_t parent, const int32_t* tokens, int32_t n) {
+    uint64_t h = 1469598103934665603ull;  // FNV-1a over the parent id and the tokens
+    auto mix = [&h](uint32_t v) {
+      for (int b = 0; b < 4; ++b) {
+        h ^= (v >> (8 * b)) & 0xffu;
+        h *= 1099511628211ull;
+      }
+    };
+    mix(static_cast<uint32_t>(parent));
+    for (int32_t i = 0; i < n; ++i) mix(static_cast<uint32_t>(tokens[i]));
+    return h;
+  }
+  // the held block whose entry is (parent, tokens), or -1
+  int32_t find_cached(int32_t parent, const int32_t* tokens) const {
+    const uint64_t key = key_of(parent, tokens, block_size);
+    auto range = prefix_index.equal_range(key);
+    for (auto it = range.first; it != range.second; ++it) {
+      const Cached& c = cached[static_cast<size_t>(it->second)];
+      if (c.parent == parent &&
+          std::equal(c.tokens.begin(), c.tokens.end(), tokens))
+        return it->second;
+    }
+    return -1;
+  }
+  void enter_cached(int32_t blk, int32_t parent, const int32_t* tokens) {
+    Cached& c = cached[static_cast<size_t>(blk)];
+    c.valid = true;
+    c.key = key_of(parent, tokens, block_size);
+    c.parent = parent;
+    c.tokens.assign(tokens, tokens + block_size);
+    prefix_index.emplace(c.key, blk);
+    ++num_cached;
+  }
+  void forget_cached(int32_t blk) {
+    Cached& c = cached[static_cast<size_t>(blk)];
+    if (!c.valid) return;
+    auto range = prefix_index.equal_range(c.key);
+    for (auto it = range.first; it != range.second; ++it) {
+      if (it->second == blk) {
+        prefix_index.erase(it);
+        break;
+      }
+    }
+    c = Cached();
+    --num_cached;
+  }
 
   bool alloc(int32_t* out) {
     if (free_list.empty()) return false;
@@ -42,7 +108,10 @@ struct pa_block_manager {
     return true;
   }
   void release(int32_t blk) {
-    if (--refcount[blk] == 0) free_list.push_back(blk);
+    if (--refcount[blk] == 0) {
+      forget_cached(blk);
+      free_list.push_back(blk);
+    }
   }
 };
 
@@ -55,6 +124,7 @@ extern "C" pa_status pa_bm_create(int32_t num_blocks, int32_t block_size,
   bm->num_blocks = num_blocks;
   bm->block_size = block_size;
   bm->refcount.assign(num_blocks, 0);
+  bm->cached.resize(static_cast<size_t>(num_blocks));
   if (free_order == nullptr) {
     for (int32_t i = 0; i < num_blocks; ++i) bm->free_list.push_back(i);
   } else {
@@ -89,6 +159,52 @@ extern "C" pa_status pa_bm_add_sequence(pa_block_manager* bm, int64_t seq, int64
     s.table.push_back(blk);
   }
   bm->seqs.emplace(seq, std::move(s));
+  return PA_OK;
+}
+
+// A new request of num_tokens prompt tokens `token_ids`: its leading full
+// blocks that match the prefix cache are shared (their key and value rows are
+// already in the pool: *cached_tokens of them, a multiple of block_size), the
+// rest are allocated, and its own full blocks are entered in the cache.  The
+// caller writes the rows of tokens cached_tokens .. num_tokens - 1 before any
+// attention reads them.  All or nothing.
+extern "C" pa_status pa_bm_add_sequence_with_prefix(pa_block_manager* bm, int64_t seq,
+                                                    const int32_t* token_ids,
+                                                    int64_t num_tokens,
+                                                    int64_t* cached_tokens) {
+  if (bm == nullptr || num_tokens < 0 || cached_tokens == nullptr ||
+      (num_tokens > 0 && token_ids == nullptr))
+    return PA_ERR_INVALID_ARG;
+  if (bm->seqs.count(seq)) return PA_ERR_INVALID_ARG;
+  const int32_t bs = bm->block_size;
+  const int64_t full = num_tokens / bs;
+  const int64_t need_all = (num_tokens + bs - 1) / bs;
+  // leading full blocks found in the cache
+  std::vector<int32_t> hits;
+  int32_t parent = -1;
+  for (int64_t i = 0; i < full; ++i) {
+    const int32_t blk = bm->find_cached(parent, token_ids + i * bs);
+    if (blk < 0) break;
+    hits.push_back(blk);
+    parent = blk;
+  }
+  const int64_t fresh = need_all - static_cast<int64_t>(hits.size());
+  if (fresh > static_cast<int64_t>(bm->free_list.size())) return PA_ERR_OUT_OF_BLOCKS;
+  pa_block_manager::Seq s;
+  s.tokens = num_tokens;
+  s.table.reserve(static_cast<size_t>(need_all));
+  for (int32_t blk : hits) {
+    ++bm->refcount[static_cast<size_t>(blk)];
+    s.table.push_back(blk);
+  }
+  for (int64_t i = static_cast<int64_t>(hits.size()); i < need_all; ++i) {
+    int32_t blk;
+    bm->alloc(&blk);
+    if (i < full) bm->enter_cached(blk, s.table.empty() ? -1 : s.table.back(), token_ids + i * bs);
+    s.table.push_back(blk);
+  }
+  bm->seqs.emplace(seq, std::move(s));
+  *cached_tokens = static_cast<int64_t>(hits.size()) * bs;
   return PA_OK;
 }
 
@@ -377,6 +493,7 @@ extern "C" pa_status pa_bm_stats(const pa_block_manager* bm, pa_bm_stats_t* out)
     }
   }
   st.waste_slots = st.held_blocks * bs - st.stored_slots;
+  st.cached_blocks = bm->num_cached;
   *out = st;
   return PA_OK;
 }

@@ -416,3 +416,71 @@ def test_native_blocks_needed_predicts_the_appends(pa):
     with pytest.raises(pa.PagedAttnError) as e:
         bm.blocks_needed([0, 0])
     assert e.value.name == "PA_ERR_INVALID_ARG"
+
+
+def _prompt(seed, n):
+    return [int(x) for x in np.random.default_rng(seed).integers(0, 32000, n)]
+
+
+def test_prefix_cache_shares_the_full_blocks_of_a_common_prompt(pa):
+    """Two requests with one 40-token prompt at block size 16: the second
+    shares the two full blocks (32 cached tokens) and gets its own partial
+    block; a third prompt sharing only the first 16 tokens shares one block."""
+    bm = pa.BlockManager(32, 16)
+    p = _prompt(1, 40)
+    assert bm.add_sequence_with_prefix(0, p) == 0
+    assert bm.add_sequence_with_prefix(1, p) == 32
+    t0, t1 = bm.block_table(0), bm.block_table(1)
+    assert t1[:2] == t0[:2] and t1[2] != t0[2]
+    assert [bm.refcount(b) for b in t0] == [2, 2, 1]
+    q = p[:16] + _prompt(2, 20)
+    assert bm.add_sequence_with_prefix(2, q) == 16
+    assert bm.block_table(2)[0] == t0[0] and bm.refcount(t0[0]) == 3
+    assert bm.stats()["cached_blocks"] == 3      # t0[0], t0[1] and seq 2's second block
+    assert bm.seq_len(1) == 40
+
+
+def test_prefix_cache_match_is_exact_and_chained(pa):
+    """A block matches only when its tokens and every token before it match:
+    the same second block after a different first block is not shared, nor is
+    a block that differs in one token."""
+    bm = pa.BlockManager(32, 4)
+    a, b = _prompt(3, 4), _prompt(4, 4)
+    y = _prompt(5, 4)
+    assert bm.add_sequence_with_prefix(0, a + y) == 0
+    assert bm.add_sequence_with_prefix(1, b + y) == 0            # y after b: no match
+    assert bm.add_sequence_with_prefix(2, a + y[:3] + [y[3] + 1]) == 4
+    assert bm.add_sequence_with_prefix(3, a + y + [7]) == 8      # both full blocks, then 1 token
+    assert bm.block_table(3)[:2] == bm.block_table(0)
+
+
+def test_prefix_cache_entries_leave_with_their_blocks(pa):
+    bm = pa.BlockManager(8, 4)
+    p = _prompt(6, 12)
+    bm.add_sequence_with_prefix(0, p)
+    bm.add_sequence_with_prefix(1, p)
+    bm.free_sequence(0)                       # blocks still held by seq 1
+    assert bm.add_sequence_with_prefix(2, p) == 12
+    bm.free_sequence(1)
+    bm.free_sequence(2)
+    assert bm.stats()["cached_blocks"] == 0 and bm.num_free() == 8
+    assert bm.add_sequence_with_prefix(3, p) == 0
+
+
+def test_prefix_cache_all_or_nothing_and_appends(pa):
+    """A request whose uncached blocks do not fit changes nothing; appending
+    after a prompt that ends on a block boundary never writes a shared
+    block (a new block is taken, no copy)."""
+    bm = pa.BlockManager(5, 4)
+    p = _prompt(7, 8)
+    bm.add_sequence_with_prefix(0, p)         # 2 blocks, both cached
+    bm.add_sequence(9, 8)                     # 2 more: 1 free
+    with pytest.raises(pa.PagedAttnError) as e:
+        bm.add_sequence_with_prefix(1, p[:4] + _prompt(8, 8))   # 1 shared + 2 new
+    assert e.value.name == "PA_ERR_OUT_OF_BLOCKS"
+    assert bm.num_free() == 1 and bm.stats()["cached_blocks"] == 2
+    assert bm.add_sequence_with_prefix(1, p) == 8   # all shared, nothing new
+    slot, cow = bm.append_slot(1)
+    assert cow is None and bm.num_free() == 0
+    assert bm.block_table(1)[:2] == bm.block_table(0)
+    assert slot // 4 == bm.block_table(1)[2]
