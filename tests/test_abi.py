@@ -484,3 +484,23 @@ def test_prefix_cache_all_or_nothing_and_appends(pa):
     assert cow is None and bm.num_free() == 0
     assert bm.block_table(1)[:2] == bm.block_table(0)
     assert slot // 4 == bm.block_table(1)[2]
+
+
+def test_c_abi_from_plain_c(pa, tmp_path):
+    """The header compiles as C99 with warnings as errors, and a C program
+    linked against the library sees the declared host-side behaviour."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    exe = tmp_path / "abi_check"
+    lib_dir = os.path.dirname(pa.LIB_PATH)
+    build = subprocess.run(
+        [cc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-I", os.path.join(ROOT, "include"),
+         os.path.join(ROOT, "tests", "c", "abi_check.c"), "-L", lib_dir, "-lpagedattn",
+         "-Wl,-rpath," + lib_dir, "-o", str(exe)], capture_output=True, text=True)
+    assert build.returncode == 0, build.stderr
+    run = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert run.returncode == 0, run.stderr
+    assert "all checks held" in run.stdout
