@@ -465,8 +465,8 @@ pa_status pa_stream_read(const void* buf, int64_t bytes, uint32_t* sink, int32_t
                          pa_stream_t stream);
 
 /* ---------------------------------------------------------------------------
- * Host block manager -- [PA] "The idea: page the KV cache" (allocate a block
- * when the previous one is full, from a free list, from anywhere in memory),
+ * Host block manager -- [PA] "The idea: page the KV cache" (a new block only
+ * once the last one has no free slot, any free block, wherever it lies),
  * "Sharing and copy-on-write" (per-block reference counts; a filled block is
  * not written again) and "How does copy-on-write work for parallel
  * sampling?" (allocate, copy, decrement, write into the copy).
@@ -483,8 +483,9 @@ pa_status pa_bm_create(int32_t num_blocks, int32_t block_size,
 void pa_bm_destroy(pa_block_manager* bm);
 /* A new sequence that already holds num_tokens tokens: ceil(n / bs) blocks. */
 pa_status pa_bm_add_sequence(pa_block_manager* bm, int64_t seq, int64_t num_tokens);
-/* Prefix caching ([PA] "Sharing and copy-on-write": requests with the same
- * system prompt share blocks; full blocks are never written again).  A new
+/* Prefix caching ([PA] "Sharing and copy-on-write": requests that begin with
+ * one system prompt can hold the same blocks; a block with no free slot is
+ * not written to again).  A new
  * sequence whose num_tokens prompt tokens are token_ids (host int32): its
  * leading FULL blocks whose tokens -- and every token before them -- match
  * a block still held in the manager are shared (refcount + 1) and

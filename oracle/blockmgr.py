@@ -6,11 +6,11 @@ A plain restatement of the host-side bookkeeping on the "PagedAttention" page
 * "The idea: page the KV cache" (the OS analogy table and the five-request
   figure): a sequence gets a new physical block from the free list only when
   its previous block is full; blocks come from anywhere.
-* "Sharing and copy-on-write": two sequences may point at the same physical
-  block; every block keeps a reference count; a block that has filled up is
-  not written again, so only a shared, partially filled last block is copied.
-* "How does copy-on-write work for parallel sampling?": all samples' tables
-  point at the prompt's blocks with refcount = number of users; a sample that
+* "Sharing and copy-on-write": one physical block may appear in several
+  tables; every block counts its holders; a block that has filled up is not
+  written again, so only a shared, partially filled last block is copied.
+* "How does copy-on-write work for parallel sampling?": the samples' tables
+  name the prompt's blocks, each counting its users; a sample that
   must append into a shared partial block takes a new block, has the tokens
   already there copied into it, drops its count on the old block and writes
   into the copy.

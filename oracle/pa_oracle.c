@@ -10,10 +10,11 @@
  * function restates one step as the pages describe it:
  *
  *   orc_slot_mapping      "PagedAttention" (shubhamtatvamasi), "How attention
- *                         reads paged memory" + the block-size-4 figure: a
- *                         block table maps logical block i to a physical
- *                         block id; token p of a sequence lives in logical
- *                         block p / block_size at offset p % block_size.
+ *                         reads paged memory" + the block-size-4 figure:
+ *                         entry i of a block table names the physical block
+ *                         that holds the sequence's logical block i; token p
+ *                         sits in logical block p / block_size at offset
+ *                         p % block_size.
  *   orc_reshape_and_cache "How PagedAttention Works in vLLM to Maximize
  *                         Memory Efficiency", "write_to_paged_cache: Direct
  *                         In-Place Updates" and "Code Example": new K/V rows

@@ -2,21 +2,23 @@
 // kernels consume: block tables, slot mappings and copy-on-write pairs.
 //
 // Rules from "PagedAttention" (shubhamtatvamasi.com):
-//  - "The idea: page the KV cache": a sequence gets a new physical block only
-//    when its previous block is full (the OS analogy: a page is allocated when
-//    first used), from a free list, from anywhere in memory;
-//  - "Sharing and copy-on-write": tables may point at the same physical block;
-//    each block keeps a reference count; a filled block is not written again;
-//  - "How does copy-on-write work for parallel sampling?": a sequence that must
-//    append into a shared, partially filled block allocates a new block, has
-//    the old contents copied into it, decrements the old block's count and
-//    writes into the copy.
+//  - "The idea: page the KV cache": a sequence takes a new physical block only
+//    once its last one has no free slot (as an OS maps a page on first use),
+//    and any free block will do, wherever it lies;
+//  - "Sharing and copy-on-write": several tables may name one physical
+//    block, which counts its holders; a block with no free slot left is
+//    never written to again;
+//  - "How does copy-on-write work for parallel sampling?": before a sequence
+//    adds a token to a partially filled block that others also hold, it takes
+//    a fresh block, gets the tokens already there duplicated into it, gives
+//    up its hold on the old block and continues in the fresh one.
 // The copy itself is the device's job (pa_copy_blocks); this manager returns
 // the (src, dst) pair.
 //
-// Prefix caching ("Sharing and copy-on-write": requests with the same system
-// prompt share blocks; full blocks are never written again, so they can be
-// shared for as long as they live): a full block added with its token ids is
+// Prefix caching ("Sharing and copy-on-write": requests that begin with one
+// system prompt can hold the same blocks, and since a block with no free slot
+// is not written to again, holding it together is safe while it lives): a
+// full block added with its token ids is
 // entered in an index under (the physical block before it, its tokens); a
 // later request whose prompt starts with the same tokens finds its leading
 // full blocks there and shares them.  The match is exact (the tokens are

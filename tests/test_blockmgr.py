@@ -1,7 +1,7 @@
 """Host block manager: the reference (oracle) manager against the pages'
-rules, CPU only.  ("PagedAttention": allocate a block when the previous one is
-full; refcounts; copy-on-write of a shared partial block; full blocks are
-never copied; at most one copy per sequence.)"""
+rules, CPU only.  ("PagedAttention": a new block only once the last one is
+out of slots; refcounts; copy-on-write of a shared partial block; full
+blocks are never copied; at most one copy per sequence.)"""
 import pytest
 
 from oracle.blockmgr import OutOfBlocks, RefBlockManager
