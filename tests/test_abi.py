@@ -504,3 +504,19 @@ def test_c_abi_from_plain_c(pa, tmp_path):
     run = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
     assert run.returncode == 0, run.stderr
     assert "all checks held" in run.stdout
+
+
+def test_import_fails_loudly_without_the_library(tmp_path):
+    """The binding has no fallback: a copy of the package without its
+    library refuses to import, naming the missing file."""
+    import shutil
+    import subprocess
+    import sys
+    pkg = tmp_path / "paged_kv_cache_343_b200"
+    pkg.mkdir()
+    shutil.copy(os.path.join(ROOT, "paged_kv_cache_343_b200", "__init__.py"), pkg / "__init__.py")
+    run = subprocess.run([sys.executable, "-c", "import paged_kv_cache_343_b200"],
+                         cwd=tmp_path, capture_output=True, text=True, timeout=300,
+                         env=dict(os.environ, PYTHONPATH=str(tmp_path)))
+    assert run.returncode != 0
+    assert "libpagedattn.so is missing" in run.stderr
