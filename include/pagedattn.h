@@ -574,6 +574,14 @@ typedef struct pa_bm_stats_t {
   int64_t cached_blocks;     /* full blocks in the prefix cache */
 } pa_bm_stats_t;
 pa_status pa_bm_stats(const pa_block_manager* bm, pa_bm_stats_t* out);
+/* A batch order for pa_decode_attention_shared_prefix: sequences holding
+ * the same leading blocks become neighbours (tables compared as words of
+ * block ids; ties keep the given order).  order (host int32, n entries)
+ * gets, for each position of the new order, the index into seqs.  The
+ * caller permutes its query rows, tables and lengths accordingly.
+ * PA_ERR_NOT_FOUND for an unknown sequence. */
+pa_status pa_bm_order_by_prefix(const pa_block_manager* bm, const int64_t* seqs, int32_t n,
+                                int32_t* order);
 /* Reference count of a physical block (-1 if out of range). */
 int32_t pa_bm_refcount(const pa_block_manager* bm, int32_t block);
 int32_t pa_bm_num_free(const pa_block_manager* bm);

@@ -184,6 +184,8 @@ def _load() -> ctypes.CDLL:
                                         ctypes.POINTER(i32), ctypes.POINTER(i32)]
     lib.pa_bm_blocks_needed.restype = ctypes.c_int
     lib.pa_bm_blocks_needed.argtypes = [p, ctypes.POINTER(i64), i32, p, ctypes.POINTER(i64)]
+    lib.pa_bm_order_by_prefix.restype = ctypes.c_int
+    lib.pa_bm_order_by_prefix.argtypes = [p, ctypes.POINTER(i64), i32, ctypes.POINTER(i32)]
     lib.pa_bm_fill_tables.restype = ctypes.c_int
     lib.pa_bm_fill_tables.argtypes = [p, ctypes.POINTER(i64), i32, p, i32, p]
     lib.pa_bm_stats.restype = ctypes.c_int
@@ -621,6 +623,16 @@ class BlockManager:
         out = (ctypes.c_int32 * max(n, 1))()
         _check(lib.pa_bm_shared_blocks(self._h, ids, n, out), "pa_bm_shared_blocks")
         return torch.tensor(list(out)[:n], dtype=torch.int32)
+
+    def order_by_prefix(self, seqs: Sequence[int]) -> list:
+        """The batch reordered so that sequences holding the same leading
+        blocks are neighbours (for decode_attention_shared_prefix): a list of
+        indices into seqs."""
+        n = len(seqs)
+        ids = (ctypes.c_int64 * max(n, 1))(*[int(x) for x in seqs])
+        out = (ctypes.c_int32 * max(n, 1))()
+        _check(lib.pa_bm_order_by_prefix(self._h, ids, n, out), "pa_bm_order_by_prefix")
+        return [int(out[i]) for i in range(n)]
 
     def tables(self, seqs: Sequence[int], width: int) -> torch.Tensor:
         """int32 [len(seqs), width] host tensor of block tables, padded with -1."""

@@ -298,6 +298,32 @@ extern "C" pa_status pa_bm_shared_blocks(const pa_block_manager* bm, const int64
   return PA_OK;
 }
 
+// A batch order that puts sequences holding the same leading blocks next to
+// each other (the samples of one prompt, requests of one cached system
+// prompt), so that pa_decode_attention_shared_prefix finds them in its
+// windows: the sequences sorted by their block tables read as words (ties
+// keep the given order).  order[i] = the index into seqs of the i-th
+// sequence of the new order.
+extern "C" pa_status pa_bm_order_by_prefix(const pa_block_manager* bm, const int64_t* seqs,
+                                           int32_t n, int32_t* order) {
+  if (bm == nullptr || n < 0 || (n > 0 && (seqs == nullptr || order == nullptr)))
+    return PA_ERR_INVALID_ARG;
+  std::vector<const std::vector<int32_t>*> tabs(static_cast<size_t>(n));
+  for (int32_t i = 0; i < n; ++i) {
+    auto it = bm->seqs.find(seqs[i]);
+    if (it == bm->seqs.end()) return PA_ERR_NOT_FOUND;
+    tabs[static_cast<size_t>(i)] = &it->second.table;
+  }
+  std::vector<int32_t> idx(static_cast<size_t>(n));
+  for (int32_t i = 0; i < n; ++i) idx[static_cast<size_t>(i)] = i;
+  std::stable_sort(idx.begin(), idx.end(), [&](int32_t a, int32_t b) {
+    return std::lexicographical_compare(tabs[a]->begin(), tabs[a]->end(), tabs[b]->begin(),
+                                        tabs[b]->end());
+  });
+  std::copy(idx.begin(), idx.end(), order);
+  return PA_OK;
+}
+
 extern "C" int32_t pa_bm_refcount(const pa_block_manager* bm, int32_t block) {
   if (bm == nullptr || block < 0 || block >= bm->num_blocks) return -1;
   return bm->refcount[block];

@@ -520,3 +520,36 @@ def test_import_fails_loudly_without_the_library(tmp_path):
                          env=dict(os.environ, PYTHONPATH=str(tmp_path)))
     assert run.returncode != 0
     assert "libpagedattn.so is missing" in run.stderr
+
+
+def test_order_by_prefix_groups_the_samples_of_a_prompt(pa):
+    """Samples of three prompts listed in a shuffled order: after
+    pa_bm_order_by_prefix each prompt's samples are neighbours, so the
+    shared-blocks counts of the reordered batch show the sharing."""
+    bm = pa.BlockManager(256, 4, np.random.default_rng(0).permutation(256).astype(np.int32))
+    sid = 0
+    owner = {}
+    for prompt, length in enumerate((22, 9, 30)):
+        bm.add_sequence(sid, length)
+        owner[sid] = prompt
+        for k in range(1, 4):
+            bm.fork(sid, sid + k)
+            owner[sid + k] = prompt
+        sid += 4
+    batch = [int(x) for x in np.random.default_rng(1).permutation(sid)]
+    order = bm.order_by_prefix(batch)
+    assert sorted(order) == list(range(sid))
+    seqs = [batch[i] for i in order]
+    groups = [owner[s] for s in seqs]
+    for g0 in range(0, sid, 4):           # each run of four is one prompt's samples
+        assert len(set(groups[g0:g0 + 4])) == 1
+        run = seqs[g0:g0 + 4]
+        shared = bm.shared_blocks(run).tolist()
+        full = -(-bm.seq_len(run[0]) // 4)
+        assert shared == [full] * 3 + [0]
+    # ties keep the given order
+    assert [s for s in seqs if owner[s] == owner[seqs[0]]] == \
+        [s for s in batch if owner[s] == owner[seqs[0]]]
+    with pytest.raises(pa.PagedAttnError) as e:
+        bm.order_by_prefix([0, 999])
+    assert e.value.name == "PA_ERR_NOT_FOUND"
