@@ -380,6 +380,8 @@ def run_ours(args, rank, world, local_rank):
     flag = torch.zeros(1, dtype=torch.int32, device=device)
     scale = W.scale_of(spec)
     stream = torch.cuda.current_stream(device)
+    # one query token per sequence, no packs: the host-planned decode applies
+    plannable = not shared and not multi
     launches_per_step = 1 + 3 + (1 if cow is not None else 0)
 
     def step():
@@ -457,70 +459,108 @@ def run_ours(args, rank, world, local_rank):
         torch.distributed.barrier()
     elapsed_ms = t_start.elapsed_time(t_end)
     # The attention call alone, for the roofline: its average duration over
-    # att_steps calls launched back to back on its stream between two events
+    # att_calls calls launched back to back on its stream between two events
     # (an event between the calls of one chain would break the programmatic
-    # dependent launch that overlaps them).
-    att_steps = min(args.steps, 500)
-    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    torch.cuda.synchronize()
-    a0.record(stream)
-    for _ in range(att_steps):
-        attention()
-    a1.record(stream)
-    torch.cuda.synchronize()
+    # dependent launch that overlaps them), whatever --steps is.
+    att_calls = args.att_calls
+
+    def chained(fn):
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        a0.record(stream)
+        for _ in range(att_calls):
+            fn()
+        a1.record(stream)
+        torch.cuda.synchronize()
+        return a0.elapsed_time(a1) / att_calls
+
+    att_avg_ms = chained(attention)
     clock_info = clocks.summary(wall0, wall1)
     clocks.stop()
-    att_avg_ms = a0.elapsed_time(a1) / att_steps
+    # the same decode with its split plan made on the host (pa_decode_plan,
+    # copied to the device once): main kernel + combine, no plan kernel
+    planned = None
+    if plannable:
+        hplan, _ = pa.decode_plan(torch.from_numpy(np.ascontiguousarray(wl["lens"])), Hq,
+                                  spec.num_kv_heads, D, spec.block_size, max_len, psize,
+                                  "fp8_e4m3" if spec.fp8 else "auto")
+        dplan = hplan.to(device)
+
+        def planned():
+            pa.decode_attention_planned(out, q, k_cache, v_cache, tables, lens, max_len, scale,
+                                        dplan, psize, ws, k_scale=k_scale, v_scale=v_scale,
+                                        error_flag=flag)
+        planned_avg_ms = chained(planned)
     read_bytes = unique_kv_bytes(spec, wl) if spec.len_dist == "shared_prefix" else bytes_step
     latency = latency_distribution(attention, read_bytes, device, stream)
+    latency_planned = (latency_distribution(planned, read_bytes, device, stream)
+                       if planned is not None else None)
     ceiling = read_ceiling(device, stream)
     if int(flag.item()) != 0:
         raise RuntimeError("device error flag %#x in the timed region" % int(flag.item()))
 
-    # ---------------- end to end: pinned host buffers through the public API
+    # ---------------- end to end: pinned host buffers through the C entry point
+    # pa_decode_step (plan on the host, one H2D copy, the kernels, one D2H copy)
     e2e_steps = max(1, min(args.steps, args.e2e_steps))
-    runner = pa.PagedDecodeStep(k_cache, v_cache, B, Hq, wl["tables"].shape[1], max_len, scale,
-                                psize, query_dtype=td, k_scale=k_scale, v_scale=v_scale,
-                                slots=2)
-
-    def fill(dst, a, dtype=None):
-        t = torch.from_numpy(np.ascontiguousarray(a))
-        dst.copy_(t.view(torch.int16).view(dtype) if dtype is not None else t)
-
-    e2e_ok = wl["slots"].shape[0] == B and cow is None and not multi
+    e2e_ok = plannable and wl["slots"].shape[0] == B
     e2e = None
     if e2e_ok:
+        ncow = 0 if cow is None else int(cow.shape[0])
+        runner = pa.DecodeStep(k_cache, v_cache, B, Hq, wl["tables"].shape[1], max_len, scale,
+                               psize, query_dtype=td, k_scale=k_scale, v_scale=v_scale,
+                               max_cow=ncow, slots=2)
+
+        def fill(dst, a, dtype=None):
+            t = torch.from_numpy(np.ascontiguousarray(a))
+            dst.copy_(t.view(torch.int16).view(dtype) if dtype is not None else t)
+
         for sl in range(2):
-            h = runner.slot_host(sl)
+            h = runner.host(sl)
             fill(h["q"], case.q, td)
             fill(h["new_k"], wl["new_k"], td)
             fill(h["new_v"], wl["new_v"], td)
             fill(h["slots"], wl["slots"])
             fill(h["tables"], wl["tables"])
             fill(h["lens"], wl["lens"])
-        for i in range(4):  # warm-up; captures each slot's kernels in a graph
-            runner.submit(i % 2)
+            if ncow:
+                fill(h["cow"], wl["cow"])
+        for i in range(4):  # warm-up
+            runner.submit(i % 2, ncow, error_flag=flag)
             runner.wait(i % 2)
         if world > 1:
             torch.distributed.barrier()
-        # every step copies its inputs in and its output out; step i + 1 is
-        # submitted before the host waits for step i, as a serving loop does
+        # serving loop: step i + 1 (its own slot and stream) is submitted
+        # before the host waits for step i, so one step's copies overlap
+        # another's kernels; every step copies its inputs in and its output out
         t0 = time.perf_counter()
-        runner.submit(0)
+        runner.submit(0, ncow, error_flag=flag)
         for i in range(1, e2e_steps):
-            runner.submit(i % 2)
+            runner.submit(i % 2, ncow, error_flag=flag)
             runner.wait((i - 1) % 2)
         runner.wait((e2e_steps - 1) % 2)
-        e2e_s = time.perf_counter() - t0
-        e2e_s = max_over_ranks(e2e_s, world, device)
+        e2e_s = max_over_ranks(time.perf_counter() - t0, world, device)
+        # the same step alone through the single call pa_decode_step (its three
+        # parts on one stream), each waited for: no overlap between steps
+        t0 = time.perf_counter()
+        for i in range(e2e_steps):
+            runner(ncow, error_flag=flag)
+        serial_s = max_over_ranks(time.perf_counter() - t0, world, device)
         e2e = {"value": round(bytes_step * e2e_steps * world / e2e_s / 1e9, 2), "unit": "GB/s",
                "h2d_bytes_per_step": runner.h2d_bytes(), "d2h_bytes_per_step": runner.d2h_bytes(),
                "steps": e2e_steps, "ms_per_step": round(e2e_s * 1e3 / e2e_steps, 4),
-               "how": "PagedDecodeStep with two slots: per step one pinned H2D copy of "
-                      "the step's inputs, reshape_and_cache + decode_attention (a CUDA "
-                      "graph per slot), one D2H copy of the output into pinned memory; "
-                      "step i + 1 is submitted before the host waits for step i's output, "
-                      "so one step's copies overlap another's kernels"}
+               "serial": {"value": round(bytes_step * e2e_steps * world / serial_s / 1e9, 2),
+                          "ms_per_step": round(serial_s * 1e3 / e2e_steps, 4),
+                          "how": "pa_decode_step (upload, run, download on one stream), each "
+                                 "step waited for before the next is issued"},
+               "how": "C ABI from pinned host buffers, two slots: per step "
+                      "pa_decode_step_upload (split plan computed on the host, one H2D copy of "
+                      "the staging buffer) on a copy stream, pa_decode_step_run "
+                      "(reshape_and_cache + the decode's main kernel + combine, no plan kernel) "
+                      "on the compute stream in submission order, pa_decode_step_download (one "
+                      "D2H copy of the output) on a second copy stream; step i + 1 is submitted "
+                      "before the host waits for step i (wall clock, max over ranks)"}
+        if int(flag.item()) != 0:
+            raise RuntimeError("device error flag %#x in the end-to-end steps" % int(flag.item()))
 
     elapsed_ms = max_over_ranks(elapsed_ms, world, device)
     att_avg_ms = max_over_ranks(att_avg_ms, world, device)
@@ -542,10 +582,7 @@ def run_ours(args, rank, world, local_rank):
         "dtype": spec.dtype + ("/e4m3 cache" if spec.fp8 else ""),
         "data": "synthetic (seeded N(0,1) values; lengths, placement and sharing per workload)",
         "config": {
-            "workload": "%s: B %d, Hq %d / Hkv %d, D %d, block %d, %s%s, lengths %s" % (
-                spec.name, spec.num_seqs, spec.num_q_heads, spec.num_kv_heads, spec.head_dim,
-                spec.block_size, spec.dtype, ", fp8 E4M3 cache" if spec.fp8 else "",
-                describe_lengths(spec)),
+            "workload": describe_workload(spec),
             "global_batch": spec.num_seqs * world, "kv_bytes_per_step": bytes_step,
             "sum_seq_len": int(wl["lens"].sum()), "partition_size": psize,
             "num_blocks": case.num_blocks, "parallelism": "dp%d (independent batches)" % world,
@@ -562,7 +599,11 @@ def run_ours(args, rank, world, local_rank):
                                 "pa_decode_attention_multi_query" if multi else
                                 "pa_decode_attention") + " (plan + main + combine launches)",
                      "bytes_per_launch": read_bytes,
-                     "peak_kind": peak_kind + " (MEASURED_PEAKS hbm_gbs, copy read+write)"},
+                     "peak_kind": ("measured (MEASURED_PEAKS.json hbm_gbs, copy read+write)"
+                                   if peak_kind == "measured" else
+                                   "fallback (6.65 TB/s copy, an earlier measurement on this "
+                                   "pool; MEASURED_PEAKS.json absent)")},
+        "attention_calls_averaged": att_calls,
         "attention_latency": latency,
         "read_ceiling": dict(ceiling, frac=round(achieved / ceiling["gbs"], 4)),
         "kv_memory": dict(kv_memory(spec, wl), block_manager={
@@ -572,6 +613,15 @@ def run_ours(args, rank, world, local_rank):
         "e2e": e2e,
         "gpu_launches": launches_per_step * args.steps,
     }
+    if planned is not None:
+        planned_avg_ms = max_over_ranks(planned_avg_ms, world, device)
+        line["attention_planned"] = {
+            "gbs": round(read_bytes / (planned_avg_ms / 1e3) / 1e9, 2),
+            "us": round(planned_avg_ms * 1e3, 2), "calls": att_calls,
+            "frac_of_peak": round(read_bytes / (planned_avg_ms / 1e3) / 1e9 / peak, 4),
+            "how": "pa_decode_attention_planned (plan from pa_decode_plan on the host, copied "
+                   "once): main kernel + combine, back to back between two events"}
+        line["attention_latency_planned"] = latency_planned
     if spec.len_dist == "shared_prefix":
         ub = unique_kv_bytes(spec, wl)
         line["config"]["unique_kv_bytes_per_step"] = ub
@@ -584,6 +634,13 @@ def run_ours(args, rank, world, local_rank):
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(spec, wl, budget_s=args.cpu_budget)
     return line
+
+
+def describe_workload(spec):
+    return "%s: B %d, Hq %d / Hkv %d, D %d, block %d, %s%s, lengths %s" % (
+        spec.name, spec.num_seqs, spec.num_q_heads, spec.num_kv_heads, spec.head_dim,
+        spec.block_size, spec.dtype, ", fp8 E4M3 cache" if spec.fp8 else "",
+        describe_lengths(spec))
 
 
 def describe_lengths(spec):
@@ -669,10 +726,18 @@ def cpu_baseline(spec, wl, budget_s=20.0):
         if total_t + t > budget_s or n >= 40:
             break
     return {"value": round(total_b / total_t / 1e9, 4), "unit": "GB/s", "cores": threads,
-            "kind": "oracle",
-            "sample": "%d full step(s) of the %s batch (%d sequences, %d tokens each step): "
-                      "reshape_and_cache + fp64 decode, %.1f s" % (
-                          n, spec.name, B, int(wl["lens"].sum()), total_t)}
+            "kind": "oracle", "sample": describe_oracle_sample(spec, wl, n, B, total_t)}
+
+
+def describe_oracle_sample(spec, wl, steps, per_step, seconds):
+    """One wording for both oracle legs (cpu_baseline and --impl reference)."""
+    B = spec.num_seqs
+    what = ("full step(s) of the %s batch (%d sequences, %d tokens each step)" % (
+        spec.name, B, int(wl["lens"].sum())) if per_step == B else
+        "step(s) of %d of the %s batch's %d sequences (seeded random sample)" % (
+            per_step, spec.name, B))
+    return "%d %s: reshape_and_cache + fp64 decode on all host cores, %.1f s timed" % (
+        steps, what, seconds)
 
 
 def run_reference(args, rank, world):
@@ -694,32 +759,39 @@ def run_reference(args, rank, world):
     wl = dict(case=case, lens=lens, tables=tables, slots=np.array(slots, np.int32),
               new_k=new_k, new_v=new_v)
     _add_queries(spec, wl)
-    # size each step so warm-up + timed steps take about args.ref_budget seconds
+    # Each step is the whole batch, as in the cpu_baseline leg, when warm-up +
+    # timed steps fit in args.ref_budget seconds; otherwise a seeded sample of
+    # the batch's sequences sized to fit.
     B = spec.num_seqs
-    t1, _ = _oracle_sample(spec, wl, np.arange(1))
-    per_seq = max(t1, 1e-4)
+    t_full, _ = _oracle_sample(spec, wl, np.arange(B))
     n_steps = args.warmup + args.steps
-    per_step = max(1, min(B, int(args.ref_budget / n_steps / per_seq)))
+    per_step = B if t_full * n_steps <= args.ref_budget else max(
+        1, min(B, int(args.ref_budget / n_steps / max(t_full / B, 1e-4))))
     rng = np.random.default_rng(0)
+
+    def pick():
+        return np.arange(B) if per_step == B else np.sort(rng.choice(B, per_step, replace=False))
+
     for _ in range(args.warmup):
-        _oracle_sample(spec, wl, np.sort(rng.choice(B, per_step, replace=False)))
+        _oracle_sample(spec, wl, pick())
     tt, tb = 0.0, 0
     for _ in range(args.steps):
-        t, b = _oracle_sample(spec, wl, np.sort(rng.choice(B, per_step, replace=False)))
+        t, b = _oracle_sample(spec, wl, pick())
         tt += t
         tb += b
     value = tb / tt / 1e9
     threads = len(os.sched_getaffinity(0))
-    sample = "%d of %d sequences per step (random, seeded), reshape_and_cache + fp64 decode" % (
-        per_step, B)
+    sample = describe_oracle_sample(spec, wl, args.steps, per_step, tt)
     return {
         "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(tt * 1e3 / args.steps, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded N(0,1) values; lengths and placement per workload)",
-        "config": {"workload": spec.name, "global_batch": spec.num_seqs,
-                   "parallelism": "host cores"},
+        "config": {"workload": describe_workload(spec), "global_batch": spec.num_seqs,
+                   "kv_bytes_per_step": kv_bytes(spec, wl["lens"]),
+                   "sum_seq_len": int(wl["lens"].sum()), "partition_size": spec.partition_size,
+                   "parallelism": "host cores (the fp64 oracle)"},
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": threads,
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
@@ -735,6 +807,8 @@ def main(argv=None):
     ap.add_argument("--workload", default="llama8b", choices=sorted(W.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=200)
+    ap.add_argument("--att-calls", type=int, default=500,
+                    help="back-to-back attention calls averaged for the roofline")
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--ref-budget", type=float, default=90.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")

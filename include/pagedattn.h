@@ -93,6 +93,8 @@ typedef struct pa_cache_strides {
 #define PA_DEVERR_TIMEOUT 0x8     /* a bounded pipeline wait gave up           */
 #define PA_DEVERR_BAD_SHARE 0x10  /* shared_blocks promised a block the tables
                                      of a pack's members do not share          */
+#define PA_DEVERR_BAD_PLAN 0x20   /* a host-computed plan was made for another
+                                     shape (nothing was computed)              */
 
 /* Human-readable name of a status code (static storage). */
 const char* pa_status_string(pa_status status);
@@ -231,7 +233,9 @@ pa_status pa_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads,
  *                  block_size).  Partials are merged by the combine pass.
  *  workspace       device scratch of at least pa_decode_workspace_bytes(),
  *                  256-byte aligned; contents need no initialisation.
- * Built shapes: head_dim 64 or 128; block_size 4..128 (power of two);
+ * Built shapes: head_dim 64 or 128; block_size 4..256 (power of two; a
+ * block longer than 16 tokens is read as several 16-token tiles, one table
+ * lookup per block);
  * num_q_heads / num_kv_heads <= 8.  Other shapes: PA_ERR_UNSUPPORTED.
  * Errors: PA_ERR_INVALID_ARG for null pointers, num_q_heads % num_kv_heads,
  * block_table_stride < ceil(max_seq_len / block_size), a partition_size that
@@ -411,6 +415,174 @@ pa_status pa_decode_attention_shared_prefix(void* out, pa_dtype out_dtype, const
                                             int32_t* device_error_flag, pa_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * Split plans computed on the host.  [PA] "How attention reads paged memory"
+ * gives the kernel each sequence's current length; pa_decode_attention reads
+ * the lengths on the device, in a one-CTA plan kernel that lays the batch's
+ * 16-token tiles end to end and cuts them into the persistent CTAs' equal
+ * shares and the split-KV segments.  A serving step knows its lengths on the
+ * host, so the same plan can be made there and copied to the device with the
+ * step's other inputs; the decode then starts with its main kernel.
+ *
+ * pa_decode_plan_bytes -- bytes of a plan for this shape on the CURRENT
+ *   device (plain decode: one query token per sequence; kv_cache_dtype
+ *   PA_KV_AUTO for 16-bit pools or PA_KV_FP8_E4M3).  num_seqs >= 1.
+ * pa_decode_plan -- writes the plan for the HOST lengths seq_lens[num_seqs]
+ *   (each in [0, max_seq_len], else PA_ERR_INVALID_ARG) into the HOST buffer
+ *   `plan` (plan_bytes >= pa_decode_plan_bytes, 4-byte aligned).  The plan is
+ *   a self-describing block of int32 words (a header naming the shape, then
+ *   the tile and segment prefix sums and each CTA's first sequence and
+ *   segment); copy it as it is to 256-byte aligned device memory.
+ *   *needs_combine (optional) gets 1 if some sequence is split into partials.
+ * pa_decode_attention_planned -- pa_decode_attention (or, with
+ *   PA_KV_FP8_E4M3, pa_decode_attention_fp8) with the plan read from the
+ *   DEVICE buffer `plan` instead of computed by a kernel: two launches (main,
+ *   combine) instead of three.  The device seq_lens must be the lengths the
+ *   plan was made from: a sequence whose length disagrees with the plan's tile
+ *   count is flagged PA_DEVERR_BAD_SEQLEN and its tiles are left out (no table
+ *   entry or pool row of it is read); a plan made for another number of
+ *   sequences, launch shape or partition size is flagged PA_DEVERR_BAD_PLAN
+ *   and nothing is computed.  Workspace: pa_decode_workspace_bytes.  Other
+ *   arguments and errors as in pa_decode_attention_strided (without strides).
+ * pa_split_plan -- the plan's arithmetic alone, for a given CTA count and
+ *   partition_size (0 or a multiple of 16), on host arrays: tiles[num_seqs+1]
+ *   (tile prefix sums), seg_base[num_seqs+1] (segment prefix sums),
+ *   start_seq[num_ctas] and first_k[num_ctas] (the sequence holding CTA c's
+ *   first tile and the index of the segment starting there), *num_segments and
+ *   *needs_combine.  Needs no GPU.
+ * ------------------------------------------------------------------------- */
+pa_status pa_decode_plan_bytes(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
+                               int32_t head_dim, int32_t block_size, int32_t max_seq_len,
+                               int32_t partition_size, pa_kv_cache_dtype kv_cache_dtype,
+                               size_t* bytes);
+pa_status pa_decode_plan(const int32_t* seq_lens, int32_t num_seqs, int32_t num_q_heads,
+                         int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                         int32_t max_seq_len, int32_t partition_size,
+                         pa_kv_cache_dtype kv_cache_dtype, void* plan, size_t plan_bytes,
+                         int32_t* needs_combine);
+pa_status pa_decode_attention_planned(void* out, pa_dtype out_dtype, const void* query,
+                                      pa_dtype query_dtype, const void* key_cache,
+                                      const void* value_cache, pa_kv_cache_dtype kv_cache_dtype,
+                                      const float* k_scale, const float* v_scale,
+                                      const int32_t* block_tables, int32_t block_table_stride,
+                                      const int32_t* seq_lens, int32_t num_seqs,
+                                      int32_t max_seq_len, int32_t num_q_heads,
+                                      int32_t num_kv_heads, int32_t head_dim, int32_t num_blocks,
+                                      int32_t block_size, float scale, int32_t partition_size,
+                                      const void* plan, void* workspace, size_t workspace_bytes,
+                                      int32_t* device_error_flag, pa_stream_t stream);
+pa_status pa_split_plan(const int32_t* seq_lens, int32_t num_seqs, int32_t max_seq_len,
+                        int32_t partition_size, int32_t num_ctas, int32_t* tiles,
+                        int32_t* seg_base, int32_t* start_seq, int32_t* first_k,
+                        int32_t* num_segments, int32_t* needs_combine);
+
+/* ---------------------------------------------------------------------------
+ * pa_decode_step -- one decode step of a batch, driven from host memory:
+ * [vLLM] "write_to_paged_cache" (the new token's K and V go into their slots)
+ * followed by [PA] "How attention reads paged memory" (each sequence's query
+ * attends its grown cache), with the copy-on-write copies of [PA] "How does
+ * copy-on-write work for parallel sampling?" first when the step has any.
+ *
+ * The caller writes the step's inputs into a HOST staging buffer laid out by
+ * pa_decode_step_layout (pinned memory, so the copy is asynchronous):
+ *   query          [num_seqs, num_q_heads, head_dim]  dtype
+ *   new_k, new_v   [num_seqs, num_kv_heads, head_dim] dtype (each sequence's
+ *                  new token)
+ *   slot_mapping   int32 [num_seqs]  (pa_bm_append_slots)
+ *   block_tables   int32 [num_seqs, table_width]
+ *   seq_lens       int32 [num_seqs]  lengths after the new token, each in
+ *                  [0, max_seq_len]
+ *   cow_pairs      int32 [max_cow, 2]; the first num_cow are copied first
+ * The call then, on `stream`, in order:
+ *   1. computes the split plan on the host from seq_lens and writes it into
+ *      the staging buffer's plan section;
+ *   2. copies the whole staging buffer to the start of device_scratch in ONE
+ *      host-to-device copy;
+ *   3. pa_copy_blocks of the num_cow pairs (if any), pa_reshape_and_cache of
+ *      the new rows, the decode's main kernel and (when some sequence is
+ *      split) its combine -- no plan kernel;
+ *   4. copies the output [num_seqs, num_q_heads, head_dim] out_dtype into
+ *      host_out in ONE device-to-host copy.
+ * It returns once everything is enqueued; host_out is valid, and the staging
+ * buffer may be rewritten, after the stream has reached that point (e.g.
+ * cudaStreamSynchronize or an event recorded after the call).  Steps in
+ * flight at once need their own staging buffer, output and device_scratch;
+ * a step whose attention reads rows an earlier step wrote must run after it
+ * (the same stream orders them).
+ *
+ *  shape           host pointer; the batch shape (pa_step_shape).
+ *  key_cache, value_cache  the pools (device), [num_blocks, block_size,
+ *                  num_kv_heads, head_dim] of dtype, or uint8 E4M3 codes with
+ *                  kv_cache_dtype PA_KV_FP8_E4M3 (then k_scale / v_scale are
+ *                  device floats, as in pa_reshape_and_cache).
+ *  device_scratch  device, 256-byte aligned, layout.device_bytes or more: the
+ *                  staging copy, the device output and the split-KV partials.
+ * Built shapes as pa_decode_attention (fp8: head_dim 128).  Errors:
+ * PA_ERR_INVALID_ARG for null pointers, a length outside [0, max_seq_len]
+ * (read from the staging buffer), num_cow outside [0, max_cow], a short
+ * scratch or a table_width below ceil(max_seq_len / block_size);
+ * PA_ERR_UNSUPPORTED / PA_ERR_CUDA as in the calls it makes.  Device-side
+ * flags as in those calls.
+ * ------------------------------------------------------------------------- */
+typedef struct pa_step_shape {
+  int32_t num_seqs;        /* sequences, one new token each                 */
+  int32_t num_q_heads;
+  int32_t num_kv_heads;
+  int32_t head_dim;
+  int32_t num_blocks;      /* pool size in blocks                           */
+  int32_t block_size;
+  int32_t table_width;     /* int32 entries per block-table row             */
+  int32_t max_seq_len;     /* bound of every length                         */
+  int32_t partition_size;  /* as in pa_decode_attention                     */
+  int32_t max_cow;         /* room for copy-on-write pairs in one step      */
+  pa_dtype dtype;          /* query and new rows: PA_F16 or PA_BF16         */
+  pa_dtype out_dtype;      /* PA_F16, PA_BF16 or PA_F32                     */
+  pa_kv_cache_dtype kv_cache_dtype;
+} pa_step_shape;
+
+typedef struct pa_step_layout {
+  size_t query, new_k, new_v, slot_mapping, block_tables, seq_lens, cow_pairs;
+                           /* byte offsets of the inputs in the staging buffer */
+  size_t plan;             /* byte offset of the plan the call writes        */
+  size_t host_bytes;       /* size of the staging buffer                     */
+  size_t out_bytes;        /* size of host_out                               */
+  size_t device_bytes;     /* size of device_scratch                         */
+} pa_step_layout;
+
+/* Layout of the staging buffer and sizes for a shape on the CURRENT device. */
+pa_status pa_decode_step_layout(const pa_step_shape* shape, pa_step_layout* layout);
+
+pa_status pa_decode_step(const pa_step_shape* shape, void* host_staging, int32_t num_cow,
+                         void* key_cache, void* value_cache, const float* k_scale,
+                         const float* v_scale, float scale, void* device_scratch,
+                         size_t device_scratch_bytes, void* host_out,
+                         int32_t* device_error_flag, pa_stream_t stream);
+
+/* The three parts of pa_decode_step, for callers that put the copies on
+ * streams of their own so they overlap other steps' kernels (the caller
+ * orders the streams, e.g. with events: upload before run, run before
+ * download; run on one stream for steps that depend on each other):
+ *   pa_decode_step_upload    1. and 2. above: plan on the host, one
+ *                            host-to-device copy of the staging buffer;
+ *   pa_decode_step_run       3.: the kernels, from the staging copy in
+ *                            device_scratch; host_staging is read on the host
+ *                            for the plan's header, which must be the one
+ *                            upload wrote for this shape (else
+ *                            PA_ERR_INVALID_ARG);
+ *   pa_decode_step_download  4.: one device-to-host copy of the output.
+ * Arguments and errors as in pa_decode_step. */
+pa_status pa_decode_step_upload(const pa_step_shape* shape, void* host_staging,
+                                void* device_scratch, size_t device_scratch_bytes,
+                                pa_stream_t stream);
+pa_status pa_decode_step_run(const pa_step_shape* shape, const void* host_staging,
+                             int32_t num_cow, void* key_cache, void* value_cache,
+                             const float* k_scale, const float* v_scale, float scale,
+                             void* device_scratch, size_t device_scratch_bytes,
+                             int32_t* device_error_flag, pa_stream_t stream);
+pa_status pa_decode_step_download(const pa_step_shape* shape, const void* device_scratch,
+                                  size_t device_scratch_bytes, void* host_out,
+                                  pa_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * pa_decode_attention_noalloc -- pa_decode_attention for callers that cannot
  * allocate device memory.  The pages have no counterpart of this entry point;
  * it exists for callers such as plugins whose host framework owns every device
@@ -427,7 +599,9 @@ pa_status pa_decode_attention_shared_prefix(void* out, pa_dtype out_dtype, const
  * routine).
  *  - The first call on each device looks up the array's device address
  *    (cudaGetSymbolAddress) with that device current; make that first call
- *    before any stream capture.
+ *    before any stream capture.  The address is kept with the id of the CUDA
+ *    context it belongs to: after a cudaDeviceReset the next call runs in a
+ *    new context and looks the address up again (again outside any capture).
  *  - All calls on a device share the one array and it keeps the last call's
  *    contents.  Nothing in it needs to start at zero: each call's first
  *    kernel rewrites the per-call bookkeeping before the others read it.
@@ -494,7 +668,12 @@ pa_status pa_bm_add_sequence(pa_block_manager* bm, int64_t seq, int64_t num_toke
  * cache (a partial last block never is).  Rows of tokens cached_tokens ..
  * num_tokens - 1 are the caller's to write (pa_reshape_and_cache) before any
  * attention reads them; the multi-query decode attends the uncached tokens
- * over the shared ones.  Matches compare token ids exactly.  A cache entry
+ * over the shared ones.  A block enters the cache when it is allocated, not
+ * when its rows are written: a hit may name blocks of a request added earlier
+ * in the same step whose rows are still to be written, so the caller writes
+ * every added request's uncached rows before any attention of that step (a
+ * request freed before its rows were written leaves such blocks empty for the
+ * requests that share them).  Matches compare token ids exactly.  A cache entry
  * lives while its block is held; blocks that return to the free list leave
  * the cache.  All or nothing (PA_ERR_OUT_OF_BLOCKS changes nothing);
  * PA_ERR_INVALID_ARG for a known seq id or NULL pointers. */

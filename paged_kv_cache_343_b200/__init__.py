@@ -27,8 +27,13 @@ Entry points (see the header for argument meaning, layout and errors):
   paged cache causally.
 * ``BlockManager``      -- the native host block manager (free list,
   refcounts, copy-on-write planning, shared-prefix counts).
-* ``PagedDecodeStep``   -- one decode step from pinned host buffers: copies in,
-  the two kernels, copy out (the end-to-end call).
+* ``decode_plan`` / ``decode_attention_planned`` -- the split plan made on the
+  host from host lengths, and the decode that reads it instead of running its
+  plan kernel.
+* ``DecodeStep``        -- one decode step from pinned host buffers through the
+  C entry points ``pa_decode_step`` / ``_upload`` / ``_run`` / ``_download``:
+  the plan on the host, one copy in, the kernels, one copy out (the
+  end-to-end call).
 """
 from __future__ import annotations
 
@@ -43,8 +48,10 @@ __all__ = [
     "decode_workspace_bytes", "decode_attention_fp8", "decode_attention_noalloc",
     "decode_attention_shared_prefix", "shared_prefix_workspace_bytes",
     "decode_attention_multi_query", "multi_query_workspace_bytes", "BlockManager",
-    "PagedDecodeStep", "DEVERR_BAD_BLOCK", "DEVERR_BAD_SLOT", "DEVERR_BAD_SEQLEN",
-    "DEVERR_TIMEOUT", "DEVERR_BAD_SHARE", "CacheStrides", "version", "stream_read",
+    "DEVERR_BAD_BLOCK", "DEVERR_BAD_SLOT", "DEVERR_BAD_SEQLEN",
+    "DEVERR_TIMEOUT", "DEVERR_BAD_SHARE", "DEVERR_BAD_PLAN", "CacheStrides", "version",
+    "stream_read", "decode_plan_bytes", "decode_plan", "decode_attention_planned", "split_plan",
+    "DecodeStep", "StepShape", "StepLayout",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpagedattn.so")
@@ -54,6 +61,7 @@ DEVERR_BAD_SLOT = 0x2
 DEVERR_BAD_SEQLEN = 0x4
 DEVERR_TIMEOUT = 0x8
 DEVERR_BAD_SHARE = 0x10
+DEVERR_BAD_PLAN = 0x20
 
 _PA_F16, _PA_BF16, _PA_F32 = 0, 1, 2
 _DTYPE_CODE = {torch.float16: _PA_F16, torch.bfloat16: _PA_BF16, torch.float32: _PA_F32}
@@ -79,6 +87,21 @@ class BmStats(ctypes.Structure):
     _fields_ = [(name, ctypes.c_int64) for name in (
         "num_blocks", "free_blocks", "held_blocks", "logical_blocks", "num_seqs", "tokens",
         "stored_slots", "waste_slots", "max_waste_per_seq", "cached_blocks")]
+
+
+class StepShape(ctypes.Structure):
+    """pa_step_shape: the batch shape of pa_decode_step."""
+    _fields_ = [(n, ctypes.c_int32) for n in (
+        "num_seqs", "num_q_heads", "num_kv_heads", "head_dim", "num_blocks", "block_size",
+        "table_width", "max_seq_len", "partition_size", "max_cow")] + [
+        ("dtype", ctypes.c_int), ("out_dtype", ctypes.c_int), ("kv_cache_dtype", ctypes.c_int)]
+
+
+class StepLayout(ctypes.Structure):
+    """pa_step_layout: where pa_decode_step's inputs sit in its staging buffer."""
+    _fields_ = [(n, ctypes.c_size_t) for n in (
+        "query", "new_k", "new_v", "slot_mapping", "block_tables", "seq_lens", "cow_pairs",
+        "plan", "host_bytes", "out_bytes", "device_bytes")]
 
 
 def _pool_strides(cache: torch.Tensor) -> Optional[CacheStrides]:
@@ -149,6 +172,31 @@ def _load() -> ctypes.CDLL:
     lib.pa_decode_attention_noalloc.argtypes = [p, ctypes.c_int, p, p, p, p, i32, p, i32, i32, i32,
                                                 i32, i32, i32, i32, ctypes.c_float, ctypes.c_int,
                                                 i32, p, p]
+    lib.pa_decode_plan_bytes.restype = ctypes.c_int
+    lib.pa_decode_plan_bytes.argtypes = [i32, i32, i32, i32, i32, i32, i32, ctypes.c_int,
+                                         ctypes.POINTER(sz)]
+    lib.pa_decode_plan.restype = ctypes.c_int
+    lib.pa_decode_plan.argtypes = [p, i32, i32, i32, i32, i32, i32, i32, ctypes.c_int, p, sz,
+                                   ctypes.POINTER(i32)]
+    lib.pa_decode_attention_planned.restype = ctypes.c_int
+    lib.pa_decode_attention_planned.argtypes = [p, ctypes.c_int, p, ctypes.c_int, p, p,
+                                                ctypes.c_int, p, p, p, i32, p, i32, i32, i32, i32,
+                                                i32, i32, i32, ctypes.c_float, i32, p, p, sz, p, p]
+    lib.pa_split_plan.restype = ctypes.c_int
+    lib.pa_split_plan.argtypes = [p, i32, i32, i32, i32, p, p, p, p, ctypes.POINTER(i32),
+                                  ctypes.POINTER(i32)]
+    lib.pa_decode_step_layout.restype = ctypes.c_int
+    lib.pa_decode_step_layout.argtypes = [ctypes.POINTER(StepShape), ctypes.POINTER(StepLayout)]
+    lib.pa_decode_step_upload.restype = ctypes.c_int
+    lib.pa_decode_step_upload.argtypes = [ctypes.POINTER(StepShape), p, p, sz, p]
+    lib.pa_decode_step_run.restype = ctypes.c_int
+    lib.pa_decode_step_run.argtypes = [ctypes.POINTER(StepShape), p, i32, p, p, p, p,
+                                       ctypes.c_float, p, sz, p, p]
+    lib.pa_decode_step_download.restype = ctypes.c_int
+    lib.pa_decode_step_download.argtypes = [ctypes.POINTER(StepShape), p, sz, p, p]
+    lib.pa_decode_step.restype = ctypes.c_int
+    lib.pa_decode_step.argtypes = [ctypes.POINTER(StepShape), p, i32, p, p, p, p, ctypes.c_float,
+                                   p, sz, p, p, p]
     lib.pa_stream_read.restype = ctypes.c_int
     lib.pa_stream_read.argtypes = [p, i64, p, i32, p]
     lib.pa_bm_create.restype = ctypes.c_int
@@ -326,6 +374,32 @@ def alloc_workspace(nbytes: int, device) -> torch.Tensor:
     return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
 
 
+def _decode_args(out: torch.Tensor, query: torch.Tensor, key_cache: torch.Tensor,
+                 value_cache: torch.Tensor, block_tables: torch.Tensor, seq_lens: torch.Tensor,
+                 allow_strided_pools: bool = True) -> Optional[CacheStrides]:
+    """Checks of the 16-bit decode entry points, made before any library call:
+    contiguous query and out of one shape, 16-bit query and pools of one dtype,
+    K and V pools of one shape and strides, int32 tables with contiguous rows,
+    int32 contiguous lengths, a supported out dtype.  Returns the pools'
+    strides (None when contiguous); allow_strided_pools=False refuses strided
+    pools instead."""
+    _need(query.dim() == 3 and query.is_contiguous(), "query must be contiguous [B, Hq, D]")
+    _need(out.shape == query.shape and out.is_contiguous(), "out must be contiguous [B, Hq, D]")
+    _need(key_cache.shape == value_cache.shape and key_cache.stride() == value_cache.stride(),
+          "K and V pools share shape and strides")
+    strides = _pool_strides(key_cache)
+    _need(allow_strided_pools or strides is None, "pools must be contiguous [nb, bs, Hkv, D]")
+    _need(block_tables.dtype == torch.int32 and block_tables.dim() == 2 and
+          block_tables.stride(1) == 1, "block_tables int32 [B, W], rows contiguous")
+    _need(seq_lens.dtype == torch.int32 and seq_lens.is_contiguous(), "seq_lens int32")
+    _need(query.dtype == key_cache.dtype == value_cache.dtype, "query and caches share a dtype")
+    _need(key_cache.shape[3] == query.shape[2], "query and pools must share head_dim")
+    _need(query.dtype in (torch.float16, torch.bfloat16), "query and pools must be float16 or "
+          "bfloat16 (fp8 code pools: decode_attention_fp8)")
+    _dtype_code(out.dtype)
+    return strides
+
+
 def decode_attention(out: torch.Tensor, query: torch.Tensor, key_cache: torch.Tensor,
                      value_cache: torch.Tensor, block_tables: torch.Tensor,
                      seq_lens: torch.Tensor, max_seq_len: int, scale: float,
@@ -335,19 +409,9 @@ def decode_attention(out: torch.Tensor, query: torch.Tensor, key_cache: torch.Te
     """out/query [B, Hq, D]; caches [nb, bs, Hkv, D] (any strided view with head_dim
     contiguous, e.g. the K and V halves of one interleaved tensor); block_tables
     int32 [B, W]; seq_lens int32 [B]."""
-    _need(query.dim() == 3 and query.is_contiguous(), "query must be contiguous [B, Hq, D]")
-    _need(out.shape == query.shape and out.is_contiguous(), "out must be contiguous [B, Hq, D]")
-    _need(key_cache.shape == value_cache.shape and key_cache.stride() == value_cache.stride(),
-          "K and V pools share shape and strides")
-    strides = _pool_strides(key_cache)
-    _need(block_tables.dtype == torch.int32 and block_tables.dim() == 2 and
-          block_tables.stride(1) == 1, "block_tables int32 [B, W], rows contiguous")
-    _need(seq_lens.dtype == torch.int32 and seq_lens.is_contiguous(), "seq_lens int32")
-    _need(query.dtype == key_cache.dtype == value_cache.dtype, "query and caches share a dtype")
+    strides = _decode_args(out, query, key_cache, value_cache, block_tables, seq_lens)
     B, hq, d = query.shape
     nb, bs, hkv, _ = key_cache.shape
-    _need(key_cache.shape[3] == d, "query and pools must share head_dim")
-    _dtype_code(out.dtype), _dtype_code(query.dtype)  # refused before any library call
     if workspace is None:
         workspace = alloc_workspace(decode_workspace_bytes(B, hq, hkv, d, bs, max_seq_len,
                                                            partition_size), query.device)
@@ -504,6 +568,231 @@ def decode_attention_multi_query(out: torch.Tensor, query: torch.Tensor, q_start
     return out
 
 
+_KV_CODE = {"auto": 0, "fp8": 1, "fp8_e4m3": 1}
+
+
+def decode_plan_bytes(num_seqs: int, num_q_heads: int, num_kv_heads: int, head_dim: int,
+                      block_size: int, max_seq_len: int, partition_size: int = 0,
+                      kv_cache_dtype: str = "auto") -> int:
+    out = ctypes.c_size_t(0)
+    _check(lib.pa_decode_plan_bytes(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
+                                    max_seq_len, partition_size, _KV_CODE[kv_cache_dtype],
+                                    ctypes.byref(out)), "pa_decode_plan_bytes")
+    return int(out.value)
+
+
+def decode_plan(seq_lens: torch.Tensor, num_q_heads: int, num_kv_heads: int, head_dim: int,
+                block_size: int, max_seq_len: int, partition_size: int = 0,
+                kv_cache_dtype: str = "auto", plan: Optional[torch.Tensor] = None):
+    """The split plan for HOST int32 lengths, computed on the host
+    (pa_decode_plan).  Returns (plan, needs_combine): plan is a host uint8
+    tensor (pinned when allocated here) to copy to 256-byte aligned device
+    memory for decode_attention_planned."""
+    _need(seq_lens.device.type == "cpu" and seq_lens.dtype == torch.int32 and
+          seq_lens.is_contiguous(), "seq_lens: contiguous int32 on the host")
+    B = seq_lens.numel()
+    n = decode_plan_bytes(B, num_q_heads, num_kv_heads, head_dim, block_size, max_seq_len,
+                          partition_size, kv_cache_dtype)
+    if plan is None:
+        plan = torch.empty(n, dtype=torch.uint8).pin_memory()
+    _need(plan.device.type == "cpu" and plan.numel() >= n and plan.is_contiguous(),
+          "plan: a contiguous host buffer of decode_plan_bytes() bytes")
+    comb = ctypes.c_int32(0)
+    _check(lib.pa_decode_plan(_ptr(seq_lens), B, num_q_heads, num_kv_heads, head_dim, block_size,
+                              max_seq_len, partition_size, _KV_CODE[kv_cache_dtype], _ptr(plan),
+                              plan.numel(), ctypes.byref(comb)), "pa_decode_plan")
+    return plan, bool(comb.value)
+
+
+def decode_attention_planned(out: torch.Tensor, query: torch.Tensor, key_cache: torch.Tensor,
+                             value_cache: torch.Tensor, block_tables: torch.Tensor,
+                             seq_lens: torch.Tensor, max_seq_len: int, scale: float,
+                             plan: torch.Tensor, partition_size: int = 0,
+                             workspace: Optional[torch.Tensor] = None,
+                             k_scale: Optional[torch.Tensor] = None,
+                             v_scale: Optional[torch.Tensor] = None,
+                             error_flag: Optional[torch.Tensor] = None,
+                             stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """decode_attention (decode_attention_fp8 for uint8 code pools, with the
+    scales) with the split plan read from the device copy `plan` of a
+    decode_plan() result: no plan kernel.  Contiguous pools."""
+    fp8 = key_cache.dtype == torch.uint8
+    if fp8:
+        _need(query.dim() == 3 and query.is_contiguous() and out.shape == query.shape and
+              out.is_contiguous(), "query / out must be contiguous [B, Hq, D]")
+        _need(value_cache.dtype == torch.uint8 and key_cache.shape == value_cache.shape and
+              key_cache.is_contiguous() and value_cache.is_contiguous(),
+              "fp8 pools: contiguous uint8 codes of one shape")
+        _need(k_scale is not None and v_scale is not None and k_scale.dtype == torch.float32 and
+              v_scale.dtype == torch.float32, "fp8 pools need float32 k_scale and v_scale")
+        _need(block_tables.dtype == torch.int32 and block_tables.dim() == 2 and
+              block_tables.stride(1) == 1, "block_tables int32 [B, W], rows contiguous")
+        _need(seq_lens.dtype == torch.int32 and seq_lens.is_contiguous(), "seq_lens int32")
+        _need(key_cache.shape[3] == query.shape[2], "query and pools must share head_dim")
+        _dtype_code(out.dtype), _dtype_code(query.dtype)
+    else:
+        _decode_args(out, query, key_cache, value_cache, block_tables, seq_lens,
+                     allow_strided_pools=False)
+    _need(plan.is_cuda and plan.is_contiguous() and plan.data_ptr() % 256 == 0,
+          "plan: the decode_plan() bytes in 256-byte aligned device memory")
+    B, hq, d = query.shape
+    nb, bs, hkv, _ = key_cache.shape
+    if workspace is None:
+        workspace = alloc_workspace(decode_workspace_bytes(B, hq, hkv, d, bs, max_seq_len,
+                                                           partition_size), query.device)
+    _check(lib.pa_decode_attention_planned(
+        _ptr(out), _dtype_code(out.dtype), _ptr(query), _dtype_code(query.dtype),
+        _ptr(key_cache), _ptr(value_cache), 1 if fp8 else 0, _ptr(k_scale), _ptr(v_scale),
+        _ptr(block_tables), block_tables.stride(0), _ptr(seq_lens), B, int(max_seq_len), hq, hkv,
+        d, nb, bs, float(scale), int(partition_size), _ptr(plan), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _ptr(error_flag), _stream_handle(stream)),
+        "pa_decode_attention_planned")
+    return out
+
+
+def split_plan(seq_lens, max_seq_len: int, partition_size: int, num_ctas: int) -> dict:
+    """pa_split_plan on host lengths (no GPU): the tile and segment prefix
+    sums and each CTA's start, as numpy arrays."""
+    import numpy as np
+    lens = np.ascontiguousarray(np.asarray(seq_lens, dtype=np.int32))
+    B = lens.size
+    tiles = np.zeros(B + 1, np.int32)
+    segs = np.zeros(B + 1, np.int32)
+    start = np.zeros(num_ctas, np.int32)
+    firstk = np.zeros(num_ctas, np.int32)
+    nseg, comb = ctypes.c_int32(0), ctypes.c_int32(0)
+    vp = lambda a: ctypes.c_void_p(a.ctypes.data)
+    _check(lib.pa_split_plan(vp(lens), B, int(max_seq_len), int(partition_size), int(num_ctas),
+                             vp(tiles), vp(segs), vp(start), vp(firstk), ctypes.byref(nseg),
+                             ctypes.byref(comb)), "pa_split_plan")
+    return {"tiles": tiles, "seg_base": segs, "start_seq": start, "first_k": firstk,
+            "num_segments": int(nseg.value), "needs_combine": bool(comb.value)}
+
+
+class DecodeStep:
+    """One decode step from pinned host memory through the C entry points
+    pa_decode_step_upload / _run / _download (argument marshalling only: the
+    library computes the split plan on the host, makes the one host-to-device
+    copy, launches the kernels and makes the one device-to-host copy).
+
+    ``host(slot)`` gives the pinned staging views to write the step's inputs
+    into (``q``, ``new_k``, ``new_v``, ``slots``, ``tables``, ``lens``,
+    ``cow``); ``submit(slot, num_cow)`` enqueues the step and returns at once;
+    ``wait(slot)`` returns the slot's pinned output once it has arrived.
+    Each slot has its own staging buffer, device scratch and output, so a
+    serving loop can fill and submit step i + 1 while step i runs.  The
+    uploads run on a copy-in stream and the downloads on a copy-out stream,
+    so they overlap other steps' kernels; the kernels of every step run on
+    one compute stream, in submission order, so a step attends the rows the
+    steps before it wrote.  A slot may be refilled once its step has been
+    waited for.  ``__call__`` runs one step with pa_decode_step (the three
+    parts on one stream) and waits for it.
+    """
+
+    def __init__(self, key_cache: torch.Tensor, value_cache: torch.Tensor, num_seqs: int,
+                 num_q_heads: int, table_width: int, max_seq_len: int, scale: float,
+                 partition_size: int = 0, query_dtype: Optional[torch.dtype] = None,
+                 out_dtype: Optional[torch.dtype] = None, k_scale: Optional[torch.Tensor] = None,
+                 v_scale: Optional[torch.Tensor] = None, max_cow: int = 0, slots: int = 1):
+        _need(slots >= 1, "at least one slot")
+        _need(key_cache.shape == value_cache.shape and key_cache.is_contiguous() and
+              value_cache.is_contiguous(), "contiguous K and V pools of one shape")
+        self.fp8 = key_cache.dtype == torch.uint8
+        _need(not self.fp8 or (query_dtype is not None and k_scale is not None and
+                               v_scale is not None), "fp8 pools need query_dtype and scales")
+        dt = query_dtype if query_dtype is not None else key_cache.dtype
+        nb, bs, hkv, d = key_cache.shape
+        self.k, self.v, self.k_scale, self.v_scale = key_cache, value_cache, k_scale, v_scale
+        self.scale = float(scale)
+        self.shape = StepShape(num_seqs, num_q_heads, hkv, d, nb, bs, table_width, max_seq_len,
+                               partition_size, max_cow, _dtype_code(dt),
+                               _dtype_code(out_dtype or dt), 1 if self.fp8 else 0)
+        lay = StepLayout()
+        _check(lib.pa_decode_step_layout(ctypes.byref(self.shape), ctypes.byref(lay)),
+               "pa_decode_step_layout")
+        self.layout = lay
+        dev = key_cache.device
+        fields = [("q", lay.query, (num_seqs, num_q_heads, d), dt),
+                  ("new_k", lay.new_k, (num_seqs, hkv, d), dt),
+                  ("new_v", lay.new_v, (num_seqs, hkv, d), dt),
+                  ("slots", lay.slot_mapping, (num_seqs,), torch.int32),
+                  ("tables", lay.block_tables, (num_seqs, table_width), torch.int32),
+                  ("lens", lay.seq_lens, (num_seqs,), torch.int32),
+                  ("cow", lay.cow_pairs, (max_cow, 2), torch.int32)]
+
+        def views(buf):
+            v = {}
+            for name, off, shape, dtype in fields:
+                n = int(torch.Size(shape).numel()) * torch.empty((), dtype=dtype).element_size()
+                v[name] = buf[off:off + n].view(dtype).view(shape)
+            return v
+
+        self._staging = [torch.zeros(lay.host_bytes, dtype=torch.uint8).pin_memory()
+                         for _ in range(slots)]
+        self._views = [views(b) for b in self._staging]
+        self._scratch = [torch.empty(lay.device_bytes, dtype=torch.uint8, device=dev)
+                         for _ in range(slots)]
+        out_shape = (num_seqs, num_q_heads, d)
+        self._outs = [torch.empty(out_shape, dtype=out_dtype or dt).pin_memory()
+                      for _ in range(slots)]
+        self.stream = torch.cuda.Stream(device=dev)       # kernels, in submission order
+        self._copy_in = torch.cuda.Stream(device=dev)
+        self._copy_out = torch.cuda.Stream(device=dev)
+        self._ev_in = [torch.cuda.Event() for _ in range(slots)]
+        self._ev_run = [torch.cuda.Event() for _ in range(slots)]
+        self._ev_out = [torch.cuda.Event() for _ in range(slots)]
+        self._pending = [False] * slots
+
+    def h2d_bytes(self) -> int:
+        return int(self.layout.host_bytes)
+
+    def d2h_bytes(self) -> int:
+        return int(self.layout.out_bytes)
+
+    def host(self, slot: int = 0) -> dict:
+        return self._views[slot]
+
+    def submit(self, slot: int = 0, num_cow: int = 0,
+               error_flag: Optional[torch.Tensor] = None) -> None:
+        _need(not self._pending[slot], "wait for the slot's previous step first")
+        sh, st, sc = ctypes.byref(self.shape), self._staging[slot], self._scratch[slot]
+        nbytes = sc.numel()
+        # the slot's scratch is free once its previous kernels have finished
+        self._copy_in.wait_event(self._ev_run[slot])
+        _check(lib.pa_decode_step_upload(sh, _ptr(st), _ptr(sc), nbytes,
+                                         _stream_handle(self._copy_in)), "pa_decode_step_upload")
+        self._ev_in[slot].record(self._copy_in)
+        self.stream.wait_event(self._ev_in[slot])
+        _check(lib.pa_decode_step_run(sh, _ptr(st), int(num_cow), _ptr(self.k), _ptr(self.v),
+                                      _ptr(self.k_scale), _ptr(self.v_scale), self.scale,
+                                      _ptr(sc), nbytes, _ptr(error_flag),
+                                      _stream_handle(self.stream)), "pa_decode_step_run")
+        self._ev_run[slot].record(self.stream)
+        self._copy_out.wait_event(self._ev_run[slot])
+        _check(lib.pa_decode_step_download(sh, _ptr(sc), nbytes, _ptr(self._outs[slot]),
+                                           _stream_handle(self._copy_out)),
+               "pa_decode_step_download")
+        self._ev_out[slot].record(self._copy_out)
+        self._pending[slot] = True
+
+    def wait(self, slot: int = 0) -> torch.Tensor:
+        self._ev_out[slot].synchronize()
+        self._pending[slot] = False
+        return self._outs[slot]
+
+    def __call__(self, num_cow: int = 0, error_flag: Optional[torch.Tensor] = None):
+        """One step through pa_decode_step on the compute stream, waited for."""
+        _need(not self._pending[0], "wait for slot 0's previous step first")
+        sc = self._scratch[0]
+        _check(lib.pa_decode_step(ctypes.byref(self.shape), _ptr(self._staging[0]),
+                                  int(num_cow), _ptr(self.k), _ptr(self.v), _ptr(self.k_scale),
+                                  _ptr(self.v_scale), self.scale, _ptr(sc), sc.numel(),
+                                  _ptr(self._outs[0]), _ptr(error_flag),
+                                  _stream_handle(self.stream)), "pa_decode_step")
+        self.stream.synchronize()
+        return self._outs[0]
+
+
 # Bytes of the library's static scratch array used by decode_attention_noalloc.
 NOALLOC_SCRATCH_BYTES = 16 << 20
 
@@ -515,12 +804,15 @@ def decode_attention_noalloc(out: torch.Tensor, query: torch.Tensor, key_cache: 
                              stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
     """decode_attention for callers that must not allocate device memory: the
     scratch is the library's static per-device array (NOALLOC_SCRATCH_BYTES),
-    so this wrapper allocates nothing either.  Shapes needing more scratch raise
+    so this wrapper allocates nothing either.  Arguments are checked as in
+    decode_attention, except that the pools must be contiguous (there is no
+    strided form of this entry point).  Shapes needing more scratch raise
     PagedAttnError PA_ERR_TOO_LARGE.  Calls overlapping on the GPU share the
     array and race; the first call on a device should precede stream capture."""
+    _decode_args(out, query, key_cache, value_cache, block_tables, seq_lens,
+                 allow_strided_pools=False)
     B, hq, d = query.shape
     nb, bs, hkv, _ = key_cache.shape
-    _need(key_cache.shape[3] == d, "query and pools must share head_dim")
     _check(lib.pa_decode_attention_noalloc(
         _ptr(out), _dtype_code(out.dtype), _ptr(query), _ptr(key_cache), _ptr(value_cache),
         _ptr(block_tables), block_tables.stride(0), _ptr(seq_lens), B, int(max_seq_len), hq, hkv,
@@ -710,172 +1002,3 @@ class BlockManager:
         d["sharing_saving"] = (1.0 - d["held_blocks"] / d["logical_blocks"]
                                if d["logical_blocks"] else 0.0)
         return d
-
-
-class PagedDecodeStep:
-    """One decode step driven from pinned host memory (the end-to-end call).
-
-    Holds, for a fixed batch shape, pinned host staging buffers and device
-    buffers of the same layout.  The caller writes the step's inputs into the
-    views of ``host`` (``q``, ``new_k``, ``new_v``, ``slots``, ``tables``,
-    ``lens``); a call copies the whole staging buffer host->device in one copy,
-    writes the new rows into the pools with reshape_and_cache, runs
-    decode_attention, copies the output into the pinned ``host_out`` in one copy
-    and waits for the stream.  With ``use_graph`` (default) the first call runs
-    eagerly and captures the step (copies and kernels) into a CUDA graph that
-    later calls replay.
-
-    Pipelined use (``slots`` >= 2): slot s has its own staging buffers
-    (``slot_host(s)``, slot 0 being ``host``) and output (``slot_out(s)``);
-    ``submit(s)`` enqueues the slot's host->device copy on a copy stream, the
-    kernels on the compute stream and the device->host copy of the output on a
-    second copy stream, ordered by events, and returns at once; ``wait(s)``
-    returns the slot's pinned output once it has arrived.  A serving loop
-    submits step i + 1 before it waits for step i, so the copies of one step
-    overlap the kernels of another.  A slot's inputs may be rewritten once its
-    previous ``submit`` has been waited for."""
-
-    _ALIGN = 256
-
-    def __init__(self, key_cache: torch.Tensor, value_cache: torch.Tensor, num_seqs: int,
-                 num_q_heads: int, table_width: int, max_seq_len: int, scale: float,
-                 partition_size: int = 0, out_dtype: Optional[torch.dtype] = None,
-                 stream: Optional[torch.cuda.Stream] = None, use_graph: bool = True,
-                 query_dtype: Optional[torch.dtype] = None,
-                 k_scale: Optional[torch.Tensor] = None, v_scale: Optional[torch.Tensor] = None,
-                 slots: int = 1):
-        """uint8 pools are fp8 (E4M3) code pools: pass query_dtype and the
-        one-element float32 device scales."""
-        _need(slots >= 1, "at least one slot")
-        self.k, self.v = key_cache, value_cache
-        nb, bs, hkv, d = key_cache.shape
-        dev = key_cache.device
-        self.fp8 = key_cache.dtype == torch.uint8
-        _need(not self.fp8 or (query_dtype is not None and k_scale is not None and
-                               v_scale is not None), "fp8 pools need query_dtype and scales")
-        self.k_scale, self.v_scale = k_scale, v_scale
-        dt = query_dtype if self.fp8 else key_cache.dtype
-        self.max_seq_len, self.scale, self.partition_size = max_seq_len, scale, partition_size
-        self.stream = stream if stream is not None else torch.cuda.Stream(device=dev)
-        self.use_graph = use_graph
-        self.graph = None
-        fields = [("q", (num_seqs, num_q_heads, d), dt), ("new_k", (num_seqs, hkv, d), dt),
-                  ("new_v", (num_seqs, hkv, d), dt), ("slots", (num_seqs,), torch.int32),
-                  ("tables", (num_seqs, table_width), torch.int32),
-                  ("lens", (num_seqs,), torch.int32)]
-        layout, off = [], 0
-        for name, shape, dtype in fields:
-            nbytes = int(torch.Size(shape).numel()) * torch.empty((), dtype=dtype).element_size()
-            layout.append((name, shape, dtype, off, nbytes))
-            off += -(-nbytes // self._ALIGN) * self._ALIGN
-        self._nbytes = off
-
-        def views(buf):
-            return {name: buf[o:o + n].view(dtype).view(shape) for name, shape, dtype, o, n in layout}
-
-        out_shape = (num_seqs, num_q_heads, d)
-        self._host_bufs = [torch.empty(off, dtype=torch.uint8).pin_memory() for _ in range(slots)]
-        self._dev_bufs = [torch.empty(off, dtype=torch.uint8, device=dev) for _ in range(slots)]
-        self._hosts = [views(b) for b in self._host_bufs]
-        self._devs = [views(b) for b in self._dev_bufs]
-        self._outs = [torch.empty(out_shape, dtype=out_dtype or dt, device=dev)
-                      for _ in range(slots)]
-        self._host_outs = [torch.empty(out_shape, dtype=out_dtype or dt).pin_memory()
-                           for _ in range(slots)]
-        # slot 0 is also the sequential call's buffers
-        self._host_buf, self._dev_buf = self._host_bufs[0], self._dev_bufs[0]
-        self.host, self.dev = self._hosts[0], self._devs[0]
-        self.out, self.host_out = self._outs[0], self._host_outs[0]
-        self.ws = alloc_workspace(decode_workspace_bytes(num_seqs, num_q_heads, hkv, d, bs,
-                                                         max_seq_len, partition_size), dev)
-        # pipelined use: copy streams, per-slot events and compute graphs
-        self._copy_in = torch.cuda.Stream(device=dev)
-        self._copy_out = torch.cuda.Stream(device=dev)
-        self._ev_in = [torch.cuda.Event() for _ in range(slots)]
-        self._ev_comp = [torch.cuda.Event() for _ in range(slots)]
-        self._ev_out = [torch.cuda.Event() for _ in range(slots)]
-        self._slot_graphs = [None] * slots
-        self._pending = [False] * slots
-
-    def h2d_bytes(self) -> int:
-        return self._nbytes
-
-    def d2h_bytes(self) -> int:
-        return self.out.numel() * self.out.element_size()
-
-    def slot_host(self, slot: int) -> dict:
-        """Pinned input views of a slot (write them before ``submit(slot)``)."""
-        return self._hosts[slot]
-
-    def slot_out(self, slot: int) -> torch.Tensor:
-        return self._host_outs[slot]
-
-    def _kernels(self, dv, out) -> None:
-        if self.fp8:
-            reshape_and_cache(dv["new_k"], dv["new_v"], self.k, self.v, dv["slots"],
-                              kv_cache_dtype="fp8_e4m3", k_scale=self.k_scale,
-                              v_scale=self.v_scale)
-            decode_attention_fp8(out, dv["q"], self.k, self.v, self.k_scale, self.v_scale,
-                                 dv["tables"], dv["lens"], self.max_seq_len, self.scale,
-                                 self.partition_size, self.ws)
-        else:
-            reshape_and_cache(dv["new_k"], dv["new_v"], self.k, self.v, dv["slots"])
-            decode_attention(out, dv["q"], self.k, self.v, dv["tables"], dv["lens"],
-                             self.max_seq_len, self.scale, self.partition_size, self.ws)
-
-    def _enqueue(self) -> None:
-        self._dev_buf.copy_(self._host_buf, non_blocking=True)
-        self._kernels(self.dev, self.out)
-        self.host_out.copy_(self.out, non_blocking=True)
-
-    def __call__(self) -> torch.Tensor:
-        if self.graph is not None:
-            with torch.cuda.stream(self.stream):
-                self.graph.replay()
-            self.stream.synchronize()
-            return self.host_out
-        with torch.cuda.stream(self.stream):
-            self._enqueue()
-        self.stream.synchronize()
-        if self.use_graph:
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=self.stream, capture_error_mode="thread_local"):
-                self._enqueue()
-            self.graph = g
-        return self.host_out
-
-    def submit(self, slot: int) -> None:
-        """Enqueue one step on a slot: copy in, kernels, copy out; no wait."""
-        _need(not self._pending[slot], "wait for the slot's previous step first")
-        cs, ci, co = self.stream, self._copy_in, self._copy_out
-        # the slot's device inputs are free once its previous kernels finished
-        ci.wait_event(self._ev_comp[slot])
-        with torch.cuda.stream(ci):
-            self._dev_bufs[slot].copy_(self._host_bufs[slot], non_blocking=True)
-            self._ev_in[slot].record(ci)
-        cs.wait_event(self._ev_in[slot])
-        g = self._slot_graphs[slot]
-        if g is not None:
-            with torch.cuda.stream(cs):
-                g.replay()
-        else:
-            with torch.cuda.stream(cs):
-                self._kernels(self._devs[slot], self._outs[slot])
-            if self.use_graph:
-                cs.synchronize()
-                g = torch.cuda.CUDAGraph()
-                with torch.cuda.graph(g, stream=cs, capture_error_mode="thread_local"):
-                    self._kernels(self._devs[slot], self._outs[slot])
-                self._slot_graphs[slot] = g
-        self._ev_comp[slot].record(cs)
-        co.wait_event(self._ev_comp[slot])
-        with torch.cuda.stream(co):
-            self._host_outs[slot].copy_(self._outs[slot], non_blocking=True)
-            self._ev_out[slot].record(co)
-        self._pending[slot] = True
-
-    def wait(self, slot: int) -> torch.Tensor:
-        """The slot's pinned output, once its device->host copy has landed."""
-        self._ev_out[slot].synchronize()
-        self._pending[slot] = False
-        return self._host_outs[slot]

@@ -30,94 +30,11 @@
 #include <cstring>
 #include <mutex>
 
+#include "pa_decode_common.cuh"
 #include "pa_device.cuh"
 #include "pa_host.h"
 
 namespace pa {
-
-constexpr int kTile = 16;            // tokens per tile (MMA M of the score product)
-constexpr int kPlanThreads = 256;
-constexpr int kCombineWarps = 4;
-
-enum : int32_t {
-  kNewSeq = 1,    // first tile of a sequence in this CTA: reload Q
-  kSegStart = 2,  // reset the online-softmax state
-  kSegEnd = 4,    // finalise and write the segment
-  kDirect = 8,    // the segment is the whole sequence: write `out` directly
-  kCausal = 16,   // several query tokens of one sequence: column c sees rows <= rel + c / G
-};
-
-constexpr int kMaxPack = 8;        // sequences per pack
-constexpr int kMaxPackCols = 32;   // query columns per KV head of a pack (4 blocks of 8)
-constexpr int kMinPackTiles = 4;   // shared prefixes shorter than this are not packed
-
-struct TileInfo {
-  int32_t b;       // sequence (the first member of a pack)
-  int32_t valid;   // tokens of this tile inside the sequence (1..16)
-  int32_t mask;    // bit t set: token t takes part (valid and its block id is good)
-  int32_t seg;     // segment id inside this head group
-  int32_t flags;
-  int32_t members;  // query rows using this tile: pack members, query tokens, or 1
-  int32_t qrow0;    // query row of column 0 (column c: row qrow0 + c / G, head c % G)
-  int32_t rel;      // kCausal: last visible tile row of column 0 (may be < 0 or > 15)
-};
-
-struct DecodeParams {
-  void* out;
-  const uint16_t* query;
-  const int32_t* block_tables;
-  const int32_t* seq_lens;
-  int64_t table_stride;
-  int32_t out_dtype;
-  int32_t num_seqs, max_seq_len, num_q_heads, group, num_blocks, block_size;
-  int32_t num_rows;        // query (and output) rows: num_seqs, or the multi-query rows
-  int32_t tiles_per_part;  // partition length in tiles (INT_MAX: no partitions)
-  float scale_log2;        // scale * log2(e)
-  int32_t ctas_per_group;  // CTAs sharing one head group's tiles
-  int32_t heads_per_cta;   // KV heads per CTA (HG)
-  int32_t nseg_cap;        // partial slots per head group
-  int32_t stages;
-  int32_t tok_box;         // tokens per TMA box: min(block_size, 16)
-  int32_t tma_mode;        // 0: one box per block per tile, 1: one per (head, d-half)
-  int32_t plan_closed;     // 1: segment bookkeeping in closed form (many cut points per
-                           //    entry); 0: walk each entry's cut points (few)
-  int32_t* plan_tiles;     // [entries + 1] tile prefix sums
-  int32_t* seg_base;       // [entries + 1] segment prefix sums (partial slots)
-  int32_t* start_seq;      // [ctas_per_group] entry holding each CTA's first tile
-  int32_t* first_k;        // [ctas_per_group] index of that tile's segment in its entry
-  // shared prompts: packs of pack_size consecutive sequences whose block tables
-  // share leading blocks are attended together over that prefix ("entries"
-  // 0 .. K-1 are the packs' prefixes, K + b the rest of sequence b)
-  const int32_t* shared_blocks;  // [num_seqs] leading blocks b shares with b + 1, or null
-  int32_t pack_size;       // sequences per window (1: no packing)
-  int32_t* pack_first;     // [num_seqs / 2] first sequence of pack k
-  int32_t* pack_n;         // [num_seqs / 2] sequences of pack k (pack_size, or 2)
-  int32_t* pack_tiles;     // [num_seqs / 2] prefix tiles of pack k
-  int32_t* seq_pack;       // [num_seqs] pack of sequence b, or -1
-  int32_t* seq_pre;        // [num_seqs] tiles of b attended through its pack
-  int32_t* meta;           // [2] number of packs K (0 without packing), number of entries E
-  // several query tokens per sequence ("multi-query"): entries are chunks of
-  // at most q_per_entry query tokens of one sequence
-  const int32_t* q_start;  // [num_seqs + 1] query rows of sequence b, or null
-  int32_t q_per_entry;
-  int32_t* ent_b;          // [rows] sequence of entry e
-  int32_t* ent_q0;         // [rows] first query row of entry e
-  int32_t* ent_nq;         // [rows] query rows of entry e
-  int32_t* ent_tok;        // [rows] tokens entry e reads: one past its last query's position
-  int32_t* q_entry;        // [rows] entry of query row r
-  int32_t cols;            // partial columns per KV head: pack_size * group
-  float* part_o;           // [groups][nseg_cap][HG][cols][head_dim]
-  float* part_ml;          // [groups][nseg_cap][HG][cols][2]  (m in log2 units, l)
-  int32_t* err;
-  const float* k_scale;    // fp8 cache only: element = code * (*k_scale)
-  const float* v_scale;
-  int32_t q_bf16;          // fp8 cache only: the query is bf16 (else fp16)
-};
-
-__device__ __forceinline__ int32_t clamp_len(int32_t L, int32_t max_len) {
-  return L < 0 ? 0 : (L > max_len ? max_len : L);
-}
-
 
 // ---------------------------------------------------------------------------
 // plan (one CTA)
@@ -526,6 +443,10 @@ __global__ void __launch_bounds__((HG * CG + 1) * 32, 1)
   __syncthreads();
   griddep_launch_dependents();
   griddep_wait();  // the plan (and all earlier work on the stream) is complete
+  if (!host_plan_matches(p)) {  // a plan made for another shape: no work at all
+    if (threadIdx.x == 0 && c == 0 && hg == 0) flag_error(p.err, PA_DEVERR_BAD_PLAN);
+    return;
+  }
 
   // entries: packs' prefixes then sequences, or query chunks (plain: the B sequences)
   const bool plain = p.pack_size == 1 && p.q_start == nullptr;
@@ -538,165 +459,9 @@ __global__ void __launch_bounds__((HG * CG + 1) * 32, 1)
   if (warp == NW) {
     // ======================= producer =======================
     if (lane != 0) return;
-    const uint64_t policy = l2_policy_evict_first();
-    const int bs = p.block_size;
-    const int TB = p.tok_box;
-    const uint32_t box_bytes = static_cast<uint32_t>(HG * DCT * TB * 128);
-    const int bpt = bs < kTile ? kTile / bs : 1;  // blocks per tile
-    const int K = plain ? 0 : p.meta[0];
-    // the entry being walked: tiles t_first .. t_first + n_e - 1 of the line,
-    // which are tiles i0 .. i0 + n_e - 1 of sequence b (of every pack member)
-    int e = p.start_seq[c];
-    int b = 0, members = 1;
-    int32_t t_first = 0, n_e = 0, i0 = 0, L_b = 0, seg_e = 0, nseg_e = 0;
-    int32_t qrow0 = 0, lim0 = 0;  // first query row; causal: position of query 0
-    bool pack = false;
-    const int32_t* row = p.block_tables;
-    auto enter = [&](int ent) {
-      t_first = p.plan_tiles[ent];
-      n_e = p.plan_tiles[ent + 1] - t_first;
-      seg_e = p.seg_base[ent];
-      nseg_e = p.seg_base[ent + 1] - seg_e;
-      pack = false;
-      if (p.q_start != nullptr) {
-        b = p.ent_b[ent];
-        members = p.ent_nq[ent];
-        i0 = 0;
-        L_b = p.ent_tok[ent];
-        qrow0 = p.ent_q0[ent];
-        lim0 = L_b - members;
-      } else if (ent < K) {
-        b = p.pack_first[ent];
-        members = p.pack_n[ent];
-        i0 = 0;
-        L_b = n_e * kTile;
-        qrow0 = b;
-        pack = true;
-      } else {
-        b = ent - K;
-        members = 1;
-        i0 = p.pack_size > 1 ? p.seq_pre[b] : 0;
-        L_b = clamp_len(p.seq_lens[b], p.max_seq_len);
-        qrow0 = b;
-      }
-      row = p.block_tables + static_cast<int64_t>(b) * p.table_stride;
-    };
-    enter(e);
-    int32_t k = p.first_k[c] - 1;  // segment index inside the entry (advanced at starts)
-    int32_t i = static_cast<int32_t>(lo - t_first);
-    bool new_seq = true;
-    int stage = 0;
-    uint32_t phase = 0;
-    int64_t issued = 0;
-    // the pack's other members must hold the same block ids
-    auto check_shared = [&](int64_t idx, int32_t id) {
-      for (int m = 1; m < members; ++m)
-        if (__ldg(row + static_cast<int64_t>(m) * p.table_stride + idx) != id)
-          flag_error(p.err, PA_DEVERR_BAD_SHARE);
-    };
-    // Tile index inside its partition: segments start at the CTA's first
-    // tile, at an entry's first tile and at every partition start, and end
-    // before the next start or at the CTA's last tile.
-    const int32_t tpp = p.tiles_per_part;
-    int32_t ip = tpp == INT_MAX ? i : i % tpp;
-    for (int64_t t = lo; t < hi; ++t, ++i) {
-      while (i >= n_e) {  // next entry that has tiles
-        enter(++e);
-        k = -1;
-        i = 0;
-        ip = 0;
-        new_seq = true;
-      }
-      const int32_t ti_seq = i0 + i;  // tile index inside the sequence
-      const int32_t valid = min(kTile, L_b - ti_seq * kTile);
-      int32_t flags = new_seq ? kNewSeq : 0;
-      if (t == lo || ip == 0) {
-        flags |= kSegStart;
-        ++k;
-      }
-      if (t == hi - 1 || i == n_e - 1 || ip == tpp - 1) flags |= kSegEnd;
-      // one segment holds the whole attention of every query row of the entry
-      if (nseg_e == 1 && !pack && i0 == 0) flags |= kDirect;
-      if (p.q_start != nullptr) flags |= kCausal;
-      new_seq = false;
-      if (++ip == tpp) ip = 0;
-      uint32_t mask = valid >= kTile ? 0xffffu : ((1u << valid) - 1u);
-      // the first block id is loaded before the wait for a free stage
-      const int64_t idx0 = bs <= kTile ? static_cast<int64_t>(ti_seq) * bpt
-                                       : static_cast<int64_t>(ti_seq) * kTile / bs;
-      const int32_t id0 = __ldg(row + idx0);
-
-      if (!mbar_wait(empty(stage), phase ^ 1u, p.err)) break;
-      const uint32_t kdst = smem_base + static_cast<uint32_t>(stage) * 2u * kTileBytes;
-      const uint32_t vdst = kdst + kTileBytes;
-      // one box per block of the tile; each copy's bytes are announced on the
-      // stage's barriers just before it is issued
-      auto issue = [&](uint32_t off, int32_t tok_off, int32_t id) {
-        mbar_expect_tx(full_k(stage), box_bytes);
-        mbar_expect_tx(full_v(stage), box_bytes);
-        if (p.tma_mode == 0) {
-          tma_load_5d(kdst + off, &tmK, full_k(stage), 0, tok_off, 0, hg * HG, id, policy);
-          tma_load_5d(vdst + off, &tmV, full_v(stage), 0, tok_off, 0, hg * HG, id, policy);
-        } else {
-          for (int hh = 0; hh < HG; ++hh) {
-            for (int dc = 0; dc < DCT; ++dc) {
-              const uint32_t o2 = off + ((hh * DCT + dc) * TB) * 128u;
-              tma_load_5d(kdst + o2, &tmK, full_k(stage), 0, dc, hg * HG + hh, tok_off, id,
-                          policy);
-              tma_load_5d(vdst + o2, &tmV, full_v(stage), 0, dc, hg * HG + hh, tok_off, id,
-                          policy);
-            }
-          }
-        }
-      };
-      if (bs <= kTile) {
-#pragma unroll
-        for (int kk = 0; kk < kTile / 4; ++kk) {  // at most 4 blocks: block_size >= 4
-          const int tok0 = kk * bs;
-          if (kk < bpt && tok0 < valid) {
-            const int64_t idx = idx0 + kk;
-            const int32_t id = kk == 0 ? id0 : __ldg(row + idx);
-            if (pack) check_shared(idx, id);
-            if (id < 0 || id >= p.num_blocks) {
-              flag_error(p.err, PA_DEVERR_BAD_BLOCK);
-              mask &= ~(((1u << bs) - 1u) << tok0);
-            } else {
-              issue(static_cast<uint32_t>(kk) * box_bytes, 0, id);
-            }
-          }
-        }
-      } else {
-        if (pack) check_shared(idx0, id0);
-        if (id0 < 0 || id0 >= p.num_blocks) {
-          flag_error(p.err, PA_DEVERR_BAD_BLOCK);
-          mask = 0;
-        } else {
-          issue(0, static_cast<int32_t>((static_cast<int64_t>(ti_seq) * kTile) % bs), id0);
-        }
-      }
-      TileInfo& ti = info[stage];
-      ti.b = b;
-      ti.valid = valid;
-      ti.mask = static_cast<int32_t>(mask);
-      ti.seg = seg_e + k;
-      ti.flags = flags;
-      ti.members = members;
-      ti.qrow0 = qrow0;
-      ti.rel = (flags & kCausal) ? lim0 - ti_seq * kTile : kTile;  // kTile: every row visible
-      // the one arrival of the phase: it completes once the announced bytes land
-      mbar_arrive(full_k(stage));
-      mbar_arrive(full_v(stage));
-      ++issued;
-      if (++stage == NS) { stage = 0; phase ^= 1u; }
-    }
-    // Wait (bounded) until every load this warp issued has landed, so that no
-    // copy is in flight into shared memory when the CTA retires.
-    for (int64_t k = (issued > NS ? issued - NS : 0); k < issued; ++k) {
-      const int s = static_cast<int>(k % NS);
-      const uint32_t par = static_cast<uint32_t>((k / NS) & 1);
-      if (!mbar_wait(full_k(s), par, p.err)) break;
-      if (!mbar_wait(full_v(s), par, p.err)) break;
-    }
+    produce_tiles<HG, DCT>(p, &tmK, &tmV, smem_base, kTileBytes, info, full_k(0), full_v(0),
+                           empty(0), NS, lo, hi, c, hg, plain,
+                           [](int32_t, int32_t) { return true; });
     return;
   }
 
@@ -1141,7 +906,7 @@ __global__ void __launch_bounds__(kCombineWarps * 32) pa_combine_narrow_kernel(c
   // this grid before touching data
   griddep_launch_dependents();
   griddep_wait();  // the main kernel's partials are complete and visible
-  if (qh >= p.num_q_heads) return;
+  if (qh >= p.num_q_heads || !host_plan_matches(p)) return;
   const int G = p.group, HG = p.heads_per_cta;
   const int kvh = qh / G, h = qh - kvh * G;
   const int hg = kvh / HG, g = kvh - hg * HG;
@@ -1222,6 +987,7 @@ __global__ void __launch_bounds__(kCombineWarps * 32) pa_combine_wide_kernel(con
   // this grid before touching data
   griddep_launch_dependents();
   griddep_wait();  // the main kernel's partials are complete and visible
+  if (!host_plan_matches(p)) return;
   const int G = p.group, HG = p.heads_per_cta;
   const int kvh = qh / G, h = qh - kvh * G;
   const int hg = kvh / HG, g = kvh - hg * HG;
@@ -1349,9 +1115,11 @@ MainKernel select_main(int D, int HG, int NB, int CG, bool bf16, bool fp8) {
 struct LaunchPlan {
   int HG = 0, groups = 0, stages = 0, tok_box = 0, threads = 0;
   int ctas_per_group = 0, tiles_per_part = INT_MAX, nseg_cap = 0;
-  int pack_size = 1, cols = 0, nb = 1, cg = 1, q_per_entry = 0;
+  int pack_size = 1, cols = 0, nb = 1, cg = 1, q_per_entry = 0, head_dim = 0;
   int64_t rows = 0;  // output rows
   bool many_partials = false;  // long sequences / partitions: closed-form plan, wide combine
+  bool umma = false;           // the tensor-memory kernel (many query columns, head_dim 128)
+  UmmaKernel ukernel = nullptr;
   size_t smem = 0;
   size_t off_tiles = 0, off_segs = 0, off_start = 0, off_firstk = 0, off_meta = 0,
          off_pack_first = 0, off_pack_n = 0, off_pack_tiles = 0, off_seq_pack = 0,
@@ -1380,7 +1148,7 @@ pa_status make_plan(int32_t num_seqs, int32_t Hq, int32_t Hkv, int32_t D, int32_
     return PA_ERR_INVALID_ARG;
   if (Hq % Hkv != 0) return PA_ERR_INVALID_ARG;
   if (D != 64 && D != 128) return PA_ERR_UNSUPPORTED;
-  if (!is_pow2(bs) || bs < 4 || bs > 128) return PA_ERR_UNSUPPORTED;
+  if (!is_pow2(bs) || bs < 4 || bs > 256) return PA_ERR_UNSUPPORTED;
   const int G = Hq / Hkv;
   if (G > 8) return PA_ERR_UNSUPPORTED;
   if (partition_size > 0 && (partition_size % kTile != 0 || partition_size % bs != 0))
@@ -1406,27 +1174,49 @@ pa_status make_plan(int32_t num_seqs, int32_t Hq, int32_t Hkv, int32_t D, int32_
   const int DCT = fp8 ? 1 : D / 64;  // 128-byte rows per (token, head) in a stage
   const int TB = bs < kTile ? bs : kTile;
   if ((HG * DCT * TB * 128) % 1024 != 0) return PA_ERR_UNSUPPORTED;
+  // Entries of many query columns (packs, query chunks) with 16-bit caches and
+  // head_dim 128 run on the tensor-memory kernel when its shape rules hold: the
+  // query columns of an entry fill whole 32-row loads (G divides 32), two or
+  // four KV heads per CTA, 8- or 16-token boxes.
+  const bool umma = (P > 1 || Qc > 0) && !fp8 && D == 128 && 32 % G == 0 && TB >= 8 &&
+                    Hkv % 2 == 0;
+  if (umma) HG = Hkv % 4 == 0 ? 4 : 2;
   lp->HG = HG;
+  lp->head_dim = D;
   lp->groups = Hkv / HG;
   lp->tok_box = TB;
-  lp->threads = (HG * CG + 1) * 32;
+  lp->threads = umma ? kUmmaThreads : (HG * CG + 1) * 32;
   lp->nb = NB;
   lp->cg = CG;
-  const size_t tile_bytes = static_cast<size_t>(kTile) * HG * D * (fp8 ? 1 : 2);
-  const size_t budget = 200 * 1024;
-  int stages = static_cast<int>(budget / (2 * tile_bytes));
-  if (stages > 6) stages = 6;
-  if (stages < 2) return PA_ERR_UNSUPPORTED;
-  lp->stages = stages;
-  lp->smem = 1024 + static_cast<size_t>(stages) * 2 * tile_bytes + stages * sizeof(TileInfo) +
-             3 * stages * sizeof(uint64_t);
-  lp->kernel = select_main(D, HG, NB, CG, bf16, fp8);
-  if (lp->kernel == nullptr) return PA_ERR_UNSUPPORTED;
-
+  lp->umma = umma;
   const DeviceInfo* dev = current_device_info();
   if (dev == nullptr) return PA_ERR_CUDA;
-  if (!ensure_smem_attr(reinterpret_cast<const void*>(lp->kernel), lp->smem)) return PA_ERR_CUDA;
-  const int per_sm = ctas_per_sm(reinterpret_cast<const void*>(lp->kernel), lp->threads, lp->smem);
+  const void* kfn = nullptr;
+  if (umma) {
+    int stages = 6;
+    while (stages > 2 &&
+           umma_smem_bytes(HG, stages) > static_cast<size_t>(dev->max_smem_optin))
+      --stages;
+    lp->stages = stages;
+    lp->smem = umma_smem_bytes(HG, stages);
+    lp->ukernel = select_umma(HG, bf16);
+    if (lp->ukernel == nullptr) return PA_ERR_UNSUPPORTED;
+    kfn = reinterpret_cast<const void*>(lp->ukernel);
+  } else {
+    const size_t tile_bytes = static_cast<size_t>(kTile) * HG * D * (fp8 ? 1 : 2);
+    const size_t budget = 200 * 1024;
+    int stages = static_cast<int>(budget / (2 * tile_bytes));
+    if (stages > 6) stages = 6;
+    if (stages < 2) return PA_ERR_UNSUPPORTED;
+    lp->stages = stages;
+    lp->smem = 1024 + static_cast<size_t>(stages) * 2 * tile_bytes +
+               stages * sizeof(TileInfo) + 3 * stages * sizeof(uint64_t);
+    lp->kernel = select_main(D, HG, NB, CG, bf16, fp8);
+    if (lp->kernel == nullptr) return PA_ERR_UNSUPPORTED;
+    kfn = reinterpret_cast<const void*>(lp->kernel);
+  }
+  if (!ensure_smem_attr(kfn, lp->smem)) return PA_ERR_CUDA;
+  const int per_sm = ctas_per_sm(kfn, lp->threads, lp->smem);
   if (per_sm < 1) return PA_ERR_CUDA;
   const int total_ctas = dev->num_sms * per_sm;
   lp->ctas_per_group = total_ctas / lp->groups > 0 ? total_ctas / lp->groups : 1;
@@ -1442,7 +1232,7 @@ pa_status make_plan(int32_t num_seqs, int32_t Hq, int32_t Hkv, int32_t D, int32_
   lp->pack_size = P;
   lp->q_per_entry = Qc;
   lp->rows = Qc > 0 ? num_rows : num_seqs;
-  lp->cols = (P > 1 || Qc > 0) ? 8 * NB * CG : G;
+  lp->cols = umma ? kMaxPackCols : (P > 1 || Qc > 0) ? 8 * NB * CG : G;
   // entries: at most num_seqs / 2 packs (pairs), then the sequences; or at
   // most one chunk per query row
   const int64_t max_packs = P > 1 ? num_seqs / 2 : 0;
@@ -1539,20 +1329,32 @@ extern "C" pa_status pa_decode_shared_prefix_workspace_bytes(
 
 namespace {
 
-// Shared by the 16-bit and the fp8 entry points.  elem_bytes is 1 for E4M3
-// codes; then q_dtype is the query's type and k_scale / v_scale are set.
-pa_status launch_decode(void* out, pa_dtype out_dtype, const void* query, pa_dtype q_dtype,
-                        const void* key_cache, const void* value_cache, int elem_bytes,
-                        const float* k_scale, const float* v_scale,
-                        const int32_t* block_tables, int32_t block_table_stride,
-                        const int32_t* seq_lens, int32_t num_seqs, int32_t max_seq_len,
-                        int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
-                        int32_t num_blocks, int32_t block_size, float scale,
-                        int32_t partition_size, const int32_t* shared_blocks, void* workspace,
-                        size_t workspace_bytes, int32_t* device_error_flag, pa_stream_t stream,
-                        const pa_cache_strides* cache_strides = nullptr,
-                        const int32_t* q_start = nullptr, int32_t num_rows = 0,
-                        int32_t max_q_len = 0) {
+// Everything one decode call launches with: the launch shape, the kernel
+// parameters and the K/V tensor maps.
+struct DecodeSetup {
+  LaunchPlan lp;
+  DecodeParams p;
+  CUtensorMap tmK, tmV;
+  CUtensorMap tmQ;  // the tensor-memory kernel's query rows
+};
+
+// Shared by the 16-bit and the fp8 entry points: validates the arguments,
+// chooses the launch shape and fills *su.  Returns PA_OK with su->p.num_seqs
+// == 0 when there is nothing to do.  elem_bytes is 1 for E4M3 codes; then
+// q_dtype is the query's type and k_scale / v_scale are set.
+pa_status setup_decode(void* out, pa_dtype out_dtype, const void* query, pa_dtype q_dtype,
+                       const void* key_cache, const void* value_cache, int elem_bytes,
+                       const float* k_scale, const float* v_scale,
+                       const int32_t* block_tables, int32_t block_table_stride,
+                       const int32_t* seq_lens, int32_t num_seqs, int32_t max_seq_len,
+                       int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                       int32_t num_blocks, int32_t block_size, float scale,
+                       int32_t partition_size, const int32_t* shared_blocks, void* workspace,
+                       size_t workspace_bytes, int32_t* device_error_flag, DecodeSetup* su,
+                       const pa_cache_strides* cache_strides = nullptr,
+                       const int32_t* q_start = nullptr, int32_t num_rows = 0,
+                       int32_t max_q_len = 0) {
+  std::memset(&su->p, 0, sizeof(su->p));
   if (num_seqs < 0 || num_rows < 0) return PA_ERR_INVALID_ARG;
   if (num_seqs == 0 || (q_start != nullptr && num_rows == 0)) return PA_OK;
   if (q_start != nullptr && (max_q_len <= 0 || !aligned(q_start, 4))) return PA_ERR_INVALID_ARG;
@@ -1565,7 +1367,8 @@ pa_status launch_decode(void* out, pa_dtype out_dtype, const void* query, pa_dty
   if (out_dtype != PA_F16 && out_dtype != PA_BF16 && out_dtype != PA_F32)
     return PA_ERR_INVALID_ARG;
   if (num_blocks <= 0 || !(scale == scale)) return PA_ERR_INVALID_ARG;
-  LaunchPlan lp;
+  LaunchPlan& lp = su->lp;
+  lp = LaunchPlan();
   if (shared_blocks != nullptr && !aligned(shared_blocks, 4)) return PA_ERR_INVALID_ARG;
   pa_status st = make_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
                            max_seq_len, partition_size, !fp8 && q_dtype == PA_BF16, fp8,
@@ -1596,7 +1399,6 @@ pa_status launch_decode(void* out, pa_dtype out_dtype, const void* query, pa_dty
   }
   const int DCT = fp8 ? 1 : D / 64;           // 128-byte rows per (token, head)
   const uint32_t inner = fp8 ? 128u : 64u;    // elements in one 128-byte row
-  CUtensorMap tmK, tmV;
   int mode = 0;
   {
     // mode 0: dims {row, tokens, d-chunks, heads, blocks}, box {row, TB, DCT, HG, 1}
@@ -1609,21 +1411,32 @@ pa_status launch_decode(void* out, pa_dtype out_dtype, const void* query, pa_dty
                                (uint64_t)block_size, (uint64_t)num_blocks};
     const uint64_t str1[4] = {128, head_b, tok_b, blk_b};
     const uint32_t box1[5] = {inner, 1, 1, (uint32_t)lp.tok_box, 1};
-    if (get_tensor_map(&tmK, key_cache, dims0, str0, box0, elem_bytes) &&
-        get_tensor_map(&tmV, value_cache, dims0, str0, box0, elem_bytes)) {
+    if (get_tensor_map(&su->tmK, key_cache, dims0, str0, box0, elem_bytes) &&
+        get_tensor_map(&su->tmV, value_cache, dims0, str0, box0, elem_bytes)) {
       mode = 0;
     } else if (lp.tok_box * 128 % 1024 == 0 &&
-               get_tensor_map(&tmK, key_cache, dims1, str1, box1, elem_bytes) &&
-               get_tensor_map(&tmV, value_cache, dims1, str1, box1, elem_bytes)) {
+               get_tensor_map(&su->tmK, key_cache, dims1, str1, box1, elem_bytes) &&
+               get_tensor_map(&su->tmV, value_cache, dims1, str1, box1, elem_bytes)) {
       mode = 1;
     } else {
       return PA_ERR_UNSUPPORTED;
     }
   }
+  if (lp.umma) {
+    // the tensor-memory kernel reads one box per (head, d-chunk) layout only
+    if (mode != 0) return PA_ERR_UNSUPPORTED;
+    // query rows [rows][Hq][D] as {64 elements, 2 d-chunks, Hq, rows}; a box
+    // is 64 elements of G heads of 32 / G rows: 32 rows of 128 bytes
+    const int G = num_q_heads / num_kv_heads;
+    const uint64_t qd[5] = {64, 2, (uint64_t)num_q_heads, (uint64_t)lp.rows, 1};
+    const uint64_t qs[4] = {128, 256, (uint64_t)num_q_heads * 256,
+                            (uint64_t)lp.rows * num_q_heads * 256};
+    const uint32_t qb[5] = {64, 1, (uint32_t)G, (uint32_t)(32 / G), 1};
+    if (!get_tensor_map(&su->tmQ, query, qd, qs, qb, 2, 4)) return PA_ERR_UNSUPPORTED;
+  }
 
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  DecodeParams p;
-  std::memset(&p, 0, sizeof(p));
+  DecodeParams& p = su->p;
   p.out = out;
   p.query = static_cast<const uint16_t*>(query);
   p.block_tables = block_tables;
@@ -1677,29 +1490,64 @@ pa_status launch_decode(void* out, pa_dtype out_dtype, const void* query, pa_dty
   p.k_scale = k_scale;
   p.v_scale = v_scale;
   p.q_bf16 = q_dtype == PA_BF16 ? 1 : 0;
+  p.out_vec16 = aligned(out, 16) ? 1 : 0;
+  return PA_OK;
+}
 
-  // All three launches use programmatic dependent launch: each may start while
-  // its predecessor runs and waits (griddepcontrol.wait) before touching data.
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (PdlLaunch(s, dim3(1), dim3(kPlanThreads))(pa_plan_kernel, p) != cudaSuccess)
+// Launches a prepared call on `s`: the plan kernel (unless the plan was
+// computed on the host, su.p.host_plan set), the main kernel and, when some
+// output row has partials to merge, the combine.  All launches use
+// programmatic dependent launch: each may start while its predecessor runs and
+// waits (griddepcontrol.wait) before touching data.
+pa_status launch_setup(const DecodeSetup& su, cudaStream_t s, bool run_combine = true) {
+  const LaunchPlan& lp = su.lp;
+  const DecodeParams& p = su.p;
+  if (p.host_plan == nullptr &&
+      PdlLaunch(s, dim3(1), dim3(kPlanThreads))(pa_plan_kernel, p) != cudaSuccess)
     return PA_ERR_CUDA;
-  if (PdlLaunch(s, dim3(lp.ctas_per_group, lp.groups), dim3(lp.threads), lp.smem)(
-          lp.kernel, tmK, tmV, p) != cudaSuccess)
-    return PA_ERR_CUDA;
+  PdlLaunch main_launch(s, dim3(lp.ctas_per_group, lp.groups), dim3(lp.threads), lp.smem);
+  const cudaError_t e2 = lp.umma ? main_launch(lp.ukernel, su.tmK, su.tmV, su.tmQ, p)
+                                 : main_launch(lp.kernel, su.tmK, su.tmV, p);
+  if (e2 != cudaSuccess) return PA_ERR_CUDA;
+  if (!run_combine) return PA_OK;
+  const int D = lp.head_dim;
   cudaError_t e3;
   if (lp.many_partials) {
-    PdlLaunch combine(s, dim3(static_cast<unsigned>(lp.rows), num_q_heads),
+    PdlLaunch combine(s, dim3(static_cast<unsigned>(lp.rows), p.num_q_heads),
                       dim3(kCombineWarps * 32));
     e3 = D == 128 ? combine(pa_combine_wide_kernel<128>, p)
                   : combine(pa_combine_wide_kernel<64>, p);
   } else {
     PdlLaunch combine(s, dim3(static_cast<unsigned>(lp.rows),
-                           (num_q_heads + kCombineWarps - 1) / kCombineWarps),
+                           (p.num_q_heads + kCombineWarps - 1) / kCombineWarps),
                       dim3(kCombineWarps * 32));
     e3 = D == 128 ? combine(pa_combine_narrow_kernel<128>, p)
                   : combine(pa_combine_narrow_kernel<64>, p);
   }
   return e3 == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+pa_status launch_decode(void* out, pa_dtype out_dtype, const void* query, pa_dtype q_dtype,
+                        const void* key_cache, const void* value_cache, int elem_bytes,
+                        const float* k_scale, const float* v_scale,
+                        const int32_t* block_tables, int32_t block_table_stride,
+                        const int32_t* seq_lens, int32_t num_seqs, int32_t max_seq_len,
+                        int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                        int32_t num_blocks, int32_t block_size, float scale,
+                        int32_t partition_size, const int32_t* shared_blocks, void* workspace,
+                        size_t workspace_bytes, int32_t* device_error_flag, pa_stream_t stream,
+                        const pa_cache_strides* cache_strides = nullptr,
+                        const int32_t* q_start = nullptr, int32_t num_rows = 0,
+                        int32_t max_q_len = 0) {
+  DecodeSetup su;
+  const pa_status st = setup_decode(
+      out, out_dtype, query, q_dtype, key_cache, value_cache, elem_bytes, k_scale, v_scale,
+      block_tables, block_table_stride, seq_lens, num_seqs, max_seq_len, num_q_heads,
+      num_kv_heads, head_dim, num_blocks, block_size, scale, partition_size, shared_blocks,
+      workspace, workspace_bytes, device_error_flag, &su, cache_strides, q_start, num_rows,
+      max_q_len);
+  if (st != PA_OK || su.p.num_seqs == 0) return st;
+  return launch_setup(su, reinterpret_cast<cudaStream_t>(stream));
 }
 
 }  // namespace
@@ -1786,6 +1634,392 @@ extern "C" pa_status pa_decode_attention_shared_prefix(
 }
 
 // ===========================================================================
+// Plans computed on the host.  The plan kernel reads the lengths on the
+// device; a serving step has them on the host already, so the same
+// bookkeeping can be done there and shipped with the step's other inputs,
+// and the decode then starts with the main kernel.  Plain decode only (one
+// query token per sequence, no packs).  Buffer layout (int32 words, 256-byte
+// aligned sections): the header (kPlanHeaderWords), then tile prefix sums
+// [B + 1], segment prefix sums [B + 1], start entry [C] and first segment
+// index [C] of each CTA.
+// ===========================================================================
+namespace {
+
+struct PlanOffsets {
+  size_t tiles, segs, start, firstk, total;
+};
+
+PlanOffsets plan_offsets(int64_t B, int64_t C) {
+  auto words = [](int64_t n) { return align_up(static_cast<size_t>(n) * 4, 256); };
+  PlanOffsets o;
+  o.tiles = 256;
+  o.segs = o.tiles + words(B + 1);
+  o.start = o.segs + words(B + 1);
+  o.firstk = o.start + words(C);
+  o.total = o.firstk + words(C);
+  return o;
+}
+
+// The plan kernel's bookkeeping for a plain decode, by walking each
+// sequence's cut points in order: the tiles of all sequences laid end to end
+// (tiles[b] = tiles before sequence b), cut wherever a partition starts
+// (every tpp tiles from a sequence's first tile) or a CTA's share starts
+// (lo(c) = floor(c N / C)); seg_base[b] = segments before sequence b;
+// start_seq[c], first_k[c] = the sequence holding lo(c) and the index of the
+// segment starting there.  Lengths are clamped to [0, max_seq_len].  Returns
+// false if the tile count does not fit in int32.
+bool split_walk(const int32_t* lens, int32_t B, int32_t max_seq_len, int32_t tpp, int32_t C,
+                int32_t* tiles, int32_t* seg_base, int32_t* start_seq, int32_t* first_k,
+                int32_t* total_segs, bool* split) {
+  int64_t N = 0;
+  for (int32_t b = 0; b < B; ++b) {
+    tiles[b] = static_cast<int32_t>(N);
+    const int32_t L = lens[b] < 0 ? 0 : (lens[b] > max_seq_len ? max_seq_len : lens[b]);
+    N += (static_cast<int64_t>(L) + kTile - 1) / kTile;
+    if (N > INT_MAX / 2) return false;
+  }
+  tiles[B] = static_cast<int32_t>(N);
+  for (int32_t c = 0; c < C; ++c) start_seq[c] = first_k[c] = 0;
+  *split = false;
+  int64_t seg = 0;
+  for (int32_t b = 0; b < B; ++b) {
+    seg_base[b] = static_cast<int32_t>(seg);
+    const int64_t t0 = tiles[b], t1 = tiles[b + 1];
+    if (t1 <= t0) continue;
+    int64_t c = (t0 * C + N - 1) / N;  // first CTA whose share starts at or after t0
+    int64_t part = t0;                 // next partition start
+    int32_t count = 0;
+    int64_t last = -1;
+    while (true) {
+      const int64_t lo_c = c * N / C;
+      const int64_t cta_pt = (c < C && lo_c < t1) ? lo_c : INT64_MAX;
+      const int64_t part_pt = part < t1 ? part : INT64_MAX;
+      if (cta_pt == INT64_MAX && part_pt == INT64_MAX) break;
+      if (cta_pt <= part_pt) {
+        const int32_t idx = (cta_pt == last) ? count - 1 : count;
+        if (cta_pt != last) {
+          ++count;
+          last = cta_pt;
+        }
+        start_seq[c] = b;
+        first_k[c] = idx;
+        ++c;
+      } else {
+        if (part_pt != last) {
+          ++count;
+          last = part_pt;
+        }
+        part = (tpp == INT_MAX) ? INT64_MAX : part + tpp;
+      }
+    }
+    seg += count;
+    if (count > 1) *split = true;
+  }
+  seg_base[B] = static_cast<int32_t>(seg);
+  *total_segs = static_cast<int32_t>(seg);
+  return true;
+}
+
+// Writes a plan for launch shape lp into `buf` (host, plan_offsets().total
+// bytes).  *needs_combine: some sequence has partials to merge.
+pa_status write_plan(const LaunchPlan& lp, const int32_t* lens, int32_t B, int32_t max_seq_len,
+                     uint8_t* buf, bool* needs_combine) {
+  const int32_t C = lp.ctas_per_group;
+  const PlanOffsets o = plan_offsets(B, C);
+  int32_t* h = reinterpret_cast<int32_t*>(buf);
+  for (int32_t b = 0; b < B; ++b)
+    if (lens[b] < 0 || lens[b] > max_seq_len) return PA_ERR_INVALID_ARG;
+  int32_t segs = 0;
+  bool split = false;
+  if (!split_walk(lens, B, max_seq_len, lp.tiles_per_part, C,
+                  reinterpret_cast<int32_t*>(buf + o.tiles), reinterpret_cast<int32_t*>(buf + o.segs),
+                  reinterpret_cast<int32_t*>(buf + o.start),
+                  reinterpret_cast<int32_t*>(buf + o.firstk), &segs, &split))
+    return PA_ERR_UNSUPPORTED;
+  if (segs > lp.nseg_cap) return PA_ERR_UNSUPPORTED;  // cannot happen: nseg_cap bounds it
+  std::memset(h, 0, kPlanHeaderWords * sizeof(int32_t));
+  h[0] = kPlanMagic;
+  h[1] = B;
+  h[2] = C;
+  h[3] = lp.tiles_per_part;
+  h[4] = reinterpret_cast<const int32_t*>(buf + o.tiles)[B];
+  h[5] = segs;
+  h[6] = split ? 1 : 0;
+  *needs_combine = split;
+  return PA_OK;
+}
+
+// Points a prepared call at a plan in device memory.
+void use_device_plan(DecodeSetup* su, const void* plan) {
+  const PlanOffsets o = plan_offsets(su->p.num_seqs, su->lp.ctas_per_group);
+  const uint8_t* d = static_cast<const uint8_t*>(plan);
+  su->p.host_plan = reinterpret_cast<const int32_t*>(d);
+  su->p.plan_tiles = reinterpret_cast<int32_t*>(const_cast<uint8_t*>(d + o.tiles));
+  su->p.seg_base = reinterpret_cast<int32_t*>(const_cast<uint8_t*>(d + o.segs));
+  su->p.start_seq = reinterpret_cast<int32_t*>(const_cast<uint8_t*>(d + o.start));
+  su->p.first_k = reinterpret_cast<int32_t*>(const_cast<uint8_t*>(d + o.firstk));
+}
+
+pa_status plan_shape(int32_t num_seqs, int32_t Hq, int32_t Hkv, int32_t D, int32_t bs,
+                     int32_t max_seq_len, int32_t partition_size, pa_kv_cache_dtype kv,
+                     LaunchPlan* lp) {
+  if (kv != PA_KV_AUTO && kv != PA_KV_FP8_E4M3) return PA_ERR_UNSUPPORTED;
+  if (num_seqs <= 0) return PA_ERR_INVALID_ARG;
+  return make_plan(num_seqs, Hq, Hkv, D, bs, max_seq_len, partition_size, true,
+                   kv == PA_KV_FP8_E4M3, false, lp);
+}
+
+}  // namespace
+
+extern "C" pa_status pa_split_plan(const int32_t* seq_lens, int32_t num_seqs, int32_t max_seq_len,
+                                   int32_t partition_size, int32_t num_ctas, int32_t* tiles,
+                                   int32_t* seg_base, int32_t* start_seq, int32_t* first_k,
+                                   int32_t* num_segments, int32_t* needs_combine) {
+  if (num_seqs <= 0 || max_seq_len < 0 || num_ctas <= 0 || num_ctas > kPlanMaxCtas ||
+      partition_size < 0 || partition_size % kTile != 0)
+    return PA_ERR_INVALID_ARG;
+  if (!seq_lens || !tiles || !seg_base || !start_seq || !first_k || !num_segments ||
+      !needs_combine)
+    return PA_ERR_INVALID_ARG;
+  for (int32_t b = 0; b < num_seqs; ++b)
+    if (seq_lens[b] < 0 || seq_lens[b] > max_seq_len) return PA_ERR_INVALID_ARG;
+  const int32_t tpp = partition_size > 0 ? partition_size / kTile : INT_MAX;
+  bool split = false;
+  if (!split_walk(seq_lens, num_seqs, max_seq_len, tpp, num_ctas, tiles, seg_base, start_seq,
+                  first_k, num_segments, &split))
+    return PA_ERR_UNSUPPORTED;
+  *needs_combine = split ? 1 : 0;
+  return PA_OK;
+}
+
+extern "C" pa_status pa_decode_plan_bytes(int32_t num_seqs, int32_t num_q_heads,
+                                          int32_t num_kv_heads, int32_t head_dim,
+                                          int32_t block_size, int32_t max_seq_len,
+                                          int32_t partition_size,
+                                          pa_kv_cache_dtype kv_cache_dtype, size_t* bytes) {
+  if (bytes == nullptr) return PA_ERR_INVALID_ARG;
+  LaunchPlan lp;
+  const pa_status st = plan_shape(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
+                                  max_seq_len, partition_size, kv_cache_dtype, &lp);
+  if (st != PA_OK) return st;
+  *bytes = plan_offsets(num_seqs, lp.ctas_per_group).total;
+  return PA_OK;
+}
+
+extern "C" pa_status pa_decode_plan(const int32_t* seq_lens, int32_t num_seqs,
+                                    int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                    int32_t block_size, int32_t max_seq_len,
+                                    int32_t partition_size, pa_kv_cache_dtype kv_cache_dtype,
+                                    void* plan, size_t plan_bytes, int32_t* needs_combine) {
+  if (seq_lens == nullptr || plan == nullptr || !aligned(plan, 4)) return PA_ERR_INVALID_ARG;
+  LaunchPlan lp;
+  pa_status st = plan_shape(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
+                            max_seq_len, partition_size, kv_cache_dtype, &lp);
+  if (st != PA_OK) return st;
+  if (plan_bytes < plan_offsets(num_seqs, lp.ctas_per_group).total) return PA_ERR_INVALID_ARG;
+  bool combine = false;
+  st = write_plan(lp, seq_lens, num_seqs, max_seq_len, static_cast<uint8_t*>(plan), &combine);
+  if (st == PA_OK && needs_combine != nullptr) *needs_combine = combine ? 1 : 0;
+  return st;
+}
+
+extern "C" pa_status pa_decode_attention_planned(
+    void* out, pa_dtype out_dtype, const void* query, pa_dtype query_dtype,
+    const void* key_cache, const void* value_cache, pa_kv_cache_dtype kv_cache_dtype,
+    const float* k_scale, const float* v_scale, const int32_t* block_tables,
+    int32_t block_table_stride, const int32_t* seq_lens, int32_t num_seqs, int32_t max_seq_len,
+    int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim, int32_t num_blocks,
+    int32_t block_size, float scale, int32_t partition_size, const void* plan, void* workspace,
+    size_t workspace_bytes, int32_t* device_error_flag, pa_stream_t stream) {
+  if (kv_cache_dtype != PA_KV_AUTO && kv_cache_dtype != PA_KV_FP8_E4M3) return PA_ERR_UNSUPPORTED;
+  if (num_seqs > 0 && (plan == nullptr || !aligned(plan, 256))) return PA_ERR_INVALID_ARG;
+  const bool fp8 = kv_cache_dtype == PA_KV_FP8_E4M3;
+  DecodeSetup su;
+  const pa_status st = setup_decode(
+      out, out_dtype, query, query_dtype, key_cache, value_cache, fp8 ? 1 : 2,
+      fp8 ? k_scale : nullptr, fp8 ? v_scale : nullptr, block_tables, block_table_stride,
+      seq_lens, num_seqs, max_seq_len, num_q_heads, num_kv_heads, head_dim, num_blocks,
+      block_size, scale, partition_size, nullptr, workspace, workspace_bytes, device_error_flag,
+      &su);
+  if (st != PA_OK || su.p.num_seqs == 0) return st;
+  use_device_plan(&su, plan);
+  return launch_setup(su, reinterpret_cast<cudaStream_t>(stream));
+}
+
+// ---------------------------------------------------------------------------
+// One decode step from host buffers.
+// ---------------------------------------------------------------------------
+namespace {
+
+pa_status step_plan(const pa_step_shape* sh, LaunchPlan* lp) {
+  if (sh == nullptr) return PA_ERR_INVALID_ARG;
+  if (sh->dtype != PA_F16 && sh->dtype != PA_BF16) return PA_ERR_UNSUPPORTED;
+  if (sh->out_dtype != PA_F16 && sh->out_dtype != PA_BF16 && sh->out_dtype != PA_F32)
+    return PA_ERR_INVALID_ARG;
+  if (sh->num_blocks <= 0 || sh->table_width <= 0 || sh->max_cow < 0) return PA_ERR_INVALID_ARG;
+  if (sh->block_size > 0 &&
+      sh->table_width < (static_cast<int64_t>(sh->max_seq_len) + sh->block_size - 1) / sh->block_size)
+    return PA_ERR_INVALID_ARG;
+  return plan_shape(sh->num_seqs, sh->num_q_heads, sh->num_kv_heads, sh->head_dim,
+                    sh->block_size, sh->max_seq_len, sh->partition_size, sh->kv_cache_dtype, lp);
+}
+
+}  // namespace
+
+extern "C" pa_status pa_decode_step_layout(const pa_step_shape* shape, pa_step_layout* layout) {
+  if (layout == nullptr) return PA_ERR_INVALID_ARG;
+  LaunchPlan lp;
+  const pa_status st = step_plan(shape, &lp);
+  if (st != PA_OK) return st;
+  const int64_t B = shape->num_seqs, Hq = shape->num_q_heads, Hkv = shape->num_kv_heads,
+                D = shape->head_dim;
+  auto sec = [](int64_t bytes) { return align_up(static_cast<size_t>(bytes), 256); };
+  pa_step_layout L;
+  std::memset(&L, 0, sizeof(L));
+  L.query = 0;
+  L.new_k = L.query + sec(B * Hq * D * 2);
+  L.new_v = L.new_k + sec(B * Hkv * D * 2);
+  L.slot_mapping = L.new_v + sec(B * Hkv * D * 2);
+  L.block_tables = L.slot_mapping + sec(B * 4);
+  L.seq_lens = L.block_tables + sec(B * static_cast<int64_t>(shape->table_width) * 4);
+  L.cow_pairs = L.seq_lens + sec(B * 4);
+  L.plan = L.cow_pairs + sec(static_cast<int64_t>(shape->max_cow) * 8);
+  L.host_bytes = L.plan + plan_offsets(B, lp.ctas_per_group).total;
+  L.out_bytes = static_cast<size_t>(B * Hq * D) * (shape->out_dtype == PA_F32 ? 4 : 2);
+  L.device_bytes = L.host_bytes + sec(static_cast<int64_t>(L.out_bytes)) + lp.total;
+  *layout = L;
+  return PA_OK;
+}
+
+namespace {
+
+// Checks shared by the step's three parts; fills the layout.
+pa_status step_check(const pa_step_shape* shape, const void* device_scratch,
+                     size_t device_scratch_bytes, pa_step_layout* L) {
+  if (shape == nullptr || device_scratch == nullptr) return PA_ERR_INVALID_ARG;
+  const pa_status st = pa_decode_step_layout(shape, L);
+  if (st != PA_OK) return st;
+  if (!aligned(device_scratch, 256) || device_scratch_bytes < L->device_bytes)
+    return PA_ERR_INVALID_ARG;
+  return PA_OK;
+}
+
+}  // namespace
+
+extern "C" pa_status pa_decode_step_upload(const pa_step_shape* shape, void* host_staging,
+                                           void* device_scratch, size_t device_scratch_bytes,
+                                           pa_stream_t stream) {
+  if (host_staging == nullptr || !aligned(host_staging, 16)) return PA_ERR_INVALID_ARG;
+  pa_step_layout L;
+  pa_status st = step_check(shape, device_scratch, device_scratch_bytes, &L);
+  if (st != PA_OK) return st;
+  LaunchPlan lp;
+  st = step_plan(shape, &lp);
+  if (st != PA_OK) return st;
+  uint8_t* h = static_cast<uint8_t*>(host_staging);
+  // the plan, from the lengths the caller wrote, goes out with the inputs
+  bool combine = false;
+  st = write_plan(lp, reinterpret_cast<const int32_t*>(h + L.seq_lens), shape->num_seqs,
+                  shape->max_seq_len, h + L.plan, &combine);
+  if (st != PA_OK) return st;
+  if (cudaMemcpyAsync(device_scratch, h, L.host_bytes, cudaMemcpyHostToDevice,
+                      reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return PA_ERR_CUDA;
+  return PA_OK;
+}
+
+extern "C" pa_status pa_decode_step_run(const pa_step_shape* shape, const void* host_staging,
+                                        int32_t num_cow, void* key_cache, void* value_cache,
+                                        const float* k_scale, const float* v_scale, float scale,
+                                        void* device_scratch, size_t device_scratch_bytes,
+                                        int32_t* device_error_flag, pa_stream_t stream) {
+  if (!host_staging || !key_cache || !value_cache) return PA_ERR_INVALID_ARG;
+  pa_step_layout L;
+  pa_status st = step_check(shape, device_scratch, device_scratch_bytes, &L);
+  if (st != PA_OK) return st;
+  if (num_cow < 0 || num_cow > shape->max_cow) return PA_ERR_INVALID_ARG;
+  const bool fp8 = shape->kv_cache_dtype == PA_KV_FP8_E4M3;
+  if (fp8 && (!k_scale || !v_scale)) return PA_ERR_INVALID_ARG;
+  const int32_t B = shape->num_seqs, Hq = shape->num_q_heads, Hkv = shape->num_kv_heads,
+                D = shape->head_dim;
+  uint8_t* d = static_cast<uint8_t*>(device_scratch);
+  uint8_t* d_out = d + L.host_bytes;
+  uint8_t* d_ws = d_out + align_up(L.out_bytes, 256);
+  const size_t ws_bytes = device_scratch_bytes - (d_ws - d);
+
+  DecodeSetup su;
+  st = setup_decode(d_out, shape->out_dtype, d + L.query, shape->dtype, key_cache, value_cache,
+                    fp8 ? 1 : 2, fp8 ? k_scale : nullptr, fp8 ? v_scale : nullptr,
+                    reinterpret_cast<const int32_t*>(d + L.block_tables), shape->table_width,
+                    reinterpret_cast<const int32_t*>(d + L.seq_lens), B, shape->max_seq_len, Hq,
+                    Hkv, D, shape->num_blocks, shape->block_size, scale, shape->partition_size,
+                    nullptr, d_ws, ws_bytes, device_error_flag, &su);
+  if (st != PA_OK) return st;
+  // the plan pa_decode_step_upload wrote into the staging buffer (its header
+  // must name this shape) is in device_scratch by the time the kernels run
+  const int32_t* hdr =
+      reinterpret_cast<const int32_t*>(static_cast<const uint8_t*>(host_staging) + L.plan);
+  if (hdr[0] != kPlanMagic || hdr[1] != B || hdr[2] != su.lp.ctas_per_group ||
+      hdr[3] != su.lp.tiles_per_part)
+    return PA_ERR_INVALID_ARG;
+  const bool combine = hdr[6] != 0;
+  use_device_plan(&su, d + L.plan);
+
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (num_cow > 0) {
+    void* kc[1] = {key_cache};
+    void* vc[1] = {value_cache};
+    const int64_t block_bytes =
+        static_cast<int64_t>(shape->block_size) * Hkv * D * (fp8 ? 1 : 2);
+    st = pa_copy_blocks(kc, vc, 1, reinterpret_cast<const int32_t*>(d + L.cow_pairs), num_cow,
+                        shape->num_blocks, block_bytes, device_error_flag, stream);
+    if (st != PA_OK) return st;
+  }
+  const int64_t row = static_cast<int64_t>(Hkv) * D;
+  st = pa_reshape_and_cache(d + L.new_k, d + L.new_v, row, row, key_cache, value_cache,
+                            reinterpret_cast<const int32_t*>(d + L.slot_mapping), B,
+                            shape->num_blocks, shape->block_size, Hkv, D, shape->dtype,
+                            shape->kv_cache_dtype, k_scale, v_scale, device_error_flag, stream);
+  if (st != PA_OK) return st;
+  return launch_setup(su, s, combine);
+}
+
+extern "C" pa_status pa_decode_step_download(const pa_step_shape* shape,
+                                             const void* device_scratch,
+                                             size_t device_scratch_bytes, void* host_out,
+                                             pa_stream_t stream) {
+  if (host_out == nullptr) return PA_ERR_INVALID_ARG;
+  pa_step_layout L;
+  const pa_status st = step_check(shape, device_scratch, device_scratch_bytes, &L);
+  if (st != PA_OK) return st;
+  const uint8_t* d_out = static_cast<const uint8_t*>(device_scratch) + L.host_bytes;
+  if (cudaMemcpyAsync(host_out, d_out, L.out_bytes, cudaMemcpyDeviceToHost,
+                      reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return PA_ERR_CUDA;
+  return PA_OK;
+}
+
+extern "C" pa_status pa_decode_step(const pa_step_shape* shape, void* host_staging,
+                                    int32_t num_cow, void* key_cache, void* value_cache,
+                                    const float* k_scale, const float* v_scale, float scale,
+                                    void* device_scratch, size_t device_scratch_bytes,
+                                    void* host_out, int32_t* device_error_flag,
+                                    pa_stream_t stream) {
+  if (!shape || !host_staging || !key_cache || !value_cache || !device_scratch || !host_out)
+    return PA_ERR_INVALID_ARG;
+  // everything the later parts refuse is refused before the first copy
+  if (num_cow < 0 || num_cow > shape->max_cow) return PA_ERR_INVALID_ARG;
+  if (shape->kv_cache_dtype == PA_KV_FP8_E4M3 && (!k_scale || !v_scale)) return PA_ERR_INVALID_ARG;
+  pa_status st = pa_decode_step_upload(shape, host_staging, device_scratch, device_scratch_bytes,
+                                       stream);
+  if (st != PA_OK) return st;
+  st = pa_decode_step_run(shape, host_staging, num_cow, key_cache, value_cache, k_scale, v_scale,
+                          scale, device_scratch, device_scratch_bytes, device_error_flag, stream);
+  if (st != PA_OK) return st;
+  return pa_decode_step_download(shape, device_scratch, device_scratch_bytes, host_out, stream);
+}
+
+// ===========================================================================
 // No-allocation variant: the same launches with the workspace in a static
 // device array of this file instead of caller-provided memory, for callers
 // that may not allocate device memory (see pa_decode_attention_noalloc in the
@@ -1797,19 +2031,51 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[PA_NOALLOC_SCRA
 namespace {
 
 std::mutex g_noalloc_mu;
-void* g_noalloc_addr[64] = {};  // device address of g_noalloc_scratch, per device
+// Device address of g_noalloc_scratch, per device, with the id of the CUDA
+// context it was looked up in: a device reset ends that context, and the next
+// call (in the new context, which has a new id) looks the address up again.
+void* g_noalloc_addr[64] = {};
+unsigned long long g_noalloc_ctx[64] = {};
 
-// Looks the array's address up on the current device the first time; later
-// calls on that device reuse it.
+// Unique id of the calling thread's current context (0 if none or unknown).
+unsigned long long current_context_id() {
+  static PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
+  static PFN_cuCtxGetId_v12000 get_id = nullptr;
+  static bool looked_up = false;
+  if (!looked_up) {
+    looked_up = true;
+    void* f1 = nullptr;
+    void* f2 = nullptr;
+    cudaDriverEntryPointQueryResult q1, q2;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f1, cudaEnableDefault, &q1) == cudaSuccess &&
+        q1 == cudaDriverEntryPointSuccess &&
+        cudaGetDriverEntryPoint("cuCtxGetId", &f2, cudaEnableDefault, &q2) == cudaSuccess &&
+        q2 == cudaDriverEntryPointSuccess) {
+      get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(f1);
+      get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(f2);
+    }
+  }
+  if (get_current == nullptr || get_id == nullptr) return 0;
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr || get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
+
+// Looks the array's address up on the current device the first time in each
+// context; later calls in that context reuse it.
 pa_status noalloc_scratch(void** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return PA_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (g_noalloc_addr[dev] == nullptr) {
+  const unsigned long long ctx = current_context_id();
+  if (g_noalloc_addr[dev] == nullptr || ctx == 0 || g_noalloc_ctx[dev] != ctx) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
       return PA_ERR_CUDA;
     g_noalloc_addr[dev] = p;
+    g_noalloc_ctx[dev] = current_context_id();  // the lookup made the context current
   }
   *out = g_noalloc_addr[dev];
   return PA_OK;

@@ -33,6 +33,7 @@ std::vector<Occupancy> g_occupancy;
 struct TmapEntry {
   const void* base;
   int elem_bytes;
+  int rank;
   uint64_t dims[5];
   uint64_t strides[4];
   uint32_t box[5];
@@ -116,10 +117,11 @@ int ctas_per_sm(const void* func, int threads, size_t smem) {
 }
 
 bool get_tensor_map(CUtensorMap* out, const void* base, const uint64_t dims[5],
-                    const uint64_t strides[4], const uint32_t box[5], int elem_bytes) {
+                    const uint64_t strides[4], const uint32_t box[5], int elem_bytes,
+                    int rank) {
   std::lock_guard<std::mutex> lock(g_mu);
   for (const TmapEntry& e : g_tmaps) {
-    if (e.base == base && e.elem_bytes == elem_bytes &&
+    if (e.base == base && e.elem_bytes == elem_bytes && e.rank == rank &&
         std::memcmp(e.dims, dims, sizeof(e.dims)) == 0 &&
         std::memcmp(e.strides, strides, sizeof(e.strides)) == 0 &&
         std::memcmp(e.box, box, sizeof(e.box)) == 0) {
@@ -130,6 +132,7 @@ bool get_tensor_map(CUtensorMap* out, const void* base, const uint64_t dims[5],
   TmapEntry e;
   e.base = base;
   e.elem_bytes = elem_bytes;
+  e.rank = rank;
   std::memcpy(e.dims, dims, sizeof(e.dims));
   std::memcpy(e.strides, strides, sizeof(e.strides));
   std::memcpy(e.box, box, sizeof(e.box));
@@ -148,7 +151,7 @@ bool get_tensor_map(CUtensorMap* out, const void* base, const uint64_t dims[5],
     const CUresult r = enc(&e.map,
                            elem_bytes == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
                                            : CU_TENSOR_MAP_DATA_TYPE_UINT16,
-                           5, const_cast<void*>(base),
+                           static_cast<cuuint32_t>(rank), const_cast<void*>(base),
                            gdims, gstr, gbox, elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE,
                            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);

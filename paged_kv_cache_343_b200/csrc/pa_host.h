@@ -35,11 +35,13 @@ inline bool aligned(const void* p, size_t a) {
   return (reinterpret_cast<uintptr_t>(p) % a) == 0;
 }
 
-// 5-D tiled tensor map with 128-byte swizzle over `base`, elements of
-// `elem_bytes` (1 or 2) bytes.  dims: innermost first; strides: bytes of dims
-// 1..4; box: elements per dim.  Returns false if the driver rejects it.
+// Tiled tensor map of `rank` (4 or 5) dimensions with 128-byte swizzle over
+// `base`, elements of `elem_bytes` (1 or 2) bytes.  dims: innermost first;
+// strides: bytes of dims 1..rank-1; box: elements per dim.  Returns false if
+// the driver rejects it.
 bool get_tensor_map(CUtensorMap* out, const void* base, const uint64_t dims[5],
-                    const uint64_t strides[4], const uint32_t box[5], int elem_bytes = 2);
+                    const uint64_t strides[4], const uint32_t box[5], int elem_bytes = 2,
+                    int rank = 5);
 
 // Launches kernels with programmatic dependent launch on `stream`: the kernel
 // may start while the previous kernel on the stream finishes and must call

@@ -31,6 +31,48 @@ int main(void) {
   CHECK(pa_stream_read((const void*)(uintptr_t)4096, 100, (uint32_t*)(uintptr_t)4096, 4, NULL) ==
         PA_ERR_INVALID_ARG);
 
+  /* the decode step from host buffers: refusals made before any device work */
+  {
+    pa_step_shape sh;
+    memset(&sh, 0, sizeof(sh));
+    sh.num_seqs = 2; sh.num_q_heads = 4; sh.num_kv_heads = 2; sh.head_dim = 64;
+    sh.num_blocks = 8; sh.block_size = 16; sh.table_width = 4; sh.max_seq_len = 64;
+    sh.dtype = PA_F16; sh.out_dtype = PA_F16; sh.kv_cache_dtype = PA_KV_AUTO;
+    char host[64];
+    pa_step_layout lay;
+    CHECK(pa_decode_step_layout(NULL, &lay) == PA_ERR_INVALID_ARG);
+    CHECK(pa_decode_step_layout(&sh, NULL) == PA_ERR_INVALID_ARG);
+    CHECK(pa_decode_step(NULL, host, 0, host, host, NULL, NULL, 0.125f, host, 64, host, NULL,
+                         NULL) == PA_ERR_INVALID_ARG);
+    CHECK(pa_decode_step(&sh, NULL, 0, host, host, NULL, NULL, 0.125f, host, 64, host, NULL,
+                         NULL) == PA_ERR_INVALID_ARG);
+    CHECK(pa_decode_step(&sh, host, 0, host, host, NULL, NULL, 0.125f, host, 64, NULL, NULL,
+                         NULL) == PA_ERR_INVALID_ARG);
+    sh.table_width = 3; /* below ceil(64 / 16) */
+    CHECK(pa_decode_step_layout(&sh, &lay) == PA_ERR_INVALID_ARG);
+    sh.table_width = 4;
+    sh.head_dim = 96; /* not a built head size */
+    CHECK(pa_decode_step_layout(&sh, &lay) == PA_ERR_UNSUPPORTED);
+    sh.head_dim = 64;
+    sh.dtype = PA_F32; /* the query and new rows are 16-bit */
+    CHECK(pa_decode_step_layout(&sh, &lay) == PA_ERR_UNSUPPORTED);
+  }
+
+  /* the split plan on the host: 4 sequences over 7 CTAs */
+  {
+    const int32_t lens4[4] = {5, 40, 0, 100};
+    int32_t tiles[5], segs[5], start[7], firstk[7], nseg = -1, comb = -1;
+    CHECK(pa_split_plan(lens4, 4, 128, 0, 7, tiles, segs, start, firstk, &nseg, &comb) == PA_OK);
+    CHECK(tiles[0] == 0 && tiles[1] == 1 && tiles[2] == 4 && tiles[3] == 4 && tiles[4] == 11);
+    CHECK(segs[4] == 7 && nseg == 7 && comb == 1);
+    CHECK(start[2] == 1 && firstk[2] == 1 && start[6] == 3 && firstk[6] == 3);
+    CHECK(pa_split_plan(lens4, 4, 64, 0, 7, tiles, segs, start, firstk, &nseg, &comb) ==
+          PA_ERR_INVALID_ARG); /* a length above max_seq_len */
+    char plan[64];
+    CHECK(pa_decode_plan(NULL, 4, 4, 2, 64, 16, 128, 0, PA_KV_AUTO, plan, 64, NULL) ==
+          PA_ERR_INVALID_ARG);
+  }
+
   /* block manager: parallel sampling with copy-on-write */
   pa_block_manager* bm = NULL;
   CHECK(pa_bm_create(16, 4, NULL, &bm) == PA_OK && bm != NULL);

@@ -206,6 +206,40 @@ def test_binding_refuses_unsupported_dtypes(pa):
                             16, 0.1)
 
 
+def test_noalloc_binding_refuses_before_any_library_call(pa):
+    """decode_attention_noalloc makes decode_attention's checks (CPU tensors:
+    a refusal here is raised before any pointer reaches the library): a uint8
+    code pool under a 16-bit query, a query of another 16-bit type, K and V of
+    different strides, a strided half of an interleaved pool (the entry point
+    has no strided form), 64-bit tables or lengths, a non-contiguous query."""
+    import torch
+    q = torch.zeros(2, 8, 128, dtype=torch.bfloat16)
+    out = torch.empty_like(q)
+    k = torch.zeros(4, 16, 2, 128, dtype=torch.bfloat16)
+    tables = torch.zeros(2, 8, dtype=torch.int32)
+    lens = torch.ones(2, dtype=torch.int32)
+    f = pa.decode_attention_noalloc
+    codes = torch.zeros(4, 16, 2, 128, dtype=torch.uint8)
+    with pytest.raises(ValueError):
+        f(out, q, codes, codes, tables, lens, 16, 0.1)
+    with pytest.raises(ValueError):
+        f(out, q, k.half(), k.half(), tables, lens, 16, 0.1)
+    kv = torch.zeros(4, 2, 16, 2, 128, dtype=torch.bfloat16)  # per-block interleaved K/V
+    with pytest.raises(ValueError, match="contiguous"):
+        f(out, q, kv[:, 0], kv[:, 1], tables, lens, 16, 0.1)
+    with pytest.raises(ValueError):
+        f(out, q, k, k.transpose(1, 2).contiguous().transpose(1, 2), tables, lens, 16, 0.1)
+    with pytest.raises(ValueError):
+        f(out, q, k, k, tables.long(), lens, 16, 0.1)
+    with pytest.raises(ValueError):
+        f(out, q, k, k, tables, lens.long(), 16, 0.1)
+    qt = torch.zeros(8, 2, 128, dtype=torch.bfloat16).transpose(0, 1)
+    with pytest.raises(ValueError):
+        f(torch.empty(2, 8, 128, dtype=torch.bfloat16), qt, k, k, tables, lens, 16, 0.1)
+    with pytest.raises(ValueError, match="unsupported dtype"):
+        f(torch.empty(q.shape, dtype=torch.float64), q, k, k, tables, lens, 16, 0.1)
+
+
 def _sampling_trace(bm, seed, prompts=3, samples=4, prompt_len=10):
     """Prompts forked into samples (parallel sampling), as both managers see it."""
     sid = 0

@@ -35,6 +35,30 @@ def test_reshape_and_cache_workloads(pa, orc, name):
     assert int(flag.item()) == 0
 
 
+@pytest.mark.parametrize("bs", [128, 256])
+def test_reshape_and_copy_large_blocks(pa, orc, bs):
+    """Blocks of 128 and 256 tokens (512 KiB per pool at 8 KV heads of 128):
+    new rows land bit-exact, and copy_blocks copies whole large blocks."""
+    spec = W.WORKLOADS["longtail"].replace(num_seqs=24, block_size=bs, seed=50 + bs)
+    prep = prepare(spec)
+    s = prep.case.spec
+    kc, vc = prep.k_pool.copy(), prep.v_pool.copy()
+    orc.reshape_and_cache(prep.case.new_k, prep.case.new_v, kc, vc, prep.new_slots)
+    nb = kc.shape[0]
+    pairs = np.stack([np.arange(0, nb // 2, 3), np.arange(nb // 2, nb, 3)[:len(range(0, nb // 2, 3))]],
+                     axis=1).astype(np.int32)
+    orc.copy_blocks([kc, vc], pairs, int(np.prod(kc.shape[1:])) * 2)
+    dk, dv = to_dev(prep.k_pool, s.dtype), to_dev(prep.v_pool, s.dtype)
+    flag = _flag()
+    pa.reshape_and_cache(to_dev(prep.case.new_k, s.dtype), to_dev(prep.case.new_v, s.dtype),
+                         dk, dv, to_dev(prep.new_slots), error_flag=flag)
+    pa.copy_blocks([dk], [dv], to_dev(pairs), error_flag=flag)
+    torch.cuda.synchronize()
+    assert np.array_equal(bits_of(dk), kc)
+    assert np.array_equal(bits_of(dv), vc)
+    assert int(flag.item()) == 0
+
+
 def test_reshape_code_example_and_padding(pa, orc):
     # the code example's shapes: pool (2, 64, 32, 8, 128) fp16, 4 rows to slots 0..3,
     # plus padding tokens (slot -1) and rows taken from a wider strided tensor

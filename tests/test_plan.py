@@ -1,0 +1,112 @@
+"""The split plan computed on the host (pa_split_plan; CPU, no GPU).
+
+The decode lays every sequence's 16-token tiles end to end, gives CTA c of C
+the tiles from lo(c) = floor(c N / C), and cuts a sequence wherever a CTA's
+share or a partition starts.  This file restates that definition tile by
+tile in Python (a set of segment starts per sequence) and checks the
+library's walk against it on random batches: the tile and segment prefix
+sums, each CTA's first sequence and segment index, and whether any sequence
+is split (which decides if the combine runs)."""
+import numpy as np
+import pytest
+
+
+@pytest.fixture(scope="module")
+def pa():
+    import importlib.util
+    import os
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    spec = importlib.util.spec_from_file_location(
+        "_pa_build", os.path.join(root, "paged_kv_cache_343_b200", "build.py"))
+    builder = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(builder)
+    builder.build()
+    import paged_kv_cache_343_b200 as pa
+    return pa
+
+
+def brute_plan(lens, max_len, partition_size, C):
+    """Segment starts enumerated tile by tile."""
+    tiles_of = [(min(max(int(L), 0), max_len) + 15) // 16 for L in lens]
+    t = np.concatenate([[0], np.cumsum(tiles_of)]).astype(np.int64)
+    N = int(t[-1])
+    tpp = partition_size // 16 if partition_size else None
+    lo = [c * N // C for c in range(C)]
+    starts = []  # per sequence: sorted segment starts (global tile index)
+    for b in range(len(lens)):
+        t0, t1 = int(t[b]), int(t[b + 1])
+        S = set()
+        for x in range(t0, t1):
+            if x == t0 or (tpp and (x - t0) % tpp == 0) or x in lo:
+                S.add(x)
+        starts.append(sorted(S))
+    seg_base = np.concatenate([[0], np.cumsum([len(S) for S in starts])]).astype(np.int32)
+    start_seq = np.zeros(C, np.int32)
+    first_k = np.zeros(C, np.int32)
+    for c in range(C):
+        if N == 0:
+            continue
+        x = lo[c]
+        b = max(i for i in range(len(lens)) if t[i] <= x and t[i + 1] > x)
+        start_seq[c] = b
+        first_k[c] = sum(1 for s in starts[b] if s < x)
+    return dict(tiles=t.astype(np.int32), seg_base=seg_base, start_seq=start_seq,
+                first_k=first_k, num_segments=int(seg_base[-1]),
+                needs_combine=any(len(S) > 1 for S in starts))
+
+
+CASES = [
+    # lengths, max_seq_len, partition_size, CTAs
+    ([5, 40, 0, 100], 128, 0, 7),
+    ([1, 5, 16, 22], 22, 0, 148),           # more CTAs than tiles: empty shares
+    ([32768] * 8, 32768, 512, 148),         # long context, 512-token partitions
+    ([0, 0, 0], 8, 0, 4),                   # nothing to attend
+    ([16, 16, 16, 16], 16, 16, 2),          # every tile its own partition
+]
+
+
+@pytest.mark.parametrize("lens,max_len,psize,C", CASES)
+def test_split_plan_matches_the_definition(pa, lens, max_len, psize, C):
+    got = pa.split_plan(lens, max_len, psize, C)
+    ref = brute_plan(lens, max_len, psize, C)
+    for k in ("tiles", "seg_base"):
+        assert np.array_equal(got[k], ref[k]), k
+    N = int(ref["tiles"][-1])
+    if N:
+        # CTAs with an empty share never read their entry; compare the others
+        lo = np.array([c * N // C for c in range(C)])
+        hi = np.array([(c + 1) * N // C for c in range(C)])
+        busy = lo < hi
+        assert np.array_equal(got["start_seq"][busy], ref["start_seq"][busy])
+        assert np.array_equal(got["first_k"][busy], ref["first_k"][busy])
+    assert got["num_segments"] == ref["num_segments"]
+    assert got["needs_combine"] == ref["needs_combine"]
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_split_plan_random_batches(pa, seed):
+    rng = np.random.default_rng(seed)
+    B = int(rng.integers(1, 90))
+    max_len = int(rng.integers(1, 3000))
+    lens = rng.integers(0, max_len + 1, B)
+    psize = int(rng.choice([0, 16, 64, 512]))
+    C = int(rng.choice([1, 3, 37, 148, 296]))
+    got = pa.split_plan(lens, max_len, psize, C)
+    ref = brute_plan(lens, max_len, psize, C)
+    assert np.array_equal(got["tiles"], ref["tiles"])
+    assert np.array_equal(got["seg_base"], ref["seg_base"])
+    N = int(ref["tiles"][-1])
+    busy = np.array([c * N // C < (c + 1) * N // C for c in range(C)])
+    assert np.array_equal(got["start_seq"][busy], ref["start_seq"][busy])
+    assert np.array_equal(got["first_k"][busy], ref["first_k"][busy])
+    assert got["needs_combine"] == ref["needs_combine"]
+
+
+def test_split_plan_refuses_bad_arguments(pa):
+    import paged_kv_cache_343_b200 as m
+    with pytest.raises(m.PagedAttnError):      # a length above max_seq_len
+        pa.split_plan([5, 300], 200, 0, 4)
+    with pytest.raises(m.PagedAttnError):      # partitions not in whole tiles
+        pa.split_plan([5, 30], 200, 24, 4)
+    with pytest.raises(m.PagedAttnError):      # no CTA
+        pa.split_plan([5, 30], 200, 0, 0)

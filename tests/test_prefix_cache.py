@@ -66,3 +66,38 @@ def test_uncached_tail_over_shared_blocks_equals_the_full_prompt(pa, orc, L, bs)
                                scale, "bf16")
     assert np.all(np.isfinite(via_shared))
     assert np.array_equal(via_shared, via_own)
+
+
+def test_two_requests_added_in_one_step_share_rows_written_once(pa, orc):
+    """Two requests with one prompt added back to back, before any row is
+    written: the second hits the first's full blocks (a block enters the cache
+    when it is allocated), so the first request's write alone fills the rows
+    both attend; the second writes only its uncached tail.  Freeing the first
+    leaves the shared blocks held by the second, still cached."""
+    L, bs, hq, hkv, d, nb = 45, 8, 4, 2, 64, 32
+    bm = pa.BlockManager(nb, bs)
+    prompt = [int(t) for t in np.random.default_rng(7).integers(0, 5000, L)]
+    assert bm.add_sequence_with_prefix(0, prompt) == 0
+    cached = bm.add_sequence_with_prefix(1, prompt)
+    assert cached == (L // bs) * bs
+    t0, t1 = bm.block_table(0), bm.block_table(1)
+    assert t1[:cached // bs] == t0[:cached // bs] and t1[-1] != t0[-1]
+    k_pool = np.full((nb, bs, hkv, d), W.NAN_BITS["bf16"], np.uint16)
+    v_pool = k_pool.copy()
+    k_rows, v_rows = _rows(L, hkv, d, 1), _rows(L, hkv, d, 2)
+    s0 = np.array([t0[p // bs] * bs + p % bs for p in range(L)], np.int32)
+    s1 = np.array([t1[p // bs] * bs + p % bs for p in range(cached, L)], np.int32)
+    orc.reshape_and_cache(k_rows, v_rows, k_pool, v_pool, s0)
+    orc.reshape_and_cache(k_rows[cached:], v_rows[cached:], k_pool, v_pool, s1)
+    n = L - cached
+    q = W.randn_bits((n, hq, d), "bf16", torch.Generator().manual_seed(3))
+    tables, lens = bm.fill_tables([0, 1], -(-L // bs))
+    qs = np.array([0, n], np.int32)
+    a = orc.decode_multi(q, qs, k_pool, v_pool, tables.numpy()[1:], lens.numpy()[1:], 0.125, "bf16")
+    b = orc.decode_multi(q, qs, k_pool, v_pool, tables.numpy()[:1], lens.numpy()[:1], 0.125, "bf16")
+    assert np.all(np.isfinite(a)) and np.array_equal(a, b)
+    bm.free_sequence(0)
+    for blk in t1[:cached // bs]:
+        assert bm.refcount(blk) == 1
+    assert bm.stats()["cached_blocks"] == cached // bs
+    assert bm.add_sequence_with_prefix(2, prompt) == cached

@@ -167,6 +167,25 @@ def test_decode_strided_matches_oracle(pa, orc, layout, psize):
     assert int(flag.item()) == 0
 
 
+@pytest.mark.parametrize("layout", LAYOUTS)
+def test_decode_strided_256_token_blocks(pa, orc, layout):
+    """256-token blocks in every layout: a tile covers a sixteenth of a block."""
+    prep = prepare(W.WORKLOADS["llama8b"].replace(num_seqs=5, len_lo=100, len_hi=1400,
+                                                  block_size=256, seed=61))
+    s = prep.case.spec
+    pools = Pools(layout, prep.k_pool, prep.v_pool, W.NAN_BITS[s.dtype], torch.bfloat16)
+    ref = orc.decode(prep.case.q, prep.k_pool, prep.v_pool, prep.tables, prep.seq_lens,
+                     W.scale_of(s), s.dtype)
+    q = to_dev(prep.case.q, s.dtype)
+    out = torch.empty(q.shape, dtype=torch.float32, device="cuda")
+    flag = torch.zeros(1, dtype=torch.int32, device="cuda")
+    pa.decode_attention(out, q, pools.k(), pools.v(), to_dev(prep.tables), to_dev(prep.seq_lens),
+                        int(prep.seq_lens.max()), W.scale_of(s), error_flag=flag)
+    torch.cuda.synchronize()
+    assert float(np.max(np.abs(as_f64(out) - ref))) <= TOL_F32
+    assert int(flag.item()) == 0
+
+
 def test_decode_fp8_head_major(pa, orc):
     """E4M3 code pools in the head-major layout (NaN codes outside the tokens)."""
     spec, prep, kc, vc = fp8_case(31, B=5, lo=200, hi=700)

@@ -75,6 +75,23 @@ def test_noalloc_matches_workspace_entry_point_twice(pa, orc, out_dtype):
         assert float(np.max(np.abs(as_f64(got) - oref))) <= max(tol, TOL_STORED if out_dtype is None else tol)
 
 
+def test_noalloc_through_the_binding(pa, orc):
+    """The Python wrapper's path (its checks, then the same C entry point)
+    gives the regular entry point's result on a reduced llama8b batch."""
+    prep = prepare(W.WORKLOADS["llama8b"].replace(num_seqs=5, len_lo=100, len_hi=900, seed=33))
+    a = _args(prep)
+    ref = torch.empty_like(a["query"])
+    pa.decode_attention(ref, **a)
+    got = torch.full_like(ref, float("nan"))
+    pa.decode_attention_noalloc(got, **a)
+    torch.cuda.synchronize()
+    assert float((got.float() - ref.float()).abs().max()) <= TOL_STORED
+    s = prep.case.spec
+    oref = orc.decode(prep.case.q, prep.k_pool, prep.v_pool, prep.tables, prep.seq_lens,
+                      W.scale_of(s), s.dtype, nthreads=4)
+    assert float(np.max(np.abs(as_f64(got) - oref))) <= TOL_STORED
+
+
 def test_noalloc_refuses_shapes_beyond_its_scratch(pa):
     # 4096 sequences of up to 32768 tokens in 16-token partitions needs far more
     # than the static array; the call must refuse before launching anything
