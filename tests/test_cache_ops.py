@@ -39,7 +39,7 @@ def test_reshape_and_cache_workloads(pa, orc, name):
 def test_reshape_and_copy_large_blocks(pa, orc, bs):
     """Blocks of 128 and 256 tokens (512 KiB per pool at 8 KV heads of 128):
     new rows land bit-exact, and copy_blocks copies whole large blocks."""
-    spec = W.WORKLOADS["longtail"].replace(num_seqs=24, block_size=bs, seed=50 + bs)
+    spec = W.WORKLOADS["longtail"].replace(num_seqs=24, new_rows=24, block_size=bs, seed=50 + bs)
     prep = prepare(spec)
     s = prep.case.spec
     kc, vc = prep.k_pool.copy(), prep.v_pool.copy()
