@@ -623,6 +623,20 @@ pa_status pa_decode_attention_noalloc(void* out, pa_dtype out_dtype, const void*
                                       int32_t* device_error_flag, pa_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * pa_set_consumer_wait_limit_ns -- a diagnostic setting, not a step of the
+ * method.  Every pipeline wait in the kernels is bounded: a wait that has not
+ * ended after its limit flags PA_DEVERR_TIMEOUT and the warp stops (nothing
+ * traps).  This sets, for decode calls made after it (process-wide), the
+ * limit of the waits of the warps that consume landed K/V stages in the
+ * warp-level main kernel; 0 restores the default of 2 s.  The loading side
+ * keeps 2 s for its own waits, including its final wait for every copy it
+ * issued, so no copy is in flight when a CTA exits.  A short limit makes a
+ * timeout happen on purpose, to test that it is reported and that the
+ * context stays usable.
+ * ------------------------------------------------------------------------- */
+void pa_set_consumer_wait_limit_ns(uint64_t ns);
+
+/* ---------------------------------------------------------------------------
  * Read-bandwidth ceiling -- a measurement aid, not a step of the method.
  * Decode is limited by reading the cache from memory ([KV] opening section),
  * so its kernels are held against the rate at which this GPU streams reads.

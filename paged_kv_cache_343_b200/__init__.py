@@ -51,7 +51,7 @@ __all__ = [
     "DEVERR_BAD_BLOCK", "DEVERR_BAD_SLOT", "DEVERR_BAD_SEQLEN",
     "DEVERR_TIMEOUT", "DEVERR_BAD_SHARE", "DEVERR_BAD_PLAN", "CacheStrides", "version",
     "stream_read", "decode_plan_bytes", "decode_plan", "decode_attention_planned", "split_plan",
-    "DecodeStep", "StepShape", "StepLayout",
+    "DecodeStep", "StepShape", "StepLayout", "set_consumer_wait_limit_ns",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpagedattn.so")
@@ -197,6 +197,8 @@ def _load() -> ctypes.CDLL:
     lib.pa_decode_step.restype = ctypes.c_int
     lib.pa_decode_step.argtypes = [ctypes.POINTER(StepShape), p, i32, p, p, p, p, ctypes.c_float,
                                    p, sz, p, p, p]
+    lib.pa_set_consumer_wait_limit_ns.restype = None
+    lib.pa_set_consumer_wait_limit_ns.argtypes = [ctypes.c_uint64]
     lib.pa_stream_read.restype = ctypes.c_int
     lib.pa_stream_read.argtypes = [p, i64, p, i32, p]
     lib.pa_bm_create.restype = ctypes.c_int
@@ -819,6 +821,12 @@ def decode_attention_noalloc(out: torch.Tensor, query: torch.Tensor, key_cache: 
         d, nb, bs, float(scale), _dtype_code(query.dtype), int(partition_size),
         _ptr(error_flag), _stream_handle(stream)), "pa_decode_attention_noalloc")
     return out
+
+
+def set_consumer_wait_limit_ns(ns: int) -> None:
+    """Diagnostic: the limit of the consuming warps' waits for the decode calls
+    that follow (0 restores the 2 s default); see the header."""
+    lib.pa_set_consumer_wait_limit_ns(int(ns))
 
 
 def stream_read(buf: torch.Tensor, sink: torch.Tensor,

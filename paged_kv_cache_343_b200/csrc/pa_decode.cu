@@ -26,6 +26,7 @@
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <climits>
 #include <cstring>
 #include <mutex>
@@ -521,7 +522,7 @@ __global__ void __launch_bounds__((HG * CG + 1) * 32, 1)
   const float sl2 = p.scale_log2 * k_scale;
 
   for (int64_t t = lo; t < hi; ++t) {
-    if (!mbar_wait(full_k(stage), phase, p.err)) break;
+    if (!mbar_wait(full_k(stage), phase, p.err, p.consumer_wait_ns)) break;
     const TileInfo ti = info[stage];
     const int ncol = ti.members * G;  // query columns of this tile, per KV head
     if (CG > 1 && col0 >= ncol) {
@@ -596,7 +597,7 @@ __global__ void __launch_bounds__((HG * CG + 1) * 32, 1)
                        : "r"(a));
         }
       }
-      if (!mbar_wait(full_v(stage), phase, p.err)) break;
+      if (!mbar_wait(full_v(stage), phase, p.err, p.consumer_wait_ns)) break;
 #pragma unroll
       for (int tt = 0; tt < 4; ++tt) {
         const int r = r8_v[tt];
@@ -722,7 +723,7 @@ __global__ void __launch_bounds__((HG * CG + 1) * 32, 1)
     }
 
     // ---- O^T[D x 8] += V^T[D x 16 tok] * P^T[16 tok x 8], per n8 block
-    if (!kFP8 && !mbar_wait(full_v(stage), phase, p.err)) break;
+    if (!kFP8 && !mbar_wait(full_v(stage), phase, p.err, p.consumer_wait_ns)) break;
     const bool partial = mask != 0xffffu;
     uint32_t z01 = 0xffffffffu, z23 = 0xffffffffu;
     if (partial) {
@@ -1329,6 +1330,20 @@ extern "C" pa_status pa_decode_shared_prefix_workspace_bytes(
 
 namespace {
 
+std::atomic<uint64_t> g_consumer_wait_ns{kWaitLimitNs};
+
+}  // namespace
+
+uint64_t pa::consumer_wait_limit_ns() {
+  return g_consumer_wait_ns.load(std::memory_order_relaxed);
+}
+
+extern "C" void pa_set_consumer_wait_limit_ns(uint64_t ns) {
+  g_consumer_wait_ns.store(ns == 0 ? kWaitLimitNs : ns, std::memory_order_relaxed);
+}
+
+namespace {
+
 // Everything one decode call launches with: the launch shape, the kernel
 // parameters and the K/V tensor maps.
 struct DecodeSetup {
@@ -1491,6 +1506,7 @@ pa_status setup_decode(void* out, pa_dtype out_dtype, const void* query, pa_dtyp
   p.v_scale = v_scale;
   p.q_bf16 = q_dtype == PA_BF16 ? 1 : 0;
   p.out_vec16 = aligned(out, 16) ? 1 : 0;
+  p.consumer_wait_ns = consumer_wait_limit_ns();
   return PA_OK;
 }
 

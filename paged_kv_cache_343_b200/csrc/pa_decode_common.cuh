@@ -96,7 +96,12 @@ struct DecodeParams {
   // the plan kernel writes them into the workspace.
   const int32_t* host_plan;
   int32_t out_vec16;       // out is 16-byte aligned (vector stores allowed)
+  uint64_t consumer_wait_ns;  // limit of the consumer warps' waits for a landed stage
 };
+
+// Limit of the consumers' waits for the next call's kernels (host side; see
+// pa_set_consumer_wait_limit_ns).
+uint64_t consumer_wait_limit_ns();
 
 // Header of a host-computed plan (int32 words): magic, num_seqs, CTAs per head
 // group, partition length in tiles, total tiles, total segments, whether some

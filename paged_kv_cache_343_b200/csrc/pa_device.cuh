@@ -71,14 +71,40 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking test of the same condition.
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Waits for the phase with the given parity to complete.  Returns false (and
-// flags PA_DEVERR_TIMEOUT) if it has not completed within kWaitLimitNs.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int32_t* err) {
+// flags PA_DEVERR_TIMEOUT) if it has not completed within limit_ns.  try_wait
+// may suspend the thread inside the hardware for a while, so limits under a
+// microsecond (diagnostics) poll with the non-blocking test instead.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int32_t* err,
+                                          uint64_t limit_ns = kWaitLimitNs) {
+  if (limit_ns < 1000) {
+    const uint64_t t0 = global_timer_ns();
+    while (!mbar_test_wait(bar, parity)) {
+      if (global_timer_ns() - t0 >= limit_ns) {
+        flag_error(err, PA_DEVERR_TIMEOUT);
+        return false;
+      }
+    }
+    return true;
+  }
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (global_timer_ns() - t0 > kWaitLimitNs) {
+    if (global_timer_ns() - t0 > limit_ns) {
       flag_error(err, PA_DEVERR_TIMEOUT);
       return false;
     }
