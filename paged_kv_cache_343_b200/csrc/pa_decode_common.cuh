@@ -129,7 +129,7 @@ using UmmaKernel = void (*)(const CUtensorMap, const CUtensorMap, const CUtensor
                             const DecodeParams);
 UmmaKernel select_umma(int HG, bool bf16);
 size_t umma_smem_bytes(int HG, int stages);
-constexpr int kUmmaThreads = 192;
+constexpr int kUmmaThreads = 256;
 
 // ---------------------------------------------------------------------------
 // The producer warp's loop (one elected lane), shared by the decode kernels:

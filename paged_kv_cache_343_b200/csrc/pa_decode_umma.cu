@@ -26,8 +26,13 @@
 // lanes 16..31 of sub-partitions 0 and 1, region r of the columns.
 //
 // Warps: 0, 1, 4, 5 softmax and epilogue (sub-partitions 0 and 1 of regions
-// 0 and 1), 2 producer (TMA: K/V tiles and each entry's query rows), 3 MMA
-// issuer (one thread) and tensor-memory owner.  Every wait is bounded.
+// 0 and 1), 2 producer (TMA: K/V tiles and each entry's query rows), 3 and 6
+// issue the S products of regions 0 and 1, 7 issues every P.V product.  One
+// thread issues a tcgen05.mma about every 60 cycles, while several issuing
+// warps overlap (measured on B200), so the small S products are spread over
+// two issuers and run ahead of the softmax (two S buffers per region), and the
+// P.V products follow it on their own.  Warp 3 owns the tensor memory.  Every
+// wait is bounded.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -42,7 +47,7 @@ namespace pa {
 namespace {
 
 constexpr int kUD = 128;             // head_dim of this kernel
-constexpr int kUThreads = kUmmaThreads;  // 6 warps
+constexpr int kUThreads = kUmmaThreads;  // 8 warps
 constexpr float kLazyLog2 = 8.0f;    // growth of a row maximum that forces a rescale
 constexpr uint32_t kQBlock = 32 * 128;   // 32 query rows of one (head, d-chunk): 4 KiB
 constexpr uint32_t kPBlock = 32 * 32;    // 32 rows of 16 tokens of P, one half: 1 KiB
@@ -65,7 +70,7 @@ __host__ __device__ inline UmmaLayout umma_layout(int HG, int NS) {
   L.info = L.p + 2u * HG * 2u * kPBlock + kPBlock;
   L.bars = L.info + static_cast<uint32_t>(NS) * sizeof(TileInfo);
   L.bars = (L.bars + 7u) & ~7u;
-  const uint32_t nbars = 3u * NS + 13u;
+  const uint32_t nbars = 3u * NS + 19u;
   L.tmem_slot = L.bars + nbars * 8u;
   L.total = L.tmem_slot + 16u;
   return L;
@@ -102,11 +107,11 @@ __global__ void __launch_bounds__(kUThreads, 1)
   const uint32_t barx = bar0 + 8u * (3 * NS);
   auto q_full = [&](int b) { return barx + 8u * b; };
   auto q_free = [&](int b) { return barx + 8u * (2 + b); };
-  auto s_full = [&](int j) { return barx + 8u * (4 + j); };
-  auto s_free = [&](int j) { return barx + 8u * (6 + j); };
-  auto p_full = [&](int j) { return barx + 8u * (8 + j); };
-  auto pv_done = [&](int j) { return barx + 8u * (10 + j); };
-  const uint32_t o_free = barx + 8u * 12;
+  auto p_full = [&](int j) { return barx + 8u * (4 + j); };
+  auto pv_done = [&](int j) { return barx + 8u * (6 + j); };
+  const uint32_t o_free = barx + 8u * 8;
+  auto s_full = [&](int r, int j) { return barx + 8u * (9 + 2 * r + j); };
+  auto s_free = [&](int r, int j) { return barx + 8u * (13 + 2 * r + j); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay.tmem_slot);
   auto q_addr = [&](int qb, int g, int dc) {
     return base + Lay.q + ((static_cast<uint32_t>(qb) * HG + g) * 2u + dc) * kQBlock;
@@ -128,15 +133,17 @@ __global__ void __launch_bounds__(kUThreads, 1)
     for (int s = 0; s < NS; ++s) {
       mbar_init(full_k(s), 1);
       mbar_init(full_v(s), 1);
-      mbar_init(empty(s), 1);  // the MMA thread's commit after the tile's P.V
+      mbar_init(empty(s), 1);  // the P.V issuer's commit after the tile's products
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(q_full(b), 1);
-      mbar_init(q_free(b), 1);
-      mbar_init(s_full(b), 1);
-      mbar_init(s_free(b), NSW);
-      mbar_init(p_full(b), NSW);
-      mbar_init(pv_done(b), 1);
+      mbar_init(q_free(b), R);        // each S issuer's commit
+      mbar_init(p_full(b), NSW);      // every softmax warp's P rows
+      mbar_init(pv_done(b), 1);       // the P.V issuer's commit
+      for (int r = 0; r < 2; ++r) {
+        mbar_init(s_full(r, b), 1);   // S issuer r's commit
+        mbar_init(s_free(r, b), 2);   // region r's two softmax warps
+      }
     }
     mbar_init(o_free, NSW);
     fence_mbar_init();
@@ -195,86 +202,89 @@ __global__ void __launch_bounds__(kUThreads, 1)
         for (int32_t n = last_n > 0 ? last_n - 1 : 0; n <= last_n; ++n)
           if (!mbar_wait(q_full(n & 1), static_cast<uint32_t>(n >> 1) & 1u, p.err)) break;
       }
-    } else if (warp == 3) {
-      // ======================= MMA issuer =======================
+    } else if ((warp == 3 || warp == 6) && (warp == 3 || R == 2)) {
+      // ======================= S issuer of region r =======================
       if (lane == 0) {
+        const int r = warp == 3 ? 0 : 1;
         const uint32_t idS = idesc_f16(kBF16, 64, 16, false, false);
-        const uint32_t idPV = idesc_f16(kBF16, 64, 128, false, true);
         int32_t n_entry = -1;
+        for (int64_t t = lo; t < hi; ++t) {
+          const int64_t u = t - lo;
+          const int s = static_cast<int>(u % NS), j = static_cast<int>(u & 1);
+          if (!mbar_wait(full_k(s), static_cast<uint32_t>((u / NS) & 1), p.err)) break;
+          if (info[s].flags & kNewSeq) {
+            ++n_entry;
+            // the previous entry's query buffer is free once its products finish
+            if (n_entry >= 1) umma_commit(q_free((n_entry - 1) & 1));
+            if (!mbar_wait(q_full(n_entry & 1), static_cast<uint32_t>(n_entry >> 1) & 1u, p.err))
+              break;
+          }
+          if (u >= 2 &&
+              !mbar_wait(s_free(r, j), static_cast<uint32_t>((u - 2) >> 1) & 1u, p.err))
+            break;
+          tc_fence_after();
+          const int qb = n_entry & 1;
+#pragma unroll
+          for (int gg = 0; gg < 2; ++gg) {
+            const int g = 2 * r + gg;
+            const uint32_t d = tmem + (static_cast<uint32_t>(gg * 16) << 16) + kSCol0 +
+                               static_cast<uint32_t>(r) * 32u + static_cast<uint32_t>(j) * 16u;
+#pragma unroll
+            for (int kc = 0; kc < 8; ++kc) {
+              const uint64_t a =
+                  smem_desc(q_addr(qb, g, kc >> 2) + (kc & 3) * 32u, 16u, 1024u, kSwizzle128);
+              const uint64_t b = smem_desc(
+                  k_addr(s) + static_cast<uint32_t>((g * 2 + (kc >> 2)) * TB) * 128u +
+                      (kc & 3) * 32u,
+                  16u, sbo_tok, kSwizzle128);
+              umma_f16_ss(d, a, b, idS, kc > 0);
+            }
+          }
+          umma_commit(s_full(r, j));
+        }
+      }
+    } else if (warp == 7) {
+      // ======================= P.V issuer =======================
+      if (lane == 0) {
+        const uint32_t idPV = idesc_f16(kBF16, 64, 128, false, true);
         uint32_t ofree_par = 0;
         bool first_seg = true;
         int64_t pv_issued = -1;  // local index of the last P.V issued
-        for (int64_t t = lo; t <= hi; ++t) {
-          if (t < hi) {  // S of tile u
-            const int64_t u = t - lo;
-            const int s = static_cast<int>(u % NS), j = static_cast<int>(u & 1);
-            if (!mbar_wait(full_k(s), static_cast<uint32_t>((u / NS) & 1), p.err)) break;
-            const int32_t fl = info[s].flags;
-            if (fl & kNewSeq) {
-              ++n_entry;
-              // the previous entry's query buffer is free once its products finish
-              if (n_entry >= 1) umma_commit(q_free((n_entry - 1) & 1));
-              if (!mbar_wait(q_full(n_entry & 1), static_cast<uint32_t>(n_entry >> 1) & 1u,
-                             p.err))
-                break;
+        for (int64_t t = lo; t < hi; ++t) {
+          const int64_t u = t - lo;
+          const int s = static_cast<int>(u % NS), j = static_cast<int>(u & 1);
+          if (!mbar_wait(p_full(j), static_cast<uint32_t>(u >> 1) & 1u, p.err)) break;
+          const bool seg_start = (info[s].flags & kSegStart) != 0;
+          if (seg_start) {
+            // the previous segment's epilogue has read its accumulator
+            if (!first_seg) {
+              if (!mbar_wait(o_free, ofree_par, p.err)) break;
+              ofree_par ^= 1u;
             }
-            if (u >= 2 && !mbar_wait(s_free(j), static_cast<uint32_t>((u - 2) >> 1) & 1u, p.err))
-              break;
-            tc_fence_after();
-            const int qb = n_entry & 1;
-#pragma unroll
-            for (int g = 0; g < HG; ++g) {
-              const uint32_t d = tmem + (static_cast<uint32_t>((g & 1) * 16) << 16) + kSCol0 +
-                                 static_cast<uint32_t>(g >> 1) * 32u + static_cast<uint32_t>(j) * 16u;
-#pragma unroll
-              for (int kc = 0; kc < 8; ++kc) {
-                const uint64_t a =
-                    smem_desc(q_addr(qb, g, kc >> 2) + (kc & 3) * 32u, 16u, 1024u, kSwizzle128);
-                const uint64_t b = smem_desc(
-                    k_addr(s) + static_cast<uint32_t>((g * 2 + (kc >> 2)) * TB) * 128u +
-                        (kc & 3) * 32u,
-                    16u, sbo_tok, kSwizzle128);
-                umma_f16_ss(d, a, b, idS, kc > 0);
-              }
-            }
-            umma_commit(s_full(j));
+            first_seg = false;
           }
-          if (t > lo) {  // P.V of tile u = t - 1 - lo
-            const int64_t u = t - 1 - lo;
-            const int s = static_cast<int>(u % NS), j = static_cast<int>(u & 1);
-            if (!mbar_wait(p_full(j), static_cast<uint32_t>(u >> 1) & 1u, p.err)) break;
-            const bool seg_start = (info[s].flags & kSegStart) != 0;
-            if (seg_start) {
-              // the previous segment's epilogue has read its accumulator
-              if (!first_seg) {
-                if (!mbar_wait(o_free, ofree_par, p.err)) break;
-                ofree_par ^= 1u;
-              }
-              first_seg = false;
-            }
-            if (!mbar_wait(full_v(s), static_cast<uint32_t>((u / NS) & 1), p.err)) break;
-            tc_fence_after();
+          if (!mbar_wait(full_v(s), static_cast<uint32_t>((u / NS) & 1), p.err)) break;
+          tc_fence_after();
 #pragma unroll
-            for (int g = 0; g < HG; ++g) {
-              const uint32_t d = tmem + (static_cast<uint32_t>((g & 1) * 16) << 16) +
-                                 static_cast<uint32_t>(g >> 1) * 128u;
-              // V[16 tokens x 128]: N = head_dim contiguous (MN-major), d-chunks
-              // TB rows apart, 8-token row groups sbo_tok apart
-              const uint64_t b =
-                  smem_desc(v_addr(s) + static_cast<uint32_t>(g * 2 * TB) * 128u,
-                            static_cast<uint32_t>(TB) * 128u, sbo_tok, kSwizzle128);
+          for (int g = 0; g < HG; ++g) {
+            const uint32_t d = tmem + (static_cast<uint32_t>((g & 1) * 16) << 16) +
+                               static_cast<uint32_t>(g >> 1) * 128u;
+            // V[16 tokens x 128]: N = head_dim contiguous (MN-major), d-chunks
+            // TB rows apart, 8-token row groups sbo_tok apart
+            const uint64_t b =
+                smem_desc(v_addr(s) + static_cast<uint32_t>(g * 2 * TB) * 128u,
+                          static_cast<uint32_t>(TB) * 128u, sbo_tok, kSwizzle128);
 #pragma unroll
-              for (int part = 0; part < 2; ++part) {
-                // P[64 x 16], K-major without swizzle: 8-row core matrices of
-                // 16 bytes, tokens 8..15 128 bytes on, row groups 256 apart
-                const uint64_t a = smem_desc(p_addr(j, g, part), 128u, 256u, kSwizzleNone);
-                umma_f16_ss(d, a, b, idPV, !(seg_start && part == 0));
-              }
+            for (int part = 0; part < 2; ++part) {
+              // P[64 x 16], K-major without swizzle: 8-row core matrices of
+              // 16 bytes, tokens 8..15 128 bytes on, row groups 256 apart
+              const uint64_t a = smem_desc(p_addr(j, g, part), 128u, 256u, kSwizzleNone);
+              umma_f16_ss(d, a, b, idPV, !(seg_start && part == 0));
             }
-            umma_commit(empty(s));
-            umma_commit(pv_done(j));
-            pv_issued = u;
           }
+          umma_commit(empty(s));
+          umma_commit(pv_done(j));
+          pv_issued = u;
         }
         // the last products have finished before tensor memory is released
         if (pv_issued >= 0)
@@ -299,13 +309,13 @@ __global__ void __launch_bounds__(kUThreads, 1)
         const uint32_t ph = static_cast<uint32_t>((u / NS) & 1);
         if (!warp_wait(full_k(s), ph, p.err)) break;
         const TileInfo ti = info[s];
-        if (!warp_wait(s_full(j), static_cast<uint32_t>(u >> 1) & 1u, p.err)) break;
+        if (!warp_wait(s_full(region, j), static_cast<uint32_t>(u >> 1) & 1u, p.err)) break;
         tc_fence_after();
         uint32_t sr[16];
         tmem_ld16(tS + static_cast<uint32_t>(j) * 16u, sr);
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(s_free(j));
+        if (lane == 0) mbar_arrive(s_free(region, j));
 
         if (ti.flags & kSegStart) {
           m_run = -INFINITY;
