@@ -38,7 +38,7 @@ import pa_workloads as W  # noqa: E402
 METRIC = "paged decode attention KV-read GB/s (% of B200 HBM peak); decode tokens/s"
 PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "decode_main_llama8b.md")
 KERNEL_SOURCES = [os.path.join(ROOT, "paged_kv_cache_343_b200", "csrc", f)
-                  for f in ("pa_decode.cu", "pa_device.cuh")]
+                  for f in ("pa_decode.cu", "pa_decode_common.cuh", "pa_device.cuh")]
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 
 

@@ -1177,11 +1177,11 @@ pa_status make_plan(int32_t num_seqs, int32_t Hq, int32_t Hkv, int32_t D, int32_
   if ((HG * DCT * TB * 128) % 1024 != 0) return PA_ERR_UNSUPPORTED;
   // Entries of many query columns (packs, query chunks) with 16-bit caches and
   // head_dim 128 run on the tensor-memory kernel when its shape rules hold: the
-  // query columns of an entry fill whole 32-row loads (G divides 32), two or
-  // four KV heads per CTA, 8- or 16-token boxes.
-  const bool umma = (P > 1 || Qc > 0) && !fp8 && D == 128 && 32 % G == 0 && TB >= 8 &&
-                    Hkv % 2 == 0;
-  if (umma) HG = Hkv % 4 == 0 ? 4 : 2;
+  // query columns of an entry fill whole 32-row loads (G divides 32), four KV
+  // heads per CTA, 16-token boxes (blocks of 16 tokens or more).
+  const bool umma = (P > 1 || Qc > 0) && !fp8 && D == 128 && 32 % G == 0 && TB == kTile &&
+                    Hkv % 4 == 0;
+  if (umma) HG = 4;
   lp->HG = HG;
   lp->head_dim = D;
   lp->groups = Hkv / HG;
@@ -1195,12 +1195,11 @@ pa_status make_plan(int32_t num_seqs, int32_t Hq, int32_t Hkv, int32_t D, int32_
   const void* kfn = nullptr;
   if (umma) {
     int stages = 6;
-    while (stages > 2 &&
-           umma_smem_bytes(HG, stages) > static_cast<size_t>(dev->max_smem_optin))
+    while (stages > 2 && umma_smem_bytes(stages) > static_cast<size_t>(dev->max_smem_optin))
       --stages;
     lp->stages = stages;
-    lp->smem = umma_smem_bytes(HG, stages);
-    lp->ukernel = select_umma(HG, bf16);
+    lp->smem = umma_smem_bytes(stages);
+    lp->ukernel = select_umma(bf16);
     if (lp->ukernel == nullptr) return PA_ERR_UNSUPPORTED;
     kfn = reinterpret_cast<const void*>(lp->ukernel);
   } else {
@@ -1415,7 +1414,18 @@ pa_status setup_decode(void* out, pa_dtype out_dtype, const void* query, pa_dtyp
   const int DCT = fp8 ? 1 : D / 64;           // 128-byte rows per (token, head)
   const uint32_t inner = fp8 ? 128u : 64u;    // elements in one 128-byte row
   int mode = 0;
-  {
+  if (lp.umma) {
+    // mode 2: dims {row, tokens, heads, d-chunks, blocks}, box {row, 16, HG, 2, 1}:
+    // the rows of one d-chunk of all HG heads are contiguous in the stage
+    const uint64_t dims2[5] = {inner, (uint64_t)block_size, (uint64_t)num_kv_heads,
+                               (uint64_t)DCT, (uint64_t)num_blocks};
+    const uint64_t str2[4] = {tok_b, head_b, 128, blk_b};
+    const uint32_t box2[5] = {inner, (uint32_t)lp.tok_box, (uint32_t)HG, (uint32_t)DCT, 1};
+    if (!get_tensor_map(&su->tmK, key_cache, dims2, str2, box2, elem_bytes) ||
+        !get_tensor_map(&su->tmV, value_cache, dims2, str2, box2, elem_bytes))
+      return PA_ERR_UNSUPPORTED;
+    mode = 2;
+  } else {
     // mode 0: dims {row, tokens, d-chunks, heads, blocks}, box {row, TB, DCT, HG, 1}
     const uint64_t dims0[5] = {inner, (uint64_t)block_size, (uint64_t)DCT,
                                (uint64_t)num_kv_heads, (uint64_t)num_blocks};
@@ -1438,8 +1448,6 @@ pa_status setup_decode(void* out, pa_dtype out_dtype, const void* query, pa_dtyp
     }
   }
   if (lp.umma) {
-    // the tensor-memory kernel reads one box per (head, d-chunk) layout only
-    if (mode != 0) return PA_ERR_UNSUPPORTED;
     // query rows [rows][Hq][D] as {64 elements, 2 d-chunks, Hq, rows}; a box
     // is 64 elements of G heads of 32 / G rows: 32 rows of 128 bytes
     const int G = num_q_heads / num_kv_heads;

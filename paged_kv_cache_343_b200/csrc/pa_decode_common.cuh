@@ -124,11 +124,12 @@ __device__ __forceinline__ int32_t clamp_len(int32_t L, int32_t max_len) {
 
 
 // The tensor-memory kernel for entries with many query columns
-// (pa_decode_umma.cu): head_dim 128, 16-bit caches, 2 or 4 KV heads per CTA.
+// (pa_decode_umma.cu): head_dim 128, 16-bit caches, 4 KV heads per CTA,
+// 16-token boxes whose rows run (d-chunk, head, token) (tma_mode 2).
 using UmmaKernel = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap,
                             const DecodeParams);
-UmmaKernel select_umma(int HG, bool bf16);
-size_t umma_smem_bytes(int HG, int stages);
+UmmaKernel select_umma(bool bf16);
+size_t umma_smem_bytes(int stages);
 constexpr int kUmmaThreads = 256;
 
 // ---------------------------------------------------------------------------
@@ -271,6 +272,9 @@ __device__ __forceinline__ void produce_tiles(const DecodeParams& p, const CUten
       if (p.tma_mode == 0) {
         tma_load_5d(kdst + off, tmK, full_k(stage), 0, tok_off, 0, hg * HG, id, policy);
         tma_load_5d(vdst + off, tmV, full_v(stage), 0, tok_off, 0, hg * HG, id, policy);
+      } else if (p.tma_mode == 2) {  // dims {row, tokens, heads, d-chunks, blocks}
+        tma_load_5d(kdst + off, tmK, full_k(stage), 0, tok_off, hg * HG, 0, id, policy);
+        tma_load_5d(vdst + off, tmV, full_v(stage), 0, tok_off, hg * HG, 0, id, policy);
       } else {
         for (int hh = 0; hh < HG; ++hh) {
           for (int dc = 0; dc < DCT; ++dc) {
