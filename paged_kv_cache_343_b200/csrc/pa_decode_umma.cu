@@ -50,9 +50,11 @@ constexpr int kUThreads = kUmmaThreads;      // 8 warps
 constexpr float kLazyLog2 = 8.0f;            // growth of a row maximum that forces a rescale
 constexpr uint32_t kUTileBytes = kTile * kUH * kUD * 2;  // K (or V) of one tile: 16 KiB
 constexpr uint32_t kUQBytes = 2 * 128 * 128;             // query rows of an entry: 32 KiB
-// tensor-memory columns: O [0, 128), S buffers [128, 256), P buffers [256, 384)
+// tensor-memory columns: O [0, 128), three S buffers [128, 320), three P
+// buffers of two halves [320, 512)
+constexpr int kUBufs = 3;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColO = 0, kColS = 128, kColP = 256;
+constexpr uint32_t kColO = 0, kColS = 128, kColP = 320;
 
 }  // namespace
 
@@ -67,7 +69,7 @@ __host__ __device__ inline UmmaLayout umma_layout(int NS) {
   L.info = L.q + 2u * kUQBytes;                        // two query buffers
   L.bars = L.info + static_cast<uint32_t>(NS) * sizeof(TileInfo);
   L.bars = (L.bars + 7u) & ~7u;
-  const uint32_t nbars = 3u * NS + 13u;
+  const uint32_t nbars = 3u * NS + 17u;
   L.tmem_slot = L.bars + nbars * 8u;
   L.total = L.tmem_slot + 16u;
   return L;
@@ -99,10 +101,10 @@ __global__ void __launch_bounds__(kUThreads, 1)
   auto q_full = [&](int b) { return barx + 8u * b; };
   auto q_free = [&](int b) { return barx + 8u * (2 + b); };
   auto s_full = [&](int j) { return barx + 8u * (4 + j); };
-  auto s_free = [&](int j) { return barx + 8u * (6 + j); };
-  auto p_full = [&](int j) { return barx + 8u * (8 + j); };
-  auto pv_done = [&](int j) { return barx + 8u * (10 + j); };
-  const uint32_t o_free = barx + 8u * 12;
+  auto s_free = [&](int j) { return barx + 8u * (7 + j); };
+  auto p_full = [&](int j) { return barx + 8u * (10 + j); };
+  auto pv_done = [&](int j) { return barx + 8u * (13 + j); };
+  const uint32_t o_free = barx + 8u * 16;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay.tmem_slot);
   // stage s: K rows (d-chunk dc, head g, token t) at ((dc * 4 + g) * 16 + t) * 128,
   // V the same 16 KiB further on
@@ -125,6 +127,8 @@ __global__ void __launch_bounds__(kUThreads, 1)
     for (int b = 0; b < 2; ++b) {
       mbar_init(q_full(b), 1);
       mbar_init(q_free(b), 1);     // the S issuer's commit
+    }
+    for (int b = 0; b < kUBufs; ++b) {
       mbar_init(s_full(b), 1);     // the S issuer's commit
       mbar_init(s_free(b), kUH);   // the four softmax warps
       mbar_init(p_full(b), kUH);
@@ -152,7 +156,7 @@ __global__ void __launch_bounds__(kUThreads, 1)
     const uint32_t zero[16] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
     const uint32_t lrow = tmem + (static_cast<uint32_t>(32 * warp) << 16);
 #pragma unroll
-    for (int k = 0; k < 8; ++k) tmem_st16(lrow + kColP + 16u * k, zero);
+    for (int k = 0; k < kUBufs * 4; ++k) tmem_st16(lrow + kColP + 16u * k, zero);
     tmem_wait_st();
   }
   griddep_launch_dependents();
@@ -201,7 +205,7 @@ __global__ void __launch_bounds__(kUThreads, 1)
         int32_t n_entry = -1;
         for (int64_t t = lo; t < hi; ++t) {
           const int64_t u = t - lo;
-          const int s = static_cast<int>(u % NS), j = static_cast<int>(u & 1);
+          const int s = static_cast<int>(u % NS), j = static_cast<int>(u % kUBufs);
           if (!mbar_wait(full_k(s), static_cast<uint32_t>((u / NS) & 1), p.err)) break;
           if (info[s].flags & kNewSeq) {
             ++n_entry;
@@ -210,7 +214,8 @@ __global__ void __launch_bounds__(kUThreads, 1)
             if (!mbar_wait(q_full(n_entry & 1), static_cast<uint32_t>(n_entry >> 1) & 1u, p.err))
               break;
           }
-          if (u >= 2 && !mbar_wait(s_free(j), static_cast<uint32_t>((u - 2) >> 1) & 1u, p.err))
+          if (u >= kUBufs &&
+              !mbar_wait(s_free(j), static_cast<uint32_t>((u / kUBufs - 1) & 1), p.err))
             break;
           tc_fence_after();
           const uint32_t qa = q_addr(n_entry & 1), ka = k_addr(s);
@@ -236,8 +241,8 @@ __global__ void __launch_bounds__(kUThreads, 1)
         int64_t pv_issued = -1;  // local index of the last P.V issued
         for (int64_t t = lo; t < hi; ++t) {
           const int64_t u = t - lo;
-          const int s = static_cast<int>(u % NS), j = static_cast<int>(u & 1);
-          if (!mbar_wait(p_full(j), static_cast<uint32_t>(u >> 1) & 1u, p.err)) break;
+          const int s = static_cast<int>(u % NS), j = static_cast<int>(u % kUBufs);
+          if (!mbar_wait(p_full(j), static_cast<uint32_t>((u / kUBufs) & 1), p.err)) break;
           const bool seg_start = (info[s].flags & kSegStart) != 0;
           if (seg_start) {
             // the previous segment's epilogue has read the accumulator
@@ -271,8 +276,8 @@ __global__ void __launch_bounds__(kUThreads, 1)
         }
         // the last products have finished before tensor memory is released
         if (pv_issued >= 0)
-          mbar_wait(pv_done(static_cast<int>(pv_issued & 1)),
-                    static_cast<uint32_t>(pv_issued >> 1) & 1u, p.err);
+          mbar_wait(pv_done(static_cast<int>(pv_issued % kUBufs)),
+                    static_cast<uint32_t>((pv_issued / kUBufs) & 1), p.err);
       }
     } else if (warp < kUH) {
       // ======================= softmax + epilogue =======================
@@ -284,14 +289,16 @@ __global__ void __launch_bounds__(kUThreads, 1)
       const uint32_t tP = lrow + kColP + static_cast<uint32_t>(h) * 8u;   // + (j * 2 + part) * 32
       const uint32_t tO = lrow + kColO;
       const float sl2 = p.scale_log2;
+      const int cdiv = col / G;  // query row of this column inside the entry
       float m_run = -INFINITY, l_run = 0.f;
       for (int64_t t = lo; t < hi; ++t) {
         const int64_t u = t - lo;
-        const int s = static_cast<int>(u % NS), j = static_cast<int>(u & 1);
+        const int s = static_cast<int>(u % NS), j = static_cast<int>(u % kUBufs);
         const uint32_t ph = static_cast<uint32_t>((u / NS) & 1);
+        const uint32_t bph = static_cast<uint32_t>((u / kUBufs) & 1);  // this buffer's use
         if (!warp_wait(full_k(s), ph, p.err)) break;
         const TileInfo ti = info[s];
-        if (!warp_wait(s_full(j), static_cast<uint32_t>(u >> 1) & 1u, p.err)) break;
+        if (!warp_wait(s_full(j), bph, p.err)) break;
         tc_fence_after();
         uint32_t sr[16];
         tmem_ld16(tS + static_cast<uint32_t>(j) * 64u, sr);
@@ -303,18 +310,33 @@ __global__ void __launch_bounds__(kUThreads, 1)
           m_run = -INFINITY;
           l_run = 0.f;
         }
-        const int ncol = ti.members * G;
-        const bool col_ok = col < ncol;
-        // column c sees tile rows up to rel + c / G (rel = 16: all)
-        const int lim = (ti.flags & kCausal) ? ti.rel + col / G : kTile;
         const uint32_t msk = static_cast<uint32_t>(ti.mask);
-        float sv[16];
-        float mx = -INFINITY;
+        // Every token of the tile visible to every column (the common case):
+        // no per-token selection.  Columns past the entry's (other queries or
+        // zero rows) are computed like the others and never written.
+        const bool full = __all_sync(
+            0xffffffffu, msk == 0xffffu && (!(ti.flags & kCausal) || ti.rel + cdiv >= kTile - 1));
+        float x[16];
 #pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          const bool ok = col_ok && ((msk >> k) & 1u) && k <= lim;
-          sv[k] = ok ? __uint_as_float(sr[k]) * sl2 : -INFINITY;
-          mx = fmaxf(mx, sv[k]);
+        for (int k = 0; k < 16; ++k) x[k] = __uint_as_float(sr[k]);
+        float mx;
+        if (full) {
+          float m8[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) m8[k] = fmaxf(x[k], x[k + 8]);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) m8[k] = fmaxf(m8[k], m8[k + 4]);
+          mx = fmaxf(fmaxf(m8[0], m8[2]), fmaxf(m8[1], m8[3])) * sl2;
+        } else {
+          // column c sees tile rows up to rel + c / G (rel = 16: all)
+          const int lim = (ti.flags & kCausal) ? ti.rel + cdiv : kTile;
+          mx = -INFINITY;
+#pragma unroll
+          for (int k = 0; k < 16; ++k) {
+            const bool ok = ((msk >> k) & 1u) && k <= lim;
+            x[k] = ok ? x[k] * sl2 : -INFINITY;
+            mx = fmaxf(mx, x[k]);
+          }
         }
         // the running maximum moves only when exceeded by 2^kLazyLog2
         bool rescale = false;
@@ -329,8 +351,8 @@ __global__ void __launch_bounds__(kUThreads, 1)
         if (__any_sync(0xffffffffu, rescale)) {
           // this row's accumulator holds earlier tiles of the segment: wait for
           // the last products into it (tile u - 1), then scale it in place
-          if (!warp_wait(pv_done(static_cast<int>((u - 1) & 1)),
-                         static_cast<uint32_t>((u - 1) >> 1) & 1u, p.err))
+          if (!warp_wait(pv_done(static_cast<int>((u - 1) % kUBufs)),
+                         static_cast<uint32_t>(((u - 1) / kUBufs) & 1), p.err))
             break;
           tc_fence_after();
 #pragma unroll 1
@@ -343,13 +365,25 @@ __global__ void __launch_bounds__(kUThreads, 1)
           }
           tmem_wait_st();
         }
-        float psum = 0.f;
+        float pw[16];
+        if (full) {
+          const float nm = -m_run;
+#pragma unroll
+          for (int k = 0; k < 16; ++k) pw[k] = ex2(fmaf(x[k], sl2, nm));
+        } else {
+#pragma unroll
+          for (int k = 0; k < 16; ++k) pw[k] = x[k] == -INFINITY ? 0.f : ex2(x[k] - m_run);
+        }
+        float ps[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) ps[k] = pw[k] + pw[k + 8];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) ps[k] += ps[k + 4];
+        const float psum = (ps[0] + ps[2]) + (ps[1] + ps[3]);
         uint32_t phi[8], plo[8];
 #pragma unroll
         for (int k = 0; k < 16; k += 2) {
-          const float p0 = sv[k] == -INFINITY ? 0.f : ex2(sv[k] - m_run);
-          const float p1 = sv[k + 1] == -INFINITY ? 0.f : ex2(sv[k + 1] - m_run);
-          psum += p0 + p1;
+          const float p0 = pw[k], p1 = pw[k + 1];
           if constexpr (kBF16) {
             // hi: the upper 16 bits of each fp32 weight (a bf16 value, by
             // truncation); lo: the exact remainder rounded to bf16
@@ -365,9 +399,8 @@ __global__ void __launch_bounds__(kUThreads, 1)
           }
         }
         l_run = l_run * alpha + psum;
-        // P buffer j was last read by the products of tile u - 2
-        if (u >= 2 && !warp_wait(pv_done(j), static_cast<uint32_t>((u - 2) >> 1) & 1u, p.err))
-          break;
+        // P buffer j was last read by the products of tile u - kUBufs
+        if (u >= kUBufs && !warp_wait(pv_done(j), bph ^ 1u, p.err)) break;
         tmem_st8(tP + static_cast<uint32_t>(j * 2) * 32u, phi);
         tmem_st8(tP + static_cast<uint32_t>(j * 2 + 1) * 32u, plo);
         tmem_wait_st();
@@ -392,13 +425,14 @@ __global__ void __launch_bounds__(kUThreads, 1)
         if (lane == 0) mbar_arrive(p_full(j));
 
         if (ti.flags & kSegEnd) {
-          if (!warp_wait(pv_done(j), static_cast<uint32_t>(u >> 1) & 1u, p.err)) break;
+          if (!warp_wait(pv_done(j), bph, p.err)) break;
           tc_fence_after();
           const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
           const bool direct = (ti.flags & kDirect) != 0;
           const bool part_ok = direct || ti.seg < p.nseg_cap;
           if (!direct && !part_ok && lane == 0) flag_error(p.err, PA_DEVERR_BAD_SEQLEN);
-          const int r = col / G;
+          const bool col_ok = col < ti.members * G;
+          const int r = cdiv;
           const int64_t orow =
               (static_cast<int64_t>(ti.qrow0) + r) * p.num_q_heads + kvh * G + (col - r * G);
           const int64_t prow =
