@@ -47,8 +47,10 @@ namespace pa {
 //   tiles[e]    = sum_{e' < e} (tiles of entry e')          (N = tiles[E] in all)
 //   segments    an entry's tiles are cut wherever a partition starts (every
 //               tiles_per_part tiles from its first tile) or a CTA's share
-//               starts (lo(c) = floor(c N / C)); each piece is one segment,
-//               numbered 0, 1, ... within the entry;
+//               starts (lo(c) of the LineCut: floor(c N / C), or with a
+//               split the packs' tiles and the sequences' tiles cut
+//               separately); each piece is one segment, numbered 0, 1, ...
+//               within the entry;
 //   seg_base[e] = sum_{e' < e} (segments of e'), so the partials of entry e
 //               occupy slots seg_base[e] .. seg_base[e + 1] - 1;
 //   start_seq[c], first_k[c]: the entry holding lo(c) and the number of
@@ -59,7 +61,7 @@ namespace pa {
 // when its share is not empty (lo(c) < lo(c + 1)), so every distinct start
 // is held once; it "coincides" when lo(c) is also a partition start of its
 // entry.  With SD, SDC the prefix sums over c of held and held-and-coincident,
-// and cnt(x) = min(C, ceil(x C / N)) the number of CTAs with lo(c) < x:
+// and cnt(x) the number of CTAs with lo(c) < x (LineCut::count_below):
 //   segments(e)  = partitions(e) + SD/SDC counts over CTAs cnt(t0) .. cnt(t1);
 //   first_k[c]   = partition starts of e below lo(c) + held starts in
 //                  [cnt(t0), c) - coincident ones among them.
@@ -99,17 +101,15 @@ __device__ __forceinline__ int32_t block_exclusive_scan(int32_t v, int32_t* warp
 // Records start_seq / first_k for every CTA whose share starts inside b and
 // returns the number of segments.
 __device__ int32_t plan_sequence_segments(const DecodeParams& p, int32_t b, int64_t t0,
-                                          int64_t t1, int64_t N, int64_t C) {
-  const int64_t q = N / C, r = N % C;
-  int64_t c = (t0 * C + N - 1) / N;  // first CTA with lo(c) >= t0
-  int64_t lo_c = c * q + (c * r) / C;
-  int64_t rem = (c * r) % C;         // lo(c + 1) = lo(c) + q + [rem + r >= C]
+                                          int64_t t1, const LineCut& cut) {
+  int64_t c = cut.count_below(t0);  // first CTA with lo(c) >= t0
+  int64_t lo_c = c < cut.C ? cut.lo(c) : INT64_MAX;
   int64_t part = t0;                 // next partition start
   const int64_t tpp = p.tiles_per_part;
   int32_t count = 0;
   int64_t last = -1;
   while (true) {
-    const int64_t cta_pt = (c < C && lo_c < t1) ? lo_c : INT64_MAX;
+    const int64_t cta_pt = (c < cut.C && lo_c < t1) ? lo_c : INT64_MAX;
     const int64_t part_pt = part < t1 ? part : INT64_MAX;
     if (cta_pt == INT64_MAX && part_pt == INT64_MAX) break;
     if (cta_pt <= part_pt) {
@@ -118,9 +118,7 @@ __device__ int32_t plan_sequence_segments(const DecodeParams& p, int32_t b, int6
       p.start_seq[c] = b;
       p.first_k[c] = idx;
       ++c;
-      rem += r;
-      lo_c += q;
-      if (rem >= C) { rem -= C; ++lo_c; }
+      lo_c = c < cut.C ? cut.lo(c) : INT64_MAX;
     } else {
       if (part_pt != last) { ++count; last = part_pt; }
       part = (tpp == INT_MAX) ? INT64_MAX : part + tpp;
@@ -296,6 +294,11 @@ __global__ void __launch_bounds__(kPlanThreads) pa_plan_kernel(DecodeParams p) {
   const int C = p.ctas_per_group;
   const int32_t tpp = p.tiles_per_part;
   const int32_t* tiles = E <= kPlanSmemTiles ? s_tiles : p.plan_tiles;
+  LineCut cut;
+  cut.C = C;
+  cut.S = p.split_ctas;
+  cut.N = N;
+  cut.NK = p.split_ctas > 0 ? tiles[K] : 0;
   if (!p.plan_closed) {  // few cut points per entry: walk them
     int32_t seg_carry = 0;
     for (int ch = 0; ch < nchunks; ++ch) {
@@ -303,7 +306,7 @@ __global__ void __launch_bounds__(kPlanThreads) pa_plan_kernel(DecodeParams p) {
       int32_t ns = 0;
       if (e < E && N > 0) {
         const int64_t t0 = tiles[e], t1 = tiles[e + 1];
-        if (t1 > t0) ns = plan_sequence_segments(p, e, t0, t1, N, C);
+        if (t1 > t0) ns = plan_sequence_segments(p, e, t0, t1, cut);
       }
       const int32_t ex = block_exclusive_scan(ns, warp_buf, &total);
       if (e < E) p.seg_base[e] = seg_carry + ex;
@@ -312,9 +315,9 @@ __global__ void __launch_bounds__(kPlanThreads) pa_plan_kernel(DecodeParams p) {
     if (tid == 0) p.seg_base[E] = seg_carry;
     return;
   }
-  auto lo_of = [&](int64_t c) { return c * N / C; };
+  auto lo_of = [&](int64_t c) { return cut.lo(c); };
   auto cnt_below = [&](int64_t x) {  // CTAs with lo(c) < x
-    return static_cast<int>(min(static_cast<int64_t>(C), (x * C + N - 1) / N));
+    return static_cast<int>(cut.count_below(x));
   };
   // ---- CTAs: the entry holding each share's start; held / coincident flags,
   // scanned together as held + coincident * 2^16 (C <= kPlanMaxCtas < 2^15)
@@ -425,8 +428,7 @@ __global__ void __launch_bounds__((HG * CG + 1) * 32, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int hg = blockIdx.y;
-  const int64_t C = p.ctas_per_group;
-  const int c = blockIdx.x;
+  const int c = p.cta_base + blockIdx.x;  // this CTA's share of the line (LineCut)
   const int B = p.num_seqs;
 
   if (threadIdx.x == 0) {
@@ -453,13 +455,17 @@ __global__ void __launch_bounds__((HG * CG + 1) * 32, 1)
   const bool plain = p.pack_size == 1 && p.q_start == nullptr;
   const int E = plain ? B : p.meta[1];
   const int64_t N = p.plan_tiles[E];
-  const int64_t lo = static_cast<int64_t>(c) * N / C;
-  const int64_t hi = static_cast<int64_t>(c + 1) * N / C;
+  const LineCut cut = line_cut(p, N);
+  const int64_t lo = cut.lo(c);
+  const int64_t hi = cut.lo(c + 1);
   if (lo >= hi) return;
 
   if (warp == NW) {
     // ======================= producer =======================
-    if (lane != 0) return;
+    if (lane != 0) {
+      check_pack_tables(p, lo, hi, c, lane - 1, 31);
+      return;
+    }
     produce_tiles<HG, DCT>(p, &tmK, &tmV, smem_base, kTileBytes, info, full_k(0), full_v(0),
                            empty(0), NS, lo, hi, c, hg, plain,
                            [](int32_t, int32_t) { return true; });
@@ -817,8 +823,7 @@ __global__ void __launch_bounds__((HG * CG + 1) * 32, 1)
             }
           }
         } else if (ti.seg < p.nseg_cap) {
-          const int64_t prow =
-              ((static_cast<int64_t>(hg) * p.nseg_cap + ti.seg) * HG + g) * p.cols;
+          const int64_t prow = part_row(p, ti.seg, kvh, 0);
           float* po = p.part_o + prow * D;
 #pragma unroll
           for (int mt = 0; mt < MTILES; ++mt) {
@@ -908,9 +913,8 @@ __global__ void __launch_bounds__(kCombineWarps * 32) pa_combine_narrow_kernel(c
   griddep_launch_dependents();
   griddep_wait();  // the main kernel's partials are complete and visible
   if (qh >= p.num_q_heads || !host_plan_matches(p)) return;
-  const int G = p.group, HG = p.heads_per_cta;
+  const int G = p.group;
   const int kvh = qh / G, h = qh - kvh * G;
-  const int hg = kvh / HG, g = kvh - hg * HG;
   const RowParts rp = row_parts(p, b, h);
   if (rp.direct || !rp.valid) return;  // written by the main kernel (or no entry)
   // partial k: k < ns from the row's own entry, then the pack's
@@ -920,7 +924,7 @@ __global__ void __launch_bounds__(kCombineWarps * 32) pa_combine_narrow_kernel(c
   auto row_of = [&](int32_t k) {
     const int32_t slot = k < nseq ? rp.s0 + k : rp.s1 + (k - nseq);
     const int col = k < nseq ? rp.col0 : rp.col1;
-    return ((static_cast<int64_t>(hg) * p.nseg_cap + slot) * HG + g) * p.cols + col;
+    return part_row(p, slot, kvh, col);
   };
   const int64_t obase = (static_cast<int64_t>(b) * p.num_q_heads + qh) * D + lane * V;
 
@@ -989,9 +993,8 @@ __global__ void __launch_bounds__(kCombineWarps * 32) pa_combine_wide_kernel(con
   griddep_launch_dependents();
   griddep_wait();  // the main kernel's partials are complete and visible
   if (!host_plan_matches(p)) return;
-  const int G = p.group, HG = p.heads_per_cta;
+  const int G = p.group;
   const int kvh = qh / G, h = qh - kvh * G;
-  const int hg = kvh / HG, g = kvh - hg * HG;
   const RowParts rp = row_parts(p, b, h);
   if (rp.direct || !rp.valid) return;  // written by the main kernel (or no entry)
   const int32_t nseq = (rp.s0 + rp.ns <= p.nseg_cap) ? rp.ns : 0;
@@ -1000,7 +1003,7 @@ __global__ void __launch_bounds__(kCombineWarps * 32) pa_combine_wide_kernel(con
   auto row_of = [&](int32_t k) {  // partial k: own entry's first, then the pack's
     const int32_t slot = k < nseq ? rp.s0 + k : rp.s1 + (k - nseq);
     const int col = k < nseq ? rp.col0 : rp.col1;
-    return ((static_cast<int64_t>(hg) * p.nseg_cap + slot) * HG + g) * p.cols + col;
+    return part_row(p, slot, kvh, col);
   };
 
   float M = -INFINITY;
@@ -1122,6 +1125,14 @@ struct LaunchPlan {
   bool umma = false;           // the tensor-memory kernel (many query columns, head_dim 128)
   UmmaKernel ukernel = nullptr;
   size_t smem = 0;
+  // split (shared prompts on the tensor-memory kernel): CTAs 0 .. split_ctas-1
+  // of the line run the packs on the tensor-memory kernel (grid split_ctas x
+  // groups); the sequences' own tiles run on the warp-level kernel `kernel`
+  // with the shape below (grid ctas_b x groups_b), as line CTAs split_ctas ..
+  // ctas_per_group - 1
+  bool split = false;
+  int split_ctas = 0, ctas_b = 0, groups_b = 0, HG_b = 0, threads_b = 0, stages_b = 0;
+  size_t smem_b = 0;
   size_t off_tiles = 0, off_segs = 0, off_start = 0, off_firstk = 0, off_meta = 0,
          off_pack_first = 0, off_pack_n = 0, off_pack_tiles = 0, off_seq_pack = 0,
          off_seq_pre = 0, off_ent = 0, off_o = 0, off_ml = 0, total = 0;
@@ -1129,6 +1140,28 @@ struct LaunchPlan {
 };
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Launch shape of the warp-level main kernel for HG heads per CTA: stages of
+// K and V tiles within a 200 KiB budget (at most 6), the kernel, threads,
+// dynamic shared memory and resident CTAs per SM (opting into the memory).
+pa_status warp_kernel_shape(int D, int HG, int NB, int CG, bool bf16, bool fp8, MainKernel* kernel,
+                            int* stages, size_t* smem, int* threads, int* per_sm) {
+  const size_t tile_bytes = static_cast<size_t>(kTile) * HG * D * (fp8 ? 1 : 2);
+  const size_t budget = 200 * 1024;
+  int ns = static_cast<int>(budget / (2 * tile_bytes));
+  if (ns > 6) ns = 6;
+  if (ns < 2) return PA_ERR_UNSUPPORTED;
+  *stages = ns;
+  *smem = 1024 + static_cast<size_t>(ns) * 2 * tile_bytes + ns * sizeof(TileInfo) +
+          3 * ns * sizeof(uint64_t);
+  *threads = (HG * CG + 1) * 32;
+  *kernel = select_main(D, HG, NB, CG, bf16, fp8);
+  if (*kernel == nullptr) return PA_ERR_UNSUPPORTED;
+  const void* kfn = reinterpret_cast<const void*>(*kernel);
+  if (!ensure_smem_attr(kfn, *smem)) return PA_ERR_CUDA;
+  *per_sm = ctas_per_sm(kfn, *threads, *smem);
+  return *per_sm >= 1 ? PA_OK : PA_ERR_CUDA;
+}
 
 bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
 
@@ -1175,12 +1208,15 @@ pa_status make_plan(int32_t num_seqs, int32_t Hq, int32_t Hkv, int32_t D, int32_
   const int DCT = fp8 ? 1 : D / 64;  // 128-byte rows per (token, head) in a stage
   const int TB = bs < kTile ? bs : kTile;
   if ((HG * DCT * TB * 128) % 1024 != 0) return PA_ERR_UNSUPPORTED;
-  // Entries of many query columns (packs, query chunks) with 16-bit caches and
-  // head_dim 128 run on the tensor-memory kernel when its shape rules hold: the
-  // query columns of an entry fill whole 32-row loads (G divides 32), four KV
-  // heads per CTA, 16-token boxes (blocks of 16 tokens or more).
-  const bool umma = (P > 1 || Qc > 0) && !fp8 && D == 128 && 32 % G == 0 && TB == kTile &&
-                    Hkv % 4 == 0;
+  // Entries whose query columns fill all 32 rows a KV head has in the
+  // tensor-memory kernel's products (packs of 32 / G samples, chunks of
+  // 32 / G query tokens), with 16-bit caches and head_dim 128, run on that
+  // kernel when its shape rules also hold: four KV heads per CTA, 16-token
+  // boxes (blocks of 16 tokens or more).  Narrower entries would leave rows
+  // of every product idle; the warp-level kernel takes them.
+  const int entry_cols = (Qc > 0 ? Qc : P) * G;
+  const bool umma = (P > 1 || Qc > 0) && entry_cols >= kMaxPackCols && !fp8 && D == 128 &&
+                    32 % G == 0 && TB == kTile && Hkv % 4 == 0;
   if (umma) HG = 4;
   lp->HG = HG;
   lp->head_dim = D;
@@ -1192,7 +1228,7 @@ pa_status make_plan(int32_t num_seqs, int32_t Hq, int32_t Hkv, int32_t D, int32_
   lp->umma = umma;
   const DeviceInfo* dev = current_device_info();
   if (dev == nullptr) return PA_ERR_CUDA;
-  const void* kfn = nullptr;
+  int per_sm = 0;
   if (umma) {
     int stages = 6;
     while (stages > 2 && umma_smem_bytes(stages) > static_cast<size_t>(dev->max_smem_optin))
@@ -1201,26 +1237,41 @@ pa_status make_plan(int32_t num_seqs, int32_t Hq, int32_t Hkv, int32_t D, int32_
     lp->smem = umma_smem_bytes(stages);
     lp->ukernel = select_umma(bf16);
     if (lp->ukernel == nullptr) return PA_ERR_UNSUPPORTED;
-    kfn = reinterpret_cast<const void*>(lp->ukernel);
+    const void* kfn = reinterpret_cast<const void*>(lp->ukernel);
+    if (!ensure_smem_attr(kfn, lp->smem)) return PA_ERR_CUDA;
+    per_sm = ctas_per_sm(kfn, lp->threads, lp->smem);
+    if (per_sm < 1) return PA_ERR_CUDA;
   } else {
-    const size_t tile_bytes = static_cast<size_t>(kTile) * HG * D * (fp8 ? 1 : 2);
-    const size_t budget = 200 * 1024;
-    int stages = static_cast<int>(budget / (2 * tile_bytes));
-    if (stages > 6) stages = 6;
-    if (stages < 2) return PA_ERR_UNSUPPORTED;
-    lp->stages = stages;
-    lp->smem = 1024 + static_cast<size_t>(stages) * 2 * tile_bytes +
-               stages * sizeof(TileInfo) + 3 * stages * sizeof(uint64_t);
-    lp->kernel = select_main(D, HG, NB, CG, bf16, fp8);
-    if (lp->kernel == nullptr) return PA_ERR_UNSUPPORTED;
-    kfn = reinterpret_cast<const void*>(lp->kernel);
+    int threads = 0;
+    const pa_status st = warp_kernel_shape(D, HG, NB, CG, bf16, fp8, &lp->kernel, &lp->stages,
+                                           &lp->smem, &threads, &per_sm);
+    if (st != PA_OK) return st;
   }
-  if (!ensure_smem_attr(kfn, lp->smem)) return PA_ERR_CUDA;
-  const int per_sm = ctas_per_sm(kfn, lp->threads, lp->smem);
-  if (per_sm < 1) return PA_ERR_CUDA;
   const int total_ctas = dev->num_sms * per_sm;
   lp->ctas_per_group = total_ctas / lp->groups > 0 ? total_ctas / lp->groups : 1;
   if (lp->ctas_per_group > kPlanMaxCtas) lp->ctas_per_group = kPlanMaxCtas;
+  if (umma && P > 1) {
+    // Shared prompts: the packs' prefixes on the tensor-memory kernel, every
+    // sequence's own tiles (one query row: G of the 32 columns) on the
+    // warp-level kernel with one column block per head, run after it.  A
+    // sequence entry is short and narrow; on the tensor-memory kernel it
+    // would cost a query load, an epilogue and whole products.
+    int HGb = 8;
+    while (Hkv % HGb != 0) HGb >>= 1;
+    int per_sm_b = 0;
+    const pa_status st = warp_kernel_shape(D, HGb, 1, 1, bf16, false, &lp->kernel, &lp->stages_b,
+                                           &lp->smem_b, &lp->threads_b, &per_sm_b);
+    if (st != PA_OK) return st;
+    lp->split = true;
+    lp->HG_b = HGb;
+    lp->groups_b = Hkv / HGb;
+    lp->ctas_b = dev->num_sms * per_sm_b / lp->groups_b;
+    if (lp->ctas_b < 1) lp->ctas_b = 1;
+    if (lp->ctas_per_group > kPlanMaxCtas / 2) lp->ctas_per_group = kPlanMaxCtas / 2;
+    if (lp->ctas_b > kPlanMaxCtas / 2) lp->ctas_b = kPlanMaxCtas / 2;
+    lp->split_ctas = lp->ctas_per_group;
+    lp->ctas_per_group += lp->ctas_b;
+  }
 
   const int64_t max_tiles = (static_cast<int64_t>(max_seq_len) + kTile - 1) / kTile;
   int64_t parts_per_seq = 1;
@@ -1266,10 +1317,9 @@ pa_status make_plan(int32_t num_seqs, int32_t Hq, int32_t Hkv, int32_t D, int32_
     off = lp->off_ent + 5 * words(num_rows);
   }
   lp->off_o = off;
-  const size_t o_bytes = static_cast<size_t>(lp->groups) * nseg * HG * lp->cols * D * sizeof(float);
+  const size_t o_bytes = static_cast<size_t>(Hkv) * nseg * lp->cols * D * sizeof(float);
   lp->off_ml = lp->off_o + align_up(o_bytes, 256);
-  const size_t ml_bytes =
-      static_cast<size_t>(lp->groups) * nseg * HG * lp->cols * 2 * sizeof(float);
+  const size_t ml_bytes = static_cast<size_t>(Hkv) * nseg * lp->cols * 2 * sizeof(float);
   lp->total = lp->off_ml + align_up(ml_bytes, 256);
   return PA_OK;
 }
@@ -1350,6 +1400,8 @@ struct DecodeSetup {
   DecodeParams p;
   CUtensorMap tmK, tmV;
   CUtensorMap tmQ;  // the tensor-memory kernel's query rows
+  CUtensorMap tmK_b, tmV_b;  // split: the warp-level kernel's K/V maps (mode_b)
+  int mode_b = 0;
 };
 
 // Shared by the 16-bit and the fp8 entry points: validates the arguments,
@@ -1413,7 +1465,35 @@ pa_status setup_decode(void* out, pa_dtype out_dtype, const void* query, pa_dtyp
   }
   const int DCT = fp8 ? 1 : D / 64;           // 128-byte rows per (token, head)
   const uint32_t inner = fp8 ? 128u : 64u;    // elements in one 128-byte row
+  // The warp-level kernel's maps for HGx heads per CTA.  mode 0: dims {row,
+  // tokens, d-chunks, heads, blocks}, box {row, TB, DCT, HGx, 1}; mode 1 (when
+  // the driver rejects mode 0): dims {row, d-chunks, heads, tokens, blocks},
+  // box {row, 1, 1, TB, 1}.
+  auto warp_maps = [&](int HGx, CUtensorMap* mk, CUtensorMap* mv, int* m) {
+    const uint64_t dims0[5] = {inner, (uint64_t)block_size, (uint64_t)DCT,
+                               (uint64_t)num_kv_heads, (uint64_t)num_blocks};
+    const uint64_t str0[4] = {tok_b, 128, head_b, blk_b};
+    const uint32_t box0[5] = {inner, (uint32_t)lp.tok_box, (uint32_t)DCT, (uint32_t)HGx, 1};
+    const uint64_t dims1[5] = {inner, (uint64_t)DCT, (uint64_t)num_kv_heads,
+                               (uint64_t)block_size, (uint64_t)num_blocks};
+    const uint64_t str1[4] = {128, head_b, tok_b, blk_b};
+    const uint32_t box1[5] = {inner, 1, 1, (uint32_t)lp.tok_box, 1};
+    if (get_tensor_map(mk, key_cache, dims0, str0, box0, elem_bytes) &&
+        get_tensor_map(mv, value_cache, dims0, str0, box0, elem_bytes)) {
+      *m = 0;
+      return true;
+    }
+    if (lp.tok_box * 128 % 1024 == 0 &&
+        get_tensor_map(mk, key_cache, dims1, str1, box1, elem_bytes) &&
+        get_tensor_map(mv, value_cache, dims1, str1, box1, elem_bytes)) {
+      *m = 1;
+      return true;
+    }
+    return false;
+  };
   int mode = 0;
+  if (lp.split && !warp_maps(lp.HG_b, &su->tmK_b, &su->tmV_b, &su->mode_b))
+    return PA_ERR_UNSUPPORTED;
   if (lp.umma) {
     // mode 2: dims {row, tokens, heads, d-chunks, blocks}, box {row, 16, HG, 2, 1}:
     // the rows of one d-chunk of all HG heads are contiguous in the stage
@@ -1425,27 +1505,8 @@ pa_status setup_decode(void* out, pa_dtype out_dtype, const void* query, pa_dtyp
         !get_tensor_map(&su->tmV, value_cache, dims2, str2, box2, elem_bytes))
       return PA_ERR_UNSUPPORTED;
     mode = 2;
-  } else {
-    // mode 0: dims {row, tokens, d-chunks, heads, blocks}, box {row, TB, DCT, HG, 1}
-    const uint64_t dims0[5] = {inner, (uint64_t)block_size, (uint64_t)DCT,
-                               (uint64_t)num_kv_heads, (uint64_t)num_blocks};
-    const uint64_t str0[4] = {tok_b, 128, head_b, blk_b};
-    const uint32_t box0[5] = {inner, (uint32_t)lp.tok_box, (uint32_t)DCT, (uint32_t)HG, 1};
-    // mode 1: dims {row, d-chunks, heads, tokens, blocks}, box {row, 1, 1, TB, 1}
-    const uint64_t dims1[5] = {inner, (uint64_t)DCT, (uint64_t)num_kv_heads,
-                               (uint64_t)block_size, (uint64_t)num_blocks};
-    const uint64_t str1[4] = {128, head_b, tok_b, blk_b};
-    const uint32_t box1[5] = {inner, 1, 1, (uint32_t)lp.tok_box, 1};
-    if (get_tensor_map(&su->tmK, key_cache, dims0, str0, box0, elem_bytes) &&
-        get_tensor_map(&su->tmV, value_cache, dims0, str0, box0, elem_bytes)) {
-      mode = 0;
-    } else if (lp.tok_box * 128 % 1024 == 0 &&
-               get_tensor_map(&su->tmK, key_cache, dims1, str1, box1, elem_bytes) &&
-               get_tensor_map(&su->tmV, value_cache, dims1, str1, box1, elem_bytes)) {
-      mode = 1;
-    } else {
-      return PA_ERR_UNSUPPORTED;
-    }
+  } else if (!warp_maps(HG, &su->tmK, &su->tmV, &mode)) {
+    return PA_ERR_UNSUPPORTED;
   }
   if (lp.umma) {
     // query rows [rows][Hq][D] as {64 elements, 2 d-chunks, Hq, rows}; a box
@@ -1476,6 +1537,8 @@ pa_status setup_decode(void* out, pa_dtype out_dtype, const void* query, pa_dtyp
   p.tiles_per_part = lp.tiles_per_part;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.ctas_per_group = lp.ctas_per_group;
+  p.split_ctas = lp.split ? lp.split_ctas : 0;
+  p.cta_base = 0;
   p.heads_per_cta = HG;
   p.nseg_cap = lp.nseg_cap;
   p.stages = lp.stages;
@@ -1529,10 +1592,20 @@ pa_status launch_setup(const DecodeSetup& su, cudaStream_t s, bool run_combine =
   if (p.host_plan == nullptr &&
       PdlLaunch(s, dim3(1), dim3(kPlanThreads))(pa_plan_kernel, p) != cudaSuccess)
     return PA_ERR_CUDA;
-  PdlLaunch main_launch(s, dim3(lp.ctas_per_group, lp.groups), dim3(lp.threads), lp.smem);
+  const int ctas_a = lp.split ? lp.split_ctas : lp.ctas_per_group;
+  PdlLaunch main_launch(s, dim3(ctas_a, lp.groups), dim3(lp.threads), lp.smem);
   const cudaError_t e2 = lp.umma ? main_launch(lp.ukernel, su.tmK, su.tmV, su.tmQ, p)
                                  : main_launch(lp.kernel, su.tmK, su.tmV, p);
   if (e2 != cudaSuccess) return PA_ERR_CUDA;
+  if (lp.split) {  // the sequences' own tiles: line CTAs split_ctas .. ctas_per_group - 1
+    DecodeParams pb = p;
+    pb.cta_base = lp.split_ctas;
+    pb.heads_per_cta = lp.HG_b;
+    pb.stages = lp.stages_b;
+    pb.tma_mode = su.mode_b;
+    PdlLaunch seq_launch(s, dim3(lp.ctas_b, lp.groups_b), dim3(lp.threads_b), lp.smem_b);
+    if (seq_launch(lp.kernel, su.tmK_b, su.tmV_b, pb) != cudaSuccess) return PA_ERR_CUDA;
+  }
   if (!run_combine) return PA_OK;
   const int D = lp.head_dim;
   cudaError_t e3;

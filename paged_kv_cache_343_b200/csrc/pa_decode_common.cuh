@@ -51,9 +51,13 @@ struct DecodeParams {
   int32_t num_rows;        // query (and output) rows: num_seqs, or the multi-query rows
   int32_t tiles_per_part;  // partition length in tiles (INT_MAX: no partitions)
   float scale_log2;        // scale * log2(e)
-  int32_t ctas_per_group;  // CTAs sharing one head group's tiles
+  int32_t ctas_per_group;  // CTAs sharing one head group's tiles (both kernels of a split)
+  int32_t split_ctas;      // 0: one kernel walks the whole line; else CTAs 0 .. split_ctas-1
+                           //    (the tensor-memory kernel) share the packs' tiles and the
+                           //    rest (the warp-level kernel) the sequences' (LineCut)
+  int32_t cta_base;        // line CTA index of this launch's blockIdx.x == 0
   int32_t heads_per_cta;   // KV heads per CTA (HG)
-  int32_t nseg_cap;        // partial slots per head group
+  int32_t nseg_cap;        // partial slots (segments)
   int32_t stages;
   int32_t tok_box;         // tokens per TMA box: min(block_size, 16)
   int32_t tma_mode;        // 0: one box per block per tile, 1: one per (head, d-half)
@@ -84,8 +88,8 @@ struct DecodeParams {
   int32_t* ent_tok;        // [rows] tokens entry e reads: one past its last query's position
   int32_t* q_entry;        // [rows] entry of query row r
   int32_t cols;            // partial columns per KV head: pack_size * group
-  float* part_o;           // [groups][nseg_cap][HG][cols][head_dim]
-  float* part_ml;          // [groups][nseg_cap][HG][cols][2]  (m in log2 units, l)
+  float* part_o;           // [nseg_cap][num_kv_heads][cols][head_dim]
+  float* part_ml;          // [nseg_cap][num_kv_heads][cols][2]  (m in log2 units, l)
   int32_t* err;
   const float* k_scale;    // fp8 cache only: element = code * (*k_scale)
   const float* v_scale;
@@ -98,6 +102,44 @@ struct DecodeParams {
   int32_t out_vec16;       // out is 16-byte aligned (vector stores allowed)
   uint64_t consumer_wait_ns;  // limit of the consumer warps' waits for a landed stage
 };
+
+// How the tile line of N tiles is cut into CTA shares [lo(c), lo(c + 1)).
+// One kernel (S == 0): evenly over the C CTAs.  Split (0 < S < C): the
+// packs' tiles [0, NK) evenly over CTAs 0 .. S-1, the sequences' tiles
+// [NK, N) evenly over CTAs S .. C-1, so no share mixes the two.
+struct LineCut {
+  int64_t C, S, N, NK;
+  __host__ __device__ int64_t lo(int64_t c) const {
+    if (S == 0) return c * N / C;
+    if (c < S) return c * NK / S;
+    return NK + (c - S) * (N - NK) / (C - S);
+  }
+  // CTAs whose share starts below x, 0 <= x <= N (lo is non-decreasing in c)
+  __host__ __device__ int64_t count_below(int64_t x) const {
+    auto cdiv = [](int64_t a, int64_t b) { return (a + b - 1) / b; };
+    if (N <= 0) return 0;
+    if (S == 0) return min(C, cdiv(x * C, N));
+    if (x <= NK) return NK > 0 ? min(S, cdiv(x * S, NK)) : 0;
+    const int64_t C2 = C - S, N2 = N - NK;
+    return S + min(C2, cdiv((x - NK) * C2, N2));
+  }
+};
+
+// The cut of a plan whose entries end at tile N (packs end at plan_tiles[K]).
+__device__ __forceinline__ LineCut line_cut(const DecodeParams& p, int64_t N) {
+  LineCut L;
+  L.C = p.ctas_per_group;
+  L.S = p.split_ctas;
+  L.N = N;
+  L.NK = p.split_ctas > 0 ? p.plan_tiles[p.meta[0]] : 0;
+  return L;
+}
+
+// Row of (segment, KV head, column) in the partial buffers.
+__host__ __device__ __forceinline__ int64_t part_row(const DecodeParams& p, int64_t seg, int kvh,
+                                                     int col) {
+  return (seg * (p.num_q_heads / p.group) + kvh) * p.cols + col;
+}
 
 // Limit of the consumers' waits for the next call's kernels (host side; see
 // pa_set_consumer_wait_limit_ns).
@@ -133,10 +175,41 @@ size_t umma_smem_bytes(int stages);
 constexpr int kUmmaThreads = 256;
 
 // ---------------------------------------------------------------------------
+// The members of a pack read the first member's blocks over the pack's tiles,
+// so their tables must hold the same ids there; a difference is flagged
+// (PA_DEVERR_BAD_SHARE).  Threads first, first + stride, ... of a warp that
+// does not load tiles take the CTA's tiles [lo, hi) in turn, away from the
+// producer's path.  Entries 0 .. K-1 of a line are the packs.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void check_pack_tables(const DecodeParams& p, int64_t lo, int64_t hi,
+                                                  int c, int first, int stride) {
+  if (p.pack_size <= 1 || p.q_start != nullptr) return;
+  const int K = p.meta[0];
+  int e = p.start_seq[c];
+  const int bs = p.block_size;
+  const int nblk = bs < kTile ? kTile / bs : 1;  // blocks a tile reads
+  for (int64_t t = lo + first; t < hi && e < K; t += stride) {
+    while (e < K && t >= p.plan_tiles[e + 1]) ++e;
+    if (e >= K) break;
+    const int64_t ti = t - p.plan_tiles[e];  // tile of the pack's prefix
+    const int members = p.pack_n[e];
+    const int32_t* row = p.block_tables + static_cast<int64_t>(p.pack_first[e]) * p.table_stride;
+    const int64_t idx0 = bs < kTile ? ti * nblk : ti * kTile / bs;
+    for (int kk = 0; kk < nblk; ++kk) {
+      const int32_t id = __ldg(row + idx0 + kk);
+#pragma unroll
+      for (int m = 1; m < kMaxPack; ++m)
+        if (m < members && __ldg(row + static_cast<int64_t>(m) * p.table_stride + idx0 + kk) != id)
+          flag_error(p.err, PA_DEVERR_BAD_SHARE);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
 // The producer warp's loop (one elected lane), shared by the decode kernels:
 // walks the CTA's tiles [lo, hi) of the tile line entry by entry, looks up
-// each tile's block ids (one table lookup per block), loads its K and V with
-// TMA into the stage ring (full_k / full_v of stage s at full_k0 + 8 s ...;
+// each tile's block ids (one tile ahead, one table lookup per block), loads
+// its K and V with TMA into the stage ring (full_k / full_v of stage s at full_k0 + 8 s ...;
 // a stage is reused once empty[s] completes), and publishes each tile's
 // TileInfo.  on_entry(n, qrow0) runs after the first tile of the CTA's n-th
 // entry has been published (n = 0, 1, ...); returning false stops the loop.
@@ -208,16 +281,19 @@ __device__ __forceinline__ void produce_tiles(const DecodeParams& p, const CUten
   int stage = 0;
   uint32_t phase = 0;
   int64_t issued = 0;
-  // blocks longer than a tile: the id of the block the last tile read, so a
-  // block's tiles after its first reuse it (one table lookup per block)
-  const int32_t* id_row = nullptr;
-  int64_t id_idx = -1;
-  int32_t id_val = -1;
-  // the pack's other members must hold the same block ids
-  auto check_shared = [&](int64_t idx, int32_t id) {
-    for (int m = 1; m < members; ++m)
-      if (__ldg(row + static_cast<int64_t>(m) * p.table_stride + idx) != id)
-        flag_error(p.err, PA_DEVERR_BAD_SHARE);
+  // Block ids of the tile after this one (same entry), loaded one tile ahead
+  // so that their latency hides behind this tile's wait and copies.  Only the
+  // ids a tile reads are loaded: blocks holding valid tokens.
+  int32_t nxt[kTile / 4];
+  bool nxt_ready = false;
+  auto load_ids = [&](int32_t ts, int32_t v, int32_t* ids) {
+    if (bs <= kTile) {
+#pragma unroll
+      for (int kk = 0; kk < kTile / 4; ++kk)  // at most 4 blocks: block_size >= 4
+        ids[kk] = (kk < bpt && kk * bs < v) ? ld_early(row + static_cast<int64_t>(ts) * bpt + kk) : -1;
+    } else {
+      ids[0] = ld_early(row + static_cast<int64_t>(ts) * kTile / bs);
+    }
   };
   // Tile index inside its partition: segments start at the CTA's first
   // tile, at an entry's first tile and at every partition start, and end
@@ -231,6 +307,7 @@ __device__ __forceinline__ void produce_tiles(const DecodeParams& p, const CUten
       i = 0;
       ip = 0;
       new_seq = true;
+      nxt_ready = false;
     }
     const int32_t ti_seq = i0 + i;  // tile index inside the sequence
     const int32_t valid = stale ? 0 : min(kTile, L_b - ti_seq * kTile);
@@ -246,19 +323,23 @@ __device__ __forceinline__ void produce_tiles(const DecodeParams& p, const CUten
     new_seq = false;
     if (++ip == tpp) ip = 0;
     uint32_t mask = valid >= kTile ? 0xffffu : ((1u << valid) - 1u);
-    // the first block id is loaded before the wait for a free stage
-    const int64_t idx0 = bs <= kTile ? static_cast<int64_t>(ti_seq) * bpt
-                                     : static_cast<int64_t>(ti_seq) * kTile / bs;
-    int32_t id0 = -1;
-    if (!stale) {
-      if (bs > kTile && row == id_row && idx0 == id_idx) {
-        id0 = id_val;
+    int32_t ids[kTile / 4];
+    if (nxt_ready) {
+#pragma unroll
+      for (int kk = 0; kk < kTile / 4; ++kk) ids[kk] = nxt[kk];
+    } else if (!stale) {
+      load_ids(ti_seq, valid, ids);
+    }
+    nxt_ready = false;
+    if (!stale && i + 1 < n_e && t + 1 < hi) {
+      const int32_t ts1 = ti_seq + 1;
+      if (bs > kTile && static_cast<int64_t>(ts1) * kTile / bs ==
+                            static_cast<int64_t>(ti_seq) * kTile / bs) {
+        nxt[0] = ids[0];  // the next tile reads the same block
       } else {
-        id0 = __ldg(row + idx0);
-        id_row = row;
-        id_idx = idx0;
-        id_val = id0;
+        load_ids(ts1, min(kTile, L_b - ts1 * kTile), nxt);
       }
+      nxt_ready = true;
     }
 
     if (!mbar_wait(empty(stage), phase ^ 1u, p.err)) break;
@@ -289,12 +370,10 @@ __device__ __forceinline__ void produce_tiles(const DecodeParams& p, const CUten
     };
     if (bs <= kTile) {
 #pragma unroll
-      for (int kk = 0; kk < kTile / 4; ++kk) {  // at most 4 blocks: block_size >= 4
+      for (int kk = 0; kk < kTile / 4; ++kk) {
         const int tok0 = kk * bs;
         if (kk < bpt && tok0 < valid) {
-          const int64_t idx = idx0 + kk;
-          const int32_t id = kk == 0 ? id0 : __ldg(row + idx);
-          if (pack) check_shared(idx, id);
+          const int32_t id = ids[kk];
           if (id < 0 || id >= p.num_blocks) {
             flag_error(p.err, PA_DEVERR_BAD_BLOCK);
             mask &= ~(((1u << bs) - 1u) << tok0);
@@ -304,12 +383,11 @@ __device__ __forceinline__ void produce_tiles(const DecodeParams& p, const CUten
         }
       }
     } else if (!stale) {
-      if (pack) check_shared(idx0, id0);
-      if (id0 < 0 || id0 >= p.num_blocks) {
+      if (ids[0] < 0 || ids[0] >= p.num_blocks) {
         flag_error(p.err, PA_DEVERR_BAD_BLOCK);
         mask = 0;
       } else {
-        issue(0, static_cast<int32_t>((static_cast<int64_t>(ti_seq) * kTile) % bs), id0);
+        issue(0, static_cast<int32_t>((static_cast<int64_t>(ti_seq) * kTile) % bs), ids[0]);
       }
     }
     TileInfo& ti = info[stage];

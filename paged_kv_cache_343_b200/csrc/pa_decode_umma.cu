@@ -29,8 +29,8 @@
 // products (warp 6) have an issuing thread each, running ahead of and behind
 // the softmax.  Warps 0..3: softmax and epilogue of heads 0..3 (tensor-memory
 // sub-partition = warp), 4: producer (TMA: K/V tiles and each entry's query
-// rows), 5: S issuer and tensor-memory owner, 6: P.V issuer.  Every wait is
-// bounded.
+// rows), 5: S issuer and tensor-memory owner, 6: P.V issuer, 7: checks that
+// a pack's members share the blocks read for them.  Every wait is bounded.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -115,8 +115,7 @@ __global__ void __launch_bounds__(kUThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int hg = blockIdx.y;
-  const int c = blockIdx.x;
-  const int64_t C = p.ctas_per_group;
+  const int c = p.cta_base + blockIdx.x;  // this CTA's share of the line (LineCut)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) {
@@ -164,10 +163,9 @@ __global__ void __launch_bounds__(kUThreads, 1)
 
   int64_t lo = 0, hi = 0;
   if (host_plan_matches(p)) {
-    const int E = p.meta[1];
-    const int64_t N = p.plan_tiles[E];
-    lo = static_cast<int64_t>(c) * N / C;
-    hi = static_cast<int64_t>(c + 1) * N / C;
+    const LineCut cut = line_cut(p, p.plan_tiles[p.meta[1]]);
+    lo = cut.lo(c);
+    hi = cut.lo(c + 1);
   } else if (threadIdx.x == 0 && c == 0 && hg == 0) {
     flag_error(p.err, PA_DEVERR_BAD_PLAN);
   }
@@ -279,6 +277,9 @@ __global__ void __launch_bounds__(kUThreads, 1)
           mbar_wait(pv_done(static_cast<int>(pv_issued % kUBufs)),
                     static_cast<uint32_t>((pv_issued / kUBufs) & 1), p.err);
       }
+    } else if (warp == 7) {
+      // ======================= pack tables =======================
+      check_pack_tables(p, lo, hi, c, lane, 32);
     } else if (warp < kUH) {
       // ======================= softmax + epilogue =======================
       const int h = warp;        // KV head inside the CTA (= tensor-memory sub-partition)
@@ -435,8 +436,7 @@ __global__ void __launch_bounds__(kUThreads, 1)
           const int r = cdiv;
           const int64_t orow =
               (static_cast<int64_t>(ti.qrow0) + r) * p.num_q_heads + kvh * G + (col - r * G);
-          const int64_t prow =
-              ((static_cast<int64_t>(hg) * p.nseg_cap + ti.seg) * kUH + h) * p.cols + col;
+          const int64_t prow = part_row(p, ti.seg, kvh, col);
 #pragma unroll 1
           for (int kk = 0; kk < 8; ++kk) {
             uint32_t o[16];

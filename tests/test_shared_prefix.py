@@ -94,7 +94,7 @@ def _check(pa, orc, spec, partition_size=0, expect_packs=True):
 
 def test_reduced_shared_prefix_matches_oracle(pa, orc):
     """The benchmark's shape (8 samples of a 2047-token prompt, 4 query heads
-    per KV head: packs of 2) at 2 prompts."""
+    per KV head: packs of 8) at 2 prompts."""
     _check(pa, orc, _spec())
 
 
@@ -133,6 +133,13 @@ def test_prefix_ends_on_a_tile(pa, orc):
     """A 256-token prompt and samples with 0..2 extra tokens: some sequences
     are attended entirely through their pack (their own entry has no tiles)."""
     _check(pa, orc, _spec(prompts=3, samples=4, prompt_len=256, extra_lo=0, extra_hi=2))
+
+
+def test_every_tile_in_a_pack(pa, orc):
+    """A 256-token prompt and no extra tokens: every tile of every sequence is
+    attended through its pack, so the sequences' own tiles (the second part
+    of the tile line) are empty."""
+    _check(pa, orc, _spec(prompts=3, samples=8, prompt_len=256, extra_lo=0, extra_hi=0))
 
 
 def test_short_prompt_is_not_packed(pa, orc):
