@@ -103,7 +103,24 @@ __device__ __forceinline__ int32_t block_exclusive_scan(int32_t v, int32_t* warp
 __device__ int32_t plan_sequence_segments(const DecodeParams& p, int32_t b, int64_t t0,
                                           int64_t t1, const LineCut& cut) {
   int64_t c = cut.count_below(t0);  // first CTA with lo(c) >= t0
-  int64_t lo_c = c < cut.C ? cut.lo(c) : INT64_MAX;
+  // lo(c) stepped in order without a division per CTA: inside a piece of
+  // the cut (Np tiles over Cp CTAs from tile base), lo(c0) = base +
+  // floor(c0 Np / Cp) and lo(c0 + 1) = lo(c0) + q + [rem + r >= Cp] with
+  // q, r = Np / Cp, Np % Cp and rem = c0 r % Cp
+  int64_t lo_c = INT64_MAX, q = 0, r = 0, rem = 0, Cp = 1;
+  auto enter_piece = [&]() {
+    if (c >= cut.C) { lo_c = INT64_MAX; return; }
+    const bool second = cut.S > 0 && c >= cut.S;
+    const int64_t base = second ? cut.NK : 0;
+    const int64_t Np = cut.S == 0 ? cut.N : (second ? cut.N - cut.NK : cut.NK);
+    const int64_t c0 = second ? c - cut.S : c;
+    Cp = cut.S == 0 ? cut.C : (second ? cut.C - cut.S : cut.S);
+    q = Np / Cp;
+    r = Np % Cp;
+    lo_c = base + c0 * q + (c0 * r) / Cp;
+    rem = (c0 * r) % Cp;
+  };
+  enter_piece();
   int64_t part = t0;                 // next partition start
   const int64_t tpp = p.tiles_per_part;
   int32_t count = 0;
@@ -118,7 +135,13 @@ __device__ int32_t plan_sequence_segments(const DecodeParams& p, int32_t b, int6
       p.start_seq[c] = b;
       p.first_k[c] = idx;
       ++c;
-      lo_c = c < cut.C ? cut.lo(c) : INT64_MAX;
+      if (c >= cut.C || c == cut.S) {
+        enter_piece();
+      } else {
+        rem += r;
+        lo_c += q;
+        if (rem >= Cp) { rem -= Cp; ++lo_c; }
+      }
     } else {
       if (part_pt != last) { ++count; last = part_pt; }
       part = (tpp == INT_MAX) ? INT64_MAX : part + tpp;
@@ -1532,6 +1555,7 @@ pa_status setup_decode(void* out, pa_dtype out_dtype, const void* query, pa_dtyp
   p.max_seq_len = max_seq_len;
   p.num_q_heads = num_q_heads;
   p.group = num_q_heads / num_kv_heads;
+  p.num_kv_heads = num_kv_heads;
   p.num_blocks = num_blocks;
   p.block_size = block_size;
   p.tiles_per_part = lp.tiles_per_part;

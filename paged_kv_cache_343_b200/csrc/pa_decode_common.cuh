@@ -47,7 +47,7 @@ struct DecodeParams {
   const int32_t* seq_lens;
   int64_t table_stride;
   int32_t out_dtype;
-  int32_t num_seqs, max_seq_len, num_q_heads, group, num_blocks, block_size;
+  int32_t num_seqs, max_seq_len, num_q_heads, num_kv_heads, group, num_blocks, block_size;
   int32_t num_rows;        // query (and output) rows: num_seqs, or the multi-query rows
   int32_t tiles_per_part;  // partition length in tiles (INT_MAX: no partitions)
   float scale_log2;        // scale * log2(e)
@@ -138,7 +138,7 @@ __device__ __forceinline__ LineCut line_cut(const DecodeParams& p, int64_t N) {
 // Row of (segment, KV head, column) in the partial buffers.
 __host__ __device__ __forceinline__ int64_t part_row(const DecodeParams& p, int64_t seg, int kvh,
                                                      int col) {
-  return (seg * (p.num_q_heads / p.group) + kvh) * p.cols + col;
+  return (seg * p.num_kv_heads + kvh) * p.cols + col;
 }
 
 // Limit of the consumers' waits for the next call's kernels (host side; see
@@ -208,8 +208,8 @@ __device__ __forceinline__ void check_pack_tables(const DecodeParams& p, int64_t
 // ---------------------------------------------------------------------------
 // The producer warp's loop (one elected lane), shared by the decode kernels:
 // walks the CTA's tiles [lo, hi) of the tile line entry by entry, looks up
-// each tile's block ids (one tile ahead, one table lookup per block), loads
-// its K and V with TMA into the stage ring (full_k / full_v of stage s at full_k0 + 8 s ...;
+// each tile's block ids (one table lookup per block), loads its K and V with
+// TMA into the stage ring (full_k / full_v of stage s at full_k0 + 8 s ...;
 // a stage is reused once empty[s] completes), and publishes each tile's
 // TileInfo.  on_entry(n, qrow0) runs after the first tile of the CTA's n-th
 // entry has been published (n = 0, 1, ...); returning false stops the loop.
@@ -281,20 +281,11 @@ __device__ __forceinline__ void produce_tiles(const DecodeParams& p, const CUten
   int stage = 0;
   uint32_t phase = 0;
   int64_t issued = 0;
-  // Block ids of the tile after this one (same entry), loaded one tile ahead
-  // so that their latency hides behind this tile's wait and copies.  Only the
-  // ids a tile reads are loaded: blocks holding valid tokens.
-  int32_t nxt[kTile / 4];
-  bool nxt_ready = false;
-  auto load_ids = [&](int32_t ts, int32_t v, int32_t* ids) {
-    if (bs <= kTile) {
-#pragma unroll
-      for (int kk = 0; kk < kTile / 4; ++kk)  // at most 4 blocks: block_size >= 4
-        ids[kk] = (kk < bpt && kk * bs < v) ? ld_early(row + static_cast<int64_t>(ts) * bpt + kk) : -1;
-    } else {
-      ids[0] = ld_early(row + static_cast<int64_t>(ts) * kTile / bs);
-    }
-  };
+  // blocks longer than a tile: the id of the block the last tile read, so a
+  // block's tiles after its first reuse it (one table lookup per block)
+  const int32_t* id_row = nullptr;
+  int64_t id_idx = -1;
+  int32_t id_val = -1;
   // Tile index inside its partition: segments start at the CTA's first
   // tile, at an entry's first tile and at every partition start, and end
   // before the next start or at the CTA's last tile.
@@ -307,7 +298,6 @@ __device__ __forceinline__ void produce_tiles(const DecodeParams& p, const CUten
       i = 0;
       ip = 0;
       new_seq = true;
-      nxt_ready = false;
     }
     const int32_t ti_seq = i0 + i;  // tile index inside the sequence
     const int32_t valid = stale ? 0 : min(kTile, L_b - ti_seq * kTile);
@@ -323,23 +313,19 @@ __device__ __forceinline__ void produce_tiles(const DecodeParams& p, const CUten
     new_seq = false;
     if (++ip == tpp) ip = 0;
     uint32_t mask = valid >= kTile ? 0xffffu : ((1u << valid) - 1u);
-    int32_t ids[kTile / 4];
-    if (nxt_ready) {
-#pragma unroll
-      for (int kk = 0; kk < kTile / 4; ++kk) ids[kk] = nxt[kk];
-    } else if (!stale) {
-      load_ids(ti_seq, valid, ids);
-    }
-    nxt_ready = false;
-    if (!stale && i + 1 < n_e && t + 1 < hi) {
-      const int32_t ts1 = ti_seq + 1;
-      if (bs > kTile && static_cast<int64_t>(ts1) * kTile / bs ==
-                            static_cast<int64_t>(ti_seq) * kTile / bs) {
-        nxt[0] = ids[0];  // the next tile reads the same block
+    // the first block id is loaded before the wait for a free stage
+    const int64_t idx0 = bs <= kTile ? static_cast<int64_t>(ti_seq) * bpt
+                                     : static_cast<int64_t>(ti_seq) * kTile / bs;
+    int32_t id0 = -1;
+    if (!stale) {
+      if (bs > kTile && row == id_row && idx0 == id_idx) {
+        id0 = id_val;
       } else {
-        load_ids(ts1, min(kTile, L_b - ts1 * kTile), nxt);
+        id0 = __ldg(row + idx0);
+        id_row = row;
+        id_idx = idx0;
+        id_val = id0;
       }
-      nxt_ready = true;
     }
 
     if (!mbar_wait(empty(stage), phase ^ 1u, p.err)) break;
@@ -373,7 +359,7 @@ __device__ __forceinline__ void produce_tiles(const DecodeParams& p, const CUten
       for (int kk = 0; kk < kTile / 4; ++kk) {
         const int tok0 = kk * bs;
         if (kk < bpt && tok0 < valid) {
-          const int32_t id = ids[kk];
+          const int32_t id = kk == 0 ? id0 : __ldg(row + idx0 + kk);
           if (id < 0 || id >= p.num_blocks) {
             flag_error(p.err, PA_DEVERR_BAD_BLOCK);
             mask &= ~(((1u << bs) - 1u) << tok0);
@@ -383,11 +369,11 @@ __device__ __forceinline__ void produce_tiles(const DecodeParams& p, const CUten
         }
       }
     } else if (!stale) {
-      if (ids[0] < 0 || ids[0] >= p.num_blocks) {
+      if (id0 < 0 || id0 >= p.num_blocks) {
         flag_error(p.err, PA_DEVERR_BAD_BLOCK);
         mask = 0;
       } else {
-        issue(0, static_cast<int32_t>((static_cast<int64_t>(ti_seq) * kTile) % bs), ids[0]);
+        issue(0, static_cast<int32_t>((static_cast<int64_t>(ti_seq) * kTile) % bs), id0);
       }
     }
     TileInfo& ti = info[stage];

@@ -125,15 +125,6 @@ __device__ __forceinline__ void griddep_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
-// Read-only 32-bit load issued exactly where it stands: the compiler may move
-// an ordinary read-only load next to its first use, which would undo a load
-// issued early on purpose to hide its latency.
-__device__ __forceinline__ int32_t ld_early(const int32_t* ptr) {
-  int32_t v;
-  asm volatile("ld.global.nc.b32 %0, [%1];" : "=r"(v) : "l"(ptr));
-  return v;
-}
-
 // ---------------------------------------------------------------- TMA
 __device__ __forceinline__ void prefetch_tmap(const void* tmap) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap))
