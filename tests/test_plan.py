@@ -110,3 +110,32 @@ def test_split_plan_refuses_bad_arguments(pa):
         pa.split_plan([5, 30], 200, 24, 4)
     with pytest.raises(m.PagedAttnError):      # no CTA
         pa.split_plan([5, 30], 200, 0, 0)
+
+
+def test_line_cut_matches_the_definition(tmp_path):
+    """The cut of the tile line into CTA shares that the plan kernel and the
+    decode kernels share (LineCut): a host program built by nvcc with the
+    library's flags checks it against its definition written out as loops
+    (even shares, the packs' tiles and the sequences' tiles cut separately
+    when a shared-prompt call runs two kernels, and the count of shares
+    starting below every tile) on the benchmark's shapes, edge cases and 400
+    random ones."""
+    import os
+    import shutil
+    import subprocess
+    nvcc = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
+    if not os.path.exists(nvcc) and shutil.which("nvcc") is None:
+        pytest.skip("no nvcc")
+    if not os.path.exists(nvcc):
+        nvcc = shutil.which("nvcc")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    exe = tmp_path / "linecut_check"
+    build = subprocess.run(
+        [nvcc, "-gencode", "arch=compute_100a,code=sm_100a", "-O2", "-std=c++17",
+         "--expt-relaxed-constexpr", "-I", os.path.join(root, "include"),
+         os.path.join(root, "tests", "c", "linecut_check.cu"), "-o", str(exe)],
+        capture_output=True, text=True, timeout=300)
+    assert build.returncode == 0, build.stderr
+    run = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
+    assert run.returncode == 0, run.stdout + run.stderr
+    assert "all checks held" in run.stdout
