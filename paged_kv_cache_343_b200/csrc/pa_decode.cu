@@ -1168,9 +1168,9 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 // K and V tiles within a 200 KiB budget (at most 6), the kernel, threads,
 // dynamic shared memory and resident CTAs per SM (opting into the memory).
 pa_status warp_kernel_shape(int D, int HG, int NB, int CG, bool bf16, bool fp8, MainKernel* kernel,
-                            int* stages, size_t* smem, int* threads, int* per_sm) {
+                            int* stages, size_t* smem, int* threads, int* per_sm,
+                            size_t budget = 200 * 1024) {
   const size_t tile_bytes = static_cast<size_t>(kTile) * HG * D * (fp8 ? 1 : 2);
-  const size_t budget = 200 * 1024;
   int ns = static_cast<int>(budget / (2 * tile_bytes));
   if (ns > 6) ns = 6;
   if (ns < 2) return PA_ERR_UNSUPPORTED;
@@ -1241,6 +1241,15 @@ pa_status make_plan(int32_t num_seqs, int32_t Hq, int32_t Hkv, int32_t D, int32_
   const bool umma = (P > 1 || Qc > 0) && entry_cols >= kMaxPackCols && !fp8 && D == 128 &&
                     32 % G == 0 && TB == kTile && Hkv % 4 == 0;
   if (umma) HG = 4;
+  // fp8 caches: two CTAs of four KV heads per SM (stages within 100 KiB)
+  // rather than one of eight, so twice the warps hide the per-tile chain of
+  // the code conversion and the MMAs (the 16-bit decode is HBM-bound and
+  // keeps eight heads per CTA: 0.5% faster in a same-GPU A/B)
+  size_t budget = 200 * 1024;
+  if (fp8 && HG == 8) {
+    HG = 4;
+    budget = 100 * 1024;
+  }
   lp->HG = HG;
   lp->head_dim = D;
   lp->groups = Hkv / HG;
@@ -1267,7 +1276,7 @@ pa_status make_plan(int32_t num_seqs, int32_t Hq, int32_t Hkv, int32_t D, int32_
   } else {
     int threads = 0;
     const pa_status st = warp_kernel_shape(D, HG, NB, CG, bf16, fp8, &lp->kernel, &lp->stages,
-                                           &lp->smem, &threads, &per_sm);
+                                           &lp->smem, &threads, &per_sm, budget);
     if (st != PA_OK) return st;
   }
   const int total_ctas = dev->num_sms * per_sm;
@@ -1279,11 +1288,11 @@ pa_status make_plan(int32_t num_seqs, int32_t Hq, int32_t Hkv, int32_t D, int32_
     // warp-level kernel with one column block per head, run after it.  A
     // sequence entry is short and narrow; on the tensor-memory kernel it
     // would cost a query load, an epilogue and whole products.
-    int HGb = 8;
+    int HGb = 4;
     while (Hkv % HGb != 0) HGb >>= 1;
     int per_sm_b = 0;
     const pa_status st = warp_kernel_shape(D, HGb, 1, 1, bf16, false, &lp->kernel, &lp->stages_b,
-                                           &lp->smem_b, &lp->threads_b, &per_sm_b);
+                                           &lp->smem_b, &lp->threads_b, &per_sm_b, 100 * 1024);
     if (st != PA_OK) return st;
     lp->split = true;
     lp->HG_b = HGb;
