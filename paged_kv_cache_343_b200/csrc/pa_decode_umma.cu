@@ -50,6 +50,7 @@ constexpr int kUThreads = kUmmaThreads;      // 8 warps
 constexpr float kLazyLog2 = 8.0f;            // growth of a row maximum that forces a rescale
 constexpr uint32_t kUTileBytes = kTile * kUH * kUD * 2;  // K (or V) of one tile: 16 KiB
 constexpr uint32_t kUQBytes = 2 * 128 * 128;             // query rows of an entry: 32 KiB
+constexpr int kUQBufs = 2;                               // query buffers (entries in flight)
 // tensor-memory columns: O [0, 128), three S buffers [128, 320), three P
 // buffers of two halves [320, 512)
 constexpr int kUBufs = 3;
@@ -66,7 +67,7 @@ struct UmmaLayout {
 __host__ __device__ inline UmmaLayout umma_layout(int NS) {
   UmmaLayout L;
   L.q = static_cast<uint32_t>(NS) * 2u * kUTileBytes;  // stages first
-  L.info = L.q + 2u * kUQBytes;                        // two query buffers
+  L.info = L.q + static_cast<uint32_t>(kUQBufs) * kUQBytes;  // the query buffers
   L.bars = L.info + static_cast<uint32_t>(NS) * sizeof(TileInfo);
   L.bars = (L.bars + 7u) & ~7u;
   const uint32_t nbars = 3u * NS + 17u;
@@ -123,7 +124,7 @@ __global__ void __launch_bounds__(kUThreads, 1)
       mbar_init(full_v(s), 1);
       mbar_init(empty(s), 1);      // the P.V issuer's commit after the tile's products
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < kUQBufs; ++b) {
       mbar_init(q_full(b), 1);
       mbar_init(q_free(b), 1);     // the S issuer's commit
     }
@@ -179,8 +180,10 @@ __global__ void __launch_bounds__(kUThreads, 1)
         produce_tiles<kUH, 2>(
             p, &tmK, &tmV, base, kUTileBytes, info, full_k(0), full_v(0), empty(0), NS, lo, hi,
             c, hg, false, [&](int32_t n, int32_t qrow0) {
-              const int qb = n & 1;
-              if (n >= 2 && !mbar_wait(q_free(qb), static_cast<uint32_t>((n - 2) >> 1) & 1u, p.err))
+              const int qb = n % kUQBufs;
+              if (n >= kUQBufs &&
+                  !mbar_wait(q_free(qb), static_cast<uint32_t>((n - kUQBufs) / kUQBufs) & 1u,
+                             p.err))
                 return false;
               // one box per (head, d-chunk): 32 / G query rows of the G query
               // heads of KV head h, i.e. the entry's 32 columns of that head
@@ -192,9 +195,10 @@ __global__ void __launch_bounds__(kUThreads, 1)
               last_n = n;
               return true;
             });
-        // the last (up to two) query loads have landed before the CTA retires
-        for (int32_t n = last_n > 0 ? last_n - 1 : 0; n <= last_n; ++n)
-          if (!mbar_wait(q_full(n & 1), static_cast<uint32_t>(n >> 1) & 1u, p.err)) break;
+        // the last query loads (one per buffer) have landed before the CTA retires
+        for (int32_t n = last_n >= kUQBufs ? last_n - kUQBufs + 1 : 0; n <= last_n; ++n)
+          if (!mbar_wait(q_full(n % kUQBufs), static_cast<uint32_t>(n / kUQBufs) & 1u, p.err))
+            break;
       }
     } else if (warp == 5) {
       // ======================= S issuer =======================
@@ -208,15 +212,16 @@ __global__ void __launch_bounds__(kUThreads, 1)
           if (info[s].flags & kNewSeq) {
             ++n_entry;
             // the previous entry's query buffer is free once its products finish
-            if (n_entry >= 1) umma_commit(q_free((n_entry - 1) & 1));
-            if (!mbar_wait(q_full(n_entry & 1), static_cast<uint32_t>(n_entry >> 1) & 1u, p.err))
+            if (n_entry >= 1) umma_commit(q_free((n_entry - 1) % kUQBufs));
+            if (!mbar_wait(q_full(n_entry % kUQBufs), static_cast<uint32_t>(n_entry / kUQBufs) & 1u,
+                           p.err))
               break;
           }
           if (u >= kUBufs &&
               !mbar_wait(s_free(j), static_cast<uint32_t>((u / kUBufs - 1) & 1), p.err))
             break;
           tc_fence_after();
-          const uint32_t qa = q_addr(n_entry & 1), ka = k_addr(s);
+          const uint32_t qa = q_addr(n_entry % kUQBufs), ka = k_addr(s);
           const uint32_t d = tmem + kColS + static_cast<uint32_t>(j) * 64u;
 #pragma unroll
           for (int kc = 0; kc < 8; ++kc) {
