@@ -447,8 +447,13 @@ pa_status pa_decode_attention_shared_prefix(void* out, pa_dtype out_dtype, const
  *   partition_size (0 or a multiple of 16), on host arrays: tiles[num_seqs+1]
  *   (tile prefix sums), seg_base[num_seqs+1] (segment prefix sums),
  *   start_seq[num_ctas] and first_k[num_ctas] (the sequence holding CTA c's
- *   first tile and the index of the segment starting there), *num_segments and
- *   *needs_combine.  Needs no GPU.
+ *   first tile and the index of the segment starting there),
+ *   cta_first_tile[num_ctas+1] (the first tile of CTA c's share; the last
+ *   entry is the tile count), *num_segments and *needs_combine.  The shares
+ *   cut the line evenly in weighted tiles: a sequence with tiles counts
+ *   PA_PLAN_ENTRY_WEIGHT tiles more (the cost of a CTA moving to it, placed
+ *   before its first tile) when num_seqs <= PA_PLAN_WEIGHTED_MAX_ENTRIES, else
+ *   nothing more.  Needs no GPU.
  * ------------------------------------------------------------------------- */
 pa_status pa_decode_plan_bytes(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
                                int32_t head_dim, int32_t block_size, int32_t max_seq_len,
@@ -470,10 +475,12 @@ pa_status pa_decode_attention_planned(void* out, pa_dtype out_dtype, const void*
                                       int32_t block_size, float scale, int32_t partition_size,
                                       const void* plan, void* workspace, size_t workspace_bytes,
                                       int32_t* device_error_flag, pa_stream_t stream);
+#define PA_PLAN_ENTRY_WEIGHT 2
+#define PA_PLAN_WEIGHTED_MAX_ENTRIES 4096
 pa_status pa_split_plan(const int32_t* seq_lens, int32_t num_seqs, int32_t max_seq_len,
                         int32_t partition_size, int32_t num_ctas, int32_t* tiles,
                         int32_t* seg_base, int32_t* start_seq, int32_t* first_k,
-                        int32_t* num_segments, int32_t* needs_combine);
+                        int32_t* cta_first_tile, int32_t* num_segments, int32_t* needs_combine);
 
 /* ---------------------------------------------------------------------------
  * pa_decode_step -- one decode step of a batch, driven from host memory:

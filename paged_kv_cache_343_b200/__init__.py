@@ -183,7 +183,7 @@ def _load() -> ctypes.CDLL:
                                                 ctypes.c_int, p, p, p, i32, p, i32, i32, i32, i32,
                                                 i32, i32, i32, ctypes.c_float, i32, p, p, sz, p, p]
     lib.pa_split_plan.restype = ctypes.c_int
-    lib.pa_split_plan.argtypes = [p, i32, i32, i32, i32, p, p, p, p, ctypes.POINTER(i32),
+    lib.pa_split_plan.argtypes = [p, i32, i32, i32, i32, p, p, p, p, p, ctypes.POINTER(i32),
                                   ctypes.POINTER(i32)]
     lib.pa_decode_step_layout.restype = ctypes.c_int
     lib.pa_decode_step_layout.argtypes = [ctypes.POINTER(StepShape), ctypes.POINTER(StepLayout)]
@@ -654,7 +654,8 @@ def decode_attention_planned(out: torch.Tensor, query: torch.Tensor, key_cache: 
 
 def split_plan(seq_lens, max_seq_len: int, partition_size: int, num_ctas: int) -> dict:
     """pa_split_plan on host lengths (no GPU): the tile and segment prefix
-    sums and each CTA's start, as numpy arrays."""
+    sums, each CTA's start and the first tile of each CTA's share, as numpy
+    arrays."""
     import numpy as np
     lens = np.ascontiguousarray(np.asarray(seq_lens, dtype=np.int32))
     B = lens.size
@@ -662,13 +663,15 @@ def split_plan(seq_lens, max_seq_len: int, partition_size: int, num_ctas: int) -
     segs = np.zeros(B + 1, np.int32)
     start = np.zeros(num_ctas, np.int32)
     firstk = np.zeros(num_ctas, np.int32)
+    ctalo = np.zeros(num_ctas + 1, np.int32)
     nseg, comb = ctypes.c_int32(0), ctypes.c_int32(0)
     vp = lambda a: ctypes.c_void_p(a.ctypes.data)
     _check(lib.pa_split_plan(vp(lens), B, int(max_seq_len), int(partition_size), int(num_ctas),
-                             vp(tiles), vp(segs), vp(start), vp(firstk), ctypes.byref(nseg),
-                             ctypes.byref(comb)), "pa_split_plan")
+                             vp(tiles), vp(segs), vp(start), vp(firstk), vp(ctalo),
+                             ctypes.byref(nseg), ctypes.byref(comb)), "pa_split_plan")
     return {"tiles": tiles, "seg_base": segs, "start_seq": start, "first_k": firstk,
-            "num_segments": int(nseg.value), "needs_combine": bool(comb.value)}
+            "cta_first_tile": ctalo, "num_segments": int(nseg.value),
+            "needs_combine": bool(comb.value)}
 
 
 class DecodeStep:

@@ -26,10 +26,12 @@
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <atomic>
 #include <climits>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "pa_decode_common.cuh"
 #include "pa_device.cuh"
@@ -96,37 +98,30 @@ __device__ __forceinline__ int32_t block_exclusive_scan(int32_t v, int32_t* warp
   return before;
 }
 
+// Smallest c in [0, C] with lo[c] >= x, i.e. the number of CTA shares that
+// start below x (lo non-decreasing, lo[C] = N >= x).
+__device__ __forceinline__ int32_t ctas_below(const int32_t* lo, int32_t C, int64_t x) {
+  int32_t a = 0, z = C;  // the answer is in [a, z]
+  while (a < z) {
+    const int32_t mid = (a + z) >> 1;
+    if (lo[mid] < x) a = mid + 1; else z = mid;
+  }
+  return a;
+}
+
 // Walks the segment starts of entry b (tiles [t0, t1)) in order: the
-// partition starts and the CTA-share starts, equal points counted once.
-// Records start_seq / first_k for every CTA whose share starts inside b and
-// returns the number of segments.
+// partition starts and the CTA-share starts (lo[c]), equal points counted
+// once.  Records start_seq / first_k for every CTA whose share starts inside
+// b and returns the number of segments.
 __device__ int32_t plan_sequence_segments(const DecodeParams& p, int32_t b, int64_t t0,
-                                          int64_t t1, const LineCut& cut) {
-  int64_t c = cut.count_below(t0);  // first CTA with lo(c) >= t0
-  // lo(c) stepped in order without a division per CTA: inside a piece of
-  // the cut (Np tiles over Cp CTAs from tile base), lo(c0) = base +
-  // floor(c0 Np / Cp) and lo(c0 + 1) = lo(c0) + q + [rem + r >= Cp] with
-  // q, r = Np / Cp, Np % Cp and rem = c0 r % Cp
-  int64_t lo_c = INT64_MAX, q = 0, r = 0, rem = 0, Cp = 1;
-  auto enter_piece = [&]() {
-    if (c >= cut.C) { lo_c = INT64_MAX; return; }
-    const bool second = cut.S > 0 && c >= cut.S;
-    const int64_t base = second ? cut.NK : 0;
-    const int64_t Np = cut.S == 0 ? cut.N : (second ? cut.N - cut.NK : cut.NK);
-    const int64_t c0 = second ? c - cut.S : c;
-    Cp = cut.S == 0 ? cut.C : (second ? cut.C - cut.S : cut.S);
-    q = Np / Cp;
-    r = Np % Cp;
-    lo_c = base + c0 * q + (c0 * r) / Cp;
-    rem = (c0 * r) % Cp;
-  };
-  enter_piece();
-  int64_t part = t0;                 // next partition start
+                                          int64_t t1, const int32_t* lo, int32_t C) {
+  int32_t c = ctas_below(lo, C, t0);  // first CTA with lo(c) >= t0
+  int64_t part = t0;                  // next partition start
   const int64_t tpp = p.tiles_per_part;
   int32_t count = 0;
   int64_t last = -1;
   while (true) {
-    const int64_t cta_pt = (c < cut.C && lo_c < t1) ? lo_c : INT64_MAX;
+    const int64_t cta_pt = (c < C && lo[c] < t1) ? lo[c] : INT64_MAX;
     const int64_t part_pt = part < t1 ? part : INT64_MAX;
     if (cta_pt == INT64_MAX && part_pt == INT64_MAX) break;
     if (cta_pt <= part_pt) {
@@ -135,13 +130,6 @@ __device__ int32_t plan_sequence_segments(const DecodeParams& p, int32_t b, int6
       p.start_seq[c] = b;
       p.first_k[c] = idx;
       ++c;
-      if (c >= cut.C || c == cut.S) {
-        enter_piece();
-      } else {
-        rem += r;
-        lo_c += q;
-        if (rem >= Cp) { rem -= Cp; ++lo_c; }
-      }
     } else {
       if (part_pt != last) { ++count; last = part_pt; }
       part = (tpp == INT_MAX) ? INT64_MAX : part + tpp;
@@ -167,6 +155,7 @@ __global__ void __launch_bounds__(kPlanThreads) pa_plan_kernel(DecodeParams p) {
   __shared__ int32_t warp_buf[kPlanWarps];
   __shared__ int32_t s_tiles[kPlanSmemTiles + 1];
   __shared__ int32_t s_sd[kPlanMaxCtas + 1], s_sdc[kPlanMaxCtas + 1];
+  __shared__ int32_t s_lo[kPlanMaxCtas + 1];  // first tile of each CTA's share
   const int tid = threadIdx.x;
   const int B = p.num_seqs;
   griddep_launch_dependents();
@@ -316,12 +305,52 @@ __global__ void __launch_bounds__(kPlanThreads) pa_plan_kernel(DecodeParams p) {
   const int64_t N = carry;
   const int C = p.ctas_per_group;
   const int32_t tpp = p.tiles_per_part;
-  const int32_t* tiles = E <= kPlanSmemTiles ? s_tiles : p.plan_tiles;
+  const bool in_smem = E <= kPlanSmemTiles;
+  const int32_t* tiles = in_smem ? s_tiles : p.plan_tiles;
+  // ---- the cut: CTA c's share starts at tile s_lo[c] (also cta_lo[c]).  The
+  // line is cut evenly (LineCut; with a split, the packs and the sequences
+  // separately) in virtual tiles, where an entry with tiles counts
+  // kEntryWeight more (its switch first); each cut is then mapped back to the
+  // real tile at that virtual position.  The virtual starts live in s_tiles
+  // while the cut is made, so only a batch whose prefix sums fit there is
+  // weighted.
+  const int64_t w = in_smem ? kEntryWeight : 0;
   LineCut cut;
   cut.C = C;
   cut.S = p.split_ctas;
-  cut.N = N;
-  cut.NK = p.split_ctas > 0 ? tiles[K] : 0;
+  if (w > 0) {
+    int32_t vcarry = 0, vtot = 0;
+    for (int ch = 0; ch < nchunks; ++ch) {
+      const int e = ch * kPlanThreads + tid;
+      const int32_t has = (e < E && p.plan_tiles[e + 1] > p.plan_tiles[e]) ? 1 : 0;
+      const int32_t ex = block_exclusive_scan(has, warp_buf, &vtot);
+      if (e < E) s_tiles[e] = p.plan_tiles[e] + static_cast<int32_t>(w) * (vcarry + ex);
+      vcarry += vtot;
+    }
+    if (tid == 0) s_tiles[E] = static_cast<int32_t>(N + w * vcarry);
+    __syncthreads();
+    cut.N = s_tiles[E];
+    cut.NK = p.split_ctas > 0 ? s_tiles[K] : 0;
+    for (int c = tid; c <= C; c += kPlanThreads) {
+      const int64_t x = cut.lo(c);
+      const int e = upper_entry(s_tiles, E + 1, x);
+      const int64_t t = e >= E ? N
+                               : entry_tile(x, s_tiles[e], p.plan_tiles[e],
+                                            p.plan_tiles[e + 1] - p.plan_tiles[e], w);
+      s_lo[c] = static_cast<int32_t>(t);
+      p.cta_lo[c] = static_cast<int32_t>(t);
+    }
+    __syncthreads();  // s_tiles is read above until here
+    for (int e = tid; e <= E; e += kPlanThreads) s_tiles[e] = p.plan_tiles[e];
+  } else {
+    cut.N = N;
+    cut.NK = p.split_ctas > 0 ? tiles[K] : 0;
+    for (int c = tid; c <= C; c += kPlanThreads) {
+      s_lo[c] = static_cast<int32_t>(cut.lo(c));
+      p.cta_lo[c] = s_lo[c];
+    }
+  }
+  __syncthreads();  // s_lo and the real prefix sums are read below
   if (!p.plan_closed) {  // few cut points per entry: walk them
     int32_t seg_carry = 0;
     for (int ch = 0; ch < nchunks; ++ch) {
@@ -329,7 +358,7 @@ __global__ void __launch_bounds__(kPlanThreads) pa_plan_kernel(DecodeParams p) {
       int32_t ns = 0;
       if (e < E && N > 0) {
         const int64_t t0 = tiles[e], t1 = tiles[e + 1];
-        if (t1 > t0) ns = plan_sequence_segments(p, e, t0, t1, cut);
+        if (t1 > t0) ns = plan_sequence_segments(p, e, t0, t1, s_lo, C);
       }
       const int32_t ex = block_exclusive_scan(ns, warp_buf, &total);
       if (e < E) p.seg_base[e] = seg_carry + ex;
@@ -338,10 +367,8 @@ __global__ void __launch_bounds__(kPlanThreads) pa_plan_kernel(DecodeParams p) {
     if (tid == 0) p.seg_base[E] = seg_carry;
     return;
   }
-  auto lo_of = [&](int64_t c) { return cut.lo(c); };
-  auto cnt_below = [&](int64_t x) {  // CTAs with lo(c) < x
-    return static_cast<int>(cut.count_below(x));
-  };
+  auto lo_of = [&](int64_t c) { return static_cast<int64_t>(s_lo[c]); };
+  auto cnt_below = [&](int64_t x) { return ctas_below(s_lo, C, x); };  // CTAs with lo(c) < x
   // ---- CTAs: the entry holding each share's start; held / coincident flags,
   // scanned together as held + coincident * 2^16 (C <= kPlanMaxCtas < 2^15)
   int32_t sd_carry = 0, sdc_carry = 0;
@@ -476,11 +503,9 @@ __global__ void __launch_bounds__((HG * CG + 1) * 32, 1)
 
   // entries: packs' prefixes then sequences, or query chunks (plain: the B sequences)
   const bool plain = p.pack_size == 1 && p.q_start == nullptr;
-  const int E = plain ? B : p.meta[1];
-  const int64_t N = p.plan_tiles[E];
-  const LineCut cut = line_cut(p, N);
-  const int64_t lo = cut.lo(c);
-  const int64_t hi = cut.lo(c + 1);
+  // this CTA's share of the tile line, as the plan cut it
+  const int64_t lo = p.cta_lo[c];
+  const int64_t hi = p.cta_lo[c + 1];
   if (lo >= hi) return;
 
   if (warp == NW) {
@@ -1156,7 +1181,7 @@ struct LaunchPlan {
   bool split = false;
   int split_ctas = 0, ctas_b = 0, groups_b = 0, HG_b = 0, threads_b = 0, stages_b = 0;
   size_t smem_b = 0;
-  size_t off_tiles = 0, off_segs = 0, off_start = 0, off_firstk = 0, off_meta = 0,
+  size_t off_tiles = 0, off_segs = 0, off_start = 0, off_firstk = 0, off_meta = 0, off_ctalo = 0,
          off_pack_first = 0, off_pack_n = 0, off_pack_tiles = 0, off_seq_pack = 0,
          off_seq_pre = 0, off_ent = 0, off_o = 0, off_ml = 0, total = 0;
   MainKernel kernel = nullptr;
@@ -1334,7 +1359,8 @@ pa_status make_plan(int32_t num_seqs, int32_t Hq, int32_t Hkv, int32_t D, int32_
   lp->off_segs = lp->off_tiles + words(entries + 1);
   lp->off_start = lp->off_segs + words(entries + 1);
   lp->off_firstk = lp->off_start + words(lp->ctas_per_group);
-  lp->off_meta = lp->off_firstk + words(lp->ctas_per_group);
+  lp->off_ctalo = lp->off_firstk + words(lp->ctas_per_group);
+  lp->off_meta = lp->off_ctalo + words(lp->ctas_per_group + 1);
   size_t off = lp->off_meta + words(2);
   if (lp->pack_size > 1) {
     lp->off_pack_first = off;
@@ -1582,6 +1608,7 @@ pa_status setup_decode(void* out, pa_dtype out_dtype, const void* query, pa_dtyp
   p.seg_base = reinterpret_cast<int32_t*>(ws + lp.off_segs);
   p.start_seq = reinterpret_cast<int32_t*>(ws + lp.off_start);
   p.first_k = reinterpret_cast<int32_t*>(ws + lp.off_firstk);
+  p.cta_lo = reinterpret_cast<int32_t*>(ws + lp.off_ctalo);
   p.meta = reinterpret_cast<int32_t*>(ws + lp.off_meta);
   if (q_start != nullptr) {
     p.q_start = q_start;
@@ -1771,12 +1798,12 @@ extern "C" pa_status pa_decode_attention_shared_prefix(
 // query token per sequence, no packs).  Buffer layout (int32 words, 256-byte
 // aligned sections): the header (kPlanHeaderWords), then tile prefix sums
 // [B + 1], segment prefix sums [B + 1], start entry [C] and first segment
-// index [C] of each CTA.
+// index [C] of each CTA, and the first tile of each CTA's share [C + 1].
 // ===========================================================================
 namespace {
 
 struct PlanOffsets {
-  size_t tiles, segs, start, firstk, total;
+  size_t tiles, segs, start, firstk, ctalo, total;
 };
 
 PlanOffsets plan_offsets(int64_t B, int64_t C) {
@@ -1786,7 +1813,8 @@ PlanOffsets plan_offsets(int64_t B, int64_t C) {
   o.segs = o.tiles + words(B + 1);
   o.start = o.segs + words(B + 1);
   o.firstk = o.start + words(C);
-  o.total = o.firstk + words(C);
+  o.ctalo = o.firstk + words(C);
+  o.total = o.ctalo + words(C + 1);
   return o;
 }
 
@@ -1794,13 +1822,15 @@ PlanOffsets plan_offsets(int64_t B, int64_t C) {
 // sequence's cut points in order: the tiles of all sequences laid end to end
 // (tiles[b] = tiles before sequence b), cut wherever a partition starts
 // (every tpp tiles from a sequence's first tile) or a CTA's share starts
-// (lo(c) = floor(c N / C)); seg_base[b] = segments before sequence b;
-// start_seq[c], first_k[c] = the sequence holding lo(c) and the index of the
-// segment starting there.  Lengths are clamped to [0, max_seq_len].  Returns
-// false if the tile count does not fit in int32.
+// (cta_lo[c]: the line cut evenly in virtual tiles, a sequence with tiles
+// counting kEntryWeight more when B fits the plan kernel's shared prefix
+// sums, as the plan kernel cuts it); seg_base[b] = segments before sequence
+// b; start_seq[c], first_k[c] = the sequence holding cta_lo[c] and the index
+// of the segment starting there.  Lengths are clamped to [0, max_seq_len].
+// Returns false if the tile count does not fit in int32.
 bool split_walk(const int32_t* lens, int32_t B, int32_t max_seq_len, int32_t tpp, int32_t C,
                 int32_t* tiles, int32_t* seg_base, int32_t* start_seq, int32_t* first_k,
-                int32_t* total_segs, bool* split) {
+                int32_t* cta_lo, int32_t* total_segs, bool* split) {
   int64_t N = 0;
   for (int32_t b = 0; b < B; ++b) {
     tiles[b] = static_cast<int32_t>(N);
@@ -1809,6 +1839,28 @@ bool split_walk(const int32_t* lens, int32_t B, int32_t max_seq_len, int32_t tpp
     if (N > INT_MAX / 2) return false;
   }
   tiles[B] = static_cast<int32_t>(N);
+  // the cut (the plan kernel's arithmetic): virtual starts, an even cut of
+  // the virtual line, each cut mapped to its real tile
+  const int64_t w = B <= kPlanSmemTiles ? kEntryWeight : 0;
+  std::vector<int64_t> vs(static_cast<size_t>(B) + 1);
+  int64_t nonempty = 0;
+  for (int32_t b = 0; b < B; ++b) {
+    vs[b] = tiles[b] + w * nonempty;
+    if (tiles[b + 1] > tiles[b]) ++nonempty;
+  }
+  vs[B] = N + w * nonempty;
+  LineCut cut;
+  cut.C = C;
+  cut.S = 0;
+  cut.N = vs[B];
+  cut.NK = 0;
+  for (int32_t c = 0; c <= C; ++c) {
+    const int64_t x = cut.lo(c);
+    // the last entry whose virtual start is at or below x
+    const int32_t e = static_cast<int32_t>(std::upper_bound(vs.begin(), vs.end(), x) - vs.begin()) - 1;
+    cta_lo[c] = static_cast<int32_t>(
+        e >= B ? N : entry_tile(x, vs[e], tiles[e], tiles[e + 1] - tiles[e], w));
+  }
   for (int32_t c = 0; c < C; ++c) start_seq[c] = first_k[c] = 0;
   *split = false;
   int64_t seg = 0;
@@ -1816,13 +1868,13 @@ bool split_walk(const int32_t* lens, int32_t B, int32_t max_seq_len, int32_t tpp
     seg_base[b] = static_cast<int32_t>(seg);
     const int64_t t0 = tiles[b], t1 = tiles[b + 1];
     if (t1 <= t0) continue;
-    int64_t c = (t0 * C + N - 1) / N;  // first CTA whose share starts at or after t0
-    int64_t part = t0;                 // next partition start
+    // first CTA whose share starts at or after t0
+    int64_t c = std::lower_bound(cta_lo, cta_lo + C, static_cast<int32_t>(t0)) - cta_lo;
+    int64_t part = t0;  // next partition start
     int32_t count = 0;
     int64_t last = -1;
     while (true) {
-      const int64_t lo_c = c * N / C;
-      const int64_t cta_pt = (c < C && lo_c < t1) ? lo_c : INT64_MAX;
+      const int64_t cta_pt = (c < C && cta_lo[c] < t1) ? cta_lo[c] : INT64_MAX;
       const int64_t part_pt = part < t1 ? part : INT64_MAX;
       if (cta_pt == INT64_MAX && part_pt == INT64_MAX) break;
       if (cta_pt <= part_pt) {
@@ -1864,7 +1916,8 @@ pa_status write_plan(const LaunchPlan& lp, const int32_t* lens, int32_t B, int32
   if (!split_walk(lens, B, max_seq_len, lp.tiles_per_part, C,
                   reinterpret_cast<int32_t*>(buf + o.tiles), reinterpret_cast<int32_t*>(buf + o.segs),
                   reinterpret_cast<int32_t*>(buf + o.start),
-                  reinterpret_cast<int32_t*>(buf + o.firstk), &segs, &split))
+                  reinterpret_cast<int32_t*>(buf + o.firstk),
+                  reinterpret_cast<int32_t*>(buf + o.ctalo), &segs, &split))
     return PA_ERR_UNSUPPORTED;
   if (segs > lp.nseg_cap) return PA_ERR_UNSUPPORTED;  // cannot happen: nseg_cap bounds it
   std::memset(h, 0, kPlanHeaderWords * sizeof(int32_t));
@@ -1888,6 +1941,7 @@ void use_device_plan(DecodeSetup* su, const void* plan) {
   su->p.seg_base = reinterpret_cast<int32_t*>(const_cast<uint8_t*>(d + o.segs));
   su->p.start_seq = reinterpret_cast<int32_t*>(const_cast<uint8_t*>(d + o.start));
   su->p.first_k = reinterpret_cast<int32_t*>(const_cast<uint8_t*>(d + o.firstk));
+  su->p.cta_lo = reinterpret_cast<int32_t*>(const_cast<uint8_t*>(d + o.ctalo));
 }
 
 pa_status plan_shape(int32_t num_seqs, int32_t Hq, int32_t Hkv, int32_t D, int32_t bs,
@@ -1904,19 +1958,20 @@ pa_status plan_shape(int32_t num_seqs, int32_t Hq, int32_t Hkv, int32_t D, int32
 extern "C" pa_status pa_split_plan(const int32_t* seq_lens, int32_t num_seqs, int32_t max_seq_len,
                                    int32_t partition_size, int32_t num_ctas, int32_t* tiles,
                                    int32_t* seg_base, int32_t* start_seq, int32_t* first_k,
-                                   int32_t* num_segments, int32_t* needs_combine) {
+                                   int32_t* cta_first_tile, int32_t* num_segments,
+                                   int32_t* needs_combine) {
   if (num_seqs <= 0 || max_seq_len < 0 || num_ctas <= 0 || num_ctas > kPlanMaxCtas ||
       partition_size < 0 || partition_size % kTile != 0)
     return PA_ERR_INVALID_ARG;
-  if (!seq_lens || !tiles || !seg_base || !start_seq || !first_k || !num_segments ||
-      !needs_combine)
+  if (!seq_lens || !tiles || !seg_base || !start_seq || !first_k || !cta_first_tile ||
+      !num_segments || !needs_combine)
     return PA_ERR_INVALID_ARG;
   for (int32_t b = 0; b < num_seqs; ++b)
     if (seq_lens[b] < 0 || seq_lens[b] > max_seq_len) return PA_ERR_INVALID_ARG;
   const int32_t tpp = partition_size > 0 ? partition_size / kTile : INT_MAX;
   bool split = false;
   if (!split_walk(seq_lens, num_seqs, max_seq_len, tpp, num_ctas, tiles, seg_base, start_seq,
-                  first_k, num_segments, &split))
+                  first_k, cta_first_tile, num_segments, &split))
     return PA_ERR_UNSUPPORTED;
   *needs_combine = split ? 1 : 0;
   return PA_OK;

@@ -65,6 +65,8 @@ struct DecodeParams {
                            //    entry); 0: walk each entry's cut points (few)
   int32_t* plan_tiles;     // [entries + 1] tile prefix sums
   int32_t* seg_base;       // [entries + 1] segment prefix sums (partial slots)
+  int32_t* cta_lo;         // [ctas_per_group + 1] first tile of each CTA's share (LineCut
+                           //    of the weighted line, entry_tile below); [C] = N
   int32_t* start_seq;      // [ctas_per_group] entry holding each CTA's first tile
   int32_t* first_k;        // [ctas_per_group] index of that tile's segment in its entry
   // shared prompts: packs of pack_size consecutive sequences whose block tables
@@ -125,14 +127,20 @@ struct LineCut {
   }
 };
 
-// The cut of a plan whose entries end at tile N (packs end at plan_tiles[K]).
-__device__ __forceinline__ LineCut line_cut(const DecodeParams& p, int64_t N) {
-  LineCut L;
-  L.C = p.ctas_per_group;
-  L.S = p.split_ctas;
-  L.N = N;
-  L.NK = p.split_ctas > 0 ? p.plan_tiles[p.meta[0]] : 0;
-  return L;
+// The cut weighs each entry switch: a CTA whose share spans several entries
+// pays an epilogue, a query load and a pipeline restart per switch, so the
+// line is cut evenly in virtual tiles where an entry with tiles counts its
+// tiles plus kEntryWeight (its switch first).  Batches of more entries than
+// the plan keeps in shared memory are cut unweighted.
+constexpr int kEntryWeight = 2;
+
+// The real tile at virtual position x of an entry that starts at virtual
+// position v_e and real tile t_e and holds n_e tiles (weight w per switch):
+// inside its switch the cut falls on its first tile.
+__host__ __device__ __forceinline__ int64_t entry_tile(int64_t x, int64_t v_e, int64_t t_e,
+                                                       int64_t n_e, int64_t w) {
+  const int64_t o = x - v_e - (n_e > 0 ? w : 0);
+  return t_e + (o < 0 ? 0 : (o > n_e ? n_e : o));
 }
 
 // Row of (segment, KV head, column) in the partial buffers.

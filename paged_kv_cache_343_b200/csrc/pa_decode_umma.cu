@@ -164,9 +164,8 @@ __global__ void __launch_bounds__(kUThreads, 1)
 
   int64_t lo = 0, hi = 0;
   if (host_plan_matches(p)) {
-    const LineCut cut = line_cut(p, p.plan_tiles[p.meta[1]]);
-    lo = cut.lo(c);
-    hi = cut.lo(c + 1);
+    lo = p.cta_lo[c];
+    hi = p.cta_lo[c + 1];
   } else if (threadIdx.x == 0 && c == 0 && hg == 0) {
     flag_error(p.err, PA_DEVERR_BAD_PLAN);
   }

@@ -58,15 +58,21 @@ int main(void) {
     CHECK(pa_decode_step_layout(&sh, &lay) == PA_ERR_UNSUPPORTED);
   }
 
-  /* the split plan on the host: 4 sequences over 7 CTAs */
+  /* the split plan on the host: 4 sequences (1, 3, 0 and 7 tiles) over 7
+   * CTAs.  Weighted line: the three sequences with tiles start at virtual
+   * tiles 0, 3 and 8 (2 more each), 17 in all; cut at 0, 2, 4, 7, 9, 12, 14,
+   * 17 -> first tiles 0, 0, 1, 3, 4, 6, 8, 11 */
   {
     const int32_t lens4[4] = {5, 40, 0, 100};
-    int32_t tiles[5], segs[5], start[7], firstk[7], nseg = -1, comb = -1;
-    CHECK(pa_split_plan(lens4, 4, 128, 0, 7, tiles, segs, start, firstk, &nseg, &comb) == PA_OK);
+    int32_t tiles[5], segs[5], start[7], firstk[7], ctalo[8], nseg = -1, comb = -1;
+    CHECK(pa_split_plan(lens4, 4, 128, 0, 7, tiles, segs, start, firstk, ctalo, &nseg, &comb) ==
+          PA_OK);
     CHECK(tiles[0] == 0 && tiles[1] == 1 && tiles[2] == 4 && tiles[3] == 4 && tiles[4] == 11);
-    CHECK(segs[4] == 7 && nseg == 7 && comb == 1);
-    CHECK(start[2] == 1 && firstk[2] == 1 && start[6] == 3 && firstk[6] == 3);
-    CHECK(pa_split_plan(lens4, 4, 64, 0, 7, tiles, segs, start, firstk, &nseg, &comb) ==
+    CHECK(ctalo[0] == 0 && ctalo[1] == 0 && ctalo[2] == 1 && ctalo[3] == 3 && ctalo[4] == 4 &&
+          ctalo[5] == 6 && ctalo[6] == 8 && ctalo[7] == 11);
+    CHECK(segs[1] == 1 && segs[2] == 3 && segs[3] == 3 && segs[4] == 6 && nseg == 6 && comb == 1);
+    CHECK(start[3] == 1 && firstk[3] == 1 && start[6] == 3 && firstk[6] == 2);
+    CHECK(pa_split_plan(lens4, 4, 64, 0, 7, tiles, segs, start, firstk, ctalo, &nseg, &comb) ==
           PA_ERR_INVALID_ARG); /* a length above max_seq_len */
     char plan[64];
     CHECK(pa_decode_plan(NULL, 4, 4, 2, 64, 16, 128, 0, PA_KV_AUTO, plan, 64, NULL) ==

@@ -1,12 +1,16 @@
 """The split plan computed on the host (pa_split_plan; CPU, no GPU).
 
-The decode lays every sequence's 16-token tiles end to end, gives CTA c of C
-the tiles from lo(c) = floor(c N / C), and cuts a sequence wherever a CTA's
-share or a partition starts.  This file restates that definition tile by
-tile in Python (a set of segment starts per sequence) and checks the
-library's walk against it on random batches: the tile and segment prefix
-sums, each CTA's first sequence and segment index, and whether any sequence
-is split (which decides if the combine runs)."""
+The decode lays every sequence's 16-token tiles end to end and cuts the
+line into C shares evenly in weighted tiles: a sequence with tiles is
+preceded by PA_PLAN_ENTRY_WEIGHT = 2 virtual tiles (the cost of a CTA moving
+to it), a cut that falls there starting the share at the sequence's first
+tile (unweighted above PA_PLAN_WEIGHTED_MAX_ENTRIES = 4096 sequences).  A
+sequence is cut wherever a CTA's share or a partition starts.  This file
+restates that definition in Python (the virtual line listed tile by tile,
+a set of segment starts per sequence) and checks the library's walk against
+it on random batches: the tile and segment prefix sums, each CTA's first
+tile, first sequence and segment index, and whether any sequence is split
+(which decides if the combine runs)."""
 import numpy as np
 import pytest
 
@@ -31,7 +35,15 @@ def brute_plan(lens, max_len, partition_size, C):
     t = np.concatenate([[0], np.cumsum(tiles_of)]).astype(np.int64)
     N = int(t[-1])
     tpp = partition_size // 16 if partition_size else None
-    lo = [c * N // C for c in range(C)]
+    # the virtual line: each sequence with tiles is W switch slots (its first
+    # tile) followed by its tiles; a cut at virtual x starts at real[x]
+    W = 2 if len(lens) <= 4096 else 0
+    real = []
+    for b, n in enumerate(tiles_of):
+        if n > 0:
+            real += [int(t[b])] * W + list(range(int(t[b]), int(t[b]) + n))
+    V = len(real)
+    lo = [real[c * V // C] if c * V // C < V else N for c in range(C + 1)]
     starts = []  # per sequence: sorted segment starts (global tile index)
     for b in range(len(lens)):
         t0, t1 = int(t[b]), int(t[b + 1])
@@ -51,7 +63,8 @@ def brute_plan(lens, max_len, partition_size, C):
         start_seq[c] = b
         first_k[c] = sum(1 for s in starts[b] if s < x)
     return dict(tiles=t.astype(np.int32), seg_base=seg_base, start_seq=start_seq,
-                first_k=first_k, num_segments=int(seg_base[-1]),
+                first_k=first_k, cta_first_tile=np.array(lo, np.int32),
+                num_segments=int(seg_base[-1]),
                 needs_combine=any(len(S) > 1 for S in starts))
 
 
@@ -69,14 +82,13 @@ CASES = [
 def test_split_plan_matches_the_definition(pa, lens, max_len, psize, C):
     got = pa.split_plan(lens, max_len, psize, C)
     ref = brute_plan(lens, max_len, psize, C)
-    for k in ("tiles", "seg_base"):
+    for k in ("tiles", "seg_base", "cta_first_tile"):
         assert np.array_equal(got[k], ref[k]), k
     N = int(ref["tiles"][-1])
     if N:
         # CTAs with an empty share never read their entry; compare the others
-        lo = np.array([c * N // C for c in range(C)])
-        hi = np.array([(c + 1) * N // C for c in range(C)])
-        busy = lo < hi
+        lo = ref["cta_first_tile"]
+        busy = lo[:-1] < lo[1:]
         assert np.array_equal(got["start_seq"][busy], ref["start_seq"][busy])
         assert np.array_equal(got["first_k"][busy], ref["first_k"][busy])
     assert got["num_segments"] == ref["num_segments"]
@@ -95,8 +107,9 @@ def test_split_plan_random_batches(pa, seed):
     ref = brute_plan(lens, max_len, psize, C)
     assert np.array_equal(got["tiles"], ref["tiles"])
     assert np.array_equal(got["seg_base"], ref["seg_base"])
-    N = int(ref["tiles"][-1])
-    busy = np.array([c * N // C < (c + 1) * N // C for c in range(C)])
+    assert np.array_equal(got["cta_first_tile"], ref["cta_first_tile"])
+    lo = ref["cta_first_tile"]
+    busy = lo[:-1] < lo[1:]
     assert np.array_equal(got["start_seq"][busy], ref["start_seq"][busy])
     assert np.array_equal(got["first_k"][busy], ref["first_k"][busy])
     assert got["needs_combine"] == ref["needs_combine"]
