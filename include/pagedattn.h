@@ -475,7 +475,7 @@ pa_status pa_decode_attention_planned(void* out, pa_dtype out_dtype, const void*
                                       int32_t block_size, float scale, int32_t partition_size,
                                       const void* plan, void* workspace, size_t workspace_bytes,
                                       int32_t* device_error_flag, pa_stream_t stream);
-#define PA_PLAN_ENTRY_WEIGHT 2
+#define PA_PLAN_ENTRY_WEIGHT 3
 #define PA_PLAN_WEIGHTED_MAX_ENTRIES 4096
 pa_status pa_split_plan(const int32_t* seq_lens, int32_t num_seqs, int32_t max_seq_len,
                         int32_t partition_size, int32_t num_ctas, int32_t* tiles,

@@ -140,6 +140,8 @@ __device__ int32_t plan_sequence_segments(const DecodeParams& p, int32_t b, int6
 
 constexpr int kPlanSmemTiles = 4096;  // entries whose prefix sums are searched in shared memory
 constexpr int kPlanMaxCtas = 2048;    // CTAs per head group the plan can describe
+static_assert(kEntryWeight == PA_PLAN_ENTRY_WEIGHT && kPlanSmemTiles == PA_PLAN_WEIGHTED_MAX_ENTRIES,
+              "the header states the plan's weighting");
 
 // Largest e in [0, n) with tiles[e] <= x (tiles non-decreasing, tiles[0] = 0 <= x).
 __device__ __forceinline__ int upper_entry(const int32_t* tiles, int n, int64_t x) {

@@ -132,7 +132,7 @@ struct LineCut {
 // line is cut evenly in virtual tiles where an entry with tiles counts its
 // tiles plus kEntryWeight (its switch first).  Batches of more entries than
 // the plan keeps in shared memory are cut unweighted.
-constexpr int kEntryWeight = 2;
+constexpr int kEntryWeight = 3;  // same-GPU A/B: 3 beat 2 and 4 on longtail and multi-query
 
 // The real tile at virtual position x of an entry that starts at virtual
 // position v_e and real tile t_e and holds n_e tiles (weight w per switch):

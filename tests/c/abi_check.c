@@ -60,16 +60,16 @@ int main(void) {
 
   /* the split plan on the host: 4 sequences (1, 3, 0 and 7 tiles) over 7
    * CTAs.  Weighted line: the three sequences with tiles start at virtual
-   * tiles 0, 3 and 8 (2 more each), 17 in all; cut at 0, 2, 4, 7, 9, 12, 14,
-   * 17 -> first tiles 0, 0, 1, 3, 4, 6, 8, 11 */
+   * tiles 0, 4 and 10 (3 more each), 20 in all; cut at 0, 2, 5, 8, 11, 14, 17,
+   * 20 -> first tiles 0, 0, 1, 2, 4, 5, 8, 11 */
   {
     const int32_t lens4[4] = {5, 40, 0, 100};
     int32_t tiles[5], segs[5], start[7], firstk[7], ctalo[8], nseg = -1, comb = -1;
     CHECK(pa_split_plan(lens4, 4, 128, 0, 7, tiles, segs, start, firstk, ctalo, &nseg, &comb) ==
           PA_OK);
     CHECK(tiles[0] == 0 && tiles[1] == 1 && tiles[2] == 4 && tiles[3] == 4 && tiles[4] == 11);
-    CHECK(ctalo[0] == 0 && ctalo[1] == 0 && ctalo[2] == 1 && ctalo[3] == 3 && ctalo[4] == 4 &&
-          ctalo[5] == 6 && ctalo[6] == 8 && ctalo[7] == 11);
+    CHECK(ctalo[0] == 0 && ctalo[1] == 0 && ctalo[2] == 1 && ctalo[3] == 2 && ctalo[4] == 4 &&
+          ctalo[5] == 5 && ctalo[6] == 8 && ctalo[7] == 11);
     CHECK(segs[1] == 1 && segs[2] == 3 && segs[3] == 3 && segs[4] == 6 && nseg == 6 && comb == 1);
     CHECK(start[3] == 1 && firstk[3] == 1 && start[6] == 3 && firstk[6] == 2);
     CHECK(pa_split_plan(lens4, 4, 64, 0, 7, tiles, segs, start, firstk, ctalo, &nseg, &comb) ==

@@ -2,7 +2,7 @@
 
 The decode lays every sequence's 16-token tiles end to end and cuts the
 line into C shares evenly in weighted tiles: a sequence with tiles is
-preceded by PA_PLAN_ENTRY_WEIGHT = 2 virtual tiles (the cost of a CTA moving
+preceded by PA_PLAN_ENTRY_WEIGHT = 3 virtual tiles (the cost of a CTA moving
 to it), a cut that falls there starting the share at the sequence's first
 tile (unweighted above PA_PLAN_WEIGHTED_MAX_ENTRIES = 4096 sequences).  A
 sequence is cut wherever a CTA's share or a partition starts.  This file
@@ -37,7 +37,7 @@ def brute_plan(lens, max_len, partition_size, C):
     tpp = partition_size // 16 if partition_size else None
     # the virtual line: each sequence with tiles is W switch slots (its first
     # tile) followed by its tiles; a cut at virtual x starts at real[x]
-    W = 2 if len(lens) <= 4096 else 0
+    W = 3 if len(lens) <= 4096 else 0
     real = []
     for b, n in enumerate(tiles_of):
         if n > 0:
