@@ -156,7 +156,12 @@ __device__ __forceinline__ int upper_entry(const int32_t* tiles, int n, int64_t 
 __global__ void __launch_bounds__(kPlanThreads) pa_plan_kernel(DecodeParams p) {
   __shared__ int32_t warp_buf[kPlanWarps];
   __shared__ int32_t s_tiles[kPlanSmemTiles + 1];
-  __shared__ int32_t s_sd[kPlanMaxCtas + 1], s_sdc[kPlanMaxCtas + 1];
+  // s_sd, s_sdc: the closed form's prefix sums over CTAs; before them the
+  // same words hold the entries' virtual starts while the line is cut
+  __shared__ int32_t s_aux[2 * (kPlanMaxCtas + 1)];
+  static_assert(2 * (kPlanMaxCtas + 1) >= kPlanSmemTiles + 1, "virtual starts fit s_aux");
+  int32_t* const s_sd = s_aux;
+  int32_t* const s_sdc = s_aux + kPlanMaxCtas + 1;
   __shared__ int32_t s_lo[kPlanMaxCtas + 1];  // first tile of each CTA's share
   const int tid = threadIdx.x;
   const int B = p.num_seqs;
@@ -313,37 +318,35 @@ __global__ void __launch_bounds__(kPlanThreads) pa_plan_kernel(DecodeParams p) {
   // line is cut evenly (LineCut; with a split, the packs and the sequences
   // separately) in virtual tiles, where an entry with tiles counts
   // kEntryWeight more (its switch first); each cut is then mapped back to the
-  // real tile at that virtual position.  The virtual starts live in s_tiles
-  // while the cut is made, so only a batch whose prefix sums fit there is
-  // weighted.
+  // real tile at that virtual position.  The virtual starts (s_vs) take the
+  // closed form's words until that form starts; a batch whose prefix sums do
+  // not fit in shared memory is cut unweighted.
   const int64_t w = in_smem ? kEntryWeight : 0;
   LineCut cut;
   cut.C = C;
   cut.S = p.split_ctas;
   if (w > 0) {
+    int32_t* const s_vs = s_aux;
     int32_t vcarry = 0, vtot = 0;
     for (int ch = 0; ch < nchunks; ++ch) {
       const int e = ch * kPlanThreads + tid;
-      const int32_t has = (e < E && p.plan_tiles[e + 1] > p.plan_tiles[e]) ? 1 : 0;
+      const int32_t has = (e < E && s_tiles[e + 1] > s_tiles[e]) ? 1 : 0;
       const int32_t ex = block_exclusive_scan(has, warp_buf, &vtot);
-      if (e < E) s_tiles[e] = p.plan_tiles[e] + static_cast<int32_t>(w) * (vcarry + ex);
+      if (e < E) s_vs[e] = s_tiles[e] + static_cast<int32_t>(w) * (vcarry + ex);
       vcarry += vtot;
     }
-    if (tid == 0) s_tiles[E] = static_cast<int32_t>(N + w * vcarry);
+    if (tid == 0) s_vs[E] = static_cast<int32_t>(N + w * vcarry);
     __syncthreads();
-    cut.N = s_tiles[E];
-    cut.NK = p.split_ctas > 0 ? s_tiles[K] : 0;
+    cut.N = s_vs[E];
+    cut.NK = p.split_ctas > 0 ? s_vs[K] : 0;
     for (int c = tid; c <= C; c += kPlanThreads) {
       const int64_t x = cut.lo(c);
-      const int e = upper_entry(s_tiles, E + 1, x);
-      const int64_t t = e >= E ? N
-                               : entry_tile(x, s_tiles[e], p.plan_tiles[e],
-                                            p.plan_tiles[e + 1] - p.plan_tiles[e], w);
+      const int e = upper_entry(s_vs, E + 1, x);
+      const int64_t t =
+          e >= E ? N : entry_tile(x, s_vs[e], s_tiles[e], s_tiles[e + 1] - s_tiles[e], w);
       s_lo[c] = static_cast<int32_t>(t);
       p.cta_lo[c] = static_cast<int32_t>(t);
     }
-    __syncthreads();  // s_tiles is read above until here
-    for (int e = tid; e <= E; e += kPlanThreads) s_tiles[e] = p.plan_tiles[e];
   } else {
     cut.N = N;
     cut.NK = p.split_ctas > 0 ? tiles[K] : 0;
@@ -352,7 +355,7 @@ __global__ void __launch_bounds__(kPlanThreads) pa_plan_kernel(DecodeParams p) {
       p.cta_lo[c] = s_lo[c];
     }
   }
-  __syncthreads();  // s_lo and the real prefix sums are read below
+  __syncthreads();  // s_lo is read below, and s_aux is free again
   if (!p.plan_closed) {  // few cut points per entry: walk them
     int32_t seg_carry = 0;
     for (int ch = 0; ch < nchunks; ++ch) {
