@@ -499,8 +499,10 @@ __global__ void __launch_bounds__((HG * CG + 1) * 32, 1)
     prefetch_tmap(&tmV);
   }
   __syncthreads();
-  griddep_launch_dependents();
   griddep_wait();  // the plan (and all earlier work on the stream) is complete
+  // the next launch (the combine) may start now: what it reads before its
+  // own wait, the plan, is complete
+  griddep_launch_dependents();
   if (!host_plan_matches(p)) {  // a plan made for another shape: no work at all
     if (threadIdx.x == 0 && c == 0 && hg == 0) flag_error(p.err, PA_DEVERR_BAD_PLAN);
     return;
@@ -921,7 +923,9 @@ __global__ void __launch_bounds__((HG * CG + 1) * 32, 1)
 // The partials of output row r, query head h (h inside its KV head's group):
 // those of its own entry (slots s0 .., column col0) and, for a pack member,
 // those of the pack's entry (slots s1 .., column col1).  direct: the main
-// kernel wrote the row itself.  valid: the row belongs to an entry.
+// kernel wrote the row itself.  valid: the row belongs to an entry.  Read
+// from L2 before the combine waits on the main kernel: the plan is complete
+// once any main CTA has let the combine start.
 struct RowParts {
   int32_t s0, ns, col0, s1, np, col1;
   bool direct, valid;
@@ -932,25 +936,25 @@ __device__ __forceinline__ RowParts row_parts(const DecodeParams& p, int r, int 
   q.s1 = q.np = q.col1 = 0;
   q.valid = true;
   if (p.q_start != nullptr) {  // query chunks: row r is column (r - first row) * G + h
-    const int e = p.q_entry[r];
-    q.valid = e >= 0 && e < p.meta[1];
+    const int e = __ldcg(p.q_entry + r);
+    q.valid = e >= 0 && e < __ldcg(p.meta + 1);
     const int ee = q.valid ? e : 0;
-    q.s0 = p.seg_base[ee];
-    q.ns = p.seg_base[ee + 1] - q.s0;
-    q.col0 = (r - p.ent_q0[ee]) * p.group + h;
+    q.s0 = __ldcg(p.seg_base + ee);
+    q.ns = __ldcg(p.seg_base + ee + 1) - q.s0;
+    q.col0 = (r - __ldcg(p.ent_q0 + ee)) * p.group + h;
     q.direct = q.ns == 1;
     return q;
   }
-  const int K = p.pack_size > 1 ? p.meta[0] : 0;
-  q.s0 = p.seg_base[K + r];
-  q.ns = p.seg_base[K + r + 1] - q.s0;
+  const int K = p.pack_size > 1 ? __ldcg(p.meta) : 0;
+  q.s0 = __ldcg(p.seg_base + K + r);
+  q.ns = __ldcg(p.seg_base + K + r + 1) - q.s0;
   q.col0 = h;
-  const int pk = p.pack_size > 1 ? p.seq_pack[r] : -1;
+  const int pk = p.pack_size > 1 ? __ldcg(p.seq_pack + r) : -1;
   q.direct = pk < 0 && q.ns == 1;
   if (pk >= 0) {
-    q.s1 = p.seg_base[pk];
-    q.np = p.seg_base[pk + 1] - q.s1;
-    q.col1 = (r - p.pack_first[pk]) * p.group + h;
+    q.s1 = __ldcg(p.seg_base + pk);
+    q.np = __ldcg(p.seg_base + pk + 1) - q.s1;
+    q.col1 = (r - __ldcg(p.pack_first + pk)) * p.group + h;
   }
   return q;
 }
@@ -961,19 +965,20 @@ __global__ void __launch_bounds__(kCombineWarps * 32) pa_combine_narrow_kernel(c
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int b = blockIdx.x;
   const int qh = blockIdx.y * kCombineWarps + warp;
+  const int G = p.group;
+  const int kvh = qh / G, h = qh - kvh * G;
+  const bool live = qh < p.num_q_heads && host_plan_matches(p);
+  RowParts rp{};
+  if (live) rp = row_parts(p, b, h);  // the plan is complete: read it before the wait
   // the next launch on the stream may start its prologue now; it waits for
   // this grid before touching data
   griddep_launch_dependents();
   griddep_wait();  // the main kernel's partials are complete and visible
-  if (qh >= p.num_q_heads || !host_plan_matches(p)) return;
-  const int G = p.group;
-  const int kvh = qh / G, h = qh - kvh * G;
-  const RowParts rp = row_parts(p, b, h);
-  if (rp.direct || !rp.valid) return;  // written by the main kernel (or no entry)
+  if (!live || rp.direct || !rp.valid) return;  // written by the main kernel (or no entry)
   // partial k: k < ns from the row's own entry, then the pack's
   const int32_t nseq = (rp.s0 + rp.ns <= p.nseg_cap) ? rp.ns : 0;
   const int32_t npack = (rp.s1 + rp.np <= p.nseg_cap) ? rp.np : 0;
-  const int32_t ntot = nseq + npack;
+  int32_t ntot = nseq + npack;
   auto row_of = [&](int32_t k) {
     const int32_t slot = k < nseq ? rp.s0 + k : rp.s1 + (k - nseq);
     const int col = k < nseq ? rp.col0 : rp.col1;
@@ -981,6 +986,48 @@ __global__ void __launch_bounds__(kCombineWarps * 32) pa_combine_narrow_kernel(c
   };
   const int64_t obase = (static_cast<int64_t>(b) * p.num_q_heads + qh) * D + lane * V;
 
+  float acc[V];
+#pragma unroll
+  for (int v = 0; v < V; ++v) acc[v] = 0.f;
+  float W = 0.f;
+  if (ntot <= kCombineRegs) {
+    // few partials: every load is issued at once, then the same arithmetic
+    // in the same order as the loops below
+    float mk[kCombineRegs], lk[kCombineRegs], ok[kCombineRegs][V];
+#pragma unroll
+    for (int k = 0; k < kCombineRegs; ++k) {
+      mk[k] = -INFINITY;
+      lk[k] = 0.f;
+#pragma unroll
+      for (int v = 0; v < V; ++v) ok[k][v] = 0.f;
+      if (k < ntot) {
+        const int64_t r = row_of(k);
+        mk[k] = p.part_ml[r * 2];
+        lk[k] = p.part_ml[r * 2 + 1];
+        const float* po = p.part_o + r * D + lane * V;
+        if constexpr (V == 4) {
+          const float4 o4 = *reinterpret_cast<const float4*>(po);
+          ok[k][0] = o4.x; ok[k][1] = o4.y; ok[k][2] = o4.z; ok[k][3] = o4.w;
+        } else {
+          const float2 o2 = *reinterpret_cast<const float2*>(po);
+          ok[k][0] = o2.x; ok[k][1] = o2.y;
+        }
+      }
+    }
+    float M = -INFINITY;
+#pragma unroll
+    for (int k = 0; k < kCombineRegs; ++k)
+      if (lk[k] > 0.f) M = fmaxf(M, mk[k]);
+#pragma unroll
+    for (int k = 0; k < kCombineRegs; ++k) {
+      if (!(lk[k] > 0.f)) continue;  // nothing attended (or no partial k): skip, never 0 * o
+      const float w = lk[k] * ex2(mk[k] - M);
+#pragma unroll
+      for (int v = 0; v < V; ++v) acc[v] += w * ok[k][v];
+      W += w;
+    }
+    ntot = 0;  // done: the loops below run no iteration
+  }
   float M = -INFINITY;
   for (int k = lane; k < ntot; k += 32) {
     const int64_t r = row_of(k);
@@ -990,10 +1037,6 @@ __global__ void __launch_bounds__(kCombineWarps * 32) pa_combine_narrow_kernel(c
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-  float acc[V];
-#pragma unroll
-  for (int v = 0; v < V; ++v) acc[v] = 0.f;
-  float W = 0.f;
 #pragma unroll 4
   for (int k = 0; k < ntot; ++k) {
     const int64_t r = row_of(k);
@@ -1041,15 +1084,16 @@ __global__ void __launch_bounds__(kCombineWarps * 32) pa_combine_wide_kernel(con
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int b = blockIdx.x;
   const int qh = blockIdx.y;
+  const int G = p.group;
+  const int kvh = qh / G, h = qh - kvh * G;
+  const bool live = host_plan_matches(p);
+  RowParts rp{};
+  if (live) rp = row_parts(p, b, h);  // the plan is complete: read it before the wait
   // the next launch on the stream may start its prologue now; it waits for
   // this grid before touching data
   griddep_launch_dependents();
   griddep_wait();  // the main kernel's partials are complete and visible
-  if (!host_plan_matches(p)) return;
-  const int G = p.group;
-  const int kvh = qh / G, h = qh - kvh * G;
-  const RowParts rp = row_parts(p, b, h);
-  if (rp.direct || !rp.valid) return;  // written by the main kernel (or no entry)
+  if (!live || rp.direct || !rp.valid) return;  // written by the main kernel (or no entry)
   const int32_t nseq = (rp.s0 + rp.ns <= p.nseg_cap) ? rp.ns : 0;
   const int32_t npack = (rp.s1 + rp.np <= p.nseg_cap) ? rp.np : 0;
   const int32_t ntot = nseq + npack;

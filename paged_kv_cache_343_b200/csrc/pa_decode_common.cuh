@@ -16,6 +16,7 @@ namespace pa {
 constexpr int kTile = 16;            // tokens per tile (MMA M of the score product)
 constexpr int kPlanThreads = 256;
 constexpr int kCombineWarps = 4;
+constexpr int kCombineRegs = 8;  // partials a combine lane loads at once (few-partial rows)
 
 enum : int32_t {
   kNewSeq = 1,    // first tile of a sequence in this CTA: reload Q

@@ -159,8 +159,10 @@ __global__ void __launch_bounds__(kUThreads, 1)
     for (int k = 0; k < kUBufs * 4; ++k) tmem_st16(lrow + kColP + 16u * k, zero);
     tmem_wait_st();
   }
-  griddep_launch_dependents();
   griddep_wait();  // the plan (and all earlier work on the stream) is complete
+  // the next launch may start now: what it reads before its own wait, the
+  // plan, is complete
+  griddep_launch_dependents();
 
   int64_t lo = 0, hi = 0;
   if (host_plan_matches(p)) {
