@@ -98,6 +98,51 @@ __device__ __forceinline__ int32_t block_exclusive_scan(int32_t v, int32_t* warp
   return before;
 }
 
+// The same for two values per thread at once (warp_buf holds 2 kPlanWarps
+// words): exclusive sums in ex[0..1], block totals in total[0..1].
+__device__ __forceinline__ void block_exclusive_scan2(int32_t v0, int32_t v1, int32_t* warp_buf,
+                                                      int32_t* ex, int32_t* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int32_t i0 = v0, i1 = v1;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int32_t u0 = __shfl_up_sync(0xffffffffu, i0, o);
+    const int32_t u1 = __shfl_up_sync(0xffffffffu, i1, o);
+    if (lane >= o) {
+      i0 += u0;
+      i1 += u1;
+    }
+  }
+  if (lane == 31) {
+    warp_buf[warp] = i0;
+    warp_buf[kPlanWarps + warp] = i1;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    int32_t w0 = lane < kPlanWarps ? warp_buf[lane] : 0;
+    int32_t w1 = lane < kPlanWarps ? warp_buf[kPlanWarps + lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int32_t u0 = __shfl_up_sync(0xffffffffu, w0, o);
+      const int32_t u1 = __shfl_up_sync(0xffffffffu, w1, o);
+      if (lane >= o) {
+        w0 += u0;
+        w1 += u1;
+      }
+    }
+    if (lane < kPlanWarps) {  // inclusive over warps
+      warp_buf[lane] = w0;
+      warp_buf[kPlanWarps + lane] = w1;
+    }
+  }
+  __syncthreads();
+  ex[0] = (warp > 0 ? warp_buf[warp - 1] : 0) + i0 - v0;
+  ex[1] = (warp > 0 ? warp_buf[kPlanWarps + warp - 1] : 0) + i1 - v1;
+  total[0] = warp_buf[kPlanWarps - 1];
+  total[1] = warp_buf[2 * kPlanWarps - 1];
+  __syncthreads();  // warp_buf is reused by the next call
+}
+
 // Smallest c in [0, C] with lo[c] >= x, i.e. the number of CTA shares that
 // start below x (lo non-decreasing, lo[C] = N >= x).
 __device__ __forceinline__ int32_t ctas_below(const int32_t* lo, int32_t C, int64_t x) {
@@ -154,7 +199,7 @@ __device__ __forceinline__ int upper_entry(const int32_t* tiles, int n, int64_t 
 }
 
 __global__ void __launch_bounds__(kPlanThreads) pa_plan_kernel(DecodeParams p) {
-  __shared__ int32_t warp_buf[kPlanWarps];
+  __shared__ int32_t warp_buf[2 * kPlanWarps];
   __shared__ int32_t s_tiles[kPlanSmemTiles + 1];
   // s_sd, s_sdc: the closed form's prefix sums over CTAs; before them the
   // same words hold the entries' virtual starts while the line is cut
@@ -284,7 +329,12 @@ __global__ void __launch_bounds__(kPlanThreads) pa_plan_kernel(DecodeParams p) {
     p.meta[1] = E;
   }
   const int nchunks = (E + kPlanThreads - 1) / kPlanThreads;
-  int32_t carry = 0, total = 0;
+  // the cut weighs entry switches when the prefix sums fit in shared memory;
+  // the entries' virtual starts (s_vs) are summed with their tiles
+  const bool in_smem = E <= kPlanSmemTiles;
+  const int64_t w = in_smem ? kEntryWeight : 0;
+  int32_t* const s_vs = s_aux;
+  int32_t carry = 0, total = 0, vcarry = 0;
   for (int ch = 0; ch < nchunks; ++ch) {
     const int e = ch * kPlanThreads + tid;
     int32_t nt = 0;
@@ -299,44 +349,39 @@ __global__ void __launch_bounds__(kPlanThreads) pa_plan_kernel(DecodeParams p) {
       nt = (clamp_len(raw, p.max_seq_len) + kTile - 1) / kTile;
       if (p.pack_size > 1) nt -= p.seq_pre[b];
     }
-    const int32_t ex = block_exclusive_scan(nt, warp_buf, &total);
-    if (e < E) p.plan_tiles[e] = carry + ex;
-    if (e < E && e <= kPlanSmemTiles) s_tiles[e] = carry + ex;
-    carry += total;
+    int32_t ex[2], tot[2];
+    block_exclusive_scan2(nt, nt > 0 ? 1 : 0, warp_buf, ex, tot);
+    if (e < E) p.plan_tiles[e] = carry + ex[0];
+    if (e < E && in_smem) {
+      s_tiles[e] = carry + ex[0];
+      s_vs[e] = carry + ex[0] + static_cast<int32_t>(w) * (vcarry + ex[1]);
+    }
+    carry += tot[0];
+    vcarry += tot[1];
   }
   if (tid == 0) {
     p.plan_tiles[E] = carry;
-    if (E <= kPlanSmemTiles) s_tiles[E] = carry;
+    if (in_smem) {
+      s_tiles[E] = carry;
+      s_vs[E] = static_cast<int32_t>(carry + w * vcarry);
+    }
   }
   __syncthreads();  // the prefix sums are read back below
   const int64_t N = carry;
   const int C = p.ctas_per_group;
   const int32_t tpp = p.tiles_per_part;
-  const bool in_smem = E <= kPlanSmemTiles;
   const int32_t* tiles = in_smem ? s_tiles : p.plan_tiles;
   // ---- the cut: CTA c's share starts at tile s_lo[c] (also cta_lo[c]).  The
   // line is cut evenly (LineCut; with a split, the packs and the sequences
   // separately) in virtual tiles, where an entry with tiles counts
   // kEntryWeight more (its switch first); each cut is then mapped back to the
-  // real tile at that virtual position.  The virtual starts (s_vs) take the
-  // closed form's words until that form starts; a batch whose prefix sums do
-  // not fit in shared memory is cut unweighted.
-  const int64_t w = in_smem ? kEntryWeight : 0;
+  // real tile at that virtual position.  The virtual starts (s_vs, summed
+  // above) take the closed form's words until that form starts; a batch whose
+  // prefix sums do not fit in shared memory is cut unweighted.
   LineCut cut;
   cut.C = C;
   cut.S = p.split_ctas;
   if (w > 0) {
-    int32_t* const s_vs = s_aux;
-    int32_t vcarry = 0, vtot = 0;
-    for (int ch = 0; ch < nchunks; ++ch) {
-      const int e = ch * kPlanThreads + tid;
-      const int32_t has = (e < E && s_tiles[e + 1] > s_tiles[e]) ? 1 : 0;
-      const int32_t ex = block_exclusive_scan(has, warp_buf, &vtot);
-      if (e < E) s_vs[e] = s_tiles[e] + static_cast<int32_t>(w) * (vcarry + ex);
-      vcarry += vtot;
-    }
-    if (tid == 0) s_vs[E] = static_cast<int32_t>(N + w * vcarry);
-    __syncthreads();
     cut.N = s_vs[E];
     cut.NK = p.split_ctas > 0 ? s_vs[K] : 0;
     for (int c = tid; c <= C; c += kPlanThreads) {
