@@ -115,6 +115,33 @@ def test_split_plan_random_batches(pa, seed):
     assert got["needs_combine"] == ref["needs_combine"]
 
 
+@pytest.mark.parametrize("B", [4096, 4097, 5000])
+def test_split_plan_weight_limit(pa, B):
+    """The switch weight applies while the batch's prefix sums fit the plan
+    kernel's shared table (PA_PLAN_WEIGHTED_MAX_ENTRIES = 4096 sequences);
+    above it the line is cut evenly in real tiles, so share c starts at
+    tile floor(c N / C)."""
+    rng = np.random.default_rng(B)
+    lens = rng.integers(0, 65, B)
+    C = 148
+    got = pa.split_plan(lens, 64, 0, C)
+    ref = brute_plan(lens, 64, 0, C)
+    assert np.array_equal(got["tiles"], ref["tiles"])
+    assert np.array_equal(got["seg_base"], ref["seg_base"])
+    assert np.array_equal(got["cta_first_tile"], ref["cta_first_tile"])
+    N = int(ref["tiles"][-1])
+    even = np.array([c * N // C for c in range(C + 1)], np.int32)
+    if B > 4096:
+        assert np.array_equal(got["cta_first_tile"], even)
+    else:
+        assert not np.array_equal(got["cta_first_tile"], even)
+    lo = ref["cta_first_tile"]
+    busy = lo[:-1] < lo[1:]
+    assert np.array_equal(got["start_seq"][busy], ref["start_seq"][busy])
+    assert np.array_equal(got["first_k"][busy], ref["first_k"][busy])
+    assert got["needs_combine"] == ref["needs_combine"]
+
+
 def test_split_plan_refuses_bad_arguments(pa):
     import paged_kv_cache_343_b200 as m
     with pytest.raises(m.PagedAttnError):      # a length above max_seq_len
